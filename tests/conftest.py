@@ -1,0 +1,19 @@
+"""Test configuration: the ``gpu`` marker and import paths.
+
+Tests marked ``gpu`` need a CUDA device and the built CUDA library; the rest
+run on any host (``pytest -m "not gpu"``).
+"""
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+HERE = os.path.dirname(os.path.abspath(__file__))
+if HERE not in sys.path:
+    sys.path.insert(0, HERE)
+
+
+def pytest_configure(config):
+    config.addinivalue_line(
+        "markers", "gpu: needs a CUDA device (B200) and the built CUDA library")
