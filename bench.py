@@ -1,0 +1,437 @@
+#!/usr/bin/env python
+"""Throughput of the fused QK-RMSNorm + RoPE forward + backward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...      (the CPU oracle, as the reference arm)
+
+A step is one forward and one backward over one batch of the workload
+(default: the Qwen2.5-0.5B-shaped batch, 8 x 2048 tokens, 14 query / 2 KV
+heads of dim 64, bf16 I/O). Inputs are resident in HBM before timing. Each
+rank keeps a ring of four input/output sets; step i runs the forward on set
+i mod 4 and the backward on set (i - 2) mod 4 (a layer's backward comes
+after the rest of the forward in training), so no kernel finds its inputs in
+the 126 MB L2: between two touches of a set ~2.5x L2 of other traffic
+passes. K steps are timed with CUDA events between a barrier and a
+synchronize on both sides; every fwd/bwd launch is also bracketed by events
+on its stream for the per-kernel roofline. N > 1 (torchrun): weak scaling,
+each rank its own batch, no collective on the data path; the time is the
+max over ranks.
+
+Rank 0 prints one JSON line. ``e2e`` repeats the step through the public
+Python API from pinned host buffers (inputs copied in, every output copied
+back, inside the timed region). ``cpu_baseline`` times the CPU oracle on a
+bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "QK-norm+RoPE fwd+bwd tokens/s and HBM GB/s (% of B200 peak), 1 GPU"
+FALLBACK_HBM_GBS = 6650.0
+NSETS, LAG = 4, 2
+KERNEL_SOURCES = ["qk_rmsnorm_rope_norm_b200/csrc/qknr_kernels.cuh",
+                  "qk_rmsnorm_rope_norm_b200/csrc/qknr_api.cu"]
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def env_rank():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)),
+            int(os.environ.get("WORLD_SIZE", 1)))
+
+
+def hbm_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback (6.65 TB/s, earlier measurement on this pool)"
+
+
+def source_hash():
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def ncu_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, or None when the
+    kernel sources changed since it was captured."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        e = d[kernel][workload]
+        if e.get("source_sha256") != source_hash():
+            return None
+        return float(e["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+# ----------------------------------------------------------------- clocks
+REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+           0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+           0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+           0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    """NVML samples of the SM clock and clock-event reasons, every few ms,
+    while the timed region runs."""
+
+    def __init__(self, device_index: int, period_s: float = 0.002):
+        self.ok = False
+        self.samples = []
+        self.period = period_s
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = self._handle(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report clocks as unknown
+            log("clock sampler unavailable:", e)
+
+    def _handle(self, idx):
+        nv = self.nv
+        try:
+            p = torch.cuda.get_device_properties(idx)
+            bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+            return nv.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+            phys = int(vis.split(",")[idx]) if vis and vis.split(",")[0].isdigit() else idx
+            return nv.nvmlDeviceGetHandleByIndex(phys)
+
+    def sample(self):
+        nv = self.nv
+        sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+        try:
+            r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+        self.samples.append((sm, r))
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.sample()
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._stop = threading.Event()
+            self.sample()
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+            self.sample()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unknown: no NVML"]}
+        busy = [s for s in self.samples if not (s[1] & 0x1)] or self.samples
+        mask = 0
+        for _, r in busy:
+            mask |= r
+        reasons = [n for b, n in REASONS.items() if mask & b]
+        return {"sm_mhz": statistics.median(s[0] for s in busy), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- our arm
+class Set:
+    """Device buffers of one batch: inputs, forward outputs, gradients."""
+
+    def __init__(self, inp: workloads.Inputs, dev):
+        w = inp.w
+        self.q, self.k = inp.q.to(dev), inp.k.to(dev)
+        self.gq, self.gk = inp.gamma_q.to(dev), inp.gamma_k.to(dev)
+        self.pos = None if inp.pos is None else inp.pos.to(dev)
+        self.dqo, self.dko = inp.dq_out.to(dev), inp.dk_out.to(dev)
+        self.qo, self.ko = torch.empty_like(self.q), torch.empty_like(self.k)
+        self.rq = torch.empty((w.B, w.S, w.Hq), dtype=torch.float32, device=dev)
+        self.rk = torch.empty((w.B, w.S, w.Hkv), dtype=torch.float32, device=dev)
+        self.dq, self.dk = torch.empty_like(self.q), torch.empty_like(self.k)
+        self.dgq = torch.empty(w.D, dtype=torch.float32, device=dev)
+        self.dgk = torch.empty(w.D, dtype=torch.float32, device=dev)
+
+
+def run_ours(args, w, inp, rank, local_rank, world):
+    import qk_rmsnorm_rope_norm_b200 as qknr
+    dev = torch.device("cuda", local_rank)
+    qknr.load_library()
+    cfg = dict(rotary_dim=w.rotary_dim, theta=w.theta, eps=w.eps)
+    sets = [Set(inp, dev) for _ in range(NSETS)]
+    stream = torch.cuda.current_stream(dev)
+    fwd = [qknr.prepare_fwd(s.q, s.k, s.gq, s.gk, s.pos, s.qo, s.ko, s.rq, s.rk, **cfg)
+           for s in sets]
+    bwd = [qknr.prepare_bwd(s.q, s.k, s.gq, s.gk, s.pos, s.rq, s.rk, s.dqo, s.dko, s.dq,
+                            s.dk, s.dgq, s.dgk, **cfg) for s in sets]
+    K, W = args.steps, args.warmup
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def step(i, e=None):
+        if e is not None:
+            e[0].record(stream)
+        fwd[i % NSETS]()
+        if e is not None:
+            e[1].record(stream)
+        bwd[(i - LAG) % NSETS]()
+        if e is not None:
+            e[2].record(stream)
+
+    for i in range(W):
+        step(i)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local_rank) as clocks:
+        t_start.record(stream)
+        for i in range(K):
+            step(W + i, ev[i])
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    total_ms = t_start.elapsed_time(t_end)
+    fwd_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / K
+    bwd_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / K
+    t = torch.tensor([total_ms, fwd_ms, bwd_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    total_ms, fwd_ms, bwd_ms = t.tolist()
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, w, inp, dev, cfg, world)
+    return dict(total_ms=total_ms, fwd_ms=fwd_ms, bwd_ms=bwd_ms, clocks=clocks.summary(),
+                e2e=e2e)
+
+
+def run_e2e(args, w, inp, dev, cfg, world):
+    """Public API from pinned host buffers: H2D inputs, fwd, bwd, D2H outputs."""
+    import qk_rmsnorm_rope_norm_b200 as qknr
+    host_in = {n: getattr(inp, n).pin_memory() for n in ("q", "k", "dq_out", "dk_out")}
+    gq, gk = inp.gamma_q.to(dev), inp.gamma_k.to(dev)
+    pos = None if inp.pos is None else inp.pos.to(dev)
+    d = {n: torch.empty_like(t, device=dev) for n, t in host_in.items()}
+    out_shapes = {"q_out": (inp.q.shape, inp.q.dtype), "k_out": (inp.k.shape, inp.k.dtype),
+                  "rstd_q": ((w.B, w.S, w.Hq), torch.float32),
+                  "rstd_k": ((w.B, w.S, w.Hkv), torch.float32),
+                  "dq": (inp.q.shape, inp.q.dtype), "dk": (inp.k.shape, inp.k.dtype),
+                  "dgamma_q": ((w.D,), torch.float32), "dgamma_k": ((w.D,), torch.float32)}
+    host_out = {n: torch.empty(s, dtype=dt).pin_memory() for n, (s, dt) in out_shapes.items()}
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+
+    def step():
+        for n, t in host_in.items():
+            d[n].copy_(t, non_blocking=True)
+        qo, ko, rq, rk = qknr.qk_norm_rope_fwd(d["q"], d["k"], gq, gk, pos, **cfg)
+        dq, dk, dgq, dgk = qknr.qk_norm_rope_bwd(d["q"], d["k"], gq, gk, pos, rq, rk,
+                                                 d["dq_out"], d["dk_out"], **cfg)
+        for n, t in (("q_out", qo), ("k_out", ko), ("rstd_q", rq), ("rstd_k", rk),
+                     ("dq", dq), ("dk", dk), ("dgamma_q", dgq), ("dgamma_k", dgk)):
+            host_out[n].copy_(t, non_blocking=True)
+
+    E = max(1, min(args.steps, args.e2e_steps))
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(E):
+        step()
+    b.record()
+    torch.cuda.synchronize(dev)
+    ms = a.elapsed_time(b) / E
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return dict(ms=float(t.item()), steps=E, h2d=h2d, d2h=d2h)
+
+
+# ------------------------------------------------------- the CPU oracle
+def oracle_sample_rate(inp, budget_s: float, tokens_per_call: int = 512, max_calls=None):
+    """Time the CPU oracle (fwd + bwd) on consecutive token chunks of the
+    workload until ``budget_s`` seconds or the workload are used up."""
+    import oracle
+    w = inp.w
+    T = w.B * w.S
+    m_all = oracle.positions(None if inp.pos is None else inp.pos.numpy(), w.B, w.S)
+    q = inp.q.reshape(T, w.Hq, w.D)
+    k = inp.k.reshape(T, w.Hkv, w.D)
+    dqo = inp.dq_out.reshape(T, w.Hq, w.D)
+    dko = inp.dk_out.reshape(T, w.Hkv, w.D)
+    orc = oracle.get()
+    done, spent, calls, t0 = 0, 0.0, 0, 0
+    per_call = []
+    while spent < budget_s and (max_calls is None or calls < max_calls):
+        t1 = min(T, t0 + tokens_per_call)
+        args = [a[t0:t1] for a in (q, k)]
+        m = m_all[t0:t1]
+        c = time.perf_counter()
+        orc.fwd(args[0], args[1], inp.gamma_q, inp.gamma_k, m, w.rotary_dim, w.theta, w.eps)
+        orc.bwd(args[0], args[1], inp.gamma_q, inp.gamma_k, m, dqo[t0:t1], dko[t0:t1],
+                w.rotary_dim, w.theta, w.eps)
+        dt = time.perf_counter() - c
+        per_call.append(dt)
+        spent += dt
+        done += t1 - t0
+        calls += 1
+        t0 = t1 % T
+    return done, spent, per_call
+
+
+def config_of(w, inp, world):
+    return {"workload": w.name, "B": w.B, "S": w.S, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
+            "rotary_dim": w.rotary_dim, "theta": w.theta, "eps": w.eps, "io_dtype": w.dtype,
+            "tokens_per_step": inp.real_tokens,
+            "l2": f"ring of {NSETS} input sets, bwd lags fwd by {LAG} steps: inputs not "
+                  f"L2-resident (> 2x 126 MB of traffic between touches)",
+            "parallelism": f"dp{world} (weak, no data-path collective)"}
+
+
+def run_reference(args, w, inp, rank, world):
+    """The reference arm: the CPU oracle as it stands, rank 0 only."""
+    if rank != 0:
+        return
+    per_step_tokens = 256
+    _, _, _ = oracle_sample_rate(inp, 1e9, per_step_tokens, max_calls=args.warmup)
+    done, spent, per_call = oracle_sample_rate(inp, 1e9, per_step_tokens, max_calls=args.steps)
+    v = done / spent
+    ms = 1000.0 * spent / args.steps
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_of(w, inp, 1),
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{per_step_tokens} consecutive tokens per step "
+                                   f"(fwd + bwd), single-threaded fp64 C"},
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=workloads.BENCH_WORKLOAD,
+                    choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-budget-s", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank, local_rank, world = env_rank()
+    w = workloads.WORKLOADS[args.workload]
+    seed = workloads.seed_for(w) + 100 * rank
+    inp = workloads.make_inputs(w, seed=seed)
+    w = inp.w
+
+    if args.impl == "reference":
+        run_reference(args, w, inp, rank, world)
+        return
+
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    r = run_ours(args, w, inp, rank, local_rank, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        done, spent, _ = oracle_sample_rate(inp, args.cpu_budget_s)
+        cpu = {"value": done / spent, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+               "sample": f"{done} consecutive tokens of the workload, fwd + bwd, "
+                         f"single-threaded fp64 C, {spent:.1f} s"}
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return
+
+    cb = workloads.contract_bytes(w, with_pos=inp.pos is not None)
+    peak, peak_src = hbm_peak()
+    tokens = inp.real_tokens
+    ms = r["total_ms"] / args.steps
+    value = world * tokens / (ms / 1e3)
+    fwd_gbs = cb["fwd"] / (r["fwd_ms"] / 1e3) / 1e9
+    bwd_gbs = cb["bwd"] / (r["bwd_ms"] / 1e3) / 1e9
+    step_gbs = (cb["fwd"] + cb["bwd"]) / (ms / 1e3) / 1e9
+    lpr = 1
+    while lpr < w.D // (2 * (16 // w.elem_bytes)):
+        lpr *= 2
+    tname = "__nv_bfloat16" if w.dtype == "bf16" else "float"
+    bwd_kernel = f"qknr_bwd_kernel<{tname}, {lpr}>"
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "io_dtype": w.dtype, "data": "synthetic", "config": config_of(w, inp, world),
+        "hbm": {"fwd_gbs": fwd_gbs, "bwd_gbs": bwd_gbs, "step_gbs": step_gbs,
+                "fwd_frac": fwd_gbs / peak, "bwd_frac": bwd_gbs / peak,
+                "step_frac": step_gbs / peak, "peak_gbs": peak, "peak_source": peak_src},
+        "fwd": {"ms": r["fwd_ms"], "tokens_per_s": world * tokens / (r["fwd_ms"] / 1e3),
+                "bytes_per_launch": cb["fwd"]},
+        "bwd": {"ms": r["bwd_ms"], "tokens_per_s": world * tokens / (r["bwd_ms"] / 1e3),
+                "bytes_per_launch": cb["bwd"]},
+        "roofline": {"bound": "hbm", "kernel": bwd_kernel, "achieved": bwd_gbs, "peak": peak,
+                     "unit": "GB/s", "frac": bwd_gbs / peak,
+                     "traffic": ncu_traffic(bwd_kernel, w.name),
+                     "algorithmic_bytes": cb["bwd"], "peak_source": peak_src},
+        "clocks": r["clocks"],
+        "gpu_launches": 2 * args.steps,
+    }
+    if r["e2e"] is not None:
+        e = r["e2e"]
+        line["e2e"] = {"value": world * tokens / (e["ms"] / 1e3), "unit": "tokens/s",
+                       "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"],
+                       "ms_per_step": e["ms"], "steps": e["steps"]}
+    line["cpu_baseline"] = cpu
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,145 @@
+/*
+ * qknr.h -- fused per-head QK-RMSNorm + rotate-half RoPE for NVIDIA B200
+ * (sm_100a): forward and backward, as a plain C ABI.
+ *
+ * What it computes. Chronicals (arXiv 2601.02609), abstract, contribution
+ * (1), fuses the query/key normalisation with the rotary embedding
+ * ("QK-RoPE") so Q and K cross HBM once. For every token and every head of
+ * Q (weight gamma_q) and of K (weight gamma_k), with x the head's D values
+ * and m the token's position:
+ *
+ *   r         = 1 / sqrt(mean_d(x_d^2) + eps)       saved as fp32
+ *   n_d       = x_d * r * gamma_d
+ *   w_i       = theta^(-2i/R),  i < R/2             (R = rotary_dim)
+ *   y_i       = n_i cos(m w_i) - n_{i+R/2} sin(m w_i)
+ *   y_{i+R/2} = n_{i+R/2} cos(m w_i) + n_i sin(m w_i)
+ *   y_d       = n_d                                 for R <= d < D
+ *
+ * The per-(token, head) inverse RMS is the one statistic kept for the
+ * backward ("QK-Normed MLA: QK normalization without full key caching",
+ * abstract). Rotating only the first R < D dims is partial RoPE ("Fractional
+ * Rotation, Full Potential? Investigating Performance and Convergence of
+ * Partial RoPE", abstract); R = 0 leaves plain per-head RMSNorm (the NoPE
+ * layers of "Rope to Nope and Back Again: A New Hybrid Attention Strategy",
+ * abstract). Optional int32 position ids carry packed sequences whose
+ * positions restart per document (Chronicals, abstract, contribution (4)).
+ *
+ * Layout. Every tensor is dense and row-major, no strides:
+ *   q, q_out, dq_out, dq   [B, S, Hq,  D]     k, k_out, dk_out, dk [B, S, Hkv, D]
+ *   rstd_q [B, S, Hq] fp32, rstd_k [B, S, Hkv] fp32
+ *   gamma_q, gamma_k [D] in the I/O dtype;  dgamma_q, dgamma_k [D] fp32
+ *   pos_ids [B, S] int32, or NULL for position = s (restarting every batch row)
+ * I/O dtype is fp32 or bf16 for all of q, k, gamma, outputs and gradients;
+ * arithmetic is fp32 with fp64 rotary-angle reduction.
+ *
+ * Pointers. All pointers are device pointers (or managed memory) owned by
+ * the caller; the library allocates nothing and keeps no state between
+ * calls, so concurrent calls on different streams are safe. Vector pointers
+ * (q, k, gamma, outputs, gradients) must be 16-byte aligned; rstd, dgamma
+ * and pos_ids 4-byte aligned. An output may alias its own input exactly
+ * (q_out == q, dq == dq_out) for in-place use; any other overlap is rejected.
+ * A tensor with zero heads (Hq == 0 or Hkv == 0) may pass NULL for its
+ * pointers. B == 0 or S == 0 is an empty problem: nothing is launched except
+ * the backward's zeroing of dgamma.
+ *
+ * Asynchrony and errors. A call validates every argument on the host first;
+ * on any failure it returns a non-zero status and enqueues nothing. On
+ * success it enqueues its work on `stream` and returns without waiting; a
+ * fault during execution surfaces at the caller's next synchronisation, as
+ * for any CUDA launch. A launch the runtime refuses returns QKNR_ERR_CUDA.
+ *
+ * Limits. 2 <= D <= 256 with D * elem_bytes a multiple of 32 (two 16-byte
+ * halves per lane); rotary_dim even, 0 <= rotary_dim <= D, and
+ * (rotary_dim / 2) * elem_bytes a multiple of 16; theta finite and > 0;
+ * eps finite and >= 0. Other shapes return QKNR_ERR_UNSUPPORTED or
+ * QKNR_ERR_INVALID_ARG.
+ */
+#ifndef QKNR_H
+#define QKNR_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define QKNR_API __attribute__((visibility("default")))
+#else
+#define QKNR_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t / CUstream; NULL is the legacy default stream. */
+struct CUstream_st;
+typedef struct CUstream_st *qknr_stream_t;
+
+typedef enum {
+    QKNR_F32 = 0,  /* 4-byte IEEE float I/O */
+    QKNR_BF16 = 1  /* 2-byte bfloat16 I/O, outputs rounded to nearest even */
+} qknr_dtype;
+
+typedef enum {
+    QKNR_OK = 0,
+    QKNR_ERR_INVALID_ARG = 1, /* bad size, NULL pointer, overlap, bad theta/eps */
+    QKNR_ERR_ALIGNMENT = 2,   /* a pointer is not aligned as stated above */
+    QKNR_ERR_UNSUPPORTED = 3, /* a valid shape this build does not handle */
+    QKNR_ERR_CUDA = 4         /* the CUDA runtime refused the launch */
+} qknr_status;
+
+/*
+ * Forward: q_out/k_out = rope(rmsnorm(q|k) * gamma), rstd_q/rstd_k = r.
+ * Chronicals (arXiv 2601.02609), abstract, contribution (1).
+ *
+ *   q, k            inputs, [B,S,Hq,D] / [B,S,Hkv,D], dtype
+ *   gamma_q/gamma_k per-dim weights [D], dtype
+ *   pos_ids         [B,S] int32 positions, or NULL (position = s)
+ *   q_out, k_out    outputs, same shapes as q, k (may equal q, k)
+ *   rstd_q, rstd_k  fp32 [B,S,Hq] / [B,S,Hkv] inverse RMS, saved for bwd
+ *   B, S, Hq, Hkv, D, rotary_dim, theta, eps   as defined above
+ *   dtype           I/O element type
+ *   stream          stream to enqueue on
+ */
+QKNR_API qknr_status qk_norm_rope_fwd(const void *q, const void *k,
+                             const void *gamma_q, const void *gamma_k,
+                             const int32_t *pos_ids,
+                             void *q_out, void *k_out,
+                             float *rstd_q, float *rstd_k,
+                             int B, int S, int Hq, int Hkv, int D,
+                             int rotary_dim, float theta, float eps,
+                             qknr_dtype dtype, qknr_stream_t stream);
+
+/*
+ * Backward of qk_norm_rope_fwd. Given the forward's inputs, its saved
+ * rstd and the upstream gradients dq_out/dk_out, writes
+ *   dq, dk            gradients w.r.t. q and k (may equal dq_out, dk_out)
+ *   dgamma_q/dgamma_k fp32 [D] gradients w.r.t. gamma, OVERWRITTEN (the
+ *                     call zeroes them on `stream` first); either may be
+ *                     NULL to skip it.
+ * Per row, with g the inverse rotation of dy and xh = x * r:
+ *   dgamma_d += g_d * xh_d;   h = g * gamma;
+ *   dx = r * (h - xh * <h, xh> / D).
+ * dgamma is summed with fp32 atomics, one pass per thread block, so its
+ * last bits may differ run to run; dq and dk are bitwise reproducible.
+ */
+QKNR_API qknr_status qk_norm_rope_bwd(const void *q, const void *k,
+                             const void *gamma_q, const void *gamma_k,
+                             const int32_t *pos_ids,
+                             const float *rstd_q, const float *rstd_k,
+                             const void *dq_out, const void *dk_out,
+                             void *dq, void *dk,
+                             float *dgamma_q, float *dgamma_k,
+                             int B, int S, int Hq, int Hkv, int D,
+                             int rotary_dim, float theta, float eps,
+                             qknr_dtype dtype, qknr_stream_t stream);
+
+/* Static English text for a status code; never NULL. */
+QKNR_API const char *qknr_strerror(qknr_status status);
+
+/* The CUDA runtime error of the last QKNR_ERR_CUDA on this thread (0 if none). */
+QKNR_API int qknr_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QKNR_H */

@@ -87,8 +87,8 @@ class Oracle:
         gq, gk = as_f64(gamma_q), as_f64(gamma_k)
         Hq, D = q.shape[-2], q.shape[-1]
         Hkv = k.shape[-2]
-        T = q.size // (Hq * D)
-        m = np.ascontiguousarray(np.asarray(m, dtype=np.int64).reshape(T))
+        m = np.ascontiguousarray(np.asarray(m, dtype=np.int64).reshape(-1))
+        T = m.size
         q_out = np.empty_like(q)
         k_out = np.empty_like(k)
         rq = np.empty(q.shape[:-1], dtype=np.float64)
@@ -111,8 +111,8 @@ class Oracle:
         gq, gk = as_f64(gamma_q), as_f64(gamma_k)
         Hq, D = q.shape[-2], q.shape[-1]
         Hkv = k.shape[-2]
-        T = q.size // (Hq * D)
-        m = np.ascontiguousarray(np.asarray(m, dtype=np.int64).reshape(T))
+        m = np.ascontiguousarray(np.asarray(m, dtype=np.int64).reshape(-1))
+        T = m.size
         dq = np.empty_like(q)
         dk = np.empty_like(k)
         dgq = np.zeros(D) if dgamma_q is None else dgamma_q

@@ -1,0 +1,270 @@
+"""Fused per-head QK-RMSNorm + rotate-half RoPE for NVIDIA B200 (sm_100a).
+
+Thin ctypes binding of ``libqknr.so`` (the C ABI declared in
+``include/qknr.h``). This module only marshals arguments: it checks tensor
+metadata, allocates outputs the caller did not pass, and hands raw device
+pointers and the current CUDA stream to the library. Every step of the
+computation runs in the library's CUDA kernels; there is no fallback, and
+every entry point raises if the library is missing or a tensor is not on a
+CUDA device.
+
+Names follow the C ABI: ``qk_norm_rope_fwd`` / ``qk_norm_rope_bwd``. The
+autograd wrapper ``QKNormRoPE`` chains them for training code.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+__all__ = ["qk_norm_rope_fwd", "qk_norm_rope_bwd", "qknr_strerror", "QKNormRoPE",
+           "prepare_fwd", "prepare_bwd", "PreparedCall",
+           "qk_norm_rope", "QKNRError", "library_path", "load_library"]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libqknr.so")
+
+QKNR_OK, QKNR_ERR_INVALID_ARG, QKNR_ERR_ALIGNMENT, QKNR_ERR_UNSUPPORTED, QKNR_ERR_CUDA = range(5)
+_DTYPES = {torch.float32: 0, torch.bfloat16: 1}
+
+_lib = None
+
+
+class QKNRError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = qknr_strerror(status)
+        if status == QKNR_ERR_CUDA:
+            msg += f" (cudaError {load_library().qknr_last_cuda_error()})"
+        super().__init__(f"{where}: {msg}")
+
+
+def library_path() -> str:
+    return LIB_PATH
+
+
+def load_library():
+    """Load ``libqknr.so`` (build it with ``python -m qk_rmsnorm_rope_norm_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m qk_rmsnorm_rope_norm_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    lib.qk_norm_rope_fwd.restype = i32
+    lib.qk_norm_rope_fwd.argtypes = [vp] * 9 + [i32] * 6 + [f32, f32, i32, vp]
+    lib.qk_norm_rope_bwd.restype = i32
+    lib.qk_norm_rope_bwd.argtypes = [vp] * 13 + [i32] * 6 + [f32, f32, i32, vp]
+    lib.qknr_strerror.restype = ctypes.c_char_p
+    lib.qknr_strerror.argtypes = [i32]
+    lib.qknr_last_cuda_error.restype = i32
+    lib.qknr_last_cuda_error.argtypes = []
+    _lib = lib
+    return lib
+
+
+def qknr_strerror(status: int) -> str:
+    return load_library().qknr_strerror(int(status)).decode()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need_cuda(name: str, t: torch.Tensor):
+    if not isinstance(t, torch.Tensor) or t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _shape(q: torch.Tensor, k: torch.Tensor):
+    if q.dim() != 4 or k.dim() != 4:
+        raise ValueError("q and k must be [B, S, H, D]")
+    B, S, Hq, D = q.shape
+    if k.shape[0] != B or k.shape[1] != S or k.shape[3] != D:
+        raise ValueError(f"k shape {tuple(k.shape)} does not match q {tuple(q.shape)}")
+    return B, S, Hq, k.shape[2], D
+
+
+def qk_norm_rope_fwd(q, k, gamma_q, gamma_k, pos_ids=None, *, rotary_dim: int,
+                     theta: float, eps: float, q_out=None, k_out=None,
+                     rstd_q=None, rstd_k=None, stream=None):
+    """Forward. Returns ``(q_out, k_out, rstd_q, rstd_k)``.
+
+    q [B,S,Hq,D], k [B,S,Hkv,D] (fp32 or bf16, contiguous, CUDA); gamma_q,
+    gamma_k [D] same dtype; pos_ids optional int32 [B,S]. Outputs not given
+    are allocated; ``q_out=q`` / ``k_out=k`` runs in place.
+    """
+    lib = load_library()
+    for n, t in (("q", q), ("k", k), ("gamma_q", gamma_q), ("gamma_k", gamma_k)):
+        _need_cuda(n, t)
+    B, S, Hq, Hkv, D = _shape(q, k)
+    if q.dtype not in _DTYPES or k.dtype != q.dtype or gamma_q.dtype != q.dtype \
+            or gamma_k.dtype != q.dtype:
+        raise ValueError("q, k, gamma_q, gamma_k must share one dtype (float32 or bfloat16)")
+    if pos_ids is not None:
+        _need_cuda("pos_ids", pos_ids)
+        if pos_ids.dtype != torch.int32 or tuple(pos_ids.shape) != (B, S):
+            raise ValueError("pos_ids must be int32 [B, S]")
+    q_out = torch.empty_like(q) if q_out is None else q_out
+    k_out = torch.empty_like(k) if k_out is None else k_out
+    if rstd_q is None:
+        rstd_q = torch.empty((B, S, Hq), dtype=torch.float32, device=q.device)
+    if rstd_k is None:
+        rstd_k = torch.empty((B, S, Hkv), dtype=torch.float32, device=q.device)
+    for n, t in (("q_out", q_out), ("k_out", k_out), ("rstd_q", rstd_q), ("rstd_k", rstd_k)):
+        _need_cuda(n, t)
+    if q_out.shape != q.shape or k_out.shape != k.shape or q_out.dtype != q.dtype \
+            or k_out.dtype != q.dtype:
+        raise ValueError("q_out / k_out must match q / k in shape and dtype")
+    if rstd_q.dtype != torch.float32 or rstd_k.dtype != torch.float32 or \
+            tuple(rstd_q.shape) != (B, S, Hq) or tuple(rstd_k.shape) != (B, S, Hkv):
+        raise ValueError("rstd_q / rstd_k must be float32 [B,S,Hq] / [B,S,Hkv]")
+    st = lib.qk_norm_rope_fwd(_ptr(q), _ptr(k), _ptr(gamma_q), _ptr(gamma_k), _ptr(pos_ids),
+                              _ptr(q_out), _ptr(k_out), _ptr(rstd_q), _ptr(rstd_k),
+                              B, S, Hq, Hkv, D, int(rotary_dim), float(theta), float(eps),
+                              _DTYPES[q.dtype], _stream(stream))
+    if st != QKNR_OK:
+        raise QKNRError(st, "qk_norm_rope_fwd")
+    return q_out, k_out, rstd_q, rstd_k
+
+
+def qk_norm_rope_bwd(q, k, gamma_q, gamma_k, pos_ids, rstd_q, rstd_k, dq_out, dk_out, *,
+                     rotary_dim: int, theta: float, eps: float, dq=None, dk=None,
+                     dgamma_q=None, dgamma_k=None, need_dgamma: bool = True, stream=None):
+    """Backward. Returns ``(dq, dk, dgamma_q, dgamma_k)`` (dgamma fp32 [D]).
+
+    ``dq=dq_out`` / ``dk=dk_out`` runs in place. With ``need_dgamma=False``
+    and no dgamma buffers given, the gamma gradients are skipped (None).
+    """
+    lib = load_library()
+    for n, t in (("q", q), ("k", k), ("gamma_q", gamma_q), ("gamma_k", gamma_k),
+                 ("rstd_q", rstd_q), ("rstd_k", rstd_k), ("dq_out", dq_out), ("dk_out", dk_out)):
+        _need_cuda(n, t)
+    B, S, Hq, Hkv, D = _shape(q, k)
+    if q.dtype not in _DTYPES or any(t.dtype != q.dtype for t in (k, gamma_q, gamma_k, dq_out, dk_out)):
+        raise ValueError("q, k, gamma, dq_out, dk_out must share one dtype")
+    if dq_out.shape != q.shape or dk_out.shape != k.shape:
+        raise ValueError("dq_out / dk_out must match q / k")
+    if rstd_q.dtype != torch.float32 or rstd_k.dtype != torch.float32 or \
+            tuple(rstd_q.shape) != (B, S, Hq) or tuple(rstd_k.shape) != (B, S, Hkv):
+        raise ValueError("rstd_q / rstd_k must be float32 [B,S,Hq] / [B,S,Hkv]")
+    if pos_ids is not None:
+        _need_cuda("pos_ids", pos_ids)
+        if pos_ids.dtype != torch.int32 or tuple(pos_ids.shape) != (B, S):
+            raise ValueError("pos_ids must be int32 [B, S]")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    if need_dgamma:
+        if dgamma_q is None:
+            dgamma_q = torch.empty(D, dtype=torch.float32, device=q.device)
+        if dgamma_k is None:
+            dgamma_k = torch.empty(D, dtype=torch.float32, device=q.device)
+    for n, t in (("dq", dq), ("dk", dk)):
+        _need_cuda(n, t)
+    for n, t in (("dgamma_q", dgamma_q), ("dgamma_k", dgamma_k)):
+        if t is not None:
+            _need_cuda(n, t)
+            if t.dtype != torch.float32 or t.numel() != D:
+                raise ValueError(f"{n} must be float32 [D]")
+    st = lib.qk_norm_rope_bwd(_ptr(q), _ptr(k), _ptr(gamma_q), _ptr(gamma_k), _ptr(pos_ids),
+                              _ptr(rstd_q), _ptr(rstd_k), _ptr(dq_out), _ptr(dk_out),
+                              _ptr(dq), _ptr(dk), _ptr(dgamma_q), _ptr(dgamma_k),
+                              B, S, Hq, Hkv, D, int(rotary_dim), float(theta), float(eps),
+                              _DTYPES[q.dtype], _stream(stream))
+    if st != QKNR_OK:
+        raise QKNRError(st, "qk_norm_rope_bwd")
+    return dq, dk, dgamma_q, dgamma_k
+
+
+class QKNormRoPE(torch.autograd.Function):
+    """Autograd wrapper: forward saves q, k, gamma and rstd; backward calls
+    ``qk_norm_rope_bwd``. gamma gradients are returned in gamma's dtype."""
+
+    @staticmethod
+    def forward(ctx, q, k, gamma_q, gamma_k, pos_ids, rotary_dim, theta, eps):
+        q_out, k_out, rq, rk = qk_norm_rope_fwd(q, k, gamma_q, gamma_k, pos_ids,
+                                                rotary_dim=rotary_dim, theta=theta, eps=eps)
+        ctx.save_for_backward(q, k, gamma_q, gamma_k, rq, rk)
+        ctx.pos_ids = pos_ids
+        ctx.cfg = (rotary_dim, theta, eps)
+        ctx.mark_non_differentiable(rq, rk)
+        return q_out, k_out
+
+    @staticmethod
+    def backward(ctx, dq_out, dk_out):
+        q, k, gq, gk, rq, rk = ctx.saved_tensors
+        R, theta, eps = ctx.cfg
+        dq, dk, dgq, dgk = qk_norm_rope_bwd(
+            q, k, gq, gk, ctx.pos_ids, rq, rk, dq_out.contiguous(), dk_out.contiguous(),
+            rotary_dim=R, theta=theta, eps=eps,
+            need_dgamma=ctx.needs_input_grad[2] or ctx.needs_input_grad[3])
+        dgq = None if dgq is None else dgq.to(gq.dtype)
+        dgk = None if dgk is None else dgk.to(gk.dtype)
+        return dq, dk, dgq, dgk, None, None, None, None
+
+
+def qk_norm_rope(q, k, gamma_q, gamma_k, pos_ids=None, *, rotary_dim: int, theta: float,
+                 eps: float):
+    """Differentiable fused op; returns ``(q_out, k_out)``."""
+    return QKNormRoPE.apply(q, k, gamma_q, gamma_k, pos_ids, rotary_dim, theta, eps)
+
+
+class PreparedCall:
+    """A C ABI call with every argument marshalled once.
+
+    ``prepare_fwd`` / ``prepare_bwd`` check the tensors exactly like
+    ``qk_norm_rope_fwd`` / ``qk_norm_rope_bwd`` and keep the ctypes argument
+    tuple, so each later ``call()`` is a single foreign call (for tight loops
+    such as benchmarks). The tensors must stay alive and unchanged in shape.
+    """
+
+    def __init__(self, fn, args, name, keep):
+        self._fn, self._args, self._name, self._keep = fn, args, name, keep
+
+    def __call__(self):
+        st = self._fn(*self._args)
+        if st != QKNR_OK:
+            raise QKNRError(st, self._name)
+
+
+def prepare_fwd(q, k, gamma_q, gamma_k, pos_ids, q_out, k_out, rstd_q, rstd_k, *,
+                rotary_dim, theta, eps, stream=None) -> PreparedCall:
+    lib = load_library()
+    # one checked call validates the tensors (and runs the op once)
+    qk_norm_rope_fwd(q, k, gamma_q, gamma_k, pos_ids, rotary_dim=rotary_dim, theta=theta,
+                     eps=eps, q_out=q_out, k_out=k_out, rstd_q=rstd_q, rstd_k=rstd_k,
+                     stream=stream)
+    B, S, Hq, Hkv, D = _shape(q, k)
+    args = (_ptr(q), _ptr(k), _ptr(gamma_q), _ptr(gamma_k), _ptr(pos_ids), _ptr(q_out),
+            _ptr(k_out), _ptr(rstd_q), _ptr(rstd_k), B, S, Hq, Hkv, D, int(rotary_dim),
+            float(theta), float(eps), _DTYPES[q.dtype], _stream(stream))
+    keep = (q, k, gamma_q, gamma_k, pos_ids, q_out, k_out, rstd_q, rstd_k)
+    return PreparedCall(lib.qk_norm_rope_fwd, args, "qk_norm_rope_fwd", keep)
+
+
+def prepare_bwd(q, k, gamma_q, gamma_k, pos_ids, rstd_q, rstd_k, dq_out, dk_out, dq, dk,
+                dgamma_q, dgamma_k, *, rotary_dim, theta, eps, stream=None) -> PreparedCall:
+    lib = load_library()
+    qk_norm_rope_bwd(q, k, gamma_q, gamma_k, pos_ids, rstd_q, rstd_k, dq_out, dk_out,
+                     rotary_dim=rotary_dim, theta=theta, eps=eps, dq=dq, dk=dk,
+                     dgamma_q=dgamma_q, dgamma_k=dgamma_k, stream=stream)
+    B, S, Hq, Hkv, D = _shape(q, k)
+    args = (_ptr(q), _ptr(k), _ptr(gamma_q), _ptr(gamma_k), _ptr(pos_ids), _ptr(rstd_q),
+            _ptr(rstd_k), _ptr(dq_out), _ptr(dk_out), _ptr(dq), _ptr(dk), _ptr(dgamma_q),
+            _ptr(dgamma_k), B, S, Hq, Hkv, D, int(rotary_dim), float(theta), float(eps),
+            _DTYPES[q.dtype], _stream(stream))
+    keep = (q, k, gamma_q, gamma_k, pos_ids, rstd_q, rstd_k, dq_out, dk_out, dq, dk,
+            dgamma_q, dgamma_k)
+    return PreparedCall(lib.qk_norm_rope_bwd, args, "qk_norm_rope_bwd", keep)

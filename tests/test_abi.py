@@ -1,0 +1,129 @@
+"""The C ABI library: it loads, exports every symbol include/qknr.h declares,
+and rejects bad arguments on the host before touching the GPU.
+
+No GPU is needed: every call here fails validation, which happens before any
+CUDA runtime call. The pointers are fake addresses that are never
+dereferenced.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import qk_rmsnorm_rope_norm_b200 as qknr
+from qk_rmsnorm_rope_norm_b200 import build as qbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qknr.h")
+
+OK, INVALID, ALIGN, UNSUP, CUDA = range(5)
+F32, BF16 = 0, 1
+
+
+@pytest.fixture(scope="module")
+def lib():
+    qbuild.build()
+    return qknr.load_library()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"#define QKNR_API.*", "", src)
+    return re.findall(r"QKNR_API\s+[\w\s\*]*?\b(\w+)\s*\(", src)
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("qk_norm_rope_fwd", "qk_norm_rope_bwd", "qknr_strerror", "qknr_last_cuda_error"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for n in declared_functions():
+        assert hasattr(lib, n), f"{n} declared in qknr.h but not exported"
+
+
+def test_library_is_sm100a_only():
+    assert "arch=compute_100a,code=sm_100a" in " ".join(qbuild.NVCC_FLAGS)
+    assert "sm_90" not in " ".join(qbuild.NVCC_FLAGS)
+
+
+def test_strerror_covers_every_status(lib):
+    for s in range(5):
+        assert len(qknr.qknr_strerror(s)) > 5
+    assert qknr.qknr_strerror(99) == "unknown status"
+
+
+# fake, 256-aligned, well separated device addresses (never dereferenced)
+def P(i, off=0):
+    return ctypes.c_void_p(0x7f0000000000 + i * (1 << 32) + off)
+
+
+def fwd(lib, B=2, S=8, Hq=4, Hkv=2, D=64, R=64, theta=1e4, eps=1e-6, dt=BF16, **ptrs):
+    p = dict(q=P(1), k=P(2), gq=P(3), gk=P(4), pos=None, qo=P(5), ko=P(6), rq=P(7), rk=P(8))
+    p.update(ptrs)
+    return lib.qk_norm_rope_fwd(p["q"], p["k"], p["gq"], p["gk"], p["pos"], p["qo"], p["ko"],
+                                p["rq"], p["rk"], B, S, Hq, Hkv, D, R, theta, eps, dt, None)
+
+
+def bwd(lib, B=2, S=8, Hq=4, Hkv=2, D=64, R=64, theta=1e4, eps=1e-6, dt=BF16, **ptrs):
+    p = dict(q=P(1), k=P(2), gq=P(3), gk=P(4), pos=None, rq=P(7), rk=P(8), dqo=P(9),
+             dko=P(10), dq=P(11), dk=P(12), dgq=P(13), dgk=P(14))
+    p.update(ptrs)
+    return lib.qk_norm_rope_bwd(p["q"], p["k"], p["gq"], p["gk"], p["pos"], p["rq"], p["rk"],
+                                p["dqo"], p["dko"], p["dq"], p["dk"], p["dgq"], p["dgk"],
+                                B, S, Hq, Hkv, D, R, theta, eps, dt, None)
+
+
+@pytest.mark.parametrize("call", [fwd, bwd], ids=["fwd", "bwd"])
+@pytest.mark.parametrize("kw,want", [
+    (dict(B=-1), INVALID), (dict(S=-3), INVALID), (dict(Hq=-1), INVALID),
+    (dict(D=0), INVALID), (dict(D=63), INVALID), (dict(R=66), INVALID),
+    (dict(R=-2), INVALID), (dict(R=31), INVALID), (dict(theta=0.0), INVALID),
+    (dict(theta=float("inf")), INVALID), (dict(theta=float("nan")), INVALID),
+    (dict(eps=-1e-6), INVALID), (dict(eps=float("nan")), INVALID), (dict(dt=7), INVALID),
+    (dict(D=512, R=512), UNSUP), (dict(D=72, R=72), UNSUP), (dict(D=64, R=8), UNSUP),
+])
+def test_shape_validation(lib, call, kw, want):
+    assert call(lib, **kw) == want
+
+
+@pytest.mark.parametrize("call", [fwd, bwd], ids=["fwd", "bwd"])
+def test_null_and_alignment(lib, call):
+    assert call(lib, q=None) == INVALID
+    assert call(lib, k=None) == INVALID
+    assert call(lib, gq=None) == INVALID
+    assert call(lib, rq=None) == INVALID
+    assert call(lib, q=P(1, 8)) == ALIGN          # vectors need 16 bytes
+    assert call(lib, gk=P(4, 4)) == ALIGN
+    assert call(lib, rk=P(8, 2)) == ALIGN         # fp32 arrays need 4 bytes
+    assert call(lib, pos=P(15, 1)) == ALIGN
+
+
+def test_fwd_overlap_rules(lib):
+    # B*S*Hq*D*2 bytes = 2*8*4*64*2 = 8 KiB per q tensor
+    assert fwd(lib, qo=P(1, 4096)) == INVALID          # partial overlap with q
+    assert fwd(lib, ko=P(5)) == INVALID                # k_out on top of q_out
+    assert fwd(lib, rq=P(5, 64)) == INVALID            # rstd inside q_out
+    assert fwd(lib, qo=P(2), ko=P(1)) == INVALID       # outputs swapped onto inputs
+
+
+def test_bwd_overlap_rules(lib):
+    assert bwd(lib, dq=P(9, 16)) == INVALID            # partial overlap with dq_out
+    assert bwd(lib, dgq=P(11, 32)) == INVALID          # dgamma inside dq
+    assert bwd(lib, dgq=P(13), dgk=P(13)) == INVALID   # both dgammas on one buffer
+    assert bwd(lib, dq=P(1)) == INVALID                # dq on top of q
+
+
+def test_zero_heads_allow_null_pointers(lib):
+    # Hkv = 0: K pointers may be NULL, but an invalid D still fails first
+    assert fwd(lib, Hkv=0, k=None, gk=None, ko=None, rk=None, D=63) == INVALID
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    q = torch.zeros(1, 2, 1, 16)
+    with pytest.raises(ValueError):
+        qknr.qk_norm_rope_fwd(q, q, q[0, 0, 0], q[0, 0, 0], rotary_dim=16, theta=1e4, eps=1e-6)
