@@ -138,6 +138,14 @@ QKNR_API const char *qknr_strerror(qknr_status status);
 /* The CUDA runtime error of the last QKNR_ERR_CUDA on this thread (0 if none). */
 QKNR_API int qknr_last_cuda_error(void);
 
+/*
+ * Diagnostic flag of the current device's pipelined kernels: non-zero if
+ * a kernel gave up an internal wait (bounded at 2 s; the results of that
+ * launch are then incomplete). Synchronises with the device. With reset
+ * != 0 the flag is cleared. Returns -1 if the flag cannot be read.
+ */
+QKNR_API int qknr_pipeline_error(int reset);
+
 #ifdef __cplusplus
 }
 #endif

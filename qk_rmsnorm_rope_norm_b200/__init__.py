@@ -21,7 +21,7 @@ import torch
 
 __all__ = ["qk_norm_rope_fwd", "qk_norm_rope_bwd", "qknr_strerror", "QKNormRoPE",
            "prepare_fwd", "prepare_bwd", "PreparedCall",
-           "qk_norm_rope", "QKNRError", "library_path", "load_library"]
+           "qk_norm_rope", "QKNRError", "library_path", "load_library", "pipeline_error"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libqknr.so")
@@ -63,12 +63,20 @@ def load_library():
     lib.qknr_strerror.argtypes = [i32]
     lib.qknr_last_cuda_error.restype = i32
     lib.qknr_last_cuda_error.argtypes = []
+    lib.qknr_pipeline_error.restype = i32
+    lib.qknr_pipeline_error.argtypes = [i32]
     _lib = lib
     return lib
 
 
 def qknr_strerror(status: int) -> str:
     return load_library().qknr_strerror(int(status)).decode()
+
+
+def pipeline_error(reset: bool = False) -> int:
+    """Non-zero if a pipelined kernel on the current device gave up a bounded
+    internal wait since the flag was last cleared (synchronises)."""
+    return int(load_library().qknr_pipeline_error(1 if reset else 0))
 
 
 def _ptr(t: Optional[torch.Tensor]):

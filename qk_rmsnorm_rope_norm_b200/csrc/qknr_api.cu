@@ -2,11 +2,12 @@
 // launch geometry and dispatch to the sm_100a kernels in qknr_kernels.cuh.
 // Declarations and the full contract are in include/qknr.h.
 #include "qknr.h"
-#include "qknr_kernels.cuh"
+#include "qknr_pipe.cuh"
 
 #include <atomic>
 #include <cmath>
 #include <cstdint>
+#include <cstdlib>
 
 namespace qknr {
 namespace {
@@ -108,6 +109,198 @@ void geometry(const void *kernel, std::atomic<int> *cache, int64_t T, int *grid,
     *grid = (int)((warps + kWarps - 1) / kWarps);
 }
 
+// ------------------------------------------------------------ pipelined
+#ifndef QKNR_FWD_PIPE_WARPS
+#define QKNR_FWD_PIPE_WARPS 16
+#endif
+#ifndef QKNR_BWD_PIPE_WARPS
+#define QKNR_BWD_PIPE_WARPS 16
+#endif
+#ifndef QKNR_PRODUCER_WARPS
+#define QKNR_PRODUCER_WARPS 4
+#endif
+constexpr int kFwdPipeWarps = QKNR_FWD_PIPE_WARPS;  // consumer warps per CTA
+constexpr int kBwdPipeWarps = QKNR_BWD_PIPE_WARPS;
+constexpr int kProducerWarps = QKNR_PRODUCER_WARPS;  // copy issue + rotary tables
+constexpr int kStageTargetBytes = 24576; // aim for ~24 KB of rows per stage
+constexpr int kStaticSmemReserve = 8192; // barriers, omega, gamma, dgamma tables
+
+int align128(int x) { return (x + 127) & ~127; }
+
+int max_dyn_smem(int dev) {
+    static std::atomic<int> cache[64];
+    if (dev >= 0 && dev < 64) {
+        int c = cache[dev].load(std::memory_order_relaxed);
+        if (c > 0) return c;
+    }
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+        n = 48 * 1024;
+    if (dev >= 0 && dev < 64) cache[dev].store(n, std::memory_order_relaxed);
+    return n;
+}
+
+// Tile and ring sizes for one problem; false when the pipelined kernels do
+// not apply (a token too large for two stages, or unaligned rstd buffers).
+bool pipe_geometry(bool bwd, int64_t T, int Hq, int Hkv, int D, int R, int esz, int dev,
+                   const void *rq, const void *rk, PipeGeom *g, int *grid, int *smem) {
+    const int rowb = D * esz, H = Hq + Hkv, half = R / 2;
+    if (bwd && ((rq && ((uintptr_t)rq & 15)) || (rk && ((uintptr_t)rk & 15)))) return false;
+    // backward tiles must start rstd blocks on 16-byte boundaries
+    int m = 1;
+    if (bwd) {
+        while ((m * Hq) % 4 || (m * Hkv) % 4) m <<= 1;  // m in {1, 2, 4}
+    }
+    const int per_tok = (bwd ? 2 : 1) * H * rowb;
+    int TT = kStageTargetBytes / (per_tok > 0 ? per_tok : 1);
+    TT = TT < 1 ? 1 : (TT > kMaxTileTokens ? kMaxTileTokens : TT);
+    TT = ((TT + m - 1) / m) * m;
+    if (TT > kMaxTileTokens) TT = kMaxTileTokens;  // a multiple of 4 already
+    if (T < TT) TT = (int)(((T + m - 1) / m) * m);
+    PipeGeom q{};
+    q.TT = TT;
+    int off = align128(TT * Hq * rowb);
+    q.off_k = off;
+    off = align128(off + TT * Hkv * rowb);
+    if (bwd) {
+        q.off_dq = off;
+        off = align128(off + TT * Hq * rowb);
+        q.off_dk = off;
+        off = align128(off + TT * Hkv * rowb);
+    }
+    q.off_cs = off;
+    off = align128(off + TT * half * 8);
+    if (bwd) {
+        q.off_rq = off;
+        off = align128(off + TT * Hq * 4);
+        q.off_rk = off;
+        off = align128(off + TT * Hkv * 4);
+    }
+    q.stage_bytes = off > 0 ? off : 128;
+    const int budget = max_dyn_smem(dev) - kStaticSmemReserve;
+    int NS = budget / q.stage_bytes;
+    if (NS > kMaxStages) NS = kMaxStages;
+    if (NS < 2) return false;
+    q.NS = NS;
+    // one CTA per SM; each owns a contiguous run of tokens (a multiple of m)
+    const int64_t sms = sm_count(dev);
+    int64_t tpc = (T + sms - 1) / sms;
+    tpc = ((tpc + m - 1) / m) * m;
+    if (tpc < 1) tpc = 1;
+    q.tpc = tpc;
+    q.mq = Hq > 1 ? (uint32_t)(0x100000000ull / (uint64_t)Hq + 1) : 0u;
+    q.mk = Hkv > 1 ? (uint32_t)(0x100000000ull / (uint64_t)Hkv + 1) : 0u;
+    *grid = (int)((T + tpc - 1) / tpc);
+    *smem = NS * q.stage_bytes;
+    *g = q;
+    return true;
+}
+
+bool allow_dyn_smem(const void *kernel, int dev, std::atomic<int> *cache, int bytes) {
+    if (dev < 0 || dev >= 64) return false;
+    if (cache[dev].load(std::memory_order_relaxed) >= bytes) return true;
+    const int want = max_dyn_smem(dev) - kStaticSmemReserve;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, want) !=
+        cudaSuccess)
+        return false;
+    cache[dev].store(want, std::memory_order_relaxed);
+    return want >= bytes;
+}
+
+bool pipe_disabled() {
+    const char *e = std::getenv("QKNR_SIMPLE_KERNELS");
+    return e && e[0] == '1';
+}
+
+template <typename T, int LPR, int U>
+qknr_status launch_fwd_pipe(const FwdArgs &a, const PipeGeom &g, int grid, int smem, int dev,
+                            cudaStream_t st, bool *launched) {
+    static std::atomic<int> smem_ok[64];
+    auto kern = qknr_fwd_pipe_kernel<T, LPR, U, kFwdPipeWarps, kProducerWarps>;
+    *launched = false;
+    if (!allow_dyn_smem((const void *)kern, dev, smem_ok, smem)) return QKNR_OK;
+    *launched = true;
+    kern<<<grid, (kFwdPipeWarps + kProducerWarps) * 32, smem, st>>>(a, g);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? QKNR_OK : cuda_fail(e);
+}
+
+template <typename T, int LPR>
+qknr_status launch_bwd_pipe(const BwdArgs &a, const PipeGeom &g, int grid, int smem, int dev,
+                            cudaStream_t st, bool *launched) {
+    static std::atomic<int> smem_ok[64];
+    auto kern = qknr_bwd_pipe_kernel<T, LPR, kBwdPipeWarps, kProducerWarps>;
+    *launched = false;
+    if (!allow_dyn_smem((const void *)kern, dev, smem_ok, smem)) return QKNR_OK;
+    *launched = true;
+    kern<<<grid, (kBwdPipeWarps + kProducerWarps) * 32, smem, st>>>(a, g);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? QKNR_OK : cuda_fail(e);
+}
+
+int next_pow2(int x) {
+    int l = 1;
+    while (l < x) l <<= 1;
+    return l;
+}
+
+// Pipelined forward when it applies: two units per lane once a row has
+// three or more (halving the per-row overhead per element).
+template <typename T>
+bool try_fwd_pipe(const FwdArgs &a, cudaStream_t st, qknr_status *status) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    PipeGeom g;
+    int grid, smem;
+    if (pipe_disabled() ||
+        !pipe_geometry(false, a.T, a.Hq, a.Hkv, a.D, a.R, (int)sizeof(T), dev, nullptr, nullptr,
+                       &g, &grid, &smem))
+        return false;
+    const int dv2 = a.D / (2 * (16 / (int)sizeof(T)));
+    bool launched = false;
+    qknr_status s = QKNR_OK;
+    if (dv2 >= 3) {
+        switch (next_pow2((dv2 + 1) / 2)) {
+            case 2: s = launch_fwd_pipe<T, 2, 2>(a, g, grid, smem, dev, st, &launched); break;
+            case 4: s = launch_fwd_pipe<T, 4, 2>(a, g, grid, smem, dev, st, &launched); break;
+            case 8: s = launch_fwd_pipe<T, 8, 2>(a, g, grid, smem, dev, st, &launched); break;
+            case 16: s = launch_fwd_pipe<T, 16, 2>(a, g, grid, smem, dev, st, &launched); break;
+        }
+    } else {
+        switch (next_pow2(dv2)) {
+            case 1: s = launch_fwd_pipe<T, 1, 1>(a, g, grid, smem, dev, st, &launched); break;
+            case 2: s = launch_fwd_pipe<T, 2, 1>(a, g, grid, smem, dev, st, &launched); break;
+        }
+    }
+    *status = s;
+    return launched;
+}
+
+template <typename T>
+bool try_bwd_pipe(const BwdArgs &a, cudaStream_t st, qknr_status *status) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    PipeGeom g;
+    int grid, smem;
+    if (pipe_disabled() ||
+        !pipe_geometry(true, a.T, a.Hq, a.Hkv, a.D, a.R, (int)sizeof(T), dev, a.rq, a.rk, &g,
+                       &grid, &smem))
+        return false;
+    const int dv2 = a.D / (2 * (16 / (int)sizeof(T)));
+    bool launched = false;
+    qknr_status s = QKNR_OK;
+    switch (next_pow2(dv2)) {
+        case 1: s = launch_bwd_pipe<T, 1>(a, g, grid, smem, dev, st, &launched); break;
+        case 2: s = launch_bwd_pipe<T, 2>(a, g, grid, smem, dev, st, &launched); break;
+        case 4: s = launch_bwd_pipe<T, 4>(a, g, grid, smem, dev, st, &launched); break;
+        case 8: s = launch_bwd_pipe<T, 8>(a, g, grid, smem, dev, st, &launched); break;
+        case 16: s = launch_bwd_pipe<T, 16>(a, g, grid, smem, dev, st, &launched); break;
+        case 32: s = launch_bwd_pipe<T, 32>(a, g, grid, smem, dev, st, &launched); break;
+    }
+    *status = s;
+    return launched;
+}
+
 template <typename T, int LPR>
 qknr_status launch_fwd(FwdArgs a, cudaStream_t st) {
     static std::atomic<int> occ[64];
@@ -134,6 +327,8 @@ qknr_status launch_bwd(BwdArgs a, cudaStream_t st) {
 
 template <typename T>
 qknr_status dispatch_fwd(const FwdArgs &a, int lpr, cudaStream_t st) {
+    qknr_status ps;
+    if (try_fwd_pipe<T>(a, st, &ps)) return ps;
     switch (lpr) {
         case 1: return launch_fwd<T, 1>(a, st);
         case 2: return launch_fwd<T, 2>(a, st);
@@ -147,6 +342,8 @@ qknr_status dispatch_fwd(const FwdArgs &a, int lpr, cudaStream_t st) {
 
 template <typename T>
 qknr_status dispatch_bwd(const BwdArgs &a, int lpr, cudaStream_t st) {
+    qknr_status ps;
+    if (try_bwd_pipe<T>(a, st, &ps)) return ps;
     switch (lpr) {
         case 1: return launch_bwd<T, 1>(a, st);
         case 2: return launch_bwd<T, 2>(a, st);
@@ -276,3 +473,14 @@ extern "C" const char *qknr_strerror(qknr_status s) {
 }
 
 extern "C" int qknr_last_cuda_error(void) { return g_last_cuda_error; }
+
+extern "C" int qknr_pipeline_error(int reset) {
+    unsigned int v = 0;
+    if (cudaMemcpyFromSymbol(&v, qknr::g_qknr_pipe_error, sizeof(v)) != cudaSuccess) return -1;
+    if (reset && v) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(qknr::g_qknr_pipe_error, &zero, sizeof(zero)) != cudaSuccess)
+            return -1;
+    }
+    return (int)v;
+}

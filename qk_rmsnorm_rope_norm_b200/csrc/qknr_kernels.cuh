@@ -155,7 +155,22 @@ __device__ __forceinline__ void fill_tables(double *s_omega, float (*s_g)[kMaxD]
     }
 }
 
-// Lane geometry for a head row of D elements, R rotary, V elements / vector.
+// Geometry of unit w of a head row of D elements (R rotary, V elements per
+// 16-byte vector): the element offsets of its two vectors. Units past the
+// row (D / 2V not a power of two) are off and point at element 0.
+template <int V> struct UnitGeom {
+    bool on, rot;
+    int eA, eB;
+    __device__ __forceinline__ UnitGeom(int w, int D, int R) {
+        const int Dv2 = D / (2 * V), Rv2 = R / (2 * V);
+        on = w < Dv2;
+        rot = w < Rv2;
+        eA = on ? (rot ? w : w + Rv2) * V : 0;
+        eB = on ? (rot ? w + Rv2 : w + Dv2) * V : 0;
+    }
+};
+
+// Lane geometry: LPR lanes per row, lane u of the group owns unit u.
 template <int LPR, int V> struct Lane {
     int u, slot;
     bool on, rot;
@@ -163,11 +178,11 @@ template <int LPR, int V> struct Lane {
     __device__ __forceinline__ Lane(int lane, int D, int R) {
         u = lane & (LPR - 1);
         slot = lane / LPR;
-        const int Dv2 = D / (2 * V), Rv2 = R / (2 * V);
-        on = u < Dv2;
-        rot = u < Rv2;
-        eA = (rot ? u : u + Rv2) * V;
-        eB = (rot ? u + Rv2 : u + Dv2) * V;
+        const UnitGeom<V> G(u, D, R);
+        on = G.on;
+        rot = G.rot;
+        eA = G.eA;
+        eB = G.eB;
     }
 };
 
@@ -274,8 +289,9 @@ qknr_fwd_kernel(const FwdArgs a) {
                         const int e = 2 * k2;
                         const float2 c0 = lane_cs(cs, L.rot, L.eA + e);
                         const float2 c1 = lane_cs(cs, L.rot, L.eA + e + 1);
-                        const float na0 = va.x * r * g[L.eA + e], na1 = va.y * r * g[L.eA + e + 1];
-                        const float nb0 = vb.x * r * g[L.eB + e], nb1 = vb.y * r * g[L.eB + e + 1];
+                        // n = (x * gamma) * r, the order the pipelined kernel uses
+                        const float na0 = va.x * g[L.eA + e] * r, na1 = va.y * g[L.eA + e + 1] * r;
+                        const float nb0 = vb.x * g[L.eB + e] * r, nb1 = vb.y * g[L.eB + e + 1] * r;
                         IO::put2(ya, k2, fmaf(na0, c0.x, -nb0 * c0.y), fmaf(na1, c1.x, -nb1 * c1.y));
                         IO::put2(yb, k2, fmaf(nb0, c0.x, na0 * c0.y), fmaf(nb1, c1.x, na1 * c1.y));
                     }

@@ -158,7 +158,7 @@ def test_explicit_positions_equal_default(cuda):
 def test_packing_boundaries_and_pass_through(cuda):
     """Exact identities of the kernel, checked bitwise against a host
     recomputation from the kernel's own rstd: at doc starts (position 0)
-    every dim of the output is (x * r) * gamma rounded once to bf16, and
+    every dim of the output is (x * gamma) * r rounded once to bf16, and
     in a partial rotary layout so is every dim >= R at every position;
     padding slots stay zero."""
     inp = workloads.make_inputs("bfd-packed", rotary_dim=32)
@@ -168,7 +168,7 @@ def test_packing_boundaries_and_pass_through(cuda):
     assert int(starts.sum()) == len(inp.doc_lengths)
     for x, g, name, rname in ((inp.q, inp.gamma_q, "q_out", "rstd_q"),
                               (inp.k, inp.gamma_k, "k_out", "rstd_k")):
-        n = ((x.float() * got[rname].unsqueeze(-1)) * g.float()).to(torch.bfloat16)
+        n = ((x.float() * g.float()) * got[rname].unsqueeze(-1)).to(torch.bfloat16)
         assert torch.equal(got[name][starts], n[starts]), f"{name} at doc starts"
         R = w.rotary_dim
         assert torch.equal(got[name][..., R:], n[..., R:]), f"{name} pass-through dims"
@@ -244,8 +244,9 @@ def test_autograd_wrapper(cuda):
     got = parity.gpu_run(inp)
     assert torch.equal(qo.detach().cpu(), got["q_out"])
     assert torch.equal(q.grad.cpu(), got["dq"]) and torch.equal(k.grad.cpu(), got["dk"])
-    torch.testing.assert_close(gq.grad.cpu(), got["dgamma_q"], rtol=1e-6, atol=1e-6)
-    torch.testing.assert_close(gk.grad.cpu(), got["dgamma_k"], rtol=1e-6, atol=1e-6)
+    # dgamma is summed with atomics in a run-dependent order: normwise check
+    for a_, b_ in ((gq.grad.cpu(), got["dgamma_q"]), (gk.grad.cpu(), got["dgamma_k"])):
+        assert float((a_ - b_).abs().max()) <= 1e-5 * float(b_.abs().max())
 
 
 def test_side_stream_and_graph_capture(cuda):
@@ -277,4 +278,51 @@ def test_side_stream_and_graph_capture(cuda):
     g.replay()
     torch.cuda.synchronize()
     assert torch.equal(qo.cpu(), ref["q_out"]) and torch.equal(dq.cpu(), ref["dq"])
-    torch.testing.assert_close(dgq.cpu(), ref["dgamma_q"], rtol=1e-5, atol=1e-5)
+    assert float((dgq.cpu() - ref["dgamma_q"]).abs().max()) <= 1e-5 * float(ref["dgamma_q"].abs().max())
+
+
+# ------------------------------------------------- simple (fallback) kernels
+@pytest.fixture
+def simple_kernels():
+    import os
+    os.environ["QKNR_SIMPLE_KERNELS"] = "1"
+    yield
+    del os.environ["QKNR_SIMPLE_KERNELS"]
+
+
+@pytest.mark.parametrize("dtype,D,R", [("bf16", 64, 64), ("bf16", 128, 32), ("bf16", 80, 16),
+                                       ("f32", 24, 16), ("f32", 128, 128)])
+def test_simple_kernels_shape_sweep(cuda, simple_kernels, dtype, D, R):
+    inp = sweep_inputs(dtype, D, R)
+    parity.check(inp, parity.gpu_run(inp))
+
+
+def test_simple_kernels_exact_identities(cuda, simple_kernels):
+    test_packing_boundaries_and_pass_through(cuda)
+
+
+def test_simple_kernels_bench_workload(cuda, simple_kernels):
+    inp = workloads.make_inputs(workloads.BENCH_WORKLOAD)
+    parity.check(inp, parity.gpu_run(inp))
+
+
+def test_simple_and_pipelined_agree(cuda):
+    """Both kernel families compute the same arithmetic; outputs agree to
+    within the rounding of the fp32 sum-of-squares order (1 bf16 ulp)."""
+    import os
+    inp = workloads.make_inputs("partial-rope-64k", B=1, S=5000)
+    a = parity.gpu_run(inp)
+    os.environ["QKNR_SIMPLE_KERNELS"] = "1"
+    try:
+        b = parity.gpu_run(inp)
+    finally:
+        del os.environ["QKNR_SIMPLE_KERNELS"]
+    for n in ("q_out", "k_out", "dq", "dk"):
+        d = (a[n].double() - b[n].double()).abs()
+        ulp = torch.from_numpy(parity.bf16_ulp(b[n].double().numpy()))
+        assert float((d / torch.clamp(ulp, min=1e-5)).max()) <= 1.0, n
+    torch.testing.assert_close(a["rstd_q"], b["rstd_q"], rtol=1e-5, atol=0)
+
+
+def test_no_pipeline_timeouts(cuda):
+    assert qknr.pipeline_error() == 0
