@@ -44,6 +44,7 @@ METRIC = "QK-norm+RoPE fwd+bwd tokens/s and HBM GB/s (% of B200 peak), 1 GPU"
 FALLBACK_HBM_GBS = 6650.0
 NSETS, LAG = 4, 2
 KERNEL_SOURCES = ["qk_rmsnorm_rope_norm_b200/csrc/qknr_kernels.cuh",
+                  "qk_rmsnorm_rope_norm_b200/csrc/qknr_pipe.cuh",
                   "qk_rmsnorm_rope_norm_b200/csrc/qknr_api.cu"]
 
 
@@ -236,8 +237,32 @@ def run_ours(args, w, inp, rank, local_rank, world):
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(args, w, inp, dev, cfg, world)
+    cb = workloads.contract_bytes(w, with_pos=inp.pos is not None)
+    floor = {"fwd_ms": copy_floor_ms(cb["fwd"], dev), "bwd_ms": copy_floor_ms(cb["bwd"], dev)}
     return dict(total_ms=total_ms, fwd_ms=fwd_ms, bwd_ms=bwd_ms, clocks=clocks.summary(),
-                e2e=e2e)
+                e2e=e2e, floor=floor)
+
+
+def copy_floor_ms(traffic_bytes: int, dev, n: int = 20) -> float:
+    """Median time of a device-to-device copy moving the same DRAM bytes
+    (traffic/2 read + traffic/2 written), each launch after an L2 flush:
+    the practical floor for a single launch of that size on this GPU."""
+    half = max(16, traffic_bytes // 2) // 2 * 2
+    src = torch.empty(half // 2, dtype=torch.bfloat16, device=dev)
+    dst = torch.empty_like(src)
+    flush = torch.empty(256 * 1024 * 1024 // 4, device=dev)
+    ts = []
+    for i in range(n + 3):
+        flush.fill_(float(i))
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        dst.copy_(src)
+        b.record()
+        torch.cuda.synchronize(dev)
+        if i >= 3:
+            ts.append(a.elapsed_time(b))
+    del src, dst, flush
+    return statistics.median(ts)
 
 
 def run_e2e(args, w, inp, dev, cfg, world):
@@ -412,7 +437,14 @@ def main():
         "io_dtype": w.dtype, "data": "synthetic", "config": config_of(w, inp, world),
         "hbm": {"fwd_gbs": fwd_gbs, "bwd_gbs": bwd_gbs, "step_gbs": step_gbs,
                 "fwd_frac": fwd_gbs / peak, "bwd_frac": bwd_gbs / peak,
-                "step_frac": step_gbs / peak, "peak_gbs": peak, "peak_source": peak_src},
+                "step_frac": step_gbs / peak, "peak_gbs": peak, "peak_source": peak_src,
+                "copy_floor": {
+                    "what": "torch copy_ moving the same DRAM bytes, one launch after an "
+                            "L2 flush (the practical floor at this size)",
+                    "fwd_gbs": cb["fwd"] / (r["floor"]["fwd_ms"] / 1e3) / 1e9,
+                    "bwd_gbs": cb["bwd"] / (r["floor"]["bwd_ms"] / 1e3) / 1e9,
+                    "fwd_frac_of_copy": r["floor"]["fwd_ms"] / r["fwd_ms"],
+                    "bwd_frac_of_copy": r["floor"]["bwd_ms"] / r["bwd_ms"]}},
         "fwd": {"ms": r["fwd_ms"], "tokens_per_s": world * tokens / (r["fwd_ms"] / 1e3),
                 "bytes_per_launch": cb["fwd"]},
         "bwd": {"ms": r["bwd_ms"], "tokens_per_s": world * tokens / (r["bwd_ms"] / 1e3),

@@ -22,10 +22,10 @@
 // registers hold gamma, the row and the dgamma partial sums in fp32, with
 // packed FP32x2 arithmetic (FFMA2/FMUL2) on element pairs.
 //
-// Every mbarrier wait is bounded by a wall-clock limit (%globaltimer); on
-// expiry the thread records an error in g_qknr_pipe_error and leaves its
-// loop, and the producer waits (again bounded) for the copies it issued
-// before the CTA exits.
+// Every mbarrier wait is bounded (about 2-4 s of SM clock cycles); on expiry
+// the thread records an error in g_qknr_pipe_error and leaves its loop, and
+// the producers wait (again bounded) for the copies they issued before the
+// CTA exits.
 #pragma once
 
 #include "qknr_kernels.cuh"
@@ -34,7 +34,7 @@ namespace qknr {
 
 constexpr int kMaxStages = 8;
 constexpr int kMaxTileTokens = 32;
-constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per wait
+constexpr long long kWaitLimitCycles = 4000000000ll;  // ~2 s per wait at 1.9 GHz
 
 // Sticky error flag of the pipelined kernels (bit 0: a wait timed out).
 __device__ unsigned int g_qknr_pipe_error;
@@ -81,21 +81,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-__device__ __forceinline__ uint64_t global_ns() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
 // Wait until the phase of parity `parity` has completed, for at most
-// kWaitLimitNs (the clock is read once per 1024 tries); false on expiry,
-// with the error flag set.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+// kWaitLimitCycles SM clock cycles (about 2-4 s; the cycle counter is cheap
+// to read, unlike the global timer); false on expiry, with the error flag
+// set. After a few tries a waiting warp may sleep between tests (backing off
+// from 32 ns to `max_sleep` ns) so waiters leave the issue slots to the warps
+// doing work.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t max_sleep = 256) {
     if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = global_ns();
+    const long long c0 = clock64();
+    uint32_t nap = 32;
 #pragma unroll 1
     for (uint32_t n = 1;; ++n) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((n & 1023u) == 0 && global_ns() - t0 > kWaitLimitNs) {
+        if (n > 2 && max_sleep) {
+            __nanosleep(nap);
+            nap = nap < max_sleep ? nap * 2 : max_sleep;
+        }
+        if ((n & 255u) == 0 && clock64() - c0 > kWaitLimitCycles) {
             atomicOr(&g_qknr_pipe_error, 1u);
             return false;
         }
@@ -300,9 +303,9 @@ template <int LPR, int V, int U> struct Units {
 // a warp reads it without bank conflicts.
 template <typename T, int V>
 __device__ __forceinline__ void fill_unit_gamma(float4 (*s_gl)[V / 2][32], const void *gq,
-                                                const void *gk, int D, int R, int nthreads) {
+                                                const void *gk, int D, int R, int tid, int nthreads) {
     constexpr int W = V / 2;
-    for (int idx = threadIdx.x; idx < 2 * W * 32; idx += nthreads) {
+    for (int idx = tid; idx < 2 * W * 32; idx += nthreads) {
         const int z = idx / (W * 32), k = (idx / 32) % W, w = idx % 32;
         const UnitGeom<V> L(w, D, R);
         const void *gp = z ? gk : gq;
@@ -340,19 +343,23 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g) {
     __shared__ __align__(8) uint64_t bars[2 * kMaxStages];
     __shared__ uint64_t s_step[kMaxHalf];
     __shared__ __align__(16) float4 s_gl[2][W][32];
+    __shared__ volatile int s_abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t full0 = smem_u32(&bars[0]), empty0 = smem_u32(&bars[kMaxStages]);
     init_barriers<NCW, NPW>(full0, empty0, g);
+    if (threadIdx.x == 0) s_abort = 0;
     __syncthreads();
 
     const Run run(a.T, g);
     const int rowb = a.D * (int)sizeof(T);
     const int half = a.R >> 1;
 
-    if (warp >= NCW) {
+    if (warp < NPW) {
         // ----------------------------------------------------- producers
-        const int pw = warp - NCW;
+        // (the lowest warp ids, which the warp schedulers favour, so the
+        // tables are ready before the consumers need them)
+        const int pw = warp;
         const uint64_t pol = evict_first_policy();
         // copies of tile `it` into its stage, counted on the stage's barrier
         auto issue = [&](int it) {
@@ -388,8 +395,16 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g) {
                 pos_next = tile_pos(a.pos, a.S, t1, s_row, (int)min((int64_t)g.TT, run.t_hi - t1), lane);
             }
             if (it >= first) {
-                if (!mbar_wait(empty0 + 8 * s, ((it / g.NS) & 1) ^ 1)) break;
-                if (pw == 0 && lane == 0) issue(it);
+                // warp 0 waits for the stage and refills it; the others block
+                // on a hardware barrier until it has (no spinning)
+                bool ok = true;
+                if (pw == 0) {
+                    ok = mbar_wait(empty0 + 8 * s, ((it / g.NS) & 1) ^ 1, 512);
+                    if (ok && lane == 0) issue(it);
+                    if (!ok) s_abort = 1;
+                }
+                producers_sync(32 * NPW);
+                if (s_abort) break;
                 issued = it + 1;
             }
             unsigned char *st = smem + (size_t)s * g.stage_bytes;
@@ -403,7 +418,7 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g) {
     } else {
         // ------------------------------------------------------ consumers
         fill_unit_gamma<T, V>(s_gl, a.Hq ? a.gq : nullptr, a.Hkv ? a.gk : nullptr, a.D, a.R,
-                              NCW * 32);
+                              threadIdx.x - NPW * 32, NCW * 32);
         consumers_sync(NCW * 32);
         const Units<LPR, V, U> L(lane, a.D, a.R);
         int offA[U], offB[U];
@@ -416,7 +431,7 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g) {
         int pc = 0;  // passes dealt before this tile, mod NCW
         for (int it = 0; it < run.ntiles; ++it) {
             const int s = it % g.NS;
-            if (!mbar_wait(full0 + 8 * s, (it / g.NS) & 1)) break;
+            if (!mbar_wait(full0 + 8 * s, (it / g.NS) & 1, 0)) break;
             const unsigned char *st = smem + (size_t)s * g.stage_bytes;
             const int64_t t0 = run.t_lo + (int64_t)it * g.TT;
             const int na = (int)min((int64_t)g.TT, run.t_hi - t0);
@@ -427,7 +442,7 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g) {
             float *r_k = a.rk + t0 * a.Hkv;
             const float4 *cs_tile = reinterpret_cast<const float4 *>(st + g.off_cs);
             const int npass = (rows + SLOTS - 1) / SLOTS;
-            int p = warp - pc;
+            int p = (warp - NPW) - pc;
             if (p < 0) p += NCW;
             for (; p < npass; p += NCW) {
                 const int j = p * SLOTS + L.slot;
@@ -505,11 +520,13 @@ qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g) {
     __shared__ __align__(8) uint64_t bars[2 * kMaxStages];
     __shared__ uint64_t s_step[kMaxHalf];
     __shared__ __align__(16) float4 s_gl[2][W][32];
+    __shared__ volatile int s_abort;
     __shared__ float s_dg[2][kMaxD];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t full0 = smem_u32(&bars[0]), empty0 = smem_u32(&bars[kMaxStages]);
     init_barriers<NCW, NPW>(full0, empty0, g);
+    if (threadIdx.x == 0) s_abort = 0;
     for (int i = threadIdx.x; i < 2 * kMaxD; i += blockDim.x) (&s_dg[0][0])[i] = 0.f;
     __syncthreads();
 
@@ -517,9 +534,11 @@ qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g) {
     const int rowb = a.D * (int)sizeof(T);
     const int half = a.R >> 1;
 
-    if (warp >= NCW) {
+    if (warp < NPW) {
         // ----------------------------------------------------- producers
-        const int pw = warp - NCW;
+        // (the lowest warp ids, which the warp schedulers favour, so the
+        // tables are ready before the consumers need them)
+        const int pw = warp;
         const uint64_t pol = evict_first_policy();
         auto issue = [&](int it) {
             const int s = it % g.NS;
@@ -527,8 +546,8 @@ qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g) {
             const int na = (int)min((int64_t)g.TT, run.t_hi - t0);
             unsigned char *st = smem + (size_t)s * g.stage_bytes;
             const uint32_t bq = (uint32_t)(na * a.Hq * rowb), bk = (uint32_t)(na * a.Hkv * rowb);
-            // inverse RMS: the 16-byte multiple of each block; a tail of up
-            // to three floats is read by the consumers directly
+            // inverse RMS: the 16-byte multiple of each block (the
+            // producers fill in a tail of up to three floats)
             const uint32_t brq = (uint32_t)(na * a.Hq * 4) & ~15u;
             const uint32_t brk = (uint32_t)(na * a.Hkv * 4) & ~15u;
             const uint32_t bar = full0 + 8 * s;
@@ -565,11 +584,29 @@ qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g) {
                 pos_next = tile_pos(a.pos, a.S, t1, s_row, (int)min((int64_t)g.TT, run.t_hi - t1), lane);
             }
             if (it >= first) {
-                if (!mbar_wait(empty0 + 8 * s, ((it / g.NS) & 1) ^ 1)) break;
-                if (pw == 0 && lane == 0) issue(it);
+                // warp 0 waits for the stage and refills it; the others block
+                // on a hardware barrier until it has (no spinning)
+                bool ok = true;
+                if (pw == 0) {
+                    ok = mbar_wait(empty0 + 8 * s, ((it / g.NS) & 1) ^ 1, 512);
+                    if (ok && lane == 0) issue(it);
+                    if (!ok) s_abort = 1;
+                }
+                producers_sync(32 * NPW);
+                if (s_abort) break;
                 issued = it + 1;
             }
             unsigned char *st = smem + (size_t)s * g.stage_bytes;
+            if (pw == 0) {
+                // inverse-RMS floats past the 16-byte multiple (at most three
+                // per tensor, only in a tensor's last, partial tile)
+                const int nq = na * a.Hq, nk = na * a.Hkv;
+                const int cq = (nq * 4 & ~15) / 4, ck = (nk * 4 & ~15) / 4;
+                if (lane < nq - cq)
+                    reinterpret_cast<float *>(st + g.off_rq)[cq + lane] = a.rq[t0 * a.Hq + cq + lane];
+                if (lane >= 4 && lane - 4 < nk - ck)
+                    reinterpret_cast<float *>(st + g.off_rk)[ck + lane - 4] = a.rk[t0 * a.Hkv + ck + lane - 4];
+            }
             tile_angles<V, NPW>(reinterpret_cast<float *>(st + g.off_cs), s_step, half, na, pos, pw, lane);
             __syncwarp();
             mbar_arrive(full0 + 8 * s);
@@ -579,7 +616,7 @@ qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g) {
     } else {
         // ------------------------------------------------------ consumers
         fill_unit_gamma<T, V>(s_gl, a.Hq ? a.gq : nullptr, a.Hkv ? a.gk : nullptr, a.D, a.R,
-                              NCW * 32);
+                              threadIdx.x - NPW * 32, NCW * 32);
         consumers_sync(NCW * 32);
         const Units<LPR, V, 1> L(lane, a.D, a.R);
         const int offA = L.eA[0] * (int)sizeof(T), offB = L.eB[0] * (int)sizeof(T);
@@ -592,19 +629,16 @@ qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g) {
         int pc = 0;
         for (int it = 0; it < run.ntiles; ++it) {
             const int s = it % g.NS;
-            if (!mbar_wait(full0 + 8 * s, (it / g.NS) & 1)) break;
+            if (!mbar_wait(full0 + 8 * s, (it / g.NS) & 1, 0)) break;
             const unsigned char *st = smem + (size_t)s * g.stage_bytes;
             const int64_t t0 = run.t_lo + (int64_t)it * g.TT;
             const int na = (int)min((int64_t)g.TT, run.t_hi - t0);
             const int rows_q = na * a.Hq, rows = na * (a.Hq + a.Hkv);
-            const int cov_q = (rows_q * 4 & ~15) / 4, cov_k = (na * a.Hkv * 4 & ~15) / 4;
             char *out_q = (char *)a.dq + t0 * a.Hq * rowb;
             char *out_k = (char *)a.dk + t0 * a.Hkv * rowb;
-            const float *gr_q = a.rq + t0 * a.Hq;
-            const float *gr_k = a.rk + t0 * a.Hkv;
             const float4 *cs_tile = reinterpret_cast<const float4 *>(st + g.off_cs);
             const int npass = (rows + SLOTS - 1) / SLOTS;
-            int p = warp - pc;
+            int p = (warp - NPW) - pc;
             if (p < 0) p += NCW;
             for (; p < npass; p += NCW) {
                 const int j = p * SLOTS + L.slot;
@@ -614,9 +648,7 @@ qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g) {
                 const unsigned char *ds = st + (tr.isq ? g.off_dq : g.off_dk) + tr.jj * rowb;
                 const Vec16 xa = lds16(xs + offA), xb = lds16(xs + offB);
                 const Vec16 da = lds16(ds + offA), db = lds16(ds + offB);
-                const bool in_smem = tr.jj < (tr.isq ? cov_q : cov_k);
-                float r = in_smem ? reinterpret_cast<const float *>(st + (tr.isq ? g.off_rq : g.off_rk))[tr.jj]
-                                  : (tr.isq ? gr_q : gr_k)[tr.jj];
+                float r = reinterpret_cast<const float *>(st + (tr.isq ? g.off_rq : g.off_rk))[tr.jj];
                 r = valid ? r : 0.f;  // rows past the tile and off lanes add nothing
                 float4 cs[W], gv[W];
                 unit_table<V>(cs_tile + tr.tl * (half >> 1), L.rot[0], uu, cs);
