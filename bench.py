@@ -42,7 +42,7 @@ import workloads  # noqa: E402
 
 METRIC = "QK-norm+RoPE fwd+bwd tokens/s and HBM GB/s (% of B200 peak), 1 GPU"
 FALLBACK_HBM_GBS = 6650.0
-NSETS, LAG = 4, 2
+NSETS, LAG = 4, 2  # ring of input sets; the backward runs LAG steps behind
 KERNEL_SOURCES = ["qk_rmsnorm_rope_norm_b200/csrc/qknr_kernels.cuh",
                   "qk_rmsnorm_rope_norm_b200/csrc/qknr_pipe.cuh",
                   "qk_rmsnorm_rope_norm_b200/csrc/qknr_api.cu"]
@@ -168,6 +168,26 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(self.samples)}
 
 
+# ------------------------------------------------------- multi-rank plumbing
+def rank_seed(w, rank: int) -> int:
+    """Each rank draws its own batch (weak scaling): seed 1000*index + 100*rank."""
+    return workloads.seed_for(w) + 100 * rank
+
+
+def max_over_ranks(values, world: int, device) -> list:
+    """Element-wise max of per-rank timings (the job is as slow as its
+    slowest rank); a no-op on one rank."""
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.tolist()
+
+
+def aggregate_tokens_per_s(world: int, tokens_per_rank: int, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank processes its own batch each step."""
+    return world * tokens_per_rank / (ms_per_step / 1e3)
+
+
 # ---------------------------------------------------------------- our arm
 class Set:
     """Device buffers of one batch: inputs, forward outputs, gradients."""
@@ -191,7 +211,8 @@ def run_ours(args, w, inp, rank, local_rank, world):
     dev = torch.device("cuda", local_rank)
     qknr.load_library()
     cfg = dict(rotary_dim=w.rotary_dim, theta=w.theta, eps=w.eps)
-    sets = [Set(inp, dev) for _ in range(NSETS)]
+    nsets = args.sets
+    sets = [Set(inp, dev) for _ in range(nsets)]
     stream = torch.cuda.current_stream(dev)
     fwd = [qknr.prepare_fwd(s.q, s.k, s.gq, s.gk, s.pos, s.qo, s.ko, s.rq, s.rk, **cfg)
            for s in sets]
@@ -204,10 +225,10 @@ def run_ours(args, w, inp, rank, local_rank, world):
     def step(i, e=None):
         if e is not None:
             e[0].record(stream)
-        fwd[i % NSETS]()
+        fwd[i % nsets]()
         if e is not None:
             e[1].record(stream)
-        bwd[(i - LAG) % NSETS]()
+        bwd[(i - LAG) % nsets]()
         if e is not None:
             e[2].record(stream)
 
@@ -229,10 +250,7 @@ def run_ours(args, w, inp, rank, local_rank, world):
     total_ms = t_start.elapsed_time(t_end)
     fwd_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / K
     bwd_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / K
-    t = torch.tensor([total_ms, fwd_ms, bwd_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    total_ms, fwd_ms, bwd_ms = t.tolist()
+    total_ms, fwd_ms, bwd_ms = max_over_ranks([total_ms, fwd_ms, bwd_ms], world, dev)
 
     e2e = None
     if not args.no_e2e:
@@ -303,11 +321,8 @@ def run_e2e(args, w, inp, dev, cfg, world):
         step()
     b.record()
     torch.cuda.synchronize(dev)
-    ms = a.elapsed_time(b) / E
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    return dict(ms=float(t.item()), steps=E, h2d=h2d, d2h=d2h)
+    ms = max_over_ranks([a.elapsed_time(b) / E], world, dev)[0]
+    return dict(ms=ms, steps=E, h2d=h2d, d2h=d2h)
 
 
 # ------------------------------------------------------- the CPU oracle
@@ -342,12 +357,29 @@ def oracle_sample_rate(inp, budget_s: float, tokens_per_call: int = 512, max_cal
     return done, spent, per_call
 
 
+cfg_args = None
+
+
+def bwd_kernel_name(w) -> str:
+    """The backward kernel the library launches for this shape (the pipelined
+    one: one row unit per lane, lanes per row the next power of two of
+    D / 16 bytes-pairs; 16 consumer and 4 producer warps)."""
+    dv2 = w.D // (2 * (16 // w.elem_bytes))
+    lpr = 1
+    while lpr < dv2:
+        lpr *= 2
+    tname = "__nv_bfloat16" if w.dtype == "bf16" else "float"
+    return f"qknr_bwd_pipe_kernel<{tname}, {lpr}, 16, 4>"
+
+
 def config_of(w, inp, world):
     return {"workload": w.name, "B": w.B, "S": w.S, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
             "rotary_dim": w.rotary_dim, "theta": w.theta, "eps": w.eps, "io_dtype": w.dtype,
             "tokens_per_step": inp.real_tokens,
             "l2": f"ring of {NSETS} input sets, bwd lags fwd by {LAG} steps: inputs not "
-                  f"L2-resident (> 2x 126 MB of traffic between touches)",
+                  f"L2-resident (> 2x 126 MB of traffic between touches)"
+                  if getattr(cfg_args, "sets", NSETS) == NSETS else
+                  f"{cfg_args.sets} input set(s): profiling run, inputs may be L2-resident",
             "parallelism": f"dp{world} (weak, no data-path collective)"}
 
 
@@ -382,17 +414,23 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=workloads.BENCH_WORKLOAD,
                     choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--sets", type=int, default=NSETS,
+                    help="input sets in the ring (4 keeps inputs out of L2; 1 for small "
+                         "profiling footprints)")
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
+    global cfg_args
+    cfg_args = args
+    if args.sets < 1:
+        ap.error("--sets must be >= 1")
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     rank, local_rank, world = env_rank()
     w = workloads.WORKLOADS[args.workload]
-    seed = workloads.seed_for(w) + 100 * rank
-    inp = workloads.make_inputs(w, seed=seed)
+    inp = workloads.make_inputs(w, seed=rank_seed(w, rank))
     w = inp.w
 
     if args.impl == "reference":
@@ -421,15 +459,11 @@ def main():
     peak, peak_src = hbm_peak()
     tokens = inp.real_tokens
     ms = r["total_ms"] / args.steps
-    value = world * tokens / (ms / 1e3)
+    value = aggregate_tokens_per_s(world, tokens, ms)
     fwd_gbs = cb["fwd"] / (r["fwd_ms"] / 1e3) / 1e9
     bwd_gbs = cb["bwd"] / (r["bwd_ms"] / 1e3) / 1e9
     step_gbs = (cb["fwd"] + cb["bwd"]) / (ms / 1e3) / 1e9
-    lpr = 1
-    while lpr < w.D // (2 * (16 // w.elem_bytes)):
-        lpr *= 2
-    tname = "__nv_bfloat16" if w.dtype == "bf16" else "float"
-    bwd_kernel = f"qknr_bwd_kernel<{tname}, {lpr}>"
+    bwd_kernel = bwd_kernel_name(w)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
@@ -445,9 +479,9 @@ def main():
                     "bwd_gbs": cb["bwd"] / (r["floor"]["bwd_ms"] / 1e3) / 1e9,
                     "fwd_frac_of_copy": r["floor"]["fwd_ms"] / r["fwd_ms"],
                     "bwd_frac_of_copy": r["floor"]["bwd_ms"] / r["bwd_ms"]}},
-        "fwd": {"ms": r["fwd_ms"], "tokens_per_s": world * tokens / (r["fwd_ms"] / 1e3),
+        "fwd": {"ms": r["fwd_ms"], "tokens_per_s": aggregate_tokens_per_s(world, tokens, r["fwd_ms"]),
                 "bytes_per_launch": cb["fwd"]},
-        "bwd": {"ms": r["bwd_ms"], "tokens_per_s": world * tokens / (r["bwd_ms"] / 1e3),
+        "bwd": {"ms": r["bwd_ms"], "tokens_per_s": aggregate_tokens_per_s(world, tokens, r["bwd_ms"]),
                 "bytes_per_launch": cb["bwd"]},
         "roofline": {"bound": "hbm", "kernel": bwd_kernel, "achieved": bwd_gbs, "peak": peak,
                      "unit": "GB/s", "frac": bwd_gbs / peak,
@@ -458,7 +492,7 @@ def main():
     }
     if r["e2e"] is not None:
         e = r["e2e"]
-        line["e2e"] = {"value": world * tokens / (e["ms"] / 1e3), "unit": "tokens/s",
+        line["e2e"] = {"value": aggregate_tokens_per_s(world, tokens, e["ms"]), "unit": "tokens/s",
                        "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"],
                        "ms_per_step": e["ms"], "steps": e["steps"]}
     line["cpu_baseline"] = cpu
