@@ -274,34 +274,56 @@ struct TileRow {
     }
 };
 
-// U units per lane: lane (slot, u) owns units u + q * LPR, q < U. Unit w
-// holds the two 16-byte vectors of a head row described in
-// qknr_kernels.cuh (rotary partners in one unit); units past D / 2V are
-// off (they read element 0 and are masked out).
-template <int LPR, int V, int U> struct Units {
+// Register pairs of a lane. Lane (slot, u) owns units u + q * LPR (q < U),
+// each unit being the two 16-byte vectors of a head row described in
+// qknr_kernels.cuh (rotary partners in one unit). Pair p holds unit
+// u + q LPR with c = (p + slot) mod 2U, q = c mod U, and its two vectors in
+// swapped order when c >= U. Load instruction k (first vectors for k < U,
+// second vectors after) then reads combination (k + slot) mod 2U, so the
+// rows of a shared-memory phase (rows are 128 or 256 bytes apart and would
+// otherwise all hit the same banks) read distinct bank groups. A swapped
+// pair computes the same rotation with the sine negated. Units past D / 2V
+// are off (they read element 0 and are masked out).
+template <int LPR, int V, int U> struct Pairs {
     int u, slot;
     bool on[U], rot[U];
-    int eA[U], eB[U];
+    int w[U];               // unit index
+    int first[U], second[U];  // element offsets of the pair's two vectors
+    int kb[U];              // gamma-table half of the first vector (0: A, V/4: B)
+    float sgn[U];           // +1, or -1 when the halves are swapped
     float mask[U];
-    __device__ __forceinline__ Units(int lane, int D, int R) {
+    __device__ __forceinline__ Pairs(int lane, int D, int R) {
         u = lane & (LPR - 1);
         slot = lane / LPR;
 #pragma unroll
-        for (int q = 0; q < U; ++q) {
-            const UnitGeom<V> G(u + q * LPR, D, R);
-            on[q] = G.on;
-            rot[q] = G.rot;
-            eA[q] = G.eA;
-            eB[q] = G.eB;
-            mask[q] = G.on ? 1.f : 0.f;
+        for (int p = 0; p < U; ++p) {
+            const int c = (p + slot) % (2 * U);
+            const bool sw = c >= U;
+            const int q = sw ? c - U : c;
+            w[p] = u + q * LPR;
+            const UnitGeom<V> G(w[p], D, R);
+            on[p] = G.on;
+            rot[p] = G.rot;
+            first[p] = sw ? G.eB : G.eA;
+            second[p] = sw ? G.eA : G.eB;
+            kb[p] = sw ? V / 4 : 0;
+            sgn[p] = sw ? -1.f : 1.f;
+            mask[p] = G.on ? 1.f : 0.f;
         }
     }
 };
 
-// Per-CTA table of gamma in unit order: s_gl[z][k][w] holds elements
-// 4k..4k+3 of unit w's A vector (k < V/4) or of its B vector, as fp32, so
-// a warp reads it without bank conflicts.
-template <typename T, int V>
+// Column swizzle of the gamma table: with at most 4 units per row group the
+// B half is stored at column w ^ 4, which keeps a phase's reads on distinct
+// banks under the pair rotation above.
+template <int LPR, int U> struct GammaSwz {
+    static constexpr int X = (LPR * U <= 4) ? 4 : 0;
+};
+
+// Per-CTA table of gamma in unit order: s_gl[z][k][w ^ (k >= V/4 ? X : 0)]
+// holds elements 4k..4k+3 of unit w's A vector (k < V/4) or 4(k - V/4)..
+// of its B vector, as fp32, so a warp reads it without bank conflicts.
+template <typename T, int V, int X>
 __device__ __forceinline__ void fill_unit_gamma(float4 (*s_gl)[V / 2][32], const void *gq,
                                                 const void *gk, int D, int R, int tid, int nthreads) {
     constexpr int W = V / 2;
@@ -315,7 +337,19 @@ __device__ __forceinline__ void fill_unit_gamma(float4 (*s_gl)[V / 2][32], const
             v = make_float4(Io<T>::to_f32(gp, e), Io<T>::to_f32(gp, e + 1),
                             Io<T>::to_f32(gp, e + 2), Io<T>::to_f32(gp, e + 3));
         }
-        s_gl[z][k][w] = v;
+        s_gl[z][k][w ^ (k >= W / 2 ? X : 0)] = v;
+    }
+}
+
+// gamma of a pair: float4 j < V/4 of its first vector, then of its second.
+template <int V, int X>
+__device__ __forceinline__ void pair_gamma(const float4 (*gl)[32], int w, int kb, float4 *gv) {
+    constexpr int W = V / 2;
+#pragma unroll
+    for (int j = 0; j < W / 2; ++j) {
+        const int k1 = kb + j, k2 = (W / 2 - kb) + j;
+        gv[j] = gl[k1][w ^ (k1 >= W / 2 ? X : 0)];
+        gv[W / 2 + j] = gl[k2][w ^ (k2 >= W / 2 ? X : 0)];
     }
 }
 
@@ -332,7 +366,8 @@ __device__ __forceinline__ void init_barriers(uint32_t full0, uint32_t empty0, c
 }
 
 // ================================================================== forward
-// Per row: y_A = r (u_A c - u_B s), y_B = r (u_B c + u_A s), u = x * gamma.
+// Per row: y_A = r (u_A c - u_B s), y_B = r (u_B c + u_A s), u = x * gamma,
+// evaluated as u_A (r c) - u_B (r s) and u_B (r c) + u_A (r s).
 template <typename T, int LPR, int U, int NCW, int NPW>
 __global__ void __launch_bounds__((NCW + NPW) * 32, 1)
 qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g) {
@@ -417,15 +452,16 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g) {
             mbar_wait(full0 + 8 * (it % g.NS), (it / g.NS) & 1);
     } else {
         // ------------------------------------------------------ consumers
-        fill_unit_gamma<T, V>(s_gl, a.Hq ? a.gq : nullptr, a.Hkv ? a.gk : nullptr, a.D, a.R,
-                              threadIdx.x - NPW * 32, NCW * 32);
+        constexpr int X = GammaSwz<LPR, U>::X;
+        fill_unit_gamma<T, V, X>(s_gl, a.Hq ? a.gq : nullptr, a.Hkv ? a.gk : nullptr, a.D, a.R,
+                                 threadIdx.x - NPW * 32, NCW * 32);
         consumers_sync(NCW * 32);
-        const Units<LPR, V, U> L(lane, a.D, a.R);
-        int offA[U], offB[U];
+        const Pairs<LPR, V, U> L(lane, a.D, a.R);
+        int off1[U], off2[U];
 #pragma unroll
         for (int q = 0; q < U; ++q) {
-            offA[q] = L.eA[q] * (int)sizeof(T);
-            offB[q] = L.eB[q] * (int)sizeof(T);
+            off1[q] = L.first[q] * (int)sizeof(T);
+            off2[q] = L.second[q] * (int)sizeof(T);
         }
         const float inv_d = 1.0f / (float)a.D;
         int pc = 0;  // passes dealt before this tile, mod NCW
@@ -451,10 +487,9 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g) {
                 const unsigned char *src = st + (tr.isq ? 0 : g.off_k) + tr.jj * rowb;
                 Vec16 xa[U], xb[U];
 #pragma unroll
-                for (int q = 0; q < U; ++q) {
-                    xa[q] = lds16(src + offA[q]);
-                    xb[q] = lds16(src + offB[q]);
-                }
+                for (int q = 0; q < U; ++q) xa[q] = lds16(src + off1[q]);
+#pragma unroll
+                for (int q = 0; q < U; ++q) xb[q] = lds16(src + off2[q]);
                 float ss = 0.f;
 #pragma unroll
                 for (int q = 0; q < U; ++q) {
@@ -475,26 +510,27 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g) {
 #pragma unroll
                 for (int q = 0; q < U; ++q) {
                     float4 cs[W], gv[W];
-                    unit_table<V>(tok, L.rot[q], L.u + q * LPR, cs);
-#pragma unroll
-                    for (int k = 0; k < W; ++k) gv[k] = s_gl[tr.isq ? 0 : 1][k][L.u + q * LPR];
+                    unit_table<V>(tok, L.rot[q], L.w[q], cs);
+                    pair_gamma<V, X>(s_gl[tr.isq ? 0 : 1], L.w[q], L.kb[q], gv);
+                    // r (and the pair's sine sign) folded into cos and sin
+                    const float rs = r * L.sgn[q];
+                    const float2 rs2 = make_float2(rs, rs);
                     Vec16 ya, yb;
 #pragma unroll
                     for (int k = 0; k < W; ++k) {
                         const float2 ga = (k & 1) ? hi2(gv[k >> 1]) : lo2(gv[k >> 1]);
                         const float2 gb = (k & 1) ? hi2(gv[W / 2 + (k >> 1)]) : lo2(gv[W / 2 + (k >> 1)]);
-                        const float2 c = lo2(cs[k]), sn = hi2(cs[k]);
+                        const float2 c = __fmul2_rn(lo2(cs[k]), r2), sn = __fmul2_rn(hi2(cs[k]), rs2);
                         const float2 ua = __fmul2_rn(IO::get2(xa[q], k), ga);
                         const float2 ub = __fmul2_rn(IO::get2(xb[q], k), gb);
-                        const float2 pa = __ffma2_rn(ua, c, __fmul2_rn(ub, neg2(sn)));
-                        const float2 pb = __ffma2_rn(ub, c, __fmul2_rn(ua, sn));
-                        const float2 oa = __fmul2_rn(pa, r2), ob = __fmul2_rn(pb, r2);
+                        const float2 oa = __ffma2_rn(ua, c, __fmul2_rn(ub, neg2(sn)));
+                        const float2 ob = __ffma2_rn(ub, c, __fmul2_rn(ua, sn));
                         IO::put2(ya, k, oa.x, oa.y);
                         IO::put2(yb, k, ob.x, ob.y);
                     }
                     if (valid && L.on[q]) {
-                        stg16(out + offA[q], ya);
-                        stg16(out + offB[q], yb);
+                        stg16(out + off1[q], ya);
+                        stg16(out + off2[q], yb);
                     }
                 }
                 if (valid && L.u == 0) __stcs((tr.isq ? r_q : r_k) + tr.jj, r);
@@ -615,14 +651,17 @@ qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g) {
             mbar_wait(full0 + 8 * (it % g.NS), (it / g.NS) & 1);
     } else {
         // ------------------------------------------------------ consumers
-        fill_unit_gamma<T, V>(s_gl, a.Hq ? a.gq : nullptr, a.Hkv ? a.gk : nullptr, a.D, a.R,
-                              threadIdx.x - NPW * 32, NCW * 32);
+        constexpr int X = GammaSwz<LPR, 1>::X;
+        fill_unit_gamma<T, V, X>(s_gl, a.Hq ? a.gq : nullptr, a.Hkv ? a.gk : nullptr, a.D, a.R,
+                                 threadIdx.x - NPW * 32, NCW * 32);
         consumers_sync(NCW * 32);
-        const Units<LPR, V, 1> L(lane, a.D, a.R);
-        const int offA = L.eA[0] * (int)sizeof(T), offB = L.eB[0] * (int)sizeof(T);
-        const int uu = L.u;
+        const Pairs<LPR, V, 1> L(lane, a.D, a.R);
+        const int off1 = L.first[0] * (int)sizeof(T), off2 = L.second[0] * (int)sizeof(T);
+        const int uu = L.w[0];
+        const float2 sg = make_float2(L.sgn[0], L.sgn[0]);
         const float inv_d = 1.0f / (float)a.D;
-        // dgamma partial sums: [k] = elements (eA + 2k, eA + 2k + 1), same for B
+        // dgamma partial sums: [k] = elements (first + 2k, first + 2k + 1),
+        // same for the second vector
         float2 aqa[W], aqb[W], aka[W], akb[W];
 #pragma unroll
         for (int k = 0; k < W; ++k) aqa[k] = aqb[k] = aka[k] = akb[k] = make_float2(0.f, 0.f);
@@ -646,14 +685,13 @@ qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g) {
                 const TileRow tr(j < rows ? j : 0, rows_q, g);
                 const unsigned char *xs = st + (tr.isq ? 0 : g.off_k) + tr.jj * rowb;
                 const unsigned char *ds = st + (tr.isq ? g.off_dq : g.off_dk) + tr.jj * rowb;
-                const Vec16 xa = lds16(xs + offA), xb = lds16(xs + offB);
-                const Vec16 da = lds16(ds + offA), db = lds16(ds + offB);
+                const Vec16 xa = lds16(xs + off1), da = lds16(ds + off1);
+                const Vec16 xb = lds16(xs + off2), db = lds16(ds + off2);
                 float r = reinterpret_cast<const float *>(st + (tr.isq ? g.off_rq : g.off_rk))[tr.jj];
                 r = valid ? r : 0.f;  // rows past the tile and off lanes add nothing
                 float4 cs[W], gv[W];
                 unit_table<V>(cs_tile + tr.tl * (half >> 1), L.rot[0], uu, cs);
-#pragma unroll
-                for (int k = 0; k < W; ++k) gv[k] = s_gl[tr.isq ? 0 : 1][k][uu];
+                pair_gamma<V, X>(s_gl[tr.isq ? 0 : 1], uu, L.kb[0], gv);
                 const float2 r2 = make_float2(r, r);
                 float2 ha[W], hb[W], xha[W], xhb[W];
                 float2 d0 = make_float2(0.f, 0.f), d1 = make_float2(0.f, 0.f);
@@ -661,7 +699,7 @@ qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g) {
                 for (int k = 0; k < W; ++k) {
                     const float2 ga = (k & 1) ? hi2(gv[k >> 1]) : lo2(gv[k >> 1]);
                     const float2 gb = (k & 1) ? hi2(gv[W / 2 + (k >> 1)]) : lo2(gv[W / 2 + (k >> 1)]);
-                    const float2 c = lo2(cs[k]), sn = hi2(cs[k]);
+                    const float2 c = lo2(cs[k]), sn = __fmul2_rn(hi2(cs[k]), sg);
                     const float2 dA = IO::get2(da, k), dB = IO::get2(db, k);
                     xha[k] = __fmul2_rn(IO::get2(xa, k), r2);
                     xhb[k] = __fmul2_rn(IO::get2(xb, k), r2);
@@ -691,16 +729,26 @@ qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g) {
                         IO::put2(ob, k, vb.x, vb.y);
                     }
                     char *out = (tr.isq ? out_q : out_k) + tr.jj * rowb;
-                    stg16(out + offA, oa);
-                    stg16(out + offB, ob);
+                    stg16(out + off1, oa);
+                    stg16(out + off2, ob);
                 }
             }
             pc = (pc + npass) % NCW;
             __syncwarp();
             if (lane == 0) mbar_arrive(empty0 + 8 * s);
         }
-        // dgamma: lanes of one unit across the warp's row slots, then the
-        // CTA's consumer warps (shared atomics)
+        // dgamma: back to (A, B) order on swapped lanes, then lanes of one
+        // unit across the warp's row slots, then the CTA's consumer warps
+        // (shared atomics)
+        const bool sw = L.sgn[0] < 0.f;
+#pragma unroll
+        for (int k = 0; k < W; ++k) {
+            const float2 q1 = aqa[k], q2 = aqb[k], k1 = aka[k], k2 = akb[k];
+            aqa[k] = sw ? q2 : q1;
+            aqb[k] = sw ? q1 : q2;
+            aka[k] = sw ? k2 : k1;
+            akb[k] = sw ? k1 : k2;
+        }
 #pragma unroll
         for (int o = LPR; o < 32; o <<= 1) {
 #pragma unroll
@@ -716,7 +764,7 @@ qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g) {
             }
         }
         if (L.slot == 0 && L.on[0]) {
-            const int eA = L.eA[0], eB = L.eB[0];
+            const int eA = sw ? L.second[0] : L.first[0], eB = sw ? L.first[0] : L.second[0];
 #pragma unroll
             for (int k = 0; k < W; ++k) {
                 atomicAdd(&s_dg[0][eA + 2 * k], aqa[k].x);
