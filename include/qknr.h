@@ -24,7 +24,8 @@
  * abstract). Optional int32 position ids carry packed sequences whose
  * positions restart per document (Chronicals, abstract, contribution (4)).
  *
- * Layout. Every tensor is dense and row-major, no strides:
+ * Layout. Every tensor is dense and row-major (the _strided forms below
+ * also take Q and K, and dQ and dK, with a token stride):
  *   q, q_out, dq_out, dq   [B, S, Hq,  D]     k, k_out, dk_out, dk [B, S, Hkv, D]
  *   rstd_q [B, S, Hq] fp32, rstd_k [B, S, Hkv] fp32
  *   gamma_q, gamma_k [D] in the I/O dtype;  dgamma_q, dgamma_k [D] fp32
@@ -127,6 +128,59 @@ QKNR_API qknr_status qk_norm_rope_bwd(const void *q, const void *k,
                              const float *rstd_q, const float *rstd_k,
                              const void *dq_out, const void *dk_out,
                              void *dq, void *dk,
+                             float *dgamma_q, float *dgamma_k,
+                             int B, int S, int Hq, int Hkv, int D,
+                             int rotary_dim, float theta, float eps,
+                             qknr_dtype dtype, qknr_stream_t stream);
+
+/*
+ * Strided-input forms, for Q and K read straight out of a fused QKV
+ * projection buffer with no copy pass in between (Chronicals, arXiv
+ * 2601.02609, abstract, contribution (1): the fused kernels remove memory
+ * traffic; reading the projection output in place is this library's reading
+ * of that, the pages give no layout). Heads stay contiguous within a token
+ * and D contiguous within a head; tokens t = b * S + s are evenly spaced:
+ *
+ *   row (t, h) of q  starts at  q + t * q_token_stride + h * D   (elements)
+ *   row (t, h) of k  starts at  k + t * k_token_stride + h * D
+ *
+ * e.g. for qkv [B, S, (Hq + 2 Hkv) * D]: q = qkv, k = qkv + Hq * D and both
+ * strides (Hq + 2 Hkv) * D. A stride must be >= H * D of its tensor and a
+ * whole number of 16 bytes (else QKNR_ERR_INVALID_ARG / QKNR_ERR_ALIGNMENT);
+ * H * D elements is the dense layout of qk_norm_rope_fwd / _bwd, which
+ * these calls then match exactly.
+ *
+ * Forward: q_out, k_out, rstd_q, rstd_k are dense as in qk_norm_rope_fwd
+ * (the layout attention kernels read). An output may alias its input only
+ * when that input is dense.
+ */
+QKNR_API qknr_status qk_norm_rope_fwd_strided(const void *q, const void *k,
+                             int64_t q_token_stride, int64_t k_token_stride,
+                             const void *gamma_q, const void *gamma_k,
+                             const int32_t *pos_ids,
+                             void *q_out, void *k_out,
+                             float *rstd_q, float *rstd_k,
+                             int B, int S, int Hq, int Hkv, int D,
+                             int rotary_dim, float theta, float eps,
+                             qknr_dtype dtype, qknr_stream_t stream);
+
+/*
+ * Backward with strided q, k (as in qk_norm_rope_fwd_strided) and strided
+ * gradients dq, dk (row (t, h) of dq at dq + t * dq_token_stride + h * D),
+ * e.g. written straight into the Q and K slots of a dQKV buffer whose V slot
+ * another kernel fills. dq_out, dk_out, rstd and dgamma are dense as in
+ * qk_norm_rope_bwd. Strided outputs may share a buffer with each other and
+ * with other tensors' slots as long as their bytes do not overlap; dq may
+ * alias dq_out (dk, dk_out) only when both are dense.
+ */
+QKNR_API qknr_status qk_norm_rope_bwd_strided(const void *q, const void *k,
+                             int64_t q_token_stride, int64_t k_token_stride,
+                             const void *gamma_q, const void *gamma_k,
+                             const int32_t *pos_ids,
+                             const float *rstd_q, const float *rstd_k,
+                             const void *dq_out, const void *dk_out,
+                             void *dq, void *dk,
+                             int64_t dq_token_stride, int64_t dk_token_stride,
                              float *dgamma_q, float *dgamma_k,
                              int B, int S, int Hq, int Hkv, int D,
                              int rotary_dim, float theta, float eps,

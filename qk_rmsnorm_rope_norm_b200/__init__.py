@@ -8,8 +8,10 @@ computation runs in the library's CUDA kernels; there is no fallback, and
 every entry point raises if the library is missing or a tensor is not on a
 CUDA device.
 
-Names follow the C ABI: ``qk_norm_rope_fwd`` / ``qk_norm_rope_bwd``. The
-autograd wrapper ``QKNormRoPE`` chains them for training code.
+Names follow the C ABI: ``qk_norm_rope_fwd`` / ``qk_norm_rope_bwd`` (which
+also take Q / K slices of a fused QKV buffer, dispatching to the
+``_strided`` entry points). The autograd wrappers ``QKNormRoPE`` and
+``QKNormRoPEFromQKV`` chain them for training code.
 """
 from __future__ import annotations
 
@@ -20,6 +22,7 @@ from typing import Optional
 import torch
 
 __all__ = ["qk_norm_rope_fwd", "qk_norm_rope_bwd", "qknr_strerror", "QKNormRoPE",
+           "QKNormRoPEFromQKV", "qk_norm_rope_qkv", "split_qkv",
            "prepare_fwd", "prepare_bwd", "PreparedCall",
            "qk_norm_rope", "QKNRError", "library_path", "load_library", "pipeline_error"]
 
@@ -59,6 +62,13 @@ def load_library():
     lib.qk_norm_rope_fwd.argtypes = [vp] * 9 + [i32] * 6 + [f32, f32, i32, vp]
     lib.qk_norm_rope_bwd.restype = i32
     lib.qk_norm_rope_bwd.argtypes = [vp] * 13 + [i32] * 6 + [f32, f32, i32, vp]
+    i64 = ctypes.c_int64
+    lib.qk_norm_rope_fwd_strided.restype = i32
+    lib.qk_norm_rope_fwd_strided.argtypes = [vp, vp, i64, i64] + [vp] * 7 + [i32] * 6 + \
+        [f32, f32, i32, vp]
+    lib.qk_norm_rope_bwd_strided.restype = i32
+    lib.qk_norm_rope_bwd_strided.argtypes = [vp, vp, i64, i64] + [vp] * 9 + [i64, i64] + \
+        [vp] * 2 + [i32] * 6 + [f32, f32, i32, vp]
     lib.qknr_strerror.restype = ctypes.c_char_p
     lib.qknr_strerror.argtypes = [i32]
     lib.qknr_last_cuda_error.restype = i32
@@ -96,6 +106,27 @@ def _need_cuda(name: str, t: torch.Tensor):
         raise ValueError(f"{name} must be contiguous")
 
 
+def _token_stride(name: str, t: torch.Tensor) -> int:
+    """Elements between consecutive tokens of a [B, S, H, D] CUDA tensor whose
+    heads and dims are dense and whose tokens (t = b * S + s) are evenly
+    spaced: a dense tensor, or a Q / K slice of a fused QKV buffer."""
+    if not isinstance(t, torch.Tensor) or t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dim() != 4:
+        raise ValueError(f"{name} must be [B, S, H, D]")
+    B, S, H, D = t.shape
+    if t.is_contiguous():
+        return H * D
+    st = t.stride()
+    ts = st[1] if S > 1 else (st[0] if B > 1 else H * D)
+    ok = (D <= 1 or st[3] == 1) and (H <= 1 or st[2] == D) and ts >= H * D
+    ok = ok and (B <= 1 or S <= 1 or st[0] == S * st[1]) and (S > 1 or B <= 1 or st[0] == ts)
+    if not ok:
+        raise ValueError(f"{name} must be dense within each token, with tokens evenly spaced "
+                         f"(strides {tuple(st)})")
+    return int(ts)
+
+
 def _shape(q: torch.Tensor, k: torch.Tensor):
     if q.dim() != 4 or k.dim() != 4:
         raise ValueError("q and k must be [B, S, H, D]")
@@ -115,7 +146,8 @@ def qk_norm_rope_fwd(q, k, gamma_q, gamma_k, pos_ids=None, *, rotary_dim: int,
     are allocated; ``q_out=q`` / ``k_out=k`` runs in place.
     """
     lib = load_library()
-    for n, t in (("q", q), ("k", k), ("gamma_q", gamma_q), ("gamma_k", gamma_k)):
+    qts, kts = _token_stride("q", q), _token_stride("k", k)
+    for n, t in (("gamma_q", gamma_q), ("gamma_k", gamma_k)):
         _need_cuda(n, t)
     B, S, Hq, Hkv, D = _shape(q, k)
     if q.dtype not in _DTYPES or k.dtype != q.dtype or gamma_q.dtype != q.dtype \
@@ -125,8 +157,8 @@ def qk_norm_rope_fwd(q, k, gamma_q, gamma_k, pos_ids=None, *, rotary_dim: int,
         _need_cuda("pos_ids", pos_ids)
         if pos_ids.dtype != torch.int32 or tuple(pos_ids.shape) != (B, S):
             raise ValueError("pos_ids must be int32 [B, S]")
-    q_out = torch.empty_like(q) if q_out is None else q_out
-    k_out = torch.empty_like(k) if k_out is None else k_out
+    q_out = torch.empty(q.shape, dtype=q.dtype, device=q.device) if q_out is None else q_out
+    k_out = torch.empty(k.shape, dtype=k.dtype, device=k.device) if k_out is None else k_out
     if rstd_q is None:
         rstd_q = torch.empty((B, S, Hq), dtype=torch.float32, device=q.device)
     if rstd_k is None:
@@ -139,13 +171,26 @@ def qk_norm_rope_fwd(q, k, gamma_q, gamma_k, pos_ids=None, *, rotary_dim: int,
     if rstd_q.dtype != torch.float32 or rstd_k.dtype != torch.float32 or \
             tuple(rstd_q.shape) != (B, S, Hq) or tuple(rstd_k.shape) != (B, S, Hkv):
         raise ValueError("rstd_q / rstd_k must be float32 [B,S,Hq] / [B,S,Hkv]")
-    st = lib.qk_norm_rope_fwd(_ptr(q), _ptr(k), _ptr(gamma_q), _ptr(gamma_k), _ptr(pos_ids),
-                              _ptr(q_out), _ptr(k_out), _ptr(rstd_q), _ptr(rstd_k),
-                              B, S, Hq, Hkv, D, int(rotary_dim), float(theta), float(eps),
-                              _DTYPES[q.dtype], _stream(stream))
+    fn, name, args = _fwd_args(lib, q, k, qts, kts, gamma_q, gamma_k, pos_ids, q_out, k_out,
+                               rstd_q, rstd_k, rotary_dim, theta, eps, stream)
+    st = fn(*args)
     if st != QKNR_OK:
-        raise QKNRError(st, "qk_norm_rope_fwd")
+        raise QKNRError(st, name)
     return q_out, k_out, rstd_q, rstd_k
+
+
+def _fwd_args(lib, q, k, qts, kts, gamma_q, gamma_k, pos_ids, q_out, k_out, rstd_q, rstd_k,
+              rotary_dim, theta, eps, stream):
+    """(C function, its name, argument tuple): the dense entry point when q and
+    k are dense, else the strided one."""
+    B, S, Hq, Hkv, D = _shape(q, k)
+    tail = (_ptr(gamma_q), _ptr(gamma_k), _ptr(pos_ids), _ptr(q_out), _ptr(k_out),
+            _ptr(rstd_q), _ptr(rstd_k), B, S, Hq, Hkv, D, int(rotary_dim), float(theta),
+            float(eps), _DTYPES[q.dtype], _stream(stream))
+    if qts == Hq * D and kts == Hkv * D:
+        return lib.qk_norm_rope_fwd, "qk_norm_rope_fwd", (_ptr(q), _ptr(k)) + tail
+    return lib.qk_norm_rope_fwd_strided, "qk_norm_rope_fwd_strided", \
+        (_ptr(q), _ptr(k), qts, kts) + tail
 
 
 def qk_norm_rope_bwd(q, k, gamma_q, gamma_k, pos_ids, rstd_q, rstd_k, dq_out, dk_out, *,
@@ -157,7 +202,8 @@ def qk_norm_rope_bwd(q, k, gamma_q, gamma_k, pos_ids, rstd_q, rstd_k, dq_out, dk
     and no dgamma buffers given, the gamma gradients are skipped (None).
     """
     lib = load_library()
-    for n, t in (("q", q), ("k", k), ("gamma_q", gamma_q), ("gamma_k", gamma_k),
+    qts, kts = _token_stride("q", q), _token_stride("k", k)
+    for n, t in (("gamma_q", gamma_q), ("gamma_k", gamma_k),
                  ("rstd_q", rstd_q), ("rstd_k", rstd_k), ("dq_out", dq_out), ("dk_out", dk_out)):
         _need_cuda(n, t)
     B, S, Hq, Hkv, D = _shape(q, k)
@@ -172,28 +218,44 @@ def qk_norm_rope_bwd(q, k, gamma_q, gamma_k, pos_ids, rstd_q, rstd_k, dq_out, dk
         _need_cuda("pos_ids", pos_ids)
         if pos_ids.dtype != torch.int32 or tuple(pos_ids.shape) != (B, S):
             raise ValueError("pos_ids must be int32 [B, S]")
-    dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty_like(k) if dk is None else dk
+    dq = torch.empty(q.shape, dtype=q.dtype, device=q.device) if dq is None else dq
+    dk = torch.empty(k.shape, dtype=k.dtype, device=k.device) if dk is None else dk
     if need_dgamma:
         if dgamma_q is None:
             dgamma_q = torch.empty(D, dtype=torch.float32, device=q.device)
         if dgamma_k is None:
             dgamma_k = torch.empty(D, dtype=torch.float32, device=q.device)
-    for n, t in (("dq", dq), ("dk", dk)):
-        _need_cuda(n, t)
+    dqts, dkts = _token_stride("dq", dq), _token_stride("dk", dk)
+    if dq.shape != q.shape or dk.shape != k.shape or dq.dtype != q.dtype or dk.dtype != q.dtype:
+        raise ValueError("dq / dk must match q / k in shape and dtype")
     for n, t in (("dgamma_q", dgamma_q), ("dgamma_k", dgamma_k)):
         if t is not None:
             _need_cuda(n, t)
             if t.dtype != torch.float32 or t.numel() != D:
                 raise ValueError(f"{n} must be float32 [D]")
-    st = lib.qk_norm_rope_bwd(_ptr(q), _ptr(k), _ptr(gamma_q), _ptr(gamma_k), _ptr(pos_ids),
-                              _ptr(rstd_q), _ptr(rstd_k), _ptr(dq_out), _ptr(dk_out),
-                              _ptr(dq), _ptr(dk), _ptr(dgamma_q), _ptr(dgamma_k),
-                              B, S, Hq, Hkv, D, int(rotary_dim), float(theta), float(eps),
-                              _DTYPES[q.dtype], _stream(stream))
+    fn, name, args = _bwd_args(lib, q, k, qts, kts, gamma_q, gamma_k, pos_ids, rstd_q, rstd_k,
+                               dq_out, dk_out, dq, dk, dqts, dkts, dgamma_q, dgamma_k,
+                               rotary_dim, theta, eps, stream)
+    st = fn(*args)
     if st != QKNR_OK:
-        raise QKNRError(st, "qk_norm_rope_bwd")
+        raise QKNRError(st, name)
     return dq, dk, dgamma_q, dgamma_k
+
+
+def _bwd_args(lib, q, k, qts, kts, gamma_q, gamma_k, pos_ids, rstd_q, rstd_k, dq_out, dk_out,
+              dq, dk, dqts, dkts, dgamma_q, dgamma_k, rotary_dim, theta, eps, stream):
+    B, S, Hq, Hkv, D = _shape(q, k)
+    tail = (B, S, Hq, Hkv, D, int(rotary_dim), float(theta), float(eps), _DTYPES[q.dtype],
+            _stream(stream))
+    if qts == Hq * D and kts == Hkv * D and dqts == Hq * D and dkts == Hkv * D:
+        return lib.qk_norm_rope_bwd, "qk_norm_rope_bwd", (
+            _ptr(q), _ptr(k), _ptr(gamma_q), _ptr(gamma_k), _ptr(pos_ids), _ptr(rstd_q),
+            _ptr(rstd_k), _ptr(dq_out), _ptr(dk_out), _ptr(dq), _ptr(dk), _ptr(dgamma_q),
+            _ptr(dgamma_k)) + tail
+    return lib.qk_norm_rope_bwd_strided, "qk_norm_rope_bwd_strided", (
+        _ptr(q), _ptr(k), qts, kts, _ptr(gamma_q), _ptr(gamma_k), _ptr(pos_ids), _ptr(rstd_q),
+        _ptr(rstd_k), _ptr(dq_out), _ptr(dk_out), _ptr(dq), _ptr(dk), dqts, dkts,
+        _ptr(dgamma_q), _ptr(dgamma_k)) + tail
 
 
 class QKNormRoPE(torch.autograd.Function):
@@ -229,6 +291,63 @@ def qk_norm_rope(q, k, gamma_q, gamma_k, pos_ids=None, *, rotary_dim: int, theta
     return QKNormRoPE.apply(q, k, gamma_q, gamma_k, pos_ids, rotary_dim, theta, eps)
 
 
+def split_qkv(qkv: torch.Tensor, Hq: int, Hkv: int):
+    """Views ``(q, k, v)`` of a fused projection output qkv [B, S, (Hq + 2 Hkv) D]:
+    q [B,S,Hq,D], k and v [B,S,Hkv,D], tokens (Hq + 2 Hkv) D elements apart."""
+    if qkv.dim() != 3 or qkv.shape[2] % (Hq + 2 * Hkv):
+        raise ValueError("qkv must be [B, S, (Hq + 2 Hkv) * D]")
+    B, S, W = qkv.shape
+    D = W // (Hq + 2 * Hkv)
+    q = qkv[..., :Hq * D].unflatten(-1, (Hq, D))
+    k = qkv[..., Hq * D:(Hq + Hkv) * D].unflatten(-1, (Hkv, D))
+    v = qkv[..., (Hq + Hkv) * D:].unflatten(-1, (Hkv, D))
+    return q, k, v
+
+
+class QKNormRoPEFromQKV(torch.autograd.Function):
+    """Fused op on a QKV projection output: q and k are read in place from
+    qkv, and the backward writes dq and dk straight into the Q and K slots of
+    one dqkv buffer (dv fills the V slot), so no split or concat is copied."""
+
+    @staticmethod
+    def forward(ctx, qkv, gamma_q, gamma_k, pos_ids, Hq, Hkv, rotary_dim, theta, eps):
+        q, k, v = split_qkv(qkv, Hq, Hkv)
+        q_out, k_out, rq, rk = qk_norm_rope_fwd(q, k, gamma_q, gamma_k, pos_ids,
+                                                rotary_dim=rotary_dim, theta=theta, eps=eps)
+        ctx.save_for_backward(qkv, gamma_q, gamma_k, rq, rk)
+        ctx.pos_ids = pos_ids
+        ctx.cfg = (Hq, Hkv, rotary_dim, theta, eps)
+        ctx.mark_non_differentiable(rq, rk)
+        return q_out, k_out, v
+
+    @staticmethod
+    def backward(ctx, dq_out, dk_out, dv):
+        qkv, gq, gk, rq, rk = ctx.saved_tensors
+        Hq, Hkv, R, theta, eps = ctx.cfg
+        q, k, _ = split_qkv(qkv, Hq, Hkv)
+        dqkv = torch.empty_like(qkv)
+        dq, dk, dvs = split_qkv(dqkv, Hq, Hkv)
+        if dv is None:
+            dvs.zero_()
+        else:
+            dvs.copy_(dv)
+        _, _, dgq, dgk = qk_norm_rope_bwd(
+            q, k, gq, gk, ctx.pos_ids, rq, rk, dq_out.contiguous(), dk_out.contiguous(),
+            rotary_dim=R, theta=theta, eps=eps, dq=dq, dk=dk,
+            need_dgamma=ctx.needs_input_grad[1] or ctx.needs_input_grad[2])
+        dgq = None if dgq is None else dgq.to(gq.dtype)
+        dgk = None if dgk is None else dgk.to(gk.dtype)
+        return dqkv, dgq, dgk, None, None, None, None, None, None
+
+
+def qk_norm_rope_qkv(qkv, gamma_q, gamma_k, pos_ids=None, *, Hq: int, Hkv: int,
+                     rotary_dim: int, theta: float, eps: float):
+    """Differentiable fused op on qkv [B, S, (Hq + 2 Hkv) D]; returns
+    ``(q_out, k_out, v)`` with q_out, k_out dense [B,S,H,D] and v a view."""
+    return QKNormRoPEFromQKV.apply(qkv, gamma_q, gamma_k, pos_ids, Hq, Hkv, rotary_dim, theta,
+                                   eps)
+
+
 class PreparedCall:
     """A C ABI call with every argument marshalled once.
 
@@ -254,12 +373,11 @@ def prepare_fwd(q, k, gamma_q, gamma_k, pos_ids, q_out, k_out, rstd_q, rstd_k, *
     qk_norm_rope_fwd(q, k, gamma_q, gamma_k, pos_ids, rotary_dim=rotary_dim, theta=theta,
                      eps=eps, q_out=q_out, k_out=k_out, rstd_q=rstd_q, rstd_k=rstd_k,
                      stream=stream)
-    B, S, Hq, Hkv, D = _shape(q, k)
-    args = (_ptr(q), _ptr(k), _ptr(gamma_q), _ptr(gamma_k), _ptr(pos_ids), _ptr(q_out),
-            _ptr(k_out), _ptr(rstd_q), _ptr(rstd_k), B, S, Hq, Hkv, D, int(rotary_dim),
-            float(theta), float(eps), _DTYPES[q.dtype], _stream(stream))
+    fn, name, args = _fwd_args(lib, q, k, _token_stride("q", q), _token_stride("k", k), gamma_q,
+                               gamma_k, pos_ids, q_out, k_out, rstd_q, rstd_k, rotary_dim,
+                               theta, eps, stream)
     keep = (q, k, gamma_q, gamma_k, pos_ids, q_out, k_out, rstd_q, rstd_k)
-    return PreparedCall(lib.qk_norm_rope_fwd, args, "qk_norm_rope_fwd", keep)
+    return PreparedCall(fn, args, name, keep)
 
 
 def prepare_bwd(q, k, gamma_q, gamma_k, pos_ids, rstd_q, rstd_k, dq_out, dk_out, dq, dk,
@@ -268,11 +386,10 @@ def prepare_bwd(q, k, gamma_q, gamma_k, pos_ids, rstd_q, rstd_k, dq_out, dk_out,
     qk_norm_rope_bwd(q, k, gamma_q, gamma_k, pos_ids, rstd_q, rstd_k, dq_out, dk_out,
                      rotary_dim=rotary_dim, theta=theta, eps=eps, dq=dq, dk=dk,
                      dgamma_q=dgamma_q, dgamma_k=dgamma_k, stream=stream)
-    B, S, Hq, Hkv, D = _shape(q, k)
-    args = (_ptr(q), _ptr(k), _ptr(gamma_q), _ptr(gamma_k), _ptr(pos_ids), _ptr(rstd_q),
-            _ptr(rstd_k), _ptr(dq_out), _ptr(dk_out), _ptr(dq), _ptr(dk), _ptr(dgamma_q),
-            _ptr(dgamma_k), B, S, Hq, Hkv, D, int(rotary_dim), float(theta), float(eps),
-            _DTYPES[q.dtype], _stream(stream))
+    fn, name, args = _bwd_args(lib, q, k, _token_stride("q", q), _token_stride("k", k), gamma_q,
+                               gamma_k, pos_ids, rstd_q, rstd_k, dq_out, dk_out, dq, dk,
+                               _token_stride("dq", dq), _token_stride("dk", dk), dgamma_q,
+                               dgamma_k, rotary_dim, theta, eps, stream)
     keep = (q, k, gamma_q, gamma_k, pos_ids, rstd_q, rstd_k, dq_out, dk_out, dq, dk,
             dgamma_q, dgamma_k)
-    return PreparedCall(lib.qk_norm_rope_bwd, args, "qk_norm_rope_bwd", keep)
+    return PreparedCall(fn, args, name, keep)

@@ -4,6 +4,8 @@
 #include "qknr.h"
 #include "qknr_pipe.cuh"
 
+#include <cudaTypedefs.h>  // PFN_cuTensorMapEncodeTiled
+
 #include <atomic>
 #include <cmath>
 #include <cstdint>
@@ -21,14 +23,37 @@ qknr_status cuda_fail(cudaError_t e) {
 
 bool aligned(const void *p, uintptr_t a) { return ((uintptr_t)p % a) == 0; }
 
+// The bytes a buffer covers: [p, p + n), and when ts > 0 only the first
+// `row` bytes of every ts-byte token step (a strided Q or K in a fused QKV
+// buffer, where the other slots belong to other tensors).
 struct Span {
     const char *p;
     size_t n;
+    size_t row = 0;
+    size_t ts = 0;
 };
+
+// Span covering T tokens of `row` bytes, `ts` bytes apart (ts == row: dense).
+Span strided(const void *p, int64_t T, size_t row, size_t ts) {
+    if (!p || T <= 0 || row == 0) return Span{(const char *)p, 0};
+    Span s{(const char *)p, (size_t)(T - 1) * ts + row};
+    if (ts != row) {
+        s.row = row;
+        s.ts = ts;
+    }
+    return s;
+}
 
 bool overlaps(Span a, Span b) {
     if (!a.p || !b.p || a.n == 0 || b.n == 0) return false;
-    return a.p < b.p + b.n && b.p < a.p + a.n;
+    if (!(a.p < b.p + b.n && b.p < a.p + a.n)) return false;
+    if (a.ts && a.ts == b.ts) {
+        // two combs of the same pitch: disjoint when b's row sits in a's gap
+        const int64_t d = (int64_t)(b.p - a.p), ts = (int64_t)a.ts;
+        const int64_t r = ((d % ts) + ts) % ts;
+        return !((int64_t)a.row <= r && r + (int64_t)b.row <= ts);
+    }
+    return true;
 }
 
 // Shape checks shared by both directions.
@@ -54,7 +79,8 @@ qknr_status check_overlaps(const Span *all, int n_all, int first_out, const int 
     for (int i = first_out; i < n_all; ++i) {
         for (int j = 0; j < n_all; ++j) {
             if (j == i || !overlaps(all[i], all[j])) continue;
-            if (j == may_equal[i - first_out] && all[j].p == all[i].p && all[j].n == all[i].n)
+            if (j == may_equal[i - first_out] && all[j].p == all[i].p && all[j].n == all[i].n &&
+                all[j].ts == all[i].ts)
                 continue;
             return QKNR_ERR_INVALID_ARG;
         }
@@ -218,28 +244,82 @@ bool pipe_disabled() {
     return e && e[0] == '1';
 }
 
+// cuTensorMapEncodeTiled from the driver, looked up once.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static std::atomic<void *> fn{nullptr};
+    static std::atomic<int> tried{0};
+    void *f = fn.load(std::memory_order_acquire);
+    if (f || tried.load(std::memory_order_acquire)) return (PFN_cuTensorMapEncodeTiled_v12000)f;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+        f = nullptr;
+    fn.store(f, std::memory_order_release);
+    tried.store(1, std::memory_order_release);
+    return (PFN_cuTensorMapEncodeTiled_v12000)f;
+}
+
+// 3-D tensor map {D, H, T} over rows whose tokens are ts bytes apart (heads
+// contiguous within a token), box {D, H, TT}: one tile's block in one copy.
+bool encode_rows(CUtensorMap *m, const void *base, int esz, int D, int H, int64_t T, int64_t ts,
+                 int TT) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc || H > 256 || D > 256 || T >= ((int64_t)1 << 31)) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T};
+    const cuuint64_t strides[2] = {(cuuint64_t)D * esz, (cuuint64_t)ts};
+    const cuuint32_t box[3] = {(cuuint32_t)D, (cuuint32_t)H, (cuuint32_t)TT};
+    const cuuint32_t unit[3] = {1, 1, 1};
+    return enc(m, esz == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+               const_cast<void *>(base), dims, strides, box, unit, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Tensor maps for strided Q / K inputs (bit 0 / 1 of the returned mask);
+// -1 when a strided input cannot be described by one (the caller then uses
+// the plain-load kernels).
+int input_maps(const void *q, const void *k, int64_t qts, int64_t kts, int Hq, int Hkv, int D,
+               int esz, int64_t T, int TT, CUtensorMap *mq, CUtensorMap *mk) {
+    const int64_t rowb = (int64_t)D * esz;
+    int mask = 0;
+    *mq = CUtensorMap{};
+    *mk = CUtensorMap{};
+    if (Hq > 0 && qts != Hq * rowb) {
+        if (!encode_rows(mq, q, esz, D, Hq, T, qts, TT)) return -1;
+        mask |= 1;
+    }
+    if (Hkv > 0 && kts != Hkv * rowb) {
+        if (!encode_rows(mk, k, esz, D, Hkv, T, kts, TT)) return -1;
+        mask |= 2;
+    }
+    return mask;
+}
+
 template <typename T, int LPR, int U>
-qknr_status launch_fwd_pipe(const FwdArgs &a, const PipeGeom &g, int grid, int smem, int dev,
-                            cudaStream_t st, bool *launched) {
+qknr_status launch_fwd_pipe(const FwdArgs &a, const PipeGeom &g, const CUtensorMap &mq,
+                            const CUtensorMap &mk, int grid, int smem, int dev, cudaStream_t st,
+                            bool *launched) {
     static std::atomic<int> smem_ok[64];
     auto kern = qknr_fwd_pipe_kernel<T, LPR, U, kFwdPipeWarps, kProducerWarps>;
     *launched = false;
     if (!allow_dyn_smem((const void *)kern, dev, smem_ok, smem)) return QKNR_OK;
     *launched = true;
-    kern<<<grid, (kFwdPipeWarps + kProducerWarps) * 32, smem, st>>>(a, g);
+    kern<<<grid, (kFwdPipeWarps + kProducerWarps) * 32, smem, st>>>(a, g, mq, mk);
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? QKNR_OK : cuda_fail(e);
 }
 
 template <typename T, int LPR>
-qknr_status launch_bwd_pipe(const BwdArgs &a, const PipeGeom &g, int grid, int smem, int dev,
-                            cudaStream_t st, bool *launched) {
+qknr_status launch_bwd_pipe(const BwdArgs &a, const PipeGeom &g, const CUtensorMap &mq,
+                            const CUtensorMap &mk, int grid, int smem, int dev, cudaStream_t st,
+                            bool *launched) {
     static std::atomic<int> smem_ok[64];
     auto kern = qknr_bwd_pipe_kernel<T, LPR, kBwdPipeWarps, kProducerWarps>;
     *launched = false;
     if (!allow_dyn_smem((const void *)kern, dev, smem_ok, smem)) return QKNR_OK;
     *launched = true;
-    kern<<<grid, (kBwdPipeWarps + kProducerWarps) * 32, smem, st>>>(a, g);
+    kern<<<grid, (kBwdPipeWarps + kProducerWarps) * 32, smem, st>>>(a, g, mq, mk);
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? QKNR_OK : cuda_fail(e);
 }
@@ -262,20 +342,23 @@ bool try_fwd_pipe(const FwdArgs &a, cudaStream_t st, qknr_status *status) {
         !pipe_geometry(false, a.T, a.Hq, a.Hkv, a.D, a.R, (int)sizeof(T), dev, nullptr, nullptr,
                        &g, &grid, &smem))
         return false;
+    CUtensorMap mq, mk;
+    g.tmap = input_maps(a.q, a.k, a.qts, a.kts, a.Hq, a.Hkv, a.D, (int)sizeof(T), a.T, g.TT, &mq, &mk);
+    if (g.tmap < 0) return false;
     const int dv2 = a.D / (2 * (16 / (int)sizeof(T)));
     bool launched = false;
     qknr_status s = QKNR_OK;
     if (dv2 >= 3) {
         switch (next_pow2((dv2 + 1) / 2)) {
-            case 2: s = launch_fwd_pipe<T, 2, 2>(a, g, grid, smem, dev, st, &launched); break;
-            case 4: s = launch_fwd_pipe<T, 4, 2>(a, g, grid, smem, dev, st, &launched); break;
-            case 8: s = launch_fwd_pipe<T, 8, 2>(a, g, grid, smem, dev, st, &launched); break;
-            case 16: s = launch_fwd_pipe<T, 16, 2>(a, g, grid, smem, dev, st, &launched); break;
+            case 2: s = launch_fwd_pipe<T, 2, 2>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
+            case 4: s = launch_fwd_pipe<T, 4, 2>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
+            case 8: s = launch_fwd_pipe<T, 8, 2>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
+            case 16: s = launch_fwd_pipe<T, 16, 2>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
         }
     } else {
         switch (next_pow2(dv2)) {
-            case 1: s = launch_fwd_pipe<T, 1, 1>(a, g, grid, smem, dev, st, &launched); break;
-            case 2: s = launch_fwd_pipe<T, 2, 1>(a, g, grid, smem, dev, st, &launched); break;
+            case 1: s = launch_fwd_pipe<T, 1, 1>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
+            case 2: s = launch_fwd_pipe<T, 2, 1>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
         }
     }
     *status = s;
@@ -292,16 +375,19 @@ bool try_bwd_pipe(const BwdArgs &a, cudaStream_t st, qknr_status *status) {
         !pipe_geometry(true, a.T, a.Hq, a.Hkv, a.D, a.R, (int)sizeof(T), dev, a.rq, a.rk, &g,
                        &grid, &smem))
         return false;
+    CUtensorMap mq, mk;
+    g.tmap = input_maps(a.q, a.k, a.qts, a.kts, a.Hq, a.Hkv, a.D, (int)sizeof(T), a.T, g.TT, &mq, &mk);
+    if (g.tmap < 0) return false;
     const int dv2 = a.D / (2 * (16 / (int)sizeof(T)));
     bool launched = false;
     qknr_status s = QKNR_OK;
     switch (next_pow2(dv2)) {
-        case 1: s = launch_bwd_pipe<T, 1>(a, g, grid, smem, dev, st, &launched); break;
-        case 2: s = launch_bwd_pipe<T, 2>(a, g, grid, smem, dev, st, &launched); break;
-        case 4: s = launch_bwd_pipe<T, 4>(a, g, grid, smem, dev, st, &launched); break;
-        case 8: s = launch_bwd_pipe<T, 8>(a, g, grid, smem, dev, st, &launched); break;
-        case 16: s = launch_bwd_pipe<T, 16>(a, g, grid, smem, dev, st, &launched); break;
-        case 32: s = launch_bwd_pipe<T, 32>(a, g, grid, smem, dev, st, &launched); break;
+        case 1: s = launch_bwd_pipe<T, 1>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
+        case 2: s = launch_bwd_pipe<T, 2>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
+        case 4: s = launch_bwd_pipe<T, 4>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
+        case 8: s = launch_bwd_pipe<T, 8>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
+        case 16: s = launch_bwd_pipe<T, 16>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
+        case 32: s = launch_bwd_pipe<T, 32>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
     }
     *status = s;
     return launched;
@@ -366,12 +452,23 @@ qknr_status dispatch_bwd(const BwdArgs &a, int lpr, cudaStream_t st) {
 
 using namespace qknr;
 
-extern "C" qknr_status qk_norm_rope_fwd(const void *q, const void *k,
-                                        const void *gamma_q, const void *gamma_k,
-                                        const int32_t *pos_ids, void *q_out, void *k_out,
-                                        float *rstd_q, float *rstd_k, int B, int S, int Hq,
-                                        int Hkv, int D, int rotary_dim, float theta, float eps,
-                                        qknr_dtype dtype, qknr_stream_t stream) {
+namespace qknr {
+namespace {
+
+// Token strides (elements) of a strided input or output: at least the rows
+// of one token, and a whole number of 16-byte steps.
+qknr_status check_stride(int64_t ts, int H, int D, size_t e) {
+    if (H == 0) return QKNR_OK;
+    if (ts < (int64_t)H * D) return QKNR_ERR_INVALID_ARG;
+    if ((ts * (int64_t)e) % 16 != 0) return QKNR_ERR_ALIGNMENT;
+    return QKNR_OK;
+}
+
+qknr_status fwd_impl(const void *q, const void *k, int64_t q_ts, int64_t k_ts,
+                     const void *gamma_q, const void *gamma_k, const int32_t *pos_ids, void *q_out,
+                     void *k_out, float *rstd_q, float *rstd_k, int B, int S, int Hq, int Hkv,
+                     int D, int rotary_dim, float theta, float eps, qknr_dtype dtype,
+                     qknr_stream_t stream) {
     qknr_status st = check_shape(B, S, Hq, Hkv, D, rotary_dim, theta, eps, dtype);
     if (st != QKNR_OK) return st;
     const int64_t T = (int64_t)B * S;
@@ -379,6 +476,8 @@ extern "C" qknr_status qk_norm_rope_fwd(const void *q, const void *k,
     const size_t e = dtype == QKNR_F32 ? 4 : 2;
     if (Hq > 0 && (!q || !q_out || !rstd_q || !gamma_q)) return QKNR_ERR_INVALID_ARG;
     if (Hkv > 0 && (!k || !k_out || !rstd_k || !gamma_k)) return QKNR_ERR_INVALID_ARG;
+    if ((st = check_stride(q_ts, Hq, D, e)) != QKNR_OK) return st;
+    if ((st = check_stride(k_ts, Hkv, D, e)) != QKNR_OK) return st;
     const void *vec[] = {q, k, gamma_q, gamma_k, q_out, k_out};
     for (const void *p : vec)
         if (p && !aligned(p, 16)) return QKNR_ERR_ALIGNMENT;
@@ -386,20 +485,22 @@ extern "C" qknr_status qk_norm_rope_fwd(const void *q, const void *k,
         (pos_ids && !aligned(pos_ids, 4)))
         return QKNR_ERR_ALIGNMENT;
 
+    const size_t rq = (size_t)Hq * D * e, rk = (size_t)Hkv * D * e;  // bytes per token
     const size_t nq = (size_t)T * Hq, nk = (size_t)T * Hkv;
     Span all[] = {
-        {(const char *)q, nq * D * e},          {(const char *)k, nk * D * e},
+        strided(q, Hq ? T : 0, rq, (size_t)q_ts * e), strided(k, Hkv ? T : 0, rk, (size_t)k_ts * e),
         {(const char *)gamma_q, Hq ? D * e : 0}, {(const char *)gamma_k, Hkv ? D * e : 0},
         {(const char *)pos_ids, pos_ids ? (size_t)T * 4 : 0},
         {(const char *)q_out, nq * D * e},      {(const char *)k_out, nk * D * e},
         {(const char *)rstd_q, nq * 4},         {(const char *)rstd_k, nk * 4},
     };
-    const int may_equal[] = {0, 1, -1, -1};  // q_out may be q, k_out may be k
+    const int may_equal[] = {0, 1, -1, -1};  // q_out may be a dense q, k_out a dense k
     if (check_overlaps(all, 9, 5, may_equal) != QKNR_OK) return QKNR_ERR_INVALID_ARG;
 
     FwdArgs a{};
     a.q = q; a.k = k; a.gq = gamma_q; a.gk = gamma_k; a.pos = pos_ids;
     a.qo = q_out; a.ko = k_out; a.rq = rstd_q; a.rk = rstd_k;
+    a.qts = q_ts * (int64_t)e; a.kts = k_ts * (int64_t)e;
     a.T = T; a.S = S; a.Hq = Hq; a.Hkv = Hkv; a.D = D; a.R = rotary_dim;
     a.theta = theta; a.eps = eps;
     const int lpr = lanes_per_row(D, (int)e);
@@ -408,14 +509,13 @@ extern "C" qknr_status qk_norm_rope_fwd(const void *q, const void *k,
                              : dispatch_fwd<__nv_bfloat16>(a, lpr, cs);
 }
 
-extern "C" qknr_status qk_norm_rope_bwd(const void *q, const void *k,
-                                        const void *gamma_q, const void *gamma_k,
-                                        const int32_t *pos_ids, const float *rstd_q,
-                                        const float *rstd_k, const void *dq_out,
-                                        const void *dk_out, void *dq, void *dk,
-                                        float *dgamma_q, float *dgamma_k, int B, int S, int Hq,
-                                        int Hkv, int D, int rotary_dim, float theta, float eps,
-                                        qknr_dtype dtype, qknr_stream_t stream) {
+qknr_status bwd_impl(const void *q, const void *k, int64_t q_ts, int64_t k_ts,
+                     const void *gamma_q, const void *gamma_k, const int32_t *pos_ids,
+                     const float *rstd_q, const float *rstd_k, const void *dq_out,
+                     const void *dk_out, void *dq, void *dk, int64_t dq_ts, int64_t dk_ts,
+                     float *dgamma_q, float *dgamma_k, int B, int S, int Hq, int Hkv, int D,
+                     int rotary_dim, float theta, float eps, qknr_dtype dtype,
+                     qknr_stream_t stream) {
     qknr_status st = check_shape(B, S, Hq, Hkv, D, rotary_dim, theta, eps, dtype);
     if (st != QKNR_OK) return st;
     const int64_t T = (int64_t)B * S;
@@ -423,6 +523,10 @@ extern "C" qknr_status qk_norm_rope_bwd(const void *q, const void *k,
     const bool work = T > 0 && Hq + Hkv > 0;
     if (work && Hq > 0 && (!q || !gamma_q || !rstd_q || !dq_out || !dq)) return QKNR_ERR_INVALID_ARG;
     if (work && Hkv > 0 && (!k || !gamma_k || !rstd_k || !dk_out || !dk)) return QKNR_ERR_INVALID_ARG;
+    if ((st = check_stride(q_ts, Hq, D, e)) != QKNR_OK) return st;
+    if ((st = check_stride(k_ts, Hkv, D, e)) != QKNR_OK) return st;
+    if ((st = check_stride(dq_ts, Hq, D, e)) != QKNR_OK) return st;
+    if ((st = check_stride(dk_ts, Hkv, D, e)) != QKNR_OK) return st;
     const void *vec[] = {q, k, gamma_q, gamma_k, dq_out, dk_out, dq, dk};
     for (const void *p : vec)
         if (p && !aligned(p, 16)) return QKNR_ERR_ALIGNMENT;
@@ -431,18 +535,20 @@ extern "C" qknr_status qk_norm_rope_bwd(const void *q, const void *k,
         (dgamma_k && !aligned(dgamma_k, 4)))
         return QKNR_ERR_ALIGNMENT;
 
-    const size_t nq = work ? (size_t)T * Hq : 0, nk = work ? (size_t)T * Hkv : 0;
+    const int64_t Tq = work && Hq ? T : 0, Tk = work && Hkv ? T : 0;
+    const size_t rq = (size_t)Hq * D * e, rk = (size_t)Hkv * D * e;  // bytes per token
+    const size_t nq = (size_t)Tq * Hq, nk = (size_t)Tk * Hkv;
     Span all[] = {
-        {(const char *)q, nq * D * e},           {(const char *)k, nk * D * e},
+        strided(q, Tq, rq, (size_t)q_ts * e),    strided(k, Tk, rk, (size_t)k_ts * e),
         {(const char *)gamma_q, Hq ? D * e : 0},  {(const char *)gamma_k, Hkv ? D * e : 0},
         {(const char *)pos_ids, pos_ids && work ? (size_t)T * 4 : 0},
         {(const char *)rstd_q, nq * 4},          {(const char *)rstd_k, nk * 4},
         {(const char *)dq_out, nq * D * e},      {(const char *)dk_out, nk * D * e},
-        {(const char *)dq, nq * D * e},          {(const char *)dk, nk * D * e},
+        strided(dq, Tq, rq, (size_t)dq_ts * e),  strided(dk, Tk, rk, (size_t)dk_ts * e),
         {(const char *)dgamma_q, dgamma_q ? (size_t)D * 4 : 0},
         {(const char *)dgamma_k, dgamma_k ? (size_t)D * 4 : 0},
     };
-    const int may_equal[] = {7, 8, -1, -1};  // dq may be dq_out, dk may be dk_out
+    const int may_equal[] = {7, 8, -1, -1};  // a dense dq may be dq_out, a dense dk dk_out
     if (check_overlaps(all, 13, 9, may_equal) != QKNR_OK) return QKNR_ERR_INVALID_ARG;
 
     cudaStream_t cs = (cudaStream_t)stream;
@@ -460,11 +566,63 @@ extern "C" qknr_status qk_norm_rope_bwd(const void *q, const void *k,
     a.q = q; a.k = k; a.gq = gamma_q; a.gk = gamma_k; a.pos = pos_ids;
     a.rq = rstd_q; a.rk = rstd_k; a.dqo = dq_out; a.dko = dk_out;
     a.dq = dq; a.dk = dk; a.dgq = dgamma_q; a.dgk = dgamma_k;
+    a.qts = q_ts * (int64_t)e; a.kts = k_ts * (int64_t)e;
+    a.dqts = dq_ts * (int64_t)e; a.dkts = dk_ts * (int64_t)e;
     a.T = T; a.S = S; a.Hq = Hq; a.Hkv = Hkv; a.D = D; a.R = rotary_dim;
     a.theta = theta; a.eps = eps;
     const int lpr = lanes_per_row(D, (int)e);
     return dtype == QKNR_F32 ? dispatch_bwd<float>(a, lpr, cs)
                              : dispatch_bwd<__nv_bfloat16>(a, lpr, cs);
+}
+
+}  // namespace
+}  // namespace qknr
+
+extern "C" qknr_status qk_norm_rope_fwd(const void *q, const void *k,
+                                        const void *gamma_q, const void *gamma_k,
+                                        const int32_t *pos_ids, void *q_out, void *k_out,
+                                        float *rstd_q, float *rstd_k, int B, int S, int Hq,
+                                        int Hkv, int D, int rotary_dim, float theta, float eps,
+                                        qknr_dtype dtype, qknr_stream_t stream) {
+    return fwd_impl(q, k, (int64_t)Hq * D, (int64_t)Hkv * D, gamma_q, gamma_k, pos_ids, q_out,
+                    k_out, rstd_q, rstd_k, B, S, Hq, Hkv, D, rotary_dim, theta, eps, dtype, stream);
+}
+
+extern "C" qknr_status qk_norm_rope_fwd_strided(const void *q, const void *k, int64_t q_token_stride,
+                                                int64_t k_token_stride, const void *gamma_q,
+                                                const void *gamma_k, const int32_t *pos_ids,
+                                                void *q_out, void *k_out, float *rstd_q,
+                                                float *rstd_k, int B, int S, int Hq, int Hkv, int D,
+                                                int rotary_dim, float theta, float eps,
+                                                qknr_dtype dtype, qknr_stream_t stream) {
+    return fwd_impl(q, k, q_token_stride, k_token_stride, gamma_q, gamma_k, pos_ids, q_out, k_out,
+                    rstd_q, rstd_k, B, S, Hq, Hkv, D, rotary_dim, theta, eps, dtype, stream);
+}
+
+extern "C" qknr_status qk_norm_rope_bwd(const void *q, const void *k,
+                                        const void *gamma_q, const void *gamma_k,
+                                        const int32_t *pos_ids, const float *rstd_q,
+                                        const float *rstd_k, const void *dq_out,
+                                        const void *dk_out, void *dq, void *dk,
+                                        float *dgamma_q, float *dgamma_k, int B, int S, int Hq,
+                                        int Hkv, int D, int rotary_dim, float theta, float eps,
+                                        qknr_dtype dtype, qknr_stream_t stream) {
+    const int64_t qts = (int64_t)Hq * D, kts = (int64_t)Hkv * D;
+    return bwd_impl(q, k, qts, kts, gamma_q, gamma_k, pos_ids, rstd_q, rstd_k, dq_out, dk_out, dq,
+                    dk, qts, kts, dgamma_q, dgamma_k, B, S, Hq, Hkv, D, rotary_dim, theta, eps,
+                    dtype, stream);
+}
+
+extern "C" qknr_status qk_norm_rope_bwd_strided(
+    const void *q, const void *k, int64_t q_token_stride, int64_t k_token_stride,
+    const void *gamma_q, const void *gamma_k, const int32_t *pos_ids, const float *rstd_q,
+    const float *rstd_k, const void *dq_out, const void *dk_out, void *dq, void *dk,
+    int64_t dq_token_stride, int64_t dk_token_stride, float *dgamma_q, float *dgamma_k, int B,
+    int S, int Hq, int Hkv, int D, int rotary_dim, float theta, float eps, qknr_dtype dtype,
+    qknr_stream_t stream) {
+    return bwd_impl(q, k, q_token_stride, k_token_stride, gamma_q, gamma_k, pos_ids, rstd_q,
+                    rstd_k, dq_out, dk_out, dq, dk, dq_token_stride, dk_token_stride, dgamma_q,
+                    dgamma_k, B, S, Hq, Hkv, D, rotary_dim, theta, eps, dtype, stream);
 }
 
 extern "C" const char *qknr_strerror(qknr_status s) {

@@ -52,6 +52,7 @@ struct FwdArgs {
     const int32_t *pos;
     void *qo, *ko;
     float *rq, *rk;
+    int64_t qts, kts;  // bytes from one token's rows of q (k) to the next token's
     int64_t T;  // tokens = B * S
     int S, Hq, Hkv, D, R;
     float theta, eps;
@@ -65,6 +66,8 @@ struct BwdArgs {
     const void *dqo, *dko;
     void *dq, *dk;
     float *dgq, *dgk;
+    int64_t qts, kts;    // token strides (bytes) of q and k
+    int64_t dqts, dkts;  // token strides (bytes) of dq and dk
     int64_t T;
     int S, Hq, Hkv, D, R;
     float theta, eps;
@@ -246,8 +249,8 @@ qknr_fwd_kernel(const FwdArgs a) {
 
     for (int64_t t = t_begin; t < t_end; ++t) {
         const int64_t pos = pit.next(t);
-        const char *qrow = (const char *)a.q + t * a.Hq * rowb;
-        const char *krow = (const char *)a.k + t * a.Hkv * rowb;
+        const char *qrow = (const char *)a.q + t * a.qts;
+        const char *krow = (const char *)a.k + t * a.kts;
         Vec16 xa[P], xb[P];
         auto load_chunk = [&](int p0) {
 #pragma unroll
@@ -367,9 +370,9 @@ qknr_bwd_kernel(const BwdArgs a) {
                 if (L.on && h < H) {
                     const bool isq = h < a.Hq;
                     const int64_t rowi = isq ? t * a.Hq + h : t * a.Hkv + (h - a.Hq);
-                    const int64_t off = rowi * rowb;
-                    const char *xrow = (const char *)(isq ? a.q : a.k) + off;
-                    const char *drow = (const char *)(isq ? a.dqo : a.dko) + off;
+                    const int hh = isq ? h : h - a.Hq;
+                    const char *xrow = (const char *)(isq ? a.q : a.k) + t * (isq ? a.qts : a.kts) + hh * rowb;
+                    const char *drow = (const char *)(isq ? a.dqo : a.dko) + rowi * rowb;
                     xa[pp] = ld16(xrow + offA);
                     xb[pp] = ld16(xrow + offB);
                     da[pp] = ld16(drow + offA);
@@ -446,8 +449,8 @@ qknr_bwd_kernel(const BwdArgs a) {
                         IO::put2(oa, k2, outA[0], outA[1]);
                         IO::put2(ob, k2, outB[0], outB[1]);
                     }
-                    const int64_t rowi = isq ? t * a.Hq + h : t * a.Hkv + (h - a.Hq);
-                    char *out = (char *)(isq ? a.dq : a.dk) + rowi * rowb;
+                    const int hh = isq ? h : h - a.Hq;
+                    char *out = (char *)(isq ? a.dq : a.dk) + t * (isq ? a.dqts : a.dkts) + hh * rowb;
                     st16(out + offA, oa);
                     st16(out + offB, ob);
                 }

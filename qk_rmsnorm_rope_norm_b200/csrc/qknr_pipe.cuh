@@ -28,6 +28,8 @@
 // CTA exits.
 #pragma once
 
+#include <cuda.h>  // CUtensorMap (the type only)
+
 #include "qknr_kernels.cuh"
 
 namespace qknr {
@@ -36,7 +38,8 @@ constexpr int kMaxStages = 8;
 constexpr int kMaxTileTokens = 32;
 constexpr long long kWaitLimitCycles = 4000000000ll;  // ~2 s per wait at 1.9 GHz
 
-// Sticky error flag of the pipelined kernels (bit 0: a wait timed out).
+// Sticky error flag of the pipelined kernels (bit 0: a wait timed out;
+// bit 1: shared memory unfit for tensor copies, nothing computed).
 __device__ unsigned int g_qknr_pipe_error;
 
 struct PipeGeom {
@@ -49,6 +52,7 @@ struct PipeGeom {
     int off_rq, off_rk;  // backward: saved inverse RMS of Q and K rows
     uint32_t mq, mk;   // jj / Hq == umulhi(jj, mq) (mq == 0: Hq == 1); same for Hkv
     int64_t tpc;       // tokens per CTA (a multiple of TT)
+    int tmap;          // bit 0 (1): Q (K) rows arrive by 3-D tensor copy (strided input)
 };
 
 // ------------------------------------------------------------ PTX helpers
@@ -123,6 +127,26 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
         "l"(src), "r"(bytes), "r"(bar), "l"(policy)
         : "memory");
 }
+// Tensor copy global -> this CTA's shared memory of the box at (c0, c1, c2)
+// of a 3-D tensor map {D, heads, tokens} (a strided Q or K: one token's rows
+// contiguous, tokens a fixed stride apart). The whole box is always counted
+// on `bar`; elements past the tensor's end read as zero.
+__device__ __forceinline__ void tensor_g2s(uint32_t dst, const CUtensorMap *map, int c0, int c1,
+                                           int c2, uint32_t bar, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar), "l"(policy)
+        : "memory");
+}
+// First token of the tensor-copy box of a tile [t0, t0 + na) in a run ending
+// at t_hi: the tile itself when it is whole, else the box that ends with the
+// run (so a partial last tile re-reads the end of the previous tile instead
+// of the next run's tokens), or token 0 when the run is shorter than a box.
+__device__ __forceinline__ int64_t box_start(int64_t t0, int64_t t_hi, int TT) {
+    return t0 + TT <= t_hi ? t0 : max((int64_t)0, t_hi - TT);
+}
+
 // 16-byte store to global memory, streaming (written once, not re-read).
 __device__ __forceinline__ void stg16(void *p, const Vec16 &v) {
     __stcs(reinterpret_cast<uint4 *>(p), make_uint4(v.w[0], v.w[1], v.w[2], v.w[3]));
@@ -370,7 +394,8 @@ __device__ __forceinline__ void init_barriers(uint32_t full0, uint32_t empty0, c
 // evaluated as u_A (r c) - u_B (r s) and u_B (r c) + u_A (r s).
 template <typename T, int LPR, int U, int NCW, int NPW>
 __global__ void __launch_bounds__((NCW + NPW) * 32, 1)
-qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g) {
+qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g, const __grid_constant__ CUtensorMap tmq,
+                     const __grid_constant__ CUtensorMap tmk) {
     using IO = Io<T>;
     constexpr int V = IO::V, W = V / 2;
     constexpr int SLOTS = 32 / LPR;
@@ -380,6 +405,12 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g) {
     __shared__ __align__(16) float4 s_gl[2][W][32];
     __shared__ volatile int s_abort;
 
+    // tensor copies land on 128-byte boundaries (the stage offsets are
+    // multiples of 128); should the dynamic base not be, report and stop
+    if (g.tmap && (smem_u32(smem) & 127u)) {
+        if (threadIdx.x == 0) atomicOr(&g_qknr_pipe_error, 2u);
+        return;
+    }
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t full0 = smem_u32(&bars[0]), empty0 = smem_u32(&bars[kMaxStages]);
     init_barriers<NCW, NPW>(full0, empty0, g);
@@ -403,10 +434,20 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g) {
             const int na = (int)min((int64_t)g.TT, run.t_hi - t0);
             unsigned char *st = smem + (size_t)s * g.stage_bytes;
             const uint32_t bq = (uint32_t)(na * a.Hq * rowb), bk = (uint32_t)(na * a.Hkv * rowb);
+            // a tensor copy moves its whole box of TT tokens
+            const uint32_t xq = (g.tmap & 1) && bq ? (uint32_t)(g.TT * a.Hq * rowb) : bq;
+            const uint32_t xk = (g.tmap & 2) && bk ? (uint32_t)(g.TT * a.Hkv * rowb) : bk;
+            const int bs = (int)box_start(t0, run.t_hi, g.TT);
             const uint32_t bar = full0 + 8 * s;
-            mbar_expect_tx(bar, bq + bk);
-            if (bq) bulk_g2s(smem_u32(st), (const char *)a.q + t0 * a.Hq * rowb, bq, bar, pol);
-            if (bk) bulk_g2s(smem_u32(st + g.off_k), (const char *)a.k + t0 * a.Hkv * rowb, bk, bar, pol);
+            mbar_expect_tx(bar, xq + xk);
+            if (bq) {
+                if (g.tmap & 1) tensor_g2s(smem_u32(st), &tmq, 0, 0, bs, bar, pol);
+                else bulk_g2s(smem_u32(st), (const char *)a.q + t0 * a.qts, bq, bar, pol);
+            }
+            if (bk) {
+                if (g.tmap & 2) tensor_g2s(smem_u32(st + g.off_k), &tmk, 0, 0, bs, bar, pol);
+                else bulk_g2s(smem_u32(st + g.off_k), (const char *)a.k + t0 * a.kts, bk, bar, pol);
+            }
         };
         // the first ring of copies goes out before any table is built
         const int first = min(g.NS, run.ntiles);
@@ -472,6 +513,10 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g) {
             const int64_t t0 = run.t_lo + (int64_t)it * g.TT;
             const int na = (int)min((int64_t)g.TT, run.t_hi - t0);
             const int rows_q = na * a.Hq, rows = na * (a.Hq + a.Hkv);
+            // tokens of a tensor-copy box before the tile (partial last tile)
+            const int skip = (int)(t0 - box_start(t0, run.t_hi, g.TT));
+            const int xq0 = (g.tmap & 1) ? skip * a.Hq * rowb : 0;
+            const int xk0 = (g.tmap & 2) ? skip * a.Hkv * rowb : 0;
             char *out_q = (char *)a.qo + t0 * a.Hq * rowb;   // the tile's first rows
             char *out_k = (char *)a.ko + t0 * a.Hkv * rowb;
             float *r_q = a.rq + t0 * a.Hq;
@@ -484,7 +529,7 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g) {
                 const int j = p * SLOTS + L.slot;
                 const bool valid = j < rows;
                 const TileRow tr(valid ? j : 0, rows_q, g);
-                const unsigned char *src = st + (tr.isq ? 0 : g.off_k) + tr.jj * rowb;
+                const unsigned char *src = st + (tr.isq ? xq0 : g.off_k + xk0) + tr.jj * rowb;
                 Vec16 xa[U], xb[U];
 #pragma unroll
                 for (int q = 0; q < U; ++q) xa[q] = lds16(src + off1[q]);
@@ -548,7 +593,8 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g) {
 // of both tensors stay in registers for the whole run.
 template <typename T, int LPR, int NCW, int NPW>
 __global__ void __launch_bounds__((NCW + NPW) * 32, 1)
-qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g) {
+qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g, const __grid_constant__ CUtensorMap tmq,
+                     const __grid_constant__ CUtensorMap tmk) {
     using IO = Io<T>;
     constexpr int V = IO::V, W = V / 2;
     constexpr int SLOTS = 32 / LPR;
@@ -559,6 +605,12 @@ qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g) {
     __shared__ volatile int s_abort;
     __shared__ float s_dg[2][kMaxD];
 
+    // tensor copies land on 128-byte boundaries (the stage offsets are
+    // multiples of 128); should the dynamic base not be, report and stop
+    if (g.tmap && (smem_u32(smem) & 127u)) {
+        if (threadIdx.x == 0) atomicOr(&g_qknr_pipe_error, 2u);
+        return;
+    }
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t full0 = smem_u32(&bars[0]), empty0 = smem_u32(&bars[kMaxStages]);
     init_barriers<NCW, NPW>(full0, empty0, g);
@@ -586,14 +638,20 @@ qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g) {
             // producers fill in a tail of up to three floats)
             const uint32_t brq = (uint32_t)(na * a.Hq * 4) & ~15u;
             const uint32_t brk = (uint32_t)(na * a.Hkv * 4) & ~15u;
+            // a tensor copy moves its whole box of TT tokens
+            const uint32_t xq = (g.tmap & 1) && bq ? (uint32_t)(g.TT * a.Hq * rowb) : bq;
+            const uint32_t xk = (g.tmap & 2) && bk ? (uint32_t)(g.TT * a.Hkv * rowb) : bk;
+            const int bs = (int)box_start(t0, run.t_hi, g.TT);
             const uint32_t bar = full0 + 8 * s;
-            mbar_expect_tx(bar, 2 * (bq + bk) + brq + brk);
+            mbar_expect_tx(bar, xq + xk + bq + bk + brq + brk);
             if (bq) {
-                bulk_g2s(smem_u32(st), (const char *)a.q + t0 * a.Hq * rowb, bq, bar, pol);
+                if (g.tmap & 1) tensor_g2s(smem_u32(st), &tmq, 0, 0, bs, bar, pol);
+                else bulk_g2s(smem_u32(st), (const char *)a.q + t0 * a.qts, bq, bar, pol);
                 bulk_g2s(smem_u32(st + g.off_dq), (const char *)a.dqo + t0 * a.Hq * rowb, bq, bar, pol);
             }
             if (bk) {
-                bulk_g2s(smem_u32(st + g.off_k), (const char *)a.k + t0 * a.Hkv * rowb, bk, bar, pol);
+                if (g.tmap & 2) tensor_g2s(smem_u32(st + g.off_k), &tmk, 0, 0, bs, bar, pol);
+                else bulk_g2s(smem_u32(st + g.off_k), (const char *)a.k + t0 * a.kts, bk, bar, pol);
                 bulk_g2s(smem_u32(st + g.off_dk), (const char *)a.dko + t0 * a.Hkv * rowb, bk, bar, pol);
             }
             if (brq) bulk_g2s(smem_u32(st + g.off_rq), a.rq + t0 * a.Hq, brq, bar, pol);
@@ -673,8 +731,12 @@ qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g) {
             const int64_t t0 = run.t_lo + (int64_t)it * g.TT;
             const int na = (int)min((int64_t)g.TT, run.t_hi - t0);
             const int rows_q = na * a.Hq, rows = na * (a.Hq + a.Hkv);
-            char *out_q = (char *)a.dq + t0 * a.Hq * rowb;
-            char *out_k = (char *)a.dk + t0 * a.Hkv * rowb;
+            // tokens of a tensor-copy box before the tile (partial last tile)
+            const int skip = (int)(t0 - box_start(t0, run.t_hi, g.TT));
+            const int xq0 = (g.tmap & 1) ? skip * a.Hq * rowb : 0;
+            const int xk0 = (g.tmap & 2) ? skip * a.Hkv * rowb : 0;
+            char *out_q = (char *)a.dq + t0 * a.dqts;
+            char *out_k = (char *)a.dk + t0 * a.dkts;
             const float4 *cs_tile = reinterpret_cast<const float4 *>(st + g.off_cs);
             const int npass = (rows + SLOTS - 1) / SLOTS;
             int p = (warp - NPW) - pc;
@@ -683,7 +745,7 @@ qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g) {
                 const int j = p * SLOTS + L.slot;
                 const bool valid = j < rows && L.on[0];
                 const TileRow tr(j < rows ? j : 0, rows_q, g);
-                const unsigned char *xs = st + (tr.isq ? 0 : g.off_k) + tr.jj * rowb;
+                const unsigned char *xs = st + (tr.isq ? xq0 : g.off_k + xk0) + tr.jj * rowb;
                 const unsigned char *ds = st + (tr.isq ? g.off_dq : g.off_dk) + tr.jj * rowb;
                 const Vec16 xa = lds16(xs + off1), da = lds16(ds + off1);
                 const Vec16 xb = lds16(xs + off2), db = lds16(ds + off2);
@@ -728,7 +790,10 @@ qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g) {
                         IO::put2(oa, k, va.x, va.y);
                         IO::put2(ob, k, vb.x, vb.y);
                     }
-                    char *out = (tr.isq ? out_q : out_k) + tr.jj * rowb;
+                    // row (tl, h) of dq / dk, whose tokens may be strided
+                    const int hz = tr.isq ? a.Hq : a.Hkv;
+                    char *out = (tr.isq ? out_q : out_k) + (int64_t)tr.tl * (tr.isq ? a.dqts : a.dkts) +
+                                (tr.jj - tr.tl * hz) * rowb;
                     stg16(out + off1, oa);
                     stg16(out + off2, ob);
                 }

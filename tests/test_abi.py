@@ -127,3 +127,40 @@ def test_binding_refuses_cpu_tensors():
     q = torch.zeros(1, 2, 1, 16)
     with pytest.raises(ValueError):
         qknr.qk_norm_rope_fwd(q, q, q[0, 0, 0], q[0, 0, 0], rotary_dim=16, theta=1e4, eps=1e-6)
+
+
+def fwd_strided(lib, qts, kts, B=2, S=8, Hq=4, Hkv=2, D=64, R=64, dt=BF16, **ptrs):
+    p = dict(q=P(1), k=P(2), gq=P(3), gk=P(4), pos=None, qo=P(5), ko=P(6), rq=P(7), rk=P(8))
+    p.update(ptrs)
+    return lib.qk_norm_rope_fwd_strided(p["q"], p["k"], qts, kts, p["gq"], p["gk"], p["pos"],
+                                        p["qo"], p["ko"], p["rq"], p["rk"], B, S, Hq, Hkv, D, R,
+                                        1e4, 1e-6, dt, None)
+
+
+def bwd_strided(lib, qts, kts, dqts, dkts, B=2, S=8, Hq=4, Hkv=2, D=64, R=64, dt=BF16, **ptrs):
+    p = dict(q=P(1), k=P(2), gq=P(3), gk=P(4), pos=None, rq=P(7), rk=P(8), dqo=P(9),
+             dko=P(10), dq=P(11), dk=P(12), dgq=P(13), dgk=P(14))
+    p.update(ptrs)
+    return lib.qk_norm_rope_bwd_strided(p["q"], p["k"], qts, kts, p["gq"], p["gk"], p["pos"],
+                                        p["rq"], p["rk"], p["dqo"], p["dko"], p["dq"], p["dk"],
+                                        dqts, dkts, p["dgq"], p["dgk"], B, S, Hq, Hkv, D, R,
+                                        1e4, 1e-6, dt, None)
+
+
+def test_strided_validation(lib):
+    ts = (4 + 2 * 2) * 64                       # a fused QKV row: Hq + 2 Hkv heads
+    assert fwd_strided(lib, 4 * 64 - 8, ts) == INVALID       # token step shorter than its rows
+    assert fwd_strided(lib, ts, 2 * 64 - 1) == INVALID
+    assert fwd_strided(lib, ts + 4, ts) == ALIGN              # 8-byte step (bf16)
+    assert fwd_strided(lib, ts, ts, dt=F32, D=64, R=64, q=P(1, 8)) == ALIGN
+    assert fwd_strided(lib, ts, ts, D=63) == INVALID          # shape checks still apply
+    # q_out over a strided q's bytes (fwd outputs are dense)
+    assert fwd_strided(lib, ts, ts, qo=P(1, 64)) == INVALID
+    assert bwd_strided(lib, ts, ts, ts, 2 * 64 - 2) == INVALID      # dk step < Hkv * D
+    assert bwd_strided(lib, ts, ts, ts + 4, ts) == ALIGN
+    # strided dq and dk whose rows overlap (dk 64 bytes into dq's rows)
+    assert bwd_strided(lib, ts, ts, ts, ts, dk=P(11, 64)) == INVALID
+    # dq on top of the strided q
+    assert bwd_strided(lib, ts, ts, ts, ts, dq=P(1)) == INVALID
+    # a strided dq may not alias dq_out
+    assert bwd_strided(lib, ts, ts, ts, ts, dq=P(9)) == INVALID
