@@ -71,6 +71,9 @@ class Oracle:
         lib.oracle_bwd_rows.restype = None
         lib.oracle_bwd_rows.argtypes = [_D, _D, _D, _I64, c_i64, c_int, c_int,
                                         c_dbl, c_dbl, _D, _D]
+        lib.oracle_rope_rows.restype = None
+        lib.oracle_rope_rows.argtypes = [_D, _I64, c_i64, c_int, c_int, c_dbl,
+                                         c_int, _D]
 
     # ---------------------------------------------------------------- scalars
     def inv_freq(self, i: int, R: int, theta: float) -> float:
@@ -143,6 +146,30 @@ class Oracle:
         self.lib.oracle_bwd_rows(_p(x), _p(g), _p(dy), _p(m, _I64), n, D, R,
                                  float(theta), float(eps), _p(dx), _p(dgr))
         return dx, dgr
+
+
+    def rope_rows(self, x, m, R: int, theta: float, inverse: bool = False):
+        """Rotation alone of rows x [n, D] at positions m [n]: R(m) x, or
+        R(m)^T x with ``inverse``."""
+        x = as_f64(x)
+        n, D = x.shape
+        m = np.ascontiguousarray(np.asarray(m, dtype=np.int64).reshape(n))
+        y = np.empty_like(x)
+        self.lib.oracle_rope_rows(_p(x), _p(m, _I64), n, D, R, float(theta),
+                                  1 if inverse else 0, _p(y))
+        return y
+
+    def rope(self, q, k, m, R: int, theta: float, inverse: bool = False):
+        """Rotation alone over tokens: q [..., Hq, D], k [..., Hkv, D],
+        m per-token positions (len T). Returns fp64 (q_out, k_out)."""
+        m = np.asarray(m, dtype=np.int64).reshape(-1)
+        out = []
+        for x in (as_f64(q), as_f64(k)):
+            H, D = x.shape[-2], x.shape[-1]
+            rows = x.reshape(-1, D)
+            y = self.rope_rows(rows, np.repeat(m, H), R, theta, inverse)
+            out.append(y.reshape(x.shape))
+        return out[0], out[1]
 
 
 _default: Optional[Oracle] = None

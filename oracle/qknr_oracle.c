@@ -38,6 +38,10 @@
  *   dgamma_d += g_d * x_d * r                        (summed over the tensor's rows)
  *   h_d     = g_d * gamma_d
  *   dx_d    = r * h_d - r^3 * x_d * (1/D) * sum_e h_e x_e
+ * Rotation alone (no normalisation), forward or inverse:
+ *   y = R(m) x, or y = R(m)^T x = R(-m) x, which strips RoPE from a rotated
+ *   row (the cross-model KV cache transfer abstract on the papers listing:
+ *   keys have RoPE stripped before mapping so the fit is position-free).
  */
 #include <math.h>
 #include <stdint.h>
@@ -187,5 +191,29 @@ void oracle_bwd_rows(const double *x, const double *gamma, const double *dy,
         memset(dgamma_rows + j * D, 0, sizeof(double) * (size_t)D);
         oracle_bwd_row(x + j * D, gamma, dy + j * D, D, R, theta, eps, m[j],
                        dx + j * D, dgamma_rows + j * D);
+    }
+}
+
+/*
+ * Rotation alone, rows x [n, D] at positions m [n]: y = R(m) x, or with
+ * inverse != 0 the transpose R(m)^T x (sine negated). Dims >= R copy through.
+ */
+void oracle_rope_rows(const double *x, const int64_t *m, int64_t n, int D,
+                      int R, double theta, int inverse, double *y)
+{
+    int half = R / 2;
+    for (int64_t j = 0; j < n; ++j) {
+        const double *xr = x + j * D;
+        double *yr = y + j * D;
+        for (int d = 0; d < D; ++d)
+            yr[d] = xr[d];
+        for (int i = 0; i < half; ++i) {
+            double phi = (double)m[j] * oracle_inv_freq(i, R, theta);
+            double c = cos(phi), s = sin(phi);
+            if (inverse)
+                s = -s;
+            yr[i] = xr[i] * c - xr[i + half] * s;
+            yr[i + half] = xr[i + half] * c + xr[i] * s;
+        }
     }
 }

@@ -349,4 +349,41 @@ def pin_gradients_nonzero(orc):
         assert np.count_nonzero(a) == a.size, f"{name} has exact zeros"
 
 
+# ------------------------------------------------------------ rotation alone
+def pin_rope_matches_complex(orc):
+    """Rotation alone equals complex multiplication by exp(j m w_i) on the
+    first R dims (a library routine), dims >= R copied."""
+    rng = np.random.default_rng(31)
+    for D, R in ((64, 64), (128, 32), (16, 0)):
+        x = _rows(rng, 6, D, 2.0)
+        m = rng.integers(-70000, 70000, 6)
+        y = orc.rope_rows(x, m, R, 1e6)
+        _close(y, _complex_rope(x, m, R, 1e6), tol=1e-12, what=f"rope D={D} R={R}")
+
+
+def pin_rope_inverse(orc):
+    """The inverse rotation is the transpose: it undoes the forward one, and
+    equals the forward rotation at -m."""
+    rng = np.random.default_rng(32)
+    D, R = 32, 24
+    x = _rows(rng, 5, D)
+    m = rng.integers(0, 2 ** 31 - 1, 5)
+    y = orc.rope_rows(x, m, R, 1e4)
+    _close(orc.rope_rows(y, m, R, 1e4, inverse=True), x, tol=1e-12, what="inverse after fwd")
+    _close(orc.rope_rows(x, m, R, 1e4, inverse=True), orc.rope_rows(x, -m, R, 1e4),
+           tol=1e-15, what="inverse = fwd at -m")
+    assert not np.allclose(orc.rope_rows(x, m, R, 1e4, inverse=True), y), "inverse == fwd"
+
+
+def pin_rope_is_fwd_without_norm(orc):
+    """With gamma = 1 and eps = 0 the fused forward is the rotation of x * r,
+    so dividing by r recovers the rotation alone."""
+    rng = np.random.default_rng(33)
+    D, R = 48, 32
+    x = _rows(rng, 4, D, 3.0)
+    m = rng.integers(0, 9000, 4)
+    y, r = orc.fwd_rows(x, np.ones(D), m, R, 5e5, 0.0)
+    _close(orc.rope_rows(x, m, R, 5e5), y / r[:, None], tol=1e-12, what="rope vs fwd / r")
+
+
 ALL_PINS = [v for k_, v in sorted(globals().items()) if k_.startswith("pin_")]

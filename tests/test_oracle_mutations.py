@@ -62,6 +62,12 @@ MUTATIONS = [
                             "oracle_fwd_row(q + row * D, gamma_q, D, R, theta, eps, (int64_t)t,", 0)]),
     ("bwd_k_dgamma_into_q", [("theta, eps, m[t], dk + row * D, dgamma_k);",
                               "theta, eps, m[t], dk + row * D, dgamma_q);", 0)]),
+    ("rope_inverse_ignored", [("            s = -s;", "            s = s;", 0)]),
+    ("rope_sin_sign_first", [("yr[i] = xr[i] * c - xr[i + half] * s;",
+                              "yr[i] = xr[i] * c + xr[i + half] * s;", 0)]),
+    ("rope_pass_through_zeroed", [("            yr[d] = xr[d];", "            yr[d] = 0.0;", 0)]),
+    ("rope_position_plus_one", [("double phi = (double)m[j] * oracle_inv_freq(i, R, theta);",
+                                 "double phi = (double)(m[j] + 1) * oracle_inv_freq(i, R, theta);", 0)]),
 ]
 
 
