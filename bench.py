@@ -190,18 +190,34 @@ def aggregate_tokens_per_s(world: int, tokens_per_rank: int, ms_per_step: float)
 
 # ---------------------------------------------------------------- our arm
 class Set:
-    """Device buffers of one batch: inputs, forward outputs, gradients."""
+    """Device buffers of one batch: inputs, forward outputs, gradients. With
+    layout "qkv", q and k are slices of a fused QKV projection buffer
+    [B, S, (Hq + 2 Hkv) D] and dq, dk slices of a dQKV buffer (the V slots
+    are never touched by the op)."""
 
-    def __init__(self, inp: workloads.Inputs, dev):
+    def __init__(self, inp: workloads.Inputs, dev, layout: str = "dense"):
         w = inp.w
         self.q, self.k = inp.q.to(dev), inp.k.to(dev)
+        if layout == "qkv":
+            import qk_rmsnorm_rope_norm_b200 as qknr
+            width = (w.Hq + 2 * w.Hkv) * w.D
+            self.qkv = torch.zeros((w.B, w.S, width), dtype=self.q.dtype, device=dev)
+            q, k, _ = qknr.split_qkv(self.qkv, w.Hq, w.Hkv)
+            q.copy_(self.q)
+            k.copy_(self.k)
+            self.q, self.k = q, k
         self.gq, self.gk = inp.gamma_q.to(dev), inp.gamma_k.to(dev)
         self.pos = None if inp.pos is None else inp.pos.to(dev)
         self.dqo, self.dko = inp.dq_out.to(dev), inp.dk_out.to(dev)
-        self.qo, self.ko = torch.empty_like(self.q), torch.empty_like(self.k)
+        self.qo = torch.empty(self.q.shape, dtype=self.q.dtype, device=dev)
+        self.ko = torch.empty(self.k.shape, dtype=self.k.dtype, device=dev)
         self.rq = torch.empty((w.B, w.S, w.Hq), dtype=torch.float32, device=dev)
         self.rk = torch.empty((w.B, w.S, w.Hkv), dtype=torch.float32, device=dev)
-        self.dq, self.dk = torch.empty_like(self.q), torch.empty_like(self.k)
+        self.dq = torch.empty(self.q.shape, dtype=self.q.dtype, device=dev)
+        self.dk = torch.empty(self.k.shape, dtype=self.k.dtype, device=dev)
+        if layout == "qkv":
+            self.dqkv = torch.zeros_like(self.qkv)
+            self.dq, self.dk, _ = qknr.split_qkv(self.dqkv, w.Hq, w.Hkv)
         self.dgq = torch.empty(w.D, dtype=torch.float32, device=dev)
         self.dgk = torch.empty(w.D, dtype=torch.float32, device=dev)
 
@@ -212,7 +228,7 @@ def run_ours(args, w, inp, rank, local_rank, world):
     qknr.load_library()
     cfg = dict(rotary_dim=w.rotary_dim, theta=w.theta, eps=w.eps)
     nsets = args.sets
-    sets = [Set(inp, dev) for _ in range(nsets)]
+    sets = [Set(inp, dev, args.layout) for _ in range(nsets)]
     stream = torch.cuda.current_stream(dev)
     fwd = [qknr.prepare_fwd(s.q, s.k, s.gq, s.gk, s.pos, s.qo, s.ko, s.rq, s.rk, **cfg)
            for s in sets]
@@ -259,6 +275,79 @@ def run_ours(args, w, inp, rank, local_rank, world):
     floor = {"fwd_ms": copy_floor_ms(cb["fwd"], dev), "bwd_ms": copy_floor_ms(cb["bwd"], dev)}
     return dict(total_ms=total_ms, fwd_ms=fwd_ms, bwd_ms=bwd_ms, clocks=clocks.summary(),
                 e2e=e2e, floor=floor)
+
+
+def run_variants(args, w, inp, dev, peak):
+    """The other entry points on the same workload, each timed like the main
+    step (a ring of input sets, CUDA events around every launch, mean over
+    the launches): the fused op on Q / K slices of a fused QKV buffer, the
+    NoPE op (qk_norm_*), and the rotation alone, forward and inverse
+    (qk_rope_apply). Bytes are each call's contract bytes."""
+    import qk_rmsnorm_rope_norm_b200 as qknr
+    lib = qknr.load_library()
+    cfg = dict(rotary_dim=w.rotary_dim, theta=w.theta, eps=w.eps)
+    stream = torch.cuda.current_stream(dev)
+    n_launch = max(50, min(args.steps, 400))
+    e = w.elem_bytes
+    rows = inp.q.numel() // w.D + inp.k.numel() // w.D
+    T = w.B * w.S
+    pos_b = 4 * T if inp.pos is not None else 0
+    cb = workloads.contract_bytes(w, with_pos=inp.pos is not None)
+    cb_nope = workloads.contract_bytes(w, with_pos=False)
+
+    def timed(calls):
+        for c in calls[:3]:
+            c()
+        torch.cuda.synchronize(dev)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(n_launch)]
+        for i, (a, b) in enumerate(ev):
+            a.record(stream)
+            calls[i % len(calls)]()
+            b.record(stream)
+        torch.cuda.synchronize(dev)
+        return sum(a.elapsed_time(b) for a, b in ev) / n_launch
+
+    def line(ms, nbytes):
+        gbs = nbytes / (ms / 1e3) / 1e9
+        return {"ms": ms, "gbs": gbs, "frac": gbs / peak, "bytes_per_launch": nbytes}
+
+    out = {}
+    qkv = [Set(inp, dev, "qkv") for _ in range(args.sets)]
+    f = [qknr.prepare_fwd(s.q, s.k, s.gq, s.gk, s.pos, s.qo, s.ko, s.rq, s.rk, **cfg) for s in qkv]
+    b = [qknr.prepare_bwd(s.q, s.k, s.gq, s.gk, s.pos, s.rq, s.rk, s.dqo, s.dko, s.dq, s.dk,
+                          s.dgq, s.dgk, **cfg) for s in qkv]
+    out["fused_qkv_layout"] = {"fwd": line(timed(f), cb["fwd"]), "bwd": line(timed(b), cb["bwd"]),
+                               "entry": "qk_norm_rope_fwd_strided / qk_norm_rope_bwd_strided"}
+    del qkv, f, b
+    dense = [Set(inp, dev) for _ in range(args.sets)]
+    P = qknr._ptr
+    dt = 0 if w.dtype == "f32" else 1
+    st = qknr._stream(None)
+
+    def nope_fwd(s):
+        a = (P(s.q), P(s.k), P(s.gq), P(s.gk), P(s.qo), P(s.ko), P(s.rq), P(s.rk), w.B, w.S,
+             w.Hq, w.Hkv, w.D, float(w.eps), dt, st)
+        return qknr.PreparedCall(lib.qk_norm_fwd, a, "qk_norm_fwd", s)
+
+    def nope_bwd(s):
+        a = (P(s.q), P(s.k), P(s.gq), P(s.gk), P(s.rq), P(s.rk), P(s.dqo), P(s.dko), P(s.dq),
+             P(s.dk), P(s.dgq), P(s.dgk), w.B, w.S, w.Hq, w.Hkv, w.D, float(w.eps), dt, st)
+        return qknr.PreparedCall(lib.qk_norm_bwd, a, "qk_norm_bwd", s)
+
+    def rope(s, inverse):
+        a = (P(s.q), P(s.k), P(s.pos), P(s.qo), P(s.ko), w.B, w.S, w.Hq, w.Hkv, w.D,
+             w.rotary_dim, float(w.theta), 1 if inverse else 0, dt, st)
+        return qknr.PreparedCall(lib.qk_rope_apply, a, "qk_rope_apply", s)
+
+    out["nope_qk_norm"] = {"fwd": line(timed([nope_fwd(s) for s in dense]), cb_nope["fwd"]),
+                           "bwd": line(timed([nope_bwd(s) for s in dense]), cb_nope["bwd"]),
+                           "entry": "qk_norm_fwd / qk_norm_bwd"}
+    rope_bytes = 2 * rows * w.D * e + pos_b
+    out["rope_only"] = {"fwd": line(timed([rope(s, False) for s in dense]), rope_bytes),
+                        "inverse": line(timed([rope(s, True) for s in dense]), rope_bytes),
+                        "entry": "qk_rope_apply"}
+    return out
 
 
 def copy_floor_ms(traffic_bytes: int, dev, n: int = 20) -> float:
@@ -380,6 +469,7 @@ def config_of(w, inp, world):
                   f"L2-resident (> 2x 126 MB of traffic between touches)"
                   if getattr(cfg_args, "sets", NSETS) == NSETS else
                   f"{cfg_args.sets} input set(s): profiling run, inputs may be L2-resident",
+            "layout": getattr(cfg_args, "layout", "dense"),
             "parallelism": f"dp{world} (weak, no data-path collective)"}
 
 
@@ -421,6 +511,11 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--variants", action="store_true",
+                    help="also time the fused-QKV, NoPE and rotation-only entry points")
+    ap.add_argument("--layout", choices=["dense", "qkv"], default="dense",
+                    help="dense [B,S,H,D] q/k, or q/k read from (and dq/dk written into) "
+                         "fused QKV buffers")
     args = ap.parse_args()
     global cfg_args
     cfg_args = args
@@ -496,6 +591,8 @@ def main():
                        "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"],
                        "ms_per_step": e["ms"], "steps": e["steps"]}
     line["cpu_baseline"] = cpu
+    if args.variants and world == 1:
+        line["variants"] = run_variants(args, w, inp, torch.device("cuda", local_rank), peak)
     print(json.dumps(line), flush=True)
 
 

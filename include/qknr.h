@@ -186,6 +186,48 @@ QKNR_API qknr_status qk_norm_rope_bwd_strided(const void *q, const void *k,
                              int rotary_dim, float theta, float eps,
                              qknr_dtype dtype, qknr_stream_t stream);
 
+/*
+ * Per-head QK-RMSNorm alone, for the layers that use no positional
+ * embedding ("Rope to Nope and Back Again: A New Hybrid Attention Strategy",
+ * abstract: NoPE and QK-Norm layers; "Fractional Rotation, Full Potential?",
+ * abstract: NoPE stabilised by QK-Norm). The same op as qk_norm_rope_fwd /
+ * _bwd with rotary_dim = 0 (no positions, no theta): q_out = q * r * gamma_q,
+ * and the backward of it. Arguments, layouts and errors as there.
+ */
+QKNR_API qknr_status qk_norm_fwd(const void *q, const void *k,
+                             const void *gamma_q, const void *gamma_k,
+                             void *q_out, void *k_out,
+                             float *rstd_q, float *rstd_k,
+                             int B, int S, int Hq, int Hkv, int D, float eps,
+                             qknr_dtype dtype, qknr_stream_t stream);
+
+QKNR_API qknr_status qk_norm_bwd(const void *q, const void *k,
+                             const void *gamma_q, const void *gamma_k,
+                             const float *rstd_q, const float *rstd_k,
+                             const void *dq_out, const void *dk_out,
+                             void *dq, void *dk,
+                             float *dgamma_q, float *dgamma_k,
+                             int B, int S, int Hq, int Hkv, int D, float eps,
+                             qknr_dtype dtype, qknr_stream_t stream);
+
+/*
+ * Rotate-half RoPE alone, no normalisation: q_out = R(m) q, k_out = R(m) k
+ * over the first rotary_dim dims (the rest copied), or with inverse != 0
+ * the transpose R(m)^T = R(-m), which strips RoPE from rotated rows, e.g.
+ * cached keys before a position-free mapping (cross-model KV cache
+ * transfer, abstract, on the papers listing the sources include). The
+ * gradient of either direction is the other direction applied to the
+ * upstream gradient, so there is no separate backward. Positions, layouts,
+ * aliasing (q_out may be q) and errors as for qk_norm_rope_fwd; no gamma,
+ * no eps, no rstd.
+ */
+QKNR_API qknr_status qk_rope_apply(const void *q, const void *k,
+                             const int32_t *pos_ids,
+                             void *q_out, void *k_out,
+                             int B, int S, int Hq, int Hkv, int D,
+                             int rotary_dim, float theta, int inverse,
+                             qknr_dtype dtype, qknr_stream_t stream);
+
 /* Static English text for a status code; never NULL. */
 QKNR_API const char *qknr_strerror(qknr_status status);
 

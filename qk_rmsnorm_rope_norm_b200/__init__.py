@@ -23,6 +23,7 @@ import torch
 
 __all__ = ["qk_norm_rope_fwd", "qk_norm_rope_bwd", "qknr_strerror", "QKNormRoPE",
            "QKNormRoPEFromQKV", "qk_norm_rope_qkv", "split_qkv",
+           "qk_norm_fwd", "qk_norm_bwd", "qk_rope_apply", "QKRoPE",
            "prepare_fwd", "prepare_bwd", "PreparedCall",
            "qk_norm_rope", "QKNRError", "library_path", "load_library", "pipeline_error"]
 
@@ -66,6 +67,12 @@ def load_library():
     lib.qk_norm_rope_fwd_strided.restype = i32
     lib.qk_norm_rope_fwd_strided.argtypes = [vp, vp, i64, i64] + [vp] * 7 + [i32] * 6 + \
         [f32, f32, i32, vp]
+    lib.qk_norm_fwd.restype = i32
+    lib.qk_norm_fwd.argtypes = [vp] * 8 + [i32] * 5 + [f32, i32, vp]
+    lib.qk_norm_bwd.restype = i32
+    lib.qk_norm_bwd.argtypes = [vp] * 12 + [i32] * 5 + [f32, i32, vp]
+    lib.qk_rope_apply.restype = i32
+    lib.qk_rope_apply.argtypes = [vp] * 5 + [i32] * 6 + [f32, i32, i32, vp]
     lib.qk_norm_rope_bwd_strided.restype = i32
     lib.qk_norm_rope_bwd_strided.argtypes = [vp, vp, i64, i64] + [vp] * 9 + [i64, i64] + \
         [vp] * 2 + [i32] * 6 + [f32, f32, i32, vp]
@@ -289,6 +296,117 @@ def qk_norm_rope(q, k, gamma_q, gamma_k, pos_ids=None, *, rotary_dim: int, theta
                  eps: float):
     """Differentiable fused op; returns ``(q_out, k_out)``."""
     return QKNormRoPE.apply(q, k, gamma_q, gamma_k, pos_ids, rotary_dim, theta, eps)
+
+
+def qk_norm_fwd(q, k, gamma_q, gamma_k, *, eps: float, q_out=None, k_out=None,
+                rstd_q=None, rstd_k=None, stream=None):
+    """Per-head QK-RMSNorm alone (the NoPE layers' op, C ``qk_norm_fwd``).
+    Returns ``(q_out, k_out, rstd_q, rstd_k)``; tensors as for
+    ``qk_norm_rope_fwd`` (dense)."""
+    lib = load_library()
+    for n, t in (("q", q), ("k", k), ("gamma_q", gamma_q), ("gamma_k", gamma_k)):
+        _need_cuda(n, t)
+    B, S, Hq, Hkv, D = _shape(q, k)
+    _same_dtype(q, k, gamma_q, gamma_k)
+    q_out = torch.empty_like(q) if q_out is None else q_out
+    k_out = torch.empty_like(k) if k_out is None else k_out
+    rstd_q = torch.empty((B, S, Hq), dtype=torch.float32, device=q.device) if rstd_q is None else rstd_q
+    rstd_k = torch.empty((B, S, Hkv), dtype=torch.float32, device=q.device) if rstd_k is None else rstd_k
+    _check_outputs(q, k, q_out, k_out, rstd_q, rstd_k)
+    st = lib.qk_norm_fwd(_ptr(q), _ptr(k), _ptr(gamma_q), _ptr(gamma_k), _ptr(q_out), _ptr(k_out),
+                         _ptr(rstd_q), _ptr(rstd_k), B, S, Hq, Hkv, D, float(eps),
+                         _DTYPES[q.dtype], _stream(stream))
+    if st != QKNR_OK:
+        raise QKNRError(st, "qk_norm_fwd")
+    return q_out, k_out, rstd_q, rstd_k
+
+
+def qk_norm_bwd(q, k, gamma_q, gamma_k, rstd_q, rstd_k, dq_out, dk_out, *, eps: float,
+                dq=None, dk=None, dgamma_q=None, dgamma_k=None, stream=None):
+    """Backward of ``qk_norm_fwd`` (C ``qk_norm_bwd``); returns
+    ``(dq, dk, dgamma_q, dgamma_k)``, dgamma fp32 [D]."""
+    lib = load_library()
+    for n, t in (("q", q), ("k", k), ("gamma_q", gamma_q), ("gamma_k", gamma_k),
+                 ("rstd_q", rstd_q), ("rstd_k", rstd_k), ("dq_out", dq_out), ("dk_out", dk_out)):
+        _need_cuda(n, t)
+    B, S, Hq, Hkv, D = _shape(q, k)
+    _same_dtype(q, k, gamma_q, gamma_k, dq_out, dk_out)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dgamma_q = torch.empty(D, dtype=torch.float32, device=q.device) if dgamma_q is None else dgamma_q
+    dgamma_k = torch.empty(D, dtype=torch.float32, device=q.device) if dgamma_k is None else dgamma_k
+    for n, t in (("dq", dq), ("dk", dk), ("dgamma_q", dgamma_q), ("dgamma_k", dgamma_k)):
+        _need_cuda(n, t)
+    st = lib.qk_norm_bwd(_ptr(q), _ptr(k), _ptr(gamma_q), _ptr(gamma_k), _ptr(rstd_q),
+                         _ptr(rstd_k), _ptr(dq_out), _ptr(dk_out), _ptr(dq), _ptr(dk),
+                         _ptr(dgamma_q), _ptr(dgamma_k), B, S, Hq, Hkv, D, float(eps),
+                         _DTYPES[q.dtype], _stream(stream))
+    if st != QKNR_OK:
+        raise QKNRError(st, "qk_norm_bwd")
+    return dq, dk, dgamma_q, dgamma_k
+
+
+def qk_rope_apply(q, k, pos_ids=None, *, rotary_dim: int, theta: float, inverse: bool = False,
+                  q_out=None, k_out=None, stream=None):
+    """Rotate-half RoPE alone (C ``qk_rope_apply``): R(m) q, R(m) k, or with
+    ``inverse`` the transpose R(-m), which strips RoPE from rotated rows.
+    Returns ``(q_out, k_out)``; ``q_out=q`` runs in place."""
+    lib = load_library()
+    for n, t in (("q", q), ("k", k)):
+        _need_cuda(n, t)
+    B, S, Hq, Hkv, D = _shape(q, k)
+    _same_dtype(q, k)
+    if pos_ids is not None:
+        _need_cuda("pos_ids", pos_ids)
+        if pos_ids.dtype != torch.int32 or tuple(pos_ids.shape) != (B, S):
+            raise ValueError("pos_ids must be int32 [B, S]")
+    q_out = torch.empty_like(q) if q_out is None else q_out
+    k_out = torch.empty_like(k) if k_out is None else k_out
+    for n, t in (("q_out", q_out), ("k_out", k_out)):
+        _need_cuda(n, t)
+    if q_out.shape != q.shape or k_out.shape != k.shape or q_out.dtype != q.dtype \
+            or k_out.dtype != q.dtype:
+        raise ValueError("q_out / k_out must match q / k in shape and dtype")
+    st = lib.qk_rope_apply(_ptr(q), _ptr(k), _ptr(pos_ids), _ptr(q_out), _ptr(k_out), B, S, Hq,
+                           Hkv, D, int(rotary_dim), float(theta), 1 if inverse else 0,
+                           _DTYPES[q.dtype], _stream(stream))
+    if st != QKNR_OK:
+        raise QKNRError(st, "qk_rope_apply")
+    return q_out, k_out
+
+
+class QKRoPE(torch.autograd.Function):
+    """Autograd wrapper of ``qk_rope_apply``: the gradient of a rotation is
+    the opposite rotation of the upstream gradient."""
+
+    @staticmethod
+    def forward(ctx, q, k, pos_ids, rotary_dim, theta, inverse):
+        ctx.cfg = (pos_ids, rotary_dim, theta, inverse)
+        return qk_rope_apply(q, k, pos_ids, rotary_dim=rotary_dim, theta=theta, inverse=inverse)
+
+    @staticmethod
+    def backward(ctx, dq_out, dk_out):
+        pos_ids, R, theta, inverse = ctx.cfg
+        dq, dk = qk_rope_apply(dq_out.contiguous(), dk_out.contiguous(), pos_ids, rotary_dim=R,
+                               theta=theta, inverse=not inverse)
+        return dq, dk, None, None, None, None
+
+
+def _same_dtype(*ts):
+    if ts[0].dtype not in _DTYPES or any(t.dtype != ts[0].dtype for t in ts):
+        raise ValueError("tensors must share one dtype (float32 or bfloat16)")
+
+
+def _check_outputs(q, k, q_out, k_out, rstd_q, rstd_k):
+    B, S, Hq, Hkv, D = _shape(q, k)
+    for n, t in (("q_out", q_out), ("k_out", k_out), ("rstd_q", rstd_q), ("rstd_k", rstd_k)):
+        _need_cuda(n, t)
+    if q_out.shape != q.shape or k_out.shape != k.shape or q_out.dtype != q.dtype \
+            or k_out.dtype != q.dtype:
+        raise ValueError("q_out / k_out must match q / k in shape and dtype")
+    if rstd_q.dtype != torch.float32 or rstd_k.dtype != torch.float32 or \
+            tuple(rstd_q.shape) != (B, S, Hq) or tuple(rstd_k.shape) != (B, S, Hkv):
+        raise ValueError("rstd_q / rstd_k must be float32 [B,S,Hq] / [B,S,Hkv]")
 
 
 def split_qkv(qkv: torch.Tensor, Hq: int, Hkv: int):

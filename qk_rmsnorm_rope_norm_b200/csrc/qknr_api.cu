@@ -468,14 +468,20 @@ qknr_status fwd_impl(const void *q, const void *k, int64_t q_ts, int64_t k_ts,
                      const void *gamma_q, const void *gamma_k, const int32_t *pos_ids, void *q_out,
                      void *k_out, float *rstd_q, float *rstd_k, int B, int S, int Hq, int Hkv,
                      int D, int rotary_dim, float theta, float eps, qknr_dtype dtype,
-                     qknr_stream_t stream) {
+                     qknr_stream_t stream, int mode = 0) {
     qknr_status st = check_shape(B, S, Hq, Hkv, D, rotary_dim, theta, eps, dtype);
     if (st != QKNR_OK) return st;
     const int64_t T = (int64_t)B * S;
     if (T == 0 || Hq + Hkv == 0) return QKNR_OK;
     const size_t e = dtype == QKNR_F32 ? 4 : 2;
-    if (Hq > 0 && (!q || !q_out || !rstd_q || !gamma_q)) return QKNR_ERR_INVALID_ARG;
-    if (Hkv > 0 && (!k || !k_out || !rstd_k || !gamma_k)) return QKNR_ERR_INVALID_ARG;
+    if (mode & kModeRopeOnly) {  // rotation alone: no gamma, no rstd
+        gamma_q = gamma_k = nullptr;
+        rstd_q = rstd_k = nullptr;
+        if ((Hq > 0 && (!q || !q_out)) || (Hkv > 0 && (!k || !k_out))) return QKNR_ERR_INVALID_ARG;
+    } else {
+        if (Hq > 0 && (!q || !q_out || !rstd_q || !gamma_q)) return QKNR_ERR_INVALID_ARG;
+        if (Hkv > 0 && (!k || !k_out || !rstd_k || !gamma_k)) return QKNR_ERR_INVALID_ARG;
+    }
     if ((st = check_stride(q_ts, Hq, D, e)) != QKNR_OK) return st;
     if ((st = check_stride(k_ts, Hkv, D, e)) != QKNR_OK) return st;
     const void *vec[] = {q, k, gamma_q, gamma_k, q_out, k_out};
@@ -492,7 +498,7 @@ qknr_status fwd_impl(const void *q, const void *k, int64_t q_ts, int64_t k_ts,
         {(const char *)gamma_q, Hq ? D * e : 0}, {(const char *)gamma_k, Hkv ? D * e : 0},
         {(const char *)pos_ids, pos_ids ? (size_t)T * 4 : 0},
         {(const char *)q_out, nq * D * e},      {(const char *)k_out, nk * D * e},
-        {(const char *)rstd_q, nq * 4},         {(const char *)rstd_k, nk * 4},
+        {(const char *)rstd_q, rstd_q ? nq * 4 : 0}, {(const char *)rstd_k, rstd_k ? nk * 4 : 0},
     };
     const int may_equal[] = {0, 1, -1, -1};  // q_out may be a dense q, k_out a dense k
     if (check_overlaps(all, 9, 5, may_equal) != QKNR_OK) return QKNR_ERR_INVALID_ARG;
@@ -502,7 +508,7 @@ qknr_status fwd_impl(const void *q, const void *k, int64_t q_ts, int64_t k_ts,
     a.qo = q_out; a.ko = k_out; a.rq = rstd_q; a.rk = rstd_k;
     a.qts = q_ts * (int64_t)e; a.kts = k_ts * (int64_t)e;
     a.T = T; a.S = S; a.Hq = Hq; a.Hkv = Hkv; a.D = D; a.R = rotary_dim;
-    a.theta = theta; a.eps = eps;
+    a.theta = theta; a.eps = eps; a.mode = mode;
     const int lpr = lanes_per_row(D, (int)e);
     cudaStream_t cs = (cudaStream_t)stream;
     return dtype == QKNR_F32 ? dispatch_fwd<float>(a, lpr, cs)
@@ -623,6 +629,35 @@ extern "C" qknr_status qk_norm_rope_bwd_strided(
     return bwd_impl(q, k, q_token_stride, k_token_stride, gamma_q, gamma_k, pos_ids, rstd_q,
                     rstd_k, dq_out, dk_out, dq, dk, dq_token_stride, dk_token_stride, dgamma_q,
                     dgamma_k, B, S, Hq, Hkv, D, rotary_dim, theta, eps, dtype, stream);
+}
+
+extern "C" qknr_status qk_norm_fwd(const void *q, const void *k, const void *gamma_q,
+                                   const void *gamma_k, void *q_out, void *k_out, float *rstd_q,
+                                   float *rstd_k, int B, int S, int Hq, int Hkv, int D, float eps,
+                                   qknr_dtype dtype, qknr_stream_t stream) {
+    return fwd_impl(q, k, (int64_t)Hq * D, (int64_t)Hkv * D, gamma_q, gamma_k, nullptr, q_out,
+                    k_out, rstd_q, rstd_k, B, S, Hq, Hkv, D, 0, 1.0f, eps, dtype, stream);
+}
+
+extern "C" qknr_status qk_norm_bwd(const void *q, const void *k, const void *gamma_q,
+                                   const void *gamma_k, const float *rstd_q, const float *rstd_k,
+                                   const void *dq_out, const void *dk_out, void *dq, void *dk,
+                                   float *dgamma_q, float *dgamma_k, int B, int S, int Hq, int Hkv,
+                                   int D, float eps, qknr_dtype dtype, qknr_stream_t stream) {
+    const int64_t qts = (int64_t)Hq * D, kts = (int64_t)Hkv * D;
+    return bwd_impl(q, k, qts, kts, gamma_q, gamma_k, nullptr, rstd_q, rstd_k, dq_out, dk_out, dq,
+                    dk, qts, kts, dgamma_q, dgamma_k, B, S, Hq, Hkv, D, 0, 1.0f, eps, dtype,
+                    stream);
+}
+
+extern "C" qknr_status qk_rope_apply(const void *q, const void *k, const int32_t *pos_ids,
+                                     void *q_out, void *k_out, int B, int S, int Hq, int Hkv,
+                                     int D, int rotary_dim, float theta, int inverse,
+                                     qknr_dtype dtype, qknr_stream_t stream) {
+    const int mode = kModeRopeOnly | (inverse ? kModeInverse : 0);
+    return fwd_impl(q, k, (int64_t)Hq * D, (int64_t)Hkv * D, nullptr, nullptr, pos_ids, q_out,
+                    k_out, nullptr, nullptr, B, S, Hq, Hkv, D, rotary_dim, theta, 0.0f, dtype,
+                    stream, mode);
 }
 
 extern "C" const char *qknr_strerror(qknr_status s) {

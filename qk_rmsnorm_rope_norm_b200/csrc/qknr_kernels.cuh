@@ -47,6 +47,10 @@ constexpr int kMaxHalf = kMaxD / 2;
 #define QKNR_BWD_MIN_CTAS 2
 #endif
 
+// Forward variants (FwdArgs::mode bits).
+constexpr int kModeRopeOnly = 1;  // rotation alone: r = 1, gamma = 1, no rstd written
+constexpr int kModeInverse = 2;   // rotate by -m (the transpose): strips RoPE
+
 struct FwdArgs {
     const void *q, *k, *gq, *gk;
     const int32_t *pos;
@@ -57,6 +61,7 @@ struct FwdArgs {
     int S, Hq, Hkv, D, R;
     float theta, eps;
     int tpw;    // consecutive tokens per warp
+    int mode;   // kModeRopeOnly | kModeInverse bits, 0 for the fused op
 };
 
 struct BwdArgs {
@@ -153,8 +158,8 @@ __device__ __forceinline__ void fill_tables(double *s_omega, float (*s_g)[kMaxD]
     for (int i = threadIdx.x; i < half; i += blockDim.x)
         s_omega[i] = pow((double)theta, -2.0 * (double)i / (double)R);
     for (int i = threadIdx.x; i < D; i += blockDim.x) {
-        s_g[0][i] = gq ? Io<T>::to_f32(gq, i) : 0.f;
-        s_g[1][i] = gk ? Io<T>::to_f32(gk, i) : 0.f;
+        s_g[0][i] = gq ? Io<T>::to_f32(gq, i) : 1.f;  // no gamma: rotation alone
+        s_g[1][i] = gk ? Io<T>::to_f32(gk, i) : 1.f;
     }
 }
 
@@ -265,7 +270,11 @@ qknr_fwd_kernel(const FwdArgs a) {
             }
         };
         load_chunk(0);
-        for (int i = lane; i < half; i += 32) cs[i] = rope_cos_sin(pos, s_omega[i]);
+        for (int i = lane; i < half; i += 32) {
+            float2 v = rope_cos_sin(pos, s_omega[i]);
+            if (a.mode & kModeInverse) v.y = -v.y;
+            cs[i] = v;
+        }
         __syncwarp();
 
         for (int p0 = 0; p0 < npass; p0 += P) {
@@ -280,7 +289,7 @@ qknr_fwd_kernel(const FwdArgs a) {
                     ss = fmaf(vb.x, vb.x, ss); ss = fmaf(vb.y, vb.y, ss);
                 }
                 ss = group_sum<LPR>(ss);
-                const float r = __frsqrt_rn(fmaf(ss, inv_d, a.eps));
+                const float r = (a.mode & kModeRopeOnly) ? 1.f : __frsqrt_rn(fmaf(ss, inv_d, a.eps));
                 const int h = (p0 + pp) * SLOTS + L.slot;
                 if (L.on && h < H) {
                     const bool isq = h < a.Hq;
@@ -303,7 +312,7 @@ qknr_fwd_kernel(const FwdArgs a) {
                     char *out = (char *)(isq ? a.qo : a.ko) + rowi * rowb;
                     st16(out + offA, ya);
                     st16(out + offB, yb);
-                    if (L.u == 0) (isq ? a.rq : a.rk)[rowi] = r;
+                    if (L.u == 0 && !(a.mode & kModeRopeOnly)) (isq ? a.rq : a.rk)[rowi] = r;
                 }
             }
         }

@@ -360,6 +360,8 @@ __device__ __forceinline__ void fill_unit_gamma(float4 (*s_gl)[V / 2][32], const
             const int e = (k < W / 2 ? L.eA + 4 * k : L.eB + 4 * (k - W / 2));
             v = make_float4(Io<T>::to_f32(gp, e), Io<T>::to_f32(gp, e + 1),
                             Io<T>::to_f32(gp, e + 2), Io<T>::to_f32(gp, e + 3));
+        } else if (L.on) {
+            v = make_float4(1.f, 1.f, 1.f, 1.f);  // no gamma: rotation alone
         }
         s_gl[z][k][w ^ (k >= W / 2 ? X : 0)] = v;
     }
@@ -499,10 +501,12 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g, const __grid_constant__ 
         consumers_sync(NCW * 32);
         const Pairs<LPR, V, U> L(lane, a.D, a.R);
         int off1[U], off2[U];
+        float sgn[U];  // sine sign of each pair (negated again for the inverse rotation)
 #pragma unroll
         for (int q = 0; q < U; ++q) {
             off1[q] = L.first[q] * (int)sizeof(T);
             off2[q] = L.second[q] * (int)sizeof(T);
+            sgn[q] = (a.mode & kModeInverse) ? -L.sgn[q] : L.sgn[q];
         }
         const float inv_d = 1.0f / (float)a.D;
         int pc = 0;  // passes dealt before this tile, mod NCW
@@ -535,20 +539,23 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g, const __grid_constant__ 
                 for (int q = 0; q < U; ++q) xa[q] = lds16(src + off1[q]);
 #pragma unroll
                 for (int q = 0; q < U; ++q) xb[q] = lds16(src + off2[q]);
-                float ss = 0.f;
+                float r = 1.f;  // rotation alone: no normalisation
+                if (!(a.mode & kModeRopeOnly)) {
+                    float ss = 0.f;
 #pragma unroll
-                for (int q = 0; q < U; ++q) {
-                    float2 s0 = make_float2(0.f, 0.f), s1 = make_float2(0.f, 0.f);
+                    for (int q = 0; q < U; ++q) {
+                        float2 s0 = make_float2(0.f, 0.f), s1 = make_float2(0.f, 0.f);
 #pragma unroll
-                    for (int k = 0; k < W; ++k) {
-                        const float2 va = IO::get2(xa[q], k), vb = IO::get2(xb[q], k);
-                        s0 = __ffma2_rn(va, va, s0);
-                        s1 = __ffma2_rn(vb, vb, s1);
+                        for (int k = 0; k < W; ++k) {
+                            const float2 va = IO::get2(xa[q], k), vb = IO::get2(xb[q], k);
+                            s0 = __ffma2_rn(va, va, s0);
+                            s1 = __ffma2_rn(vb, vb, s1);
+                        }
+                        ss = fmaf(L.mask[q], (s0.x + s1.x) + (s0.y + s1.y), ss);
                     }
-                    ss = fmaf(L.mask[q], (s0.x + s1.x) + (s0.y + s1.y), ss);
+                    ss = group_sum<LPR>(ss);
+                    r = rsqrtf(fmaf(ss, inv_d, a.eps));
                 }
-                ss = group_sum<LPR>(ss);
-                const float r = rsqrtf(fmaf(ss, inv_d, a.eps));
                 const float2 r2 = make_float2(r, r);
                 const float4 *tok = cs_tile + tr.tl * (half >> 1);
                 char *out = (tr.isq ? out_q : out_k) + tr.jj * rowb;
@@ -558,7 +565,7 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g, const __grid_constant__ 
                     unit_table<V>(tok, L.rot[q], L.w[q], cs);
                     pair_gamma<V, X>(s_gl[tr.isq ? 0 : 1], L.w[q], L.kb[q], gv);
                     // r (and the pair's sine sign) folded into cos and sin
-                    const float rs = r * L.sgn[q];
+                    const float rs = r * sgn[q];
                     const float2 rs2 = make_float2(rs, rs);
                     Vec16 ya, yb;
 #pragma unroll
@@ -578,7 +585,7 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g, const __grid_constant__ 
                         stg16(out + off2[q], yb);
                     }
                 }
-                if (valid && L.u == 0) __stcs((tr.isq ? r_q : r_k) + tr.jj, r);
+                if (valid && L.u == 0 && !(a.mode & kModeRopeOnly)) __stcs((tr.isq ? r_q : r_k) + tr.jj, r);
             }
             pc = (pc + npass) % NCW;
             __syncwarp();

@@ -164,3 +164,32 @@ def test_strided_validation(lib):
     assert bwd_strided(lib, ts, ts, ts, ts, dq=P(1)) == INVALID
     # a strided dq may not alias dq_out
     assert bwd_strided(lib, ts, ts, ts, ts, dq=P(9)) == INVALID
+
+
+def test_nope_and_rope_only_validation(lib):
+    # qk_norm_fwd(q, k, gq, gk, qo, ko, rq, rk, B, S, Hq, Hkv, D, eps, dtype, stream)
+    def norm_fwd(D=64, eps=1e-6, q=P(1), rq=P(7)):
+        return lib.qk_norm_fwd(q, P(2), P(3), P(4), P(5), P(6), rq, P(8), 2, 8, 4, 2, D, eps,
+                               BF16, None)
+
+    assert norm_fwd(D=63) == INVALID
+    assert norm_fwd(eps=-1.0) == INVALID
+    assert norm_fwd(q=None) == INVALID
+    assert norm_fwd(rq=None) == INVALID              # the norm saves rstd
+    assert norm_fwd(q=P(1, 8)) == ALIGN
+    assert lib.qk_norm_bwd(P(1), P(2), P(3), P(4), P(7), P(8), P(9), P(10), P(9, 16), P(12),
+                           P(13), P(14), 2, 8, 4, 2, 64, 1e-6, BF16, None) == INVALID
+
+    # qk_rope_apply(q, k, pos, qo, ko, B, S, Hq, Hkv, D, R, theta, inverse, dtype, stream)
+    def rope(D=64, R=64, theta=1e4, q=P(1), qo=P(5), pos=None):
+        return lib.qk_rope_apply(q, P(2), pos, qo, P(6), 2, 8, 4, 2, D, R, theta, 1, BF16, None)
+
+    assert rope(D=63) == INVALID
+    assert rope(R=66) == INVALID
+    assert rope(theta=0.0) == INVALID
+    assert rope(D=64, R=8) == UNSUP
+    assert rope(q=None) == INVALID
+    assert rope(qo=None) == INVALID
+    assert rope(qo=P(1, 4096)) == INVALID            # partial overlap with q
+    assert rope(q=P(1, 8)) == ALIGN
+    assert rope(pos=P(15, 2)) == ALIGN
