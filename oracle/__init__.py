@@ -71,6 +71,12 @@ class Oracle:
         lib.oracle_bwd_rows.restype = None
         lib.oracle_bwd_rows.argtypes = [_D, _D, _D, _I64, c_i64, c_int, c_int,
                                         c_dbl, c_dbl, _D, _D]
+        lib.oracle_ln_fwd_rows.restype = None
+        lib.oracle_ln_fwd_rows.argtypes = [_D, _D, _I64, c_i64, c_int, c_int,
+                                           c_dbl, c_dbl, _D, _D]
+        lib.oracle_ln_bwd_rows.restype = None
+        lib.oracle_ln_bwd_rows.argtypes = [_D, _D, _D, _I64, c_i64, c_int,
+                                           c_int, c_dbl, c_dbl, _D, _D]
         lib.oracle_rope_rows.restype = None
         lib.oracle_rope_rows.argtypes = [_D, _I64, c_i64, c_int, c_int, c_dbl,
                                          c_int, _D]
@@ -147,6 +153,50 @@ class Oracle:
                                  float(theta), float(eps), _p(dx), _p(dgr))
         return dx, dgr
 
+
+    def ln_fwd_rows(self, x, gamma, m, R: int, theta: float, eps: float):
+        """Mean-centred (QK-LayerNorm) forward of independent rows."""
+        x, g = as_f64(x), as_f64(gamma)
+        n, D = x.shape
+        m = np.ascontiguousarray(np.asarray(m, dtype=np.int64).reshape(n))
+        y = np.empty_like(x)
+        r = np.empty(n)
+        self.lib.oracle_ln_fwd_rows(_p(x), _p(g), _p(m, _I64), n, D, R,
+                                    float(theta), float(eps), _p(y), _p(r))
+        return y, r
+
+    def ln_bwd_rows(self, x, gamma, dy, m, R: int, theta: float, eps: float):
+        """Mean-centred backward of independent rows; (dx, per-row dgamma terms)."""
+        x, g, dy = as_f64(x), as_f64(gamma), as_f64(dy)
+        n, D = x.shape
+        m = np.ascontiguousarray(np.asarray(m, dtype=np.int64).reshape(n))
+        dx = np.empty_like(x)
+        dgr = np.empty_like(x)
+        self.lib.oracle_ln_bwd_rows(_p(x), _p(g), _p(dy), _p(m, _I64), n, D, R,
+                                    float(theta), float(eps), _p(dx), _p(dgr))
+        return dx, dgr
+
+    def ln_fwd(self, q, k, gamma_q, gamma_k, m, R: int, theta: float, eps: float):
+        """Mean-centred forward over tokens, shaped like ``fwd``."""
+        m = np.asarray(m, dtype=np.int64).reshape(-1)
+        out = []
+        for x, g in ((as_f64(q), gamma_q), (as_f64(k), gamma_k)):
+            H, D = x.shape[-2], x.shape[-1]
+            y, r = self.ln_fwd_rows(x.reshape(-1, D), g, np.repeat(m, H), R, theta, eps)
+            out += [y.reshape(x.shape), r.reshape(x.shape[:-1])]
+        return out[0], out[2], out[1], out[3]
+
+    def ln_bwd(self, q, k, gamma_q, gamma_k, m, dq_out, dk_out, R: int, theta: float,
+               eps: float):
+        """Mean-centred backward over tokens, shaped like ``bwd``."""
+        m = np.asarray(m, dtype=np.int64).reshape(-1)
+        out = []
+        for x, g, dy in ((as_f64(q), gamma_q, dq_out), (as_f64(k), gamma_k, dk_out)):
+            H, D = x.shape[-2], x.shape[-1]
+            dx, t = self.ln_bwd_rows(x.reshape(-1, D), g, as_f64(dy).reshape(-1, D),
+                                     np.repeat(m, H), R, theta, eps)
+            out += [dx.reshape(x.shape), t.sum(axis=0)]
+        return out[0], out[2], out[1], out[3]
 
     def rope_rows(self, x, m, R: int, theta: float, inverse: bool = False):
         """Rotation alone of rows x [n, D] at positions m [n]: R(m) x, or

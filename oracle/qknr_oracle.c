@@ -38,6 +38,13 @@
  *   dgamma_d += g_d * x_d * r                        (summed over the tensor's rows)
  *   h_d     = g_d * gamma_d
  *   dx_d    = r * h_d - r^3 * x_d * (1/D) * sum_e h_e x_e
+ * Mean-centred variant (QK-LayerNorm: "Nyonic Technical Report", abstract,
+ * names QK-LayerNorm with rotary embeddings; weight only, no bias):
+ *   mu      = (1/D) * sum_d x_d
+ *   r       = 1 / sqrt((1/D) * sum_d (x_d - mu)^2 + eps)    (saved)
+ *   n_d     = (x_d - mu) * r * gamma_d, then the same rotation
+ *   backward: xh = (x - mu) r, dgamma += g xh, h = g gamma,
+ *   dx_d    = r * (h_d - (1/D) sum_e h_e - xh_d (1/D) sum_e h_e xh_e)
  * Rotation alone (no normalisation), forward or inverse:
  *   y = R(m) x, or y = R(m)^T x = R(-m) x, which strips RoPE from a rotated
  *   row (the cross-model KV cache transfer abstract on the papers listing:
@@ -216,4 +223,97 @@ void oracle_rope_rows(const double *x, const int64_t *m, int64_t n, int D,
             yr[i + half] = xr[i + half] * c + xr[i] * s;
         }
     }
+}
+
+/* Mean of one row. */
+double oracle_mean(const double *x, int D)
+{
+    double s = 0.0;
+    for (int d = 0; d < D; ++d)
+        s += x[d];
+    return s / (double)D;
+}
+
+/* Inverse standard deviation of one row about its mean: 1 / sqrt(var + eps). */
+double oracle_ln_rstd(const double *x, int D, double eps)
+{
+    double mu = oracle_mean(x, D);
+    double var = 0.0;
+    for (int d = 0; d < D; ++d)
+        var += (x[d] - mu) * (x[d] - mu);
+    var /= (double)D;
+    return 1.0 / sqrt(var + eps);
+}
+
+/* Mean-centred forward of rows x [n, D] at positions m [n]. */
+void oracle_ln_fwd_rows(const double *x, const double *gamma, const int64_t *m,
+                        int64_t n, int D, int R, double theta, double eps,
+                        double *y, double *rstd)
+{
+    int half = R / 2;
+    double *nr = (double *)malloc(sizeof(double) * (size_t)D);
+    for (int64_t j = 0; j < n; ++j) {
+        const double *xr = x + j * D;
+        double *yr = y + j * D;
+        double mu = oracle_mean(xr, D);
+        double r = oracle_ln_rstd(xr, D, eps);
+        for (int d = 0; d < D; ++d)
+            nr[d] = (xr[d] - mu) * r * gamma[d];
+        for (int d = 0; d < D; ++d)
+            yr[d] = nr[d];
+        for (int i = 0; i < half; ++i) {
+            double phi = (double)m[j] * oracle_inv_freq(i, R, theta);
+            double c = cos(phi), s = sin(phi);
+            yr[i] = nr[i] * c - nr[i + half] * s;
+            yr[i + half] = nr[i + half] * c + nr[i] * s;
+        }
+        rstd[j] = r;
+    }
+    free(nr);
+}
+
+/*
+ * Mean-centred backward of rows: dx [n, D]; dgamma_rows [n, D] holds each
+ * row's own term g * xh (not summed).
+ */
+void oracle_ln_bwd_rows(const double *x, const double *gamma, const double *dy,
+                        const int64_t *m, int64_t n, int D, int R,
+                        double theta, double eps, double *dx,
+                        double *dgamma_rows)
+{
+    int half = R / 2;
+    double *g = (double *)malloc(sizeof(double) * (size_t)D);
+    double *h = (double *)malloc(sizeof(double) * (size_t)D);
+    double *xh = (double *)malloc(sizeof(double) * (size_t)D);
+    for (int64_t j = 0; j < n; ++j) {
+        const double *xr = x + j * D, *dyr = dy + j * D;
+        double mu = oracle_mean(xr, D);
+        double r = oracle_ln_rstd(xr, D, eps);
+        for (int d = 0; d < D; ++d)
+            g[d] = dyr[d];
+        for (int i = 0; i < half; ++i) {
+            double phi = (double)m[j] * oracle_inv_freq(i, R, theta);
+            double c = cos(phi), s = sin(phi);
+            g[i] = dyr[i] * c + dyr[i + half] * s;
+            g[i + half] = -dyr[i] * s + dyr[i + half] * c;
+        }
+        for (int d = 0; d < D; ++d)
+            xh[d] = (xr[d] - mu) * r;
+        for (int d = 0; d < D; ++d)
+            dgamma_rows[j * D + d] = g[d] * xh[d];
+        for (int d = 0; d < D; ++d)
+            h[d] = g[d] * gamma[d];
+        double mean_h = 0.0, mean_hx = 0.0;
+        for (int e = 0; e < D; ++e) {
+            mean_h += h[e];
+            mean_hx += h[e] * xh[e];
+        }
+        mean_h /= (double)D;
+        mean_hx /= (double)D;
+        for (int d = 0; d < D; ++d)
+            dx[j * D + d] = r * (h[d] - mean_h - xh[d] * mean_hx);
+    }
+    free(g);
+    free(h);
+    free(xh);
 }

@@ -386,4 +386,88 @@ def pin_rope_is_fwd_without_norm(orc):
     _close(orc.rope_rows(x, m, R, 5e5), y / r[:, None], tol=1e-12, what="rope vs fwd / r")
 
 
+# ----------------------------------------------------- mean-centred variant
+def pin_ln_matches_library(orc):
+    """rotary_dim = 0: the mean-centred forward is torch's layer_norm with the
+    weight and no bias (fp64); with a rotary span it is that, rotated as a
+    complex multiplication."""
+    rng = np.random.default_rng(41)
+    for D, R, eps in ((16, 0, 1e-5), (64, 64, 1e-6), (48, 16, 0.3)):
+        x = _rows(rng, 7, D, 2.5) + rng.standard_normal((7, 1)) * 3.0
+        g = _gamma(rng, D)
+        m = rng.integers(0, 50000, 7)
+        y, r = orc.ln_fwd_rows(x, g, m, R, 1e4, eps)
+        xt = torch.as_tensor(x)
+        ln = F.layer_norm(xt, (D,), weight=torch.as_tensor(g), eps=eps).numpy()
+        _close(y, _complex_rope(ln, m, R, 1e4), what=f"layer_norm D={D} R={R}")
+        var = x.var(axis=1)
+        _close(r, 1.0 / np.sqrt(var + eps), tol=1e-13, what="ln rstd")
+
+
+def pin_ln_shift_invariance(orc):
+    """Adding a constant to every element of a row leaves the mean-centred
+    output unchanged."""
+    rng = np.random.default_rng(42)
+    D, R = 32, 32
+    x = _rows(rng, 5, D)
+    g = _gamma(rng, D)
+    m = rng.integers(0, 1000, 5)
+    y0, _ = orc.ln_fwd_rows(x, g, m, R, 1e4, 1e-6)
+    y1, _ = orc.ln_fwd_rows(x + 7.25, g, m, R, 1e4, 1e-6)
+    _close(y1, y0, tol=1e-11, what="shift invariance")
+
+
+def pin_ln_bwd_finite_differences(orc):
+    """Central differences of sum(y * dy) for every element of dx and dgamma."""
+    rng = np.random.default_rng(43)
+    n, D, R, eps = 3, 8, 4, 1e-3
+    x = _rows(rng, n, D, 1.5) + 0.7
+    g = _gamma(rng, D)
+    dy = _rows(rng, n, D)
+    m = rng.integers(0, 100, n)
+    dx, dgr = orc.ln_bwd_rows(x, g, dy, m, R, 1e4, eps)
+
+    def loss(xx, gg):
+        y, _ = orc.ln_fwd_rows(xx, gg, m, R, 1e4, eps)
+        return float(np.sum(y * dy))
+
+    h = 1e-6
+    num = np.zeros_like(x)
+    for idx in np.ndindex(*x.shape):
+        xp, xm = x.copy(), x.copy()
+        xp[idx] += h
+        xm[idx] -= h
+        num[idx] = (loss(xp, g) - loss(xm, g)) / (2 * h)
+    _close(dx, num, tol=1e-7, what="ln dx finite differences")
+    numg = np.zeros(D)
+    for d in range(D):
+        gp, gm = g.copy(), g.copy()
+        gp[d] += h
+        gm[d] -= h
+        numg[d] = (loss(x, gp) - loss(x, gm)) / (2 * h)
+    _close(dgr.sum(axis=0), numg, tol=1e-7, what="ln dgamma finite differences")
+
+
+def pin_ln_bwd_matches_autograd(orc):
+    """torch autograd through layer_norm and a complex-multiplication rotation."""
+    rng = np.random.default_rng(44)
+    n, D, R, eps = 6, 32, 16, 1e-5
+    x = _rows(rng, n, D, 2.0) - 1.0
+    g = _gamma(rng, D)
+    dy = _rows(rng, n, D)
+    m = rng.integers(0, 9000, n)
+    xt = torch.tensor(x, requires_grad=True)
+    gt = torch.tensor(g, requires_grad=True)
+    ln = F.layer_norm(xt, (D,), weight=gt, eps=eps)
+    half = R // 2
+    ang = torch.tensor(m, dtype=torch.float64)[:, None] * torch.pow(
+        torch.tensor(1e4, dtype=torch.float64), -2.0 * torch.arange(half, dtype=torch.float64) / R)
+    z = torch.complex(ln[:, :half], ln[:, half:R]) * torch.polar(torch.ones_like(ang), ang)
+    y = torch.cat([z.real, z.imag, ln[:, R:]], dim=1)
+    (y * torch.tensor(dy)).sum().backward()
+    dx, dgr = orc.ln_bwd_rows(x, g, dy, m, R, 1e4, eps)
+    _close(dx, xt.grad.numpy(), tol=1e-12, what="ln dx vs autograd")
+    _close(dgr.sum(axis=0), gt.grad.numpy(), tol=1e-12, what="ln dgamma vs autograd")
+
+
 ALL_PINS = [v for k_, v in sorted(globals().items()) if k_.startswith("pin_")]

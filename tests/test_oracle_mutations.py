@@ -62,6 +62,18 @@ MUTATIONS = [
                             "oracle_fwd_row(q + row * D, gamma_q, D, R, theta, eps, (int64_t)t,", 0)]),
     ("bwd_k_dgamma_into_q", [("theta, eps, m[t], dk + row * D, dgamma_k);",
                               "theta, eps, m[t], dk + row * D, dgamma_q);", 0)]),
+    ("ln_mean_not_subtracted", [("            nr[d] = (xr[d] - mu) * r * gamma[d];",
+                                 "            nr[d] = xr[d] * r * gamma[d];", 0)]),
+    ("ln_variance_not_centred", [("        var += (x[d] - mu) * (x[d] - mu);",
+                                  "        var += x[d] * x[d];", 0)]),
+    ("ln_mean_over_D_minus_1", [("    return s / (double)D;", "    return s / (double)(D - 1);", 0)]),
+    ("ln_bwd_mean_h_dropped", [("r * (h[d] - mean_h - xh[d] * mean_hx);",
+                                "r * (h[d] - xh[d] * mean_hx);", 0)]),
+    ("ln_bwd_projection_dropped", [("r * (h[d] - mean_h - xh[d] * mean_hx);",
+                                    "r * (h[d] - mean_h);", 0)]),
+    ("ln_bwd_xh_not_centred", [("            xh[d] = (xr[d] - mu) * r;", "            xh[d] = xr[d] * r;", 0)]),
+    ("ln_bwd_unrotate_sign", [("            g[i + half] = -dyr[i] * s + dyr[i + half] * c;",
+                               "            g[i + half] = dyr[i] * s + dyr[i + half] * c;", 0)]),
     ("rope_inverse_ignored", [("            s = -s;", "            s = s;", 0)]),
     ("rope_sin_sign_first", [("yr[i] = xr[i] * c - xr[i + half] * s;",
                               "yr[i] = xr[i] * c + xr[i + half] * s;", 0)]),
