@@ -281,8 +281,9 @@ def run_variants(args, w, inp, dev, peak):
     """The other entry points on the same workload, each timed like the main
     step (a ring of input sets, CUDA events around every launch, mean over
     the launches): the fused op on Q / K slices of a fused QKV buffer, the
-    NoPE op (qk_norm_*), and the rotation alone, forward and inverse
-    (qk_rope_apply). Bytes are each call's contract bytes."""
+    NoPE op (qk_norm_*), the mean-centred form (qk_layernorm_rope_*), the
+    statistic alone (qk_rms_stats) and the rotation alone, forward and
+    inverse (qk_rope_apply). Bytes are each call's contract bytes."""
     import qk_rmsnorm_rope_norm_b200 as qknr
     lib = qknr.load_library()
     cfg = dict(rotary_dim=w.rotary_dim, theta=w.theta, eps=w.eps)
@@ -343,7 +344,20 @@ def run_variants(args, w, inp, dev, peak):
     out["nope_qk_norm"] = {"fwd": line(timed([nope_fwd(s) for s in dense]), cb_nope["fwd"]),
                            "bwd": line(timed([nope_bwd(s) for s in dense]), cb_nope["bwd"]),
                            "entry": "qk_norm_fwd / qk_norm_bwd"}
+    ln = dict(cfg, norm="layer")
+    f = [qknr.prepare_fwd(s.q, s.k, s.gq, s.gk, s.pos, s.qo, s.ko, s.rq, s.rk, **ln) for s in dense]
+    b = [qknr.prepare_bwd(s.q, s.k, s.gq, s.gk, s.pos, s.rq, s.rk, s.dqo, s.dko, s.dq, s.dk,
+                          s.dgq, s.dgk, **ln) for s in dense]
+    out["qk_layernorm_rope"] = {"fwd": line(timed(f), cb["fwd"]), "bwd": line(timed(b), cb["bwd"]),
+                                "entry": "qk_layernorm_rope_fwd / qk_layernorm_rope_bwd"}
     rope_bytes = 2 * rows * w.D * e + pos_b
+    def stats(s):
+        a = (P(s.q), P(s.k), P(s.rq), P(s.rk), w.B, w.S, w.Hq, w.Hkv, w.D, float(w.eps), dt, st)
+        return qknr.PreparedCall(lib.qk_rms_stats, a, "qk_rms_stats", s)
+
+    out["rms_stats"] = {"fwd": line(timed([stats(s) for s in dense]),
+                                    rows * w.D * e + 4 * rows),
+                        "entry": "qk_rms_stats"}
     out["rope_only"] = {"fwd": line(timed([rope(s, False) for s in dense]), rope_bytes),
                         "inverse": line(timed([rope(s, True) for s in dense]), rope_bytes),
                         "entry": "qk_rope_apply"}

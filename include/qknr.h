@@ -187,6 +187,39 @@ QKNR_API qknr_status qk_norm_rope_bwd_strided(const void *q, const void *k,
                              qknr_dtype dtype, qknr_stream_t stream);
 
 /*
+ * Mean-centred form (QK-LayerNorm, "Nyonic Technical Report", abstract:
+ * rotary embeddings with QK-LayerNorm): per (token, head) row
+ *   mu = mean_d x_d,  r = 1 / sqrt(mean_d (x_d - mu)^2 + eps)  (saved fp32)
+ *   n_d = (x_d - mu) * r * gamma_d,  then the same rotate-half RoPE,
+ * with the learned weight and no bias (the page names no bias). Backward,
+ * with g the inverse rotation of dy and xh = (x - mu) r:
+ *   dgamma_d += g_d xh_d;  h = g * gamma;
+ *   dx = r * (h - mean(h) - xh * mean(h * xh)).
+ * The mean is recomputed from x in the backward, so rstd is still the one
+ * saved statistic. Arguments, layouts, aliasing and errors exactly as for
+ * qk_norm_rope_fwd / qk_norm_rope_bwd.
+ */
+QKNR_API qknr_status qk_layernorm_rope_fwd(const void *q, const void *k,
+                             const void *gamma_q, const void *gamma_k,
+                             const int32_t *pos_ids,
+                             void *q_out, void *k_out,
+                             float *rstd_q, float *rstd_k,
+                             int B, int S, int Hq, int Hkv, int D,
+                             int rotary_dim, float theta, float eps,
+                             qknr_dtype dtype, qknr_stream_t stream);
+
+QKNR_API qknr_status qk_layernorm_rope_bwd(const void *q, const void *k,
+                             const void *gamma_q, const void *gamma_k,
+                             const int32_t *pos_ids,
+                             const float *rstd_q, const float *rstd_k,
+                             const void *dq_out, const void *dk_out,
+                             void *dq, void *dk,
+                             float *dgamma_q, float *dgamma_k,
+                             int B, int S, int Hq, int Hkv, int D,
+                             int rotary_dim, float theta, float eps,
+                             qknr_dtype dtype, qknr_stream_t stream);
+
+/*
  * Per-head QK-RMSNorm alone, for the layers that use no positional
  * embedding ("Rope to Nope and Back Again: A New Hybrid Attention Strategy",
  * abstract: NoPE and QK-Norm layers; "Fractional Rotation, Full Potential?",
@@ -207,6 +240,24 @@ QKNR_API qknr_status qk_norm_bwd(const void *q, const void *k,
                              const void *dq_out, const void *dk_out,
                              void *dq, void *dk,
                              float *dgamma_q, float *dgamma_k,
+                             int B, int S, int Hq, int Hkv, int D, float eps,
+                             qknr_dtype dtype, qknr_stream_t stream);
+
+/*
+ * The inverse-RMS statistic alone: rstd = 1 / sqrt(mean_d x_d^2 + eps) for
+ * every (token, head) row of q and of k, fp32 [B,S,Hq] / [B,S,Hkv], with no
+ * normalised rows written. This is the dynamic half of a split RMSNorm:
+ * "QK-Normed MLA: QK normalization without full key caching", abstract,
+ * absorbs the static key-side weight into the query projection and keeps
+ * one inverse-RMS scalar per token and KV group, computed here from the
+ * projected rows (one read of the rows, 4 bytes written per row). Equal bit
+ * for bit to the rstd that qk_norm_fwd saves (and qk_norm_rope_fwd when
+ * rotary_dim is 0 or D; with a partial span its fp32 sum is taken in another
+ * order, within the same D * 2^-24 bound). Either tensor may have zero
+ * heads; layouts, alignment and errors as for qk_norm_rope_fwd.
+ */
+QKNR_API qknr_status qk_rms_stats(const void *q, const void *k,
+                             float *rstd_q, float *rstd_k,
                              int B, int S, int Hq, int Hkv, int D, float eps,
                              qknr_dtype dtype, qknr_stream_t stream);
 

@@ -23,7 +23,7 @@ import torch
 
 __all__ = ["qk_norm_rope_fwd", "qk_norm_rope_bwd", "qknr_strerror", "QKNormRoPE",
            "QKNormRoPEFromQKV", "qk_norm_rope_qkv", "split_qkv",
-           "qk_norm_fwd", "qk_norm_bwd", "qk_rope_apply", "QKRoPE",
+           "qk_norm_fwd", "qk_norm_bwd", "qk_rope_apply", "QKRoPE", "qk_rms_stats",
            "prepare_fwd", "prepare_bwd", "PreparedCall",
            "qk_norm_rope", "QKNRError", "library_path", "load_library", "pipeline_error"]
 
@@ -67,10 +67,15 @@ def load_library():
     lib.qk_norm_rope_fwd_strided.restype = i32
     lib.qk_norm_rope_fwd_strided.argtypes = [vp, vp, i64, i64] + [vp] * 7 + [i32] * 6 + \
         [f32, f32, i32, vp]
+    for n in ("qk_layernorm_rope_fwd", "qk_layernorm_rope_bwd"):
+        fn, ref = getattr(lib, n), getattr(lib, n.replace("layernorm", "norm"))
+        fn.restype, fn.argtypes = ref.restype, ref.argtypes
     lib.qk_norm_fwd.restype = i32
     lib.qk_norm_fwd.argtypes = [vp] * 8 + [i32] * 5 + [f32, i32, vp]
     lib.qk_norm_bwd.restype = i32
     lib.qk_norm_bwd.argtypes = [vp] * 12 + [i32] * 5 + [f32, i32, vp]
+    lib.qk_rms_stats.restype = i32
+    lib.qk_rms_stats.argtypes = [vp] * 4 + [i32] * 5 + [f32, i32, vp]
     lib.qk_rope_apply.restype = i32
     lib.qk_rope_apply.argtypes = [vp] * 5 + [i32] * 6 + [f32, i32, i32, vp]
     lib.qk_norm_rope_bwd_strided.restype = i32
@@ -145,12 +150,13 @@ def _shape(q: torch.Tensor, k: torch.Tensor):
 
 def qk_norm_rope_fwd(q, k, gamma_q, gamma_k, pos_ids=None, *, rotary_dim: int,
                      theta: float, eps: float, q_out=None, k_out=None,
-                     rstd_q=None, rstd_k=None, stream=None):
+                     rstd_q=None, rstd_k=None, stream=None, norm: str = "rms"):
     """Forward. Returns ``(q_out, k_out, rstd_q, rstd_k)``.
 
     q [B,S,Hq,D], k [B,S,Hkv,D] (fp32 or bf16, contiguous, CUDA); gamma_q,
     gamma_k [D] same dtype; pos_ids optional int32 [B,S]. Outputs not given
-    are allocated; ``q_out=q`` / ``k_out=k`` runs in place.
+    are allocated; ``q_out=q`` / ``k_out=k`` runs in place. ``norm="layer"``
+    selects the mean-centred form (C ``qk_layernorm_rope_fwd``; dense q, k).
     """
     lib = load_library()
     qts, kts = _token_stride("q", q), _token_stride("k", k)
@@ -179,7 +185,7 @@ def qk_norm_rope_fwd(q, k, gamma_q, gamma_k, pos_ids=None, *, rotary_dim: int,
             tuple(rstd_q.shape) != (B, S, Hq) or tuple(rstd_k.shape) != (B, S, Hkv):
         raise ValueError("rstd_q / rstd_k must be float32 [B,S,Hq] / [B,S,Hkv]")
     fn, name, args = _fwd_args(lib, q, k, qts, kts, gamma_q, gamma_k, pos_ids, q_out, k_out,
-                               rstd_q, rstd_k, rotary_dim, theta, eps, stream)
+                               rstd_q, rstd_k, rotary_dim, theta, eps, stream, norm)
     st = fn(*args)
     if st != QKNR_OK:
         raise QKNRError(st, name)
@@ -187,13 +193,19 @@ def qk_norm_rope_fwd(q, k, gamma_q, gamma_k, pos_ids=None, *, rotary_dim: int,
 
 
 def _fwd_args(lib, q, k, qts, kts, gamma_q, gamma_k, pos_ids, q_out, k_out, rstd_q, rstd_k,
-              rotary_dim, theta, eps, stream):
+              rotary_dim, theta, eps, stream, norm="rms"):
     """(C function, its name, argument tuple): the dense entry point when q and
     k are dense, else the strided one."""
     B, S, Hq, Hkv, D = _shape(q, k)
     tail = (_ptr(gamma_q), _ptr(gamma_k), _ptr(pos_ids), _ptr(q_out), _ptr(k_out),
             _ptr(rstd_q), _ptr(rstd_k), B, S, Hq, Hkv, D, int(rotary_dim), float(theta),
             float(eps), _DTYPES[q.dtype], _stream(stream))
+    if norm not in ("rms", "layer"):
+        raise ValueError("norm must be 'rms' or 'layer'")
+    if norm == "layer":
+        if qts != Hq * D or kts != Hkv * D:
+            raise ValueError("the mean-centred form takes dense q and k")
+        return lib.qk_layernorm_rope_fwd, "qk_layernorm_rope_fwd", (_ptr(q), _ptr(k)) + tail
     if qts == Hq * D and kts == Hkv * D:
         return lib.qk_norm_rope_fwd, "qk_norm_rope_fwd", (_ptr(q), _ptr(k)) + tail
     return lib.qk_norm_rope_fwd_strided, "qk_norm_rope_fwd_strided", \
@@ -202,7 +214,8 @@ def _fwd_args(lib, q, k, qts, kts, gamma_q, gamma_k, pos_ids, q_out, k_out, rstd
 
 def qk_norm_rope_bwd(q, k, gamma_q, gamma_k, pos_ids, rstd_q, rstd_k, dq_out, dk_out, *,
                      rotary_dim: int, theta: float, eps: float, dq=None, dk=None,
-                     dgamma_q=None, dgamma_k=None, need_dgamma: bool = True, stream=None):
+                     dgamma_q=None, dgamma_k=None, need_dgamma: bool = True, stream=None,
+                     norm: str = "rms"):
     """Backward. Returns ``(dq, dk, dgamma_q, dgamma_k)`` (dgamma fp32 [D]).
 
     ``dq=dq_out`` / ``dk=dk_out`` runs in place. With ``need_dgamma=False``
@@ -242,7 +255,7 @@ def qk_norm_rope_bwd(q, k, gamma_q, gamma_k, pos_ids, rstd_q, rstd_k, dq_out, dk
                 raise ValueError(f"{n} must be float32 [D]")
     fn, name, args = _bwd_args(lib, q, k, qts, kts, gamma_q, gamma_k, pos_ids, rstd_q, rstd_k,
                                dq_out, dk_out, dq, dk, dqts, dkts, dgamma_q, dgamma_k,
-                               rotary_dim, theta, eps, stream)
+                               rotary_dim, theta, eps, stream, norm)
     st = fn(*args)
     if st != QKNR_OK:
         raise QKNRError(st, name)
@@ -250,12 +263,18 @@ def qk_norm_rope_bwd(q, k, gamma_q, gamma_k, pos_ids, rstd_q, rstd_k, dq_out, dk
 
 
 def _bwd_args(lib, q, k, qts, kts, gamma_q, gamma_k, pos_ids, rstd_q, rstd_k, dq_out, dk_out,
-              dq, dk, dqts, dkts, dgamma_q, dgamma_k, rotary_dim, theta, eps, stream):
+              dq, dk, dqts, dkts, dgamma_q, dgamma_k, rotary_dim, theta, eps, stream, norm="rms"):
     B, S, Hq, Hkv, D = _shape(q, k)
     tail = (B, S, Hq, Hkv, D, int(rotary_dim), float(theta), float(eps), _DTYPES[q.dtype],
             _stream(stream))
-    if qts == Hq * D and kts == Hkv * D and dqts == Hq * D and dkts == Hkv * D:
-        return lib.qk_norm_rope_bwd, "qk_norm_rope_bwd", (
+    dense = qts == Hq * D and kts == Hkv * D and dqts == Hq * D and dkts == Hkv * D
+    if norm not in ("rms", "layer"):
+        raise ValueError("norm must be 'rms' or 'layer'")
+    if norm == "layer" and not dense:
+        raise ValueError("the mean-centred form takes dense q, k, dq and dk")
+    if dense:
+        fn = lib.qk_layernorm_rope_bwd if norm == "layer" else lib.qk_norm_rope_bwd
+        return fn, fn.__name__, (
             _ptr(q), _ptr(k), _ptr(gamma_q), _ptr(gamma_k), _ptr(pos_ids), _ptr(rstd_q),
             _ptr(rstd_k), _ptr(dq_out), _ptr(dk_out), _ptr(dq), _ptr(dk), _ptr(dgamma_q),
             _ptr(dgamma_k)) + tail
@@ -270,32 +289,34 @@ class QKNormRoPE(torch.autograd.Function):
     ``qk_norm_rope_bwd``. gamma gradients are returned in gamma's dtype."""
 
     @staticmethod
-    def forward(ctx, q, k, gamma_q, gamma_k, pos_ids, rotary_dim, theta, eps):
+    def forward(ctx, q, k, gamma_q, gamma_k, pos_ids, rotary_dim, theta, eps, norm="rms"):
         q_out, k_out, rq, rk = qk_norm_rope_fwd(q, k, gamma_q, gamma_k, pos_ids,
-                                                rotary_dim=rotary_dim, theta=theta, eps=eps)
+                                                rotary_dim=rotary_dim, theta=theta, eps=eps,
+                                                norm=norm)
         ctx.save_for_backward(q, k, gamma_q, gamma_k, rq, rk)
         ctx.pos_ids = pos_ids
-        ctx.cfg = (rotary_dim, theta, eps)
+        ctx.cfg = (rotary_dim, theta, eps, norm)
         ctx.mark_non_differentiable(rq, rk)
         return q_out, k_out
 
     @staticmethod
     def backward(ctx, dq_out, dk_out):
         q, k, gq, gk, rq, rk = ctx.saved_tensors
-        R, theta, eps = ctx.cfg
+        R, theta, eps, norm = ctx.cfg
         dq, dk, dgq, dgk = qk_norm_rope_bwd(
             q, k, gq, gk, ctx.pos_ids, rq, rk, dq_out.contiguous(), dk_out.contiguous(),
             rotary_dim=R, theta=theta, eps=eps,
-            need_dgamma=ctx.needs_input_grad[2] or ctx.needs_input_grad[3])
+            need_dgamma=ctx.needs_input_grad[2] or ctx.needs_input_grad[3], norm=norm)
         dgq = None if dgq is None else dgq.to(gq.dtype)
         dgk = None if dgk is None else dgk.to(gk.dtype)
-        return dq, dk, dgq, dgk, None, None, None, None
+        return dq, dk, dgq, dgk, None, None, None, None, None
 
 
 def qk_norm_rope(q, k, gamma_q, gamma_k, pos_ids=None, *, rotary_dim: int, theta: float,
-                 eps: float):
-    """Differentiable fused op; returns ``(q_out, k_out)``."""
-    return QKNormRoPE.apply(q, k, gamma_q, gamma_k, pos_ids, rotary_dim, theta, eps)
+                 eps: float, norm: str = "rms"):
+    """Differentiable fused op; returns ``(q_out, k_out)``. ``norm="layer"``
+    is the mean-centred (QK-LayerNorm) form."""
+    return QKNormRoPE.apply(q, k, gamma_q, gamma_k, pos_ids, rotary_dim, theta, eps, norm)
 
 
 def qk_norm_fwd(q, k, gamma_q, gamma_k, *, eps: float, q_out=None, k_out=None,
@@ -373,6 +394,28 @@ def qk_rope_apply(q, k, pos_ids=None, *, rotary_dim: int, theta: float, inverse:
     if st != QKNR_OK:
         raise QKNRError(st, "qk_rope_apply")
     return q_out, k_out
+
+
+def qk_rms_stats(q, k, *, eps: float, rstd_q=None, rstd_k=None, stream=None):
+    """Inverse-RMS statistic alone (C ``qk_rms_stats``): fp32 ``(rstd_q,
+    rstd_k)`` [B,S,Hq] / [B,S,Hkv], no normalised rows written."""
+    lib = load_library()
+    for n, t in (("q", q), ("k", k)):
+        _need_cuda(n, t)
+    B, S, Hq, Hkv, D = _shape(q, k)
+    _same_dtype(q, k)
+    rstd_q = torch.empty((B, S, Hq), dtype=torch.float32, device=q.device) if rstd_q is None else rstd_q
+    rstd_k = torch.empty((B, S, Hkv), dtype=torch.float32, device=q.device) if rstd_k is None else rstd_k
+    for n, t in (("rstd_q", rstd_q), ("rstd_k", rstd_k)):
+        _need_cuda(n, t)
+    if rstd_q.dtype != torch.float32 or rstd_k.dtype != torch.float32 or \
+            tuple(rstd_q.shape) != (B, S, Hq) or tuple(rstd_k.shape) != (B, S, Hkv):
+        raise ValueError("rstd_q / rstd_k must be float32 [B,S,Hq] / [B,S,Hkv]")
+    st = lib.qk_rms_stats(_ptr(q), _ptr(k), _ptr(rstd_q), _ptr(rstd_k), B, S, Hq, Hkv, D,
+                          float(eps), _DTYPES[q.dtype], _stream(stream))
+    if st != QKNR_OK:
+        raise QKNRError(st, "qk_rms_stats")
+    return rstd_q, rstd_k
 
 
 class QKRoPE(torch.autograd.Function):
@@ -485,29 +528,30 @@ class PreparedCall:
 
 
 def prepare_fwd(q, k, gamma_q, gamma_k, pos_ids, q_out, k_out, rstd_q, rstd_k, *,
-                rotary_dim, theta, eps, stream=None) -> PreparedCall:
+                rotary_dim, theta, eps, stream=None, norm="rms") -> PreparedCall:
     lib = load_library()
     # one checked call validates the tensors (and runs the op once)
     qk_norm_rope_fwd(q, k, gamma_q, gamma_k, pos_ids, rotary_dim=rotary_dim, theta=theta,
                      eps=eps, q_out=q_out, k_out=k_out, rstd_q=rstd_q, rstd_k=rstd_k,
-                     stream=stream)
+                     stream=stream, norm=norm)
     fn, name, args = _fwd_args(lib, q, k, _token_stride("q", q), _token_stride("k", k), gamma_q,
                                gamma_k, pos_ids, q_out, k_out, rstd_q, rstd_k, rotary_dim,
-                               theta, eps, stream)
+                               theta, eps, stream, norm)
     keep = (q, k, gamma_q, gamma_k, pos_ids, q_out, k_out, rstd_q, rstd_k)
     return PreparedCall(fn, args, name, keep)
 
 
 def prepare_bwd(q, k, gamma_q, gamma_k, pos_ids, rstd_q, rstd_k, dq_out, dk_out, dq, dk,
-                dgamma_q, dgamma_k, *, rotary_dim, theta, eps, stream=None) -> PreparedCall:
+                dgamma_q, dgamma_k, *, rotary_dim, theta, eps, stream=None,
+                norm="rms") -> PreparedCall:
     lib = load_library()
     qk_norm_rope_bwd(q, k, gamma_q, gamma_k, pos_ids, rstd_q, rstd_k, dq_out, dk_out,
                      rotary_dim=rotary_dim, theta=theta, eps=eps, dq=dq, dk=dk,
-                     dgamma_q=dgamma_q, dgamma_k=dgamma_k, stream=stream)
+                     dgamma_q=dgamma_q, dgamma_k=dgamma_k, stream=stream, norm=norm)
     fn, name, args = _bwd_args(lib, q, k, _token_stride("q", q), _token_stride("k", k), gamma_q,
                                gamma_k, pos_ids, rstd_q, rstd_k, dq_out, dk_out, dq, dk,
                                _token_stride("dq", dq), _token_stride("dk", dk), dgamma_q,
-                               dgamma_k, rotary_dim, theta, eps, stream)
+                               dgamma_k, rotary_dim, theta, eps, stream, norm)
     keep = (q, k, gamma_q, gamma_k, pos_ids, rstd_q, rstd_k, dq_out, dk_out, dq, dk,
             dgamma_q, dgamma_k)
     return PreparedCall(fn, args, name, keep)

@@ -296,12 +296,12 @@ int input_maps(const void *q, const void *k, int64_t qts, int64_t kts, int Hq, i
     return mask;
 }
 
-template <typename T, int LPR, int U>
+template <typename T, int LPR, int U, bool LN>
 qknr_status launch_fwd_pipe(const FwdArgs &a, const PipeGeom &g, const CUtensorMap &mq,
                             const CUtensorMap &mk, int grid, int smem, int dev, cudaStream_t st,
                             bool *launched) {
     static std::atomic<int> smem_ok[64];
-    auto kern = qknr_fwd_pipe_kernel<T, LPR, U, kFwdPipeWarps, kProducerWarps>;
+    auto kern = qknr_fwd_pipe_kernel<T, LPR, U, kFwdPipeWarps, kProducerWarps, LN>;
     *launched = false;
     if (!allow_dyn_smem((const void *)kern, dev, smem_ok, smem)) return QKNR_OK;
     *launched = true;
@@ -310,12 +310,12 @@ qknr_status launch_fwd_pipe(const FwdArgs &a, const PipeGeom &g, const CUtensorM
     return e == cudaSuccess ? QKNR_OK : cuda_fail(e);
 }
 
-template <typename T, int LPR>
+template <typename T, int LPR, bool LN>
 qknr_status launch_bwd_pipe(const BwdArgs &a, const PipeGeom &g, const CUtensorMap &mq,
                             const CUtensorMap &mk, int grid, int smem, int dev, cudaStream_t st,
                             bool *launched) {
     static std::atomic<int> smem_ok[64];
-    auto kern = qknr_bwd_pipe_kernel<T, LPR, kBwdPipeWarps, kProducerWarps>;
+    auto kern = qknr_bwd_pipe_kernel<T, LPR, kBwdPipeWarps, kProducerWarps, LN>;
     *launched = false;
     if (!allow_dyn_smem((const void *)kern, dev, smem_ok, smem)) return QKNR_OK;
     *launched = true;
@@ -332,7 +332,7 @@ int next_pow2(int x) {
 
 // Pipelined forward when it applies: two units per lane once a row has
 // three or more (halving the per-row overhead per element).
-template <typename T>
+template <typename T, bool LN>
 bool try_fwd_pipe(const FwdArgs &a, cudaStream_t st, qknr_status *status) {
     int dev = 0;
     cudaGetDevice(&dev);
@@ -350,22 +350,22 @@ bool try_fwd_pipe(const FwdArgs &a, cudaStream_t st, qknr_status *status) {
     qknr_status s = QKNR_OK;
     if (dv2 >= 3) {
         switch (next_pow2((dv2 + 1) / 2)) {
-            case 2: s = launch_fwd_pipe<T, 2, 2>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
-            case 4: s = launch_fwd_pipe<T, 4, 2>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
-            case 8: s = launch_fwd_pipe<T, 8, 2>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
-            case 16: s = launch_fwd_pipe<T, 16, 2>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
+            case 2: s = launch_fwd_pipe<T, 2, 2, LN>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
+            case 4: s = launch_fwd_pipe<T, 4, 2, LN>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
+            case 8: s = launch_fwd_pipe<T, 8, 2, LN>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
+            case 16: s = launch_fwd_pipe<T, 16, 2, LN>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
         }
     } else {
         switch (next_pow2(dv2)) {
-            case 1: s = launch_fwd_pipe<T, 1, 1>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
-            case 2: s = launch_fwd_pipe<T, 2, 1>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
+            case 1: s = launch_fwd_pipe<T, 1, 1, LN>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
+            case 2: s = launch_fwd_pipe<T, 2, 1, LN>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
         }
     }
     *status = s;
     return launched;
 }
 
-template <typename T>
+template <typename T, bool LN>
 bool try_bwd_pipe(const BwdArgs &a, cudaStream_t st, qknr_status *status) {
     int dev = 0;
     cudaGetDevice(&dev);
@@ -382,21 +382,21 @@ bool try_bwd_pipe(const BwdArgs &a, cudaStream_t st, qknr_status *status) {
     bool launched = false;
     qknr_status s = QKNR_OK;
     switch (next_pow2(dv2)) {
-        case 1: s = launch_bwd_pipe<T, 1>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
-        case 2: s = launch_bwd_pipe<T, 2>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
-        case 4: s = launch_bwd_pipe<T, 4>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
-        case 8: s = launch_bwd_pipe<T, 8>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
-        case 16: s = launch_bwd_pipe<T, 16>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
-        case 32: s = launch_bwd_pipe<T, 32>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
+        case 1: s = launch_bwd_pipe<T, 1, LN>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
+        case 2: s = launch_bwd_pipe<T, 2, LN>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
+        case 4: s = launch_bwd_pipe<T, 4, LN>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
+        case 8: s = launch_bwd_pipe<T, 8, LN>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
+        case 16: s = launch_bwd_pipe<T, 16, LN>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
+        case 32: s = launch_bwd_pipe<T, 32, LN>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
     }
     *status = s;
     return launched;
 }
 
-template <typename T, int LPR>
+template <typename T, int LPR, bool LN>
 qknr_status launch_fwd(FwdArgs a, cudaStream_t st) {
     static std::atomic<int> occ[64];
-    auto kern = qknr_fwd_kernel<T, LPR>;
+    auto kern = qknr_fwd_kernel<T, LPR, LN>;
     int grid, tpw;
     geometry((const void *)kern, occ, a.T, &grid, &tpw);
     a.tpw = tpw;
@@ -405,10 +405,10 @@ qknr_status launch_fwd(FwdArgs a, cudaStream_t st) {
     return e == cudaSuccess ? QKNR_OK : cuda_fail(e);
 }
 
-template <typename T, int LPR>
+template <typename T, int LPR, bool LN>
 qknr_status launch_bwd(BwdArgs a, cudaStream_t st) {
     static std::atomic<int> occ[64];
-    auto kern = qknr_bwd_kernel<T, LPR>;
+    auto kern = qknr_bwd_kernel<T, LPR, LN>;
     int grid, tpw;
     geometry((const void *)kern, occ, a.T, &grid, &tpw);
     a.tpw = tpw;
@@ -417,32 +417,32 @@ qknr_status launch_bwd(BwdArgs a, cudaStream_t st) {
     return e == cudaSuccess ? QKNR_OK : cuda_fail(e);
 }
 
-template <typename T>
+template <typename T, bool LN>
 qknr_status dispatch_fwd(const FwdArgs &a, int lpr, cudaStream_t st) {
     qknr_status ps;
-    if (try_fwd_pipe<T>(a, st, &ps)) return ps;
+    if (try_fwd_pipe<T, LN>(a, st, &ps)) return ps;
     switch (lpr) {
-        case 1: return launch_fwd<T, 1>(a, st);
-        case 2: return launch_fwd<T, 2>(a, st);
-        case 4: return launch_fwd<T, 4>(a, st);
-        case 8: return launch_fwd<T, 8>(a, st);
-        case 16: return launch_fwd<T, 16>(a, st);
-        case 32: return launch_fwd<T, 32>(a, st);
+        case 1: return launch_fwd<T, 1, LN>(a, st);
+        case 2: return launch_fwd<T, 2, LN>(a, st);
+        case 4: return launch_fwd<T, 4, LN>(a, st);
+        case 8: return launch_fwd<T, 8, LN>(a, st);
+        case 16: return launch_fwd<T, 16, LN>(a, st);
+        case 32: return launch_fwd<T, 32, LN>(a, st);
     }
     return QKNR_ERR_UNSUPPORTED;
 }
 
-template <typename T>
+template <typename T, bool LN>
 qknr_status dispatch_bwd(const BwdArgs &a, int lpr, cudaStream_t st) {
     qknr_status ps;
-    if (try_bwd_pipe<T>(a, st, &ps)) return ps;
+    if (try_bwd_pipe<T, LN>(a, st, &ps)) return ps;
     switch (lpr) {
-        case 1: return launch_bwd<T, 1>(a, st);
-        case 2: return launch_bwd<T, 2>(a, st);
-        case 4: return launch_bwd<T, 4>(a, st);
-        case 8: return launch_bwd<T, 8>(a, st);
-        case 16: return launch_bwd<T, 16>(a, st);
-        case 32: return launch_bwd<T, 32>(a, st);
+        case 1: return launch_bwd<T, 1, LN>(a, st);
+        case 2: return launch_bwd<T, 2, LN>(a, st);
+        case 4: return launch_bwd<T, 4, LN>(a, st);
+        case 8: return launch_bwd<T, 8, LN>(a, st);
+        case 16: return launch_bwd<T, 16, LN>(a, st);
+        case 32: return launch_bwd<T, 32, LN>(a, st);
     }
     return QKNR_ERR_UNSUPPORTED;
 }
@@ -478,6 +478,10 @@ qknr_status fwd_impl(const void *q, const void *k, int64_t q_ts, int64_t k_ts,
         gamma_q = gamma_k = nullptr;
         rstd_q = rstd_k = nullptr;
         if ((Hq > 0 && (!q || !q_out)) || (Hkv > 0 && (!k || !k_out))) return QKNR_ERR_INVALID_ARG;
+    } else if (mode & kModeStatsOnly) {  // rstd alone: no gamma, no rows written
+        gamma_q = gamma_k = nullptr;
+        q_out = k_out = nullptr;
+        if ((Hq > 0 && (!q || !rstd_q)) || (Hkv > 0 && (!k || !rstd_k))) return QKNR_ERR_INVALID_ARG;
     } else {
         if (Hq > 0 && (!q || !q_out || !rstd_q || !gamma_q)) return QKNR_ERR_INVALID_ARG;
         if (Hkv > 0 && (!k || !k_out || !rstd_k || !gamma_k)) return QKNR_ERR_INVALID_ARG;
@@ -511,8 +515,11 @@ qknr_status fwd_impl(const void *q, const void *k, int64_t q_ts, int64_t k_ts,
     a.theta = theta; a.eps = eps; a.mode = mode;
     const int lpr = lanes_per_row(D, (int)e);
     cudaStream_t cs = (cudaStream_t)stream;
-    return dtype == QKNR_F32 ? dispatch_fwd<float>(a, lpr, cs)
-                             : dispatch_fwd<__nv_bfloat16>(a, lpr, cs);
+    if (mode & kModeLayerNorm)
+        return dtype == QKNR_F32 ? dispatch_fwd<float, true>(a, lpr, cs)
+                                 : dispatch_fwd<__nv_bfloat16, true>(a, lpr, cs);
+    return dtype == QKNR_F32 ? dispatch_fwd<float, false>(a, lpr, cs)
+                             : dispatch_fwd<__nv_bfloat16, false>(a, lpr, cs);
 }
 
 qknr_status bwd_impl(const void *q, const void *k, int64_t q_ts, int64_t k_ts,
@@ -521,7 +528,7 @@ qknr_status bwd_impl(const void *q, const void *k, int64_t q_ts, int64_t k_ts,
                      const void *dk_out, void *dq, void *dk, int64_t dq_ts, int64_t dk_ts,
                      float *dgamma_q, float *dgamma_k, int B, int S, int Hq, int Hkv, int D,
                      int rotary_dim, float theta, float eps, qknr_dtype dtype,
-                     qknr_stream_t stream) {
+                     qknr_stream_t stream, int mode = 0) {
     qknr_status st = check_shape(B, S, Hq, Hkv, D, rotary_dim, theta, eps, dtype);
     if (st != QKNR_OK) return st;
     const int64_t T = (int64_t)B * S;
@@ -577,8 +584,11 @@ qknr_status bwd_impl(const void *q, const void *k, int64_t q_ts, int64_t k_ts,
     a.T = T; a.S = S; a.Hq = Hq; a.Hkv = Hkv; a.D = D; a.R = rotary_dim;
     a.theta = theta; a.eps = eps;
     const int lpr = lanes_per_row(D, (int)e);
-    return dtype == QKNR_F32 ? dispatch_bwd<float>(a, lpr, cs)
-                             : dispatch_bwd<__nv_bfloat16>(a, lpr, cs);
+    if (mode & kModeLayerNorm)
+        return dtype == QKNR_F32 ? dispatch_bwd<float, true>(a, lpr, cs)
+                                 : dispatch_bwd<__nv_bfloat16, true>(a, lpr, cs);
+    return dtype == QKNR_F32 ? dispatch_bwd<float, false>(a, lpr, cs)
+                             : dispatch_bwd<__nv_bfloat16, false>(a, lpr, cs);
 }
 
 }  // namespace
@@ -631,6 +641,28 @@ extern "C" qknr_status qk_norm_rope_bwd_strided(
                     dgamma_k, B, S, Hq, Hkv, D, rotary_dim, theta, eps, dtype, stream);
 }
 
+extern "C" qknr_status qk_layernorm_rope_fwd(const void *q, const void *k, const void *gamma_q,
+                                             const void *gamma_k, const int32_t *pos_ids,
+                                             void *q_out, void *k_out, float *rstd_q,
+                                             float *rstd_k, int B, int S, int Hq, int Hkv, int D,
+                                             int rotary_dim, float theta, float eps,
+                                             qknr_dtype dtype, qknr_stream_t stream) {
+    return fwd_impl(q, k, (int64_t)Hq * D, (int64_t)Hkv * D, gamma_q, gamma_k, pos_ids, q_out,
+                    k_out, rstd_q, rstd_k, B, S, Hq, Hkv, D, rotary_dim, theta, eps, dtype, stream,
+                    kModeLayerNorm);
+}
+
+extern "C" qknr_status qk_layernorm_rope_bwd(
+    const void *q, const void *k, const void *gamma_q, const void *gamma_k, const int32_t *pos_ids,
+    const float *rstd_q, const float *rstd_k, const void *dq_out, const void *dk_out, void *dq,
+    void *dk, float *dgamma_q, float *dgamma_k, int B, int S, int Hq, int Hkv, int D,
+    int rotary_dim, float theta, float eps, qknr_dtype dtype, qknr_stream_t stream) {
+    const int64_t qts = (int64_t)Hq * D, kts = (int64_t)Hkv * D;
+    return bwd_impl(q, k, qts, kts, gamma_q, gamma_k, pos_ids, rstd_q, rstd_k, dq_out, dk_out, dq,
+                    dk, qts, kts, dgamma_q, dgamma_k, B, S, Hq, Hkv, D, rotary_dim, theta, eps,
+                    dtype, stream, kModeLayerNorm);
+}
+
 extern "C" qknr_status qk_norm_fwd(const void *q, const void *k, const void *gamma_q,
                                    const void *gamma_k, void *q_out, void *k_out, float *rstd_q,
                                    float *rstd_k, int B, int S, int Hq, int Hkv, int D, float eps,
@@ -648,6 +680,14 @@ extern "C" qknr_status qk_norm_bwd(const void *q, const void *k, const void *gam
     return bwd_impl(q, k, qts, kts, gamma_q, gamma_k, nullptr, rstd_q, rstd_k, dq_out, dk_out, dq,
                     dk, qts, kts, dgamma_q, dgamma_k, B, S, Hq, Hkv, D, 0, 1.0f, eps, dtype,
                     stream);
+}
+
+extern "C" qknr_status qk_rms_stats(const void *q, const void *k, float *rstd_q, float *rstd_k,
+                                    int B, int S, int Hq, int Hkv, int D, float eps,
+                                    qknr_dtype dtype, qknr_stream_t stream) {
+    return fwd_impl(q, k, (int64_t)Hq * D, (int64_t)Hkv * D, nullptr, nullptr, nullptr, nullptr,
+                    nullptr, rstd_q, rstd_k, B, S, Hq, Hkv, D, 0, 1.0f, eps, dtype, stream,
+                    kModeStatsOnly);
 }
 
 extern "C" qknr_status qk_rope_apply(const void *q, const void *k, const int32_t *pos_ids,

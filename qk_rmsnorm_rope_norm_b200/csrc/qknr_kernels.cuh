@@ -50,6 +50,8 @@ constexpr int kMaxHalf = kMaxD / 2;
 // Forward variants (FwdArgs::mode bits).
 constexpr int kModeRopeOnly = 1;  // rotation alone: r = 1, gamma = 1, no rstd written
 constexpr int kModeInverse = 2;   // rotate by -m (the transpose): strips RoPE
+constexpr int kModeStatsOnly = 4; // write rstd only, no normalised rows
+constexpr int kModeLayerNorm = 8; // mean-centred (QK-LayerNorm): host-side choice of kernel
 
 struct FwdArgs {
     const void *q, *k, *gq, *gk;
@@ -61,7 +63,7 @@ struct FwdArgs {
     int S, Hq, Hkv, D, R;
     float theta, eps;
     int tpw;    // consecutive tokens per warp
-    int mode;   // kModeRopeOnly | kModeInverse bits, 0 for the fused op
+    int mode;   // kMode* bits, 0 for the fused op
 };
 
 struct BwdArgs {
@@ -223,7 +225,8 @@ struct PosIter {
 // =================================================================== forward
 // A warp covers 32 / LPR rows of one token per pass; P passes are loaded
 // together so each lane keeps 2 * P 16-byte loads in flight.
-template <typename T, int LPR>
+// LN: the mean-centred variant (QK-LayerNorm): x - mean(x) in place of x.
+template <typename T, int LPR, bool LN>
 __global__ void __launch_bounds__(kThreads, QKNR_FWD_MIN_CTAS)
 qknr_fwd_kernel(const FwdArgs a) {
     using IO = Io<T>;
@@ -281,10 +284,23 @@ qknr_fwd_kernel(const FwdArgs a) {
             if (p0) load_chunk(p0);
 #pragma unroll
             for (int pp = 0; pp < P; ++pp) {
+                float mu = 0.f;
+                if (LN) {
+                    float sx = 0.f;
+#pragma unroll
+                    for (int k2 = 0; k2 < V / 2; ++k2) {
+                        const float2 va = IO::get2(xa[pp], k2), vb = IO::get2(xb[pp], k2);
+                        sx += (va.x + va.y) + (vb.x + vb.y);
+                    }
+                    mu = group_sum<LPR>(sx) * inv_d;
+                }
                 float ss = 0.f;
 #pragma unroll
                 for (int k2 = 0; k2 < V / 2; ++k2) {
-                    const float2 va = IO::get2(xa[pp], k2), vb = IO::get2(xb[pp], k2);
+                    float2 va = IO::get2(xa[pp], k2), vb = IO::get2(xb[pp], k2);
+                    if (LN && L.on) {
+                        va.x -= mu; va.y -= mu; vb.x -= mu; vb.y -= mu;
+                    }
                     ss = fmaf(va.x, va.x, ss); ss = fmaf(va.y, va.y, ss);
                     ss = fmaf(vb.x, vb.x, ss); ss = fmaf(vb.y, vb.y, ss);
                 }
@@ -297,7 +313,10 @@ qknr_fwd_kernel(const FwdArgs a) {
                     Vec16 ya, yb;
 #pragma unroll
                     for (int k2 = 0; k2 < V / 2; ++k2) {
-                        const float2 va = IO::get2(xa[pp], k2), vb = IO::get2(xb[pp], k2);
+                        float2 va = IO::get2(xa[pp], k2), vb = IO::get2(xb[pp], k2);
+                        if (LN) {
+                            va.x -= mu; va.y -= mu; vb.x -= mu; vb.y -= mu;
+                        }
                         const int e = 2 * k2;
                         const float2 c0 = lane_cs(cs, L.rot, L.eA + e);
                         const float2 c1 = lane_cs(cs, L.rot, L.eA + e + 1);
@@ -310,8 +329,10 @@ qknr_fwd_kernel(const FwdArgs a) {
                     const int hh = isq ? h : h - a.Hq;
                     const int64_t rowi = isq ? t * a.Hq + hh : t * a.Hkv + hh;
                     char *out = (char *)(isq ? a.qo : a.ko) + rowi * rowb;
-                    st16(out + offA, ya);
-                    st16(out + offB, yb);
+                    if (!(a.mode & kModeStatsOnly)) {
+                        st16(out + offA, ya);
+                        st16(out + offB, yb);
+                    }
                     if (L.u == 0 && !(a.mode & kModeRopeOnly)) (isq ? a.rq : a.rk)[rowi] = r;
                 }
             }
@@ -325,7 +346,9 @@ qknr_fwd_kernel(const FwdArgs a) {
 // dx = r (h - xh <h, xh> / D). The row is walked twice from the packed
 // registers (once for <h, xh> and the dgamma terms, once for dx) so that no
 // fp32 copy of the row is kept.
-template <typename T, int LPR>
+// LN: the mean-centred variant: xh = (x - mean) r and
+// dx = r (h - mean(h) - xh <h, xh> / D).
+template <typename T, int LPR, bool LN>
 __global__ void __launch_bounds__(kThreads, QKNR_BWD_MIN_CTAS)
 qknr_bwd_kernel(const BwdArgs a) {
     using IO = Io<T>;
@@ -402,9 +425,19 @@ qknr_bwd_kernel(const BwdArgs a) {
                 const bool isq = h < a.Hq;
                 const float *g = s_g[isq ? 0 : 1];
                 const float r = rr[pp];
+                float mu = 0.f;
+                if (LN) {
+                    float sx = 0.f;
+#pragma unroll
+                    for (int k2 = 0; k2 < V / 2; ++k2) {
+                        const float2 xa2 = IO::get2(xa[pp], k2), xb2 = IO::get2(xb[pp], k2);
+                        sx += (xa2.x + xa2.y) + (xb2.x + xb2.y);
+                    }
+                    mu = group_sum<LPR>(sx) * inv_d;
+                }
                 // walk 1: <h, xh> and the dgamma terms g * xh, four elements
-                // of each half at a time
-                float dot = 0.f;
+                // of each half at a time (and, mean-centred, sum of h)
+                float dot = 0.f, sh = 0.f;
                 float4 (*acc)[32] = isq ? acc_q : acc_k;
 #pragma unroll
                 for (int qd = 0; qd < V / 4; ++qd) {
@@ -418,13 +451,15 @@ qknr_bwd_kernel(const BwdArgs a) {
                             const int e = 2 * k2 + q;
                             const float2 c = lane_cs(cs, L.rot, L.eA + e);
                             const float dA = q ? da2.y : da2.x, dB = q ? db2.y : db2.x;
-                            const float xA = (q ? xa2.y : xa2.x) * r, xB = (q ? xb2.y : xb2.x) * r;
+                            const float xA = ((q ? xa2.y : xa2.x) - mu) * r;
+                            const float xB = ((q ? xb2.y : xb2.x) - mu) * r;
                             const float gA = fmaf(dA, c.x, dB * c.y);
                             const float gB = fmaf(dB, c.x, -dA * c.y);
                             tA[e & 3] = gA * xA;
                             tB[e & 3] = gB * xB;
                             dot = fmaf(gA * g[L.eA + e], xA, dot);
                             dot = fmaf(gB * g[L.eB + e], xB, dot);
+                            if (LN) sh += gA * g[L.eA + e] + gB * g[L.eB + e];
                         }
                     }
                     float4 &sa = acc[qd][lane];
@@ -436,6 +471,7 @@ qknr_bwd_kernel(const BwdArgs a) {
                     sb = vb;
                 }
                 dot = group_sum<LPR>(dot) * inv_d;
+                const float mh = LN ? group_sum<LPR>(sh) * inv_d : 0.f;
                 if (L.on && h < H) {
                     // walk 2: dx = r (h - xh * dot)
                     Vec16 oa, ob;
@@ -449,11 +485,12 @@ qknr_bwd_kernel(const BwdArgs a) {
                             const int e = 2 * k2 + q;
                             const float2 c = lane_cs(cs, L.rot, L.eA + e);
                             const float dA = q ? da2.y : da2.x, dB = q ? db2.y : db2.x;
-                            const float xA = (q ? xa2.y : xa2.x) * r, xB = (q ? xb2.y : xb2.x) * r;
+                            const float xA = ((q ? xa2.y : xa2.x) - mu) * r;
+                            const float xB = ((q ? xb2.y : xb2.x) - mu) * r;
                             const float hA = fmaf(dA, c.x, dB * c.y) * g[L.eA + e];
                             const float hB = fmaf(dB, c.x, -dA * c.y) * g[L.eB + e];
-                            outA[q] = r * fmaf(-xA, dot, hA);
-                            outB[q] = r * fmaf(-xB, dot, hB);
+                            outA[q] = r * fmaf(-xA, dot, LN ? hA - mh : hA);
+                            outB[q] = r * fmaf(-xB, dot, LN ? hB - mh : hB);
                         }
                         IO::put2(oa, k2, outA[0], outA[1]);
                         IO::put2(ob, k2, outB[0], outB[1]);

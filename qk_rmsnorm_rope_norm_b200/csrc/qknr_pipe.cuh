@@ -394,7 +394,8 @@ __device__ __forceinline__ void init_barriers(uint32_t full0, uint32_t empty0, c
 // ================================================================== forward
 // Per row: y_A = r (u_A c - u_B s), y_B = r (u_B c + u_A s), u = x * gamma,
 // evaluated as u_A (r c) - u_B (r s) and u_B (r c) + u_A (r s).
-template <typename T, int LPR, int U, int NCW, int NPW>
+// LN: the mean-centred variant (QK-LayerNorm): x - mean(x) in place of x.
+template <typename T, int LPR, int U, int NCW, int NPW, bool LN>
 __global__ void __launch_bounds__((NCW + NPW) * 32, 1)
 qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g, const __grid_constant__ CUtensorMap tmq,
                      const __grid_constant__ CUtensorMap tmk) {
@@ -540,6 +541,20 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g, const __grid_constant__ 
 #pragma unroll
                 for (int q = 0; q < U; ++q) xb[q] = lds16(src + off2[q]);
                 float r = 1.f;  // rotation alone: no normalisation
+                float2 nm2 = make_float2(0.f, 0.f);  // -mean (mean-centred variant)
+                if (LN) {
+                    float sx = 0.f;
+#pragma unroll
+                    for (int q = 0; q < U; ++q) {
+                        float2 s0 = make_float2(0.f, 0.f);
+#pragma unroll
+                        for (int k = 0; k < W; ++k)
+                            s0 = __fadd2_rn(s0, __fadd2_rn(IO::get2(xa[q], k), IO::get2(xb[q], k)));
+                        sx = fmaf(L.mask[q], s0.x + s0.y, sx);
+                    }
+                    const float mu = group_sum<LPR>(sx) * inv_d;
+                    nm2 = make_float2(-mu, -mu);
+                }
                 if (!(a.mode & kModeRopeOnly)) {
                     float ss = 0.f;
 #pragma unroll
@@ -547,7 +562,11 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g, const __grid_constant__ 
                         float2 s0 = make_float2(0.f, 0.f), s1 = make_float2(0.f, 0.f);
 #pragma unroll
                         for (int k = 0; k < W; ++k) {
-                            const float2 va = IO::get2(xa[q], k), vb = IO::get2(xb[q], k);
+                            float2 va = IO::get2(xa[q], k), vb = IO::get2(xb[q], k);
+                            if (LN) {
+                                va = __fadd2_rn(va, nm2);
+                                vb = __fadd2_rn(vb, nm2);
+                            }
                             s0 = __ffma2_rn(va, va, s0);
                             s1 = __ffma2_rn(vb, vb, s1);
                         }
@@ -560,7 +579,7 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g, const __grid_constant__ 
                 const float4 *tok = cs_tile + tr.tl * (half >> 1);
                 char *out = (tr.isq ? out_q : out_k) + tr.jj * rowb;
 #pragma unroll
-                for (int q = 0; q < U; ++q) {
+                for (int q = 0; q < U && !(a.mode & kModeStatsOnly); ++q) {
                     float4 cs[W], gv[W];
                     unit_table<V>(tok, L.rot[q], L.w[q], cs);
                     pair_gamma<V, X>(s_gl[tr.isq ? 0 : 1], L.w[q], L.kb[q], gv);
@@ -573,8 +592,13 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g, const __grid_constant__ 
                         const float2 ga = (k & 1) ? hi2(gv[k >> 1]) : lo2(gv[k >> 1]);
                         const float2 gb = (k & 1) ? hi2(gv[W / 2 + (k >> 1)]) : lo2(gv[W / 2 + (k >> 1)]);
                         const float2 c = __fmul2_rn(lo2(cs[k]), r2), sn = __fmul2_rn(hi2(cs[k]), rs2);
-                        const float2 ua = __fmul2_rn(IO::get2(xa[q], k), ga);
-                        const float2 ub = __fmul2_rn(IO::get2(xb[q], k), gb);
+                        float2 xa2 = IO::get2(xa[q], k), xb2 = IO::get2(xb[q], k);
+                        if (LN) {
+                            xa2 = __fadd2_rn(xa2, nm2);
+                            xb2 = __fadd2_rn(xb2, nm2);
+                        }
+                        const float2 ua = __fmul2_rn(xa2, ga);
+                        const float2 ub = __fmul2_rn(xb2, gb);
                         const float2 oa = __ffma2_rn(ua, c, __fmul2_rn(ub, neg2(sn)));
                         const float2 ob = __ffma2_rn(ub, c, __fmul2_rn(ua, sn));
                         IO::put2(ya, k, oa.x, oa.y);
@@ -598,7 +622,9 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g, const __grid_constant__ 
 // Per row: g = R^T dy; xh = x r; h = g gamma; dgamma += g xh;
 // dx = r (h - xh <h, xh> / D). One unit per lane: the dgamma partial sums
 // of both tensors stay in registers for the whole run.
-template <typename T, int LPR, int NCW, int NPW>
+// LN: the mean-centred variant: x_hat = (x - mean) r and
+// dx = r (h - mean(h) - x_hat <h, x_hat> / D).
+template <typename T, int LPR, int NCW, int NPW, bool LN>
 __global__ void __launch_bounds__((NCW + NPW) * 32, 1)
 qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g, const __grid_constant__ CUtensorMap tmq,
                      const __grid_constant__ CUtensorMap tmk) {
@@ -762,16 +788,26 @@ qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g, const __grid_constant__ 
                 unit_table<V>(cs_tile + tr.tl * (half >> 1), L.rot[0], uu, cs);
                 pair_gamma<V, X>(s_gl[tr.isq ? 0 : 1], uu, L.kb[0], gv);
                 const float2 r2 = make_float2(r, r);
+                float2 nmr2 = make_float2(0.f, 0.f);  // -mean * r (mean-centred variant)
+                if (LN) {
+                    float2 s0 = make_float2(0.f, 0.f);
+#pragma unroll
+                    for (int k = 0; k < W; ++k)
+                        s0 = __fadd2_rn(s0, __fadd2_rn(IO::get2(xa, k), IO::get2(xb, k)));
+                    const float mu = group_sum<LPR>(L.on[0] ? s0.x + s0.y : 0.f) * inv_d;
+                    nmr2 = make_float2(-mu * r, -mu * r);
+                }
                 float2 ha[W], hb[W], xha[W], xhb[W];
                 float2 d0 = make_float2(0.f, 0.f), d1 = make_float2(0.f, 0.f);
+                float2 e0 = make_float2(0.f, 0.f);  // sum of h (mean-centred variant)
 #pragma unroll
                 for (int k = 0; k < W; ++k) {
                     const float2 ga = (k & 1) ? hi2(gv[k >> 1]) : lo2(gv[k >> 1]);
                     const float2 gb = (k & 1) ? hi2(gv[W / 2 + (k >> 1)]) : lo2(gv[W / 2 + (k >> 1)]);
                     const float2 c = lo2(cs[k]), sn = __fmul2_rn(hi2(cs[k]), sg);
                     const float2 dA = IO::get2(da, k), dB = IO::get2(db, k);
-                    xha[k] = __fmul2_rn(IO::get2(xa, k), r2);
-                    xhb[k] = __fmul2_rn(IO::get2(xb, k), r2);
+                    xha[k] = LN ? __ffma2_rn(IO::get2(xa, k), r2, nmr2) : __fmul2_rn(IO::get2(xa, k), r2);
+                    xhb[k] = LN ? __ffma2_rn(IO::get2(xb, k), r2, nmr2) : __fmul2_rn(IO::get2(xb, k), r2);
                     const float2 gA = __ffma2_rn(dA, c, __fmul2_rn(dB, sn));
                     const float2 gB = __ffma2_rn(dB, c, __fmul2_rn(dA, neg2(sn)));
                     if (tr.isq) {
@@ -785,15 +821,19 @@ qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g, const __grid_constant__ 
                     hb[k] = __fmul2_rn(gB, gb);
                     d0 = __ffma2_rn(ha[k], xha[k], d0);
                     d1 = __ffma2_rn(hb[k], xhb[k], d1);
+                    if (LN) e0 = __fadd2_rn(e0, __fadd2_rn(ha[k], hb[k]));
                 }
                 const float dot = group_sum<LPR>((d0.x + d1.x) + (d0.y + d1.y)) * inv_d;
+                const float mh = LN ? group_sum<LPR>(e0.x + e0.y) * inv_d : 0.f;
                 if (valid) {
-                    const float2 nd = make_float2(-dot, -dot);
+                    const float2 nd = make_float2(-dot, -dot), nmh = make_float2(-mh, -mh);
                     Vec16 oa, ob;
 #pragma unroll
                     for (int k = 0; k < W; ++k) {
-                        const float2 va = __fmul2_rn(__ffma2_rn(xha[k], nd, ha[k]), r2);
-                        const float2 vb = __fmul2_rn(__ffma2_rn(xhb[k], nd, hb[k]), r2);
+                        const float2 pa = LN ? __fadd2_rn(ha[k], nmh) : ha[k];
+                        const float2 pb = LN ? __fadd2_rn(hb[k], nmh) : hb[k];
+                        const float2 va = __fmul2_rn(__ffma2_rn(xha[k], nd, pa), r2);
+                        const float2 vb = __fmul2_rn(__ffma2_rn(xhb[k], nd, pb), r2);
                         IO::put2(oa, k, va.x, va.y);
                         IO::put2(ob, k, vb.x, vb.y);
                     }

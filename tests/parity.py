@@ -36,8 +36,9 @@ def bf16_ulp(x: np.ndarray) -> np.ndarray:
     return np.exp2(np.floor(np.log2(a)) - 7)
 
 
-def gpu_run(inp: workloads.Inputs, device="cuda", fwd_only=False):
-    """Run the CUDA fwd (+ bwd) through the C ABI on ``inp``; CPU results."""
+def gpu_run(inp: workloads.Inputs, device="cuda", fwd_only=False, norm="rms"):
+    """Run the CUDA fwd (+ bwd) through the C ABI on ``inp``; CPU results.
+    ``norm="layer"``: the mean-centred (QK-LayerNorm) entry points."""
     import qk_rmsnorm_rope_norm_b200 as qknr
     w = inp.w
     dev = torch.device(device)
@@ -45,13 +46,13 @@ def gpu_run(inp: workloads.Inputs, device="cuda", fwd_only=False):
     gq, gk = inp.gamma_q.to(dev), inp.gamma_k.to(dev)
     pos = None if inp.pos is None else inp.pos.to(dev)
     qo, ko, rq, rk = qknr.qk_norm_rope_fwd(q, k, gq, gk, pos, rotary_dim=w.rotary_dim,
-                                           theta=w.theta, eps=w.eps)
+                                           theta=w.theta, eps=w.eps, norm=norm)
     out = {"q_out": qo, "k_out": ko, "rstd_q": rq, "rstd_k": rk}
     if not fwd_only:
         dqo, dko = inp.dq_out.to(dev), inp.dk_out.to(dev)
         dq, dk, dgq, dgk = qknr.qk_norm_rope_bwd(q, k, gq, gk, pos, rq, rk, dqo, dko,
                                                  rotary_dim=w.rotary_dim, theta=w.theta,
-                                                 eps=w.eps)
+                                                 eps=w.eps, norm=norm)
         out.update(dq=dq, dk=dk, dgamma_q=dgq, dgamma_k=dgk)
     torch.cuda.synchronize()
     return {n: t.cpu() for n, t in out.items()}
@@ -112,9 +113,10 @@ class Stats:
 
 
 def compare_with_oracle(inp: workloads.Inputs, got: dict, chunk_tokens: int = 4096,
-                        bwd: bool = True) -> Stats:
+                        bwd: bool = True, norm: str = "rms") -> Stats:
     """Every element of the GPU results against the oracle, token chunk by
-    token chunk (the oracle runs in fp64 on the CPU)."""
+    token chunk (the oracle runs in fp64 on the CPU). ``norm="layer"``
+    compares with the oracle's mean-centred form."""
     w = inp.w
     T = w.B * w.S
     st = Stats(w.dtype, w.D)
@@ -130,8 +132,9 @@ def compare_with_oracle(inp: workloads.Inputs, got: dict, chunk_tokens: int = 40
     for t0 in range(0, T, chunk_tokens):
         t1 = min(T, t0 + chunk_tokens)
         m = m_all[t0:t1]
-        qo, ko, rq, rk = orc.fwd(q[t0:t1], k[t0:t1], inp.gamma_q, inp.gamma_k, m,
-                                 w.rotary_dim, w.theta, w.eps)
+        fwd = orc.ln_fwd if norm == "layer" else orc.fwd
+        qo, ko, rq, rk = fwd(q[t0:t1], k[t0:t1], inp.gamma_q, inp.gamma_k, m,
+                             w.rotary_dim, w.theta, w.eps)
         st.elem("q_out", oracle.as_f64(view("q_out", w.Hq)[t0:t1]), qo)
         st.elem("k_out", oracle.as_f64(view("k_out", w.Hkv)[t0:t1]), ko)
         st.rstd(oracle.as_f64(view("rstd_q", w.Hq, 1)[t0:t1]).reshape(-1), rq.reshape(-1))
@@ -139,9 +142,14 @@ def compare_with_oracle(inp: workloads.Inputs, got: dict, chunk_tokens: int = 40
         if bwd:
             dqo = inp.dq_out.reshape(T, w.Hq, w.D)[t0:t1]
             dko = inp.dk_out.reshape(T, w.Hkv, w.D)[t0:t1]
-            dq, dk, dgq, dgk = orc.bwd(q[t0:t1], k[t0:t1], inp.gamma_q, inp.gamma_k, m,
-                                       dqo, dko, w.rotary_dim, w.theta, w.eps,
-                                       dgamma_q=dgq, dgamma_k=dgk)
+            if norm == "layer":
+                dq, dk, cq, ck = orc.ln_bwd(q[t0:t1], k[t0:t1], inp.gamma_q, inp.gamma_k, m,
+                                            dqo, dko, w.rotary_dim, w.theta, w.eps)
+                dgq, dgk = dgq + cq, dgk + ck
+            else:
+                dq, dk, dgq, dgk = orc.bwd(q[t0:t1], k[t0:t1], inp.gamma_q, inp.gamma_k, m,
+                                           dqo, dko, w.rotary_dim, w.theta, w.eps,
+                                           dgamma_q=dgq, dgamma_k=dgk)
             st.elem("dq", oracle.as_f64(view("dq", w.Hq)[t0:t1]), dq)
             st.elem("dk", oracle.as_f64(view("dk", w.Hkv)[t0:t1]), dk)
     st.dgamma = {"dgamma_q": (got["dgamma_q"].numpy(), dgq),

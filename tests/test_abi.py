@@ -193,3 +193,30 @@ def test_nope_and_rope_only_validation(lib):
     assert rope(qo=P(1, 4096)) == INVALID            # partial overlap with q
     assert rope(q=P(1, 8)) == ALIGN
     assert rope(pos=P(15, 2)) == ALIGN
+
+
+def test_rms_stats_validation(lib):
+    def stats(D=64, eps=1e-6, q=P(1), rq=P(7), rk=P(8)):
+        return lib.qk_rms_stats(q, P(2), rq, rk, 2, 8, 4, 2, D, eps, BF16, None)
+
+    assert stats(D=63) == INVALID
+    assert stats(eps=float("nan")) == INVALID
+    assert stats(q=None) == INVALID
+    assert stats(rq=None) == INVALID
+    assert stats(rq=P(7, 2)) == ALIGN
+    assert stats(rk=P(7, 64)) == INVALID             # the two statistics overlap
+
+
+def test_layernorm_entries_validate_like_rmsnorm(lib):
+    def ln_fwd(D=64, R=64, eps=1e-6, q=P(1)):
+        return lib.qk_layernorm_rope_fwd(q, P(2), P(3), P(4), None, P(5), P(6), P(7), P(8),
+                                         2, 8, 4, 2, D, R, 1e4, eps, BF16, None)
+
+    assert ln_fwd(D=63) == INVALID
+    assert ln_fwd(R=8) == UNSUP
+    assert ln_fwd(eps=-1.0) == INVALID
+    assert ln_fwd(q=None) == INVALID
+    assert ln_fwd(q=P(1, 8)) == ALIGN
+    assert lib.qk_layernorm_rope_bwd(P(1), P(2), P(3), P(4), None, P(7), P(8), P(9), P(10),
+                                     P(9, 16), P(12), P(13), P(14), 2, 8, 4, 2, 64, 64, 1e4,
+                                     1e-6, BF16, None) == INVALID

@@ -1,11 +1,12 @@
-"""The NoPE and rotation-only entry points (qk_norm_fwd / qk_norm_bwd and
-qk_rope_apply) through the C ABI.
+"""The NoPE, rotation-only and statistics-only entry points (qk_norm_fwd /
+qk_norm_bwd, qk_rope_apply, qk_rms_stats) through the C ABI.
 
 qk_norm_* must equal qk_norm_rope_* at rotary_dim = 0 bit for bit (the same
 kernels), and match the oracle. qk_rope_apply, forward and inverse, is checked
 element by element against the oracle's rotation alone (``rope_rows``),
 including extreme and negative positions and partial rotary spans; position 0
-and the dims past rotary_dim must come back bitwise unchanged. Both kernel
+and the dims past rotary_dim must come back bitwise unchanged. qk_rms_stats
+must equal the rstd the fused forward saves at rotary_dim = 0, bit for bit. Both kernel
 families (pipelined and plain-load) are covered.
 """
 import os
@@ -167,6 +168,27 @@ def test_qk_norm_is_rotary_dim_zero(cuda, kernels, name, over):
     for n in ("q_out", "k_out", "rstd_q", "rstd_k", "dq", "dk"):
         assert torch.equal(got[n], dense[n]), n
     parity.check(inp, got)
+
+
+@pytest.mark.parametrize("name,over", [("qwen2.5-0.5b", dict(B=2, S=333)),
+                                       ("llama3-8b-qknorm", dict(B=1, S=300)),
+                                       ("tiny", dict()),
+                                       ("tiny", dict(B=3, S=37, Hq=5, Hkv=3, D=24, rotary_dim=16))])
+def test_rms_stats_equal_saved_rstd(cuda, kernels, name, over):
+    """qk_rms_stats equals, bit for bit, the rstd the fused forward saves with
+    no rotary span (same lane layout, so the same fp32 summation order), and
+    the oracle's inverse RMS to the fp32 bound."""
+    inp = workloads.make_inputs(name, **dict(over, rotary_dim=0))
+    w = inp.w
+    dense = parity.gpu_run(inp, fwd_only=True)
+    rq, rk = qknr.qk_rms_stats(inp.q.to(cuda), inp.k.to(cuda), eps=w.eps)
+    torch.cuda.synchronize()
+    assert torch.equal(rq.cpu(), dense["rstd_q"]) and torch.equal(rk.cpu(), dense["rstd_k"])
+    rows = inp.q.double().numpy().reshape(-1, w.D)
+    _, ref_q = oracle.get().fwd_rows(rows, np.ones(w.D), np.zeros(len(rows), np.int64), 0,
+                                     w.theta, w.eps)
+    rel = np.abs(rq.cpu().double().numpy().reshape(-1) - ref_q) / ref_q
+    assert float(rel.max()) <= w.D * 2.0 ** -24
 
 
 def test_no_pipeline_timeouts(cuda):
