@@ -296,32 +296,61 @@ int input_maps(const void *q, const void *k, int64_t qts, int64_t kts, int Hq, i
     return mask;
 }
 
+template <typename T, int LPR, int U, bool LN, bool TM>
+qknr_status launch_fwd_pipe_tm(const FwdArgs &a, const PipeGeom &g, const CUtensorMap &mq,
+                               const CUtensorMap &mk, int grid, int smem, int dev, cudaStream_t st,
+                               bool *launched) {
+    static std::atomic<int> smem_ok[64];
+    auto kern = qknr_fwd_pipe_kernel<T, LPR, U, kFwdPipeWarps, kProducerWarps, LN, TM>;
+    *launched = false;
+    if (!allow_dyn_smem((const void *)kern, dev, smem_ok, smem)) return QKNR_OK;
+    *launched = true;
+    typename MapsArg<TM>::type maps{};
+    if constexpr (TM) maps = TensorMaps{mq, mk};
+    kern<<<grid, (kFwdPipeWarps + kProducerWarps) * 32, smem, st>>>(a, g, maps);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? QKNR_OK : cuda_fail(e);
+}
+
+template <typename T, int LPR, bool LN, bool TM>
+qknr_status launch_bwd_pipe_tm(const BwdArgs &a, const PipeGeom &g, const CUtensorMap &mq,
+                               const CUtensorMap &mk, int grid, int smem, int dev, cudaStream_t st,
+                               bool *launched) {
+    static std::atomic<int> smem_ok[64];
+    auto kern = qknr_bwd_pipe_kernel<T, LPR, kBwdPipeWarps, kProducerWarps, LN, TM>;
+    *launched = false;
+    if (!allow_dyn_smem((const void *)kern, dev, smem_ok, smem)) return QKNR_OK;
+    *launched = true;
+    typename MapsArg<TM>::type maps{};
+    if constexpr (TM) maps = TensorMaps{mq, mk};
+    kern<<<grid, (kBwdPipeWarps + kProducerWarps) * 32, smem, st>>>(a, g, maps);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? QKNR_OK : cuda_fail(e);
+}
+
+// The tensor-copy instantiation only for the forms that take strided inputs
+// (the fused RMSNorm op); every other form is dense.
 template <typename T, int LPR, int U, bool LN>
 qknr_status launch_fwd_pipe(const FwdArgs &a, const PipeGeom &g, const CUtensorMap &mq,
                             const CUtensorMap &mk, int grid, int smem, int dev, cudaStream_t st,
                             bool *launched) {
-    static std::atomic<int> smem_ok[64];
-    auto kern = qknr_fwd_pipe_kernel<T, LPR, U, kFwdPipeWarps, kProducerWarps, LN>;
-    *launched = false;
-    if (!allow_dyn_smem((const void *)kern, dev, smem_ok, smem)) return QKNR_OK;
-    *launched = true;
-    kern<<<grid, (kFwdPipeWarps + kProducerWarps) * 32, smem, st>>>(a, g, mq, mk);
-    cudaError_t e = cudaGetLastError();
-    return e == cudaSuccess ? QKNR_OK : cuda_fail(e);
+    if constexpr (!LN) {
+        if (g.tmap)
+            return launch_fwd_pipe_tm<T, LPR, U, LN, true>(a, g, mq, mk, grid, smem, dev, st,
+                                                           launched);
+    }
+    return launch_fwd_pipe_tm<T, LPR, U, LN, false>(a, g, mq, mk, grid, smem, dev, st, launched);
 }
 
 template <typename T, int LPR, bool LN>
 qknr_status launch_bwd_pipe(const BwdArgs &a, const PipeGeom &g, const CUtensorMap &mq,
                             const CUtensorMap &mk, int grid, int smem, int dev, cudaStream_t st,
                             bool *launched) {
-    static std::atomic<int> smem_ok[64];
-    auto kern = qknr_bwd_pipe_kernel<T, LPR, kBwdPipeWarps, kProducerWarps, LN>;
-    *launched = false;
-    if (!allow_dyn_smem((const void *)kern, dev, smem_ok, smem)) return QKNR_OK;
-    *launched = true;
-    kern<<<grid, (kBwdPipeWarps + kProducerWarps) * 32, smem, st>>>(a, g, mq, mk);
-    cudaError_t e = cudaGetLastError();
-    return e == cudaSuccess ? QKNR_OK : cuda_fail(e);
+    if constexpr (!LN) {
+        if (g.tmap)
+            return launch_bwd_pipe_tm<T, LPR, LN, true>(a, g, mq, mk, grid, smem, dev, st, launched);
+    }
+    return launch_bwd_pipe_tm<T, LPR, LN, false>(a, g, mq, mk, grid, smem, dev, st, launched);
 }
 
 int next_pow2(int x) {

@@ -139,6 +139,24 @@ __device__ __forceinline__ void tensor_g2s(uint32_t dst, const CUtensorMap *map,
         "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar), "l"(policy)
         : "memory");
 }
+// Tensor maps of strided Q and K, a kernel parameter only of the TM
+// instantiations (the dense ones take an empty one).
+struct TensorMaps {
+    CUtensorMap q, k;
+};
+struct NoTensorMaps {};
+template <bool TM> struct MapsArg {
+    using type = NoTensorMaps;
+};
+template <> struct MapsArg<true> {
+    using type = TensorMaps;
+};
+template <bool TM>
+__device__ __forceinline__ const CUtensorMap *map_of(const typename MapsArg<TM>::type &m, int z) {
+    if constexpr (TM) return z ? &m.k : &m.q;
+    else return nullptr;
+}
+
 // First token of the tensor-copy box of a tile [t0, t0 + na) in a run ending
 // at t_hi: the tile itself when it is whole, else the box that ends with the
 // run (so a partial last tile re-reads the end of the previous tile instead
@@ -394,12 +412,17 @@ __device__ __forceinline__ void init_barriers(uint32_t full0, uint32_t empty0, c
 // ================================================================== forward
 // Per row: y_A = r (u_A c - u_B s), y_B = r (u_B c + u_A s), u = x * gamma,
 // evaluated as u_A (r c) - u_B (r s) and u_B (r c) + u_A (r s).
-// LN: the mean-centred variant (QK-LayerNorm): x - mean(x) in place of x.
-template <typename T, int LPR, int U, int NCW, int NPW, bool LN>
+// LN: the mean-centred variant (QK-LayerNorm, x - mean(x) in place of x).
+// The mode word of FwdArgs selects the rotation alone, the inverse rotation
+// or the statistic alone (0: the fused op). TM: Q / K rows arrive by 3-D
+// tensor copy (strided inputs); the dense instantiations hold no
+// tensor-copy code.
+template <typename T, int LPR, int U, int NCW, int NPW, bool LN, bool TM>
 __global__ void __launch_bounds__((NCW + NPW) * 32, 1)
-qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g, const __grid_constant__ CUtensorMap tmq,
-                     const __grid_constant__ CUtensorMap tmk) {
+qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g,
+                     const __grid_constant__ typename MapsArg<TM>::type maps) {
     using IO = Io<T>;
+    const int mode = a.mode;
     constexpr int V = IO::V, W = V / 2;
     constexpr int SLOTS = 32 / LPR;
     extern __shared__ __align__(128) unsigned char smem[];
@@ -410,7 +433,8 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g, const __grid_constant__ 
 
     // tensor copies land on 128-byte boundaries (the stage offsets are
     // multiples of 128); should the dynamic base not be, report and stop
-    if (g.tmap && (smem_u32(smem) & 127u)) {
+    const int tmap = TM ? g.tmap : 0;
+    if (tmap && (smem_u32(smem) & 127u)) {
         if (threadIdx.x == 0) atomicOr(&g_qknr_pipe_error, 2u);
         return;
     }
@@ -438,17 +462,17 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g, const __grid_constant__ 
             unsigned char *st = smem + (size_t)s * g.stage_bytes;
             const uint32_t bq = (uint32_t)(na * a.Hq * rowb), bk = (uint32_t)(na * a.Hkv * rowb);
             // a tensor copy moves its whole box of TT tokens
-            const uint32_t xq = (g.tmap & 1) && bq ? (uint32_t)(g.TT * a.Hq * rowb) : bq;
-            const uint32_t xk = (g.tmap & 2) && bk ? (uint32_t)(g.TT * a.Hkv * rowb) : bk;
+            const uint32_t xq = (tmap & 1) && bq ? (uint32_t)(g.TT * a.Hq * rowb) : bq;
+            const uint32_t xk = (tmap & 2) && bk ? (uint32_t)(g.TT * a.Hkv * rowb) : bk;
             const int bs = (int)box_start(t0, run.t_hi, g.TT);
             const uint32_t bar = full0 + 8 * s;
             mbar_expect_tx(bar, xq + xk);
             if (bq) {
-                if (g.tmap & 1) tensor_g2s(smem_u32(st), &tmq, 0, 0, bs, bar, pol);
+                if (tmap & 1) tensor_g2s(smem_u32(st), map_of<TM>(maps, 0), 0, 0, bs, bar, pol);
                 else bulk_g2s(smem_u32(st), (const char *)a.q + t0 * a.qts, bq, bar, pol);
             }
             if (bk) {
-                if (g.tmap & 2) tensor_g2s(smem_u32(st + g.off_k), &tmk, 0, 0, bs, bar, pol);
+                if (tmap & 2) tensor_g2s(smem_u32(st + g.off_k), map_of<TM>(maps, 1), 0, 0, bs, bar, pol);
                 else bulk_g2s(smem_u32(st + g.off_k), (const char *)a.k + t0 * a.kts, bk, bar, pol);
             }
         };
@@ -507,7 +531,7 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g, const __grid_constant__ 
         for (int q = 0; q < U; ++q) {
             off1[q] = L.first[q] * (int)sizeof(T);
             off2[q] = L.second[q] * (int)sizeof(T);
-            sgn[q] = (a.mode & kModeInverse) ? -L.sgn[q] : L.sgn[q];
+            sgn[q] = (mode & kModeInverse) ? -L.sgn[q] : L.sgn[q];
         }
         const float inv_d = 1.0f / (float)a.D;
         int pc = 0;  // passes dealt before this tile, mod NCW
@@ -520,8 +544,8 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g, const __grid_constant__ 
             const int rows_q = na * a.Hq, rows = na * (a.Hq + a.Hkv);
             // tokens of a tensor-copy box before the tile (partial last tile)
             const int skip = (int)(t0 - box_start(t0, run.t_hi, g.TT));
-            const int xq0 = (g.tmap & 1) ? skip * a.Hq * rowb : 0;
-            const int xk0 = (g.tmap & 2) ? skip * a.Hkv * rowb : 0;
+            const int xq0 = (tmap & 1) ? skip * a.Hq * rowb : 0;
+            const int xk0 = (tmap & 2) ? skip * a.Hkv * rowb : 0;
             char *out_q = (char *)a.qo + t0 * a.Hq * rowb;   // the tile's first rows
             char *out_k = (char *)a.ko + t0 * a.Hkv * rowb;
             float *r_q = a.rq + t0 * a.Hq;
@@ -555,7 +579,7 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g, const __grid_constant__ 
                     const float mu = group_sum<LPR>(sx) * inv_d;
                     nm2 = make_float2(-mu, -mu);
                 }
-                if (!(a.mode & kModeRopeOnly)) {
+                if (!(mode & kModeRopeOnly)) {
                     float ss = 0.f;
 #pragma unroll
                     for (int q = 0; q < U; ++q) {
@@ -579,7 +603,7 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g, const __grid_constant__ 
                 const float4 *tok = cs_tile + tr.tl * (half >> 1);
                 char *out = (tr.isq ? out_q : out_k) + tr.jj * rowb;
 #pragma unroll
-                for (int q = 0; q < U && !(a.mode & kModeStatsOnly); ++q) {
+                for (int q = 0; q < U && !(mode & kModeStatsOnly); ++q) {
                     float4 cs[W], gv[W];
                     unit_table<V>(tok, L.rot[q], L.w[q], cs);
                     pair_gamma<V, X>(s_gl[tr.isq ? 0 : 1], L.w[q], L.kb[q], gv);
@@ -609,7 +633,7 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g, const __grid_constant__ 
                         stg16(out + off2[q], yb);
                     }
                 }
-                if (valid && L.u == 0 && !(a.mode & kModeRopeOnly)) __stcs((tr.isq ? r_q : r_k) + tr.jj, r);
+                if (valid && L.u == 0 && !(mode & kModeRopeOnly)) __stcs((tr.isq ? r_q : r_k) + tr.jj, r);
             }
             pc = (pc + npass) % NCW;
             __syncwarp();
@@ -623,11 +647,11 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g, const __grid_constant__ 
 // dx = r (h - xh <h, xh> / D). One unit per lane: the dgamma partial sums
 // of both tensors stay in registers for the whole run.
 // LN: the mean-centred variant: x_hat = (x - mean) r and
-// dx = r (h - mean(h) - x_hat <h, x_hat> / D).
-template <typename T, int LPR, int NCW, int NPW, bool LN>
+// dx = r (h - mean(h) - x_hat <h, x_hat> / D). TM as for the forward.
+template <typename T, int LPR, int NCW, int NPW, bool LN, bool TM>
 __global__ void __launch_bounds__((NCW + NPW) * 32, 1)
-qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g, const __grid_constant__ CUtensorMap tmq,
-                     const __grid_constant__ CUtensorMap tmk) {
+qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g,
+                     const __grid_constant__ typename MapsArg<TM>::type maps) {
     using IO = Io<T>;
     constexpr int V = IO::V, W = V / 2;
     constexpr int SLOTS = 32 / LPR;
@@ -640,7 +664,8 @@ qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g, const __grid_constant__ 
 
     // tensor copies land on 128-byte boundaries (the stage offsets are
     // multiples of 128); should the dynamic base not be, report and stop
-    if (g.tmap && (smem_u32(smem) & 127u)) {
+    const int tmap = TM ? g.tmap : 0;
+    if (tmap && (smem_u32(smem) & 127u)) {
         if (threadIdx.x == 0) atomicOr(&g_qknr_pipe_error, 2u);
         return;
     }
@@ -672,18 +697,18 @@ qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g, const __grid_constant__ 
             const uint32_t brq = (uint32_t)(na * a.Hq * 4) & ~15u;
             const uint32_t brk = (uint32_t)(na * a.Hkv * 4) & ~15u;
             // a tensor copy moves its whole box of TT tokens
-            const uint32_t xq = (g.tmap & 1) && bq ? (uint32_t)(g.TT * a.Hq * rowb) : bq;
-            const uint32_t xk = (g.tmap & 2) && bk ? (uint32_t)(g.TT * a.Hkv * rowb) : bk;
+            const uint32_t xq = (tmap & 1) && bq ? (uint32_t)(g.TT * a.Hq * rowb) : bq;
+            const uint32_t xk = (tmap & 2) && bk ? (uint32_t)(g.TT * a.Hkv * rowb) : bk;
             const int bs = (int)box_start(t0, run.t_hi, g.TT);
             const uint32_t bar = full0 + 8 * s;
             mbar_expect_tx(bar, xq + xk + bq + bk + brq + brk);
             if (bq) {
-                if (g.tmap & 1) tensor_g2s(smem_u32(st), &tmq, 0, 0, bs, bar, pol);
+                if (tmap & 1) tensor_g2s(smem_u32(st), map_of<TM>(maps, 0), 0, 0, bs, bar, pol);
                 else bulk_g2s(smem_u32(st), (const char *)a.q + t0 * a.qts, bq, bar, pol);
                 bulk_g2s(smem_u32(st + g.off_dq), (const char *)a.dqo + t0 * a.Hq * rowb, bq, bar, pol);
             }
             if (bk) {
-                if (g.tmap & 2) tensor_g2s(smem_u32(st + g.off_k), &tmk, 0, 0, bs, bar, pol);
+                if (tmap & 2) tensor_g2s(smem_u32(st + g.off_k), map_of<TM>(maps, 1), 0, 0, bs, bar, pol);
                 else bulk_g2s(smem_u32(st + g.off_k), (const char *)a.k + t0 * a.kts, bk, bar, pol);
                 bulk_g2s(smem_u32(st + g.off_dk), (const char *)a.dko + t0 * a.Hkv * rowb, bk, bar, pol);
             }
@@ -766,8 +791,8 @@ qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g, const __grid_constant__ 
             const int rows_q = na * a.Hq, rows = na * (a.Hq + a.Hkv);
             // tokens of a tensor-copy box before the tile (partial last tile)
             const int skip = (int)(t0 - box_start(t0, run.t_hi, g.TT));
-            const int xq0 = (g.tmap & 1) ? skip * a.Hq * rowb : 0;
-            const int xk0 = (g.tmap & 2) ? skip * a.Hkv * rowb : 0;
+            const int xq0 = (tmap & 1) ? skip * a.Hq * rowb : 0;
+            const int xk0 = (tmap & 2) ? skip * a.Hkv * rowb : 0;
             char *out_q = (char *)a.dq + t0 * a.dqts;
             char *out_k = (char *)a.dk + t0 * a.dkts;
             const float4 *cs_tile = reinterpret_cast<const float4 *>(st + g.off_cs);
