@@ -147,6 +147,10 @@ void geometry(const void *kernel, std::atomic<int> *cache, int64_t T, int *grid,
 #endif
 constexpr int kFwdPipeWarps = QKNR_FWD_PIPE_WARPS;  // consumer warps per CTA
 constexpr int kBwdPipeWarps = QKNR_BWD_PIPE_WARPS;
+// The mean-centred kernels keep more per-row state; with 12 consumer warps
+// (512 threads) their registers fit without spilling.
+constexpr int kBwdPipeWarpsLN = 12;
+constexpr int kFwdPipeWarpsLN = 12;
 constexpr int kProducerWarps = QKNR_PRODUCER_WARPS;  // copy issue + rotary tables
 #ifndef QKNR_STAGE_TARGET_BYTES
 #define QKNR_STAGE_TARGET_BYTES 81920
@@ -301,13 +305,14 @@ qknr_status launch_fwd_pipe_tm(const FwdArgs &a, const PipeGeom &g, const CUtens
                                const CUtensorMap &mk, int grid, int smem, int dev, cudaStream_t st,
                                bool *launched) {
     static std::atomic<int> smem_ok[64];
-    auto kern = qknr_fwd_pipe_kernel<T, LPR, U, kFwdPipeWarps, kProducerWarps, LN, TM>;
+    constexpr int NCW = LN ? kFwdPipeWarpsLN : kFwdPipeWarps;
+    auto kern = qknr_fwd_pipe_kernel<T, LPR, U, NCW, kProducerWarps, LN, TM>;
     *launched = false;
     if (!allow_dyn_smem((const void *)kern, dev, smem_ok, smem)) return QKNR_OK;
     *launched = true;
     typename MapsArg<TM>::type maps{};
     if constexpr (TM) maps = TensorMaps{mq, mk};
-    kern<<<grid, (kFwdPipeWarps + kProducerWarps) * 32, smem, st>>>(a, g, maps);
+    kern<<<grid, (NCW + kProducerWarps) * 32, smem, st>>>(a, g, maps);
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? QKNR_OK : cuda_fail(e);
 }
@@ -317,13 +322,14 @@ qknr_status launch_bwd_pipe_tm(const BwdArgs &a, const PipeGeom &g, const CUtens
                                const CUtensorMap &mk, int grid, int smem, int dev, cudaStream_t st,
                                bool *launched) {
     static std::atomic<int> smem_ok[64];
-    auto kern = qknr_bwd_pipe_kernel<T, LPR, kBwdPipeWarps, kProducerWarps, LN, TM>;
+    constexpr int NCW = LN ? kBwdPipeWarpsLN : kBwdPipeWarps;
+    auto kern = qknr_bwd_pipe_kernel<T, LPR, NCW, kProducerWarps, LN, TM>;
     *launched = false;
     if (!allow_dyn_smem((const void *)kern, dev, smem_ok, smem)) return QKNR_OK;
     *launched = true;
     typename MapsArg<TM>::type maps{};
     if constexpr (TM) maps = TensorMaps{mq, mk};
-    kern<<<grid, (kBwdPipeWarps + kProducerWarps) * 32, smem, st>>>(a, g, maps);
+    kern<<<grid, (NCW + kProducerWarps) * 32, smem, st>>>(a, g, maps);
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? QKNR_OK : cuda_fail(e);
 }
