@@ -466,14 +466,15 @@ cfg_args = None
 def bwd_kernel_name(w) -> str:
     """The backward kernel the library launches for this shape (the pipelined
     one: one row unit per lane, lanes per row the next power of two of
-    D / 16 bytes-pairs; 16 consumer and 4 producer warps; 0: the RMSNorm
-    form, as ncu prints the template flag)."""
+    D / 16 bytes-pairs; 12 consumer and 4 producer warps; then the
+    mean-centred and tensor-copy flags, 0 and 0 for the dense RMSNorm form,
+    as ncu prints them)."""
     dv2 = w.D // (2 * (16 // w.elem_bytes))
     lpr = 1
     while lpr < dv2:
         lpr *= 2
     tname = "__nv_bfloat16" if w.dtype == "bf16" else "float"
-    return f"qknr_bwd_pipe_kernel<{tname}, {lpr}, 16, 4, 0>"
+    return f"qknr_bwd_pipe_kernel<{tname}, {lpr}, 12, 4, 0, 0>"
 
 
 def config_of(w, inp, world):
