@@ -308,11 +308,23 @@ struct TileRow {
     bool isq;
     int jj;  // row index within its tensor's block of the tile
     int tl;  // token within the tile
-    __device__ __forceinline__ TileRow(int j, int rows_q, const PipeGeom &g) {
-        isq = j < rows_q;
-        jj = isq ? j : j - rows_q;
+    __device__ __forceinline__ TileRow(bool q, int j, const PipeGeom &g) {
+        isq = q;
+        jj = j;
         const uint32_t m = isq ? g.mq : g.mk;
         tl = m ? (int)__umulhi((uint32_t)jj, m) : jj;
+    }
+};
+
+// Row passes of a tile: the Q rows, then the K rows from a fresh pass, so
+// every pass is all Q or all K (the tensor is uniform across the warp).
+struct TilePasses {
+    int pq, npass, rows_q, rows_k;
+    __device__ __forceinline__ TilePasses(int na, int Hq, int Hkv, int slots) {
+        rows_q = na * Hq;
+        rows_k = na * Hkv;
+        pq = (rows_q + slots - 1) / slots;
+        npass = pq + (rows_k + slots - 1) / slots;
     }
 };
 
@@ -541,7 +553,7 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g,
             const unsigned char *st = smem + (size_t)s * g.stage_bytes;
             const int64_t t0 = run.t_lo + (int64_t)it * g.TT;
             const int na = (int)min((int64_t)g.TT, run.t_hi - t0);
-            const int rows_q = na * a.Hq, rows = na * (a.Hq + a.Hkv);
+
             // tokens of a tensor-copy box before the tile (partial last tile)
             const int skip = (int)(t0 - box_start(t0, run.t_hi, g.TT));
             const int xq0 = (tmap & 1) ? skip * a.Hq * rowb : 0;
@@ -551,13 +563,15 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g,
             float *r_q = a.rq + t0 * a.Hq;
             float *r_k = a.rk + t0 * a.Hkv;
             const float4 *cs_tile = reinterpret_cast<const float4 *>(st + g.off_cs);
-            const int npass = (rows + SLOTS - 1) / SLOTS;
+            const TilePasses tp(na, a.Hq, a.Hkv, SLOTS);
+            const int npass = tp.npass;
             int p = (warp - NPW) - pc;
             if (p < 0) p += NCW;
             for (; p < npass; p += NCW) {
-                const int j = p * SLOTS + L.slot;
-                const bool valid = j < rows;
-                const TileRow tr(valid ? j : 0, rows_q, g);
+                const bool isq = p < tp.pq;  // uniform across the warp
+                const int j = (isq ? p : p - tp.pq) * SLOTS + L.slot;
+                const bool valid = j < (isq ? tp.rows_q : tp.rows_k);
+                const TileRow tr(isq, valid ? j : 0, g);
                 const unsigned char *src = st + (tr.isq ? xq0 : g.off_k + xk0) + tr.jj * rowb;
                 Vec16 xa[U], xb[U];
 #pragma unroll
@@ -788,7 +802,7 @@ qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g,
             const unsigned char *st = smem + (size_t)s * g.stage_bytes;
             const int64_t t0 = run.t_lo + (int64_t)it * g.TT;
             const int na = (int)min((int64_t)g.TT, run.t_hi - t0);
-            const int rows_q = na * a.Hq, rows = na * (a.Hq + a.Hkv);
+
             // tokens of a tensor-copy box before the tile (partial last tile)
             const int skip = (int)(t0 - box_start(t0, run.t_hi, g.TT));
             const int xq0 = (tmap & 1) ? skip * a.Hq * rowb : 0;
@@ -796,13 +810,16 @@ qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g,
             char *out_q = (char *)a.dq + t0 * a.dqts;
             char *out_k = (char *)a.dk + t0 * a.dkts;
             const float4 *cs_tile = reinterpret_cast<const float4 *>(st + g.off_cs);
-            const int npass = (rows + SLOTS - 1) / SLOTS;
+            const TilePasses tp(na, a.Hq, a.Hkv, SLOTS);
+            const int npass = tp.npass;
             int p = (warp - NPW) - pc;
             if (p < 0) p += NCW;
             for (; p < npass; p += NCW) {
-                const int j = p * SLOTS + L.slot;
-                const bool valid = j < rows && L.on[0];
-                const TileRow tr(j < rows ? j : 0, rows_q, g);
+                const bool isq = p < tp.pq;  // uniform across the warp
+                const int j = (isq ? p : p - tp.pq) * SLOTS + L.slot;
+                const bool in = j < (isq ? tp.rows_q : tp.rows_k);
+                const bool valid = in && L.on[0];
+                const TileRow tr(isq, in ? j : 0, g);
                 const unsigned char *xs = st + (tr.isq ? xq0 : g.off_k + xk0) + tr.jj * rowb;
                 const unsigned char *ds = st + (tr.isq ? g.off_dq : g.off_dk) + tr.jj * rowb;
                 const Vec16 xa = lds16(xs + off1), da = lds16(ds + off1);
