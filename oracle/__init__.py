@@ -77,6 +77,12 @@ class Oracle:
         lib.oracle_ln_bwd_rows.restype = None
         lib.oracle_ln_bwd_rows.argtypes = [_D, _D, _D, _I64, c_i64, c_int,
                                            c_int, c_dbl, c_dbl, _D, _D]
+        lib.oracle_lw_fwd.restype = None
+        lib.oracle_lw_fwd.argtypes = [_D, _D, _I64, c_i64, c_int, c_int, c_int,
+                                      c_dbl, c_dbl, _D, _D]
+        lib.oracle_lw_bwd.restype = None
+        lib.oracle_lw_bwd.argtypes = [_D, _D, _D, _I64, c_i64, c_int, c_int,
+                                      c_int, c_dbl, c_dbl, _D, _D]
         lib.oracle_rope_rows.restype = None
         lib.oracle_rope_rows.argtypes = [_D, _I64, c_i64, c_int, c_int, c_dbl,
                                          c_int, _D]
@@ -197,6 +203,32 @@ class Oracle:
                                      np.repeat(m, H), R, theta, eps)
             out += [dx.reshape(x.shape), t.sum(axis=0)]
         return out[0], out[2], out[1], out[3]
+
+    def lw_fwd(self, x, gamma, m, R: int, theta: float, eps: float):
+        """Layerwise forward of one tensor x [..., H, D] (leading dims are
+        tokens), gamma [H*D]: one statistic per token over all its heads.
+        Returns (y like x, rstd [tokens])."""
+        x, g = as_f64(x), as_f64(gamma).reshape(-1)
+        H, D = x.shape[-2], x.shape[-1]
+        T = x.size // (H * D)
+        m = np.ascontiguousarray(np.asarray(m, dtype=np.int64).reshape(T))
+        y = np.empty_like(x)
+        r = np.empty(T)
+        self.lib.oracle_lw_fwd(_p(x), _p(g), _p(m, _I64), T, H, D, R, float(theta),
+                               float(eps), _p(y), _p(r))
+        return y, r
+
+    def lw_bwd(self, x, gamma, dy, m, R: int, theta: float, eps: float):
+        """Layerwise backward of one tensor; returns (dx like x, dgamma [H*D])."""
+        x, g, dy = as_f64(x), as_f64(gamma).reshape(-1), as_f64(dy)
+        H, D = x.shape[-2], x.shape[-1]
+        T = x.size // (H * D)
+        m = np.ascontiguousarray(np.asarray(m, dtype=np.int64).reshape(T))
+        dx = np.empty_like(x)
+        dg = np.zeros(H * D)
+        self.lib.oracle_lw_bwd(_p(x), _p(g), _p(dy), _p(m, _I64), T, H, D, R,
+                               float(theta), float(eps), _p(dx), _p(dg))
+        return dx, dg
 
     def rope_rows(self, x, m, R: int, theta: float, inverse: bool = False):
         """Rotation alone of rows x [n, D] at positions m [n]: R(m) x, or

@@ -45,6 +45,14 @@
  *   n_d     = (x_d - mu) * r * gamma_d, then the same rotation
  *   backward: xh = (x - mu) r, dgamma += g xh, h = g gamma,
  *   dx_d    = r * (h_d - (1/D) sum_e h_e - xh_d (1/D) sum_e h_e xh_e)
+ * Layerwise variant ("SwiftQK: Fast and Communication-Efficient Tensor
+ * Parallelism for Query-Key Normalization", abstract: the normalisation
+ * factor depends on the full hidden vector): per token, over all H heads,
+ *   r_t     = 1 / sqrt((1/(H D)) * sum_{h,d} x[h,d]^2 + eps)   (saved)
+ *   n[h,d]  = x[h,d] * r_t * gamma[h*D + d]   (gamma over the full hidden),
+ *   then the same rotation on every head row; backward, per token:
+ *   xh = x r_t, dgamma[h*D + d] += g xh, hh = g gamma,
+ *   dx = r_t * (hh - xh * (1/(H D)) * sum_{h,d} hh xh)
  * Rotation alone (no normalisation), forward or inverse:
  *   y = R(m) x, or y = R(m)^T x = R(-m) x, which strips RoPE from a rotated
  *   row (the cross-model KV cache transfer abstract on the papers listing:
@@ -316,4 +324,75 @@ void oracle_ln_bwd_rows(const double *x, const double *gamma, const double *dy,
     free(g);
     free(h);
     free(xh);
+}
+
+/*
+ * Layerwise forward: x [T, H, D] (one tensor), gamma [H*D], m [T]; y like x,
+ * rstd [T] (one statistic per token over its whole hidden vector).
+ */
+void oracle_lw_fwd(const double *x, const double *gamma, const int64_t *m,
+                   int64_t T, int H, int D, int R, double theta, double eps,
+                   double *y, double *rstd)
+{
+    int half = R / 2;
+    int64_t HD = (int64_t)H * D;
+    for (int64_t t = 0; t < T; ++t) {
+        const double *xt = x + t * HD;
+        double *yt = y + t * HD;
+        double ss = 0.0;
+        for (int64_t e = 0; e < HD; ++e)
+            ss += xt[e] * xt[e];
+        double r = 1.0 / sqrt(ss / (double)HD + eps);
+        rstd[t] = r;
+        for (int h = 0; h < H; ++h) {
+            const double *xr = xt + (int64_t)h * D;
+            double *yr = yt + (int64_t)h * D;
+            for (int d = 0; d < D; ++d)
+                yr[d] = xr[d] * r * gamma[h * D + d];
+            for (int i = 0; i < half; ++i) {
+                double phi = (double)m[t] * oracle_inv_freq(i, R, theta);
+                double c = cos(phi), s = sin(phi);
+                double a = yr[i], b = yr[i + half];
+                yr[i] = a * c - b * s;
+                yr[i + half] = b * c + a * s;
+            }
+        }
+    }
+}
+
+/* Layerwise backward: dx like x; dgamma [H*D] accumulated into. */
+void oracle_lw_bwd(const double *x, const double *gamma, const double *dy,
+                   const int64_t *m, int64_t T, int H, int D, int R,
+                   double theta, double eps, double *dx, double *dgamma)
+{
+    int half = R / 2;
+    int64_t HD = (int64_t)H * D;
+    double *g = (double *)malloc(sizeof(double) * (size_t)HD);
+    for (int64_t t = 0; t < T; ++t) {
+        const double *xt = x + t * HD, *dyt = dy + t * HD;
+        double ss = 0.0;
+        for (int64_t e = 0; e < HD; ++e)
+            ss += xt[e] * xt[e];
+        double r = 1.0 / sqrt(ss / (double)HD + eps);
+        for (int h = 0; h < H; ++h) {
+            const double *dr = dyt + (int64_t)h * D;
+            double *gr = g + (int64_t)h * D;
+            for (int d = 0; d < D; ++d)
+                gr[d] = dr[d];
+            for (int i = 0; i < half; ++i) {
+                double phi = (double)m[t] * oracle_inv_freq(i, R, theta);
+                double c = cos(phi), s = sin(phi);
+                gr[i] = dr[i] * c + dr[i + half] * s;
+                gr[i + half] = -dr[i] * s + dr[i + half] * c;
+            }
+        }
+        double dot = 0.0;
+        for (int64_t e = 0; e < HD; ++e) {
+            dgamma[e] += g[e] * xt[e] * r;
+            dot += g[e] * gamma[e] * xt[e] * r;
+        }
+        for (int64_t e = 0; e < HD; ++e)
+            dx[t * HD + e] = r * (g[e] * gamma[e] - xt[e] * r * dot / (double)HD);
+    }
+    free(g);
 }

@@ -470,4 +470,65 @@ def pin_ln_bwd_matches_autograd(orc):
     _close(dgr.sum(axis=0), gt.grad.numpy(), tol=1e-12, what="ln dgamma vs autograd")
 
 
+# ----------------------------------------------------------- layerwise variant
+def pin_lw_matches_library(orc):
+    """Layerwise forward: torch rms_norm over each token's whole hidden vector
+    (H * D, weight over the hidden), then complex-multiplication RoPE on each
+    head row."""
+    rng = np.random.default_rng(51)
+    for H, D, R in ((3, 8, 8), (4, 16, 0), (2, 32, 16)):
+        T = 6
+        x = rng.standard_normal((T, H, D)) * 2.0
+        g = 1.0 + 0.1 * rng.standard_normal(H * D)
+        m = rng.integers(0, 40000, T)
+        y, r = orc.lw_fwd(x, g, m, R, 1e4, 1e-6)
+        xt = torch.as_tensor(x.reshape(T, H * D))
+        n = F.rms_norm(xt, (H * D,), weight=torch.as_tensor(g), eps=1e-6).numpy().reshape(T, H, D)
+        want = _complex_rope(n.reshape(T * H, D), np.repeat(m, H), R, 1e4).reshape(T, H, D)
+        _close(y, want, what=f"layerwise H={H} D={D} R={R}")
+        _close(r, 1.0 / np.sqrt((x.reshape(T, -1) ** 2).mean(axis=1) + 1e-6), tol=1e-13,
+               what="layerwise rstd")
+
+
+def pin_lw_one_head_is_per_head(orc):
+    """With one head the layerwise form is the per-head form."""
+    rng = np.random.default_rng(52)
+    T, D, R = 7, 32, 32
+    x = rng.standard_normal((T, 1, D))
+    g = _gamma(rng, D)
+    m = rng.integers(0, 9000, T)
+    y, r = orc.lw_fwd(x, g, m, R, 1e4, 1e-5)
+    y1, r1 = orc.fwd_rows(x.reshape(T, D), g, m, R, 1e4, 1e-5)
+    _close(y.reshape(T, D), y1, tol=1e-13, what="layerwise H=1 vs per head")
+    _close(r, r1, tol=1e-13, what="layerwise H=1 rstd")
+    dy = rng.standard_normal((T, 1, D))
+    dx, dg = orc.lw_bwd(x, g, dy, m, R, 1e4, 1e-5)
+    dx1, t1 = orc.bwd_rows(x.reshape(T, D), g, dy.reshape(T, D), m, R, 1e4, 1e-5)
+    _close(dx.reshape(T, D), dx1, tol=1e-12, what="layerwise H=1 dx")
+    _close(dg, t1.sum(axis=0), tol=1e-12, what="layerwise H=1 dgamma")
+
+
+def pin_lw_bwd_matches_autograd(orc):
+    """Layerwise backward against torch autograd through rms_norm over the
+    hidden vector and complex-multiplication RoPE per head."""
+    rng = np.random.default_rng(53)
+    T, H, D, R, eps = 4, 3, 16, 8, 1e-4
+    x = rng.standard_normal((T, H, D)) * 1.5
+    g = 1.0 + 0.1 * rng.standard_normal(H * D)
+    dy = rng.standard_normal((T, H, D))
+    m = rng.integers(0, 5000, T)
+    xt = torch.tensor(x, requires_grad=True)
+    gt = torch.tensor(g, requires_grad=True)
+    n = F.rms_norm(xt.reshape(T, H * D), (H * D,), weight=gt, eps=eps).reshape(T, H, D)
+    half = R // 2
+    ang = torch.tensor(m, dtype=torch.float64)[:, None, None] * torch.pow(
+        torch.tensor(1e4, dtype=torch.float64), -2.0 * torch.arange(half, dtype=torch.float64) / R)
+    z = torch.complex(n[..., :half], n[..., half:R]) * torch.polar(torch.ones_like(ang), ang)
+    y = torch.cat([z.real, z.imag, n[..., R:]], dim=-1)
+    (y * torch.tensor(dy)).sum().backward()
+    dx, dg = orc.lw_bwd(x, g, dy, m, R, 1e4, eps)
+    _close(dx, xt.grad.numpy(), tol=1e-12, what="layerwise dx vs autograd")
+    _close(dg, gt.grad.numpy(), tol=1e-12, what="layerwise dgamma vs autograd")
+
+
 ALL_PINS = [v for k_, v in sorted(globals().items()) if k_.startswith("pin_")]

@@ -74,6 +74,14 @@ MUTATIONS = [
     ("ln_bwd_xh_not_centred", [("            xh[d] = (xr[d] - mu) * r;", "            xh[d] = xr[d] * r;", 0)]),
     ("ln_bwd_unrotate_sign", [("            g[i + half] = -dyr[i] * s + dyr[i + half] * c;",
                                "            g[i + half] = dyr[i] * s + dyr[i + half] * c;", 0)]),
+    ("lw_mean_over_D_only", [("        double r = 1.0 / sqrt(ss / (double)HD + eps);\n        rstd[t] = r;",
+                              "        double r = 1.0 / sqrt(ss / (double)D + eps);\n        rstd[t] = r;", 0)]),
+    ("lw_gamma_per_dim_only", [("                yr[d] = xr[d] * r * gamma[h * D + d];",
+                                "                yr[d] = xr[d] * r * gamma[d];", 0)]),
+    ("lw_bwd_dot_dropped", [("dx[t * HD + e] = r * (g[e] * gamma[e] - xt[e] * r * dot / (double)HD);",
+                             "dx[t * HD + e] = r * (g[e] * gamma[e]);", 0)]),
+    ("lw_bwd_dgamma_without_r", [("            dgamma[e] += g[e] * xt[e] * r;",
+                                  "            dgamma[e] += g[e] * xt[e];", 0)]),
     ("rope_inverse_ignored", [("            s = -s;", "            s = s;", 0)]),
     ("rope_sin_sign_first", [("yr[i] = xr[i] * c - xr[i + half] * s;",
                               "yr[i] = xr[i] * c + xr[i + half] * s;", 0)]),
