@@ -361,7 +361,85 @@ def run_variants(args, w, inp, dev, peak):
     out["rope_only"] = {"fwd": line(timed([rope(s, False) for s in dense]), rope_bytes),
                         "inverse": line(timed([rope(s, True) for s in dense]), rope_bytes),
                         "entry": "qk_rope_apply"}
+    out.update(layerwise_variants(w, dense, dev, timed, line))
     return out
+
+
+def layerwise_variants(w, dense, dev, timed, line):
+    """Layerwise (all-heads) QK-norm on the same rows, gamma over the full
+    hidden vector and one statistic per token and tensor. "one_pass": one
+    rank holds every head, one launch each way. "tp_phases": the sequence a
+    tensor-parallel rank runs (stats, then normalise; dots, then backward),
+    here with every head on one GPU and no exchange between the phases, so it
+    times the extra pass over the rows that sharding costs. Bytes are the
+    op's contract bytes (each row read once and written once, dy read once,
+    rstd [T] per tensor)."""
+    import qk_rmsnorm_rope_norm_b200 as qknr
+    lib = qknr.load_library()
+    P = qknr._ptr
+    dt = 0 if w.dtype == "f32" else 1
+    st = qknr._stream(None)
+    T = w.B * w.S
+    e = w.elem_bytes
+    H = w.Hq + w.Hkv
+    pos_b = 4 * T if dense[0].pos is not None else 0
+    gbytes = H * w.D * e
+    fwd_b = 2 * T * H * w.D * e + 4 * T * (int(w.Hq > 0) + int(w.Hkv > 0)) + pos_b + gbytes
+    bwd_b = 3 * T * H * w.D * e + 4 * T * (int(w.Hq > 0) + int(w.Hkv > 0)) + pos_b + gbytes
+    gq, gk = workloads.layerwise_gamma(w, 17)
+    gq, gk = gq.to(dev), gk.to(dev)
+    bufs = []
+    for s in dense:
+        bufs.append(dict(rq=torch.empty(T, device=dev), rk=torch.empty(T, device=dev),
+                         sq=torch.empty(T, device=dev), sk=torch.empty(T, device=dev),
+                         dgq=torch.empty(w.Hq * w.D, device=dev),
+                         dgk=torch.empty(w.Hkv * w.D, device=dev)))
+
+    def fwd(s, b, sums):
+        sq, sk = (P(b["sq"]), P(b["sk"])) if sums else (None, None)
+        return (P(s.q), P(s.k), P(gq), P(gk), P(s.pos), sq, sk, P(s.qo), P(s.ko), P(b["rq"]),
+                P(b["rk"]), w.B, w.S, w.Hq, w.Hkv, w.Hq, w.Hkv, w.D, w.rotary_dim,
+                float(w.theta), float(w.eps), dt, st)
+
+    def bwd(s, b, sums):
+        sq, sk = (P(b["sq"]), P(b["sk"])) if sums else (None, None)
+        return (P(s.q), P(s.k), P(gq), P(gk), P(s.pos), P(b["rq"]), P(b["rk"]), P(s.dqo),
+                P(s.dko), sq, sk, P(s.dq), P(s.dk), P(b["dgq"]), P(b["dgk"]), w.B, w.S, w.Hq,
+                w.Hkv, w.Hq, w.Hkv, w.D, w.rotary_dim, float(w.theta), dt, st)
+
+    def stats(s, b):
+        return (P(s.q), P(s.k), P(b["sq"]), P(b["sk"]), w.B, w.S, w.Hq, w.Hkv, w.D, dt, st)
+
+    def dots(s, b):
+        return (P(s.q), P(s.k), P(gq), P(gk), P(s.pos), P(b["rq"]), P(b["rk"]), P(s.dqo),
+                P(s.dko), P(b["sq"]), P(b["sk"]), w.B, w.S, w.Hq, w.Hkv, w.D, w.rotary_dim,
+                float(w.theta), dt, st)
+
+    C = qknr.PreparedCall
+
+    def seq(*calls):
+        def run():
+            for c in calls:
+                c()
+        return run
+
+    one_f = [C(lib.qk_layerwise_norm_rope_fwd, fwd(s, b, False), "lw fwd", s)
+             for s, b in zip(dense, bufs)]
+    one_b = [C(lib.qk_layerwise_norm_rope_bwd, bwd(s, b, False), "lw bwd", s)
+             for s, b in zip(dense, bufs)]
+    two_f = [seq(C(lib.qk_layerwise_stats, stats(s, b), "lw stats", s),
+                 C(lib.qk_layerwise_norm_rope_fwd, fwd(s, b, True), "lw fwd", s))
+             for s, b in zip(dense, bufs)]
+    two_b = [seq(C(lib.qk_layerwise_bwd_dots, dots(s, b), "lw dots", s),
+                 C(lib.qk_layerwise_norm_rope_bwd, bwd(s, b, True), "lw bwd", s))
+             for s, b in zip(dense, bufs)]
+    return {
+        "layerwise_one_pass": {"fwd": line(timed(one_f), fwd_b), "bwd": line(timed(one_b), bwd_b),
+                               "entry": "qk_layerwise_norm_rope_fwd / _bwd, sums NULL"},
+        "layerwise_tp_phases": {"fwd": line(timed(two_f), fwd_b),
+                                "bwd": line(timed(two_b), bwd_b),
+                                "entry": "qk_layerwise_stats + _fwd; qk_layerwise_bwd_dots + _bwd"},
+    }
 
 
 def copy_floor_ms(traffic_bytes: int, dev, n: int = 20) -> float:

@@ -279,6 +279,89 @@ QKNR_API qknr_status qk_rope_apply(const void *q, const void *k,
                              int rotary_dim, float theta, int inverse,
                              qknr_dtype dtype, qknr_stream_t stream);
 
+/*
+ * Layerwise QK-RMSNorm + RoPE under tensor parallelism. "SwiftQK: Fast and
+ * Communication-Efficient Tensor Parallelism for Query-Key Normalization"
+ * (abstract, on the papers listing the sources include): a layerwise
+ * QK-norm normalises each token's whole hidden vector (all heads of q, and
+ * separately all heads of k), so when the heads are split over ranks only
+ * one scalar statistic per token and tensor has to cross GPUs. Each rank
+ * holds Hq of the Hq_total query heads and Hkv of the Hkv_total key heads
+ * (dense [B,S,Hq,D] / [B,S,Hkv,D] rows) and the matching slices of the
+ * learned weights: gamma_q [Hq*D], gamma_k [Hkv*D], the rank's part of the
+ * full-hidden gamma. Per token t (T = B*S):
+ *
+ *   1. qk_layerwise_stats: s_t = sum over the rank's heads and dims of x^2,
+ *      fp32 [T] (sumsq_q from q, sumsq_k from k).
+ *   2. the caller sums s_t over the ranks (an all-reduce of T fp32 values;
+ *      with one rank, nothing), giving S_t.
+ *   3. qk_layerwise_norm_rope_fwd: r_t = 1/sqrt(S_t/(H_total*D) + eps),
+ *      saved fp32 [T] in rstd_q / rstd_k; out = R(m) (x r_t gamma) on every
+ *      head row, the rotate-half rotation of qk_norm_rope_fwd.
+ *
+ * Backward: with g = R(m)^T dy, hh = g gamma and xh = x r_t,
+ *   4. qk_layerwise_bwd_dots: p_t = sum over the rank of hh . xh, fp32 [T].
+ *   5. the caller sums p_t over the ranks, giving P_t.
+ *   6. qk_layerwise_norm_rope_bwd: dx = r_t (hh - xh P_t/(H_total*D)) and
+ *      dgamma[h*D + d] = sum over tokens of g xh (the rank's slice; fp32,
+ *      zeroed by the call, may be NULL).
+ *
+ * One rank holding every head (Hq_total = Hq, Hkv_total = Hkv) may pass
+ * NULL for both sumsq pointers of step 3, or both dot pointers of step 6:
+ * the call then takes the statistic itself in the same pass (steps 1-2 or
+ * 4-5 skipped; each row is read again from cache, not from HBM). NULL sums
+ * with totals above the local counts are QKNR_ERR_INVALID_ARG.
+ *
+ * pos_ids as for qk_norm_rope_fwd (NULL: position s of each row). Either
+ * tensor may have zero local heads (its pointers are then unused). Rows,
+ * gamma, outputs: 16-byte aligned; fp32 vectors: 4-byte aligned. Shapes as
+ * for qk_norm_rope_fwd; Hq_total >= Hq, Hkv_total >= Hkv (else
+ * QKNR_ERR_INVALID_ARG). The backward keeps the rank's dgamma partial sums
+ * in shared memory: (Hq + Hkv) * D * 4 bytes at most 200 KiB, else
+ * QKNR_ERR_UNSUPPORTED. No output may overlap an input or another output
+ * (QKNR_ERR_INVALID_ARG), except exactly in place: q_out = q, k_out = k,
+ * dq = dq_out, dk = dk_out. T = 0 or no heads: nothing launched (the
+ * backward still zeroes dgamma).
+ */
+QKNR_API qknr_status qk_layerwise_stats(const void *q, const void *k,
+                             float *sumsq_q, float *sumsq_k,
+                             int B, int S, int Hq, int Hkv, int D,
+                             qknr_dtype dtype, qknr_stream_t stream);
+
+QKNR_API qknr_status qk_layerwise_norm_rope_fwd(const void *q, const void *k,
+                             const void *gamma_q, const void *gamma_k,
+                             const int32_t *pos_ids,
+                             const float *sumsq_q, const float *sumsq_k,
+                             void *q_out, void *k_out,
+                             float *rstd_q, float *rstd_k,
+                             int B, int S, int Hq, int Hkv,
+                             int Hq_total, int Hkv_total, int D,
+                             int rotary_dim, float theta, float eps,
+                             qknr_dtype dtype, qknr_stream_t stream);
+
+QKNR_API qknr_status qk_layerwise_bwd_dots(const void *q, const void *k,
+                             const void *gamma_q, const void *gamma_k,
+                             const int32_t *pos_ids,
+                             const float *rstd_q, const float *rstd_k,
+                             const void *dq_out, const void *dk_out,
+                             float *dot_q, float *dot_k,
+                             int B, int S, int Hq, int Hkv, int D,
+                             int rotary_dim, float theta,
+                             qknr_dtype dtype, qknr_stream_t stream);
+
+QKNR_API qknr_status qk_layerwise_norm_rope_bwd(const void *q, const void *k,
+                             const void *gamma_q, const void *gamma_k,
+                             const int32_t *pos_ids,
+                             const float *rstd_q, const float *rstd_k,
+                             const void *dq_out, const void *dk_out,
+                             const float *dot_q, const float *dot_k,
+                             void *dq, void *dk,
+                             float *dgamma_q, float *dgamma_k,
+                             int B, int S, int Hq, int Hkv,
+                             int Hq_total, int Hkv_total, int D,
+                             int rotary_dim, float theta,
+                             qknr_dtype dtype, qknr_stream_t stream);
+
 /* Static English text for a status code; never NULL. */
 QKNR_API const char *qknr_strerror(qknr_status status);
 

@@ -25,7 +25,10 @@ __all__ = ["qk_norm_rope_fwd", "qk_norm_rope_bwd", "qknr_strerror", "QKNormRoPE"
            "QKNormRoPEFromQKV", "qk_norm_rope_qkv", "split_qkv",
            "qk_norm_fwd", "qk_norm_bwd", "qk_rope_apply", "QKRoPE", "qk_rms_stats",
            "prepare_fwd", "prepare_bwd", "PreparedCall",
-           "qk_norm_rope", "QKNRError", "library_path", "load_library", "pipeline_error"]
+           "qk_norm_rope", "QKNRError", "library_path", "load_library", "pipeline_error",
+           "qk_layerwise_stats", "qk_layerwise_norm_rope_fwd", "qk_layerwise_bwd_dots",
+           "qk_layerwise_norm_rope_bwd", "QKLayerwiseNormRoPE", "qk_layerwise_norm_rope",
+           "all_reduce_stats"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libqknr.so")
@@ -81,6 +84,14 @@ def load_library():
     lib.qk_norm_rope_bwd_strided.restype = i32
     lib.qk_norm_rope_bwd_strided.argtypes = [vp, vp, i64, i64] + [vp] * 9 + [i64, i64] + \
         [vp] * 2 + [i32] * 6 + [f32, f32, i32, vp]
+    lib.qk_layerwise_stats.restype = i32
+    lib.qk_layerwise_stats.argtypes = [vp] * 4 + [i32] * 5 + [i32, vp]
+    lib.qk_layerwise_norm_rope_fwd.restype = i32
+    lib.qk_layerwise_norm_rope_fwd.argtypes = [vp] * 11 + [i32] * 8 + [f32, f32, i32, vp]
+    lib.qk_layerwise_bwd_dots.restype = i32
+    lib.qk_layerwise_bwd_dots.argtypes = [vp] * 11 + [i32] * 6 + [f32, i32, vp]
+    lib.qk_layerwise_norm_rope_bwd.restype = i32
+    lib.qk_layerwise_norm_rope_bwd.argtypes = [vp] * 15 + [i32] * 8 + [f32, i32, vp]
     lib.qknr_strerror.restype = ctypes.c_char_p
     lib.qknr_strerror.argtypes = [i32]
     lib.qknr_last_cuda_error.restype = i32
@@ -555,3 +566,244 @@ def prepare_bwd(q, k, gamma_q, gamma_k, pos_ids, rstd_q, rstd_k, dq_out, dk_out,
     keep = (q, k, gamma_q, gamma_k, pos_ids, rstd_q, rstd_k, dq_out, dk_out, dq, dk,
             dgamma_q, dgamma_k)
     return PreparedCall(fn, args, name, keep)
+
+
+# --------------------------------------------------------------------------
+# Layerwise QK-norm under tensor parallelism ("SwiftQK: Fast and
+# Communication-Efficient Tensor Parallelism for Query-Key Normalization",
+# abstract): each rank holds a slice of the heads; the statistic of the full
+# hidden vector is one fp32 per token and tensor, summed over the ranks.
+
+
+def _token_vec(name, t, T, device):
+    if t is None:
+        return torch.empty(T, dtype=torch.float32, device=device)
+    _need_cuda(name, t)
+    if t.dtype != torch.float32 or t.numel() != T:
+        raise ValueError(f"{name} must be float32 with B*S = {T} elements")
+    return t
+
+
+def _lw_inputs(q, k, gamma_q, gamma_k, pos_ids):
+    for n, t in (("q", q), ("k", k), ("gamma_q", gamma_q), ("gamma_k", gamma_k)):
+        _need_cuda(n, t)
+    B, S, Hq, Hkv, D = _shape(q, k)
+    _same_dtype(q, k, gamma_q, gamma_k)
+    if gamma_q.numel() != Hq * D or gamma_k.numel() != Hkv * D:
+        raise ValueError(f"gamma_q / gamma_k must hold Hq*D = {Hq * D} / Hkv*D = {Hkv * D} "
+                         "elements (this rank's slice of the full-hidden weight)")
+    if pos_ids is not None:
+        _need_cuda("pos_ids", pos_ids)
+        if pos_ids.dtype != torch.int32 or tuple(pos_ids.shape) != (B, S):
+            raise ValueError("pos_ids must be int32 [B, S]")
+    return B, S, Hq, Hkv, D
+
+
+def _totals(Hq, Hkv, Hq_total, Hkv_total, group):
+    world = 1
+    if group is not None:
+        import torch.distributed as dist
+        world = dist.get_world_size(group)
+    return (Hq * world if Hq_total is None else int(Hq_total),
+            Hkv * world if Hkv_total is None else int(Hkv_total))
+
+
+def _sharded(q, k, Hq_total, Hkv_total, group) -> bool:
+    """True when some heads live on other ranks (the statistics must be
+    exchanged); False when this rank holds every head (one pass each way)."""
+    if group is not None:
+        import torch.distributed as dist
+        if dist.get_world_size(group) > 1:
+            return True
+    return Hq_total != q.shape[2] or Hkv_total != k.shape[2]
+
+
+def all_reduce_stats(tensors, group=None):
+    """Sum per-token partial statistics over the ranks of ``group`` (NCCL on
+    GPUs, any torch.distributed backend); no-op without a group or with one
+    rank. Both tensors go in one call when they can be viewed as one buffer."""
+    if group is None:
+        return tensors
+    import torch.distributed as dist
+    if dist.get_world_size(group) == 1:
+        return tensors
+    flat = torch.cat([t.reshape(-1) for t in tensors])
+    dist.all_reduce(flat, op=dist.ReduceOp.SUM, group=group)
+    out, off = [], 0
+    for t in tensors:
+        n = t.numel()
+        t.copy_(flat[off:off + n].view_as(t))
+        out.append(t)
+        off += n
+    return out
+
+
+def qk_layerwise_stats(q, k, *, sumsq_q=None, sumsq_k=None, stream=None):
+    """Per-token partial sums of squares over this rank's heads (C
+    ``qk_layerwise_stats``): fp32 ``(sumsq_q, sumsq_k)``, [B*S] each."""
+    lib = load_library()
+    for n, t in (("q", q), ("k", k)):
+        _need_cuda(n, t)
+    B, S, Hq, Hkv, D = _shape(q, k)
+    _same_dtype(q, k)
+    sumsq_q = _token_vec("sumsq_q", sumsq_q, B * S, q.device)
+    sumsq_k = _token_vec("sumsq_k", sumsq_k, B * S, q.device)
+    st = lib.qk_layerwise_stats(_ptr(q), _ptr(k), _ptr(sumsq_q), _ptr(sumsq_k), B, S, Hq, Hkv,
+                                D, _DTYPES[q.dtype], _stream(stream))
+    if st != QKNR_OK:
+        raise QKNRError(st, "qk_layerwise_stats")
+    return sumsq_q, sumsq_k
+
+
+def qk_layerwise_norm_rope_fwd(q, k, gamma_q, gamma_k, pos_ids, sumsq_q, sumsq_k, *,
+                               rotary_dim: int, theta: float, eps: float, Hq_total: int,
+                               Hkv_total: int, q_out=None, k_out=None, rstd_q=None,
+                               rstd_k=None, stream=None):
+    """Normalise with the all-rank sums of squares and rotate (C
+    ``qk_layerwise_norm_rope_fwd``). Returns ``(q_out, k_out, rstd_q, rstd_k)``,
+    rstd fp32 [B*S]. ``sumsq_q = sumsq_k = None``: this rank holds every
+    head, and the statistic is taken in the same pass."""
+    lib = load_library()
+    B, S, Hq, Hkv, D = _lw_inputs(q, k, gamma_q, gamma_k, pos_ids)
+    T = B * S
+    if sumsq_q is not None or sumsq_k is not None:
+        sumsq_q = _token_vec("sumsq_q", sumsq_q, T, q.device)
+        sumsq_k = _token_vec("sumsq_k", sumsq_k, T, q.device)
+    q_out = torch.empty_like(q) if q_out is None else q_out
+    k_out = torch.empty_like(k) if k_out is None else k_out
+    for n, t in (("q_out", q_out), ("k_out", k_out)):
+        _need_cuda(n, t)
+    if q_out.shape != q.shape or k_out.shape != k.shape or q_out.dtype != q.dtype \
+            or k_out.dtype != q.dtype:
+        raise ValueError("q_out / k_out must match q / k in shape and dtype")
+    rstd_q = _token_vec("rstd_q", rstd_q, T, q.device)
+    rstd_k = _token_vec("rstd_k", rstd_k, T, q.device)
+    st = lib.qk_layerwise_norm_rope_fwd(
+        _ptr(q), _ptr(k), _ptr(gamma_q), _ptr(gamma_k), _ptr(pos_ids), _ptr(sumsq_q),
+        _ptr(sumsq_k), _ptr(q_out), _ptr(k_out), _ptr(rstd_q), _ptr(rstd_k), B, S, Hq, Hkv,
+        int(Hq_total), int(Hkv_total), D, int(rotary_dim), float(theta), float(eps),
+        _DTYPES[q.dtype], _stream(stream))
+    if st != QKNR_OK:
+        raise QKNRError(st, "qk_layerwise_norm_rope_fwd")
+    return q_out, k_out, rstd_q, rstd_k
+
+
+def qk_layerwise_bwd_dots(q, k, gamma_q, gamma_k, pos_ids, rstd_q, rstd_k, dq_out, dk_out, *,
+                          rotary_dim: int, theta: float, dot_q=None, dot_k=None, stream=None):
+    """Per-token partial sums of (g gamma) . (x rstd) over this rank's heads,
+    g the un-rotated upstream gradient (C ``qk_layerwise_bwd_dots``)."""
+    lib = load_library()
+    B, S, Hq, Hkv, D = _lw_inputs(q, k, gamma_q, gamma_k, pos_ids)
+    T = B * S
+    for n, t, ref in (("dq_out", dq_out, q), ("dk_out", dk_out, k)):
+        _need_cuda(n, t)
+        if t.shape != ref.shape or t.dtype != ref.dtype:
+            raise ValueError(f"{n} must match its input in shape and dtype")
+    rstd_q = _token_vec("rstd_q", rstd_q, T, q.device)
+    rstd_k = _token_vec("rstd_k", rstd_k, T, q.device)
+    dot_q = _token_vec("dot_q", dot_q, T, q.device)
+    dot_k = _token_vec("dot_k", dot_k, T, q.device)
+    st = lib.qk_layerwise_bwd_dots(
+        _ptr(q), _ptr(k), _ptr(gamma_q), _ptr(gamma_k), _ptr(pos_ids), _ptr(rstd_q),
+        _ptr(rstd_k), _ptr(dq_out), _ptr(dk_out), _ptr(dot_q), _ptr(dot_k), B, S, Hq, Hkv, D,
+        int(rotary_dim), float(theta), _DTYPES[q.dtype], _stream(stream))
+    if st != QKNR_OK:
+        raise QKNRError(st, "qk_layerwise_bwd_dots")
+    return dot_q, dot_k
+
+
+def qk_layerwise_norm_rope_bwd(q, k, gamma_q, gamma_k, pos_ids, rstd_q, rstd_k, dq_out, dk_out,
+                               dot_q, dot_k, *, rotary_dim: int, theta: float, Hq_total: int,
+                               Hkv_total: int, dq=None, dk=None, dgamma_q=None, dgamma_k=None,
+                               need_dgamma: bool = True, stream=None):
+    """dq, dk and this rank's dgamma slices from the all-rank dot sums (C
+    ``qk_layerwise_norm_rope_bwd``). Returns ``(dq, dk, dgamma_q, dgamma_k)``;
+    dgamma fp32 [Hq*D] / [Hkv*D], or None without ``need_dgamma``.
+    ``dot_q = dot_k = None``: this rank holds every head, and the dots are
+    taken in the same pass."""
+    lib = load_library()
+    B, S, Hq, Hkv, D = _lw_inputs(q, k, gamma_q, gamma_k, pos_ids)
+    T = B * S
+    for n, t, ref in (("dq_out", dq_out, q), ("dk_out", dk_out, k)):
+        _need_cuda(n, t)
+        if t.shape != ref.shape or t.dtype != ref.dtype:
+            raise ValueError(f"{n} must match its input in shape and dtype")
+    for n, t in (("rstd_q", rstd_q), ("rstd_k", rstd_k), ("dot_q", dot_q), ("dot_k", dot_k)):
+        _token_vec(n, t, T, q.device) if t is not None else None
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    for n, t, ref in (("dq", dq, q), ("dk", dk, k)):
+        _need_cuda(n, t)
+        if t.shape != ref.shape or t.dtype != ref.dtype:
+            raise ValueError(f"{n} must match its input in shape and dtype")
+    if need_dgamma:
+        dgamma_q = torch.empty(Hq * D, dtype=torch.float32, device=q.device) \
+            if dgamma_q is None else dgamma_q
+        dgamma_k = torch.empty(Hkv * D, dtype=torch.float32, device=q.device) \
+            if dgamma_k is None else dgamma_k
+        for n, t, m in (("dgamma_q", dgamma_q, Hq * D), ("dgamma_k", dgamma_k, Hkv * D)):
+            _need_cuda(n, t)
+            if t.dtype != torch.float32 or t.numel() != m:
+                raise ValueError(f"{n} must be float32 with {m} elements")
+    st = lib.qk_layerwise_norm_rope_bwd(
+        _ptr(q), _ptr(k), _ptr(gamma_q), _ptr(gamma_k), _ptr(pos_ids), _ptr(rstd_q),
+        _ptr(rstd_k), _ptr(dq_out), _ptr(dk_out), _ptr(dot_q), _ptr(dot_k), _ptr(dq), _ptr(dk),
+        _ptr(dgamma_q if need_dgamma else None), _ptr(dgamma_k if need_dgamma else None),
+        B, S, Hq, Hkv, int(Hq_total), int(Hkv_total), D, int(rotary_dim), float(theta),
+        _DTYPES[q.dtype], _stream(stream))
+    if st != QKNR_OK:
+        raise QKNRError(st, "qk_layerwise_norm_rope_bwd")
+    return dq, dk, (dgamma_q if need_dgamma else None), (dgamma_k if need_dgamma else None)
+
+
+class QKLayerwiseNormRoPE(torch.autograd.Function):
+    """Autograd wrapper of the layerwise path: stats -> sum over ``group``
+    -> normalise and rotate; backward: dots -> sum over ``group`` -> dx and
+    dgamma. The gradients of gamma are this rank's slices (they are not
+    reduced over the group: each rank owns its slice)."""
+
+    @staticmethod
+    def forward(ctx, q, k, gamma_q, gamma_k, pos_ids, rotary_dim, theta, eps, Hq_total,
+                Hkv_total, group):
+        sq = sk = None
+        if _sharded(q, k, Hq_total, Hkv_total, group):
+            sq, sk = qk_layerwise_stats(q, k)
+            all_reduce_stats([sq, sk], group)
+        qo, ko, rq, rk = qk_layerwise_norm_rope_fwd(
+            q, k, gamma_q, gamma_k, pos_ids, sq, sk, rotary_dim=rotary_dim, theta=theta, eps=eps,
+            Hq_total=Hq_total, Hkv_total=Hkv_total)
+        ctx.save_for_backward(q, k, gamma_q, gamma_k, rq, rk)
+        ctx.cfg = (pos_ids, rotary_dim, theta, Hq_total, Hkv_total, group)
+        return qo, ko
+
+    @staticmethod
+    def backward(ctx, dq_out, dk_out):
+        q, k, gq, gk, rq, rk = ctx.saved_tensors
+        pos_ids, R, theta, Hqt, Hkvt, group = ctx.cfg
+        dq_out, dk_out = dq_out.contiguous(), dk_out.contiguous()
+        pq = pk = None
+        if _sharded(q, k, Hqt, Hkvt, group):
+            pq, pk = qk_layerwise_bwd_dots(q, k, gq, gk, pos_ids, rq, rk, dq_out, dk_out,
+                                           rotary_dim=R, theta=theta)
+            all_reduce_stats([pq, pk], group)
+        need = ctx.needs_input_grad[2] or ctx.needs_input_grad[3]
+        dq, dk, dgq, dgk = qk_layerwise_norm_rope_bwd(
+            q, k, gq, gk, pos_ids, rq, rk, dq_out, dk_out, pq, pk, rotary_dim=R, theta=theta,
+            Hq_total=Hqt, Hkv_total=Hkvt, need_dgamma=need)
+        if need:
+            dgq, dgk = dgq.view_as(gq).to(gq.dtype), dgk.view_as(gk).to(gk.dtype)
+        return dq, dk, dgq, dgk, None, None, None, None, None, None, None
+
+
+def qk_layerwise_norm_rope(q, k, gamma_q, gamma_k, pos_ids=None, *, rotary_dim: int,
+                           theta: float, eps: float, Hq_total: Optional[int] = None,
+                           Hkv_total: Optional[int] = None, group=None):
+    """Layerwise QK-RMSNorm + RoPE with autograd. q, k hold this rank's
+    heads; gamma_q / gamma_k this rank's [Hq*D] / [Hkv*D] slices of the
+    full-hidden weights. The head totals default to the local counts times
+    the group size (an even split)."""
+    B, S, Hq, Hkv, D = _shape(q, k)
+    Hqt, Hkvt = _totals(Hq, Hkv, Hq_total, Hkv_total, group)
+    return QKLayerwiseNormRoPE.apply(q.contiguous(), k.contiguous(), gamma_q.contiguous(),
+                                     gamma_k.contiguous(), pos_ids, rotary_dim, theta, eps, Hqt,
+                                     Hkvt, group)

@@ -16,8 +16,9 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libqknr.so")
-SOURCES = [os.path.join(CSRC, "qknr_api.cu")]
+SOURCES = [os.path.join(CSRC, "qknr_api.cu"), os.path.join(CSRC, "qknr_layerwise.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, "qknr_kernels.cuh"),
+                  os.path.join(CSRC, "qknr_pipe.cuh"),
                   os.path.join(INCLUDE, "qknr.h")]
 
 NVCC_FLAGS = [

@@ -12,14 +12,17 @@
 #include <cstdlib>
 
 namespace qknr {
-namespace {
 
 thread_local int g_last_cuda_error = 0;
 
+// Records the CUDA error behind a QKNR_ERR_CUDA (every entry point of the
+// library, in either source file, reports through here).
 qknr_status cuda_fail(cudaError_t e) {
     g_last_cuda_error = (int)e;
     return QKNR_ERR_CUDA;
 }
+
+namespace {
 
 bool aligned(const void *p, uintptr_t a) { return ((uintptr_t)p % a) == 0; }
 

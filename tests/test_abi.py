@@ -220,3 +220,53 @@ def test_layernorm_entries_validate_like_rmsnorm(lib):
     assert lib.qk_layernorm_rope_bwd(P(1), P(2), P(3), P(4), None, P(7), P(8), P(9), P(10),
                                      P(9, 16), P(12), P(13), P(14), 2, 8, 4, 2, 64, 64, 1e4,
                                      1e-6, BF16, None) == INVALID
+
+
+def test_layerwise_validation(lib):
+    def stats(D=64, q=P(1), sq=P(7), sk=P(8), Hq=4):
+        return lib.qk_layerwise_stats(q, P(2), sq, sk, 2, 8, Hq, 2, D, BF16, None)
+
+    assert stats(D=63) == INVALID
+    assert stats(D=512) == UNSUP
+    assert stats(q=None) == INVALID
+    assert stats(sq=P(7, 2)) == ALIGN
+    assert stats(sk=P(7, 32)) == INVALID            # the two sums overlap
+    assert stats(sq=P(1, 64)) == INVALID            # a sum written over q
+
+    def fwd(Hq_total=8, Hkv_total=4, qo=P(5), rq=P(9), eps=1e-6, R=64):
+        return lib.qk_layerwise_norm_rope_fwd(P(1), P(2), P(3), P(4), None, P(7), P(8), qo,
+                                              P(6), rq, P(10), 2, 8, 4, 2, Hq_total, Hkv_total,
+                                              64, R, 1e4, eps, BF16, None)
+
+    assert fwd(Hq_total=3) == INVALID               # total below the local head count
+    assert fwd(Hkv_total=1) == INVALID
+    assert fwd(eps=-1.0) == INVALID
+    assert fwd(R=8) == UNSUP
+    assert fwd(qo=P(5, 8)) == ALIGN
+    assert fwd(qo=P(1, 256)) == INVALID             # q_out partly over q
+    assert fwd(rq=P(7)) == INVALID                  # rstd written over the sums
+    assert fwd(rq=None) == INVALID
+    # no sums: only a rank holding every head may take the statistic itself
+    assert lib.qk_layerwise_norm_rope_fwd(P(1), P(2), P(3), P(4), None, None, None, P(5), P(6),
+                                          P(9), P(10), 2, 8, 4, 2, 8, 2, 64, 64, 1e4, 1e-6,
+                                          BF16, None) == INVALID
+
+    def dots(dq=P(11)):
+        return lib.qk_layerwise_bwd_dots(P(1), P(2), P(3), P(4), None, P(7), P(8), dq, P(12),
+                                         P(13), P(14), 2, 8, 4, 2, 64, 64, 1e4, BF16, None)
+
+    assert dots(dq=None) == INVALID
+    assert dots(dq=P(13)) == INVALID                # upstream gradient under dot_q
+
+    def bwd(Hq=4, dgq=P(17), dq=P(15)):
+        return lib.qk_layerwise_norm_rope_bwd(P(1), P(2), P(3), P(4), None, P(7), P(8), P(11),
+                                              P(12), P(13), P(14), dq, P(16), dgq, P(18), 2, 8,
+                                              Hq, 2, 512, 2, 128, 128, 1e4, BF16, None)
+
+    assert bwd(Hq=511) == UNSUP                     # dgamma partials exceed shared memory
+    assert bwd(dq=P(11, 16)) == INVALID             # dq partly over dq_out
+    assert bwd(dgq=P(17, 2)) == ALIGN
+    assert bwd(dq=None) == INVALID
+    assert lib.qk_layerwise_norm_rope_bwd(P(1), P(2), P(3), P(4), None, P(7), P(8), P(11),
+                                          P(12), None, None, P(15), P(16), P(17), P(18), 2, 8,
+                                          4, 2, 4, 4, 128, 128, 1e4, BF16, None) == INVALID

@@ -61,3 +61,68 @@ def test_aggregate_is_whole_job():
     import bench
     assert bench.aggregate_tokens_per_s(4, 1000, 2.0) == pytest.approx(2_000_000.0)
     assert bench.max_over_ranks([1.5, 2.5], 1, torch.device("cpu")) == [1.5, 2.5]
+
+
+def _lw_worker(rank, world, port, out):
+    """One rank of a layerwise (all-heads) QK-norm under tensor parallelism:
+    it holds a slice of the heads, sums squares over its slice, and the
+    binding's exchange sums the per-token partials over the group."""
+    import datetime
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    import numpy as np
+    import workloads
+    import qk_rmsnorm_rope_norm_b200 as qknr
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        inp = workloads.make_inputs("tiny", seed=21, Hq=4, Hkv=2)
+        w = inp.w
+        hq, hk = w.Hq // world, w.Hkv // world
+        q = inp.q[:, :, rank * hq:(rank + 1) * hq].double().numpy()
+        k = inp.k[:, :, rank * hk:(rank + 1) * hk].double().numpy()
+        sq = torch.from_numpy((q ** 2).sum(axis=(2, 3)).reshape(-1).astype(np.float32))
+        sk = torch.from_numpy((k ** 2).sum(axis=(2, 3)).reshape(-1).astype(np.float32))
+        qknr.all_reduce_stats([sq, sk], dist.group.WORLD)
+        totals = qknr._totals(hq, hk, None, None, dist.group.WORLD)
+        out[rank] = (sq.numpy().tolist(), sk.numpy().tolist(), totals)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_layerwise_stats_exchange_two_gloo_ranks():
+    import numpy as np
+    import oracle
+    import workloads
+    world = 2
+    port = _free_port()
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_lw_worker, args=(world, port, out), nprocs=world, start_method="spawn",
+                       join=True)
+    inp = workloads.make_inputs("tiny", seed=21, Hq=4, Hkv=2)
+    w = inp.w
+    T = w.B * w.S
+    m = oracle.positions(None, w.B, w.S)
+    for rank in range(world):
+        sq, sk, totals = out[rank]
+        assert totals == (w.Hq, w.Hkv)
+        # the exchanged statistic gives the oracle's full-hidden inverse RMS
+        for s, x, H in ((sq, inp.q, w.Hq), (sk, inp.k, w.Hkv)):
+            _, r = oracle.get().lw_fwd(x.reshape(T, H, w.D), np.ones(H * w.D), m, 0, w.theta,
+                                       w.eps)
+            got = 1.0 / np.sqrt(np.asarray(s, np.float64) / (H * w.D) + w.eps)
+            assert np.abs(got / r - 1).max() <= H * w.D * 2.0 ** -24
+    assert out[0][0] == out[1][0] and out[0][1] == out[1][1]
+
+
+def test_layerwise_exchange_without_group_is_identity():
+    import qk_rmsnorm_rope_norm_b200 as qknr
+    a, b = torch.arange(4.0), torch.ones(3)
+    ra, rb = qknr.all_reduce_stats([a, b], None)
+    assert ra is a and rb is b and torch.equal(a, torch.arange(4.0))
+    assert qknr._totals(4, 2, None, None, None) == (4, 2)
+    assert qknr._totals(4, 2, 16, 8, None) == (16, 8)

@@ -1,0 +1,260 @@
+"""Layerwise QK-RMSNorm + RoPE under tensor parallelism (the qk_layerwise_*
+entry points) against the oracle's layerwise functions (``lw_fwd`` /
+``lw_bwd``: one statistic per token over all heads, gamma over the full
+hidden vector).
+
+One rank holding every head is checked element by element against the
+oracle. Tensor parallelism is emulated on one GPU: the heads are split into
+W slices ("ranks"), each slice runs stats / dots on its own, the per-token
+partial sums are added (the all-reduce a multi-GPU run makes over NCCL),
+and each slice then normalises its heads; the concatenated outputs and the
+per-slice dgamma must match the oracle on the full tensor. No kernel waits
+on another slice, so this needs one GPU only.
+"""
+import pytest
+import torch
+
+import oracle
+import parity
+import workloads
+import qk_rmsnorm_rope_norm_b200 as qknr
+from qk_rmsnorm_rope_norm_b200 import build as qbuild
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def cuda():
+    assert torch.cuda.is_available(), "the gpu tests need a CUDA device"
+    qbuild.build()
+    qknr.load_library()
+    return torch.device("cuda")
+
+
+def lw_inputs(name, seed=None, **over):
+    inp = workloads.make_inputs(name, seed=seed, **over)
+    gq, gk = workloads.layerwise_gamma(inp.w, 17 if seed is None else seed)
+    return inp, gq, gk
+
+
+def positions_of(inp):
+    w = inp.w
+    return oracle.positions(None if inp.pos is None else inp.pos.numpy(), w.B, w.S)
+
+
+def run_ranks(inp, gq, gk, cuda, world=1, local=False):
+    """fwd + bwd with the heads split into ``world`` even slices; the
+    partial sums of the slices are added on the device between the calls.
+    ``local`` (one slice only): no separate stats / dots calls, the fwd and
+    bwd take the statistics in their own pass. Returns CPU results over all
+    heads (rstd per token)."""
+    w = inp.w
+    assert w.Hq % world == 0 and w.Hkv % world == 0
+    hq, hk, D = w.Hq // world, w.Hkv // world, w.D
+    cfg = dict(rotary_dim=w.rotary_dim, theta=w.theta)
+    pos = None if inp.pos is None else inp.pos.to(cuda)
+    q, k = inp.q.to(cuda), inp.k.to(cuda)
+    dqo, dko = inp.dq_out.to(cuda), inp.dk_out.to(cuda)
+    gqd, gkd = gq.to(cuda), gk.to(cuda)
+    sl = []
+    for r in range(world):
+        sq_, sk_ = slice(r * hq, (r + 1) * hq), slice(r * hk, (r + 1) * hk)
+        sl.append(dict(q=q[:, :, sq_].contiguous(), k=k[:, :, sk_].contiguous(),
+                       dqo=dqo[:, :, sq_].contiguous(), dko=dko[:, :, sk_].contiguous(),
+                       gq=gqd[r * hq * D:(r + 1) * hq * D], gk=gkd[r * hk * D:(r + 1) * hk * D]))
+    assert world == 1 or not local
+    stats = [qknr.qk_layerwise_stats(s["q"], s["k"]) for s in sl]
+    Sq = sum(s[0] for s in stats)
+    Sk = sum(s[1] for s in stats)
+    if local:
+        Sq_in = Sk_in = None
+    else:
+        Sq_in, Sk_in = Sq, Sk
+    fw = [qknr.qk_layerwise_norm_rope_fwd(s["q"], s["k"], s["gq"], s["gk"], pos, Sq_in, Sk_in,
+                                          eps=w.eps, Hq_total=w.Hq, Hkv_total=w.Hkv, **cfg)
+          for s in sl]
+    dots = [qknr.qk_layerwise_bwd_dots(s["q"], s["k"], s["gq"], s["gk"], pos, f[2], f[3],
+                                       s["dqo"], s["dko"], **cfg) for s, f in zip(sl, fw)]
+    Pq = sum(d[0] for d in dots)
+    Pk = sum(d[1] for d in dots)
+    Pq_in, Pk_in = (None, None) if local else (Pq, Pk)
+    bw = [qknr.qk_layerwise_norm_rope_bwd(s["q"], s["k"], s["gq"], s["gk"], pos, f[2], f[3],
+                                          s["dqo"], s["dko"], Pq_in, Pk_in, Hq_total=w.Hq,
+                                          Hkv_total=w.Hkv, **cfg) for s, f in zip(sl, fw)]
+    torch.cuda.synchronize()
+    cat = lambda xs, d: torch.cat(xs, dim=d).cpu()
+    return {"q_out": cat([f[0] for f in fw], 2), "k_out": cat([f[1] for f in fw], 2),
+            "rstd_q": fw[0][2].cpu(), "rstd_k": fw[0][3].cpu(),
+            "rstd_q_all": [f[2].cpu() for f in fw],
+            "dq": cat([b[0] for b in bw], 2), "dk": cat([b[1] for b in bw], 2),
+            "dgamma_q": cat([b[2] for b in bw], 0), "dgamma_k": cat([b[3] for b in bw], 0),
+            "sumsq_q": Sq.cpu(), "dot_q": Pq.cpu()}
+
+
+def check_vs_oracle(inp, gq, gk, got):
+    """Element bounds of parity.py (fp32 1e-5 max-abs; bf16 2e-2 max-abs where
+    |ref| < 4 and one bf16 ulp everywhere); rstd to (H D) 2^-24 relative
+    (an fp32 sum over the whole hidden vector); dgamma to its normwise
+    tolerance."""
+    w = inp.w
+    o = oracle.get()
+    m = positions_of(inp)
+    T = w.B * w.S
+    st_q = parity.Stats(w.dtype, max(w.Hq, 1) * w.D)
+    st_k = parity.Stats(w.dtype, max(w.Hkv, 1) * w.D)
+    dg = {}
+    for name, x, g, dy, st, H in (("q", inp.q, gq, inp.dq_out, st_q, w.Hq),
+                                  ("k", inp.k, gk, inp.dk_out, st_k, w.Hkv)):
+        if H == 0:
+            continue
+        x3 = x.reshape(T, H, w.D)
+        y, r = o.lw_fwd(x3, g, m, w.rotary_dim, w.theta, w.eps)
+        dx, dgr = o.lw_bwd(x3, g, dy.reshape(T, H, w.D), m, w.rotary_dim, w.theta, w.eps)
+        st.elem(f"{name}_out", got[f"{name}_out"].double().numpy().reshape(-1), y.reshape(-1))
+        st.rstd(got[f"rstd_{name}"].double().numpy().reshape(-1), r)
+        st.elem(f"d{name}", got[f"d{name}"].double().numpy().reshape(-1), dx.reshape(-1))
+        dg[f"dgamma_{name}"] = (got[f"dgamma_{name}"].double().numpy(), dgr)
+    st_q.check({k_: v for k_, v in dg.items() if k_ == "dgamma_q"})
+    st_k.check({k_: v for k_, v in dg.items() if k_ == "dgamma_k"})
+
+
+CASES = [
+    ("tiny", dict()),
+    ("tiny", dict(B=3, S=37, Hq=5, Hkv=3, D=24, rotary_dim=16)),
+    ("qwen2.5-0.5b", dict(B=2, S=129)),
+    ("llama3-8b-qknorm", dict(B=1, S=97)),
+    ("partial-rope-64k", dict(S=300)),
+    ("bfd-packed", dict()),
+]
+
+
+@pytest.mark.parametrize("local", [False, True], ids=["two-phase", "one-pass"])
+@pytest.mark.parametrize("name,over", CASES,
+                         ids=[f"{n}-{'-'.join(f'{k}{v}' for k, v in o.items())}"
+                              for n, o in CASES])
+def test_layerwise_one_rank_vs_oracle(cuda, name, over, local):
+    inp, gq, gk = lw_inputs(name, **over)
+    check_vs_oracle(inp, gq, gk, run_ranks(inp, gq, gk, cuda, world=1, local=local))
+
+
+@pytest.mark.parametrize("name,over", [("qwen2.5-0.5b", dict(B=2, S=300)),
+                                       ("llama3-8b-qknorm", dict(B=1, S=150)),
+                                       ("partial-rope-64k", dict(S=211)),
+                                       ("tiny", dict(B=3, S=37, Hq=5, Hkv=3, D=24,
+                                                     rotary_dim=16))])
+def test_layerwise_one_pass_equals_two_phase(cuda, name, over):
+    """The one-pass calls take the statistics with the same lane layout and
+    order as qk_layerwise_stats / qk_layerwise_bwd_dots: bit for bit the same
+    rstd, outputs and dx (dgamma, summed with atomics, to its tolerance)."""
+    inp, gq, gk = lw_inputs(name, **over)
+    two = run_ranks(inp, gq, gk, cuda)
+    one = run_ranks(inp, gq, gk, cuda, local=True)
+    for n in ("q_out", "k_out", "rstd_q", "rstd_k", "dq", "dk"):
+        assert torch.equal(one[n], two[n]), n
+    for n in ("dgamma_q", "dgamma_k"):
+        ref = two[n].double()
+        assert float((one[n].double() - ref).abs().max() / ref.abs().max()) <= 1e-5, n
+
+
+@pytest.mark.parametrize("world", [2, 4, 8])
+def test_layerwise_tp_slices_vs_oracle(cuda, world):
+    inp, gq, gk = lw_inputs("llama3-8b-qknorm", B=2, S=65)
+    got = run_ranks(inp, gq, gk, cuda, world=world)
+    # every slice saved the same statistic (it used the summed totals)
+    for r in got["rstd_q_all"][1:]:
+        assert torch.equal(r, got["rstd_q_all"][0])
+    check_vs_oracle(inp, gq, gk, got)
+
+
+def test_layerwise_tp_matches_one_rank(cuda):
+    # the slices change only the fp32 summation order of the statistics
+    inp, gq, gk = lw_inputs("qwen2.5-0.5b", B=1, S=200, Hq=16, Hkv=4)
+    one = run_ranks(inp, gq, gk, cuda, world=1)
+    two = run_ranks(inp, gq, gk, cuda, world=2)
+    rel = float(((one["sumsq_q"] - two["sumsq_q"]).abs() / one["sumsq_q"]).max())
+    assert rel <= 16 * 64 * 2.0 ** -24
+    for n in ("q_out", "k_out", "dq", "dk"):
+        a, b = one[n].float(), two[n].float()
+        # at most about one bf16 rounding apart
+        assert bool(((a - b).abs() <= 2e-2 + b.abs() * 2.0 ** -7).all()), n
+
+
+def test_layerwise_one_head_is_per_head(cuda):
+    """With one head per tensor the layerwise statistic is the per-head one:
+    the same values as qk_norm_rope_* (to rounding; different kernels)."""
+    inp, _, _ = lw_inputs("llama3-8b-qknorm", B=2, S=50, Hq=1, Hkv=1, dtype="f32")
+    w = inp.w
+    got = run_ranks(inp, inp.gamma_q, inp.gamma_k, cuda)
+    dense = parity.gpu_run(inp)
+    for n in ("q_out", "k_out", "dq", "dk"):
+        assert float((got[n] - dense[n]).abs().max()) <= 1e-5, n
+    for n in ("rstd_q", "rstd_k"):
+        a, b = got[n].reshape(-1), dense[n].reshape(-1)
+        assert float(((a - b).abs() / b).max()) <= w.D * 2.0 ** -24, n
+    for n in ("dgamma_q", "dgamma_k"):
+        ref = dense[n].double()
+        assert float((got[n].double() - ref).abs().max() / ref.abs().max()) <= 1e-5, n
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(4, 0), (0, 4), (33, 1)])
+def test_layerwise_head_counts(cuda, Hq, Hkv):
+    inp, gq, gk = lw_inputs("qwen2.5-0.5b", seed=5, B=2, S=41, Hq=Hq, Hkv=Hkv)
+    got = run_ranks(inp, gq, gk, cuda)
+    check_vs_oracle(inp, gq, gk, got)
+
+
+def test_layerwise_autograd(cuda):
+    inp, gq, gk = lw_inputs("qwen2.5-0.5b", B=2, S=65)
+    w = inp.w
+    q = inp.q.to(cuda).requires_grad_(True)
+    k = inp.k.to(cuda).requires_grad_(True)
+    gqd = gq.to(cuda).requires_grad_(True)
+    gkd = gk.to(cuda).requires_grad_(True)
+    qo, ko = qknr.qk_layerwise_norm_rope(q, k, gqd, gkd, rotary_dim=w.rotary_dim, theta=w.theta,
+                                         eps=w.eps)
+    torch.autograd.backward([qo, ko], [inp.dq_out.to(cuda), inp.dk_out.to(cuda)])
+    got = run_ranks(inp, gq, gk, cuda)
+    assert torch.equal(qo.detach().cpu(), got["q_out"])
+    assert torch.equal(ko.detach().cpu(), got["k_out"])
+    assert torch.equal(q.grad.cpu(), got["dq"]) and torch.equal(k.grad.cpu(), got["dk"])
+    for a, b in ((gqd.grad, got["dgamma_q"]), (gkd.grad, got["dgamma_k"])):
+        ref = b.double()
+        rel = float((a.double().cpu() - ref).abs().max() / ref.abs().max())
+        assert rel <= 1e-2   # dgamma is returned in gamma's dtype (bf16)
+
+
+def test_layerwise_in_place(cuda):
+    inp, gq, gk = lw_inputs("qwen2.5-0.5b", B=1, S=100)
+    w = inp.w
+    ref = run_ranks(inp, gq, gk, cuda)
+    q, k = inp.q.to(cuda), inp.k.to(cuda)
+    gqd, gkd = gq.to(cuda), gk.to(cuda)
+    sq, sk = qknr.qk_layerwise_stats(q, k)
+    qknr.qk_layerwise_norm_rope_fwd(q, k, gqd, gkd, None, sq, sk, rotary_dim=w.rotary_dim,
+                                    theta=w.theta, eps=w.eps, Hq_total=w.Hq, Hkv_total=w.Hkv,
+                                    q_out=q, k_out=k)
+    torch.cuda.synchronize()
+    assert torch.equal(q.cpu(), ref["q_out"]) and torch.equal(k.cpu(), ref["k_out"])
+
+
+def test_layerwise_errors(cuda):
+    inp, gq, gk = lw_inputs("qwen2.5-0.5b", B=1, S=16)
+    w = inp.w
+    q, k = inp.q.to(cuda), inp.k.to(cuda)
+    gqd, gkd = gq.to(cuda), gk.to(cuda)
+    sq, sk = qknr.qk_layerwise_stats(q, k)
+    with pytest.raises(qknr.QKNRError):    # totals below the local head counts
+        qknr.qk_layerwise_norm_rope_fwd(q, k, gqd, gkd, None, sq, sk, rotary_dim=64, theta=1e4,
+                                        eps=1e-6, Hq_total=w.Hq - 1, Hkv_total=w.Hkv)
+    with pytest.raises(ValueError):        # a per-head gamma is not a layerwise one
+        qknr.qk_layerwise_norm_rope_fwd(q, k, gqd[:w.D], gkd, None, sq, sk, rotary_dim=64,
+                                        theta=1e4, eps=1e-6, Hq_total=w.Hq, Hkv_total=w.Hkv)
+    # the backward's dgamma partial sums must fit in shared memory
+    big = torch.zeros(1, 4, 512, 128, dtype=torch.bfloat16, device=cuda)
+    gbig = torch.ones(512 * 128, dtype=torch.bfloat16, device=cuda)
+    r = torch.ones(4, device=cuda)
+    with pytest.raises(qknr.QKNRError) as e:
+        qknr.qk_layerwise_norm_rope_bwd(big, big[:, :, :0], gbig, gbig[:0], None, r, r, big,
+                                        big[:, :, :0].contiguous(), r, r, rotary_dim=128,
+                                        theta=1e4, Hq_total=512, Hkv_total=0)
+    assert e.value.status == qknr.QKNR_ERR_UNSUPPORTED

@@ -263,6 +263,17 @@ def make_inputs(w: Workload | str, seed: Optional[int] = None,
                   lengths, rows)
 
 
+def layerwise_gamma(w: Workload, seed: int) -> tuple:
+    """Full-hidden weights of the layerwise (all-heads) QK-norm: gamma_q
+    [Hq*D], gamma_k [Hkv*D], each ``1 + 0.1 * N(0, 1)`` drawn in float32 from
+    ``default_rng([seed, 2])`` (q first) and rounded once to the I/O dtype."""
+    rng = np.random.default_rng([seed, 2])
+    td = w.torch_dtype
+    gq = (1.0 + 0.1 * rng.standard_normal(w.Hq * w.D)).astype(np.float32)
+    gk = (1.0 + 0.1 * rng.standard_normal(w.Hkv * w.D)).astype(np.float32)
+    return torch.from_numpy(gq).to(td), torch.from_numpy(gk).to(td)
+
+
 def contract_bytes(w: Workload, with_pos: bool = False) -> dict:
     """Minimum HBM bytes each direction must move (per launch).
 
