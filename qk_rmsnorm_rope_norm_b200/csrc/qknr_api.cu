@@ -756,6 +756,10 @@ extern "C" const char *qknr_strerror(qknr_status s) {
 
 extern "C" int qknr_last_cuda_error(void) { return g_last_cuda_error; }
 
+namespace qknr {
+int lw_pipeline_error(int reset);  // the layerwise kernels' flag, same bits
+}
+
 extern "C" int qknr_pipeline_error(int reset) {
     unsigned int v = 0;
     if (cudaMemcpyFromSymbol(&v, qknr::g_qknr_pipe_error, sizeof(v)) != cudaSuccess) return -1;
@@ -764,5 +768,7 @@ extern "C" int qknr_pipeline_error(int reset) {
         if (cudaMemcpyToSymbol(qknr::g_qknr_pipe_error, &zero, sizeof(zero)) != cudaSuccess)
             return -1;
     }
-    return (int)v;
+    const int lw = qknr::lw_pipeline_error(reset);
+    if (lw < 0) return -1;
+    return (int)(v | (unsigned int)lw);
 }

@@ -25,6 +25,7 @@
 #include "qknr_kernels.cuh"
 
 #include <cstdint>
+#include <cstdlib>
 
 namespace qknr {
 
@@ -349,6 +350,453 @@ __global__ void __launch_bounds__(kThreads) qknr_lw_bwd_kernel(const LwArgs a) {
     }
 }
 
+// ------------------------------------------------------------------------
+// Pipelined kernels. One producer warp streams stages of TT whole tokens
+// (their Q rows, K rows and, backward, the upstream gradients: each one
+// contiguous range) into a shared-memory ring with 1-D bulk copies and
+// fills the stage's (cos, sin) table; G * NTG consumer warps (at most
+// kLwCWMax, chosen per shape so that every warp owns the same number of
+// head blocks) share each stage. Consumer warp w owns head block set
+// {wb + G nb} (a block is the SLOTS rows one warp covers at once) of token
+// group tg (tokens tg, tg + NTG, ...), so
+// the rows, gamma elements and dgamma sums a lane touches are the same for
+// the whole kernel: dgamma is summed in registers and added to global
+// memory once per lane at the end. Per-token sums over all heads are
+// reduced across the G warps of a token through a small shared table and a
+// per-stage barrier, in a fixed order, so the one-pass and the two-phase
+// calls add the same terms in the same order.
+constexpr int kLwCWMax = 15;                   // consumer warps at most (+1: 16 warps, 128 registers)
+constexpr int kLwThreadsMax = (kLwCWMax + 1) * 32;  // + the producer warp
+constexpr int kLwNBMax = 2;                    // head blocks one consumer warp may own
+constexpr int kLwMaxStages = 4;
+constexpr int kLwStageTarget = 48 * 1024;
+constexpr int kLwRingBytes = 200 * 1024;
+constexpr int kMaxTileTokensLw = 32;
+constexpr int kLwSmemBytes = 220 * 1024;       // dynamic shared memory at most
+constexpr long long kLwWaitCycles = 4000000000ll;  // ~2 s per wait at 1.9 GHz
+
+enum LwMode { kLwStats = 0, kLwFwd = 1, kLwDots = 2, kLwBwd = 3 };
+
+// Sticky error flag of the pipelined layerwise kernels (bit 0: a wait gave
+// up, the launch's results are then incomplete; bit 1: shared memory not
+// aligned for bulk copies, nothing computed).
+__device__ unsigned int g_lw_error;
+
+struct LwGeom {
+    int TT, NS, stage_bytes;
+    int off_k, off_dq, off_dk, off_cs;  // sections of a stage (Q rows at 0)
+    int off_sc;                         // stage: per-token scalars float4 {rq, rk, sq, sk}
+    int off_parts;                      // per-token partial sums [NS][TT][G] float2
+    int off_gamma;                      // gamma_q then gamma_k rows, I/O dtype
+    int G, NTG, HB;                     // warps per token, token groups, head blocks
+    int64_t tpc;                        // tokens per CTA (a multiple of TT)
+};
+
+__device__ __forceinline__ uint32_t lw_smem_u32(const void *p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void lw_bar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void lw_bar_expect(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void lw_bar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool lw_bar_test(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(20000u)
+        : "memory");
+    return ok != 0;
+}
+// Wait for the phase of parity `parity`, for at most kLwWaitCycles; false
+// (with the error flag set) if it never completes.
+__device__ __forceinline__ bool lw_wait(uint32_t bar, uint32_t parity) {
+    if (lw_bar_test(bar, parity)) return true;
+    const long long c0 = clock64();
+    uint32_t nap = 32;
+#pragma unroll 1
+    for (uint32_t n = 1;; ++n) {
+        if (lw_bar_test(bar, parity)) return true;
+        if (n > 2) {
+            __nanosleep(nap);
+            nap = nap < 256 ? nap * 2 : 256;
+        }
+        if ((n & 255u) == 0 && clock64() - c0 > kLwWaitCycles) {
+            atomicOr(&g_lw_error, 1u);
+            return false;
+        }
+    }
+}
+// Bulk copy global -> shared (dst, src, bytes multiples of 16), counted in
+// bytes on `bar`; the rows are read once, so they may leave L2 first.
+__device__ __forceinline__ void lw_bulk(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar,
+                                        uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1], %2, [%3], %4;" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(bar), "l"(policy)
+        : "memory");
+}
+__device__ __forceinline__ uint64_t lw_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ void lw_st_stream(void *p, const Vec16 &v) {
+    __stcs(reinterpret_cast<uint4 *>(p), make_uint4(v.w[0], v.w[1], v.w[2], v.w[3]));
+}
+
+// Stage row of token j, head h (local Q heads, then K heads) in section
+// `q0` (Q rows) / `k0` (K rows).
+__device__ __forceinline__ const unsigned char *stage_row(const unsigned char *q0,
+                                                          const unsigned char *k0, int j, int h,
+                                                          int Hq, int Hkv, int rowb) {
+    return h < Hq ? q0 + (j * Hq + h) * rowb : k0 + (j * Hkv + (h - Hq)) * rowb;
+}
+
+template <typename T, int LPR, int MODE>
+__global__ void __launch_bounds__(kLwThreadsMax, 1)
+    qknr_lw_pipe_kernel(const LwArgs a, const LwGeom g) {
+    using IO = Io<T>;
+    constexpr int V = IO::V, SLOTS = 32 / LPR, E = (int)sizeof(T);
+    constexpr bool kDy = MODE == kLwDots || MODE == kLwBwd;
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ uint64_t s_step[kMaxHalf];      // fixed-point angle step per rotary pair
+    __shared__ int32_t s_pos[kMaxTileTokensLw];  // producer: positions of the stage's tokens
+    const int half = a.R >> 1;
+    const int nthr = blockDim.x, ncw = g.G * g.NTG;  // consumer warps; the producer is warp ncw
+    for (int i = threadIdx.x; i < half; i += nthr) s_step[i] = turn_step(i, a.R, a.theta);
+    const uint32_t bar0 = lw_smem_u32(smem);  // full[NS], empty[NS], parts[NS]
+    if (bar0 & 127u) {  // bulk copies need 16-byte aligned stages: compute nothing
+        if (threadIdx.x == 0) atomicOr(&g_lw_error, 2u);
+        return;
+    }
+    unsigned char *ring = smem + 128;
+    float2 *parts_all = reinterpret_cast<float2 *>(smem + g.off_parts);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t t_lo = (int64_t)blockIdx.x * g.tpc;
+    const int64_t t_hi = min(a.T, t_lo + g.tpc);
+    const int ntiles = t_hi > t_lo ? (int)((t_hi - t_lo + g.TT - 1) / g.TT) : 0;
+    const int H = a.Hq + a.Hkv, rowb = a.D * E;
+    unsigned char *s_gamma = smem + g.off_gamma;  // every CTA reads the weights once
+    if (MODE != kLwStats) {  // (the statistics alone take no weights: gq, gk unset)
+        const int nq = a.Hq * rowb / 16, nk = a.Hkv * rowb / 16;
+        for (int i = threadIdx.x; i < nq + nk; i += nthr) {
+            const Vec16 v = i < nq ? ld16((const char *)a.gq + 16 * i)
+                                   : ld16((const char *)a.gk + 16 * (i - nq));
+            st16(s_gamma + 16 * i, v);
+        }
+    }
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < g.NS; ++s) {
+            lw_bar_init(bar0 + 8 * s, 32);                   // the producer warp's lanes
+            lw_bar_init(bar0 + 8 * (g.NS + s), ncw);       // one per consumer warp
+            lw_bar_init(bar0 + 8 * (2 * g.NS + s), ncw);   // one per consumer warp
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+
+    if (warp == ncw) {
+        // ---------------------------------------------------------- producer
+        const uint64_t pol = lw_evict_first();
+        int issued = 0;
+        for (int i = 0; i < ntiles; ++i) {
+            const int s = i % g.NS;
+            const uint32_t ph = (uint32_t)(i / g.NS) & 1u;
+            if (i >= g.NS && !lw_wait(bar0 + 8 * (g.NS + s), ph ^ 1u)) break;
+            const int64_t t0 = t_lo + (int64_t)i * g.TT;
+            const int na = (int)min((int64_t)g.TT, t_hi - t0);
+            unsigned char *st = ring + (size_t)s * g.stage_bytes;
+            const uint32_t full = bar0 + 8 * s;
+            if (lane == 0) {
+                const uint32_t bq = (uint32_t)(na * a.Hq * rowb);
+                const uint32_t bk = (uint32_t)(na * a.Hkv * rowb);
+                lw_bar_expect(full, (kDy ? 2u : 1u) * (bq + bk));
+                if (bq) lw_bulk(lw_smem_u32(st), (const char *)a.q + t0 * a.Hq * rowb, bq, full, pol);
+                if (bk)
+                    lw_bulk(lw_smem_u32(st + g.off_k), (const char *)a.k + t0 * a.Hkv * rowb, bk,
+                            full, pol);
+                if (kDy && bq)
+                    lw_bulk(lw_smem_u32(st + g.off_dq), (const char *)a.dqo + t0 * a.Hq * rowb, bq,
+                            full, pol);
+                if (kDy && bk)
+                    lw_bulk(lw_smem_u32(st + g.off_dk), (const char *)a.dko + t0 * a.Hkv * rowb, bk,
+                            full, pol);
+            }
+            {
+                // per-token scalars the consumers need: saved rstd (backward),
+                // all-rank totals (second phase of a sharded call)
+                const bool totals = (MODE == kLwFwd || MODE == kLwBwd) &&
+                                    !(a.sq == nullptr && a.sk == nullptr);
+                if (lane < na && (kDy || totals)) {
+                    const int64_t t = t0 + lane;
+                    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (kDy) {
+                        v.x = a.Hq ? a.rq[t] : 0.f;
+                        v.y = a.Hkv ? a.rk[t] : 0.f;
+                    }
+                    if (totals) {
+                        v.z = a.Hq ? a.sq[t] : 0.f;
+                        v.w = a.Hkv ? a.sk[t] : 0.f;
+                    }
+                    reinterpret_cast<float4 *>(st + g.off_sc)[lane] = v;
+                }
+            }
+            if (MODE != kLwStats && half > 0) {
+                // positions (the given ids, else s within the batch row), then
+                // the (cos, sin) table of the stage, one angle per lane at a time
+                if (lane < na) {
+                    const int64_t t = t0 + lane;
+                    s_pos[lane] = a.pos ? a.pos[t] : (int32_t)(t % a.S);
+                }
+                __syncwarp();
+                float2 *cs = reinterpret_cast<float2 *>(st + g.off_cs);
+                for (int idx = lane; idx < na * half; idx += 32) {
+                    const int j = idx / half, i2 = idx - j * half;
+                    cs[idx] = rope_cos_sin_fixed(s_pos[j], s_step[i2]);
+                }
+                __syncwarp();
+            }
+            lw_bar_arrive(full);
+            ++issued;
+        }
+        // leave only once every copy issued has landed
+        for (int i = max(0, issued - g.NS); i < issued; ++i)
+            if (!lw_wait(bar0 + 8 * (i % g.NS), (uint32_t)(i / g.NS) & 1u)) break;
+        return;
+    }
+
+    // -------------------------------------------------------------- consumers
+    const int tg = warp / g.G, wb = warp % g.G;
+    const Lane<LPR, V> L(lane, a.D, a.R);
+    const Lane<LPR, V> Ls(lane, a.D, 0);  // layout of the sums of squares
+    const int offA = L.eA * E, offB = L.eB * E;
+    const int offSA = Ls.eA * E, offSB = Ls.eB * E;
+    const bool local = (MODE == kLwFwd || MODE == kLwBwd) && a.sq == nullptr && a.sk == nullptr;
+    const bool need_parts = MODE == kLwStats || MODE == kLwDots || local;
+    float acc[kLwNBMax][2 * V];
+#pragma unroll
+    for (int nb = 0; nb < kLwNBMax; ++nb)
+#pragma unroll
+        for (int e = 0; e < 2 * V; ++e) acc[nb][e] = 0.f;
+
+    for (int i = 0; i < ntiles; ++i) {
+        const int s = i % g.NS;
+        const uint32_t ph = (uint32_t)(i / g.NS) & 1u;
+        if (!lw_wait(bar0 + 8 * s, ph)) break;
+        const int64_t t0 = t_lo + (int64_t)i * g.TT;
+        const int na = (int)min((int64_t)g.TT, t_hi - t0);
+        const unsigned char *st = ring + (size_t)s * g.stage_bytes;
+        const unsigned char *xq = st, *xk = st + g.off_k;
+        const unsigned char *dq0 = st + g.off_dq, *dk0 = st + g.off_dk;
+        const float2 *cs_st = reinterpret_cast<const float2 *>(st + g.off_cs);
+        const float4 *sc = reinterpret_cast<const float4 *>(st + g.off_sc);
+        float2 *parts = parts_all + (size_t)s * g.TT * g.G;
+
+        if (need_parts) {
+            // this warp's share of each token's sums: x^2, or (g gamma).(x r)
+            for (int j = tg; j < na; j += g.NTG) {
+                float rq = 0.f, rk = 0.f;
+                if (kDy) {
+                    const float4 v = sc[j];
+                    rq = v.x;
+                    rk = v.y;
+                }
+                const float2 *cs = cs_st + j * half;
+                float pq = 0.f, pk = 0.f;
+#pragma unroll
+                for (int nb = 0; nb < kLwNBMax; ++nb) {
+                    const int b = wb + nb * g.G;
+                    if (b >= g.HB) break;
+                    const int h = b * SLOTS + L.slot;
+                    if (!(L.on && h < H)) continue;
+                    const bool isq = h < a.Hq;
+                    const unsigned char *row = stage_row(xq, xk, j, h, a.Hq, a.Hkv, rowb);
+                    float p = 0.f;
+                    if (!kDy) {
+                        const Vec16 xa = ld16(row + offSA), xb = ld16(row + offSB);
+#pragma unroll
+                        for (int k2 = 0; k2 < V / 2; ++k2) {
+                            const float2 va = IO::get2(xa, k2), vb = IO::get2(xb, k2);
+                            p = fmaf(va.x, va.x, p); p = fmaf(va.y, va.y, p);
+                            p = fmaf(vb.x, vb.x, p); p = fmaf(vb.y, vb.y, p);
+                        }
+                    } else {
+                        const unsigned char *drow = stage_row(dq0, dk0, j, h, a.Hq, a.Hkv, rowb);
+                        const unsigned char *grow = s_gamma + h * rowb;
+                        const Vec16 xa = ld16(row + offA), xb = ld16(row + offB);
+                        const Vec16 da = ld16(drow + offA), db = ld16(drow + offB);
+                        const Vec16 ga = ld16(grow + offA), gb = ld16(grow + offB);
+#pragma unroll
+                        for (int k2 = 0; k2 < V / 2; ++k2) {
+                            const float2 va = IO::get2(xa, k2), vb = IO::get2(xb, k2);
+                            const float2 ea = IO::get2(da, k2), eb = IO::get2(db, k2);
+                            const float2 wa = IO::get2(ga, k2), wb2 = IO::get2(gb, k2);
+#pragma unroll
+                            for (int q = 0; q < 2; ++q) {
+                                const float2 c = lane_cs(cs, L.rot, L.eA + 2 * k2 + q);
+                                const float dA = q ? ea.y : ea.x, dB = q ? eb.y : eb.x;
+                                const float gA = fmaf(dA, c.x, dB * c.y);
+                                const float gB = fmaf(dB, c.x, -dA * c.y);
+                                p = fmaf(gA * (q ? wa.y : wa.x), q ? va.y : va.x, p);
+                                p = fmaf(gB * (q ? wb2.y : wb2.x), q ? vb.y : vb.x, p);
+                            }
+                        }
+                        p *= isq ? rq : rk;
+                    }
+                    if (isq) pq += p;
+                    else pk += p;
+                }
+                pq = warp_sum(pq);
+                pk = warp_sum(pk);
+                if (lane == 0) parts[j * g.G + wb] = make_float2(pq, pk);
+            }
+            __syncwarp();
+            const uint32_t pbar = bar0 + 8 * (2 * g.NS + s);
+            if (lane == 0) lw_bar_arrive(pbar);
+            if (!lw_wait(pbar, ph)) break;
+            if ((MODE == kLwStats || MODE == kLwDots) && wb == 0 && lane == 0) {
+                for (int j = tg; j < na; j += g.NTG) {
+                    float2 tot = parts[j * g.G];
+                    for (int w2 = 1; w2 < g.G; ++w2) {
+                        tot.x += parts[j * g.G + w2].x;
+                        tot.y += parts[j * g.G + w2].y;
+                    }
+                    if (a.Hq) a.wq[t0 + j] = tot.x;
+                    if (a.Hkv) a.wk[t0 + j] = tot.y;
+                }
+            }
+        }
+
+        if (MODE == kLwFwd || MODE == kLwBwd) {
+            for (int j = tg; j < na; j += g.NTG) {
+                const int64_t t = t0 + j;
+                float2 tot;
+                if (local) {
+                    tot = parts[j * g.G];
+                    for (int w2 = 1; w2 < g.G; ++w2) {
+                        tot.x += parts[j * g.G + w2].x;
+                        tot.y += parts[j * g.G + w2].y;
+                    }
+                } else {
+                    const float4 v = sc[j];
+                    tot = make_float2(v.z, v.w);
+                }
+                float rq, rk;
+                if (MODE == kLwFwd) {
+                    rq = a.Hq ? rsqrtf(fmaf(tot.x, a.inv_q, a.eps)) : 0.f;
+                    rk = a.Hkv ? rsqrtf(fmaf(tot.y, a.inv_k, a.eps)) : 0.f;
+                    if (wb == 0 && lane == 0) {
+                        if (a.Hq) a.wq[t] = rq;
+                        if (a.Hkv) a.wk[t] = rk;
+                    }
+                } else {
+                    const float4 v = sc[j];
+                    rq = v.x;
+                    rk = v.y;
+                }
+                // backward: dx = r (hh - (x r) P / (H_total D)); nq, nk: factors of x
+                const float nq = -rq * tot.x * a.inv_q, nk = -rk * tot.y * a.inv_k;
+                const float2 *cs = cs_st + j * half;
+#pragma unroll
+                for (int nb = 0; nb < kLwNBMax; ++nb) {
+                    const int b = wb + nb * g.G;
+                    if (b >= g.HB) break;
+                    const int h = b * SLOTS + L.slot;
+                    if (!(L.on && h < H)) continue;
+                    const bool isq = h < a.Hq;
+                    const int hh = isq ? h : h - a.Hq;
+                    const unsigned char *row = stage_row(xq, xk, j, h, a.Hq, a.Hkv, rowb);
+                    const unsigned char *grow = s_gamma + h * rowb;
+                    char *out = (char *)(isq ? a.qo : a.ko) +
+                                ((isq ? t * a.Hq : t * a.Hkv) + hh) * rowb;
+                    const Vec16 xa = ld16(row + offA), xb = ld16(row + offB);
+                    const Vec16 ga = ld16(grow + offA), gb = ld16(grow + offB);
+                    const float r = isq ? rq : rk;
+                    Vec16 oa, ob;
+                    if (MODE == kLwFwd) {
+#pragma unroll
+                        for (int k2 = 0; k2 < V / 2; ++k2) {
+                            const float2 va = IO::get2(xa, k2), vb = IO::get2(xb, k2);
+                            const float2 wa = IO::get2(ga, k2), wb2 = IO::get2(gb, k2);
+                            const int e = 2 * k2;
+                            const float2 c0 = lane_cs(cs, L.rot, L.eA + e);
+                            const float2 c1 = lane_cs(cs, L.rot, L.eA + e + 1);
+                            const float na0 = va.x * wa.x * r, na1 = va.y * wa.y * r;
+                            const float nb0 = vb.x * wb2.x * r, nb1 = vb.y * wb2.y * r;
+                            IO::put2(oa, k2, fmaf(na0, c0.x, -nb0 * c0.y),
+                                     fmaf(na1, c1.x, -nb1 * c1.y));
+                            IO::put2(ob, k2, fmaf(nb0, c0.x, na0 * c0.y),
+                                     fmaf(nb1, c1.x, na1 * c1.y));
+                        }
+                    } else {
+                        const unsigned char *drow = stage_row(dq0, dk0, j, h, a.Hq, a.Hkv, rowb);
+                        const Vec16 da = ld16(drow + offA), db = ld16(drow + offB);
+                        const float nd = isq ? nq : nk;
+#pragma unroll
+                        for (int k2 = 0; k2 < V / 2; ++k2) {
+                            const float2 va = IO::get2(xa, k2), vb = IO::get2(xb, k2);
+                            const float2 ea = IO::get2(da, k2), eb = IO::get2(db, k2);
+                            const float2 wa = IO::get2(ga, k2), wb2 = IO::get2(gb, k2);
+                            float outA[2], outB[2];
+#pragma unroll
+                            for (int q = 0; q < 2; ++q) {
+                                const int e = 2 * k2 + q;
+                                const float2 c = lane_cs(cs, L.rot, L.eA + e);
+                                const float dA = q ? ea.y : ea.x, dB = q ? eb.y : eb.x;
+                                const float xA = q ? va.y : va.x, xB = q ? vb.y : vb.x;
+                                const float gA = fmaf(dA, c.x, dB * c.y);
+                                const float gB = fmaf(dB, c.x, -dA * c.y);
+                                const float hA = gA * (q ? wa.y : wa.x);
+                                const float hB = gB * (q ? wb2.y : wb2.x);
+                                outA[q] = r * fmaf(xA, nd, hA);
+                                outB[q] = r * fmaf(xB, nd, hB);
+                                acc[nb][e] = fmaf(gA * xA, r, acc[nb][e]);
+                                acc[nb][V + e] = fmaf(gB * xB, r, acc[nb][V + e]);
+                            }
+                            IO::put2(oa, k2, outA[0], outA[1]);
+                            IO::put2(ob, k2, outB[0], outB[1]);
+                        }
+                    }
+                    lw_st_stream(out + offA, oa);
+                    lw_st_stream(out + offB, ob);
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) lw_bar_arrive(bar0 + 8 * (g.NS + s));
+    }
+
+    if (MODE == kLwBwd) {
+        // this lane's dgamma sums (fixed rows and elements) into the rank's slice
+#pragma unroll
+        for (int nb = 0; nb < kLwNBMax; ++nb) {
+            const int b = wb + nb * g.G;
+            if (b >= g.HB) break;
+            const int h = b * SLOTS + L.slot;
+            if (!(L.on && h < H)) continue;
+            const bool isq = h < a.Hq;
+            float *dg = isq ? a.dgq : a.dgk;
+            if (!dg) continue;
+            dg += (isq ? h : h - a.Hq) * a.D;
+#pragma unroll
+            for (int e = 0; e < V; ++e) {
+                atomicAdd(dg + L.eA + e, acc[nb][e]);
+                atomicAdd(dg + L.eB + e, acc[nb][V + e]);
+            }
+        }
+    }
+}
+
 int lpr_of(int D, int esz) {
     const int dv2 = D / (2 * (16 / esz));
     int l = 1;
@@ -382,8 +830,93 @@ qknr_status cuda_status() {
 
 enum class LwKernel { kStats, kFwd, kDots, kBwd };
 
+bool simple_kernels_forced() {
+    const char *e = std::getenv("QKNR_SIMPLE_KERNELS");
+    return e && e[0] && e[0] != '0';
+}
+
+// Stage and ring sizes of the pipelined kernels for this shape, or false if
+// the shape does not fit them (the plain-load kernels run instead).
+bool lw_plan(int mode, const LwArgs &a, int esz, int lpr, int sms, LwGeom *g, int *grid,
+             int *smem, int *threads) {
+    const int slots = 32 / lpr, H = a.Hq + a.Hkv;
+    const int HB = (H + slots - 1) / slots;
+    // head blocks per warp, warps per token, token groups: every warp owns
+    // NB blocks (the last one maybe fewer), at most kLwCWMax warps
+    const int NB = (HB + kLwCWMax - 1) / kLwCWMax;
+    if (NB > kLwNBMax) return false;
+    const int G = (HB + NB - 1) / NB;
+    const int NTG = kLwCWMax / G;
+    const bool dy = mode == kLwDots || mode == kLwBwd;
+    const int64_t rowb = (int64_t)a.D * esz;
+    const int64_t xq = (int64_t)a.Hq * rowb, xk = (int64_t)a.Hkv * rowb;  // per token
+    const int64_t csb = mode == kLwStats ? 0 : (int64_t)(a.R / 2) * 8;
+    const int64_t per = (dy ? 2 : 1) * (xq + xk) + csb + 16;  // + the per-token scalars
+    int64_t TT = kLwStageTarget / per;
+    TT = TT > kMaxTileTokensLw ? kMaxTileTokensLw : TT;
+    TT = (TT / NTG) * NTG;
+    if (TT < NTG) TT = NTG;
+    if (TT > kMaxTileTokensLw) return false;
+    const int64_t stage = ((TT * per + 127) / 128) * 128;
+    const int64_t gbytes = ((xq + xk + 127) / 128) * 128;
+    const int64_t budget = kLwSmemBytes - 128 - TT * G * 8 * kLwMaxStages - 128 - gbytes;
+    int64_t NS = (budget < kLwRingBytes ? budget : kLwRingBytes) / stage;
+    if (NS > kLwMaxStages) NS = kLwMaxStages;
+    if (NS < 2) return false;
+    g->TT = (int)TT;
+    g->NS = (int)NS;
+    g->stage_bytes = (int)stage;
+    g->off_k = (int)(TT * xq);
+    g->off_dq = (int)(TT * (xq + xk));
+    g->off_dk = (int)(TT * (2 * xq + xk));
+    g->off_cs = (int)(TT * (dy ? 2 : 1) * (xq + xk));
+    g->off_sc = g->off_cs + (int)(TT * csb);
+    g->off_parts = 128 + (int)(NS * stage);
+    g->off_gamma = g->off_parts + (int)(((NS * TT * G * 8 + 127) / 128) * 128);
+    g->G = G;
+    g->NTG = NTG;
+    g->HB = HB;
+    const int64_t tiles = (a.T + TT - 1) / TT;
+    int64_t nb = tiles < sms ? tiles : sms;
+    const int64_t tiles_per = (tiles + nb - 1) / nb;
+    g->tpc = tiles_per * TT;
+    nb = (a.T + g->tpc - 1) / g->tpc;
+    *grid = (int)nb;
+    *smem = g->off_gamma + (int)gbytes;
+    *threads = (G * NTG + 1) * 32;
+    return true;
+}
+
+template <typename T, int LPR, int MODE>
+qknr_status lw_pipe_launch(const LwArgs &a, const LwGeom &g, int grid, int smem, int threads,
+                           cudaStream_t st) {
+    auto kern = qknr_lw_pipe_kernel<T, LPR, MODE>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return cuda_fail(e);
+    kern<<<grid, threads, smem, st>>>(a, g);
+    return cuda_status();
+}
+
 template <typename T, int LPR>
 qknr_status lw_launch_t(LwKernel which, const LwArgs &a, cudaStream_t st) {
+    if (!simple_kernels_forced()) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        const int mode = which == LwKernel::kStats ? kLwStats
+                         : which == LwKernel::kFwd ? kLwFwd
+                         : which == LwKernel::kDots ? kLwDots
+                                                    : kLwBwd;
+        LwGeom g;
+        int grid, smem, thr;
+        if (lw_plan(mode, a, (int)sizeof(T), LPR, sm_count_of(dev), &g, &grid, &smem, &thr)) {
+            switch (mode) {
+                case kLwStats: return lw_pipe_launch<T, LPR, kLwStats>(a, g, grid, smem, thr, st);
+                case kLwFwd: return lw_pipe_launch<T, LPR, kLwFwd>(a, g, grid, smem, thr, st);
+                case kLwDots: return lw_pipe_launch<T, LPR, kLwDots>(a, g, grid, smem, thr, st);
+                default: return lw_pipe_launch<T, LPR, kLwBwd>(a, g, grid, smem, thr, st);
+            }
+        }
+    }
     int grid, tpw;
     lw_geometry(a.T, &grid, &tpw);
     LwArgs b = a;
@@ -472,6 +1005,22 @@ qknr_status lw_run(LwKernel which, LwArgs a, qknr_dtype dtype, qknr_stream_t str
 }
 
 }  // namespace
+}  // namespace qknr
+
+namespace qknr {
+
+// The pipelined layerwise kernels' error flag (see g_lw_error); -1 if it
+// cannot be read.
+int lw_pipeline_error(int reset) {
+    unsigned int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_lw_error, sizeof(v)) != cudaSuccess) return -1;
+    if (reset && v) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(g_lw_error, &zero, sizeof(zero)) != cudaSuccess) return -1;
+    }
+    return (int)v;
+}
+
 }  // namespace qknr
 
 using namespace qknr;

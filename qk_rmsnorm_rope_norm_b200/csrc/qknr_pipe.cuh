@@ -210,25 +210,6 @@ __device__ __forceinline__ int cs_slot(int P) {
     return W * u + (k + ((u * W) >> 3)) % W;
 }
 
-// Rotary angle in fixed point. F = round(2^64 * frac(omega / 2pi)) is the
-// angle step per position in units of 2^-64 turns, so pos * F mod 2^64 is
-// the angle mod one turn (integer wrap-around does the reduction; negative
-// positions work in two's complement). Its top 32 bits, as a signed turn
-// fraction in [-1/2, 1/2), feed the hardware sin/cos (absolute error
-// ~2^-21 on [-pi, pi]). The error of F (~1e-16 relative) times |pos| < 2^31
-// keeps the angle within ~2.4e-7 rad at the largest positions.
-__device__ __forceinline__ uint64_t turn_step(int i, int R, float theta) {
-    const double w = pow((double)theta, -2.0 * (double)i / (double)R);
-    return __double2ull_rn(w * 0.15915494309189533577 * 18446744073709551616.0);
-}
-__device__ __forceinline__ float2 rope_cos_sin_fixed(int32_t pos, uint64_t F) {
-    const uint32_t p = (uint32_t)pos, flo = (uint32_t)F, fhi = (uint32_t)(F >> 32);
-    const uint32_t hi = __umulhi(p, flo) + p * fhi - (pos < 0 ? flo : 0u);
-    const float turns = (float)(int32_t)hi * 2.3283064365386963e-10f;  // 2^-32
-    float s, c;
-    __sincosf(turns * 6.2831853071795865f, &s, &c);
-    return make_float2(c, s);
-}
 
 // Producers: fill the stage's (cos, sin) table for na tokens. The NW = 32 *
 // NPW producer lanes each own one angle index i and one token group; with

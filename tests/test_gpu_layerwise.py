@@ -4,13 +4,16 @@ entry points) against the oracle's layerwise functions (``lw_fwd`` /
 hidden vector).
 
 One rank holding every head is checked element by element against the
-oracle. Tensor parallelism is emulated on one GPU: the heads are split into
+oracle, for both kernel families (the pipelined kernels, and the plain-load
+kernels that serve shapes the pipeline's shared-memory ring cannot hold). Tensor parallelism is emulated on one GPU: the heads are split into
 W slices ("ranks"), each slice runs stats / dots on its own, the per-token
 partial sums are added (the all-reduce a multi-GPU run makes over NCCL),
 and each slice then normalises its heads; the concatenated outputs and the
 per-slice dgamma must match the oracle on the full tensor. No kernel waits
 on another slice, so this needs one GPU only.
 """
+import os
+
 import pytest
 import torch
 
@@ -29,6 +32,14 @@ def cuda():
     qbuild.build()
     qknr.load_library()
     return torch.device("cuda")
+
+
+@pytest.fixture(params=["pipelined", "plain"])
+def kernels(request):
+    if request.param == "plain":
+        os.environ["QKNR_SIMPLE_KERNELS"] = "1"
+    yield request.param
+    os.environ.pop("QKNR_SIMPLE_KERNELS", None)
 
 
 def lw_inputs(name, seed=None, **over):
@@ -132,7 +143,7 @@ CASES = [
 @pytest.mark.parametrize("name,over", CASES,
                          ids=[f"{n}-{'-'.join(f'{k}{v}' for k, v in o.items())}"
                               for n, o in CASES])
-def test_layerwise_one_rank_vs_oracle(cuda, name, over, local):
+def test_layerwise_one_rank_vs_oracle(cuda, kernels, name, over, local):
     inp, gq, gk = lw_inputs(name, **over)
     check_vs_oracle(inp, gq, gk, run_ranks(inp, gq, gk, cuda, world=1, local=local))
 
@@ -142,7 +153,7 @@ def test_layerwise_one_rank_vs_oracle(cuda, name, over, local):
                                        ("partial-rope-64k", dict(S=211)),
                                        ("tiny", dict(B=3, S=37, Hq=5, Hkv=3, D=24,
                                                      rotary_dim=16))])
-def test_layerwise_one_pass_equals_two_phase(cuda, name, over):
+def test_layerwise_one_pass_equals_two_phase(cuda, kernels, name, over):
     """The one-pass calls take the statistics with the same lane layout and
     order as qk_layerwise_stats / qk_layerwise_bwd_dots: bit for bit the same
     rstd, outputs and dx (dgamma, summed with atomics, to its tolerance)."""
@@ -157,7 +168,7 @@ def test_layerwise_one_pass_equals_two_phase(cuda, name, over):
 
 
 @pytest.mark.parametrize("world", [2, 4, 8])
-def test_layerwise_tp_slices_vs_oracle(cuda, world):
+def test_layerwise_tp_slices_vs_oracle(cuda, kernels, world):
     inp, gq, gk = lw_inputs("llama3-8b-qknorm", B=2, S=65)
     got = run_ranks(inp, gq, gk, cuda, world=world)
     # every slice saved the same statistic (it used the summed totals)
@@ -197,7 +208,7 @@ def test_layerwise_one_head_is_per_head(cuda):
 
 
 @pytest.mark.parametrize("Hq,Hkv", [(4, 0), (0, 4), (33, 1)])
-def test_layerwise_head_counts(cuda, Hq, Hkv):
+def test_layerwise_head_counts(cuda, kernels, Hq, Hkv):
     inp, gq, gk = lw_inputs("qwen2.5-0.5b", seed=5, B=2, S=41, Hq=Hq, Hkv=Hkv)
     got = run_ranks(inp, gq, gk, cuda)
     check_vs_oracle(inp, gq, gk, got)
@@ -258,3 +269,21 @@ def test_layerwise_errors(cuda):
                                         big[:, :, :0].contiguous(), r, r, rotary_dim=128,
                                         theta=1e4, Hq_total=512, Hkv_total=0)
     assert e.value.status == qknr.QKNR_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("B,S", [(1, 1), (1, 3), (2, 5), (3, 41), (1, 4099)])
+def test_layerwise_token_counts(cuda, B, S):
+    # ragged last stages and CTAs with a single partial stage
+    inp, gq, gk = lw_inputs("llama3-8b-qknorm", seed=9, B=B, S=S, Hq=6, Hkv=2)
+    check_vs_oracle(inp, gq, gk, run_ranks(inp, gq, gk, cuda, local=True))
+
+
+def test_layerwise_large_hidden_falls_back(cuda):
+    # 72 heads of 256 fp32 elements per token: too big for the ring; the
+    # plain-load kernels serve it
+    inp, gq, gk = lw_inputs("tiny", seed=2, B=1, S=9, Hq=64, Hkv=8, D=256, rotary_dim=128)
+    check_vs_oracle(inp, gq, gk, run_ranks(inp, gq, gk, cuda, local=True))
+
+
+def test_layerwise_no_pipeline_timeouts(cuda):
+    assert qknr.pipeline_error() == 0
