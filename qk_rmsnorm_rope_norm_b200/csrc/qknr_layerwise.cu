@@ -462,6 +462,32 @@ __device__ __forceinline__ const unsigned char *stage_row(const unsigned char *q
     return h < Hq ? q0 + (j * Hq + h) * rowb : k0 + (j * Hkv + (h - Hq)) * rowb;
 }
 
+__device__ __forceinline__ float2 neg2f(float2 v) { return make_float2(-v.x, -v.y); }
+
+// Token j's sums over all heads: its G per-warp partials added in warp order
+// (the same order wherever a total is formed).
+__device__ __forceinline__ float2 token_total(const float2 *parts, int j, int G) {
+    float2 tot = parts[j * G];
+    for (int w2 = 1; w2 < G; ++w2) {
+        const float2 p = parts[j * G + w2];
+        tot.x += p.x;
+        tot.y += p.y;
+    }
+    return tot;
+}
+
+// A lane's (cos, sin) pairs for elements eA .. eA + V - 1 of token table
+// `tok` (float4 per pair, pair k of unit w at k U + w, U = hp / (V / 2));
+// (1, 1, 0, 0) on lanes past the rotary span.
+template <int V, typename LaneT>
+__device__ __forceinline__ void lane_cs4(float4 (&c)[V / 2], const float4 *tok, const LaneT &L,
+                                         int U) {
+    const int w = L.eA / V;
+#pragma unroll
+    for (int k = 0; k < V / 2; ++k)
+        c[k] = L.rot ? tok[k * U + w] : make_float4(1.f, 1.f, 0.f, 0.f);
+}
+
 template <typename T, int LPR, int MODE>
 __global__ void __launch_bounds__(kLwThreadsMax, 1)
     qknr_lw_pipe_kernel(const LwArgs a, const LwGeom g) {
@@ -559,10 +585,19 @@ __global__ void __launch_bounds__(kLwThreadsMax, 1)
                     s_pos[lane] = a.pos ? a.pos[t] : (int32_t)(t % a.S);
                 }
                 __syncwarp();
-                float2 *cs = reinterpret_cast<float2 *>(st + g.off_cs);
-                for (int idx = lane; idx < na * half; idx += 32) {
-                    const int j = idx / half, i2 = idx - j * half;
-                    cs[idx] = rope_cos_sin_fixed(s_pos[j], s_step[i2]);
+                // pair P of a token: (c_2P, c_2P+1, s_2P, s_2P+1), one float4,
+                // stored at (P mod W) U + P / W (W pairs per lane, U rotating
+                // units) so that the lanes of a row read consecutive entries
+                float4 *cs = reinterpret_cast<float4 *>(st + g.off_cs);
+                constexpr int W = V / 2;
+                const int hp = half >> 1, U = hp / W;
+#pragma unroll 2
+                for (int idx = lane; idx < na * hp; idx += 32) {
+                    const int j = idx / hp, P = idx - j * hp;
+                    const float2 c0 = rope_cos_sin_fixed(s_pos[j], s_step[2 * P]);
+                    const float2 c1 = rope_cos_sin_fixed(s_pos[j], s_step[2 * P + 1]);
+                    const int pw = P / W;
+                    cs[j * hp + (P - pw * W) * U + pw] = make_float4(c0.x, c1.x, c0.y, c1.y);
                 }
                 __syncwarp();
             }
@@ -581,13 +616,15 @@ __global__ void __launch_bounds__(kLwThreadsMax, 1)
     const Lane<LPR, V> Ls(lane, a.D, 0);  // layout of the sums of squares
     const int offA = L.eA * E, offB = L.eB * E;
     const int offSA = Ls.eA * E, offSB = Ls.eB * E;
+    const int hp = half >> 1;  // rotary pairs per token
     const bool local = (MODE == kLwFwd || MODE == kLwBwd) && a.sq == nullptr && a.sk == nullptr;
     const bool need_parts = MODE == kLwStats || MODE == kLwDots || local;
-    float acc[kLwNBMax][2 * V];
+    constexpr int kUA = (MODE == kLwStats || MODE == kLwFwd) ? 4 : 2;  // tokens per partial-sum round
+    float2 acc[kLwNBMax][V];  // dgamma sums: pairs of the A vector, then of the B vector
 #pragma unroll
     for (int nb = 0; nb < kLwNBMax; ++nb)
 #pragma unroll
-        for (int e = 0; e < 2 * V; ++e) acc[nb][e] = 0.f;
+        for (int k = 0; k < V; ++k) acc[nb][k] = make_float2(0.f, 0.f);
 
     for (int i = 0; i < ntiles; ++i) {
         const int s = i % g.NS;
@@ -598,79 +635,93 @@ __global__ void __launch_bounds__(kLwThreadsMax, 1)
         const unsigned char *st = ring + (size_t)s * g.stage_bytes;
         const unsigned char *xq = st, *xk = st + g.off_k;
         const unsigned char *dq0 = st + g.off_dq, *dk0 = st + g.off_dk;
-        const float2 *cs_st = reinterpret_cast<const float2 *>(st + g.off_cs);
+        const float4 *cs_st = reinterpret_cast<const float4 *>(st + g.off_cs);
         const float4 *sc = reinterpret_cast<const float4 *>(st + g.off_sc);
         float2 *parts = parts_all + (size_t)s * g.TT * g.G;
 
         if (need_parts) {
-            // this warp's share of each token's sums: x^2, or (g gamma).(x r)
-            for (int j = tg; j < na; j += g.NTG) {
-                float rq = 0.f, rk = 0.f;
-                if (kDy) {
-                    const float4 v = sc[j];
-                    rq = v.x;
-                    rk = v.y;
-                }
-                const float2 *cs = cs_st + j * half;
-                float pq = 0.f, pk = 0.f;
+            // this warp's share of each token's sums, x^2 or (g gamma).(x r),
+            // kUA tokens per round so that their warp reductions overlap
+            for (int j0 = tg; j0 < na; j0 += kUA * g.NTG) {
+                float vq[kUA], vk[kUA];
 #pragma unroll
-                for (int nb = 0; nb < kLwNBMax; ++nb) {
-                    const int b = wb + nb * g.G;
-                    if (b >= g.HB) break;
-                    const int h = b * SLOTS + L.slot;
-                    if (!(L.on && h < H)) continue;
-                    const bool isq = h < a.Hq;
-                    const unsigned char *row = stage_row(xq, xk, j, h, a.Hq, a.Hkv, rowb);
-                    float p = 0.f;
-                    if (!kDy) {
-                        const Vec16 xa = ld16(row + offSA), xb = ld16(row + offSB);
-#pragma unroll
-                        for (int k2 = 0; k2 < V / 2; ++k2) {
-                            const float2 va = IO::get2(xa, k2), vb = IO::get2(xb, k2);
-                            p = fmaf(va.x, va.x, p); p = fmaf(va.y, va.y, p);
-                            p = fmaf(vb.x, vb.x, p); p = fmaf(vb.y, vb.y, p);
-                        }
-                    } else {
-                        const unsigned char *drow = stage_row(dq0, dk0, j, h, a.Hq, a.Hkv, rowb);
-                        const unsigned char *grow = s_gamma + h * rowb;
-                        const Vec16 xa = ld16(row + offA), xb = ld16(row + offB);
-                        const Vec16 da = ld16(drow + offA), db = ld16(drow + offB);
-                        const Vec16 ga = ld16(grow + offA), gb = ld16(grow + offB);
-#pragma unroll
-                        for (int k2 = 0; k2 < V / 2; ++k2) {
-                            const float2 va = IO::get2(xa, k2), vb = IO::get2(xb, k2);
-                            const float2 ea = IO::get2(da, k2), eb = IO::get2(db, k2);
-                            const float2 wa = IO::get2(ga, k2), wb2 = IO::get2(gb, k2);
-#pragma unroll
-                            for (int q = 0; q < 2; ++q) {
-                                const float2 c = lane_cs(cs, L.rot, L.eA + 2 * k2 + q);
-                                const float dA = q ? ea.y : ea.x, dB = q ? eb.y : eb.x;
-                                const float gA = fmaf(dA, c.x, dB * c.y);
-                                const float gB = fmaf(dB, c.x, -dA * c.y);
-                                p = fmaf(gA * (q ? wa.y : wa.x), q ? va.y : va.x, p);
-                                p = fmaf(gB * (q ? wb2.y : wb2.x), q ? vb.y : vb.x, p);
-                            }
-                        }
-                        p *= isq ? rq : rk;
+                for (int u = 0; u < kUA; ++u) {
+                    const int j = j0 + u * g.NTG;
+                    vq[u] = vk[u] = 0.f;
+                    if (j >= na) continue;
+                    float4 c[V / 2];
+                    float r2q = 0.f, r2k = 0.f;
+                    if (kDy) {
+                        lane_cs4<V>(c, cs_st + j * hp, L, hp / (V / 2));
+                        const float4 sv = sc[j];
+                        r2q = sv.x;
+                        r2k = sv.y;
                     }
-                    if (isq) pq += p;
-                    else pk += p;
+#pragma unroll
+                    for (int nb = 0; nb < kLwNBMax; ++nb) {
+                        const int b = wb + nb * g.G;
+                        if (b >= g.HB) break;
+                        const int h = b * SLOTS + L.slot;
+                        if (!(L.on && h < H)) continue;
+                        const bool isq = h < a.Hq;
+                        const unsigned char *row = stage_row(xq, xk, j, h, a.Hq, a.Hkv, rowb);
+                        float2 p2 = make_float2(0.f, 0.f);
+                        if (!kDy) {
+                            const Vec16 xa = ld16(row + offSA), xb = ld16(row + offSB);
+#pragma unroll
+                            for (int k2 = 0; k2 < V / 2; ++k2) {
+                                const float2 va = IO::get2(xa, k2), vb = IO::get2(xb, k2);
+                                p2 = __ffma2_rn(va, va, p2);
+                                p2 = __ffma2_rn(vb, vb, p2);
+                            }
+                            const float p = p2.x + p2.y;
+                            vq[u] += isq ? p : 0.f;
+                            vk[u] += isq ? 0.f : p;
+                        } else {
+                            const unsigned char *drow = stage_row(dq0, dk0, j, h, a.Hq, a.Hkv, rowb);
+                            const unsigned char *grow = s_gamma + h * rowb;
+                            const Vec16 xa = ld16(row + offA), xb = ld16(row + offB);
+                            const Vec16 da = ld16(drow + offA), db = ld16(drow + offB);
+                            const Vec16 ga = ld16(grow + offA), gb = ld16(grow + offB);
+#pragma unroll
+                            for (int k2 = 0; k2 < V / 2; ++k2) {
+                                const float2 c2 = make_float2(c[k2].x, c[k2].y);
+                                const float2 s2 = make_float2(c[k2].z, c[k2].w);
+                                const float2 ea = IO::get2(da, k2), eb = IO::get2(db, k2);
+                                const float2 gA = __ffma2_rn(ea, c2, __fmul2_rn(eb, s2));
+                                const float2 gB = __ffma2_rn(eb, c2, __fmul2_rn(ea, neg2f(s2)));
+                                p2 = __ffma2_rn(__fmul2_rn(gA, IO::get2(ga, k2)), IO::get2(xa, k2), p2);
+                                p2 = __ffma2_rn(__fmul2_rn(gB, IO::get2(gb, k2)), IO::get2(xb, k2), p2);
+                            }
+                            const float p = (p2.x + p2.y) * (isq ? r2q : r2k);
+                            vq[u] += isq ? p : 0.f;
+                            vk[u] += isq ? 0.f : p;
+                        }
+                    }
                 }
-                pq = warp_sum(pq);
-                pk = warp_sum(pk);
-                if (lane == 0) parts[j * g.G + wb] = make_float2(pq, pk);
+#pragma unroll
+                for (int o = 16; o; o >>= 1)
+#pragma unroll
+                    for (int u = 0; u < kUA; ++u) {
+                        vq[u] += __shfl_xor_sync(0xffffffffu, vq[u], o);
+                        vk[u] += __shfl_xor_sync(0xffffffffu, vk[u], o);
+                    }
+                if (lane == 0) {
+#pragma unroll
+                    for (int u = 0; u < kUA; ++u) {
+                        const int j = j0 + u * g.NTG;
+                        if (j < na) parts[j * g.G + wb] = make_float2(vq[u], vk[u]);
+                    }
+                }
             }
             __syncwarp();
             const uint32_t pbar = bar0 + 8 * (2 * g.NS + s);
             if (lane == 0) lw_bar_arrive(pbar);
             if (!lw_wait(pbar, ph)) break;
-            if ((MODE == kLwStats || MODE == kLwDots) && wb == 0 && lane == 0) {
-                for (int j = tg; j < na; j += g.NTG) {
-                    float2 tot = parts[j * g.G];
-                    for (int w2 = 1; w2 < g.G; ++w2) {
-                        tot.x += parts[j * g.G + w2].x;
-                        tot.y += parts[j * g.G + w2].y;
-                    }
+            if ((MODE == kLwStats || MODE == kLwDots) && warp == 0) {
+                // lane j: token j's total over the G warps, in warp order
+                for (int j = lane; j < na; j += 32) {
+                    const float2 tot = token_total(parts, j, g.G);
                     if (a.Hq) a.wq[t0 + j] = tot.x;
                     if (a.Hkv) a.wk[t0 + j] = tot.y;
                 }
@@ -678,97 +729,99 @@ __global__ void __launch_bounds__(kLwThreadsMax, 1)
         }
 
         if (MODE == kLwFwd || MODE == kLwBwd) {
-            for (int j = tg; j < na; j += g.NTG) {
-                const int64_t t = t0 + j;
-                float2 tot;
+            // per-token totals: lane j holds token j's (j < 32; TT <= 32)
+            float2 my_tot = make_float2(0.f, 0.f);
+            if (lane < na) {
                 if (local) {
-                    tot = parts[j * g.G];
-                    for (int w2 = 1; w2 < g.G; ++w2) {
-                        tot.x += parts[j * g.G + w2].x;
-                        tot.y += parts[j * g.G + w2].y;
-                    }
+                    my_tot = token_total(parts, lane, g.G);
                 } else {
-                    const float4 v = sc[j];
-                    tot = make_float2(v.z, v.w);
+                    const float4 v = sc[lane];
+                    my_tot = make_float2(v.z, v.w);
                 }
-                float rq, rk;
-                if (MODE == kLwFwd) {
-                    rq = a.Hq ? rsqrtf(fmaf(tot.x, a.inv_q, a.eps)) : 0.f;
-                    rk = a.Hkv ? rsqrtf(fmaf(tot.y, a.inv_k, a.eps)) : 0.f;
-                    if (wb == 0 && lane == 0) {
-                        if (a.Hq) a.wq[t] = rq;
-                        if (a.Hkv) a.wk[t] = rk;
-                    }
-                } else {
-                    const float4 v = sc[j];
-                    rq = v.x;
-                    rk = v.y;
-                }
-                // backward: dx = r (hh - (x r) P / (H_total D)); nq, nk: factors of x
-                const float nq = -rq * tot.x * a.inv_q, nk = -rk * tot.y * a.inv_k;
-                const float2 *cs = cs_st + j * half;
+            }
+            // two tokens per round, their work interleaved
+            for (int j0 = tg; j0 < na; j0 += 2 * g.NTG) {
 #pragma unroll
-                for (int nb = 0; nb < kLwNBMax; ++nb) {
-                    const int b = wb + nb * g.G;
-                    if (b >= g.HB) break;
-                    const int h = b * SLOTS + L.slot;
-                    if (!(L.on && h < H)) continue;
-                    const bool isq = h < a.Hq;
-                    const int hh = isq ? h : h - a.Hq;
-                    const unsigned char *row = stage_row(xq, xk, j, h, a.Hq, a.Hkv, rowb);
-                    const unsigned char *grow = s_gamma + h * rowb;
-                    char *out = (char *)(isq ? a.qo : a.ko) +
-                                ((isq ? t * a.Hq : t * a.Hkv) + hh) * rowb;
-                    const Vec16 xa = ld16(row + offA), xb = ld16(row + offB);
-                    const Vec16 ga = ld16(grow + offA), gb = ld16(grow + offB);
-                    const float r = isq ? rq : rk;
-                    Vec16 oa, ob;
+                for (int u = 0; u < 2; ++u) {
+                    const int j = j0 + u * g.NTG;
+                    const int jj = j < na ? j : j0;
+                    const float2 tot = make_float2(__shfl_sync(0xffffffffu, my_tot.x, jj),
+                                                   __shfl_sync(0xffffffffu, my_tot.y, jj));
+                    if (j >= na) continue;
+                    const int64_t t = t0 + j;
+                    float rq, rk;
                     if (MODE == kLwFwd) {
-#pragma unroll
-                        for (int k2 = 0; k2 < V / 2; ++k2) {
-                            const float2 va = IO::get2(xa, k2), vb = IO::get2(xb, k2);
-                            const float2 wa = IO::get2(ga, k2), wb2 = IO::get2(gb, k2);
-                            const int e = 2 * k2;
-                            const float2 c0 = lane_cs(cs, L.rot, L.eA + e);
-                            const float2 c1 = lane_cs(cs, L.rot, L.eA + e + 1);
-                            const float na0 = va.x * wa.x * r, na1 = va.y * wa.y * r;
-                            const float nb0 = vb.x * wb2.x * r, nb1 = vb.y * wb2.y * r;
-                            IO::put2(oa, k2, fmaf(na0, c0.x, -nb0 * c0.y),
-                                     fmaf(na1, c1.x, -nb1 * c1.y));
-                            IO::put2(ob, k2, fmaf(nb0, c0.x, na0 * c0.y),
-                                     fmaf(nb1, c1.x, na1 * c1.y));
+                        rq = a.Hq ? rsqrtf(fmaf(tot.x, a.inv_q, a.eps)) : 0.f;
+                        rk = a.Hkv ? rsqrtf(fmaf(tot.y, a.inv_k, a.eps)) : 0.f;
+                        if (wb == 0 && lane == 0) {
+                            if (a.Hq) a.wq[t] = rq;
+                            if (a.Hkv) a.wk[t] = rk;
                         }
                     } else {
-                        const unsigned char *drow = stage_row(dq0, dk0, j, h, a.Hq, a.Hkv, rowb);
-                        const Vec16 da = ld16(drow + offA), db = ld16(drow + offB);
-                        const float nd = isq ? nq : nk;
-#pragma unroll
-                        for (int k2 = 0; k2 < V / 2; ++k2) {
-                            const float2 va = IO::get2(xa, k2), vb = IO::get2(xb, k2);
-                            const float2 ea = IO::get2(da, k2), eb = IO::get2(db, k2);
-                            const float2 wa = IO::get2(ga, k2), wb2 = IO::get2(gb, k2);
-                            float outA[2], outB[2];
-#pragma unroll
-                            for (int q = 0; q < 2; ++q) {
-                                const int e = 2 * k2 + q;
-                                const float2 c = lane_cs(cs, L.rot, L.eA + e);
-                                const float dA = q ? ea.y : ea.x, dB = q ? eb.y : eb.x;
-                                const float xA = q ? va.y : va.x, xB = q ? vb.y : vb.x;
-                                const float gA = fmaf(dA, c.x, dB * c.y);
-                                const float gB = fmaf(dB, c.x, -dA * c.y);
-                                const float hA = gA * (q ? wa.y : wa.x);
-                                const float hB = gB * (q ? wb2.y : wb2.x);
-                                outA[q] = r * fmaf(xA, nd, hA);
-                                outB[q] = r * fmaf(xB, nd, hB);
-                                acc[nb][e] = fmaf(gA * xA, r, acc[nb][e]);
-                                acc[nb][V + e] = fmaf(gB * xB, r, acc[nb][V + e]);
-                            }
-                            IO::put2(oa, k2, outA[0], outA[1]);
-                            IO::put2(ob, k2, outB[0], outB[1]);
-                        }
+                        const float4 v = sc[j];
+                        rq = v.x;
+                        rk = v.y;
                     }
-                    lw_st_stream(out + offA, oa);
-                    lw_st_stream(out + offB, ob);
+                    // backward: dx = r (hh - (x r) P / (H_total D)); nq, nk: factors of x
+                    const float nq = -rq * tot.x * a.inv_q, nk = -rk * tot.y * a.inv_k;
+                    float4 c[V / 2];
+                    lane_cs4<V>(c, cs_st + j * hp, L, hp / (V / 2));
+#pragma unroll
+                    for (int nb = 0; nb < kLwNBMax; ++nb) {
+                        const int b = wb + nb * g.G;
+                        if (b >= g.HB) break;
+                        const int h = b * SLOTS + L.slot;
+                        if (!(L.on && h < H)) continue;
+                        const bool isq = h < a.Hq;
+                        const int hh = isq ? h : h - a.Hq;
+                        const unsigned char *row = stage_row(xq, xk, j, h, a.Hq, a.Hkv, rowb);
+                        const unsigned char *grow = s_gamma + h * rowb;
+                        char *out = (char *)(isq ? a.qo : a.ko) +
+                                    ((isq ? t * a.Hq : t * a.Hkv) + hh) * rowb;
+                        const Vec16 xa = ld16(row + offA), xb = ld16(row + offB);
+                        const Vec16 ga = ld16(grow + offA), gb = ld16(grow + offB);
+                        const float r = isq ? rq : rk;
+                        const float2 r2 = make_float2(r, r);
+                        Vec16 oa, ob;
+                        if (MODE == kLwFwd) {
+#pragma unroll
+                            for (int k2 = 0; k2 < V / 2; ++k2) {
+                                const float2 c2 = make_float2(c[k2].x, c[k2].y);
+                                const float2 s2 = make_float2(c[k2].z, c[k2].w);
+                                const float2 nA = __fmul2_rn(__fmul2_rn(IO::get2(xa, k2), IO::get2(ga, k2)), r2);
+                                const float2 nB = __fmul2_rn(__fmul2_rn(IO::get2(xb, k2), IO::get2(gb, k2)), r2);
+                                const float2 yA = __ffma2_rn(nA, c2, __fmul2_rn(nB, neg2f(s2)));
+                                const float2 yB = __ffma2_rn(nB, c2, __fmul2_rn(nA, s2));
+                                IO::put2(oa, k2, yA.x, yA.y);
+                                IO::put2(ob, k2, yB.x, yB.y);
+                            }
+                        } else {
+                            const unsigned char *drow = stage_row(dq0, dk0, j, h, a.Hq, a.Hkv, rowb);
+                            const Vec16 da = ld16(drow + offA), db = ld16(drow + offB);
+                            const float nd = isq ? nq : nk;
+                            const float2 nd2 = make_float2(nd, nd);
+#pragma unroll
+                            for (int k2 = 0; k2 < V / 2; ++k2) {
+                                const float2 c2 = make_float2(c[k2].x, c[k2].y);
+                                const float2 s2 = make_float2(c[k2].z, c[k2].w);
+                                const float2 ea = IO::get2(da, k2), eb = IO::get2(db, k2);
+                                const float2 va = IO::get2(xa, k2), vb = IO::get2(xb, k2);
+                                const float2 gA = __ffma2_rn(ea, c2, __fmul2_rn(eb, s2));
+                                const float2 gB = __ffma2_rn(eb, c2, __fmul2_rn(ea, neg2f(s2)));
+                                const float2 hA = __fmul2_rn(gA, IO::get2(ga, k2));
+                                const float2 hB = __fmul2_rn(gB, IO::get2(gb, k2));
+                                const float2 oA = __fmul2_rn(r2, __ffma2_rn(va, nd2, hA));
+                                const float2 oB = __fmul2_rn(r2, __ffma2_rn(vb, nd2, hB));
+                                acc[nb][k2] = __ffma2_rn(__fmul2_rn(gA, va), r2, acc[nb][k2]);
+                                acc[nb][V / 2 + k2] =
+                                    __ffma2_rn(__fmul2_rn(gB, vb), r2, acc[nb][V / 2 + k2]);
+                                IO::put2(oa, k2, oA.x, oA.y);
+                                IO::put2(ob, k2, oB.x, oB.y);
+                            }
+                        }
+                        lw_st_stream(out + offA, oa);
+                        lw_st_stream(out + offB, ob);
+                    }
                 }
             }
         }
@@ -789,9 +842,11 @@ __global__ void __launch_bounds__(kLwThreadsMax, 1)
             if (!dg) continue;
             dg += (isq ? h : h - a.Hq) * a.D;
 #pragma unroll
-            for (int e = 0; e < V; ++e) {
-                atomicAdd(dg + L.eA + e, acc[nb][e]);
-                atomicAdd(dg + L.eB + e, acc[nb][V + e]);
+            for (int k2 = 0; k2 < V / 2; ++k2) {
+                atomicAdd(dg + L.eA + 2 * k2, acc[nb][k2].x);
+                atomicAdd(dg + L.eA + 2 * k2 + 1, acc[nb][k2].y);
+                atomicAdd(dg + L.eB + 2 * k2, acc[nb][V / 2 + k2].x);
+                atomicAdd(dg + L.eB + 2 * k2 + 1, acc[nb][V / 2 + k2].y);
             }
         }
     }
