@@ -488,8 +488,14 @@ __device__ __forceinline__ void lane_cs4(float4 (&c)[V / 2], const float4 *tok, 
         c[k] = L.rot ? tok[k * U + w] : make_float4(1.f, 1.f, 0.f, 0.f);
 }
 
+// Without upstream gradients (statistics, forward) two CTAs share an SM
+// (64 registers a thread, half the shared memory each); with them, one.
+template <int MODE> struct LwCtas {
+    static constexpr int value = (MODE == kLwDots || MODE == kLwBwd) ? 1 : 2;
+};
+
 template <typename T, int LPR, int MODE>
-__global__ void __launch_bounds__(kLwThreadsMax, 1)
+__global__ void __launch_bounds__(kLwThreadsMax, LwCtas<MODE>::value)
     qknr_lw_pipe_kernel(const LwArgs a, const LwGeom g) {
     using IO = Io<T>;
     constexpr int V = IO::V, SLOTS = 32 / LPR, E = (int)sizeof(T);
@@ -534,13 +540,59 @@ __global__ void __launch_bounds__(kLwThreadsMax, 1)
     if (warp == ncw) {
         // ---------------------------------------------------------- producer
         const uint64_t pol = lw_evict_first();
+        const bool totals = (MODE == kLwFwd || MODE == kLwBwd) &&
+                            !(a.sq == nullptr && a.sk == nullptr);
+        const bool need_sc = kDy || totals, need_cs = MODE != kLwStats && half > 0;
+        int s_cur = (int)(t_lo % a.S);  // row position of the tile's first token
+        // (cos, sin) work split, fixed for the kernel. Pair P of a token is
+        // stored at (P mod W) U + P / W (W = V/2 pairs per lane, U = hp / W
+        // rotating units) so that the lanes of a row read consecutive entries.
+        const int cs_hp = half >> 1;
+        const int cs_tpp = (cs_hp > 0 && cs_hp <= 32) ? 32 / cs_hp : 0;  // tokens per pass
+        int cs_jo = 0, cs_P = -1, cs_dst = 0;
+        uint64_t cs_F0 = 0, cs_F1 = 0;
+        if (cs_tpp > 0 && lane < cs_tpp * cs_hp) {
+            cs_jo = lane / cs_hp;
+            cs_P = lane - cs_jo * cs_hp;
+            cs_F0 = s_step[2 * cs_P];
+            cs_F1 = s_step[2 * cs_P + 1];
+            const int pw = cs_P / (V / 2);
+            cs_dst = (cs_P - pw * (V / 2)) * (cs_hp / (V / 2)) + pw;
+        }
         int issued = 0;
         for (int i = 0; i < ntiles; ++i) {
             const int s = i % g.NS;
             const uint32_t ph = (uint32_t)(i / g.NS) & 1u;
-            if (i >= g.NS && !lw_wait(bar0 + 8 * (g.NS + s), ph ^ 1u)) break;
             const int64_t t0 = t_lo + (int64_t)i * g.TT;
             const int na = (int)min((int64_t)g.TT, t_hi - t0);
+            // this stage's per-token values, loaded before the wait for the
+            // slot so that their latency overlaps it: saved rstd (backward),
+            // all-rank totals (second phase of a sharded call), positions
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            int32_t pos = 0;
+            if (lane < na) {
+                const int64_t t = t0 + lane;
+                if (kDy) {
+                    v.x = a.Hq ? a.rq[t] : 0.f;
+                    v.y = a.Hkv ? a.rk[t] : 0.f;
+                }
+                if (totals) {
+                    v.z = a.Hq ? a.sq[t] : 0.f;
+                    v.w = a.Hkv ? a.sk[t] : 0.f;
+                }
+                if (need_cs) {
+                    if (a.pos) {
+                        pos = a.pos[t];
+                    } else {
+                        int p = s_cur + lane;
+                        while (p >= a.S) p -= a.S;
+                        pos = p;
+                    }
+                }
+            }
+            s_cur += g.TT;
+            while (s_cur >= a.S) s_cur -= a.S;
+            if (i >= g.NS && !lw_wait(bar0 + 8 * (g.NS + s), ph ^ 1u)) break;
             unsigned char *st = ring + (size_t)s * g.stage_bytes;
             const uint32_t full = bar0 + 8 * s;
             if (lane == 0) {
@@ -558,46 +610,34 @@ __global__ void __launch_bounds__(kLwThreadsMax, 1)
                     lw_bulk(lw_smem_u32(st + g.off_dk), (const char *)a.dko + t0 * a.Hkv * rowb, bk,
                             full, pol);
             }
-            {
-                // per-token scalars the consumers need: saved rstd (backward),
-                // all-rank totals (second phase of a sharded call)
-                const bool totals = (MODE == kLwFwd || MODE == kLwBwd) &&
-                                    !(a.sq == nullptr && a.sk == nullptr);
-                if (lane < na && (kDy || totals)) {
-                    const int64_t t = t0 + lane;
-                    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-                    if (kDy) {
-                        v.x = a.Hq ? a.rq[t] : 0.f;
-                        v.y = a.Hkv ? a.rk[t] : 0.f;
-                    }
-                    if (totals) {
-                        v.z = a.Hq ? a.sq[t] : 0.f;
-                        v.w = a.Hkv ? a.sk[t] : 0.f;
-                    }
-                    reinterpret_cast<float4 *>(st + g.off_sc)[lane] = v;
-                }
-            }
-            if (MODE != kLwStats && half > 0) {
-                // positions (the given ids, else s within the batch row), then
-                // the (cos, sin) table of the stage, one angle per lane at a time
-                if (lane < na) {
-                    const int64_t t = t0 + lane;
-                    s_pos[lane] = a.pos ? a.pos[t] : (int32_t)(t % a.S);
-                }
+            if (need_sc && lane < na) reinterpret_cast<float4 *>(st + g.off_sc)[lane] = v;
+            if (need_cs) {
+                if (lane < na) s_pos[lane] = pos;
                 __syncwarp();
-                // pair P of a token: (c_2P, c_2P+1, s_2P, s_2P+1), one float4,
-                // stored at (P mod W) U + P / W (W pairs per lane, U rotating
-                // units) so that the lanes of a row read consecutive entries
+                // pair P of a token: (c_2P, c_2P+1, s_2P, s_2P+1), one float4
                 float4 *cs = reinterpret_cast<float4 *>(st + g.off_cs);
-                constexpr int W = V / 2;
-                const int hp = half >> 1, U = hp / W;
-#pragma unroll 2
-                for (int idx = lane; idx < na * hp; idx += 32) {
-                    const int j = idx / hp, P = idx - j * hp;
-                    const float2 c0 = rope_cos_sin_fixed(s_pos[j], s_step[2 * P]);
-                    const float2 c1 = rope_cos_sin_fixed(s_pos[j], s_step[2 * P + 1]);
-                    const int pw = P / W;
-                    cs[j * hp + (P - pw * W) * U + pw] = make_float4(c0.x, c1.x, c0.y, c1.y);
+                if (cs_tpp > 0) {
+                    // hp <= 32: lane (jo, P) takes pair P of tokens jo, jo + tpp, ...
+                    if (cs_P >= 0)
+                        for (int j = cs_jo; j < na; j += cs_tpp) {
+                            const int32_t m = s_pos[j];
+                            const float2 c0 = rope_cos_sin_fixed(m, cs_F0);
+                            const float2 c1 = rope_cos_sin_fixed(m, cs_F1);
+                            cs[j * cs_hp + cs_dst] = make_float4(c0.x, c1.x, c0.y, c1.y);
+                        }
+                } else {
+                    // hp > 32: lane takes pairs P = lane + 32 k of every token
+                    for (int P = lane; P < cs_hp; P += 32) {
+                        const uint64_t F0 = s_step[2 * P], F1 = s_step[2 * P + 1];
+                        const int pw = P / (V / 2);
+                        const int dst = (P - pw * (V / 2)) * (cs_hp / (V / 2)) + pw;
+                        for (int j = 0; j < na; ++j) {
+                            const int32_t m = s_pos[j];
+                            const float2 c0 = rope_cos_sin_fixed(m, F0);
+                            const float2 c1 = rope_cos_sin_fixed(m, F1);
+                            cs[j * cs_hp + dst] = make_float4(c0.x, c1.x, c0.y, c1.y);
+                        }
+                    }
                 }
                 __syncwarp();
             }
@@ -619,7 +659,7 @@ __global__ void __launch_bounds__(kLwThreadsMax, 1)
     const int hp = half >> 1;  // rotary pairs per token
     const bool local = (MODE == kLwFwd || MODE == kLwBwd) && a.sq == nullptr && a.sk == nullptr;
     const bool need_parts = MODE == kLwStats || MODE == kLwDots || local;
-    constexpr int kUA = (MODE == kLwStats || MODE == kLwFwd) ? 4 : 2;  // tokens per partial-sum round
+    constexpr int kUA = 2;  // tokens per partial-sum round
     float2 acc[kLwNBMax][V];  // dgamma sums: pairs of the A vector, then of the B vector
 #pragma unroll
     for (int nb = 0; nb < kLwNBMax; ++nb)
@@ -739,10 +779,12 @@ __global__ void __launch_bounds__(kLwThreadsMax, 1)
                     my_tot = make_float2(v.z, v.w);
                 }
             }
-            // two tokens per round, their work interleaved
-            for (int j0 = tg; j0 < na; j0 += 2 * g.NTG) {
+            // kUB tokens per round, their work interleaved (one when two
+            // CTAs share the SM's registers)
+            constexpr int kUB = LwCtas<MODE>::value == 1 ? 2 : 1;
+            for (int j0 = tg; j0 < na; j0 += kUB * g.NTG) {
 #pragma unroll
-                for (int u = 0; u < 2; ++u) {
+                for (int u = 0; u < kUB; ++u) {
                     const int j = j0 + u * g.NTG;
                     const int jj = j < na ? j : j0;
                     const float2 tot = make_float2(__shfl_sync(0xffffffffu, my_tot.x, jj),
@@ -830,17 +872,21 @@ __global__ void __launch_bounds__(kLwThreadsMax, 1)
     }
 
     if (MODE == kLwBwd) {
-        // this lane's dgamma sums (fixed rows and elements) into the rank's slice
+        // dgamma: the token groups of this CTA own the same elements, so sum
+        // them in shared memory (the ring, free now) first, then one global
+        // atomic add per element and CTA
+        float *s_red = reinterpret_cast<float *>(ring);
+        const int nel = H * a.D, ct = ncw * 32;
+        asm volatile("bar.sync 1, %0;" ::"r"(ct) : "memory");
+        for (int e = threadIdx.x; e < nel; e += ct) s_red[e] = 0.f;
+        asm volatile("bar.sync 1, %0;" ::"r"(ct) : "memory");
 #pragma unroll
         for (int nb = 0; nb < kLwNBMax; ++nb) {
             const int b = wb + nb * g.G;
             if (b >= g.HB) break;
             const int h = b * SLOTS + L.slot;
             if (!(L.on && h < H)) continue;
-            const bool isq = h < a.Hq;
-            float *dg = isq ? a.dgq : a.dgk;
-            if (!dg) continue;
-            dg += (isq ? h : h - a.Hq) * a.D;
+            float *dg = s_red + h * a.D;
 #pragma unroll
             for (int k2 = 0; k2 < V / 2; ++k2) {
                 atomicAdd(dg + L.eA + 2 * k2, acc[nb][k2].x);
@@ -848,6 +894,12 @@ __global__ void __launch_bounds__(kLwThreadsMax, 1)
                 atomicAdd(dg + L.eB + 2 * k2, acc[nb][V / 2 + k2].x);
                 atomicAdd(dg + L.eB + 2 * k2 + 1, acc[nb][V / 2 + k2].y);
             }
+        }
+        asm volatile("bar.sync 1, %0;" ::"r"(ct) : "memory");
+        const int nq = a.Hq * a.D;
+        for (int e = threadIdx.x; e < nel; e += ct) {
+            float *dg = e < nq ? a.dgq + e : a.dgk + (e - nq);
+            if ((e < nq ? a.dgq : a.dgk) != nullptr) atomicAdd(dg, s_red[e]);
         }
     }
 }
@@ -914,10 +966,12 @@ bool lw_plan(int mode, const LwArgs &a, int esz, int lpr, int sms, LwGeom *g, in
     if (TT > kMaxTileTokensLw) return false;
     const int64_t stage = ((TT * per + 127) / 128) * 128;
     const int64_t gbytes = ((xq + xk + 127) / 128) * 128;
-    const int64_t budget = kLwSmemBytes - 128 - TT * G * 8 * kLwMaxStages - 128 - gbytes;
+    const int ctas = dy ? 1 : 2;  // CTAs per SM (LwCtas)
+    const int64_t budget = kLwSmemBytes / ctas - 128 - TT * G * 8 * kLwMaxStages - 128 - gbytes;
     int64_t NS = (budget < kLwRingBytes ? budget : kLwRingBytes) / stage;
     if (NS > kLwMaxStages) NS = kLwMaxStages;
     if (NS < 2) return false;
+    if (mode == kLwBwd && NS * stage < (int64_t)H * a.D * 4) return false;  // dgamma sums
     g->TT = (int)TT;
     g->NS = (int)NS;
     g->stage_bytes = (int)stage;
@@ -932,7 +986,7 @@ bool lw_plan(int mode, const LwArgs &a, int esz, int lpr, int sms, LwGeom *g, in
     g->NTG = NTG;
     g->HB = HB;
     const int64_t tiles = (a.T + TT - 1) / TT;
-    int64_t nb = tiles < sms ? tiles : sms;
+    int64_t nb = tiles < (int64_t)sms * ctas ? tiles : (int64_t)sms * ctas;
     const int64_t tiles_per = (tiles + nb - 1) / nb;
     g->tpc = tiles_per * TT;
     nb = (a.T + g->tpc - 1) / g->tpc;
