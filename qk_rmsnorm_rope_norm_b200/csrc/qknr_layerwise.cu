@@ -366,7 +366,6 @@ __global__ void __launch_bounds__(kThreads) qknr_lw_bwd_kernel(const LwArgs a) {
 // per-stage barrier, in a fixed order, so the one-pass and the two-phase
 // calls add the same terms in the same order.
 constexpr int kLwCWMax = 15;                   // consumer warps at most (+1: 16 warps, 128 registers)
-constexpr int kLwThreadsMax = (kLwCWMax + 1) * 32;  // + the producer warp
 constexpr int kLwNBMax = 2;                    // head blocks one consumer warp may own
 constexpr int kLwMaxStages = 4;
 constexpr int kLwStageTarget = 48 * 1024;
@@ -488,14 +487,17 @@ __device__ __forceinline__ void lane_cs4(float4 (&c)[V / 2], const float4 *tok, 
         c[k] = L.rot ? tok[k * U + w] : make_float4(1.f, 1.f, 0.f, 0.f);
 }
 
-// Without upstream gradients (statistics, forward) two CTAs share an SM
-// (64 registers a thread, half the shared memory each); with them, one.
+// Without upstream gradients (statistics, forward) two CTAs of at most 11
+// consumer warps share an SM (24 warps, 80 registers a thread, half the
+// shared memory each); with them, one CTA of at most 15 (128 registers).
 template <int MODE> struct LwCtas {
     static constexpr int value = (MODE == kLwDots || MODE == kLwBwd) ? 1 : 2;
+    static constexpr int cw_max = value == 1 ? kLwCWMax : 11;
+    static constexpr int threads_max = (cw_max + 1) * 32;
 };
 
 template <typename T, int LPR, int MODE>
-__global__ void __launch_bounds__(kLwThreadsMax, LwCtas<MODE>::value)
+__global__ void __launch_bounds__(LwCtas<MODE>::threads_max, LwCtas<MODE>::value)
     qknr_lw_pipe_kernel(const LwArgs a, const LwGeom g) {
     using IO = Io<T>;
     constexpr int V = IO::V, SLOTS = 32 / LPR, E = (int)sizeof(T);
@@ -950,11 +952,12 @@ bool lw_plan(int mode, const LwArgs &a, int esz, int lpr, int sms, LwGeom *g, in
     const int HB = (H + slots - 1) / slots;
     // head blocks per warp, warps per token, token groups: every warp owns
     // NB blocks (the last one maybe fewer), at most kLwCWMax warps
-    const int NB = (HB + kLwCWMax - 1) / kLwCWMax;
+    const bool dy = mode == kLwDots || mode == kLwBwd;
+    const int cw_max = dy ? LwCtas<kLwBwd>::cw_max : LwCtas<kLwFwd>::cw_max;
+    const int NB = (HB + cw_max - 1) / cw_max;
     if (NB > kLwNBMax) return false;
     const int G = (HB + NB - 1) / NB;
-    const int NTG = kLwCWMax / G;
-    const bool dy = mode == kLwDots || mode == kLwBwd;
+    const int NTG = cw_max / G;
     const int64_t rowb = (int64_t)a.D * esz;
     const int64_t xq = (int64_t)a.Hq * rowb, xk = (int64_t)a.Hkv * rowb;  // per token
     const int64_t csb = mode == kLwStats ? 0 : (int64_t)(a.R / 2) * 8;
