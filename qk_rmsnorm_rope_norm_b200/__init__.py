@@ -11,7 +11,10 @@ CUDA device.
 Names follow the C ABI: ``qk_norm_rope_fwd`` / ``qk_norm_rope_bwd`` (which
 also take Q / K slices of a fused QKV buffer, dispatching to the
 ``_strided`` entry points). The autograd wrappers ``QKNormRoPE`` and
-``QKNormRoPEFromQKV`` chain them for training code.
+``QKNormRoPEFromQKV`` chain them for training code. The layerwise form for
+tensor parallelism (``qk_layerwise_*``) is chained by
+``QKLayerwiseNormRoPE``, which sums the per-token partial statistics over a
+``torch.distributed`` group between its kernel calls.
 """
 from __future__ import annotations
 
@@ -729,7 +732,8 @@ def qk_layerwise_norm_rope_bwd(q, k, gamma_q, gamma_k, pos_ids, rstd_q, rstd_k, 
         if t.shape != ref.shape or t.dtype != ref.dtype:
             raise ValueError(f"{n} must match its input in shape and dtype")
     for n, t in (("rstd_q", rstd_q), ("rstd_k", rstd_k), ("dot_q", dot_q), ("dot_k", dot_k)):
-        _token_vec(n, t, T, q.device) if t is not None else None
+        if t is not None:  # (None dot sums: the one-pass backward)
+            _token_vec(n, t, T, q.device)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     for n, t, ref in (("dq", dq, q), ("dk", dk, k)):

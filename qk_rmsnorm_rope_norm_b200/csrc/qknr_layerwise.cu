@@ -351,30 +351,31 @@ __global__ void __launch_bounds__(kThreads) qknr_lw_bwd_kernel(const LwArgs a) {
 }
 
 // ------------------------------------------------------------------------
-// Pipelined kernels. One producer warp streams stages of TT whole tokens
-// (their Q rows, K rows and, backward, the upstream gradients: each one
-// contiguous range) into a shared-memory ring with 1-D bulk copies and
-// fills the stage's (cos, sin) table; G * NTG consumer warps (at most
-// kLwCWMax, chosen per shape so that every warp owns the same number of
+// Pipelined dots and backward (the statistics and the forward use the
+// plain-load kernels above). One producer warp streams stages of TT whole
+// tokens (their Q rows, K rows and upstream gradients: each one contiguous
+// range) into a shared-memory ring with 1-D bulk copies and fills the
+// stage's (cos, sin) table and per-token scalars; G * NTG consumer warps (at
+// most kLwCWMax, chosen per shape so that every warp owns the same number of
 // head blocks) share each stage. Consumer warp w owns head block set
 // {wb + G nb} (a block is the SLOTS rows one warp covers at once) of token
-// group tg (tokens tg, tg + NTG, ...), so
-// the rows, gamma elements and dgamma sums a lane touches are the same for
-// the whole kernel: dgamma is summed in registers and added to global
-// memory once per lane at the end. Per-token sums over all heads are
+// group tg (tokens tg, tg + NTG, ...), so the rows, gamma elements and
+// dgamma sums a lane touches are the same for the whole kernel: dgamma is
+// summed in registers, then per CTA in shared memory, and added to global
+// memory once per element and CTA. Per-token sums over all heads are
 // reduced across the G warps of a token through a small shared table and a
 // per-stage barrier, in a fixed order, so the one-pass and the two-phase
 // calls add the same terms in the same order.
 constexpr int kLwCWMax = 15;                   // consumer warps at most (+1: 16 warps, 128 registers)
 constexpr int kLwNBMax = 2;                    // head blocks one consumer warp may own
 constexpr int kLwMaxStages = 4;
-constexpr int kLwStageTarget = 48 * 1024;
+constexpr int kLwStageTarget = 96 * 1024;
 constexpr int kLwRingBytes = 200 * 1024;
 constexpr int kMaxTileTokensLw = 32;
 constexpr int kLwSmemBytes = 220 * 1024;       // dynamic shared memory at most
 constexpr long long kLwWaitCycles = 4000000000ll;  // ~2 s per wait at 1.9 GHz
 
-enum LwMode { kLwStats = 0, kLwFwd = 1, kLwDots = 2, kLwBwd = 3 };
+enum LwMode { kLwDots = 0, kLwBwd = 1 };
 
 // Sticky error flag of the pipelined layerwise kernels (bit 0: a wait gave
 // up, the launch's results are then incomplete; bit 1: shared memory not
@@ -487,21 +488,11 @@ __device__ __forceinline__ void lane_cs4(float4 (&c)[V / 2], const float4 *tok, 
         c[k] = L.rot ? tok[k * U + w] : make_float4(1.f, 1.f, 0.f, 0.f);
 }
 
-// Without upstream gradients (statistics, forward) two CTAs of at most 11
-// consumer warps share an SM (24 warps, 80 registers a thread, half the
-// shared memory each); with them, one CTA of at most 15 (128 registers).
-template <int MODE> struct LwCtas {
-    static constexpr int value = (MODE == kLwDots || MODE == kLwBwd) ? 1 : 2;
-    static constexpr int cw_max = value == 1 ? kLwCWMax : 11;
-    static constexpr int threads_max = (cw_max + 1) * 32;
-};
-
 template <typename T, int LPR, int MODE>
-__global__ void __launch_bounds__(LwCtas<MODE>::threads_max, LwCtas<MODE>::value)
+__global__ void __launch_bounds__((kLwCWMax + 1) * 32, 1)
     qknr_lw_pipe_kernel(const LwArgs a, const LwGeom g) {
     using IO = Io<T>;
     constexpr int V = IO::V, SLOTS = 32 / LPR, E = (int)sizeof(T);
-    constexpr bool kDy = MODE == kLwDots || MODE == kLwBwd;
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ uint64_t s_step[kMaxHalf];      // fixed-point angle step per rotary pair
     __shared__ int32_t s_pos[kMaxTileTokensLw];  // producer: positions of the stage's tokens
@@ -521,7 +512,7 @@ __global__ void __launch_bounds__(LwCtas<MODE>::threads_max, LwCtas<MODE>::value
     const int ntiles = t_hi > t_lo ? (int)((t_hi - t_lo + g.TT - 1) / g.TT) : 0;
     const int H = a.Hq + a.Hkv, rowb = a.D * E;
     unsigned char *s_gamma = smem + g.off_gamma;  // every CTA reads the weights once
-    if (MODE != kLwStats) {  // (the statistics alone take no weights: gq, gk unset)
+    {
         const int nq = a.Hq * rowb / 16, nk = a.Hkv * rowb / 16;
         for (int i = threadIdx.x; i < nq + nk; i += nthr) {
             const Vec16 v = i < nq ? ld16((const char *)a.gq + 16 * i)
@@ -542,9 +533,8 @@ __global__ void __launch_bounds__(LwCtas<MODE>::threads_max, LwCtas<MODE>::value
     if (warp == ncw) {
         // ---------------------------------------------------------- producer
         const uint64_t pol = lw_evict_first();
-        const bool totals = (MODE == kLwFwd || MODE == kLwBwd) &&
-                            !(a.sq == nullptr && a.sk == nullptr);
-        const bool need_sc = kDy || totals, need_cs = MODE != kLwStats && half > 0;
+        const bool totals = MODE == kLwBwd && !(a.sq == nullptr && a.sk == nullptr);
+        const bool need_cs = half > 0;
         int s_cur = (int)(t_lo % a.S);  // row position of the tile's first token
         // (cos, sin) work split, fixed for the kernel. Pair P of a token is
         // stored at (P mod W) U + P / W (W = V/2 pairs per lane, U = hp / W
@@ -568,16 +558,14 @@ __global__ void __launch_bounds__(LwCtas<MODE>::threads_max, LwCtas<MODE>::value
             const int64_t t0 = t_lo + (int64_t)i * g.TT;
             const int na = (int)min((int64_t)g.TT, t_hi - t0);
             // this stage's per-token values, loaded before the wait for the
-            // slot so that their latency overlaps it: saved rstd (backward),
-            // all-rank totals (second phase of a sharded call), positions
+            // slot so that their latency overlaps it: saved rstd, all-rank
+            // totals (second phase of a sharded call), positions
             float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
             int32_t pos = 0;
             if (lane < na) {
                 const int64_t t = t0 + lane;
-                if (kDy) {
-                    v.x = a.Hq ? a.rq[t] : 0.f;
-                    v.y = a.Hkv ? a.rk[t] : 0.f;
-                }
+                v.x = a.Hq ? a.rq[t] : 0.f;
+                v.y = a.Hkv ? a.rk[t] : 0.f;
                 if (totals) {
                     v.z = a.Hq ? a.sq[t] : 0.f;
                     v.w = a.Hkv ? a.sk[t] : 0.f;
@@ -600,19 +588,19 @@ __global__ void __launch_bounds__(LwCtas<MODE>::threads_max, LwCtas<MODE>::value
             if (lane == 0) {
                 const uint32_t bq = (uint32_t)(na * a.Hq * rowb);
                 const uint32_t bk = (uint32_t)(na * a.Hkv * rowb);
-                lw_bar_expect(full, (kDy ? 2u : 1u) * (bq + bk));
+                lw_bar_expect(full, 2u * (bq + bk));
                 if (bq) lw_bulk(lw_smem_u32(st), (const char *)a.q + t0 * a.Hq * rowb, bq, full, pol);
                 if (bk)
                     lw_bulk(lw_smem_u32(st + g.off_k), (const char *)a.k + t0 * a.Hkv * rowb, bk,
                             full, pol);
-                if (kDy && bq)
+                if (bq)
                     lw_bulk(lw_smem_u32(st + g.off_dq), (const char *)a.dqo + t0 * a.Hq * rowb, bq,
                             full, pol);
-                if (kDy && bk)
+                if (bk)
                     lw_bulk(lw_smem_u32(st + g.off_dk), (const char *)a.dko + t0 * a.Hkv * rowb, bk,
                             full, pol);
             }
-            if (need_sc && lane < na) reinterpret_cast<float4 *>(st + g.off_sc)[lane] = v;
+            if (lane < na) reinterpret_cast<float4 *>(st + g.off_sc)[lane] = v;
             if (need_cs) {
                 if (lane < na) s_pos[lane] = pos;
                 __syncwarp();
@@ -655,12 +643,10 @@ __global__ void __launch_bounds__(LwCtas<MODE>::threads_max, LwCtas<MODE>::value
     // -------------------------------------------------------------- consumers
     const int tg = warp / g.G, wb = warp % g.G;
     const Lane<LPR, V> L(lane, a.D, a.R);
-    const Lane<LPR, V> Ls(lane, a.D, 0);  // layout of the sums of squares
     const int offA = L.eA * E, offB = L.eB * E;
-    const int offSA = Ls.eA * E, offSB = Ls.eB * E;
     const int hp = half >> 1;  // rotary pairs per token
-    const bool local = (MODE == kLwFwd || MODE == kLwBwd) && a.sq == nullptr && a.sk == nullptr;
-    const bool need_parts = MODE == kLwStats || MODE == kLwDots || local;
+    const bool local = MODE == kLwBwd && a.sq == nullptr && a.sk == nullptr;
+    const bool need_parts = MODE == kLwDots || local;
     constexpr int kUA = 2;  // tokens per partial-sum round
     float2 acc[kLwNBMax][V];  // dgamma sums: pairs of the A vector, then of the B vector
 #pragma unroll
@@ -682,8 +668,8 @@ __global__ void __launch_bounds__(LwCtas<MODE>::threads_max, LwCtas<MODE>::value
         float2 *parts = parts_all + (size_t)s * g.TT * g.G;
 
         if (need_parts) {
-            // this warp's share of each token's sums, x^2 or (g gamma).(x r),
-            // kUA tokens per round so that their warp reductions overlap
+            // this warp's share of each token's (g gamma).(x r), kUA tokens
+            // per round so that their warp reductions overlap
             for (int j0 = tg; j0 < na; j0 += kUA * g.NTG) {
                 float vq[kUA], vk[kUA];
 #pragma unroll
@@ -692,13 +678,9 @@ __global__ void __launch_bounds__(LwCtas<MODE>::threads_max, LwCtas<MODE>::value
                     vq[u] = vk[u] = 0.f;
                     if (j >= na) continue;
                     float4 c[V / 2];
-                    float r2q = 0.f, r2k = 0.f;
-                    if (kDy) {
-                        lane_cs4<V>(c, cs_st + j * hp, L, hp / (V / 2));
-                        const float4 sv = sc[j];
-                        r2q = sv.x;
-                        r2k = sv.y;
-                    }
+                    lane_cs4<V>(c, cs_st + j * hp, L, hp / (V / 2));
+                    const float4 sv = sc[j];
+                    const float r2q = sv.x, r2k = sv.y;
 #pragma unroll
                     for (int nb = 0; nb < kLwNBMax; ++nb) {
                         const int b = wb + nb * g.G;
@@ -707,38 +689,25 @@ __global__ void __launch_bounds__(LwCtas<MODE>::threads_max, LwCtas<MODE>::value
                         if (!(L.on && h < H)) continue;
                         const bool isq = h < a.Hq;
                         const unsigned char *row = stage_row(xq, xk, j, h, a.Hq, a.Hkv, rowb);
+                        const unsigned char *drow = stage_row(dq0, dk0, j, h, a.Hq, a.Hkv, rowb);
+                        const unsigned char *grow = s_gamma + h * rowb;
+                        const Vec16 xa = ld16(row + offA), xb = ld16(row + offB);
+                        const Vec16 da = ld16(drow + offA), db = ld16(drow + offB);
+                        const Vec16 ga = ld16(grow + offA), gb = ld16(grow + offB);
                         float2 p2 = make_float2(0.f, 0.f);
-                        if (!kDy) {
-                            const Vec16 xa = ld16(row + offSA), xb = ld16(row + offSB);
 #pragma unroll
-                            for (int k2 = 0; k2 < V / 2; ++k2) {
-                                const float2 va = IO::get2(xa, k2), vb = IO::get2(xb, k2);
-                                p2 = __ffma2_rn(va, va, p2);
-                                p2 = __ffma2_rn(vb, vb, p2);
-                            }
-                            const float p = p2.x + p2.y;
-                            vq[u] += isq ? p : 0.f;
-                            vk[u] += isq ? 0.f : p;
-                        } else {
-                            const unsigned char *drow = stage_row(dq0, dk0, j, h, a.Hq, a.Hkv, rowb);
-                            const unsigned char *grow = s_gamma + h * rowb;
-                            const Vec16 xa = ld16(row + offA), xb = ld16(row + offB);
-                            const Vec16 da = ld16(drow + offA), db = ld16(drow + offB);
-                            const Vec16 ga = ld16(grow + offA), gb = ld16(grow + offB);
-#pragma unroll
-                            for (int k2 = 0; k2 < V / 2; ++k2) {
-                                const float2 c2 = make_float2(c[k2].x, c[k2].y);
-                                const float2 s2 = make_float2(c[k2].z, c[k2].w);
-                                const float2 ea = IO::get2(da, k2), eb = IO::get2(db, k2);
-                                const float2 gA = __ffma2_rn(ea, c2, __fmul2_rn(eb, s2));
-                                const float2 gB = __ffma2_rn(eb, c2, __fmul2_rn(ea, neg2f(s2)));
-                                p2 = __ffma2_rn(__fmul2_rn(gA, IO::get2(ga, k2)), IO::get2(xa, k2), p2);
-                                p2 = __ffma2_rn(__fmul2_rn(gB, IO::get2(gb, k2)), IO::get2(xb, k2), p2);
-                            }
-                            const float p = (p2.x + p2.y) * (isq ? r2q : r2k);
-                            vq[u] += isq ? p : 0.f;
-                            vk[u] += isq ? 0.f : p;
+                        for (int k2 = 0; k2 < V / 2; ++k2) {
+                            const float2 c2 = make_float2(c[k2].x, c[k2].y);
+                            const float2 s2 = make_float2(c[k2].z, c[k2].w);
+                            const float2 ea = IO::get2(da, k2), eb = IO::get2(db, k2);
+                            const float2 gA = __ffma2_rn(ea, c2, __fmul2_rn(eb, s2));
+                            const float2 gB = __ffma2_rn(eb, c2, __fmul2_rn(ea, neg2f(s2)));
+                            p2 = __ffma2_rn(__fmul2_rn(gA, IO::get2(ga, k2)), IO::get2(xa, k2), p2);
+                            p2 = __ffma2_rn(__fmul2_rn(gB, IO::get2(gb, k2)), IO::get2(xb, k2), p2);
                         }
+                        const float p = (p2.x + p2.y) * (isq ? r2q : r2k);
+                        vq[u] += isq ? p : 0.f;
+                        vk[u] += isq ? 0.f : p;
                     }
                 }
 #pragma unroll
@@ -760,7 +729,7 @@ __global__ void __launch_bounds__(LwCtas<MODE>::threads_max, LwCtas<MODE>::value
             const uint32_t pbar = bar0 + 8 * (2 * g.NS + s);
             if (lane == 0) lw_bar_arrive(pbar);
             if (!lw_wait(pbar, ph)) break;
-            if ((MODE == kLwStats || MODE == kLwDots) && warp == 0) {
+            if (MODE == kLwDots && warp == 0) {
                 // lane j: token j's total over the G warps, in warp order
                 for (int j = lane; j < na; j += 32) {
                     const float2 tot = token_total(parts, j, g.G);
@@ -770,7 +739,7 @@ __global__ void __launch_bounds__(LwCtas<MODE>::threads_max, LwCtas<MODE>::value
             }
         }
 
-        if (MODE == kLwFwd || MODE == kLwBwd) {
+        if (MODE == kLwBwd) {
             // per-token totals: lane j holds token j's (j < 32; TT <= 32)
             float2 my_tot = make_float2(0.f, 0.f);
             if (lane < na) {
@@ -781,32 +750,19 @@ __global__ void __launch_bounds__(LwCtas<MODE>::threads_max, LwCtas<MODE>::value
                     my_tot = make_float2(v.z, v.w);
                 }
             }
-            // kUB tokens per round, their work interleaved (one when two
-            // CTAs share the SM's registers)
-            constexpr int kUB = LwCtas<MODE>::value == 1 ? 2 : 1;
-            for (int j0 = tg; j0 < na; j0 += kUB * g.NTG) {
+            // two tokens per round, their work interleaved
+            for (int j0 = tg; j0 < na; j0 += 2 * g.NTG) {
 #pragma unroll
-                for (int u = 0; u < kUB; ++u) {
+                for (int u = 0; u < 2; ++u) {
                     const int j = j0 + u * g.NTG;
                     const int jj = j < na ? j : j0;
                     const float2 tot = make_float2(__shfl_sync(0xffffffffu, my_tot.x, jj),
                                                    __shfl_sync(0xffffffffu, my_tot.y, jj));
                     if (j >= na) continue;
                     const int64_t t = t0 + j;
-                    float rq, rk;
-                    if (MODE == kLwFwd) {
-                        rq = a.Hq ? rsqrtf(fmaf(tot.x, a.inv_q, a.eps)) : 0.f;
-                        rk = a.Hkv ? rsqrtf(fmaf(tot.y, a.inv_k, a.eps)) : 0.f;
-                        if (wb == 0 && lane == 0) {
-                            if (a.Hq) a.wq[t] = rq;
-                            if (a.Hkv) a.wk[t] = rk;
-                        }
-                    } else {
-                        const float4 v = sc[j];
-                        rq = v.x;
-                        rk = v.y;
-                    }
-                    // backward: dx = r (hh - (x r) P / (H_total D)); nq, nk: factors of x
+                    const float4 sv = sc[j];
+                    const float rq = sv.x, rk = sv.y;
+                    // dx = r (hh - (x r) P / (H_total D)); nq, nk: the factors of x
                     const float nq = -rq * tot.x * a.inv_q, nk = -rk * tot.y * a.inv_k;
                     float4 c[V / 2];
                     lane_cs4<V>(c, cs_st + j * hp, L, hp / (V / 2));
@@ -819,49 +775,33 @@ __global__ void __launch_bounds__(LwCtas<MODE>::threads_max, LwCtas<MODE>::value
                         const bool isq = h < a.Hq;
                         const int hh = isq ? h : h - a.Hq;
                         const unsigned char *row = stage_row(xq, xk, j, h, a.Hq, a.Hkv, rowb);
+                        const unsigned char *drow = stage_row(dq0, dk0, j, h, a.Hq, a.Hkv, rowb);
                         const unsigned char *grow = s_gamma + h * rowb;
                         char *out = (char *)(isq ? a.qo : a.ko) +
                                     ((isq ? t * a.Hq : t * a.Hkv) + hh) * rowb;
                         const Vec16 xa = ld16(row + offA), xb = ld16(row + offB);
+                        const Vec16 da = ld16(drow + offA), db = ld16(drow + offB);
                         const Vec16 ga = ld16(grow + offA), gb = ld16(grow + offB);
-                        const float r = isq ? rq : rk;
-                        const float2 r2 = make_float2(r, r);
+                        const float r = isq ? rq : rk, nd = isq ? nq : nk;
+                        const float2 r2 = make_float2(r, r), nd2 = make_float2(nd, nd);
                         Vec16 oa, ob;
-                        if (MODE == kLwFwd) {
 #pragma unroll
-                            for (int k2 = 0; k2 < V / 2; ++k2) {
-                                const float2 c2 = make_float2(c[k2].x, c[k2].y);
-                                const float2 s2 = make_float2(c[k2].z, c[k2].w);
-                                const float2 nA = __fmul2_rn(__fmul2_rn(IO::get2(xa, k2), IO::get2(ga, k2)), r2);
-                                const float2 nB = __fmul2_rn(__fmul2_rn(IO::get2(xb, k2), IO::get2(gb, k2)), r2);
-                                const float2 yA = __ffma2_rn(nA, c2, __fmul2_rn(nB, neg2f(s2)));
-                                const float2 yB = __ffma2_rn(nB, c2, __fmul2_rn(nA, s2));
-                                IO::put2(oa, k2, yA.x, yA.y);
-                                IO::put2(ob, k2, yB.x, yB.y);
-                            }
-                        } else {
-                            const unsigned char *drow = stage_row(dq0, dk0, j, h, a.Hq, a.Hkv, rowb);
-                            const Vec16 da = ld16(drow + offA), db = ld16(drow + offB);
-                            const float nd = isq ? nq : nk;
-                            const float2 nd2 = make_float2(nd, nd);
-#pragma unroll
-                            for (int k2 = 0; k2 < V / 2; ++k2) {
-                                const float2 c2 = make_float2(c[k2].x, c[k2].y);
-                                const float2 s2 = make_float2(c[k2].z, c[k2].w);
-                                const float2 ea = IO::get2(da, k2), eb = IO::get2(db, k2);
-                                const float2 va = IO::get2(xa, k2), vb = IO::get2(xb, k2);
-                                const float2 gA = __ffma2_rn(ea, c2, __fmul2_rn(eb, s2));
-                                const float2 gB = __ffma2_rn(eb, c2, __fmul2_rn(ea, neg2f(s2)));
-                                const float2 hA = __fmul2_rn(gA, IO::get2(ga, k2));
-                                const float2 hB = __fmul2_rn(gB, IO::get2(gb, k2));
-                                const float2 oA = __fmul2_rn(r2, __ffma2_rn(va, nd2, hA));
-                                const float2 oB = __fmul2_rn(r2, __ffma2_rn(vb, nd2, hB));
-                                acc[nb][k2] = __ffma2_rn(__fmul2_rn(gA, va), r2, acc[nb][k2]);
-                                acc[nb][V / 2 + k2] =
-                                    __ffma2_rn(__fmul2_rn(gB, vb), r2, acc[nb][V / 2 + k2]);
-                                IO::put2(oa, k2, oA.x, oA.y);
-                                IO::put2(ob, k2, oB.x, oB.y);
-                            }
+                        for (int k2 = 0; k2 < V / 2; ++k2) {
+                            const float2 c2 = make_float2(c[k2].x, c[k2].y);
+                            const float2 s2 = make_float2(c[k2].z, c[k2].w);
+                            const float2 ea = IO::get2(da, k2), eb = IO::get2(db, k2);
+                            const float2 va = IO::get2(xa, k2), vb = IO::get2(xb, k2);
+                            const float2 gA = __ffma2_rn(ea, c2, __fmul2_rn(eb, s2));
+                            const float2 gB = __ffma2_rn(eb, c2, __fmul2_rn(ea, neg2f(s2)));
+                            const float2 hA = __fmul2_rn(gA, IO::get2(ga, k2));
+                            const float2 hB = __fmul2_rn(gB, IO::get2(gb, k2));
+                            const float2 oA = __fmul2_rn(r2, __ffma2_rn(va, nd2, hA));
+                            const float2 oB = __fmul2_rn(r2, __ffma2_rn(vb, nd2, hB));
+                            acc[nb][k2] = __ffma2_rn(__fmul2_rn(gA, va), r2, acc[nb][k2]);
+                            acc[nb][V / 2 + k2] =
+                                __ffma2_rn(__fmul2_rn(gB, vb), r2, acc[nb][V / 2 + k2]);
+                            IO::put2(oa, k2, oA.x, oA.y);
+                            IO::put2(ob, k2, oB.x, oB.y);
                         }
                         lw_st_stream(out + offA, oa);
                         lw_st_stream(out + offB, ob);
@@ -944,24 +884,23 @@ bool simple_kernels_forced() {
     return e && e[0] && e[0] != '0';
 }
 
-// Stage and ring sizes of the pipelined kernels for this shape, or false if
-// the shape does not fit them (the plain-load kernels run instead).
+// Stage and ring sizes of the pipelined (dots, backward) kernels for this
+// shape, or false if the shape does not fit them (the plain-load kernels run
+// instead).
 bool lw_plan(int mode, const LwArgs &a, int esz, int lpr, int sms, LwGeom *g, int *grid,
              int *smem, int *threads) {
     const int slots = 32 / lpr, H = a.Hq + a.Hkv;
     const int HB = (H + slots - 1) / slots;
     // head blocks per warp, warps per token, token groups: every warp owns
     // NB blocks (the last one maybe fewer), at most kLwCWMax warps
-    const bool dy = mode == kLwDots || mode == kLwBwd;
-    const int cw_max = dy ? LwCtas<kLwBwd>::cw_max : LwCtas<kLwFwd>::cw_max;
-    const int NB = (HB + cw_max - 1) / cw_max;
+    const int NB = (HB + kLwCWMax - 1) / kLwCWMax;
     if (NB > kLwNBMax) return false;
     const int G = (HB + NB - 1) / NB;
-    const int NTG = cw_max / G;
+    const int NTG = kLwCWMax / G;
     const int64_t rowb = (int64_t)a.D * esz;
     const int64_t xq = (int64_t)a.Hq * rowb, xk = (int64_t)a.Hkv * rowb;  // per token
-    const int64_t csb = mode == kLwStats ? 0 : (int64_t)(a.R / 2) * 8;
-    const int64_t per = (dy ? 2 : 1) * (xq + xk) + csb + 16;  // + the per-token scalars
+    const int64_t csb = (int64_t)(a.R / 2) * 8;
+    const int64_t per = 2 * (xq + xk) + csb + 16;  // rows, gradients, angles, scalars
     int64_t TT = kLwStageTarget / per;
     TT = TT > kMaxTileTokensLw ? kMaxTileTokensLw : TT;
     TT = (TT / NTG) * NTG;
@@ -969,19 +908,18 @@ bool lw_plan(int mode, const LwArgs &a, int esz, int lpr, int sms, LwGeom *g, in
     if (TT > kMaxTileTokensLw) return false;
     const int64_t stage = ((TT * per + 127) / 128) * 128;
     const int64_t gbytes = ((xq + xk + 127) / 128) * 128;
-    const int ctas = dy ? 1 : 2;  // CTAs per SM (LwCtas)
-    const int64_t budget = kLwSmemBytes / ctas - 128 - TT * G * 8 * kLwMaxStages - 128 - gbytes;
+    const int64_t budget = kLwSmemBytes - 128 - TT * G * 8 * kLwMaxStages - 128 - gbytes;
     int64_t NS = (budget < kLwRingBytes ? budget : kLwRingBytes) / stage;
     if (NS > kLwMaxStages) NS = kLwMaxStages;
     if (NS < 2) return false;
-    if (mode == kLwBwd && NS * stage < (int64_t)H * a.D * 4) return false;  // dgamma sums
+    if (NS * stage < (int64_t)H * a.D * 4) return false;  // the backward's dgamma sums
     g->TT = (int)TT;
     g->NS = (int)NS;
     g->stage_bytes = (int)stage;
     g->off_k = (int)(TT * xq);
     g->off_dq = (int)(TT * (xq + xk));
     g->off_dk = (int)(TT * (2 * xq + xk));
-    g->off_cs = (int)(TT * (dy ? 2 : 1) * (xq + xk));
+    g->off_cs = (int)(TT * 2 * (xq + xk));
     g->off_sc = g->off_cs + (int)(TT * csb);
     g->off_parts = 128 + (int)(NS * stage);
     g->off_gamma = g->off_parts + (int)(((NS * TT * G * 8 + 127) / 128) * 128);
@@ -989,7 +927,7 @@ bool lw_plan(int mode, const LwArgs &a, int esz, int lpr, int sms, LwGeom *g, in
     g->NTG = NTG;
     g->HB = HB;
     const int64_t tiles = (a.T + TT - 1) / TT;
-    int64_t nb = tiles < (int64_t)sms * ctas ? tiles : (int64_t)sms * ctas;
+    int64_t nb = tiles < (int64_t)sms ? tiles : (int64_t)sms;
     const int64_t tiles_per = (tiles + nb - 1) / nb;
     g->tpc = tiles_per * TT;
     nb = (a.T + g->tpc - 1) / g->tpc;
@@ -1011,22 +949,20 @@ qknr_status lw_pipe_launch(const LwArgs &a, const LwGeom &g, int grid, int smem,
 
 template <typename T, int LPR>
 qknr_status lw_launch_t(LwKernel which, const LwArgs &a, cudaStream_t st) {
-    if (!simple_kernels_forced()) {
+    // The statistics and the forward read a token's rows, reduce and write:
+    // one warp per token with plain loads measured faster on B200 than the
+    // staged pipeline (whose per-stage cross-warp sum costs more than it
+    // saves there), so only the dots and the backward, whose dgamma sums
+    // need fixed row ownership, take the pipeline.
+    if (!simple_kernels_forced() && (which == LwKernel::kDots || which == LwKernel::kBwd)) {
         int dev = 0;
         cudaGetDevice(&dev);
-        const int mode = which == LwKernel::kStats ? kLwStats
-                         : which == LwKernel::kFwd ? kLwFwd
-                         : which == LwKernel::kDots ? kLwDots
-                                                    : kLwBwd;
+        const int mode = which == LwKernel::kDots ? kLwDots : kLwBwd;
         LwGeom g;
         int grid, smem, thr;
         if (lw_plan(mode, a, (int)sizeof(T), LPR, sm_count_of(dev), &g, &grid, &smem, &thr)) {
-            switch (mode) {
-                case kLwStats: return lw_pipe_launch<T, LPR, kLwStats>(a, g, grid, smem, thr, st);
-                case kLwFwd: return lw_pipe_launch<T, LPR, kLwFwd>(a, g, grid, smem, thr, st);
-                case kLwDots: return lw_pipe_launch<T, LPR, kLwDots>(a, g, grid, smem, thr, st);
-                default: return lw_pipe_launch<T, LPR, kLwBwd>(a, g, grid, smem, thr, st);
-            }
+            return mode == kLwDots ? lw_pipe_launch<T, LPR, kLwDots>(a, g, grid, smem, thr, st)
+                                   : lw_pipe_launch<T, LPR, kLwBwd>(a, g, grid, smem, thr, st);
         }
     }
     int grid, tpw;
