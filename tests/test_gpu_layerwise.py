@@ -287,3 +287,52 @@ def test_layerwise_large_hidden_falls_back(cuda):
 
 def test_layerwise_no_pipeline_timeouts(cuda):
     assert qknr.pipeline_error() == 0
+
+
+@pytest.mark.parametrize("dtype,D,R", [("bf16", 128, 0), ("f32", 64, 0), ("f32", 64, 16),
+                                       ("bf16", 64, 32)])
+def test_layerwise_rotary_spans_and_dtypes(cuda, kernels, dtype, D, R):
+    # NoPE (no rotary span), partial spans, fp32 I/O; one rank and two slices
+    inp, gq, gk = lw_inputs("tiny", seed=6, B=2, S=45, Hq=8, Hkv=4, D=D, rotary_dim=R,
+                            dtype=dtype)
+    for world in (1, 2):
+        check_vs_oracle(inp, gq, gk, run_ranks(inp, gq, gk, cuda, world=world))
+    check_vs_oracle(inp, gq, gk, run_ranks(inp, gq, gk, cuda, local=True))
+
+
+def test_layerwise_extreme_positions(cuda, kernels):
+    import numpy as np
+    inp, gq, gk = lw_inputs("tiny", seed=3, B=2, S=40, Hq=6, Hkv=2, D=128, rotary_dim=64,
+                            dtype="bf16", theta=1e4)
+    rng = np.random.default_rng(3)
+    pos = rng.integers(-2 ** 31, 2 ** 31 - 1, size=(2, 40))
+    pos.reshape(-1)[:6] = [0, 1, -1, 2 ** 31 - 1, -(2 ** 31), 65535]
+    inp.pos = torch.from_numpy(pos.astype(np.int32))
+    check_vs_oracle(inp, gq, gk, run_ranks(inp, gq, gk, cuda, local=True))
+    check_vs_oracle(inp, gq, gk, run_ranks(inp, gq, gk, cuda, world=2))
+
+
+def test_layerwise_full_size_sampled(cuda):
+    """The Llama-3-8B-shaped batch at full size (32,768 tokens, 40 heads), one
+    pass each way as the bench times it; outputs, rstd and dX of 384 sampled
+    tokens against the oracle (each token's statistic involves that token
+    only). dgamma is a sum over every token and is checked at the smaller
+    sizes above."""
+    import numpy as np
+    inp, gq, gk = lw_inputs("llama3-8b-qknorm")
+    w = inp.w
+    got = run_ranks(inp, gq, gk, cuda, local=True)
+    T = w.B * w.S
+    pick = np.sort(np.random.default_rng(11).choice(T, 384, replace=False))
+    pick[:2] = [0, T - 1]
+    m = positions_of(inp)[pick]
+    o = oracle.get()
+    for name, x, g, dy, H in (("q", inp.q, gq, inp.dq_out, w.Hq), ("k", inp.k, gk, inp.dk_out, w.Hkv)):
+        st = parity.Stats(w.dtype, H * w.D)
+        x3 = x.reshape(T, H, w.D)[pick]
+        y, r = o.lw_fwd(x3, g, m, w.rotary_dim, w.theta, w.eps)
+        dx, _ = o.lw_bwd(x3, g, dy.reshape(T, H, w.D)[pick], m, w.rotary_dim, w.theta, w.eps)
+        st.elem(f"{name}_out", got[f"{name}_out"].reshape(T, H, w.D)[pick].double().numpy(), y)
+        st.rstd(got[f"rstd_{name}"].reshape(T)[pick].double().numpy(), r)
+        st.elem(f"d{name}", got[f"d{name}"].reshape(T, H, w.D)[pick].double().numpy(), dx)
+        st.check()
