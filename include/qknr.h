@@ -309,7 +309,8 @@ QKNR_API qknr_status qk_rope_apply(const void *q, const void *k,
  * One rank holding every head (Hq_total = Hq, Hkv_total = Hkv) may pass
  * NULL for both sumsq pointers of step 3, or both dot pointers of step 6:
  * the call then takes the statistic itself in the same pass (steps 1-2 or
- * 4-5 skipped; each row is read again from cache, not from HBM). NULL sums
+ * 4-5 skipped; the second read of each row comes from on-chip memory or
+ * L2, mostly). NULL sums
  * with totals above the local counts are QKNR_ERR_INVALID_ARG.
  *
  * pos_ids as for qk_norm_rope_fwd (NULL: position s of each row). Either
