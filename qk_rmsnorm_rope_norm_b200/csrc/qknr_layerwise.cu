@@ -17,10 +17,16 @@
 //             dgamma[h D + d] += g x r_t, g = R^T dy
 //
 // The exchange itself (an all-reduce of one fp32 per token and tensor) is
-// the caller's: NCCL through torch.distributed in the Python binding.
-// One warp walks all of a token's local heads, so each per-token sum is one
-// warp reduction. gamma rows are read with the same 16-byte vectors as x rows
-// (they are cached; every token reuses them).
+// the caller's: NCCL through torch.distributed in the Python binding. A rank
+// holding every head passes no totals and gets one pass each way.
+//
+// Two kernel families. Plain-load kernels: one warp walks all of a token's
+// local heads, so each per-token sum is one warp reduction; gamma rows are
+// read with the same 16-byte vectors as x rows (they are cached; every token
+// reuses them). They serve the statistics and the forward, and every shape
+// the pipeline below does not take. Pipelined kernels (further down): the
+// dots and the backward, staged through shared memory by bulk copies, with
+// dgamma summed in registers.
 #include "qknr.h"
 #include "qknr_kernels.cuh"
 
@@ -38,7 +44,7 @@ constexpr int kLwMaxDgammaBytes = 200 * 1024;
 struct LwArgs {
     const void *q, *k;        // this rank's heads: [T, Hq, D], [T, Hkv, D]
     const void *gq, *gk;      // gamma slices [Hq * D], [Hkv * D]
-    const int32_t *pos;
+    const int32_t *pos;       // position ids [T] or NULL (s within the batch row)
     const void *dqo, *dko;    // upstream gradients (backward)
     void *qo, *ko;            // forward outputs, or dq, dk (backward)
     const float *sq, *sk;     // per-token totals over ranks (S_t or P_t)
