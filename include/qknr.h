@@ -324,6 +324,29 @@ QKNR_API qknr_status qk_rope_apply(const void *q, const void *k,
  * dq = dq_out, dk = dk_out. T = 0 or no heads: nothing launched (the
  * backward still zeroes dgamma).
  */
+/*
+ * Launch geometry of the layerwise pipelined kernels for a shape, for
+ * inspection and host-side checks; no CUDA call is made. mode 0: the dots
+ * (qk_layerwise_bwd_dots), 1: the backward (qk_layerwise_norm_rope_bwd);
+ * sms: the SM count to plan for. geom (19 int64, caller-owned) receives
+ *   [0] 1 if the pipelined kernel runs for this shape, 0 if the plain-load
+ *       kernel does (then the rest is 0),
+ *   [1] lanes per head row, [2] tokens per stage, [3] stages,
+ *   [4] bytes per stage, [5..9] byte offsets within a stage of the K rows,
+ *       dQ_out rows, dK_out rows, (cos, sin) table and per-token scalars,
+ *   [10] offset of the per-token partial-sum table and [11] of the gamma
+ *       table in the dynamic shared memory,
+ *   [12] warps per token, [13] token groups, [14] head blocks,
+ *   [15] tokens per CTA, [16] CTAs, [17] dynamic shared memory bytes,
+ *   [18] threads per CTA.
+ * Shapes are checked as for qk_layerwise_norm_rope_bwd (with the totals
+ * equal to the local head counts); a bad mode, sms or NULL geom is
+ * QKNR_ERR_INVALID_ARG.
+ */
+QKNR_API qknr_status qk_layerwise_geometry(int mode, int B, int S, int Hq, int Hkv, int D,
+                             int rotary_dim, qknr_dtype dtype, int sms,
+                             int64_t *geom);
+
 QKNR_API qknr_status qk_layerwise_stats(const void *q, const void *k,
                              float *sumsq_q, float *sumsq_k,
                              int B, int S, int Hq, int Hkv, int D,

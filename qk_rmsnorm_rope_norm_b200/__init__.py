@@ -31,7 +31,7 @@ __all__ = ["qk_norm_rope_fwd", "qk_norm_rope_bwd", "qknr_strerror", "QKNormRoPE"
            "qk_norm_rope", "QKNRError", "library_path", "load_library", "pipeline_error",
            "qk_layerwise_stats", "qk_layerwise_norm_rope_fwd", "qk_layerwise_bwd_dots",
            "qk_layerwise_norm_rope_bwd", "QKLayerwiseNormRoPE", "qk_layerwise_norm_rope",
-           "all_reduce_stats"]
+           "all_reduce_stats", "layerwise_geometry"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libqknr.so")
@@ -95,6 +95,8 @@ def load_library():
     lib.qk_layerwise_bwd_dots.argtypes = [vp] * 11 + [i32] * 6 + [f32, i32, vp]
     lib.qk_layerwise_norm_rope_bwd.restype = i32
     lib.qk_layerwise_norm_rope_bwd.argtypes = [vp] * 15 + [i32] * 8 + [f32, i32, vp]
+    lib.qk_layerwise_geometry.restype = i32
+    lib.qk_layerwise_geometry.argtypes = [i32] * 9 + [vp]
     lib.qknr_strerror.restype = ctypes.c_char_p
     lib.qknr_strerror.argtypes = [i32]
     lib.qknr_last_cuda_error.restype = i32
@@ -811,3 +813,21 @@ def qk_layerwise_norm_rope(q, k, gamma_q, gamma_k, pos_ids=None, *, rotary_dim: 
     return QKLayerwiseNormRoPE.apply(q.contiguous(), k.contiguous(), gamma_q.contiguous(),
                                      gamma_k.contiguous(), pos_ids, rotary_dim, theta, eps, Hqt,
                                      Hkvt, group)
+
+
+_GEOM_KEYS = ("pipelined", "lpr", "TT", "NS", "stage_bytes", "off_k", "off_dq", "off_dk",
+              "off_cs", "off_sc", "off_parts", "off_gamma", "G", "NTG", "HB", "tpc", "grid",
+              "smem", "threads")
+
+
+def layerwise_geometry(mode: str, B: int, S: int, Hq: int, Hkv: int, D: int, rotary_dim: int,
+                       dtype=torch.bfloat16, sms: int = 148) -> dict:
+    """Launch geometry of the pipelined layerwise ``"dots"`` or ``"bwd"``
+    kernel for a shape (C ``qk_layerwise_geometry``; host only, no GPU)."""
+    lib = load_library()
+    out = (ctypes.c_int64 * len(_GEOM_KEYS))()
+    st = lib.qk_layerwise_geometry({"dots": 0, "bwd": 1}[mode], B, S, Hq, Hkv, D, rotary_dim,
+                                   _DTYPES[dtype], sms, ctypes.cast(out, ctypes.c_void_p))
+    if st != QKNR_OK:
+        raise QKNRError(st, "qk_layerwise_geometry")
+    return dict(zip(_GEOM_KEYS, (int(v) for v in out)))

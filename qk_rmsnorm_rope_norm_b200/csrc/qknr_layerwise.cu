@@ -40,6 +40,7 @@ qknr_status cuda_fail(cudaError_t e);  // defined beside the per-head entry poin
 namespace {
 
 constexpr int kLwMaxDgammaBytes = 200 * 1024;
+constexpr int kLwGeomLen = 19;  // entries qk_layerwise_geometry writes
 
 struct LwArgs {
     const void *q, *k;        // this rank's heads: [T, Hq, D], [T, Hkv, D]
@@ -395,7 +396,7 @@ struct LwGeom {
     int off_parts;                      // per-token partial sums [NS][TT][G] float2
     int off_gamma;                      // gamma_q then gamma_k rows, I/O dtype
     int G, NTG, HB;                     // warps per token, token groups, head blocks
-    int64_t tpc;                        // tokens per CTA (a multiple of TT)
+    int64_t tpc;                        // tokens per CTA
 };
 
 __device__ __forceinline__ uint32_t lw_smem_u32(const void *p) {
@@ -932,10 +933,11 @@ bool lw_plan(int mode, const LwArgs &a, int esz, int lpr, int sms, LwGeom *g, in
     g->G = G;
     g->NTG = NTG;
     g->HB = HB;
+    // one CTA per SM, the tokens split evenly (a CTA's last stage may be
+    // partial), so no SM idles for want of whole stages
     const int64_t tiles = (a.T + TT - 1) / TT;
     int64_t nb = tiles < (int64_t)sms ? tiles : (int64_t)sms;
-    const int64_t tiles_per = (tiles + nb - 1) / nb;
-    g->tpc = tiles_per * TT;
+    g->tpc = (a.T + nb - 1) / nb;
     nb = (a.T + g->tpc - 1) / g->tpc;
     *grid = (int)nb;
     *smem = g->off_gamma + (int)gbytes;
@@ -1078,6 +1080,30 @@ int lw_pipeline_error(int reset) {
 }  // namespace qknr
 
 using namespace qknr;
+
+extern "C" qknr_status qk_layerwise_geometry(int mode, int B, int S, int Hq, int Hkv, int D,
+                                             int rotary_dim, qknr_dtype dtype, int sms,
+                                             int64_t *geom) {
+    if (!geom || (mode != 0 && mode != 1) || sms < 1) return QKNR_ERR_INVALID_ARG;
+    qknr_status s = lw_check(B, S, Hq, Hkv, Hq, Hkv, D, rotary_dim, 1.f, 0.f, dtype);
+    if (s != QKNR_OK) return s;
+    if (mode == 1 && (int64_t)(Hq + Hkv) * D * 4 > kLwMaxDgammaBytes) return QKNR_ERR_UNSUPPORTED;
+    for (int i = 0; i < kLwGeomLen; ++i) geom[i] = 0;
+    const int esz = dtype == QKNR_F32 ? 4 : 2;
+    LwArgs a{};
+    a.T = (int64_t)B * S; a.S = S; a.Hq = Hq; a.Hkv = Hkv; a.D = D; a.R = rotary_dim;
+    if (a.T == 0 || Hq + Hkv == 0) return QKNR_OK;
+    const int lpr = lpr_of(D, esz);
+    LwGeom g;
+    int grid, smem, thr;
+    if (!lw_plan(mode == 0 ? kLwDots : kLwBwd, a, esz, lpr, sms, &g, &grid, &smem, &thr))
+        return QKNR_OK;
+    const int64_t v[kLwGeomLen] = {1, lpr, g.TT, g.NS, g.stage_bytes, g.off_k, g.off_dq,
+                                   g.off_dk, g.off_cs, g.off_sc, g.off_parts, g.off_gamma, g.G,
+                                   g.NTG, g.HB, g.tpc, grid, smem, thr};
+    for (int i = 0; i < kLwGeomLen; ++i) geom[i] = v[i];
+    return QKNR_OK;
+}
 
 extern "C" qknr_status qk_layerwise_stats(const void *q, const void *k, float *sumsq_q,
                                           float *sumsq_k, int B, int S, int Hq, int Hkv, int D,
