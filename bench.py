@@ -5,22 +5,24 @@
     python bench.py --impl reference ...      (the CPU oracle, as the reference arm)
 
 A step is one forward and one backward over one batch of the workload
-(default: the Qwen2.5-0.5B-shaped batch, 8 x 2048 tokens, 14 query / 2 KV
-heads of dim 64, bf16 I/O). Inputs are resident in HBM before timing. Each
-rank keeps a ring of four input/output sets; step i runs the forward on set
-i mod 4 and the backward on set (i - 2) mod 4 (a layer's backward comes
+(default: the largest single-GPU configuration, partial RoPE at long
+context: one row of 65,536 tokens, 32 query / 8 KV heads of dim 128, rotary
+on the first 32 dims, bf16 I/O). Inputs are resident in HBM before timing.
+Each rank keeps a ring of four input/output sets; step i runs the forward on
+set i mod 4 and the backward on set (i - 2) mod 4 (a layer's backward comes
 after the rest of the forward in training), so no kernel finds its inputs in
-the 126 MB L2: between two touches of a set ~2.5x L2 of other traffic
-passes. K steps are timed with CUDA events between a barrier and a
+the 126 MB L2. K steps are timed with CUDA events between a barrier and a
 synchronize on both sides; every fwd/bwd launch is also bracketed by events
 on its stream for the per-kernel roofline. N > 1 (torchrun): weak scaling,
 each rank its own batch, no collective on the data path; the time is the
 max over ranks.
 
-Rank 0 prints one JSON line. ``e2e`` repeats the step through the public
-Python API from pinned host buffers (inputs copied in, every output copied
-back, inside the timed region). ``cpu_baseline`` times the CPU oracle on a
-bounded sample of the same workload.
+Rank 0 prints one JSON line. ``per_config`` times the other workloads the
+same way (their own rings, forward and backward each). ``e2e`` repeats the
+step through the public Python API from pinned host buffers (inputs copied
+in, every output copied back, inside the timed region). ``cpu_baseline``
+times the CPU oracle on a bounded sample of the same workload, on one host
+core and on all of them.
 """
 from __future__ import annotations
 
@@ -28,10 +30,12 @@ import argparse
 import hashlib
 import json
 import os
+import platform
 import statistics
 import sys
 import threading
 import time
+from concurrent.futures import ThreadPoolExecutor
 
 import torch
 
@@ -43,6 +47,9 @@ import workloads  # noqa: E402
 METRIC = "QK-norm+RoPE fwd+bwd tokens/s and HBM GB/s (% of B200 peak), 1 GPU"
 FALLBACK_HBM_GBS = 6650.0
 NSETS, LAG = 4, 2  # ring of input sets; the backward runs LAG steps behind
+# the workloads timed beside the headline one (one GPU each); the tiny fp32
+# case is a parity check, not a throughput workload
+PER_CONFIG = ("qwen2.5-0.5b", "llama3-8b-qknorm", "partial-rope-64k", "bfd-packed")
 KERNEL_SOURCES = ["qk_rmsnorm_rope_norm_b200/csrc/qknr_kernels.cuh",
                   "qk_rmsnorm_rope_norm_b200/csrc/qknr_pipe.cuh",
                   "qk_rmsnorm_rope_norm_b200/csrc/qknr_api.cu"]
@@ -222,19 +229,21 @@ class Set:
         self.dgk = torch.empty(w.D, dtype=torch.float32, device=dev)
 
 
-def run_ours(args, w, inp, rank, local_rank, world):
+def measure(w, inp, dev, steps: int, warmup: int, nsets: int, layout: str = "dense",
+            world: int = 1, clocks=None):
+    """Time ``steps`` fwd + bwd steps of workload ``w`` on a ring of ``nsets``
+    input sets (after ``warmup`` untimed steps), events around every launch.
+    Returns the total, mean forward and mean backward milliseconds, the max
+    over ranks when ``world`` > 1."""
     import qk_rmsnorm_rope_norm_b200 as qknr
-    dev = torch.device("cuda", local_rank)
-    qknr.load_library()
     cfg = dict(rotary_dim=w.rotary_dim, theta=w.theta, eps=w.eps)
-    nsets = args.sets
-    sets = [Set(inp, dev, args.layout) for _ in range(nsets)]
+    sets = [Set(inp, dev, layout) for _ in range(nsets)]
     stream = torch.cuda.current_stream(dev)
     fwd = [qknr.prepare_fwd(s.q, s.k, s.gq, s.gk, s.pos, s.qo, s.ko, s.rq, s.rk, **cfg)
            for s in sets]
     bwd = [qknr.prepare_bwd(s.q, s.k, s.gq, s.gk, s.pos, s.rq, s.rk, s.dqo, s.dko, s.dq,
                             s.dk, s.dgq, s.dgk, **cfg) for s in sets]
-    K, W = args.steps, args.warmup
+    K, W = steps, warmup
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
 
@@ -254,7 +263,7 @@ def run_ours(args, w, inp, rank, local_rank, world):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
-    with ClockSampler(local_rank) as clocks:
+    with (clocks if clocks is not None else _Null()):
         t_start.record(stream)
         for i in range(K):
             step(W + i, ev[i])
@@ -266,8 +275,27 @@ def run_ours(args, w, inp, rank, local_rank, world):
     total_ms = t_start.elapsed_time(t_end)
     fwd_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / K
     bwd_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / K
-    total_ms, fwd_ms, bwd_ms = max_over_ranks([total_ms, fwd_ms, bwd_ms], world, dev)
+    del fwd, bwd, sets
+    return max_over_ranks([total_ms, fwd_ms, bwd_ms], world, dev)
 
+
+class _Null:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        return False
+
+
+def run_ours(args, w, inp, rank, local_rank, world):
+    import qk_rmsnorm_rope_norm_b200 as qknr
+    dev = torch.device("cuda", local_rank)
+    qknr.load_library()
+    cfg = dict(rotary_dim=w.rotary_dim, theta=w.theta, eps=w.eps)
+    clocks = ClockSampler(local_rank)  # NVML start-up stays outside the timed region
+    total_ms, fwd_ms, bwd_ms = measure(w, inp, dev, args.steps, args.warmup, args.sets,
+                                       args.layout, world, clocks)
+    torch.cuda.empty_cache()
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(args, w, inp, dev, cfg, world)
@@ -275,6 +303,58 @@ def run_ours(args, w, inp, rank, local_rank, world):
     floor = {"fwd_ms": copy_floor_ms(cb["fwd"], dev), "bwd_ms": copy_floor_ms(cb["bwd"], dev)}
     return dict(total_ms=total_ms, fwd_ms=fwd_ms, bwd_ms=bwd_ms, clocks=clocks.summary(),
                 e2e=e2e, floor=floor)
+
+
+def device_limits(dev):
+    """SM count and opt-in shared memory per block of ``dev`` (for the plan)."""
+    p = torch.cuda.get_device_properties(dev)
+    return p.multi_processor_count, int(getattr(p, "shared_memory_per_block_optin", 0) or 0)
+
+
+def kernels_of(w, dev, layout: str = "dense"):
+    """The forward and backward kernels the library launches for ``w``."""
+    import qk_rmsnorm_rope_norm_b200 as qknr
+    sms, optin = device_limits(dev)
+    strided = 3 if layout == "qkv" else 0
+    return tuple(qknr.kernel_name(kind, w.B, w.S, w.Hq, w.Hkv, w.D, w.rotary_dim,
+                                  w.torch_dtype, strided, sms, optin) for kind in ("fwd", "bwd"))
+
+
+def per_config_line(w, inp, fwd_ms, bwd_ms, peak, dev, steps):
+    cb = workloads.contract_bytes(w, with_pos=inp.pos is not None)
+    kf, kb = kernels_of(w, dev)
+    tok = inp.real_tokens
+
+    def one(ms, nbytes, kern):
+        gbs = nbytes / (ms / 1e3) / 1e9
+        return {"ms": ms, "gbs": gbs, "frac": gbs / peak, "tokens_per_s": tok / (ms / 1e3),
+                "bytes_per_launch": nbytes, "kernel": kern}
+
+    return {"fwd": one(fwd_ms, cb["fwd"], kf), "bwd": one(bwd_ms, cb["bwd"], kb),
+            "fwd_bwd_tokens_per_s": tok / ((fwd_ms + bwd_ms) / 1e3), "tokens": tok,
+            "steps": steps}
+
+
+def run_per_config(args, main_w, main_r, rank, dev, peak):
+    """Every throughput workload on its own ring, timed like the main step;
+    the headline workload's entry repeats the main measurement."""
+    out = {}
+    for name in PER_CONFIG:
+        if name == main_w.name:
+            w, inp = main_w, main_inp_cache[0]
+            fwd_ms, bwd_ms, steps = main_r["fwd_ms"], main_r["bwd_ms"], args.steps
+        else:
+            base = workloads.WORKLOADS[name]
+            inp = workloads.make_inputs(base, seed=rank_seed(base, rank))
+            w = inp.w
+            steps = args.per_config_steps
+            _, fwd_ms, bwd_ms = measure(w, inp, dev, steps, max(3, args.warmup), NSETS)
+            torch.cuda.empty_cache()
+        out[name] = per_config_line(w, inp, fwd_ms, bwd_ms, peak, dev, steps)
+    return out
+
+
+main_inp_cache = [None]
 
 
 def run_variants(args, w, inp, dev, peak):
@@ -507,9 +587,33 @@ def run_e2e(args, w, inp, dev, cfg, world):
 
 
 # ------------------------------------------------------- the CPU oracle
-def oracle_sample_rate(inp, budget_s: float, tokens_per_call: int = 512, max_calls=None):
-    """Time the CPU oracle (fwd + bwd) on consecutive token chunks of the
-    workload until ``budget_s`` seconds or the workload are used up."""
+def host_cores() -> int:
+    """Cores this process may run on."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    return platform.processor() or "unknown"
+
+
+def oracle_rate(inp, budget_s: float, threads: int, tokens_per_call: int = 256,
+                rounds=None):
+    """Time the CPU oracle (fwd + bwd, unmodified) on consecutive token chunks
+    of the workload with ``threads`` host threads, each taking the next chunk
+    until ``budget_s`` seconds of wall time have passed (or, with ``rounds``,
+    exactly ``rounds`` chunks per thread). The oracle is C called through
+    ctypes, which releases the GIL, so the threads run on separate cores.
+    Returns (tokens, wall seconds, per-round wall times)."""
     import oracle
     w = inp.w
     T = w.B * w.S
@@ -519,40 +623,58 @@ def oracle_sample_rate(inp, budget_s: float, tokens_per_call: int = 512, max_cal
     dqo = inp.dq_out.reshape(T, w.Hq, w.D)
     dko = inp.dk_out.reshape(T, w.Hkv, w.D)
     orc = oracle.get()
-    done, spent, calls, t0 = 0, 0.0, 0, 0
-    per_call = []
-    while spent < budget_s and (max_calls is None or calls < max_calls):
-        t1 = min(T, t0 + tokens_per_call)
-        args = [a[t0:t1] for a in (q, k)]
+    lock = threading.Lock()
+    nxt = [0]
+
+    def chunk():
+        with lock:
+            t0 = nxt[0]
+            t1 = min(T, t0 + tokens_per_call)
+            nxt[0] = t1 % T
         m = m_all[t0:t1]
-        c = time.perf_counter()
-        orc.fwd(args[0], args[1], inp.gamma_q, inp.gamma_k, m, w.rotary_dim, w.theta, w.eps)
-        orc.bwd(args[0], args[1], inp.gamma_q, inp.gamma_k, m, dqo[t0:t1], dko[t0:t1],
+        orc.fwd(q[t0:t1], k[t0:t1], inp.gamma_q, inp.gamma_k, m, w.rotary_dim, w.theta, w.eps)
+        orc.bwd(q[t0:t1], k[t0:t1], inp.gamma_q, inp.gamma_k, m, dqo[t0:t1], dko[t0:t1],
                 w.rotary_dim, w.theta, w.eps)
-        dt = time.perf_counter() - c
-        per_call.append(dt)
-        spent += dt
-        done += t1 - t0
-        calls += 1
-        t0 = t1 % T
-    return done, spent, per_call
+        return t1 - t0
+
+    def worker(deadline, n):
+        done, calls = 0, 0
+        while (n is None and time.perf_counter() < deadline) or (n is not None and calls < n):
+            done += chunk()
+            calls += 1
+        return done
+
+    per_round = []
+    with ThreadPoolExecutor(threads) as ex:
+        if rounds is None:
+            c = time.perf_counter()
+            done = sum(ex.map(worker, [c + budget_s] * threads, [None] * threads))
+            wall = time.perf_counter() - c
+        else:
+            done, wall = 0, 0.0
+            for _ in range(rounds):
+                c = time.perf_counter()
+                done += sum(ex.map(worker, [0.0] * threads, [1] * threads))
+                dt = time.perf_counter() - c
+                per_round.append(dt)
+                wall += dt
+    return done, wall, per_round
+
+
+def cpu_baseline(inp, budget_s: float) -> dict:
+    """The oracle on all host cores (the reported value) and on one core."""
+    cores = host_cores()
+    d1, s1, _ = oracle_rate(inp, budget_s / 2, 1)
+    dn, sn, _ = oracle_rate(inp, budget_s / 2, cores)
+    return {"value": dn / sn, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "nproc": os.cpu_count(), "cpu_model": cpu_model(),
+            "one_core": {"value": d1 / s1, "cores": 1, "tokens": d1, "seconds": s1},
+            "sample": f"consecutive 256-token chunks of the workload, fwd + bwd, unmodified "
+                      f"fp64 C oracle; {cores} threads (one per core): {dn} tokens in "
+                      f"{sn:.1f} s; one thread: {d1} tokens in {s1:.1f} s"}
 
 
 cfg_args = None
-
-
-def bwd_kernel_name(w) -> str:
-    """The backward kernel the library launches for this shape (the pipelined
-    one: one row unit per lane, lanes per row the next power of two of
-    D / 16 bytes-pairs; 12 consumer and 4 producer warps; then the
-    mean-centred and tensor-copy flags, 0 and 0 for the dense RMSNorm form,
-    as ncu prints them)."""
-    dv2 = w.D // (2 * (16 // w.elem_bytes))
-    lpr = 1
-    while lpr < dv2:
-        lpr *= 2
-    tname = "__nv_bfloat16" if w.dtype == "bf16" else "float"
-    return f"qknr_bwd_pipe_kernel<{tname}, {lpr}, 12, 4, 0, 0>"
 
 
 def config_of(w, inp, world):
@@ -568,12 +690,14 @@ def config_of(w, inp, world):
 
 
 def run_reference(args, w, inp, rank, world):
-    """The reference arm: the CPU oracle as it stands, rank 0 only."""
+    """The reference arm: the CPU oracle as it stands, on every host core,
+    rank 0 only. A step is one round in which every core runs the oracle
+    (fwd + bwd) on the next 256-token chunk of the workload."""
     if rank != 0:
         return
-    per_step_tokens = 256
-    _, _, _ = oracle_sample_rate(inp, 1e9, per_step_tokens, max_calls=args.warmup)
-    done, spent, per_call = oracle_sample_rate(inp, 1e9, per_step_tokens, max_calls=args.steps)
+    cores = host_cores()
+    oracle_rate(inp, 0.0, cores, rounds=args.warmup)
+    done, spent, per_round = oracle_rate(inp, 0.0, cores, rounds=args.steps)
     v = done / spent
     ms = 1000.0 * spent / args.steps
     line = {
@@ -581,9 +705,11 @@ def run_reference(args, w, inp, rank, world):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": config_of(w, inp, 1),
-        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                         "sample": f"{per_step_tokens} consecutive tokens per step "
-                                   f"(fwd + bwd), single-threaded fp64 C"},
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "nproc": os.cpu_count(), "cpu_model": cpu_model(),
+                         "sample": f"each step: {cores} threads (one per core) each run the "
+                                   f"unmodified fp64 C oracle, fwd + bwd, on the next 256 "
+                                   f"consecutive tokens of the workload"},
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -598,6 +724,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=workloads.BENCH_WORKLOAD,
                     choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--seq-len", type=int, default=0,
+                    help="override S of the workload (smaller profiling captures; the "
+                         "line's config records it)")
     ap.add_argument("--sets", type=int, default=NSETS,
                     help="input sets in the ring (4 keeps inputs out of L2; 1 for small "
                          "profiling footprints)")
@@ -605,6 +734,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--per-config-steps", type=int, default=200,
+                    help="timed steps of each other workload in per_config")
+    ap.add_argument("--no-per-config", action="store_true")
     ap.add_argument("--variants", action="store_true",
                     help="also time the fused-QKV, NoPE and rotation-only entry points")
     ap.add_argument("--layout", choices=["dense", "qkv"], default="dense",
@@ -619,40 +751,47 @@ def main():
         ap.error("--warmup must be >= 3")
     rank, local_rank, world = env_rank()
     w = workloads.WORKLOADS[args.workload]
-    inp = workloads.make_inputs(w, seed=rank_seed(w, rank))
+    over = {"S": args.seq_len} if args.seq_len > 0 and not w.packed else {}
+    inp = workloads.make_inputs(w, seed=rank_seed(w, rank), **over)
     w = inp.w
+    main_inp_cache[0] = inp
 
     if args.impl == "reference":
         run_reference(args, w, inp, rank, world)
         return
 
     torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
     if world > 1:
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                             device_id=torch.device("cuda", local_rank))
+                                             device_id=dev)
     r = run_ours(args, w, inp, rank, local_rank, world)
-
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        done, spent, _ = oracle_sample_rate(inp, args.cpu_budget_s)
-        cpu = {"value": done / spent, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-               "sample": f"{done} consecutive tokens of the workload, fwd + bwd, "
-                         f"single-threaded fp64 C, {spent:.1f} s"}
     if world > 1:
         torch.distributed.destroy_process_group()
     if rank != 0:
         return
 
-    cb = workloads.contract_bytes(w, with_pos=inp.pos is not None)
     peak, peak_src = hbm_peak()
+    per_config = None
+    if world == 1 and not args.no_per_config:
+        per_config = run_per_config(args, w, r, rank, dev, peak)
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(inp, args.cpu_budget_s)
+
+    cb = workloads.contract_bytes(w, with_pos=inp.pos is not None)
     tokens = inp.real_tokens
     ms = r["total_ms"] / args.steps
     value = aggregate_tokens_per_s(world, tokens, ms)
     fwd_gbs = cb["fwd"] / (r["fwd_ms"] / 1e3) / 1e9
     bwd_gbs = cb["bwd"] / (r["bwd_ms"] / 1e3) / 1e9
     step_gbs = (cb["fwd"] + cb["bwd"]) / (ms / 1e3) / 1e9
-    bwd_kernel = bwd_kernel_name(w)
+    fwd_kernel, bwd_kernel = kernels_of(w, dev, args.layout)
+    # the dominant kernel: the one with the larger share of the step
+    dom = "bwd" if r["bwd_ms"] >= r["fwd_ms"] else "fwd"
+    dom_kernel = bwd_kernel if dom == "bwd" else fwd_kernel
+    dom_gbs = bwd_gbs if dom == "bwd" else fwd_gbs
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
@@ -669,13 +808,13 @@ def main():
                     "fwd_frac_of_copy": r["floor"]["fwd_ms"] / r["fwd_ms"],
                     "bwd_frac_of_copy": r["floor"]["bwd_ms"] / r["bwd_ms"]}},
         "fwd": {"ms": r["fwd_ms"], "tokens_per_s": aggregate_tokens_per_s(world, tokens, r["fwd_ms"]),
-                "bytes_per_launch": cb["fwd"]},
+                "bytes_per_launch": cb["fwd"], "kernel": fwd_kernel},
         "bwd": {"ms": r["bwd_ms"], "tokens_per_s": aggregate_tokens_per_s(world, tokens, r["bwd_ms"]),
-                "bytes_per_launch": cb["bwd"]},
-        "roofline": {"bound": "hbm", "kernel": bwd_kernel, "achieved": bwd_gbs, "peak": peak,
-                     "unit": "GB/s", "frac": bwd_gbs / peak,
-                     "traffic": ncu_traffic(bwd_kernel, w.name),
-                     "algorithmic_bytes": cb["bwd"], "peak_source": peak_src},
+                "bytes_per_launch": cb["bwd"], "kernel": bwd_kernel},
+        "roofline": {"bound": "hbm", "kernel": dom_kernel, "direction": dom, "achieved": dom_gbs,
+                     "peak": peak, "unit": "GB/s", "frac": dom_gbs / peak,
+                     "traffic": ncu_traffic(dom_kernel, w.name),
+                     "algorithmic_bytes": cb[dom], "peak_source": peak_src},
         "clocks": r["clocks"],
         "gpu_launches": 2 * args.steps,
     }
@@ -685,8 +824,10 @@ def main():
                        "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"],
                        "ms_per_step": e["ms"], "steps": e["steps"]}
     line["cpu_baseline"] = cpu
+    if per_config is not None:
+        line["per_config"] = per_config
     if args.variants and world == 1:
-        line["variants"] = run_variants(args, w, inp, torch.device("cuda", local_rank), peak)
+        line["variants"] = run_variants(args, w, inp, dev, peak)
     print(json.dumps(line), flush=True)
 
 

@@ -33,9 +33,14 @@
  * I/O dtype is fp32 or bf16 for all of q, k, gamma, outputs and gradients;
  * arithmetic is fp32 with fp64 rotary-angle reduction.
  *
- * Pointers. All pointers are device pointers (or managed memory) owned by
- * the caller; the library allocates nothing and keeps no state between
- * calls, so concurrent calls on different streams are safe. Vector pointers
+ * Pointers and state. All pointers are device pointers (or managed memory)
+ * owned by the caller; the library allocates no memory. It does keep a
+ * little state: per-device caches of the SM count, the shared-memory limit,
+ * kernel occupancy and kernel attributes (filled on first use, thread-safe),
+ * and one sticky device flag per kernel family that a kernel sets when it
+ * gives up a bounded internal wait (read and cleared by
+ * qknr_pipeline_error). Neither affects results, so concurrent calls on
+ * different streams are safe. Vector pointers
  * (q, k, gamma, outputs, gradients) must be 16-byte aligned; rstd, dgamma
  * and pos_ids 4-byte aligned. An output may alias its own input exactly
  * (q_out == q, dq == dq_out) for in-place use; any other overlap is rejected.
@@ -49,8 +54,9 @@
  * fault during execution surfaces at the caller's next synchronisation, as
  * for any CUDA launch. A launch the runtime refuses returns QKNR_ERR_CUDA.
  *
- * Limits. 2 <= D <= 256 with D * elem_bytes a multiple of 32 (two 16-byte
- * halves per lane); rotary_dim even, 0 <= rotary_dim <= D, and
+ * Limits. 2 <= D <= 256 with D * elem_bytes a multiple of 16 (whole 16-byte
+ * vectors; with an odd number of them per row the call runs the plain-load
+ * kernels); rotary_dim even, 0 <= rotary_dim <= D, and
  * (rotary_dim / 2) * elem_bytes a multiple of 16; theta finite and > 0;
  * eps finite and >= 0. Other shapes return QKNR_ERR_UNSUPPORTED or
  * QKNR_ERR_INVALID_ARG.
@@ -324,29 +330,6 @@ QKNR_API qknr_status qk_rope_apply(const void *q, const void *k,
  * dq = dq_out, dk = dk_out. T = 0 or no heads: nothing launched (the
  * backward still zeroes dgamma).
  */
-/*
- * Launch geometry of the layerwise pipelined kernels for a shape, for
- * inspection and host-side checks; no CUDA call is made. mode 0: the dots
- * (qk_layerwise_bwd_dots), 1: the backward (qk_layerwise_norm_rope_bwd);
- * sms: the SM count to plan for. geom (19 int64, caller-owned) receives
- *   [0] 1 if the pipelined kernel runs for this shape, 0 if the plain-load
- *       kernel does (then the rest is 0),
- *   [1] lanes per head row, [2] tokens per stage, [3] stages,
- *   [4] bytes per stage, [5..9] byte offsets within a stage of the K rows,
- *       dQ_out rows, dK_out rows, (cos, sin) table and per-token scalars,
- *   [10] offset of the per-token partial-sum table and [11] of the gamma
- *       table in the dynamic shared memory,
- *   [12] warps per token, [13] token groups, [14] head blocks,
- *   [15] tokens per CTA, [16] CTAs, [17] dynamic shared memory bytes,
- *   [18] threads per CTA.
- * Shapes are checked as for qk_layerwise_norm_rope_bwd (with the totals
- * equal to the local head counts); a bad mode, sms or NULL geom is
- * QKNR_ERR_INVALID_ARG.
- */
-QKNR_API qknr_status qk_layerwise_geometry(int mode, int B, int S, int Hq, int Hkv, int D,
-                             int rotary_dim, qknr_dtype dtype, int sms,
-                             int64_t *geom);
-
 QKNR_API qknr_status qk_layerwise_stats(const void *q, const void *k,
                              float *sumsq_q, float *sumsq_k,
                              int B, int S, int Hq, int Hkv, int D,
@@ -385,6 +368,59 @@ QKNR_API qknr_status qk_layerwise_norm_rope_bwd(const void *q, const void *k,
                              int Hq_total, int Hkv_total, int D,
                              int rotary_dim, float theta,
                              qknr_dtype dtype, qknr_stream_t stream);
+
+/*
+ * Launch geometry of the layerwise pipelined kernels for a shape, for
+ * inspection and host-side checks; no CUDA call is made. mode 0: the dots
+ * (qk_layerwise_bwd_dots), 1: the backward (qk_layerwise_norm_rope_bwd);
+ * sms: the SM count to plan for. geom (19 int64, caller-owned) receives
+ *   [0] 1 if the plan for `sms` SMs is the pipelined kernel, 0 if it is
+ *       the plain-load kernel (then the rest is 0); this is the plan the
+ *       library follows on a device with `sms` SMs unless the environment
+ *       variable QKNR_SIMPLE_KERNELS=1 forces the plain-load kernels,
+ *   [1] lanes per head row, [2] tokens per stage, [3] stages,
+ *   [4] bytes per stage, [5..9] byte offsets within a stage of the K rows,
+ *       dQ_out rows, dK_out rows, (cos, sin) table and per-token scalars,
+ *   [10] offset of the per-token partial-sum table and [11] of the gamma
+ *       table in the dynamic shared memory,
+ *   [12] warps per token, [13] token groups, [14] head blocks,
+ *   [15] tokens per CTA, [16] CTAs, [17] dynamic shared memory bytes,
+ *   [18] threads per CTA.
+ * Shapes are checked as for qk_layerwise_norm_rope_bwd (with the totals
+ * equal to the local head counts); a bad mode, sms or NULL geom is
+ * QKNR_ERR_INVALID_ARG.
+ */
+QKNR_API qknr_status qk_layerwise_geometry(int mode, int B, int S, int Hq, int Hkv, int D,
+                             int rotary_dim, qknr_dtype dtype, int sms,
+                             int64_t *geom);
+
+/*
+ * Launch plan of the per-head entry points for a shape, for inspection and
+ * host-side checks (profilers name the kernel by these template values); no
+ * CUDA call is made. kind 0: every forward form (qk_norm_rope_fwd and
+ * _strided, qk_norm_fwd, qk_rope_apply, qk_rms_stats); 1: the backward
+ * (qk_norm_rope_bwd and _strided, qk_norm_bwd); 2 / 3: the mean-centred
+ * forward / backward (qk_layernorm_rope_*). strided: bit 0 (1) when q (k)
+ * has a token stride other than its dense one. sms: the SM count to plan
+ * for; smem_optin: shared memory per block available by opt-in (0: 227 KB,
+ * B200's). plan (14 int64, caller-owned) receives
+ *   [0] 1 if the plan is the pipelined kernel, 0 if the plain-load kernel
+ *       (then only [1], [2], [5] and [13] are set); the library follows it
+ *       on a device with these limits unless QKNR_SIMPLE_KERNELS=1,
+ *   [1] lanes per head row, [2] units (pairs of 16-byte vectors) per lane,
+ *   [3] consumer warps, [4] producer warps, [5] 1 if mean-centred,
+ *   [6] tensor-copy mask (bit 0 q, bit 1 k), [7] tokens per tile,
+ *   [8] stages in the ring, [9] bytes per stage, [10] tokens per CTA,
+ *   [11] CTAs, [12] dynamic shared memory bytes, [13] threads per CTA.
+ * The pipelined kernels are named qknr_fwd_pipe_kernel<T, [1], [2], [3],
+ * [4], [5], [6] != 0> and qknr_bwd_pipe_kernel<T, [1], [3], [4], [5],
+ * [6] != 0>. Shapes are checked as for the entry points; a bad kind,
+ * strided, sms or NULL plan is QKNR_ERR_INVALID_ARG. B * S == 0 or no heads:
+ * all zeros.
+ */
+QKNR_API qknr_status qk_norm_rope_plan(int kind, int B, int S, int Hq, int Hkv, int D,
+                             int rotary_dim, qknr_dtype dtype, int strided, int sms,
+                             int smem_optin, int64_t *plan);
 
 /* Static English text for a status code; never NULL. */
 QKNR_API const char *qknr_strerror(qknr_status status);

@@ -31,7 +31,7 @@ __all__ = ["qk_norm_rope_fwd", "qk_norm_rope_bwd", "qknr_strerror", "QKNormRoPE"
            "qk_norm_rope", "QKNRError", "library_path", "load_library", "pipeline_error",
            "qk_layerwise_stats", "qk_layerwise_norm_rope_fwd", "qk_layerwise_bwd_dots",
            "qk_layerwise_norm_rope_bwd", "QKLayerwiseNormRoPE", "qk_layerwise_norm_rope",
-           "all_reduce_stats", "layerwise_geometry"]
+           "all_reduce_stats", "layerwise_geometry", "launch_plan", "kernel_name"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libqknr.so")
@@ -97,6 +97,8 @@ def load_library():
     lib.qk_layerwise_norm_rope_bwd.argtypes = [vp] * 15 + [i32] * 8 + [f32, i32, vp]
     lib.qk_layerwise_geometry.restype = i32
     lib.qk_layerwise_geometry.argtypes = [i32] * 9 + [vp]
+    lib.qk_norm_rope_plan.restype = i32
+    lib.qk_norm_rope_plan.argtypes = [i32] * 11 + [vp]
     lib.qknr_strerror.restype = ctypes.c_char_p
     lib.qknr_strerror.argtypes = [i32]
     lib.qknr_last_cuda_error.restype = i32
@@ -831,3 +833,40 @@ def layerwise_geometry(mode: str, B: int, S: int, Hq: int, Hkv: int, D: int, rot
     if st != QKNR_OK:
         raise QKNRError(st, "qk_layerwise_geometry")
     return dict(zip(_GEOM_KEYS, (int(v) for v in out)))
+
+
+_PLAN_KEYS = ("pipelined", "lpr", "units", "consumer_warps", "producer_warps", "ln", "tmap",
+              "TT", "NS", "stage_bytes", "tpc", "grid", "smem", "threads")
+_PLAN_KINDS = {"fwd": 0, "bwd": 1, "ln_fwd": 2, "ln_bwd": 3}
+
+
+def launch_plan(kind: str, B: int, S: int, Hq: int, Hkv: int, D: int, rotary_dim: int,
+                dtype=torch.bfloat16, strided: int = 0, sms: int = 148,
+                smem_optin: int = 0) -> dict:
+    """Launch plan of the per-head entry points (C ``qk_norm_rope_plan``; host
+    only, no GPU): ``kind`` is "fwd", "bwd", "ln_fwd" or "ln_bwd"."""
+    lib = load_library()
+    out = (ctypes.c_int64 * len(_PLAN_KEYS))()
+    st = lib.qk_norm_rope_plan(_PLAN_KINDS[kind], B, S, Hq, Hkv, D, rotary_dim, _DTYPES[dtype],
+                               strided, sms, smem_optin, ctypes.cast(out, ctypes.c_void_p))
+    if st != QKNR_OK:
+        raise QKNRError(st, "qk_norm_rope_plan")
+    return dict(zip(_PLAN_KEYS, (int(v) for v in out)))
+
+
+def kernel_name(kind: str, B: int, S: int, Hq: int, Hkv: int, D: int, rotary_dim: int,
+                dtype=torch.bfloat16, strided: int = 0, sms: int = 148,
+                smem_optin: int = 0) -> str:
+    """The kernel a call of this shape launches, named as profilers print it
+    (template arguments included), from the library's own launch plan."""
+    p = launch_plan(kind, B, S, Hq, Hkv, D, rotary_dim, dtype, strided, sms, smem_optin)
+    t = "__nv_bfloat16" if dtype == torch.bfloat16 else "float"
+    bwd = kind.endswith("bwd")
+    if not p["pipelined"]:
+        return f"qknr_{'bwd' if bwd else 'fwd'}_kernel<{t}, {p['lpr']}, {p['ln']}>"
+    tm = int(p["tmap"] != 0)
+    if bwd:
+        return (f"qknr_bwd_pipe_kernel<{t}, {p['lpr']}, {p['consumer_warps']}, "
+                f"{p['producer_warps']}, {p['ln']}, {tm}>")
+    return (f"qknr_fwd_pipe_kernel<{t}, {p['lpr']}, {p['units']}, {p['consumer_warps']}, "
+            f"{p['producer_warps']}, {p['ln']}, {tm}>")

@@ -70,7 +70,7 @@ qknr_status check_shape(int B, int S, int Hq, int Hkv, int D, int R,
     if (!(eps >= 0.f) || !std::isfinite(eps)) return QKNR_ERR_INVALID_ARG;
     const int e = dtype == QKNR_F32 ? 4 : 2;
     if (D > kMaxD) return QKNR_ERR_UNSUPPORTED;
-    if ((D * e) % 32 != 0) return QKNR_ERR_UNSUPPORTED;
+    if ((D * e) % 16 != 0) return QKNR_ERR_UNSUPPORTED;
     if (((R / 2) * e) % 16 != 0) return QKNR_ERR_UNSUPPORTED;
     return QKNR_OK;
 }
@@ -91,13 +91,17 @@ qknr_status check_overlaps(const Span *all, int n_all, int first_out, const int 
     return QKNR_OK;
 }
 
-int lanes_per_row(int D, int e) {
-    const int V = 16 / e;
-    const int units = D / (2 * V);
+// Units (pairs of 16-byte vectors) of a row: an odd count of vectors leaves
+// the last pass-through unit with one vector.
+int units_per_row(int D, int e) { return (D / (16 / e) + 1) / 2; }
+
+int next_pow2(int x) {
     int l = 1;
-    while (l < units) l <<= 1;
+    while (l < x) l <<= 1;
     return l;
 }
+
+int lanes_per_row(int D, int e) { return next_pow2(units_per_row(D, e)); }
 
 // Occupancy (resident CTAs per SM) of one kernel on one device. `cache` is
 // owned by the kernel's launcher (one array per template instantiation).
@@ -160,6 +164,10 @@ constexpr int kBwdPipeWarps = QKNR_BWD_PIPE_WARPS;
 constexpr int kBwdPipeWarpsLN = 12;
 constexpr int kFwdPipeWarpsLN = 12;
 constexpr int kProducerWarps = QKNR_PRODUCER_WARPS;  // copy issue + rotary tables
+constexpr int fwd_pipe_warps(int lpr, int u, bool ln) {
+    return ln ? kFwdPipeWarpsLN : (lpr * u <= 4 ? kFwdPipeWarpsShortRow : kFwdPipeWarps);
+}
+constexpr int bwd_pipe_warps(bool ln) { return ln ? kBwdPipeWarpsLN : kBwdPipeWarps; }
 #ifndef QKNR_STAGE_TARGET_BYTES
 #define QKNR_STAGE_TARGET_BYTES 81920
 #endif
@@ -168,6 +176,8 @@ constexpr int kProducerWarps = QKNR_PRODUCER_WARPS;  // copy issue + rotary tabl
 // copy and each full/empty hand-off has a fixed cost.
 constexpr int kStageTargetBytes = QKNR_STAGE_TARGET_BYTES;
 constexpr int kStaticSmemReserve = 8192; // barriers, angle steps, gamma, dgamma tables
+constexpr int kDefaultSmemOptin = 232448;  // B200: 227 KB of shared memory per block, opt-in
+constexpr int kPlanLen = 14;             // entries qk_norm_rope_plan writes
 
 int align128(int x) { return (x + 127) & ~127; }
 
@@ -184,11 +194,30 @@ int max_dyn_smem(int dev) {
     return n;
 }
 
+// The launch plan of one call: which kernel runs and with what geometry.
+// The dispatch below and the qk_norm_rope_plan query both come from here.
+struct Plan {
+    bool pipe;        // the pipelined kernel (else the plain-load one)
+    int lpr, u;       // lanes per head row, units per lane
+    int ncw, npw;     // consumer and producer warps
+    bool ln;          // mean-centred instantiation
+    PipeGeom g;
+    int grid, smem, threads;
+};
+
 // Tile and ring sizes for one problem; false when the pipelined kernels do
-// not apply (a token too large for two stages, or unaligned rstd buffers).
-bool pipe_geometry(bool bwd, int64_t T, int Hq, int Hkv, int D, int R, int esz, int dev,
-                   const void *rq, const void *rk, PipeGeom *g, int *grid, int *smem) {
+// not apply (an odd number of 16-byte vectors per row, a token too large for
+// two stages, or unaligned rstd buffers). `sms` CTAs at most, `optin` bytes
+// of shared memory per block.
+bool plan_pipe(bool bwd, bool ln, int64_t T, int Hq, int Hkv, int D, int R, int esz, int sms,
+               int optin, const void *rq, const void *rk, Plan *p) {
     const int rowb = D * esz, H = Hq + Hkv, half = R / 2;
+    const int units = units_per_row(D, esz);
+    *p = Plan{};
+    p->lpr = next_pow2(units);
+    p->u = 1;
+    p->threads = kThreads;
+    if ((D / (16 / esz)) & 1) return false;  // a half unit: the plain-load kernels take it
     if (bwd && ((rq && ((uintptr_t)rq & 15)) || (rk && ((uintptr_t)rk & 15)))) return false;
     // backward tiles must start rstd blocks on 16-byte boundaries
     int m = 1;
@@ -221,22 +250,32 @@ bool pipe_geometry(bool bwd, int64_t T, int Hq, int Hkv, int D, int R, int esz, 
         off = align128(off + TT * Hkv * 4);
     }
     q.stage_bytes = off > 0 ? off : 128;
-    const int budget = max_dyn_smem(dev) - kStaticSmemReserve;
+    const int budget = optin - kStaticSmemReserve;
     int NS = budget / q.stage_bytes;
     if (NS > kMaxStages) NS = kMaxStages;
     if (NS < 2) return false;
     q.NS = NS;
     // one CTA per SM; each owns a contiguous run of tokens (a multiple of m)
-    const int64_t sms = sm_count(dev);
     int64_t tpc = (T + sms - 1) / sms;
     tpc = ((tpc + m - 1) / m) * m;
     if (tpc < 1) tpc = 1;
     q.tpc = tpc;
     q.mq = Hq > 1 ? (uint32_t)(0x100000000ull / (uint64_t)Hq + 1) : 0u;
     q.mk = Hkv > 1 ? (uint32_t)(0x100000000ull / (uint64_t)Hkv + 1) : 0u;
-    *grid = (int)((T + tpc - 1) / tpc);
-    *smem = NS * q.stage_bytes;
-    *g = q;
+    // the kernel instantiation: two units per lane once a forward row has
+    // three or more (halving the per-row overhead per element)
+    if (!bwd && units >= 3) {
+        p->u = 2;
+        p->lpr = next_pow2((units + 1) / 2);
+    }
+    p->ncw = bwd ? bwd_pipe_warps(ln) : fwd_pipe_warps(p->lpr, p->u, ln);
+    p->npw = kProducerWarps;
+    p->ln = ln;
+    p->pipe = true;
+    p->g = q;
+    p->grid = (int)((T + tpc - 1) / tpc);
+    p->smem = NS * q.stage_bytes;
+    p->threads = (p->ncw + p->npw) * 32;
     return true;
 }
 
@@ -313,7 +352,7 @@ qknr_status launch_fwd_pipe_tm(const FwdArgs &a, const PipeGeom &g, const CUtens
                                const CUtensorMap &mk, int grid, int smem, int dev, cudaStream_t st,
                                bool *launched) {
     static std::atomic<int> smem_ok[64];
-    constexpr int NCW = LN ? kFwdPipeWarpsLN : (LPR * U <= 4 ? kFwdPipeWarpsShortRow : kFwdPipeWarps);
+    constexpr int NCW = fwd_pipe_warps(LPR, U, LN);
     auto kern = qknr_fwd_pipe_kernel<T, LPR, U, NCW, kProducerWarps, LN, TM>;
     *launched = false;
     if (!allow_dyn_smem((const void *)kern, dev, smem_ok, smem)) return QKNR_OK;
@@ -330,7 +369,7 @@ qknr_status launch_bwd_pipe_tm(const BwdArgs &a, const PipeGeom &g, const CUtens
                                const CUtensorMap &mk, int grid, int smem, int dev, cudaStream_t st,
                                bool *launched) {
     static std::atomic<int> smem_ok[64];
-    constexpr int NCW = LN ? kBwdPipeWarpsLN : kBwdPipeWarps;
+    constexpr int NCW = bwd_pipe_warps(LN);
     auto kern = qknr_bwd_pipe_kernel<T, LPR, NCW, kProducerWarps, LN, TM>;
     *launched = false;
     if (!allow_dyn_smem((const void *)kern, dev, smem_ok, smem)) return QKNR_OK;
@@ -367,39 +406,32 @@ qknr_status launch_bwd_pipe(const BwdArgs &a, const PipeGeom &g, const CUtensorM
     return launch_bwd_pipe_tm<T, LPR, LN, false>(a, g, mq, mk, grid, smem, dev, st, launched);
 }
 
-int next_pow2(int x) {
-    int l = 1;
-    while (l < x) l <<= 1;
-    return l;
-}
-
-// Pipelined forward when it applies: two units per lane once a row has
-// three or more (halving the per-row overhead per element).
+// Pipelined forward when the plan takes it.
 template <typename T, bool LN>
 bool try_fwd_pipe(const FwdArgs &a, cudaStream_t st, qknr_status *status) {
     int dev = 0;
     cudaGetDevice(&dev);
-    PipeGeom g;
-    int grid, smem;
+    Plan p;
     if (pipe_disabled() ||
-        !pipe_geometry(false, a.T, a.Hq, a.Hkv, a.D, a.R, (int)sizeof(T), dev, nullptr, nullptr,
-                       &g, &grid, &smem))
+        !plan_pipe(false, LN, a.T, a.Hq, a.Hkv, a.D, a.R, (int)sizeof(T), sm_count(dev),
+                   max_dyn_smem(dev), nullptr, nullptr, &p))
         return false;
+    PipeGeom g = p.g;
     CUtensorMap mq, mk;
     g.tmap = input_maps(a.q, a.k, a.qts, a.kts, a.Hq, a.Hkv, a.D, (int)sizeof(T), a.T, g.TT, &mq, &mk);
     if (g.tmap < 0) return false;
-    const int dv2 = a.D / (2 * (16 / (int)sizeof(T)));
+    const int grid = p.grid, smem = p.smem;
     bool launched = false;
     qknr_status s = QKNR_OK;
-    if (dv2 >= 3) {
-        switch (next_pow2((dv2 + 1) / 2)) {
+    if (p.u == 2) {
+        switch (p.lpr) {
             case 2: s = launch_fwd_pipe<T, 2, 2, LN>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
             case 4: s = launch_fwd_pipe<T, 4, 2, LN>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
             case 8: s = launch_fwd_pipe<T, 8, 2, LN>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
             case 16: s = launch_fwd_pipe<T, 16, 2, LN>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
         }
     } else {
-        switch (next_pow2(dv2)) {
+        switch (p.lpr) {
             case 1: s = launch_fwd_pipe<T, 1, 1, LN>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
             case 2: s = launch_fwd_pipe<T, 2, 1, LN>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
         }
@@ -412,19 +444,19 @@ template <typename T, bool LN>
 bool try_bwd_pipe(const BwdArgs &a, cudaStream_t st, qknr_status *status) {
     int dev = 0;
     cudaGetDevice(&dev);
-    PipeGeom g;
-    int grid, smem;
+    Plan p;
     if (pipe_disabled() ||
-        !pipe_geometry(true, a.T, a.Hq, a.Hkv, a.D, a.R, (int)sizeof(T), dev, a.rq, a.rk, &g,
-                       &grid, &smem))
+        !plan_pipe(true, LN, a.T, a.Hq, a.Hkv, a.D, a.R, (int)sizeof(T), sm_count(dev),
+                   max_dyn_smem(dev), a.rq, a.rk, &p))
         return false;
+    PipeGeom g = p.g;
     CUtensorMap mq, mk;
     g.tmap = input_maps(a.q, a.k, a.qts, a.kts, a.Hq, a.Hkv, a.D, (int)sizeof(T), a.T, g.TT, &mq, &mk);
     if (g.tmap < 0) return false;
-    const int dv2 = a.D / (2 * (16 / (int)sizeof(T)));
+    const int grid = p.grid, smem = p.smem;
     bool launched = false;
     qknr_status s = QKNR_OK;
-    switch (next_pow2(dv2)) {
+    switch (p.lpr) {
         case 1: s = launch_bwd_pipe<T, 1, LN>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
         case 2: s = launch_bwd_pipe<T, 2, LN>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
         case 4: s = launch_bwd_pipe<T, 4, LN>(a, g, mq, mk, grid, smem, dev, st, &launched); break;
@@ -743,12 +775,42 @@ extern "C" qknr_status qk_rope_apply(const void *q, const void *k, const int32_t
                     stream, mode);
 }
 
+extern "C" qknr_status qk_norm_rope_plan(int kind, int B, int S, int Hq, int Hkv, int D,
+                                         int rotary_dim, qknr_dtype dtype, int strided, int sms,
+                                         int smem_optin, int64_t *plan) {
+    if (!plan || kind < 0 || kind > 3 || strided < 0 || strided > 3 || sms < 1 ||
+        smem_optin < 0)
+        return QKNR_ERR_INVALID_ARG;
+    const qknr_status st = check_shape(B, S, Hq, Hkv, D, rotary_dim, 1.f, 0.f, dtype);
+    if (st != QKNR_OK) return st;
+    for (int i = 0; i < kPlanLen; ++i) plan[i] = 0;
+    const int64_t T = (int64_t)B * S;
+    const int esz = dtype == QKNR_F32 ? 4 : 2;
+    if (T == 0 || Hq + Hkv == 0) return QKNR_OK;
+    Plan p;
+    const bool bwd = kind & 1, ln = (kind & 2) != 0;
+    if (!plan_pipe(bwd, ln, T, Hq, Hkv, D, rotary_dim, esz, sms,
+                   smem_optin ? smem_optin : kDefaultSmemOptin, nullptr, nullptr, &p)) {
+        plan[1] = lanes_per_row(D, esz);
+        plan[2] = 1;
+        plan[5] = ln;
+        plan[13] = kThreads;
+        return QKNR_OK;
+    }
+    // tensor copies serve strided inputs of the RMSNorm forms only
+    const int tm = ln ? 0 : ((strided & 1) && Hq ? 1 : 0) | ((strided & 2) && Hkv ? 2 : 0);
+    const int64_t v[kPlanLen] = {1, p.lpr, p.u, p.ncw, p.npw, p.ln, tm, p.g.TT, p.g.NS,
+                                 p.g.stage_bytes, p.g.tpc, p.grid, p.smem, p.threads};
+    for (int i = 0; i < kPlanLen; ++i) plan[i] = v[i];
+    return QKNR_OK;
+}
+
 extern "C" const char *qknr_strerror(qknr_status s) {
     switch (s) {
         case QKNR_OK: return "success";
         case QKNR_ERR_INVALID_ARG: return "invalid argument (size, NULL pointer, overlap, theta or eps)";
         case QKNR_ERR_ALIGNMENT: return "pointer not aligned (16 bytes for vectors, 4 for fp32/int32 arrays)";
-        case QKNR_ERR_UNSUPPORTED: return "unsupported shape (D <= 256, D*elem a multiple of 32, (R/2)*elem a multiple of 16)";
+        case QKNR_ERR_UNSUPPORTED: return "unsupported shape (D <= 256, D*elem a multiple of 16, (R/2)*elem a multiple of 16)";
         case QKNR_ERR_CUDA: return "the CUDA runtime refused the launch (see qknr_last_cuda_error)";
     }
     return "unknown status";

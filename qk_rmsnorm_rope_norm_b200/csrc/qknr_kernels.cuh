@@ -186,24 +186,31 @@ __device__ __forceinline__ void fill_tables(double *s_omega, float (*s_g)[kMaxD]
 }
 
 // Geometry of unit w of a head row of D elements (R rotary, V elements per
-// 16-byte vector): the element offsets of its two vectors. Units past the
-// row (D / 2V not a power of two) are off and point at element 0.
+// 16-byte vector): the element offsets of its two vectors. The R / V rotary
+// vectors form R / 2V units (w, w + R / 2V), so every rotary pair (i, i + R/2)
+// sits in one unit; the P pass-through vectors form ceil(P / 2) units
+// (j, j + ceil(P / 2)) after them. With P odd the last pass-through unit has
+// no second vector (onB false; eB then repeats eA and must not be used).
+// Units past the row (the unit count not a power of two) are off and point
+// at element 0.
 template <int V> struct UnitGeom {
-    bool on, rot;
+    bool on, rot, onB;
     int eA, eB;
     __device__ __forceinline__ UnitGeom(int w, int D, int R) {
-        const int Dv2 = D / (2 * V), Rv2 = R / (2 * V);
-        on = w < Dv2;
+        const int Rv2 = R / (2 * V), P = D / V - 2 * Rv2, hp = (P + 1) >> 1;
+        const int j = w - Rv2;
+        on = w < Rv2 + hp;
         rot = w < Rv2;
-        eA = on ? (rot ? w : w + Rv2) * V : 0;
-        eB = on ? (rot ? w + Rv2 : w + Dv2) * V : 0;
+        onB = rot || (on && j + hp < P);
+        eA = on ? (rot ? w : 2 * Rv2 + j) * V : 0;
+        eB = onB ? (rot ? w + Rv2 : 2 * Rv2 + j + hp) * V : eA;
     }
 };
 
 // Lane geometry: LPR lanes per row, lane u of the group owns unit u.
 template <int LPR, int V> struct Lane {
     int u, slot;
-    bool on, rot;
+    bool on, rot, onB;
     int eA, eB;  // element offsets of the lane's two vectors
     __device__ __forceinline__ Lane(int lane, int D, int R) {
         u = lane & (LPR - 1);
@@ -211,6 +218,7 @@ template <int LPR, int V> struct Lane {
         const UnitGeom<V> G(u, D, R);
         on = G.on;
         rot = G.rot;
+        onB = G.onB;
         eA = G.eA;
         eB = G.eB;
     }
@@ -288,7 +296,7 @@ qknr_fwd_kernel(const FwdArgs a) {
                 if (L.on && h < H) {
                     const char *row = h < a.Hq ? qrow + h * rowb : krow + (h - a.Hq) * rowb;
                     xa[pp] = ld16(row + offA);
-                    xb[pp] = ld16(row + offB);
+                    if (L.onB) xb[pp] = ld16(row + offB);  // a half unit keeps B = 0
                 }
             }
         };
@@ -319,7 +327,10 @@ qknr_fwd_kernel(const FwdArgs a) {
                 for (int k2 = 0; k2 < V / 2; ++k2) {
                     float2 va = IO::get2(xa[pp], k2), vb = IO::get2(xb[pp], k2);
                     if (LN && L.on) {
-                        va.x -= mu; va.y -= mu; vb.x -= mu; vb.y -= mu;
+                        va.x -= mu; va.y -= mu;
+                        if (L.onB) {
+                            vb.x -= mu; vb.y -= mu;
+                        }
                     }
                     ss = fmaf(va.x, va.x, ss); ss = fmaf(va.y, va.y, ss);
                     ss = fmaf(vb.x, vb.x, ss); ss = fmaf(vb.y, vb.y, ss);
@@ -351,7 +362,7 @@ qknr_fwd_kernel(const FwdArgs a) {
                     char *out = (char *)(isq ? a.qo : a.ko) + rowi * rowb;
                     if (!(a.mode & kModeStatsOnly)) {
                         st16(out + offA, ya);
-                        st16(out + offB, yb);
+                        if (L.onB) st16(out + offB, yb);
                     }
                     if (L.u == 0 && !(a.mode & kModeRopeOnly)) (isq ? a.rq : a.rk)[rowi] = r;
                 }
@@ -426,9 +437,11 @@ qknr_bwd_kernel(const BwdArgs a) {
                     const char *xrow = (const char *)(isq ? a.q : a.k) + t * (isq ? a.qts : a.kts) + hh * rowb;
                     const char *drow = (const char *)(isq ? a.dqo : a.dko) + rowi * rowb;
                     xa[pp] = ld16(xrow + offA);
-                    xb[pp] = ld16(xrow + offB);
                     da[pp] = ld16(drow + offA);
-                    db[pp] = ld16(drow + offB);
+                    if (L.onB) {  // a half unit keeps B = 0 (no gradient, no dgamma term)
+                        xb[pp] = ld16(xrow + offB);
+                        db[pp] = ld16(drow + offB);
+                    }
                     rr[pp] = (isq ? a.rq : a.rk)[rowi];
                 }
             }
@@ -472,7 +485,7 @@ qknr_bwd_kernel(const BwdArgs a) {
                             const float2 c = lane_cs(cs, L.rot, L.eA + e);
                             const float dA = q ? da2.y : da2.x, dB = q ? db2.y : db2.x;
                             const float xA = ((q ? xa2.y : xa2.x) - mu) * r;
-                            const float xB = ((q ? xb2.y : xb2.x) - mu) * r;
+                            const float xB = L.onB ? ((q ? xb2.y : xb2.x) - mu) * r : 0.f;
                             const float gA = fmaf(dA, c.x, dB * c.y);
                             const float gB = fmaf(dB, c.x, -dA * c.y);
                             tA[e & 3] = gA * xA;
@@ -506,7 +519,7 @@ qknr_bwd_kernel(const BwdArgs a) {
                             const float2 c = lane_cs(cs, L.rot, L.eA + e);
                             const float dA = q ? da2.y : da2.x, dB = q ? db2.y : db2.x;
                             const float xA = ((q ? xa2.y : xa2.x) - mu) * r;
-                            const float xB = ((q ? xb2.y : xb2.x) - mu) * r;
+                            const float xB = L.onB ? ((q ? xb2.y : xb2.x) - mu) * r : 0.f;
                             const float hA = fmaf(dA, c.x, dB * c.y) * g[L.eA + e];
                             const float hB = fmaf(dB, c.x, -dA * c.y) * g[L.eB + e];
                             outA[q] = r * fmaf(-xA, dot, LN ? hA - mh : hA);
@@ -518,7 +531,7 @@ qknr_bwd_kernel(const BwdArgs a) {
                     const int hh = isq ? h : h - a.Hq;
                     char *out = (char *)(isq ? a.dq : a.dk) + t * (isq ? a.dqts : a.dkts) + hh * rowb;
                     st16(out + offA, oa);
-                    st16(out + offB, ob);
+                    if (L.onB) st16(out + offB, ob);
                 }
             }
         }
@@ -546,7 +559,7 @@ qknr_bwd_kernel(const BwdArgs a) {
 #pragma unroll
             for (int e = 0; e < V; ++e) {
                 atomicAdd(&s_dg[z][L.eA + e], v[e]);
-                atomicAdd(&s_dg[z][L.eB + e], v[V + e]);
+                if (L.onB) atomicAdd(&s_dg[z][L.eB + e], v[V + e]);
             }
         }
     }

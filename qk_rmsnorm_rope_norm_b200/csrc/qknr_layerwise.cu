@@ -103,7 +103,7 @@ __device__ __forceinline__ float2 token_sumsq(const LwArgs &a, const Lane<LPR, I
         const int h = p + L.slot;
         if (!(L.on && h < H)) continue;
         const char *row = row_of<T>(a.q, a.k, a, t, h);
-        const Vec16 xa = ld16(row + offA), xb = ld16(row + offB);
+        const Vec16 xa = ld16(row + offA), xb = L.onB ? ld16(row + offB) : zero16();
         float s = 0.f;
 #pragma unroll
         for (int k2 = 0; k2 < V / 2; ++k2) {
@@ -136,9 +136,10 @@ __device__ __forceinline__ float2 token_dots(const LwArgs &a, const Lane<LPR, Io
         const char *row = (const char *)(isq ? a.q : a.k) + ri * rowb;
         const char *drow = (const char *)(isq ? a.dqo : a.dko) + ri * rowb;
         const char *grow = (const char *)(isq ? a.gq : a.gk) + hh * rowb;
-        const Vec16 xa = ld16(row + offA), xb = ld16(row + offB);
-        const Vec16 da = ld16(drow + offA), db = ld16(drow + offB);
-        const Vec16 ga = ld16(grow + offA), gb = ld16(grow + offB);
+        // a half unit (odd vector count) keeps its B vectors at zero
+        const Vec16 xa = ld16(row + offA), xb = L.onB ? ld16(row + offB) : zero16();
+        const Vec16 da = ld16(drow + offA), db = L.onB ? ld16(drow + offB) : zero16();
+        const Vec16 ga = ld16(grow + offA), gb = L.onB ? ld16(grow + offB) : zero16();
         float dot = 0.f;
 #pragma unroll
         for (int k2 = 0; k2 < V / 2; ++k2) {
@@ -223,8 +224,8 @@ __global__ void __launch_bounds__(kThreads) qknr_lw_fwd_kernel(const LwArgs a) {
             const int64_t ri = (isq ? t * a.Hq : t * a.Hkv) + hh;
             const char *row = (const char *)(isq ? a.q : a.k) + ri * rowb;
             const char *grow = (const char *)(isq ? a.gq : a.gk) + hh * rowb;
-            const Vec16 xa = ld16(row + offA), xb = ld16(row + offB);
-            const Vec16 ga = ld16(grow + offA), gb = ld16(grow + offB);
+            const Vec16 xa = ld16(row + offA), xb = L.onB ? ld16(row + offB) : zero16();
+            const Vec16 ga = ld16(grow + offA), gb = L.onB ? ld16(grow + offB) : zero16();
             const float r = isq ? rq : rk;
             Vec16 ya, yb;
 #pragma unroll
@@ -240,7 +241,7 @@ __global__ void __launch_bounds__(kThreads) qknr_lw_fwd_kernel(const LwArgs a) {
             }
             char *out = (char *)(isq ? a.qo : a.ko) + ri * rowb;
             st16(out + offA, ya);
-            st16(out + offB, yb);
+            if (L.onB) st16(out + offB, yb);
         }
     }
 }
@@ -316,9 +317,9 @@ __global__ void __launch_bounds__(kThreads) qknr_lw_bwd_kernel(const LwArgs a) {
             const char *row = (const char *)(isq ? a.q : a.k) + ri * rowb;
             const char *drow = (const char *)(isq ? a.dqo : a.dko) + ri * rowb;
             const char *grow = (const char *)(isq ? a.gq : a.gk) + hh * rowb;
-            const Vec16 xa = ld16(row + offA), xb = ld16(row + offB);
-            const Vec16 da = ld16(drow + offA), db = ld16(drow + offB);
-            const Vec16 ga = ld16(grow + offA), gb = ld16(grow + offB);
+            const Vec16 xa = ld16(row + offA), xb = L.onB ? ld16(row + offB) : zero16();
+            const Vec16 da = ld16(drow + offA), db = L.onB ? ld16(drow + offB) : zero16();
+            const Vec16 ga = ld16(grow + offA), gb = L.onB ? ld16(grow + offB) : zero16();
             const float r = isq ? rq : rk, nd = isq ? nq : nk;
             float *dg = s_dg + (isq ? 0 : a.Hq * a.D) + hh * a.D;
             Vec16 oa, ob;
@@ -339,14 +340,14 @@ __global__ void __launch_bounds__(kThreads) qknr_lw_bwd_kernel(const LwArgs a) {
                     outA[q] = r * fmaf(xA, nd, hA);
                     outB[q] = r * fmaf(xB, nd, hB);
                     atomicAdd(dg + L.eA + e, gA * xA * r);
-                    atomicAdd(dg + L.eB + e, gB * xB * r);
+                    if (L.onB) atomicAdd(dg + L.eB + e, gB * xB * r);
                 }
                 IO::put2(oa, k2, outA[0], outA[1]);
                 IO::put2(ob, k2, outB[0], outB[1]);
             }
             char *out = (char *)(isq ? a.qo : a.ko) + ri * rowb;
             st16(out + offA, oa);
-            st16(out + offB, ob);
+            if (L.onB) st16(out + offB, ob);
         }
     }
     __syncthreads();
@@ -854,9 +855,9 @@ __global__ void __launch_bounds__((kLwCWMax + 1) * 32, 1)
 }
 
 int lpr_of(int D, int esz) {
-    const int dv2 = D / (2 * (16 / esz));
+    const int units = (D / (16 / esz) + 1) / 2;  // the last one may be a half unit
     int l = 1;
-    while (l < dv2) l <<= 1;
+    while (l < units) l <<= 1;
     return l;
 }
 
@@ -896,6 +897,7 @@ bool simple_kernels_forced() {
 // instead).
 bool lw_plan(int mode, const LwArgs &a, int esz, int lpr, int sms, LwGeom *g, int *grid,
              int *smem, int *threads) {
+    if ((a.D / (16 / esz)) & 1) return false;  // a half unit: the plain-load kernels take it
     const int slots = 32 / lpr, H = a.Hq + a.Hkv;
     const int HB = (H + slots - 1) / slots;
     // head blocks per warp, warps per token, token groups: every warp owns
@@ -1019,7 +1021,7 @@ qknr_status lw_check(int B, int S, int Hq, int Hkv, int Hq_total, int Hkv_total,
     if (!(theta > 0.f) || !(theta < 3.0e38f)) return QKNR_ERR_INVALID_ARG;
     if (!(eps >= 0.f) || !(eps < 3.0e38f)) return QKNR_ERR_INVALID_ARG;
     const int e = dtype == QKNR_F32 ? 4 : 2;
-    if (D > kMaxD || (D * e) % 32 != 0 || ((R / 2) * e) % 16 != 0) return QKNR_ERR_UNSUPPORTED;
+    if (D > kMaxD || (D * e) % 16 != 0 || ((R / 2) * e) % 16 != 0) return QKNR_ERR_UNSUPPORTED;
     return QKNR_OK;
 }
 

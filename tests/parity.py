@@ -3,12 +3,14 @@
 Tolerances (written here, used by every parity test):
 
 * fp32 I/O: max-abs 1e-5 on q_out, k_out, dq, dk.
-* bf16 I/O: max-abs 2e-2 on elements whose oracle value is "of order 1"
-  (|ref| < 4, where half a bf16 ulp is at most 1/64); on every element the
-  GPU value must be within one bf16 ulp of the exact value (faithful
-  rounding: the fp32 result rounded once to nearest even), with an absolute
-  floor of 1e-5 for values near zero. Above |ref| = 8 half an ulp alone is
-  1/32 > 2e-2, so faithful rounding is the meaningful bound there.
+* bf16 I/O: max-abs 2e-2 on every element whose oracle value has |ref| < 8
+  (below 8 half a bf16 ulp is at most 1/64, so a correctly rounded result
+  meets 2e-2 with room for the fp32 arithmetic); on every element,
+  |ref| >= 8 included, the GPU value must be within one bf16 ulp of the
+  exact value (faithful rounding: the fp32 result rounded once to nearest
+  even), with an absolute floor of 1e-5 for values near zero. From |ref| = 8
+  up half an ulp alone is 1/32 > 2e-2, so faithful rounding is the
+  meaningful bound there; the count of such elements is reported.
 * rstd (fp32 in both cases): relative D * 2^-24, the worst-case error of an
   fp32 sum of D squares (the root halves it).
 * dgamma: normwise relative error max|gpu - ref| / max|ref| <= 1e-3 (bf16),
@@ -18,6 +20,9 @@ Tolerances (written here, used by every parity test):
 """
 from __future__ import annotations
 
+import os
+from concurrent.futures import ThreadPoolExecutor
+
 import numpy as np
 import torch
 
@@ -26,7 +31,7 @@ import workloads
 
 ABS_TOL = {"f32": 1e-5, "bf16": 2e-2}
 DGAMMA_REL = {"f32": 1e-5, "bf16": 1e-3}
-ORDER_ONE = 4.0
+ORDER_ONE = 8.0
 ULP_FLOOR = 1e-5
 
 
@@ -107,30 +112,68 @@ class Stats:
                 assert rel <= DGAMMA_REL[self.dtype], f"{n}: normwise rel err {rel:.3e}"
                 assert np.abs(got).max() > 0, f"{n} is zero"
 
+    def merge(self, other: "Stats"):
+        """Fold in the statistics of another chunk of the same tensors."""
+        for n, m in other.max_abs.items():
+            self.max_abs[n] = max(self.max_abs.get(n, 0.0), m)
+        for n, u in other.max_ulp.items():
+            self.max_ulp[n] = max(self.max_ulp.get(n, 0.0), u)
+        for n, c in other.n_big.items():
+            self.n_big[n] = self.n_big.get(n, 0) + c
+        self.rstd_rel = max(self.rstd_rel, other.rstd_rel)
+
     def summary(self):
         return dict(max_abs=self.max_abs, max_ulp=self.max_ulp, n_big=self.n_big,
                     rstd_rel=self.rstd_rel)
 
 
-def compare_with_oracle(inp: workloads.Inputs, got: dict, chunk_tokens: int = 4096,
+def _workers() -> int:
+    try:
+        n = len(os.sched_getaffinity(0))
+    except Exception:
+        n = os.cpu_count() or 1
+    return max(1, min(n, 32))
+
+
+def ordered_map(fn, items, workers=None):
+    """fn over items on a pool of host threads (the oracle is C called through
+    ctypes, which releases the GIL), results in item order, at most 2x
+    ``workers`` chunks in flight so memory stays bounded."""
+    items = list(items)
+    workers = workers or _workers()
+    if workers == 1 or len(items) <= 1:
+        for it in items:
+            yield fn(it)
+        return
+    with ThreadPoolExecutor(workers) as ex:
+        pending = []
+        i = 0
+        while i < len(items) or pending:
+            while i < len(items) and len(pending) < 2 * workers:
+                pending.append(ex.submit(fn, items[i]))
+                i += 1
+            yield pending.pop(0).result()
+
+
+def compare_with_oracle(inp: workloads.Inputs, got: dict, chunk_tokens: int = 1024,
                         bwd: bool = True, norm: str = "rms") -> Stats:
     """Every element of the GPU results against the oracle, token chunk by
-    token chunk (the oracle runs in fp64 on the CPU). ``norm="layer"``
+    token chunk (the oracle runs in fp64 on the CPU, chunks on parallel host
+    threads; dgamma partials are added in chunk order). ``norm="layer"``
     compares with the oracle's mean-centred form."""
     w = inp.w
     T = w.B * w.S
-    st = Stats(w.dtype, w.D)
     orc = oracle.get()
     m_all = oracle.positions(None if inp.pos is None else inp.pos.numpy(), w.B, w.S)
     q = inp.q.reshape(T, w.Hq, w.D)
     k = inp.k.reshape(T, w.Hkv, w.D)
+
     def view(name, H, last=w.D):
         return got[name].reshape(T, H, last)
 
-    dgq = np.zeros(w.D)
-    dgk = np.zeros(w.D)
-    for t0 in range(0, T, chunk_tokens):
+    def one(t0):
         t1 = min(T, t0 + chunk_tokens)
+        st = Stats(w.dtype, w.D)
         m = m_all[t0:t1]
         fwd = orc.ln_fwd if norm == "layer" else orc.fwd
         qo, ko, rq, rk = fwd(q[t0:t1], k[t0:t1], inp.gamma_q, inp.gamma_k, m,
@@ -139,25 +182,35 @@ def compare_with_oracle(inp: workloads.Inputs, got: dict, chunk_tokens: int = 40
         st.elem("k_out", oracle.as_f64(view("k_out", w.Hkv)[t0:t1]), ko)
         st.rstd(oracle.as_f64(view("rstd_q", w.Hq, 1)[t0:t1]).reshape(-1), rq.reshape(-1))
         st.rstd(oracle.as_f64(view("rstd_k", w.Hkv, 1)[t0:t1]).reshape(-1), rk.reshape(-1))
+        cq = ck = None
         if bwd:
             dqo = inp.dq_out.reshape(T, w.Hq, w.D)[t0:t1]
             dko = inp.dk_out.reshape(T, w.Hkv, w.D)[t0:t1]
             if norm == "layer":
                 dq, dk, cq, ck = orc.ln_bwd(q[t0:t1], k[t0:t1], inp.gamma_q, inp.gamma_k, m,
                                             dqo, dko, w.rotary_dim, w.theta, w.eps)
-                dgq, dgk = dgq + cq, dgk + ck
             else:
-                dq, dk, dgq, dgk = orc.bwd(q[t0:t1], k[t0:t1], inp.gamma_q, inp.gamma_k, m,
-                                           dqo, dko, w.rotary_dim, w.theta, w.eps,
-                                           dgamma_q=dgq, dgamma_k=dgk)
+                dq, dk, cq, ck = orc.bwd(q[t0:t1], k[t0:t1], inp.gamma_q, inp.gamma_k, m,
+                                         dqo, dko, w.rotary_dim, w.theta, w.eps)
             st.elem("dq", oracle.as_f64(view("dq", w.Hq)[t0:t1]), dq)
             st.elem("dk", oracle.as_f64(view("dk", w.Hkv)[t0:t1]), dk)
-    st.dgamma = {"dgamma_q": (got["dgamma_q"].numpy(), dgq),
-                 "dgamma_k": (got["dgamma_k"].numpy(), dgk)} if bwd else None
-    return st
+        return st, cq, ck
+
+    total = Stats(w.dtype, w.D)
+    dgq = np.zeros(w.D)
+    dgk = np.zeros(w.D)
+    for st, cq, ck in ordered_map(one, range(0, T, chunk_tokens)):
+        total.merge(st)
+        if cq is not None:
+            dgq, dgk = dgq + cq, dgk + ck
+    total.dgamma = {"dgamma_q": (got["dgamma_q"].numpy(), dgq),
+                    "dgamma_k": (got["dgamma_k"].numpy(), dgk)} if bwd else None
+    return total
 
 
 def check(inp, got, **kw) -> Stats:
     st = compare_with_oracle(inp, got, **kw)
+    if st.n_big:
+        print("elements with |ref| >= %g (held to one bf16 ulp):" % ORDER_ONE, st.n_big)
     st.check(st.dgamma)
     return st

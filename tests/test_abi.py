@@ -1,9 +1,10 @@
 """The C ABI library: it loads, exports every symbol include/qknr.h declares,
 and rejects bad arguments on the host before touching the GPU.
 
-No GPU is needed: every call here fails validation, which happens before any
-CUDA runtime call. The pointers are fake addresses that are never
-dereferenced.
+No GPU is needed: every call here either fails validation, which happens
+before any CUDA runtime call, or is an empty problem (B = 0) that returns
+before one, or is a host-only plan query. The pointers are fake addresses
+that are never dereferenced.
 """
 import ctypes
 import os
@@ -88,6 +89,28 @@ def bwd(lib, B=2, S=8, Hq=4, Hkv=2, D=64, R=64, theta=1e4, eps=1e-6, dt=BF16, **
 ])
 def test_shape_validation(lib, call, kw, want):
     assert call(lib, **kw) == want
+
+
+@pytest.mark.parametrize("dt,D,R", [(BF16, 72, 64), (BF16, 72, 0), (BF16, 8, 0),
+                                    (BF16, 40, 16), (F32, 12, 8), (F32, 20, 16), (F32, 4, 0)])
+def test_sixteen_byte_rows_accepted(lib, dt, D, R):
+    # D * elem_bytes a multiple of 16 is enough: an odd vector count per row
+    # runs the plain-load kernels (empty problems launch nothing; the plan
+    # query makes no CUDA call)
+    assert fwd(lib, B=0, D=D, R=R, dt=dt) == OK
+    assert bwd(lib, B=0, D=D, R=R, dt=dt, dgq=None, dgk=None) == OK
+    plan = (ctypes.c_int64 * 14)()
+    for kind in range(4):
+        assert lib.qk_norm_rope_plan(kind, 2, 8, 4, 2, D, R, dt, 0, 148, 0,
+                                     ctypes.cast(plan, ctypes.c_void_p)) == OK
+        assert plan[0] == 0 and plan[13] == 256
+    assert lib.qk_layerwise_stats(P(1), P(2), P(7), P(8), 0, 8, 4, 2, D, dt, None) == OK
+
+
+@pytest.mark.parametrize("dt,D", [(BF16, 4), (BF16, 12), (F32, 2), (F32, 6)])
+def test_rows_not_whole_vectors_rejected(lib, dt, D):
+    assert fwd(lib, D=D, R=0, dt=dt) == UNSUP
+    assert bwd(lib, D=D, R=0, dt=dt) == UNSUP
 
 
 @pytest.mark.parametrize("call", [fwd, bwd], ids=["fwd", "bwd"])

@@ -57,7 +57,8 @@ def test_layernorm_vs_oracle(cuda, kernels, name, over):
 
 
 SHAPES = [("bf16", 16, 16), ("bf16", 64, 32), ("bf16", 80, 80), ("bf16", 128, 0),
-          ("bf16", 256, 64), ("f32", 8, 8), ("f32", 24, 16), ("f32", 128, 128)]
+          ("bf16", 256, 64), ("f32", 8, 8), ("f32", 24, 16), ("f32", 128, 128),
+          ("bf16", 72, 64), ("bf16", 40, 16), ("f32", 12, 8), ("f32", 20, 0)]
 
 
 @pytest.mark.parametrize("dtype,D,R", SHAPES, ids=[f"{a}-D{b}-R{c}" for a, b, c in SHAPES])

@@ -104,7 +104,7 @@ def run_ranks(inp, gq, gk, cuda, world=1, local=False):
 
 def check_vs_oracle(inp, gq, gk, got):
     """Element bounds of parity.py (fp32 1e-5 max-abs; bf16 2e-2 max-abs where
-    |ref| < 4 and one bf16 ulp everywhere); rstd to (H D) 2^-24 relative
+    |ref| < 8 and one bf16 ulp everywhere); rstd to (H D) 2^-24 relative
     (an fp32 sum over the whole hidden vector); dgamma to its normwise
     tolerance."""
     w = inp.w
@@ -290,7 +290,7 @@ def test_layerwise_no_pipeline_timeouts(cuda):
 
 
 @pytest.mark.parametrize("dtype,D,R", [("bf16", 128, 0), ("f32", 64, 0), ("f32", 64, 16),
-                                       ("bf16", 64, 32)])
+                                       ("bf16", 64, 32), ("bf16", 72, 64), ("f32", 12, 8)])
 def test_layerwise_rotary_spans_and_dtypes(cuda, kernels, dtype, D, R):
     # NoPE (no rotary span), partial spans, fp32 I/O; one rank and two slices
     inp, gq, gk = lw_inputs("tiny", seed=6, B=2, S=45, Hq=8, Hkv=4, D=D, rotary_dim=R,

@@ -77,7 +77,11 @@ SHAPES = [("bf16", 16, 16), ("bf16", 16, 0), ("bf16", 32, 16), ("bf16", 64, 32),
           ("bf16", 128, 0), ("bf16", 128, 32), ("bf16", 128, 128), ("bf16", 192, 64),
           ("bf16", 256, 256), ("bf16", 256, 32),
           ("f32", 8, 8), ("f32", 16, 8), ("f32", 24, 16), ("f32", 64, 64),
-          ("f32", 128, 32), ("f32", 128, 128), ("f32", 256, 256), ("f32", 256, 0)]
+          ("f32", 128, 32), ("f32", 128, 128), ("f32", 256, 256), ("f32", 256, 0),
+          # an odd number of 16-byte vectors per row: the last pass-through unit
+          # has one vector (the plain-load kernels take these shapes)
+          ("bf16", 8, 0), ("bf16", 40, 16), ("bf16", 72, 64), ("bf16", 72, 0),
+          ("bf16", 120, 48), ("f32", 4, 0), ("f32", 12, 8), ("f32", 20, 16), ("f32", 12, 0)]
 
 
 @pytest.mark.parametrize("dtype,D,R", SHAPES, ids=[f"{a}-D{b}-R{c}" for a, b, c in SHAPES])

@@ -47,7 +47,7 @@ def positions_of(inp):
 
 def check_elems(dtype, name, got, ref):
     """Elementwise bound of parity.py: fp32 max-abs 1e-5; bf16 max-abs 2e-2
-    where |ref| < 4 and within one bf16 ulp everywhere."""
+    where |ref| < 8 and within one bf16 ulp everywhere."""
     st = parity.Stats(dtype, got.shape[-1])
     st.elem(name, got.double().numpy().reshape(-1), np.asarray(ref).reshape(-1))
     tol = parity.ABS_TOL[dtype]
@@ -74,6 +74,8 @@ ROPE_CASES = [
     ("bfd-packed", dict()),
     ("tiny", dict()),
     ("tiny", dict(B=3, S=37, Hq=5, Hkv=3, D=24, rotary_dim=16)),
+    ("tiny", dict(B=3, S=37, Hq=5, Hkv=3, D=20, rotary_dim=16)),
+    ("llama3-8b-qknorm", dict(B=1, S=77, Hq=4, Hkv=2, D=72, rotary_dim=64)),
 ]
 
 

@@ -93,7 +93,7 @@ WORKLOADS = {
                            row_cap=4096, doc_len_range=(64, 4096), index=4),
 }
 
-BENCH_WORKLOAD = "qwen2.5-0.5b"
+BENCH_WORKLOAD = "partial-rope-64k"
 
 
 def seed_for(w: Workload, k: int = 0) -> int:
