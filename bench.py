@@ -232,9 +232,14 @@ class Set:
 def measure(w, inp, dev, steps: int, warmup: int, nsets: int, layout: str = "dense",
             world: int = 1, clocks=None):
     """Time ``steps`` fwd + bwd steps of workload ``w`` on a ring of ``nsets``
-    input sets (after ``warmup`` untimed steps), events around every launch.
-    Returns the total, mean forward and mean backward milliseconds, the max
-    over ranks when ``world`` > 1."""
+    input sets (after ``warmup`` untimed steps): first with events only at
+    the two ends (the step time; the kernels run back to back, each one's
+    prologue overlapping the previous one's tail), then the same number of
+    steps again with events around every launch (the per-kernel split; an
+    event between two launches serialises them, so this split includes the
+    launch gaps the first pass hides). Returns the total, mean forward, mean
+    backward and split-pass total milliseconds, the max over ranks when
+    ``world`` > 1."""
     import qk_rmsnorm_rope_norm_b200 as qknr
     cfg = dict(rotary_dim=w.rotary_dim, theta=w.theta, eps=w.eps)
     sets = [Set(inp, dev, layout) for _ in range(nsets)]
@@ -266,17 +271,24 @@ def measure(w, inp, dev, steps: int, warmup: int, nsets: int, layout: str = "den
     with (clocks if clocks is not None else _Null()):
         t_start.record(stream)
         for i in range(K):
-            step(W + i, ev[i])
+            step(W + i)
         t_end.record(stream)
         torch.cuda.synchronize(dev)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
     total_ms = t_start.elapsed_time(t_end)
+    s_start, s_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s_start.record(stream)
+    for i in range(K):
+        step(W + K + i, ev[i])
+    s_end.record(stream)
+    torch.cuda.synchronize(dev)
+    split_ms = s_start.elapsed_time(s_end)
     fwd_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / K
     bwd_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / K
     del fwd, bwd, sets
-    return max_over_ranks([total_ms, fwd_ms, bwd_ms], world, dev)
+    return max_over_ranks([total_ms, fwd_ms, bwd_ms, split_ms], world, dev)
 
 
 class _Null:
@@ -293,16 +305,16 @@ def run_ours(args, w, inp, rank, local_rank, world):
     qknr.load_library()
     cfg = dict(rotary_dim=w.rotary_dim, theta=w.theta, eps=w.eps)
     clocks = ClockSampler(local_rank)  # NVML start-up stays outside the timed region
-    total_ms, fwd_ms, bwd_ms = measure(w, inp, dev, args.steps, args.warmup, args.sets,
-                                       args.layout, world, clocks)
+    total_ms, fwd_ms, bwd_ms, split_ms = measure(w, inp, dev, args.steps, args.warmup,
+                                                 args.sets, args.layout, world, clocks)
     torch.cuda.empty_cache()
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(args, w, inp, dev, cfg, world)
     cb = workloads.contract_bytes(w, with_pos=inp.pos is not None)
     floor = {"fwd_ms": copy_floor_ms(cb["fwd"], dev), "bwd_ms": copy_floor_ms(cb["bwd"], dev)}
-    return dict(total_ms=total_ms, fwd_ms=fwd_ms, bwd_ms=bwd_ms, clocks=clocks.summary(),
-                e2e=e2e, floor=floor)
+    return dict(total_ms=total_ms, fwd_ms=fwd_ms, bwd_ms=bwd_ms, split_ms=split_ms,
+                clocks=clocks.summary(), e2e=e2e, floor=floor)
 
 
 def device_limits(dev):
@@ -348,9 +360,11 @@ def run_per_config(args, main_w, main_r, rank, dev, peak):
             inp = workloads.make_inputs(base, seed=rank_seed(base, rank))
             w = inp.w
             steps = args.per_config_steps
-            _, fwd_ms, bwd_ms = measure(w, inp, dev, steps, max(3, args.warmup), NSETS)
+            total_ms, fwd_ms, bwd_ms, _ = measure(w, inp, dev, steps, max(3, args.warmup), NSETS)
             torch.cuda.empty_cache()
         out[name] = per_config_line(w, inp, fwd_ms, bwd_ms, peak, dev, steps)
+        out[name]["ms_per_step"] = (main_r["total_ms"] / args.steps if name == main_w.name
+                                    else total_ms / steps)
     return out
 
 
@@ -807,6 +821,9 @@ def main():
                     "bwd_gbs": cb["bwd"] / (r["floor"]["bwd_ms"] / 1e3) / 1e9,
                     "fwd_frac_of_copy": r["floor"]["fwd_ms"] / r["fwd_ms"],
                     "bwd_frac_of_copy": r["floor"]["bwd_ms"] / r["bwd_ms"]}},
+        "split_pass": {"ms_per_step": r["split_ms"] / args.steps,
+                       "what": "the same steps again with an event around every launch; "
+                               "fwd.ms and bwd.ms come from it"},
         "fwd": {"ms": r["fwd_ms"], "tokens_per_s": aggregate_tokens_per_s(world, tokens, r["fwd_ms"]),
                 "bytes_per_launch": cb["fwd"], "kernel": fwd_kernel},
         "bwd": {"ms": r["bwd_ms"], "tokens_per_s": aggregate_tokens_per_s(world, tokens, r["bwd_ms"]),

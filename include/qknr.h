@@ -429,6 +429,20 @@ QKNR_API const char *qknr_strerror(qknr_status status);
 QKNR_API int qknr_last_cuda_error(void);
 
 /*
+ * Diagnostic of the timeout path: launches on `stream` a one-block kernel in
+ * which one thread waits, with the same bounded wait the pipelined kernels
+ * of `family` use (0: the per-head kernels, 1: the layerwise kernels), on a
+ * shared-memory barrier that nothing completes, for at most limit_cycles SM
+ * clock cycles (1 <= limit_cycles <= 2^31; the clock is read every 256th
+ * test of the barrier, each test bounded by its suspend hint, so the wait
+ * lasts a few milliseconds at least). The wait gives up, sets bit 0 of the
+ * flag qknr_pipeline_error reports, and the kernel returns; nothing else is
+ * touched and the context stays usable. A bad family or limit is
+ * QKNR_ERR_INVALID_ARG; a refused launch QKNR_ERR_CUDA.
+ */
+QKNR_API qknr_status qknr_wait_selftest(int family, int64_t limit_cycles, qknr_stream_t stream);
+
+/*
  * Diagnostic flag of the current device's pipelined kernels: non-zero if
  * a kernel gave up an internal wait (bounded at 2 s; the results of that
  * launch are then incomplete). Synchronises with the device. With reset

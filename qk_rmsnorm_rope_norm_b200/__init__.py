@@ -31,7 +31,8 @@ __all__ = ["qk_norm_rope_fwd", "qk_norm_rope_bwd", "qknr_strerror", "QKNormRoPE"
            "qk_norm_rope", "QKNRError", "library_path", "load_library", "pipeline_error",
            "qk_layerwise_stats", "qk_layerwise_norm_rope_fwd", "qk_layerwise_bwd_dots",
            "qk_layerwise_norm_rope_bwd", "QKLayerwiseNormRoPE", "qk_layerwise_norm_rope",
-           "all_reduce_stats", "layerwise_geometry", "launch_plan", "kernel_name"]
+           "all_reduce_stats", "layerwise_geometry", "launch_plan", "kernel_name",
+           "wait_selftest"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libqknr.so")
@@ -105,6 +106,8 @@ def load_library():
     lib.qknr_last_cuda_error.argtypes = []
     lib.qknr_pipeline_error.restype = i32
     lib.qknr_pipeline_error.argtypes = [i32]
+    lib.qknr_wait_selftest.restype = i32
+    lib.qknr_wait_selftest.argtypes = [i32, i64, vp]
     _lib = lib
     return lib
 
@@ -117,6 +120,15 @@ def pipeline_error(reset: bool = False) -> int:
     """Non-zero if a pipelined kernel on the current device gave up a bounded
     internal wait since the flag was last cleared (synchronises)."""
     return int(load_library().qknr_pipeline_error(1 if reset else 0))
+
+
+def wait_selftest(family: int = 0, limit_cycles: int = 100_000, stream=None) -> None:
+    """Run the bounded-wait self-test of a kernel family (0: per-head, 1:
+    layerwise): a wait on a barrier nothing completes gives up and sets the
+    flag that ``pipeline_error`` reports."""
+    st = load_library().qknr_wait_selftest(int(family), int(limit_cycles), _stream(stream))
+    if st != QKNR_OK:
+        raise QKNRError(st, "qknr_wait_selftest")
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -825,10 +837,12 @@ _GEOM_KEYS = ("pipelined", "lpr", "TT", "NS", "stage_bytes", "off_k", "off_dq", 
 def layerwise_geometry(mode: str, B: int, S: int, Hq: int, Hkv: int, D: int, rotary_dim: int,
                        dtype=torch.bfloat16, sms: int = 148) -> dict:
     """Launch geometry of the pipelined layerwise ``"dots"`` or ``"bwd"``
-    kernel for a shape (C ``qk_layerwise_geometry``; host only, no GPU)."""
+    kernel, or of the ``"tok"`` kernel (statistics and forward), for a shape
+    (C ``qk_layerwise_geometry``; host only, no GPU)."""
     lib = load_library()
     out = (ctypes.c_int64 * len(_GEOM_KEYS))()
-    st = lib.qk_layerwise_geometry({"dots": 0, "bwd": 1}[mode], B, S, Hq, Hkv, D, rotary_dim,
+    st = lib.qk_layerwise_geometry({"dots": 0, "bwd": 1, "tok": 2}[mode], B, S, Hq, Hkv, D,
+                                   rotary_dim,
                                    _DTYPES[dtype], sms, ctypes.cast(out, ctypes.c_void_p))
     if st != QKNR_OK:
         raise QKNRError(st, "qk_layerwise_geometry")

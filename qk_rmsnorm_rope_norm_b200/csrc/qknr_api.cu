@@ -10,6 +10,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstdlib>
+#include <utility>
 
 namespace qknr {
 
@@ -295,6 +296,33 @@ bool pipe_disabled() {
     return e && e[0] == '1';
 }
 
+// Programmatic dependent launch of the pipelined kernels (they wait for the
+// previous kernel of the stream before touching global memory and let the
+// next one start its prologue early); QKNR_PDL=0 launches them plainly.
+bool pdl_enabled() {
+    static const bool on = [] {
+        const char *e = std::getenv("QKNR_PDL");
+        return !(e && e[0] == '0');
+    }();
+    return on;
+}
+
+template <typename... P, typename... A>
+cudaError_t launch_pipe(void (*kern)(P...), int grid, int threads, int smem, cudaStream_t st,
+                        A &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3((unsigned)threads);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = pdl_enabled() ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<A>(args)...);
+}
+
 // cuTensorMapEncodeTiled from the driver, looked up once.
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     static std::atomic<void *> fn{nullptr};
@@ -359,8 +387,7 @@ qknr_status launch_fwd_pipe_tm(const FwdArgs &a, const PipeGeom &g, const CUtens
     *launched = true;
     typename MapsArg<TM>::type maps{};
     if constexpr (TM) maps = TensorMaps{mq, mk};
-    kern<<<grid, (NCW + kProducerWarps) * 32, smem, st>>>(a, g, maps);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pipe(kern, grid, (NCW + kProducerWarps) * 32, smem, st, a, g, maps);
     return e == cudaSuccess ? QKNR_OK : cuda_fail(e);
 }
 
@@ -376,8 +403,7 @@ qknr_status launch_bwd_pipe_tm(const BwdArgs &a, const PipeGeom &g, const CUtens
     *launched = true;
     typename MapsArg<TM>::type maps{};
     if constexpr (TM) maps = TensorMaps{mq, mk};
-    kern<<<grid, (NCW + kProducerWarps) * 32, smem, st>>>(a, g, maps);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pipe(kern, grid, (NCW + kProducerWarps) * 32, smem, st, a, g, maps);
     return e == cudaSuccess ? QKNR_OK : cuda_fail(e);
 }
 
@@ -820,6 +846,17 @@ extern "C" int qknr_last_cuda_error(void) { return g_last_cuda_error; }
 
 namespace qknr {
 int lw_pipeline_error(int reset);  // the layerwise kernels' flag, same bits
+qknr_status lw_wait_selftest(long long limit, cudaStream_t st);
+}
+
+extern "C" qknr_status qknr_wait_selftest(int family, int64_t limit_cycles, qknr_stream_t stream) {
+    if ((family != 0 && family != 1) || limit_cycles < 1 || limit_cycles > ((int64_t)1 << 31))
+        return QKNR_ERR_INVALID_ARG;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (family == 1) return qknr::lw_wait_selftest((long long)limit_cycles, st);
+    qknr::qknr_wait_selftest_kernel<<<1, 32, 0, st>>>((long long)limit_cycles);
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? QKNR_OK : cuda_fail(e);
 }
 
 extern "C" int qknr_pipeline_error(int reset) {

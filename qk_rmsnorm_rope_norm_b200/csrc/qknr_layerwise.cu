@@ -381,6 +381,7 @@ constexpr int kLwStageTarget = 96 * 1024;
 constexpr int kLwRingBytes = 200 * 1024;
 constexpr int kMaxTileTokensLw = 32;
 constexpr int kLwSmemBytes = 220 * 1024;       // dynamic shared memory at most
+constexpr int kLwTokStageTarget = 96 * 1024;   // statistics / forward stage
 constexpr long long kLwWaitCycles = 4000000000ll;  // ~2 s per wait at 1.9 GHz
 
 enum LwMode { kLwDots = 0, kLwBwd = 1 };
@@ -424,9 +425,11 @@ __device__ __forceinline__ bool lw_bar_test(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// Wait for the phase of parity `parity`, for at most kLwWaitCycles; false
-// (with the error flag set) if it never completes.
-__device__ __forceinline__ bool lw_wait(uint32_t bar, uint32_t parity) {
+// Wait for the phase of parity `parity`, for at most `limit` cycles (by
+// default kLwWaitCycles); false (with the error flag set) if it never
+// completes.
+__device__ __forceinline__ bool lw_wait(uint32_t bar, uint32_t parity,
+                                        long long limit = kLwWaitCycles) {
     if (lw_bar_test(bar, parity)) return true;
     const long long c0 = clock64();
     uint32_t nap = 32;
@@ -437,11 +440,22 @@ __device__ __forceinline__ bool lw_wait(uint32_t bar, uint32_t parity) {
             __nanosleep(nap);
             nap = nap < 256 ? nap * 2 : 256;
         }
-        if ((n & 255u) == 0 && clock64() - c0 > kLwWaitCycles) {
+        if ((n & 255u) == 0 && clock64() - c0 > limit) {
             atomicOr(&g_lw_error, 1u);
             return false;
         }
     }
+}
+
+// Diagnostic: lw_wait with a limit of `limit` cycles on a barrier nothing
+// arrives on (see qknr_wait_selftest_kernel).
+__global__ void qknr_lw_wait_selftest_kernel(long long limit) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x != 0) return;
+    const uint32_t b = lw_smem_u32(&bar);
+    lw_bar_init(b, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    lw_wait(b, 0, limit);
 }
 // Bulk copy global -> shared (dst, src, bytes multiples of 16), counted in
 // bytes on `bar`; the rows are read once, so they may leave L2 first.
@@ -496,6 +510,59 @@ __device__ __forceinline__ void lane_cs4(float4 (&c)[V / 2], const float4 *tok, 
         c[k] = L.rot ? tok[k * U + w] : make_float4(1.f, 1.f, 0.f, 0.f);
 }
 
+// The producer warp's share of a stage's (cos, sin) table: pair P of a token
+// (angles 2P, 2P + 1) is one float4 (c_2P, c_2P+1, s_2P, s_2P+1) stored at
+// (P mod W) U + P / W (W = V/2 pairs per lane, U = hp / W rotating units), so
+// the lanes of a row read consecutive entries. The work split is fixed for
+// the kernel: with hp <= 32 pairs lane (jo, P) takes pair P of tokens jo,
+// jo + tpp, ... (tpp = 32 / hp tokens per pass); beyond that every lane loops
+// over pairs lane + 32 k of every token.
+template <int V> struct LwCsWork {
+    int hp, tpp, jo, P, dst;
+    uint64_t F0, F1;
+    __device__ __forceinline__ LwCsWork(const uint64_t *s_step, int half, int lane) {
+        hp = half >> 1;
+        tpp = (hp > 0 && hp <= 32) ? 32 / hp : 0;
+        jo = 0;
+        P = -1;
+        dst = 0;
+        F0 = F1 = 0;
+        if (tpp > 0 && lane < tpp * hp) {
+            jo = lane / hp;
+            P = lane - jo * hp;
+            F0 = s_step[2 * P];
+            F1 = s_step[2 * P + 1];
+            const int pw = P / (V / 2);
+            dst = (P - pw * (V / 2)) * (hp / (V / 2)) + pw;
+        }
+    }
+    // table of na tokens whose positions are s_pos[0..na)
+    __device__ __forceinline__ void fill(float4 *cs, const int32_t *s_pos, const uint64_t *s_step,
+                                         int na, int lane) const {
+        if (tpp > 0) {
+            if (P >= 0)
+                for (int j = jo; j < na; j += tpp) {
+                    const int32_t m = s_pos[j];
+                    const float2 c0 = rope_cos_sin_fixed(m, F0);
+                    const float2 c1 = rope_cos_sin_fixed(m, F1);
+                    cs[j * hp + dst] = make_float4(c0.x, c1.x, c0.y, c1.y);
+                }
+        } else {
+            for (int q = lane; q < hp; q += 32) {
+                const uint64_t G0 = s_step[2 * q], G1 = s_step[2 * q + 1];
+                const int pw = q / (V / 2);
+                const int d = (q - pw * (V / 2)) * (hp / (V / 2)) + pw;
+                for (int j = 0; j < na; ++j) {
+                    const int32_t m = s_pos[j];
+                    const float2 c0 = rope_cos_sin_fixed(m, G0);
+                    const float2 c1 = rope_cos_sin_fixed(m, G1);
+                    cs[j * hp + d] = make_float4(c0.x, c1.x, c0.y, c1.y);
+                }
+            }
+        }
+    }
+};
+
 template <typename T, int LPR, int MODE>
 __global__ void __launch_bounds__((kLwCWMax + 1) * 32, 1)
     qknr_lw_pipe_kernel(const LwArgs a, const LwGeom g) {
@@ -512,8 +579,10 @@ __global__ void __launch_bounds__((kLwCWMax + 1) * 32, 1)
         if (threadIdx.x == 0) atomicOr(&g_lw_error, 2u);
         return;
     }
+    __shared__ int s_abort;  // a consumer warp gave up a wait: skip the dgamma phase
     unsigned char *ring = smem + 128;
     float2 *parts_all = reinterpret_cast<float2 *>(smem + g.off_parts);
+    if (threadIdx.x == 0) s_abort = 0;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t t_lo = (int64_t)blockIdx.x * g.tpc;
     const int64_t t_hi = min(a.T, t_lo + g.tpc);
@@ -544,21 +613,7 @@ __global__ void __launch_bounds__((kLwCWMax + 1) * 32, 1)
         const bool totals = MODE == kLwBwd && !(a.sq == nullptr && a.sk == nullptr);
         const bool need_cs = half > 0;
         int s_cur = (int)(t_lo % a.S);  // row position of the tile's first token
-        // (cos, sin) work split, fixed for the kernel. Pair P of a token is
-        // stored at (P mod W) U + P / W (W = V/2 pairs per lane, U = hp / W
-        // rotating units) so that the lanes of a row read consecutive entries.
-        const int cs_hp = half >> 1;
-        const int cs_tpp = (cs_hp > 0 && cs_hp <= 32) ? 32 / cs_hp : 0;  // tokens per pass
-        int cs_jo = 0, cs_P = -1, cs_dst = 0;
-        uint64_t cs_F0 = 0, cs_F1 = 0;
-        if (cs_tpp > 0 && lane < cs_tpp * cs_hp) {
-            cs_jo = lane / cs_hp;
-            cs_P = lane - cs_jo * cs_hp;
-            cs_F0 = s_step[2 * cs_P];
-            cs_F1 = s_step[2 * cs_P + 1];
-            const int pw = cs_P / (V / 2);
-            cs_dst = (cs_P - pw * (V / 2)) * (cs_hp / (V / 2)) + pw;
-        }
+        const LwCsWork<V> csw(s_step, half, lane);
         int issued = 0;
         for (int i = 0; i < ntiles; ++i) {
             const int s = i % g.NS;
@@ -612,31 +667,7 @@ __global__ void __launch_bounds__((kLwCWMax + 1) * 32, 1)
             if (need_cs) {
                 if (lane < na) s_pos[lane] = pos;
                 __syncwarp();
-                // pair P of a token: (c_2P, c_2P+1, s_2P, s_2P+1), one float4
-                float4 *cs = reinterpret_cast<float4 *>(st + g.off_cs);
-                if (cs_tpp > 0) {
-                    // hp <= 32: lane (jo, P) takes pair P of tokens jo, jo + tpp, ...
-                    if (cs_P >= 0)
-                        for (int j = cs_jo; j < na; j += cs_tpp) {
-                            const int32_t m = s_pos[j];
-                            const float2 c0 = rope_cos_sin_fixed(m, cs_F0);
-                            const float2 c1 = rope_cos_sin_fixed(m, cs_F1);
-                            cs[j * cs_hp + cs_dst] = make_float4(c0.x, c1.x, c0.y, c1.y);
-                        }
-                } else {
-                    // hp > 32: lane takes pairs P = lane + 32 k of every token
-                    for (int P = lane; P < cs_hp; P += 32) {
-                        const uint64_t F0 = s_step[2 * P], F1 = s_step[2 * P + 1];
-                        const int pw = P / (V / 2);
-                        const int dst = (P - pw * (V / 2)) * (cs_hp / (V / 2)) + pw;
-                        for (int j = 0; j < na; ++j) {
-                            const int32_t m = s_pos[j];
-                            const float2 c0 = rope_cos_sin_fixed(m, F0);
-                            const float2 c1 = rope_cos_sin_fixed(m, F1);
-                            cs[j * cs_hp + dst] = make_float4(c0.x, c1.x, c0.y, c1.y);
-                        }
-                    }
-                }
+                csw.fill(reinterpret_cast<float4 *>(st + g.off_cs), s_pos, s_step, na, lane);
                 __syncwarp();
             }
             lw_bar_arrive(full);
@@ -665,7 +696,10 @@ __global__ void __launch_bounds__((kLwCWMax + 1) * 32, 1)
     for (int i = 0; i < ntiles; ++i) {
         const int s = i % g.NS;
         const uint32_t ph = (uint32_t)(i / g.NS) & 1u;
-        if (!lw_wait(bar0 + 8 * s, ph)) break;
+        if (!lw_wait(bar0 + 8 * s, ph)) {
+            s_abort = 1;
+            break;
+        }
         const int64_t t0 = t_lo + (int64_t)i * g.TT;
         const int na = (int)min((int64_t)g.TT, t_hi - t0);
         const unsigned char *st = ring + (size_t)s * g.stage_bytes;
@@ -736,7 +770,10 @@ __global__ void __launch_bounds__((kLwCWMax + 1) * 32, 1)
             __syncwarp();
             const uint32_t pbar = bar0 + 8 * (2 * g.NS + s);
             if (lane == 0) lw_bar_arrive(pbar);
-            if (!lw_wait(pbar, ph)) break;
+            if (!lw_wait(pbar, ph)) {
+                s_abort = 1;
+                break;
+            }
             if (MODE == kLwDots && warp == 0) {
                 // lane j: token j's total over the G warps, in warp order
                 for (int j = lane; j < na; j += 32) {
@@ -824,10 +861,13 @@ __global__ void __launch_bounds__((kLwCWMax + 1) * 32, 1)
     if (MODE == kLwBwd) {
         // dgamma: the token groups of this CTA own the same elements, so sum
         // them in shared memory (the ring, free now) first, then one global
-        // atomic add per element and CTA
+        // atomic add per element and CTA. After a consumer gave up a wait the
+        // ring may still be receiving copies, so the phase is skipped (the
+        // launch's results are incomplete then, and the error flag says so).
         float *s_red = reinterpret_cast<float *>(ring);
         const int nel = H * a.D, ct = ncw * 32;
         asm volatile("bar.sync 1, %0;" ::"r"(ct) : "memory");
+        if (s_abort) return;
         for (int e = threadIdx.x; e < nel; e += ct) s_red[e] = 0.f;
         asm volatile("bar.sync 1, %0;" ::"r"(ct) : "memory");
 #pragma unroll
@@ -851,6 +891,242 @@ __global__ void __launch_bounds__((kLwCWMax + 1) * 32, 1)
             float *dg = e < nq ? a.dgq + e : a.dgk + (e - nq);
             if ((e < nq ? a.dgq : a.dgk) != nullptr) atomicAdd(dg, s_red[e]);
         }
+    }
+}
+
+// ------------------------------------------------------------------------
+// Pipelined statistics and forward. One producer warp streams stages of TT
+// whole tokens (a stage's Q rows and K rows are two contiguous ranges) into
+// the ring with bulk copies and writes the stage's per-token totals (second
+// phase of a sharded call) and (cos, sin) table. Each consumer warp takes
+// whole tokens, dealt round-robin and continuing across stages: it sums x^2
+// over the token's rows in shared memory (one warp reduction per tensor, no
+// cross-warp exchange), then normalises, rotates and stores every row of the
+// token. Every row crosses HBM once. The statistics and the one-pass forward
+// run the same summation, so the two-phase and one-pass results agree bit
+// for bit.
+enum LwTokMode { kTokStats = 0, kTokFwd = 1 };
+
+struct LwTokGeom {
+    int TT, NS, stage_bytes;
+    int off_k, off_cs, off_sc;  // sections of a stage (Q rows at 0); scalars float2 {sq, sk}
+    int off_gamma;              // gamma_q then gamma_k rows, I/O dtype
+    int ncw;                    // consumer warps
+    int64_t tpc;                // tokens per CTA
+};
+
+// Sums of x^2 over the rows of one token held in shared memory (Q rows at
+// xq, K rows at xk), the warp totals in every lane.
+template <typename T, int LPR>
+__device__ __forceinline__ float2 tok_sumsq(const unsigned char *xq, const unsigned char *xk,
+                                            const Lane<LPR, Io<T>::V> &L, int Hq, int H,
+                                            int rowb, int offA, int offB) {
+    using IO = Io<T>;
+    constexpr int V = IO::V, SLOTS = 32 / LPR;
+    float2 pq = make_float2(0.f, 0.f), pk = make_float2(0.f, 0.f);
+    for (int p = 0; p < H; p += SLOTS) {
+        const int h = p + L.slot;
+        if (!(L.on && h < H)) continue;
+        const bool isq = h < Hq;
+        const unsigned char *row = isq ? xq + h * rowb : xk + (h - Hq) * rowb;
+        const Vec16 xa = ld16(row + offA), xb = ld16(row + offB);
+        float2 s0 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int k2 = 0; k2 < V / 2; ++k2) {
+            const float2 va = IO::get2(xa, k2), vb = IO::get2(xb, k2);
+            s0 = __ffma2_rn(va, va, s0);
+            s0 = __ffma2_rn(vb, vb, s0);
+        }
+        if (isq) pq = __fadd2_rn(pq, s0);
+        else pk = __fadd2_rn(pk, s0);
+    }
+    float q = pq.x + pq.y, k = pk.x + pk.y;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        q += __shfl_xor_sync(0xffffffffu, q, o);
+        k += __shfl_xor_sync(0xffffffffu, k, o);
+    }
+    return make_float2(q, k);
+}
+
+template <typename T, int LPR, int MODE>
+__global__ void __launch_bounds__((kLwCWMax + 1) * 32, 1)
+    qknr_lw_tok_kernel(const LwArgs a, const LwTokGeom g) {
+    using IO = Io<T>;
+    constexpr int V = IO::V, SLOTS = 32 / LPR, E = (int)sizeof(T);
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ uint64_t s_step[kMaxHalf];        // fixed-point angle step per rotary pair
+    __shared__ int32_t s_pos[kMaxTileTokensLw];  // producer: positions of the stage's tokens
+    const int half = MODE == kTokFwd ? a.R >> 1 : 0;
+    const int nthr = blockDim.x, ncw = g.ncw;  // the producer is warp ncw
+    for (int i = threadIdx.x; i < half; i += nthr) s_step[i] = turn_step(i, a.R, a.theta);
+    const uint32_t bar0 = lw_smem_u32(smem);  // full[NS], empty[NS]
+    if (bar0 & 127u) {  // bulk copies need 16-byte aligned stages: compute nothing
+        if (threadIdx.x == 0) atomicOr(&g_lw_error, 2u);
+        return;
+    }
+    unsigned char *ring = smem + 128;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t t_lo = (int64_t)blockIdx.x * g.tpc;
+    const int64_t t_hi = min(a.T, t_lo + g.tpc);
+    const int ntiles = t_hi > t_lo ? (int)((t_hi - t_lo + g.TT - 1) / g.TT) : 0;
+    const int H = a.Hq + a.Hkv, rowb = a.D * E;
+    const unsigned char *s_gamma = smem + g.off_gamma;
+    if (MODE == kTokFwd) {  // every CTA reads the weights once
+        const int nq = a.Hq * rowb / 16, nk = a.Hkv * rowb / 16;
+        for (int i = threadIdx.x; i < nq + nk; i += nthr) {
+            const Vec16 v = i < nq ? ld16((const char *)a.gq + 16 * i)
+                                   : ld16((const char *)a.gk + 16 * (i - nq));
+            st16(smem + g.off_gamma + 16 * i, v);
+        }
+    }
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < g.NS; ++s) {
+            lw_bar_init(bar0 + 8 * s, 32);              // the producer warp's lanes
+            lw_bar_init(bar0 + 8 * (g.NS + s), ncw);    // one per consumer warp
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    const bool local = a.sq == nullptr && a.sk == nullptr;
+
+    if (warp == ncw) {
+        // ---------------------------------------------------------- producer
+        const uint64_t pol = lw_evict_first();
+        const bool totals = MODE == kTokFwd && !local;
+        int s_cur = (int)(t_lo % a.S);  // row position of the tile's first token
+        const LwCsWork<V> csw(s_step, half, lane);
+        int issued = 0;
+        for (int i = 0; i < ntiles; ++i) {
+            const int s = i % g.NS;
+            const uint32_t ph = (uint32_t)(i / g.NS) & 1u;
+            const int64_t t0 = t_lo + (int64_t)i * g.TT;
+            const int na = (int)min((int64_t)g.TT, t_hi - t0);
+            // per-token values, loaded before the wait for the slot
+            float2 v = make_float2(0.f, 0.f);
+            int32_t pos = 0;
+            if (lane < na) {
+                const int64_t t = t0 + lane;
+                if (totals) {
+                    v.x = a.Hq ? a.sq[t] : 0.f;
+                    v.y = a.Hkv ? a.sk[t] : 0.f;
+                }
+                if (half > 0) {
+                    if (a.pos) {
+                        pos = a.pos[t];
+                    } else {
+                        int p = s_cur + lane;
+                        while (p >= a.S) p -= a.S;
+                        pos = p;
+                    }
+                }
+            }
+            s_cur += g.TT;
+            while (s_cur >= a.S) s_cur -= a.S;
+            if (i >= g.NS && !lw_wait(bar0 + 8 * (g.NS + s), ph ^ 1u)) break;
+            unsigned char *st = ring + (size_t)s * g.stage_bytes;
+            const uint32_t full = bar0 + 8 * s;
+            if (lane == 0) {
+                const uint32_t bq = (uint32_t)(na * a.Hq * rowb);
+                const uint32_t bk = (uint32_t)(na * a.Hkv * rowb);
+                lw_bar_expect(full, bq + bk);
+                if (bq) lw_bulk(lw_smem_u32(st), (const char *)a.q + t0 * a.Hq * rowb, bq, full, pol);
+                if (bk)
+                    lw_bulk(lw_smem_u32(st + g.off_k), (const char *)a.k + t0 * a.Hkv * rowb, bk,
+                            full, pol);
+            }
+            if (totals && lane < na) reinterpret_cast<float2 *>(st + g.off_sc)[lane] = v;
+            if (half > 0) {
+                if (lane < na) s_pos[lane] = pos;
+                __syncwarp();
+                csw.fill(reinterpret_cast<float4 *>(st + g.off_cs), s_pos, s_step, na, lane);
+                __syncwarp();
+            }
+            lw_bar_arrive(full);
+            ++issued;
+        }
+        // leave only once every copy issued has landed
+        for (int i = max(0, issued - g.NS); i < issued; ++i)
+            if (!lw_wait(bar0 + 8 * (i % g.NS), (uint32_t)(i / g.NS) & 1u)) break;
+        return;
+    }
+
+    // ---------------------------------------------------------------- consumers
+    const Lane<LPR, V> L(lane, a.D, a.R);
+    const int offA = L.eA * E, offB = L.eB * E;
+    // the sums use the lane layout without a rotary span (the statistics
+    // call has none), so every call adds the same terms in the same order
+    const Lane<LPR, V> Ls(lane, a.D, 0);
+    const int offAs = Ls.eA * E, offBs = Ls.eB * E;
+    const int hp = half >> 1;  // rotary pairs per token
+    int pc = 0;                // tokens dealt before this stage, mod ncw
+    for (int i = 0; i < ntiles; ++i) {
+        const int s = i % g.NS;
+        if (!lw_wait(bar0 + 8 * s, (uint32_t)(i / g.NS) & 1u)) break;
+        const int64_t t0 = t_lo + (int64_t)i * g.TT;
+        const int na = (int)min((int64_t)g.TT, t_hi - t0);
+        const unsigned char *st = ring + (size_t)s * g.stage_bytes;
+        int j = warp - pc;
+        if (j < 0) j += ncw;
+        for (; j < na; j += ncw) {
+            const int64_t t = t0 + j;
+            const unsigned char *xq = st + j * a.Hq * rowb;
+            const unsigned char *xk = st + g.off_k + j * a.Hkv * rowb;
+            float2 tot;
+            if (MODE == kTokStats || local) {
+                tot = tok_sumsq<T, LPR>(xq, xk, Ls, a.Hq, H, rowb, offAs, offBs);
+            } else {
+                tot = reinterpret_cast<const float2 *>(st + g.off_sc)[j];
+            }
+            if (MODE == kTokStats) {
+                if (lane == 0) {
+                    if (a.Hq) a.wq[t] = tot.x;
+                    if (a.Hkv) a.wk[t] = tot.y;
+                }
+                continue;
+            }
+            const float rq = a.Hq ? rsqrtf(fmaf(tot.x, a.inv_q, a.eps)) : 0.f;
+            const float rk = a.Hkv ? rsqrtf(fmaf(tot.y, a.inv_k, a.eps)) : 0.f;
+            if (lane == 0) {
+                if (a.Hq) a.wq[t] = rq;
+                if (a.Hkv) a.wk[t] = rk;
+            }
+            float4 c[V / 2];
+            lane_cs4<V>(c, reinterpret_cast<const float4 *>(st + g.off_cs) + j * hp, L,
+                        hp / (V / 2));
+            for (int p = 0; p < H; p += SLOTS) {
+                const int h = p + L.slot;
+                if (!(L.on && h < H)) continue;
+                const bool isq = h < a.Hq;
+                const int hh = isq ? h : h - a.Hq;
+                const unsigned char *row = isq ? xq + h * rowb : xk + hh * rowb;
+                const unsigned char *grow = s_gamma + h * rowb;
+                const Vec16 xa = ld16(row + offA), xb = ld16(row + offB);
+                const Vec16 ga = ld16(grow + offA), gb = ld16(grow + offB);
+                const float r = isq ? rq : rk;
+                const float2 r2 = make_float2(r, r);
+                Vec16 ya, yb;
+#pragma unroll
+                for (int k2 = 0; k2 < V / 2; ++k2) {
+                    // r folded into cos and sin: y_A = u_A (r c) - u_B (r s),
+                    // y_B = u_B (r c) + u_A (r s), u = x gamma
+                    const float2 cr = __fmul2_rn(make_float2(c[k2].x, c[k2].y), r2);
+                    const float2 sr = __fmul2_rn(make_float2(c[k2].z, c[k2].w), r2);
+                    const float2 ua = __fmul2_rn(IO::get2(xa, k2), IO::get2(ga, k2));
+                    const float2 ub = __fmul2_rn(IO::get2(xb, k2), IO::get2(gb, k2));
+                    const float2 oa = __ffma2_rn(ua, cr, __fmul2_rn(ub, neg2f(sr)));
+                    const float2 ob = __ffma2_rn(ub, cr, __fmul2_rn(ua, sr));
+                    IO::put2(ya, k2, oa.x, oa.y);
+                    IO::put2(yb, k2, ob.x, ob.y);
+                }
+                char *out = (char *)(isq ? a.qo : a.ko) + ((isq ? t * a.Hq : t * a.Hkv) + hh) * rowb;
+                lw_st_stream(out + offA, ya);
+                lw_st_stream(out + offB, yb);
+            }
+        }
+        pc = (pc + na) % ncw;
+        __syncwarp();
+        if (lane == 0) lw_bar_arrive(bar0 + 8 * (g.NS + s));
     }
 }
 
@@ -947,6 +1223,55 @@ bool lw_plan(int mode, const LwArgs &a, int esz, int lpr, int sms, LwGeom *g, in
     return true;
 }
 
+// Stage and ring sizes of the pipelined statistics and forward, or false if
+// the shape does not fit them. One plan serves both kernels (the statistics
+// leave the angle and weight sections unused), so a shape runs both phases of
+// a sharded call in the same kernel family as the one-pass forward.
+bool lw_tok_plan(const LwArgs &a, int esz, int sms, LwTokGeom *g, int *grid, int *smem,
+                 int *threads) {
+    if ((a.D / (16 / esz)) & 1) return false;  // a half unit: the plain-load kernels take it
+    const int64_t rowb = (int64_t)a.D * esz;
+    const int64_t xq = (int64_t)a.Hq * rowb, xk = (int64_t)a.Hkv * rowb;  // per token
+    const int64_t csb = (int64_t)(a.R / 2) * 8;
+    const int64_t per = xq + xk + csb + 8;  // rows, angles, totals
+    int64_t TT = kLwTokStageTarget / per;
+    TT = TT > kMaxTileTokensLw ? kMaxTileTokensLw : (TT < 1 ? 1 : TT);
+    const int64_t off_cs = TT * (xq + xk);
+    const int64_t off_sc = off_cs + TT * csb;
+    const int64_t stage = ((off_sc + TT * 8 + 127) / 128) * 128;
+    const int64_t gbytes = ((xq + xk + 127) / 128) * 128;
+    const int64_t budget = kLwSmemBytes - 128 - gbytes;
+    int64_t NS = (budget < kLwRingBytes ? budget : kLwRingBytes) / stage;
+    if (NS > kLwMaxStages) NS = kLwMaxStages;
+    if (NS < 2 || off_cs > (1 << 20) - 1) return false;
+    g->TT = (int)TT;
+    g->NS = (int)NS;
+    g->stage_bytes = (int)stage;
+    g->off_k = (int)(TT * xq);
+    g->off_cs = (int)off_cs;
+    g->off_sc = (int)off_sc;
+    g->off_gamma = 128 + (int)(NS * stage);
+    g->ncw = kLwCWMax;
+    const int64_t tiles = (a.T + TT - 1) / TT;
+    int64_t nb = tiles < (int64_t)sms ? tiles : (int64_t)sms;
+    g->tpc = (a.T + nb - 1) / nb;
+    nb = (a.T + g->tpc - 1) / g->tpc;
+    *grid = (int)nb;
+    *smem = g->off_gamma + (int)gbytes;
+    *threads = (g->ncw + 1) * 32;
+    return true;
+}
+
+template <typename T, int LPR, int MODE>
+qknr_status lw_tok_launch(const LwArgs &a, const LwTokGeom &g, int grid, int smem, int threads,
+                          cudaStream_t st) {
+    auto kern = qknr_lw_tok_kernel<T, LPR, MODE>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return cuda_fail(e);
+    kern<<<grid, threads, smem, st>>>(a, g);
+    return cuda_status();
+}
+
 template <typename T, int LPR, int MODE>
 qknr_status lw_pipe_launch(const LwArgs &a, const LwGeom &g, int grid, int smem, int threads,
                            cudaStream_t st) {
@@ -959,11 +1284,21 @@ qknr_status lw_pipe_launch(const LwArgs &a, const LwGeom &g, int grid, int smem,
 
 template <typename T, int LPR>
 qknr_status lw_launch_t(LwKernel which, const LwArgs &a, cudaStream_t st) {
-    // The statistics and the forward read a token's rows, reduce and write:
-    // one warp per token with plain loads measured faster on B200 than the
-    // staged pipeline (whose per-stage cross-warp sum costs more than it
-    // saves there), so only the dots and the backward, whose dgamma sums
-    // need fixed row ownership, take the pipeline.
+    // The statistics and the forward take the token-per-warp pipeline (no
+    // cross-warp sums); the dots and the backward, whose dgamma sums need
+    // fixed row ownership, take the head-block pipeline. Shapes neither fits
+    // run the plain-load kernels.
+    if (!simple_kernels_forced() && (which == LwKernel::kStats || which == LwKernel::kFwd)) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        LwTokGeom g;
+        int grid, smem, thr;
+        if (lw_tok_plan(a, (int)sizeof(T), sm_count_of(dev), &g, &grid, &smem, &thr)) {
+            return which == LwKernel::kStats
+                       ? lw_tok_launch<T, LPR, kTokStats>(a, g, grid, smem, thr, st)
+                       : lw_tok_launch<T, LPR, kTokFwd>(a, g, grid, smem, thr, st);
+        }
+    }
     if (!simple_kernels_forced() && (which == LwKernel::kDots || which == LwKernel::kBwd)) {
         int dev = 0;
         cudaGetDevice(&dev);
@@ -1067,6 +1402,12 @@ qknr_status lw_run(LwKernel which, LwArgs a, qknr_dtype dtype, qknr_stream_t str
 
 namespace qknr {
 
+// Launches the layerwise family's wait self-test.
+qknr_status lw_wait_selftest(long long limit, cudaStream_t st) {
+    qknr_lw_wait_selftest_kernel<<<1, 32, 0, st>>>(limit);
+    return cuda_status();
+}
+
 // The pipelined layerwise kernels' error flag (see g_lw_error); -1 if it
 // cannot be read.
 int lw_pipeline_error(int reset) {
@@ -1086,7 +1427,7 @@ using namespace qknr;
 extern "C" qknr_status qk_layerwise_geometry(int mode, int B, int S, int Hq, int Hkv, int D,
                                              int rotary_dim, qknr_dtype dtype, int sms,
                                              int64_t *geom) {
-    if (!geom || (mode != 0 && mode != 1) || sms < 1) return QKNR_ERR_INVALID_ARG;
+    if (!geom || mode < 0 || mode > 2 || sms < 1) return QKNR_ERR_INVALID_ARG;
     qknr_status s = lw_check(B, S, Hq, Hkv, Hq, Hkv, D, rotary_dim, 1.f, 0.f, dtype);
     if (s != QKNR_OK) return s;
     if (mode == 1 && (int64_t)(Hq + Hkv) * D * 4 > kLwMaxDgammaBytes) return QKNR_ERR_UNSUPPORTED;
@@ -1096,8 +1437,18 @@ extern "C" qknr_status qk_layerwise_geometry(int mode, int B, int S, int Hq, int
     a.T = (int64_t)B * S; a.S = S; a.Hq = Hq; a.Hkv = Hkv; a.D = D; a.R = rotary_dim;
     if (a.T == 0 || Hq + Hkv == 0) return QKNR_OK;
     const int lpr = lpr_of(D, esz);
-    LwGeom g;
     int grid, smem, thr;
+    if (mode == 2) {
+        LwTokGeom t;
+        if (!lw_tok_plan(a, esz, sms, &t, &grid, &smem, &thr)) return QKNR_OK;
+        const int64_t v[kLwGeomLen] = {1, lpr, t.TT, t.NS, t.stage_bytes, t.off_k, 0, 0,
+                                       t.off_cs, t.off_sc, 0, t.off_gamma, 1, t.ncw,
+                                       (Hq + Hkv + 32 / lpr - 1) / (32 / lpr), t.tpc, grid, smem,
+                                       thr};
+        for (int i = 0; i < kLwGeomLen; ++i) geom[i] = v[i];
+        return QKNR_OK;
+    }
+    LwGeom g;
     if (!lw_plan(mode == 0 ? kLwDots : kLwBwd, a, esz, lpr, sms, &g, &grid, &smem, &thr))
         return QKNR_OK;
     const int64_t v[kLwGeomLen] = {1, lpr, g.TT, g.NS, g.stage_bytes, g.off_k, g.off_dq,

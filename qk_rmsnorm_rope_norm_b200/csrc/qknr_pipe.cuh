@@ -86,12 +86,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 // Wait until the phase of parity `parity` has completed, for at most
-// kWaitLimitCycles SM clock cycles (about 2-4 s; the cycle counter is cheap
-// to read, unlike the global timer); false on expiry, with the error flag
-// set. After a few tries a waiting warp may sleep between tests (backing off
-// from 32 ns to `max_sleep` ns) so waiters leave the issue slots to the warps
-// doing work.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t max_sleep = 256) {
+// `limit` SM clock cycles (by default kWaitLimitCycles, about 2-4 s; the
+// cycle counter is cheap to read, unlike the global timer); false on expiry,
+// with the error flag set. After a few tries a waiting warp may sleep between
+// tests (backing off from 32 ns to `max_sleep` ns) so waiters leave the issue
+// slots to the warps doing work. The clock is read every 256th test, and
+// every test is itself bounded (its suspend hint), so the wait ends.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t max_sleep = 256,
+                                          long long limit = kWaitLimitCycles) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long c0 = clock64();
     uint32_t nap = 32;
@@ -102,12 +104,39 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_
             __nanosleep(nap);
             nap = nap < max_sleep ? nap * 2 : max_sleep;
         }
-        if ((n & 255u) == 0 && clock64() - c0 > kWaitLimitCycles) {
+        if ((n & 255u) == 0 && clock64() - c0 > limit) {
             atomicOr(&g_qknr_pipe_error, 1u);
             return false;
         }
     }
 }
+
+// Diagnostic: one thread waits, with mbar_wait and a limit of `limit`
+// cycles, on a barrier nothing arrives on, so the wait gives up and sets the
+// error flag; the kernel then returns. It checks the timeout path without a
+// fault or a hang.
+__global__ void qknr_wait_selftest_kernel(long long limit) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x != 0) return;
+    const uint32_t b = smem_u32(&bar);
+    mbar_init(b, 1);
+    fence_mbar_init();
+    mbar_wait(b, 0, 256, limit);
+}
+// Programmatic dependent launch. The pipelined kernels are launched with
+// programmatic stream serialization allowed, so a kernel's CTAs may start
+// while the previous kernel of the stream is still finishing: everything
+// before grid_dep_wait() touches only the CTA's own shared memory (and, on
+// the misaligned-shared-memory error path, the library's own error flag), and
+// no input or output is read or written before it returns (the previous
+// kernel has then completed and its writes are visible). grid_dep_launch() lets the next
+// kernel of the stream start its own prologue once every CTA of this one has
+// passed that point. Both are no-ops for a launch without the attribute.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Named barrier over the consumer warps only (id 1; id 0 is __syncthreads).
 __device__ __forceinline__ void consumers_sync(int nthreads) {
     asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
@@ -435,11 +464,15 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g,
     const uint32_t full0 = smem_u32(&bars[0]), empty0 = smem_u32(&bars[kMaxStages]);
     init_barriers<NCW, NPW>(full0, empty0, g);
     if (threadIdx.x == 0) s_abort = 0;
+    const int half = a.R >> 1;
+    // the angle steps depend on the arguments only: taken before the wait
+    for (int i = threadIdx.x; i < half; i += blockDim.x) s_step[i] = turn_step(i, a.R, a.theta);
+    grid_dep_wait();
+    grid_dep_launch();
     __syncthreads();
 
     const Run run(a.T, g);
     const int rowb = a.D * (int)sizeof(T);
-    const int half = a.R >> 1;
 
     if (warp < NPW) {
         // ----------------------------------------------------- producers
@@ -473,8 +506,6 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g,
         const int first = min(g.NS, run.ntiles);
         if (pw == 0 && lane == 0)
             for (int it = 0; it < first; ++it) issue(it);
-        for (int i = pw * 32 + lane; i < half; i += 32 * NPW) s_step[i] = turn_step(i, a.R, a.theta);
-        producers_sync(32 * NPW);
         int issued = first;
         int s_row = run.ntiles ? (int)(run.t_lo % a.S) : 0;  // row position of the tile's first token
         int32_t pos_next = tile_pos(a.pos, a.S, run.t_lo, s_row,
@@ -669,11 +700,15 @@ qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g,
     init_barriers<NCW, NPW>(full0, empty0, g);
     if (threadIdx.x == 0) s_abort = 0;
     for (int i = threadIdx.x; i < 2 * kMaxD; i += blockDim.x) (&s_dg[0][0])[i] = 0.f;
+    const int half = a.R >> 1;
+    // the angle steps depend on the arguments only: taken before the wait
+    for (int i = threadIdx.x; i < half; i += blockDim.x) s_step[i] = turn_step(i, a.R, a.theta);
+    grid_dep_wait();
+    grid_dep_launch();
     __syncthreads();
 
     const Run run(a.T, g);
     const int rowb = a.D * (int)sizeof(T);
-    const int half = a.R >> 1;
 
     if (warp < NPW) {
         // ----------------------------------------------------- producers
@@ -713,8 +748,6 @@ qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g,
         const int first = min(g.NS, run.ntiles);
         if (pw == 0 && lane == 0)
             for (int it = 0; it < first; ++it) issue(it);
-        for (int i = pw * 32 + lane; i < half; i += 32 * NPW) s_step[i] = turn_step(i, a.R, a.theta);
-        producers_sync(32 * NPW);
         int issued = first;
         int s_row = run.ntiles ? (int)(run.t_lo % a.S) : 0;  // row position of the tile's first token
         int32_t pos_next = tile_pos(a.pos, a.S, run.t_lo, s_row,

@@ -293,3 +293,24 @@ def test_layerwise_validation(lib):
     assert lib.qk_layerwise_norm_rope_bwd(P(1), P(2), P(3), P(4), None, P(7), P(8), P(11),
                                           P(12), None, None, P(15), P(16), P(17), P(18), 2, 8,
                                           4, 2, 4, 4, 128, 128, 1e4, BF16, None) == INVALID
+
+
+def test_wait_selftest_validation(lib):
+    # bad family or limit: refused before any CUDA call
+    assert lib.qknr_wait_selftest(2, 1000, None) == INVALID
+    assert lib.qknr_wait_selftest(0, 0, None) == INVALID
+    assert lib.qknr_wait_selftest(1, 1 << 40, None) == INVALID
+
+
+def test_plan_query_validation(lib):
+    plan = (ctypes.c_int64 * 14)()
+    pp = ctypes.cast(plan, ctypes.c_void_p)
+    assert lib.qk_norm_rope_plan(4, 2, 8, 4, 2, 64, 64, BF16, 0, 148, 0, pp) == INVALID
+    assert lib.qk_norm_rope_plan(0, 2, 8, 4, 2, 64, 64, BF16, 4, 148, 0, pp) == INVALID
+    assert lib.qk_norm_rope_plan(0, 2, 8, 4, 2, 64, 64, BF16, 0, 0, 0, pp) == INVALID
+    assert lib.qk_norm_rope_plan(0, 2, 8, 4, 2, 64, 64, BF16, 0, 148, 0, None) == INVALID
+    assert lib.qk_norm_rope_plan(0, 2, 8, 4, 2, 63, 0, BF16, 0, 148, 0, pp) == INVALID
+    assert lib.qk_norm_rope_plan(1, 2, 8, 4, 2, 64, 8, BF16, 0, 148, 0, pp) == UNSUP
+    # the bench shapes: pipelined, one CTA per SM at most
+    assert lib.qk_norm_rope_plan(1, 1, 65536, 32, 8, 128, 32, BF16, 0, 148, 0, pp) == OK
+    assert plan[0] == 1 and plan[11] == 148 and plan[13] == (plan[3] + plan[4]) * 32

@@ -159,3 +159,112 @@ def test_geometry_rejects_bad_arguments(lib):
         qknr.layerwise_geometry("bwd", 1, 8, 4, 2, 64, 64, sms=0)
     g = qknr.layerwise_geometry("bwd", 1, 9, 64, 8, 256, 128, torch.float32)
     assert g["pipelined"] == 0  # too large for the ring: the plain-load kernels
+
+
+def replay_tok(B, S, Hq, Hkv, D, R, dtype, sms=148):
+    """The statistics / forward pipeline: CTA token runs, stages of TT
+    tokens, whole tokens dealt round-robin to the consumer warps (continuing
+    across stages), every row of a token covered by the warp's lanes, the
+    producer's (cos, sin) work split, and the shared-memory sections."""
+    g = qknr.layerwise_geometry("tok", B, S, Hq, Hkv, D, R, dtype, sms)
+    if not g["pipelined"]:
+        return None
+    e = 4 if dtype == torch.float32 else 2
+    V = 16 // e
+    Dv2 = D // (2 * V)
+    rowb = D * e
+    H = Hq + Hkv
+    T = B * S
+    lpr, TT, NS, stage, ncw = g["lpr"], g["TT"], g["NS"], g["stage_bytes"], g["NTG"]
+    slots = 32 // lpr
+    assert g["G"] == 1 and ncw <= MAX_CONSUMER_WARPS and g["threads"] == (ncw + 1) * 32
+    assert 1 <= TT <= 32
+    assert g["off_k"] == TT * Hq * rowb and g["off_cs"] == TT * H * rowb
+    assert g["off_sc"] == g["off_cs"] + TT * (R // 2) * 8
+    assert g["off_sc"] + 8 * TT <= stage and stage % 128 == 0
+    for k in ("off_k", "off_cs", "off_sc"):
+        assert g[k] % 16 == 0, k
+    assert TT * H * rowb <= TX_LIMIT
+    assert NS >= 2 and g["off_gamma"] == 128 + NS * stage
+    assert g["smem"] >= g["off_gamma"] + H * rowb and g["smem"] <= SMEM_LIMIT
+    # the producer's (cos, sin) table: every (token, angle pair) exactly once,
+    # inside the token's hp float4 entries
+    hp = R // 4
+    if hp:
+        tpp = 32 // hp if hp <= 32 else 0
+        for na in {TT, max(1, TT - 1), 1}:
+            cells = set()
+            for lane in range(32):
+                if tpp:
+                    if lane >= tpp * hp:
+                        continue
+                    jo, P = divmod(lane, hp)
+                    pairs, toks = [P], range(jo, na, tpp)
+                else:
+                    pairs, toks = range(lane, hp, 32), range(na)
+                for P in pairs:
+                    pw = P // (V // 2)
+                    dst = (P - pw * (V // 2)) * (hp // (V // 2)) + pw
+                    assert 0 <= dst < hp
+                    for j in toks:
+                        assert (j, dst) not in cells
+                        cells.add((j, dst))
+            assert len(cells) == na * hp
+    # CTA runs, stages, token dealing, rows of a token
+    grid, tpc = g["grid"], g["tpc"]
+    assert 1 <= grid <= sms and (grid - 1) * tpc < T <= grid * tpc
+    seen = set()
+    for cta in range(grid):
+        t_lo, t_hi = cta * tpc, min(T, (cta + 1) * tpc)
+        pc = 0
+        for i in range(ceil_div(t_hi - t_lo, TT)):
+            t0 = t_lo + i * TT
+            na = min(TT, t_hi - t0)
+            assert 1 <= na <= TT and t0 + na <= T
+            for w in range(ncw):
+                j = (w - pc) % ncw
+                for jj in range(j, na, ncw):
+                    for p in range(0, H, slots):
+                        for lane in range(32):
+                            slot, u = divmod(lane, lpr)
+                            h = p + slot
+                            if u >= Dv2 or h >= H:
+                                continue
+                            key = (t0 + jj, h, u)
+                            assert key not in seen, key
+                            seen.add(key)
+            pc = (pc + na) % ncw
+    assert len(seen) == T * H * Dv2
+    return g
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=[f"{s[2]}x{s[3]}x{s[4]}-R{s[5]}-T{s[0] * s[1]}"
+                                               for s in SHAPES])
+def test_token_plan_of_listed_shapes(lib, shape):
+    assert replay_tok(*shape) is not None
+
+
+def test_token_plan_of_random_shapes(lib):
+    rng = random.Random(11)
+    planned = 0
+    for _ in range(60):
+        dt = rng.choice([torch.bfloat16, torch.float32])
+        e = 4 if dt == torch.float32 else 2
+        D = rng.choice([d for d in (16, 24, 32, 48, 64, 96, 128, 192, 256) if d * e % 32 == 0])
+        R = rng.choice([r for r in range(0, D + 1, 2) if (r // 2) * e % 16 == 0])
+        Hq, Hkv = rng.randint(0, 40), rng.randint(0, 9)
+        if Hq + Hkv == 0:
+            continue
+        B, S = rng.randint(1, 3), rng.randint(1, 90)
+        planned += replay_tok(B, S, Hq, Hkv, D, R, dt, rng.choice([148, 132, 7])) is not None
+    assert planned > 40
+
+
+def test_token_plan_of_bench_shapes(lib):
+    # the bench shapes take the token pipeline and keep every SM busy
+    for shape in ((8, 2048, 14, 2, 64, 64), (4, 8192, 32, 8, 128, 128),
+                  (1, 65536, 32, 8, 128, 32)):
+        g = qknr.layerwise_geometry("tok", *shape, torch.bfloat16, 148)
+        assert g["pipelined"] and g["grid"] == 148
+    # an odd number of 16-byte vectors per row runs the plain-load kernels
+    assert not qknr.layerwise_geometry("tok", 1, 64, 4, 2, 72, 64, torch.bfloat16)["pipelined"]
