@@ -8,12 +8,13 @@ A step is one forward and one backward over one batch of the workload
 (default: the largest single-GPU configuration, partial RoPE at long
 context: one row of 65,536 tokens, 32 query / 8 KV heads of dim 128, rotary
 on the first 32 dims, bf16 I/O). Inputs are resident in HBM before timing.
-Each rank keeps a ring of four input/output sets; step i runs the forward on
-set i mod 4 and the backward on set (i - 2) mod 4 (a layer's backward comes
-after the rest of the forward in training), so no kernel finds its inputs in
-the 126 MB L2. K steps are timed with CUDA events between a barrier and a
-synchronize on both sides; every fwd/bwd launch is also bracketed by events
-on its stream for the per-kernel roofline. N > 1 (torchrun): weak scaling,
+Each rank keeps a ring of input/output sets (four, more for small
+workloads); step i runs the forward on set i and the backward on set i - 2
+(a layer's backward comes after the rest of the forward in training), so no
+kernel finds its inputs in the 126 MB L2. K steps are timed with CUDA events
+between a barrier and a synchronize on both sides, with no event between the
+launches; then K forward launches alone and K backward launches alone, back
+to back, give the per-kernel times for the roofline. N > 1 (torchrun): weak scaling,
 each rank its own batch, no collective on the data path; the time is the
 max over ranks.
 
@@ -47,6 +48,7 @@ import workloads  # noqa: E402
 METRIC = "QK-norm+RoPE fwd+bwd tokens/s and HBM GB/s (% of B200 peak), 1 GPU"
 FALLBACK_HBM_GBS = 6650.0
 NSETS, LAG = 4, 2  # ring of input sets; the backward runs LAG steps behind
+L2_BYTES = 126 * 1024 * 1024
 # the workloads timed beside the headline one (one GPU each); the tiny fp32
 # case is a parity check, not a throughput workload
 PER_CONFIG = ("qwen2.5-0.5b", "llama3-8b-qknorm", "partial-rope-64k", "bfd-packed")
@@ -229,17 +231,25 @@ class Set:
         self.dgk = torch.empty(w.D, dtype=torch.float32, device=dev)
 
 
+def ring_sets(w, nsets: int) -> int:
+    """Input sets in the ring: at least ``nsets``, and enough that ~2.5x the
+    126 MB L2 of other traffic passes between two touches of a set even in a
+    loop of one direction alone."""
+    cb = workloads.contract_bytes(w)
+    need = int(2.5 * L2_BYTES / max(1, min(cb["fwd"], cb["bwd"]))) + 2
+    return max(nsets, min(need, 16))
+
+
 def measure(w, inp, dev, steps: int, warmup: int, nsets: int, layout: str = "dense",
             world: int = 1, clocks=None):
-    """Time ``steps`` fwd + bwd steps of workload ``w`` on a ring of ``nsets``
-    input sets (after ``warmup`` untimed steps): first with events only at
-    the two ends (the step time; the kernels run back to back, each one's
-    prologue overlapping the previous one's tail), then the same number of
-    steps again with events around every launch (the per-kernel split; an
-    event between two launches serialises them, so this split includes the
-    launch gaps the first pass hides). Returns the total, mean forward, mean
-    backward and split-pass total milliseconds, the max over ranks when
-    ``world`` > 1."""
+    """Time ``steps`` fwd + bwd steps of workload ``w`` on a ring of input
+    sets (after ``warmup`` untimed steps), with events only at the two ends
+    of the timed region (the step time: the kernels run back to back, each
+    one's prologue overlapping the previous one's tail). Then each direction
+    alone: ``steps`` forward launches back to back, and ``steps`` backward
+    launches, each loop timed by events at its ends (the per-kernel times).
+    Returns the step total, the mean forward and mean backward launch
+    milliseconds, the max over ranks when ``world`` > 1."""
     import qk_rmsnorm_rope_norm_b200 as qknr
     cfg = dict(rotary_dim=w.rotary_dim, theta=w.theta, eps=w.eps)
     sets = [Set(inp, dev, layout) for _ in range(nsets)]
@@ -249,18 +259,13 @@ def measure(w, inp, dev, steps: int, warmup: int, nsets: int, layout: str = "den
     bwd = [qknr.prepare_bwd(s.q, s.k, s.gq, s.gk, s.pos, s.rq, s.rk, s.dqo, s.dko, s.dq,
                             s.dk, s.dgq, s.dgk, **cfg) for s in sets]
     K, W = steps, warmup
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
 
-    def step(i, e=None):
-        if e is not None:
-            e[0].record(stream)
+    def step(i):
         fwd[i % nsets]()
-        if e is not None:
-            e[1].record(stream)
         bwd[(i - LAG) % nsets]()
-        if e is not None:
-            e[2].record(stream)
+
+    def events():
+        return torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
 
     for i in range(W):
         step(i)
@@ -268,27 +273,30 @@ def measure(w, inp, dev, steps: int, warmup: int, nsets: int, layout: str = "den
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
+    t0, t1 = events()
     with (clocks if clocks is not None else _Null()):
-        t_start.record(stream)
+        t0.record(stream)
         for i in range(K):
             step(W + i)
-        t_end.record(stream)
+        t1.record(stream)
         torch.cuda.synchronize(dev)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
-    total_ms = t_start.elapsed_time(t_end)
-    s_start, s_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s_start.record(stream)
-    for i in range(K):
-        step(W + K + i, ev[i])
-    s_end.record(stream)
-    torch.cuda.synchronize(dev)
-    split_ms = s_start.elapsed_time(s_end)
-    fwd_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / K
-    bwd_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / K
+    total_ms = t0.elapsed_time(t1)
+    per = []
+    for calls in (fwd, bwd):
+        for i in range(3):
+            calls[i % nsets]()
+        a, b = events()
+        a.record(stream)
+        for i in range(K):
+            calls[(W + i) % nsets]()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        per.append(a.elapsed_time(b) / K)
     del fwd, bwd, sets
-    return max_over_ranks([total_ms, fwd_ms, bwd_ms, split_ms], world, dev)
+    return max_over_ranks([total_ms, per[0], per[1]], world, dev)
 
 
 class _Null:
@@ -305,15 +313,16 @@ def run_ours(args, w, inp, rank, local_rank, world):
     qknr.load_library()
     cfg = dict(rotary_dim=w.rotary_dim, theta=w.theta, eps=w.eps)
     clocks = ClockSampler(local_rank)  # NVML start-up stays outside the timed region
-    total_ms, fwd_ms, bwd_ms, split_ms = measure(w, inp, dev, args.steps, args.warmup,
-                                                 args.sets, args.layout, world, clocks)
+    nsets = ring_sets(w, args.sets) if args.sets == NSETS else args.sets
+    total_ms, fwd_ms, bwd_ms = measure(w, inp, dev, args.steps, args.warmup, nsets,
+                                       args.layout, world, clocks)
     torch.cuda.empty_cache()
     e2e = None
     if not args.no_e2e:
         e2e = run_e2e(args, w, inp, dev, cfg, world)
     cb = workloads.contract_bytes(w, with_pos=inp.pos is not None)
     floor = {"fwd_ms": copy_floor_ms(cb["fwd"], dev), "bwd_ms": copy_floor_ms(cb["bwd"], dev)}
-    return dict(total_ms=total_ms, fwd_ms=fwd_ms, bwd_ms=bwd_ms, split_ms=split_ms,
+    return dict(total_ms=total_ms, fwd_ms=fwd_ms, bwd_ms=bwd_ms, nsets=nsets,
                 clocks=clocks.summary(), e2e=e2e, floor=floor)
 
 
@@ -360,7 +369,8 @@ def run_per_config(args, main_w, main_r, rank, dev, peak):
             inp = workloads.make_inputs(base, seed=rank_seed(base, rank))
             w = inp.w
             steps = args.per_config_steps
-            total_ms, fwd_ms, bwd_ms, _ = measure(w, inp, dev, steps, max(3, args.warmup), NSETS)
+            total_ms, fwd_ms, bwd_ms = measure(w, inp, dev, steps, max(3, args.warmup),
+                                               ring_sets(w, NSETS))
             torch.cuda.empty_cache()
         out[name] = per_config_line(w, inp, fwd_ms, bwd_ms, peak, dev, steps)
         out[name]["ms_per_step"] = (main_r["total_ms"] / args.steps if name == main_w.name
@@ -373,8 +383,8 @@ main_inp_cache = [None]
 
 def run_variants(args, w, inp, dev, peak):
     """The other entry points on the same workload, each timed like the main
-    step (a ring of input sets, CUDA events around every launch, mean over
-    the launches): the fused op on Q / K slices of a fused QKV buffer, the
+    step's per-kernel loops (a ring of input sets, launches back to back,
+    CUDA events at the loop ends, mean over the launches): the fused op on Q / K slices of a fused QKV buffer, the
     NoPE op (qk_norm_*), the mean-centred form (qk_layernorm_rope_*), the
     statistic alone (qk_rms_stats) and the rotation alone, forward and
     inverse (qk_rope_apply). Bytes are each call's contract bytes."""
@@ -394,28 +404,28 @@ def run_variants(args, w, inp, dev, peak):
         for c in calls[:3]:
             c()
         torch.cuda.synchronize(dev)
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(n_launch)]
-        for i, (a, b) in enumerate(ev):
-            a.record(stream)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(n_launch):
             calls[i % len(calls)]()
-            b.record(stream)
+        b.record(stream)
         torch.cuda.synchronize(dev)
-        return sum(a.elapsed_time(b) for a, b in ev) / n_launch
+        return a.elapsed_time(b) / n_launch
 
     def line(ms, nbytes):
         gbs = nbytes / (ms / 1e3) / 1e9
         return {"ms": ms, "gbs": gbs, "frac": gbs / peak, "bytes_per_launch": nbytes}
 
     out = {}
-    qkv = [Set(inp, dev, "qkv") for _ in range(args.sets)]
+    nsets = ring_sets(w, args.sets)
+    qkv = [Set(inp, dev, "qkv") for _ in range(nsets)]
     f = [qknr.prepare_fwd(s.q, s.k, s.gq, s.gk, s.pos, s.qo, s.ko, s.rq, s.rk, **cfg) for s in qkv]
     b = [qknr.prepare_bwd(s.q, s.k, s.gq, s.gk, s.pos, s.rq, s.rk, s.dqo, s.dko, s.dq, s.dk,
                           s.dgq, s.dgk, **cfg) for s in qkv]
     out["fused_qkv_layout"] = {"fwd": line(timed(f), cb["fwd"]), "bwd": line(timed(b), cb["bwd"]),
                                "entry": "qk_norm_rope_fwd_strided / qk_norm_rope_bwd_strided"}
     del qkv, f, b
-    dense = [Set(inp, dev) for _ in range(args.sets)]
+    dense = [Set(inp, dev) for _ in range(nsets)]
     P = qknr._ptr
     dt = 0 if w.dtype == "f32" else 1
     st = qknr._stream(None)
@@ -527,12 +537,36 @@ def layerwise_variants(w, dense, dev, timed, line):
     two_b = [seq(C(lib.qk_layerwise_bwd_dots, dots(s, b), "lw dots", s),
                  C(lib.qk_layerwise_norm_rope_bwd, bwd(s, b, True), "lw bwd", s))
              for s, b in zip(dense, bufs)]
+    def no_exchange(buf, span):  # one GPU: the sums are already the totals
+        return None
+
+    def chunked_f(s):
+        def run():
+            qknr.layerwise_chunked_fwd(s.q, s.k, gq, gk, s.pos, rotary_dim=w.rotary_dim,
+                                       theta=w.theta, eps=w.eps, Hq_total=w.Hq, Hkv_total=w.Hkv,
+                                       exchange=no_exchange,
+                                       chunks=qknr.DEFAULT_EXCHANGE_CHUNKS)
+        return run
+
+    def chunked_b(s, b):
+        def run():
+            qknr.layerwise_chunked_bwd(s.q, s.k, gq, gk, s.pos, b["rq"], b["rk"], s.dqo, s.dko,
+                                       rotary_dim=w.rotary_dim, theta=w.theta, Hq_total=w.Hq,
+                                       Hkv_total=w.Hkv, exchange=no_exchange,
+                                       chunks=qknr.DEFAULT_EXCHANGE_CHUNKS)
+        return run
+
     return {
         "layerwise_one_pass": {"fwd": line(timed(one_f), fwd_b), "bwd": line(timed(one_b), bwd_b),
                                "entry": "qk_layerwise_norm_rope_fwd / _bwd, sums NULL"},
         "layerwise_tp_phases": {"fwd": line(timed(two_f), fwd_b),
                                 "bwd": line(timed(two_b), bwd_b),
                                 "entry": "qk_layerwise_stats + _fwd; qk_layerwise_bwd_dots + _bwd"},
+        "layerwise_tp_chunked": {
+            "fwd": line(timed([chunked_f(s) for s in dense]), fwd_b),
+            "bwd": line(timed([chunked_b(s, b) for s, b in zip(dense, bufs)]), bwd_b),
+            "entry": f"layerwise_chunked_fwd / _bwd, {qknr.DEFAULT_EXCHANGE_CHUNKS} token chunks, "
+                     "side-stream exchange (here a no-op: one GPU holds every head)"},
     }
 
 
@@ -695,8 +729,8 @@ def config_of(w, inp, world):
     return {"workload": w.name, "B": w.B, "S": w.S, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
             "rotary_dim": w.rotary_dim, "theta": w.theta, "eps": w.eps, "io_dtype": w.dtype,
             "tokens_per_step": inp.real_tokens,
-            "l2": f"ring of {NSETS} input sets, bwd lags fwd by {LAG} steps: inputs not "
-                  f"L2-resident (> 2x 126 MB of traffic between touches)"
+            "l2": f"ring of {ring_sets(w, NSETS)} input sets, bwd lags fwd by {LAG} steps: "
+                  f"inputs not L2-resident (>= 2.5x 126 MB of traffic between touches)"
                   if getattr(cfg_args, "sets", NSETS) == NSETS else
                   f"{cfg_args.sets} input set(s): profiling run, inputs may be L2-resident",
             "layout": getattr(cfg_args, "layout", "dense"),
@@ -821,9 +855,8 @@ def main():
                     "bwd_gbs": cb["bwd"] / (r["floor"]["bwd_ms"] / 1e3) / 1e9,
                     "fwd_frac_of_copy": r["floor"]["fwd_ms"] / r["fwd_ms"],
                     "bwd_frac_of_copy": r["floor"]["bwd_ms"] / r["bwd_ms"]}},
-        "split_pass": {"ms_per_step": r["split_ms"] / args.steps,
-                       "what": "the same steps again with an event around every launch; "
-                               "fwd.ms and bwd.ms come from it"},
+        "per_kernel_timing": f"fwd.ms and bwd.ms: {args.steps} launches of each direction "
+                             f"alone, back to back on the same ring, events at the loop ends",
         "fwd": {"ms": r["fwd_ms"], "tokens_per_s": aggregate_tokens_per_s(world, tokens, r["fwd_ms"]),
                 "bytes_per_launch": cb["fwd"], "kernel": fwd_kernel},
         "bwd": {"ms": r["bwd_ms"], "tokens_per_s": aggregate_tokens_per_s(world, tokens, r["bwd_ms"]),

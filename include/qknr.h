@@ -370,9 +370,31 @@ QKNR_API qknr_status qk_layerwise_norm_rope_bwd(const void *q, const void *k,
                              qknr_dtype dtype, qknr_stream_t stream);
 
 /*
+ * qk_layerwise_norm_rope_bwd that adds to dgamma_q / dgamma_k instead of
+ * overwriting them (no zeroing): for a backward split into token chunks,
+ * each chunk's call adds its tokens' share, and the caller zeroes dgamma
+ * once before the first. Everything else as qk_layerwise_norm_rope_bwd.
+ */
+QKNR_API qknr_status qk_layerwise_norm_rope_bwd_acc(const void *q, const void *k,
+                             const void *gamma_q, const void *gamma_k,
+                             const int32_t *pos_ids,
+                             const float *rstd_q, const float *rstd_k,
+                             const void *dq_out, const void *dk_out,
+                             const float *dot_q, const float *dot_k,
+                             void *dq, void *dk,
+                             float *dgamma_q, float *dgamma_k,
+                             int B, int S, int Hq, int Hkv,
+                             int Hq_total, int Hkv_total, int D,
+                             int rotary_dim, float theta,
+                             qknr_dtype dtype, qknr_stream_t stream);
+
+/*
  * Launch geometry of the layerwise pipelined kernels for a shape, for
  * inspection and host-side checks; no CUDA call is made. mode 0: the dots
- * (qk_layerwise_bwd_dots), 1: the backward (qk_layerwise_norm_rope_bwd);
+ * (qk_layerwise_bwd_dots), 1: the backward (qk_layerwise_norm_rope_bwd),
+ * 2: the statistics and the forward (qk_layerwise_stats,
+ * qk_layerwise_norm_rope_fwd: one warp per token, so [12] is 1 and [13]
+ * the consumer warps, with no dQ_out / dK_out or partial-sum sections);
  * sms: the SM count to plan for. geom (19 int64, caller-owned) receives
  *   [0] 1 if the plan for `sms` SMs is the pipelined kernel, 0 if it is
  *       the plain-load kernel (then the rest is 0); this is the plan the

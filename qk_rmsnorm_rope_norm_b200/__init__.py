@@ -32,7 +32,8 @@ __all__ = ["qk_norm_rope_fwd", "qk_norm_rope_bwd", "qknr_strerror", "QKNormRoPE"
            "qk_layerwise_stats", "qk_layerwise_norm_rope_fwd", "qk_layerwise_bwd_dots",
            "qk_layerwise_norm_rope_bwd", "QKLayerwiseNormRoPE", "qk_layerwise_norm_rope",
            "all_reduce_stats", "layerwise_geometry", "launch_plan", "kernel_name",
-           "wait_selftest"]
+           "wait_selftest", "token_chunks", "run_chunked", "layerwise_chunked_fwd",
+           "layerwise_chunked_bwd"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libqknr.so")
@@ -96,6 +97,8 @@ def load_library():
     lib.qk_layerwise_bwd_dots.argtypes = [vp] * 11 + [i32] * 6 + [f32, i32, vp]
     lib.qk_layerwise_norm_rope_bwd.restype = i32
     lib.qk_layerwise_norm_rope_bwd.argtypes = [vp] * 15 + [i32] * 8 + [f32, i32, vp]
+    lib.qk_layerwise_norm_rope_bwd_acc.restype = i32
+    lib.qk_layerwise_norm_rope_bwd_acc.argtypes = lib.qk_layerwise_norm_rope_bwd.argtypes
     lib.qk_layerwise_geometry.restype = i32
     lib.qk_layerwise_geometry.argtypes = [i32] * 9 + [vp]
     lib.qk_norm_rope_plan.restype = i32
@@ -734,12 +737,13 @@ def qk_layerwise_bwd_dots(q, k, gamma_q, gamma_k, pos_ids, rstd_q, rstd_k, dq_ou
 def qk_layerwise_norm_rope_bwd(q, k, gamma_q, gamma_k, pos_ids, rstd_q, rstd_k, dq_out, dk_out,
                                dot_q, dot_k, *, rotary_dim: int, theta: float, Hq_total: int,
                                Hkv_total: int, dq=None, dk=None, dgamma_q=None, dgamma_k=None,
-                               need_dgamma: bool = True, stream=None):
+                               need_dgamma: bool = True, accumulate: bool = False, stream=None):
     """dq, dk and this rank's dgamma slices from the all-rank dot sums (C
     ``qk_layerwise_norm_rope_bwd``). Returns ``(dq, dk, dgamma_q, dgamma_k)``;
     dgamma fp32 [Hq*D] / [Hkv*D], or None without ``need_dgamma``.
     ``dot_q = dot_k = None``: this rank holds every head, and the dots are
-    taken in the same pass."""
+    taken in the same pass. ``accumulate``: add to the given dgamma instead
+    of overwriting it (C ``qk_layerwise_norm_rope_bwd_acc``)."""
     lib = load_library()
     B, S, Hq, Hkv, D = _lw_inputs(q, k, gamma_q, gamma_k, pos_ids)
     T = B * S
@@ -756,6 +760,8 @@ def qk_layerwise_norm_rope_bwd(q, k, gamma_q, gamma_k, pos_ids, rstd_q, rstd_k, 
         _need_cuda(n, t)
         if t.shape != ref.shape or t.dtype != ref.dtype:
             raise ValueError(f"{n} must match its input in shape and dtype")
+    if accumulate and need_dgamma and (dgamma_q is None or dgamma_k is None):
+        raise ValueError("accumulate needs the dgamma buffers to add to")
     if need_dgamma:
         dgamma_q = torch.empty(Hq * D, dtype=torch.float32, device=q.device) \
             if dgamma_q is None else dgamma_q
@@ -765,7 +771,8 @@ def qk_layerwise_norm_rope_bwd(q, k, gamma_q, gamma_k, pos_ids, rstd_q, rstd_k, 
             _need_cuda(n, t)
             if t.dtype != torch.float32 or t.numel() != m:
                 raise ValueError(f"{n} must be float32 with {m} elements")
-    st = lib.qk_layerwise_norm_rope_bwd(
+    fn = lib.qk_layerwise_norm_rope_bwd_acc if accumulate else lib.qk_layerwise_norm_rope_bwd
+    st = fn(
         _ptr(q), _ptr(k), _ptr(gamma_q), _ptr(gamma_k), _ptr(pos_ids), _ptr(rstd_q),
         _ptr(rstd_k), _ptr(dq_out), _ptr(dk_out), _ptr(dot_q), _ptr(dot_k), _ptr(dq), _ptr(dk),
         _ptr(dgamma_q if need_dgamma else None), _ptr(dgamma_k if need_dgamma else None),
@@ -776,6 +783,179 @@ def qk_layerwise_norm_rope_bwd(q, k, gamma_q, gamma_k, pos_ids, rstd_q, rstd_k, 
     return dq, dk, (dgamma_q if need_dgamma else None), (dgamma_k if need_dgamma else None)
 
 
+def token_chunks(T: int, n: int):
+    """[t0, t1) ranges of ``n`` near-equal runs covering tokens 0..T-1."""
+    n = max(1, min(int(n), T)) if T > 0 else 1
+    return [(T * i // n, T * (i + 1) // n) for i in range(n)]
+
+
+def run_chunked(n: int, partial, exchange, finish, lag: int = 1):
+    """The exchange schedule of a sharded layerwise call, over ``n`` token
+    chunks: ``partial(i)`` enqueues chunk i's per-token partial sums,
+    ``exchange(i)`` starts their sum over the ranks (on a side stream, or as
+    an asynchronous collective), and ``finish(i)`` waits for that sum and
+    enqueues the element-wise pass of chunk i. Chunk i is finished only after
+    chunk i + ``lag``'s partial sums are enqueued, so the exchange of chunk i
+    runs while the next chunk's statistics are taken ("SwiftQK", abstract:
+    the exchange of scalar statistics overlapped with element-wise work)."""
+    for i in range(n):
+        partial(i)
+        exchange(i)
+        if i >= lag:
+            finish(i - lag)
+    for j in range(max(0, n - lag), n):
+        finish(j)
+
+
+_COMM_STREAMS = {}
+
+
+def _comm_stream(device) -> torch.cuda.Stream:
+    idx = torch.device(device).index
+    if idx is None:
+        idx = torch.cuda.current_device()
+    st = _COMM_STREAMS.get(idx)
+    if st is None:
+        st = _COMM_STREAMS[idx] = torch.cuda.Stream(device=idx)
+    return st
+
+
+def _flat_tokens(t: torch.Tensor) -> torch.Tensor:
+    B, S = t.shape[0], t.shape[1]
+    return t.reshape((B * S,) + tuple(t.shape[2:]))
+
+
+def _chunk_positions(pos_ids, B: int, S: int, device) -> torch.Tensor:
+    """Every token's position as int32 [B*S] (the given ids, else s)."""
+    if pos_ids is not None:
+        return pos_ids.reshape(B * S)
+    return (torch.arange(B * S, device=device, dtype=torch.int64) % S).to(torch.int32)
+
+
+def _all_reduce_exchange(group):
+    import torch.distributed as dist
+
+    def ex(buf, span):
+        dist.all_reduce(buf, op=dist.ReduceOp.SUM, group=group)
+    return ex
+
+
+def layerwise_chunked_fwd(q, k, gamma_q, gamma_k, pos_ids, *, rotary_dim: int, theta: float,
+                          eps: float, Hq_total: int, Hkv_total: int, exchange, chunks: int = 4):
+    """Forward of a rank holding a slice of the heads, in token chunks:
+    stats of chunk i -> ``exchange(buf, (t0, t1))`` of its [2, n] partial
+    sums (q row, k row) of tokens [t0, t1), on a side stream (the default
+    exchange is an all-reduce over the group) -> normalise and rotate chunk
+    i, with chunk i's exchange overlapping chunk i + 1's statistics
+    (``run_chunked``).
+    Returns ``(q_out, k_out, rstd_q, rstd_k)``, rstd fp32 [B*S]."""
+    B, S, Hq, Hkv, D = _lw_inputs(q, k, gamma_q, gamma_k, pos_ids)
+    T = B * S
+    dev = q.device
+    q_out, k_out = torch.empty_like(q), torch.empty_like(k)
+    rstd_q = torch.empty(T, dtype=torch.float32, device=dev)
+    rstd_k = torch.empty(T, dtype=torch.float32, device=dev)
+    if T == 0:
+        return q_out, k_out, rstd_q, rstd_k
+    pos = _chunk_positions(pos_ids, B, S, dev)
+    qf, kf, qof, kof = (_flat_tokens(t) for t in (q, k, q_out, k_out))
+    spans = token_chunks(T, chunks)
+    comp, comm = torch.cuda.current_stream(dev), _comm_stream(dev)
+    bufs = [torch.empty((2, t1 - t0), dtype=torch.float32, device=dev) for t0, t1 in spans]
+    done = [None] * len(spans)
+
+    def view(t, i):
+        t0, t1 = spans[i]
+        return t[t0:t1].unsqueeze(0)
+
+    def partial(i):
+        qk_layerwise_stats(view(qf, i), view(kf, i), sumsq_q=bufs[i][0], sumsq_k=bufs[i][1],
+                           stream=comp)
+
+    def exch(i):
+        ev = torch.cuda.Event()
+        ev.record(comp)
+        with torch.cuda.stream(comm):
+            comm.wait_event(ev)
+            exchange(bufs[i], spans[i])
+            done[i] = torch.cuda.Event()
+            done[i].record(comm)
+
+    def finish(i):
+        t0, t1 = spans[i]
+        comp.wait_event(done[i])
+        qk_layerwise_norm_rope_fwd(
+            view(qf, i), view(kf, i), gamma_q, gamma_k, pos[t0:t1].unsqueeze(0), bufs[i][0],
+            bufs[i][1], rotary_dim=rotary_dim, theta=theta, eps=eps, Hq_total=Hq_total,
+            Hkv_total=Hkv_total, q_out=view(qof, i), k_out=view(kof, i),
+            rstd_q=rstd_q[t0:t1], rstd_k=rstd_k[t0:t1], stream=comp)
+
+    run_chunked(len(spans), partial, exch, finish)
+    return q_out, k_out, rstd_q, rstd_k
+
+
+def layerwise_chunked_bwd(q, k, gamma_q, gamma_k, pos_ids, rstd_q, rstd_k, dq_out, dk_out, *,
+                          rotary_dim: int, theta: float, Hq_total: int, Hkv_total: int,
+                          exchange, chunks: int = 4, need_dgamma: bool = True):
+    """Backward of a rank holding a slice of the heads, in token chunks:
+    dots of chunk i -> ``exchange(buf, (t0, t1))`` -> dx and the chunk's dgamma share
+    (added into one dgamma per tensor, zeroed once), overlapped as in
+    ``layerwise_chunked_fwd``. Returns ``(dq, dk, dgamma_q, dgamma_k)``."""
+    B, S, Hq, Hkv, D = _lw_inputs(q, k, gamma_q, gamma_k, pos_ids)
+    T = B * S
+    dev = q.device
+    dq, dk = torch.empty_like(q), torch.empty_like(k)
+    dgq = dgk = None
+    if need_dgamma:
+        dgq = torch.zeros(Hq * D, dtype=torch.float32, device=dev)
+        dgk = torch.zeros(Hkv * D, dtype=torch.float32, device=dev)
+    if T == 0:
+        return dq, dk, dgq, dgk
+    pos = _chunk_positions(pos_ids, B, S, dev)
+    qf, kf, dqof, dkof, dqf, dkf = (_flat_tokens(t) for t in (q, k, dq_out, dk_out, dq, dk))
+    rq, rk = rstd_q.reshape(T), rstd_k.reshape(T)
+    spans = token_chunks(T, chunks)
+    comp, comm = torch.cuda.current_stream(dev), _comm_stream(dev)
+    bufs = [torch.empty((2, t1 - t0), dtype=torch.float32, device=dev) for t0, t1 in spans]
+    done = [None] * len(spans)
+
+    def view(t, i):
+        t0, t1 = spans[i]
+        return t[t0:t1].unsqueeze(0)
+
+    def partial(i):
+        t0, t1 = spans[i]
+        qk_layerwise_bwd_dots(view(qf, i), view(kf, i), gamma_q, gamma_k,
+                              pos[t0:t1].unsqueeze(0), rq[t0:t1], rk[t0:t1], view(dqof, i),
+                              view(dkof, i), rotary_dim=rotary_dim, theta=theta,
+                              dot_q=bufs[i][0], dot_k=bufs[i][1], stream=comp)
+
+    def exch(i):
+        ev = torch.cuda.Event()
+        ev.record(comp)
+        with torch.cuda.stream(comm):
+            comm.wait_event(ev)
+            exchange(bufs[i], spans[i])
+            done[i] = torch.cuda.Event()
+            done[i].record(comm)
+
+    def finish(i):
+        t0, t1 = spans[i]
+        comp.wait_event(done[i])
+        qk_layerwise_norm_rope_bwd(
+            view(qf, i), view(kf, i), gamma_q, gamma_k, pos[t0:t1].unsqueeze(0), rq[t0:t1],
+            rk[t0:t1], view(dqof, i), view(dkof, i), bufs[i][0], bufs[i][1],
+            rotary_dim=rotary_dim, theta=theta, Hq_total=Hq_total, Hkv_total=Hkv_total,
+            dq=view(dqf, i), dk=view(dkf, i), dgamma_q=dgq, dgamma_k=dgk,
+            need_dgamma=need_dgamma, accumulate=need_dgamma, stream=comp)
+
+    run_chunked(len(spans), partial, exch, finish)
+    return dq, dk, dgq, dgk
+
+
+DEFAULT_EXCHANGE_CHUNKS = 4
+
+
 class QKLayerwiseNormRoPE(torch.autograd.Function):
     """Autograd wrapper of the layerwise path: stats -> sum over ``group``
     -> normalise and rotate; backward: dots -> sum over ``group`` -> dx and
@@ -784,49 +964,57 @@ class QKLayerwiseNormRoPE(torch.autograd.Function):
 
     @staticmethod
     def forward(ctx, q, k, gamma_q, gamma_k, pos_ids, rotary_dim, theta, eps, Hq_total,
-                Hkv_total, group):
-        sq = sk = None
+                Hkv_total, group, chunks):
         if _sharded(q, k, Hq_total, Hkv_total, group):
-            sq, sk = qk_layerwise_stats(q, k)
-            all_reduce_stats([sq, sk], group)
-        qo, ko, rq, rk = qk_layerwise_norm_rope_fwd(
-            q, k, gamma_q, gamma_k, pos_ids, sq, sk, rotary_dim=rotary_dim, theta=theta, eps=eps,
-            Hq_total=Hq_total, Hkv_total=Hkv_total)
+            # stats -> sum over the ranks -> normalise, chunk by chunk, each
+            # chunk's exchange overlapping the next chunk's statistics
+            qo, ko, rq, rk = layerwise_chunked_fwd(
+                q, k, gamma_q, gamma_k, pos_ids, rotary_dim=rotary_dim, theta=theta, eps=eps,
+                Hq_total=Hq_total, Hkv_total=Hkv_total, exchange=_all_reduce_exchange(group),
+                chunks=chunks)
+        else:
+            qo, ko, rq, rk = qk_layerwise_norm_rope_fwd(
+                q, k, gamma_q, gamma_k, pos_ids, None, None, rotary_dim=rotary_dim, theta=theta,
+                eps=eps, Hq_total=Hq_total, Hkv_total=Hkv_total)
         ctx.save_for_backward(q, k, gamma_q, gamma_k, rq, rk)
-        ctx.cfg = (pos_ids, rotary_dim, theta, Hq_total, Hkv_total, group)
+        ctx.cfg = (pos_ids, rotary_dim, theta, Hq_total, Hkv_total, group, chunks)
         return qo, ko
 
     @staticmethod
     def backward(ctx, dq_out, dk_out):
         q, k, gq, gk, rq, rk = ctx.saved_tensors
-        pos_ids, R, theta, Hqt, Hkvt, group = ctx.cfg
+        pos_ids, R, theta, Hqt, Hkvt, group, chunks = ctx.cfg
         dq_out, dk_out = dq_out.contiguous(), dk_out.contiguous()
-        pq = pk = None
-        if _sharded(q, k, Hqt, Hkvt, group):
-            pq, pk = qk_layerwise_bwd_dots(q, k, gq, gk, pos_ids, rq, rk, dq_out, dk_out,
-                                           rotary_dim=R, theta=theta)
-            all_reduce_stats([pq, pk], group)
         need = ctx.needs_input_grad[2] or ctx.needs_input_grad[3]
-        dq, dk, dgq, dgk = qk_layerwise_norm_rope_bwd(
-            q, k, gq, gk, pos_ids, rq, rk, dq_out, dk_out, pq, pk, rotary_dim=R, theta=theta,
-            Hq_total=Hqt, Hkv_total=Hkvt, need_dgamma=need)
+        if _sharded(q, k, Hqt, Hkvt, group):
+            dq, dk, dgq, dgk = layerwise_chunked_bwd(
+                q, k, gq, gk, pos_ids, rq, rk, dq_out, dk_out, rotary_dim=R, theta=theta,
+                Hq_total=Hqt, Hkv_total=Hkvt, exchange=_all_reduce_exchange(group),
+                chunks=chunks, need_dgamma=need)
+        else:
+            dq, dk, dgq, dgk = qk_layerwise_norm_rope_bwd(
+                q, k, gq, gk, pos_ids, rq, rk, dq_out, dk_out, None, None, rotary_dim=R,
+                theta=theta, Hq_total=Hqt, Hkv_total=Hkvt, need_dgamma=need)
         if need:
             dgq, dgk = dgq.view_as(gq).to(gq.dtype), dgk.view_as(gk).to(gk.dtype)
-        return dq, dk, dgq, dgk, None, None, None, None, None, None, None
+        return dq, dk, dgq, dgk, None, None, None, None, None, None, None, None
 
 
 def qk_layerwise_norm_rope(q, k, gamma_q, gamma_k, pos_ids=None, *, rotary_dim: int,
                            theta: float, eps: float, Hq_total: Optional[int] = None,
-                           Hkv_total: Optional[int] = None, group=None):
+                           Hkv_total: Optional[int] = None, group=None,
+                           chunks: int = DEFAULT_EXCHANGE_CHUNKS):
     """Layerwise QK-RMSNorm + RoPE with autograd. q, k hold this rank's
     heads; gamma_q / gamma_k this rank's [Hq*D] / [Hkv*D] slices of the
     full-hidden weights. The head totals default to the local counts times
-    the group size (an even split)."""
+    the group size (an even split). A sharded call exchanges the per-token
+    sums in ``chunks`` token chunks, each chunk's all-reduce overlapping the
+    next chunk's statistics."""
     B, S, Hq, Hkv, D = _shape(q, k)
     Hqt, Hkvt = _totals(Hq, Hkv, Hq_total, Hkv_total, group)
     return QKLayerwiseNormRoPE.apply(q.contiguous(), k.contiguous(), gamma_q.contiguous(),
                                      gamma_k.contiguous(), pos_ids, rotary_dim, theta, eps, Hqt,
-                                     Hkvt, group)
+                                     Hkvt, group, int(chunks))
 
 
 _GEOM_KEYS = ("pipelined", "lpr", "TT", "NS", "stage_bytes", "off_k", "off_dq", "off_dk",

@@ -1548,12 +1548,14 @@ extern "C" qknr_status qk_layerwise_bwd_dots(
     return lw_run(LwKernel::kDots, a, dtype, stream);
 }
 
-extern "C" qknr_status qk_layerwise_norm_rope_bwd(
-    const void *q, const void *k, const void *gamma_q, const void *gamma_k,
-    const int32_t *pos_ids, const float *rstd_q, const float *rstd_k, const void *dq_out,
-    const void *dk_out, const float *dot_q, const float *dot_k, void *dq, void *dk,
-    float *dgamma_q, float *dgamma_k, int B, int S, int Hq, int Hkv, int Hq_total, int Hkv_total,
-    int D, int rotary_dim, float theta, qknr_dtype dtype, qknr_stream_t stream) {
+namespace {
+qknr_status lw_bwd_impl(const void *q, const void *k, const void *gamma_q, const void *gamma_k,
+                        const int32_t *pos_ids, const float *rstd_q, const float *rstd_k,
+                        const void *dq_out, const void *dk_out, const float *dot_q,
+                        const float *dot_k, void *dq, void *dk, float *dgamma_q, float *dgamma_k,
+                        int B, int S, int Hq, int Hkv, int Hq_total, int Hkv_total, int D,
+                        int rotary_dim, float theta, qknr_dtype dtype, qknr_stream_t stream,
+                        bool zero_dgamma) {
     qknr_status s = lw_check(B, S, Hq, Hkv, Hq_total, Hkv_total, D, rotary_dim, theta, 0.f, dtype);
     if (s != QKNR_OK) return s;
     // the block's dgamma partial sums live in shared memory
@@ -1587,10 +1589,10 @@ extern "C" qknr_status qk_layerwise_norm_rope_bwd(
     }
     cudaStream_t st = (cudaStream_t)stream;
     cudaError_t ce;
-    if (dgamma_q && Hq &&
+    if (zero_dgamma && dgamma_q && Hq &&
         (ce = cudaMemsetAsync(dgamma_q, 0, (size_t)Hq * D * 4, st)) != cudaSuccess)
         return cuda_fail(ce);
-    if (dgamma_k && Hkv &&
+    if (zero_dgamma && dgamma_k && Hkv &&
         (ce = cudaMemsetAsync(dgamma_k, 0, (size_t)Hkv * D * 4, st)) != cudaSuccess)
         return cuda_fail(ce);
     if (!work) return QKNR_OK;
@@ -1602,4 +1604,27 @@ extern "C" qknr_status qk_layerwise_norm_rope_bwd(
     a.inv_q = Hq_total ? 1.f / ((float)Hq_total * (float)D) : 0.f;
     a.inv_k = Hkv_total ? 1.f / ((float)Hkv_total * (float)D) : 0.f;
     return lw_run(LwKernel::kBwd, a, dtype, stream);
+}
+}  // namespace
+
+extern "C" qknr_status qk_layerwise_norm_rope_bwd(
+    const void *q, const void *k, const void *gamma_q, const void *gamma_k,
+    const int32_t *pos_ids, const float *rstd_q, const float *rstd_k, const void *dq_out,
+    const void *dk_out, const float *dot_q, const float *dot_k, void *dq, void *dk,
+    float *dgamma_q, float *dgamma_k, int B, int S, int Hq, int Hkv, int Hq_total, int Hkv_total,
+    int D, int rotary_dim, float theta, qknr_dtype dtype, qknr_stream_t stream) {
+    return lw_bwd_impl(q, k, gamma_q, gamma_k, pos_ids, rstd_q, rstd_k, dq_out, dk_out, dot_q,
+                       dot_k, dq, dk, dgamma_q, dgamma_k, B, S, Hq, Hkv, Hq_total, Hkv_total, D,
+                       rotary_dim, theta, dtype, stream, true);
+}
+
+extern "C" qknr_status qk_layerwise_norm_rope_bwd_acc(
+    const void *q, const void *k, const void *gamma_q, const void *gamma_k,
+    const int32_t *pos_ids, const float *rstd_q, const float *rstd_k, const void *dq_out,
+    const void *dk_out, const float *dot_q, const float *dot_k, void *dq, void *dk,
+    float *dgamma_q, float *dgamma_k, int B, int S, int Hq, int Hkv, int Hq_total, int Hkv_total,
+    int D, int rotary_dim, float theta, qknr_dtype dtype, qknr_stream_t stream) {
+    return lw_bwd_impl(q, k, gamma_q, gamma_k, pos_ids, rstd_q, rstd_k, dq_out, dk_out, dot_q,
+                       dot_k, dq, dk, dgamma_q, dgamma_k, B, S, Hq, Hkv, Hq_total, Hkv_total, D,
+                       rotary_dim, theta, dtype, stream, false);
 }

@@ -336,3 +336,62 @@ def test_layerwise_full_size_sampled(cuda):
         st.rstd(got[f"rstd_{name}"].reshape(T)[pick].double().numpy(), r)
         st.elem(f"d{name}", got[f"d{name}"].reshape(T, H, w.D)[pick].double().numpy(), dx)
         st.check()
+
+
+@pytest.mark.parametrize("name,over,chunks", [("llama3-8b-qknorm", dict(B=2, S=97), 4),
+                                              ("partial-rope-64k", dict(S=1000), 3),
+                                              ("bfd-packed", dict(), 4),
+                                              ("tiny", dict(B=3, S=37, Hq=6, Hkv=2, D=24,
+                                                            rotary_dim=16), 7)])
+def test_layerwise_chunked_schedule_vs_oracle(cuda, name, over, chunks):
+    """The binding's chunked exchange schedule (stats of a chunk, its sums
+    exchanged on a side stream, the chunk normalised once they are in, the
+    next chunk's stats overlapping the exchange), for each of two emulated
+    ranks on one GPU: the exchange adds the other slice's partial sums of the
+    chunk's tokens, as an all-reduce over two ranks would. The concatenated
+    outputs and the per-slice dgamma must match the oracle on the full
+    tensor; the outputs equal the unchunked two-phase calls bit for bit."""
+    inp, gq, gk = lw_inputs(name, **over)
+    w = inp.w
+    hq, hk, D = w.Hq // 2, w.Hkv // 2, w.D
+    cfg = dict(rotary_dim=w.rotary_dim, theta=w.theta)
+    pos = None if inp.pos is None else inp.pos.to(cuda)
+    q, k = inp.q.to(cuda), inp.k.to(cuda)
+    dqo, dko = inp.dq_out.to(cuda), inp.dk_out.to(cuda)
+    gqd, gkd = gq.to(cuda), gk.to(cuda)
+    sl = []
+    for r in range(2):
+        sq_, sk_ = slice(r * hq, (r + 1) * hq), slice(r * hk, (r + 1) * hk)
+        sl.append(dict(q=q[:, :, sq_].contiguous(), k=k[:, :, sk_].contiguous(),
+                       dqo=dqo[:, :, sq_].contiguous(), dko=dko[:, :, sk_].contiguous(),
+                       gq=gqd[r * hq * D:(r + 1) * hq * D], gk=gkd[r * hk * D:(r + 1) * hk * D]))
+    stats = [qknr.qk_layerwise_stats(s["q"], s["k"]) for s in sl]
+
+    def exchange_with(other):
+        def ex(buf, span):
+            t0, t1 = span
+            buf[0] += other[0][t0:t1]
+            buf[1] += other[1][t0:t1]
+        return ex
+
+    fw = [qknr.layerwise_chunked_fwd(s["q"], s["k"], s["gq"], s["gk"], pos, eps=w.eps,
+                                     Hq_total=w.Hq, Hkv_total=w.Hkv,
+                                     exchange=exchange_with(stats[1 - r]), chunks=chunks, **cfg)
+          for r, s in enumerate(sl)]
+    dots = [qknr.qk_layerwise_bwd_dots(s["q"], s["k"], s["gq"], s["gk"], pos, f[2], f[3],
+                                       s["dqo"], s["dko"], **cfg) for s, f in zip(sl, fw)]
+    bw = [qknr.layerwise_chunked_bwd(s["q"], s["k"], s["gq"], s["gk"], pos, f[2], f[3],
+                                     s["dqo"], s["dko"], Hq_total=w.Hq, Hkv_total=w.Hkv,
+                                     exchange=exchange_with(dots[1 - r]), chunks=chunks, **cfg)
+          for r, (s, f) in enumerate(zip(sl, fw))]
+    torch.cuda.synchronize()
+    cat = lambda xs, d: torch.cat(xs, dim=d).cpu()
+    got = {"q_out": cat([f[0] for f in fw], 2), "k_out": cat([f[1] for f in fw], 2),
+           "rstd_q": fw[0][2].cpu(), "rstd_k": fw[0][3].cpu(),
+           "dq": cat([b[0] for b in bw], 2), "dk": cat([b[1] for b in bw], 2),
+           "dgamma_q": cat([b[2] for b in bw], 0), "dgamma_k": cat([b[3] for b in bw], 0)}
+    assert torch.equal(fw[0][2], fw[1][2]) and torch.equal(fw[0][3], fw[1][3])
+    check_vs_oracle(inp, gq, gk, got)
+    two = run_ranks(inp, gq, gk, cuda, world=2)
+    for n in ("q_out", "k_out", "dq", "dk"):
+        assert torch.equal(got[n], two[n]), n
