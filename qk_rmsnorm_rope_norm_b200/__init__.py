@@ -33,7 +33,7 @@ __all__ = ["qk_norm_rope_fwd", "qk_norm_rope_bwd", "qknr_strerror", "QKNormRoPE"
            "qk_layerwise_norm_rope_bwd", "QKLayerwiseNormRoPE", "qk_layerwise_norm_rope",
            "all_reduce_stats", "layerwise_geometry", "launch_plan", "kernel_name",
            "wait_selftest", "token_chunks", "run_chunked", "layerwise_chunked_fwd",
-           "layerwise_chunked_bwd"]
+           "layerwise_chunked_bwd", "MIN_CHUNK_TOKENS"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libqknr.so")
@@ -840,116 +840,151 @@ def _all_reduce_exchange(group):
     return ex
 
 
+MIN_CHUNK_TOKENS = 4096  # a chunk's kernels should outlast their launch and event overhead
+
+
+class _Chunks:
+    """Token chunks of one sharded layerwise call and the direct library
+    arguments of each chunk (the tensors are checked once, by the caller)."""
+
+    def __init__(self, q, k, chunks, pos_ids, min_chunk):
+        B, S, Hq, Hkv, D = _shape(q, k)
+        self.T = T = B * S
+        n = max(1, min(int(chunks), T // max(1, int(min_chunk)))) if T else 1
+        self.spans = token_chunks(T, n)
+        self.dev = q.device
+        self.Hq, self.Hkv, self.D = Hq, Hkv, D
+        self.esz = q.element_size()
+        self.dt = _DTYPES[q.dtype]
+        self.pos = _chunk_positions(pos_ids, B, S, q.device)
+        self.comp, self.comm = torch.cuda.current_stream(q.device), _comm_stream(q.device)
+        self.st = _stream(self.comp)
+        self.bufs = [torch.empty((2, t1 - t0), dtype=torch.float32, device=q.device)
+                     for t0, t1 in self.spans]
+        self.done = [None] * len(self.spans)
+
+    def rows(self, t: torch.Tensor, i: int, H: int):
+        """Pointer to token spans[i][0] of a [B, S, H, D] tensor (None without heads)."""
+        if t is None or H == 0:
+            return None
+        return ctypes.c_void_p(t.data_ptr() + self.spans[i][0] * H * self.D * self.esz)
+
+    def vec(self, t: torch.Tensor, i: int):
+        """Pointer to token spans[i][0] of a per-token fp32 or int32 vector."""
+        return None if t is None else ctypes.c_void_p(t.data_ptr() + 4 * self.spans[i][0])
+
+    def sums(self, i: int):
+        b = self.bufs[i]
+        n = b.shape[1]
+        return ctypes.c_void_p(b.data_ptr()), ctypes.c_void_p(b.data_ptr() + 4 * n)
+
+    def n(self, i: int) -> int:
+        return self.spans[i][1] - self.spans[i][0]
+
+    def exchange(self, i: int, fn):
+        ev = torch.cuda.Event()
+        ev.record(self.comp)
+        with torch.cuda.stream(self.comm):
+            self.comm.wait_event(ev)
+            fn(self.bufs[i], self.spans[i])
+            self.done[i] = torch.cuda.Event()
+            self.done[i].record(self.comm)
+
+    def wait(self, i: int):
+        self.comp.wait_event(self.done[i])
+
+
+def _ok(st: int, where: str):
+    if st != QKNR_OK:
+        raise QKNRError(st, where)
+
+
 def layerwise_chunked_fwd(q, k, gamma_q, gamma_k, pos_ids, *, rotary_dim: int, theta: float,
-                          eps: float, Hq_total: int, Hkv_total: int, exchange, chunks: int = 4):
+                          eps: float, Hq_total: int, Hkv_total: int, exchange, chunks: int = 4,
+                          min_chunk: int = MIN_CHUNK_TOKENS):
     """Forward of a rank holding a slice of the heads, in token chunks:
     stats of chunk i -> ``exchange(buf, (t0, t1))`` of its [2, n] partial
     sums (q row, k row) of tokens [t0, t1), on a side stream (the default
     exchange is an all-reduce over the group) -> normalise and rotate chunk
     i, with chunk i's exchange overlapping chunk i + 1's statistics
-    (``run_chunked``).
-    Returns ``(q_out, k_out, rstd_q, rstd_k)``, rstd fp32 [B*S]."""
+    (``run_chunked``). The tokens are cut into ``chunks`` runs of at least
+    ``min_chunk`` tokens (fewer runs for short calls). Returns ``(q_out, k_out,
+    rstd_q, rstd_k)``, rstd fp32 [B*S]."""
+    lib = load_library()
     B, S, Hq, Hkv, D = _lw_inputs(q, k, gamma_q, gamma_k, pos_ids)
     T = B * S
-    dev = q.device
     q_out, k_out = torch.empty_like(q), torch.empty_like(k)
-    rstd_q = torch.empty(T, dtype=torch.float32, device=dev)
-    rstd_k = torch.empty(T, dtype=torch.float32, device=dev)
+    rstd_q = torch.empty(T, dtype=torch.float32, device=q.device)
+    rstd_k = torch.empty(T, dtype=torch.float32, device=q.device)
     if T == 0:
         return q_out, k_out, rstd_q, rstd_k
-    pos = _chunk_positions(pos_ids, B, S, dev)
-    qf, kf, qof, kof = (_flat_tokens(t) for t in (q, k, q_out, k_out))
-    spans = token_chunks(T, chunks)
-    comp, comm = torch.cuda.current_stream(dev), _comm_stream(dev)
-    bufs = [torch.empty((2, t1 - t0), dtype=torch.float32, device=dev) for t0, t1 in spans]
-    done = [None] * len(spans)
-
-    def view(t, i):
-        t0, t1 = spans[i]
-        return t[t0:t1].unsqueeze(0)
+    c = _Chunks(q, k, chunks, pos_ids, min_chunk)
+    gq, gk = _ptr(gamma_q), _ptr(gamma_k)
 
     def partial(i):
-        qk_layerwise_stats(view(qf, i), view(kf, i), sumsq_q=bufs[i][0], sumsq_k=bufs[i][1],
-                           stream=comp)
-
-    def exch(i):
-        ev = torch.cuda.Event()
-        ev.record(comp)
-        with torch.cuda.stream(comm):
-            comm.wait_event(ev)
-            exchange(bufs[i], spans[i])
-            done[i] = torch.cuda.Event()
-            done[i].record(comm)
+        sq, sk = c.sums(i)
+        _ok(lib.qk_layerwise_stats(c.rows(q, i, Hq), c.rows(k, i, Hkv), sq, sk, 1, c.n(i), Hq,
+                                   Hkv, D, c.dt, c.st), "qk_layerwise_stats")
 
     def finish(i):
-        t0, t1 = spans[i]
-        comp.wait_event(done[i])
-        qk_layerwise_norm_rope_fwd(
-            view(qf, i), view(kf, i), gamma_q, gamma_k, pos[t0:t1].unsqueeze(0), bufs[i][0],
-            bufs[i][1], rotary_dim=rotary_dim, theta=theta, eps=eps, Hq_total=Hq_total,
-            Hkv_total=Hkv_total, q_out=view(qof, i), k_out=view(kof, i),
-            rstd_q=rstd_q[t0:t1], rstd_k=rstd_k[t0:t1], stream=comp)
+        c.wait(i)
+        sq, sk = c.sums(i)
+        _ok(lib.qk_layerwise_norm_rope_fwd(
+            c.rows(q, i, Hq), c.rows(k, i, Hkv), gq, gk, c.vec(c.pos, i), sq, sk,
+            c.rows(q_out, i, Hq), c.rows(k_out, i, Hkv), c.vec(rstd_q, i), c.vec(rstd_k, i), 1,
+            c.n(i), Hq, Hkv, int(Hq_total), int(Hkv_total), D, int(rotary_dim), float(theta),
+            float(eps), c.dt, c.st), "qk_layerwise_norm_rope_fwd")
 
-    run_chunked(len(spans), partial, exch, finish)
+    run_chunked(len(c.spans), partial, lambda i: c.exchange(i, exchange), finish)
     return q_out, k_out, rstd_q, rstd_k
 
 
 def layerwise_chunked_bwd(q, k, gamma_q, gamma_k, pos_ids, rstd_q, rstd_k, dq_out, dk_out, *,
                           rotary_dim: int, theta: float, Hq_total: int, Hkv_total: int,
-                          exchange, chunks: int = 4, need_dgamma: bool = True):
+                          exchange, chunks: int = 4, need_dgamma: bool = True,
+                          min_chunk: int = MIN_CHUNK_TOKENS):
     """Backward of a rank holding a slice of the heads, in token chunks:
-    dots of chunk i -> ``exchange(buf, (t0, t1))`` -> dx and the chunk's dgamma share
-    (added into one dgamma per tensor, zeroed once), overlapped as in
-    ``layerwise_chunked_fwd``. Returns ``(dq, dk, dgamma_q, dgamma_k)``."""
+    dots of chunk i -> ``exchange(buf, (t0, t1))`` -> dx and the chunk's
+    dgamma share (added into one dgamma per tensor, zeroed once), overlapped
+    as in ``layerwise_chunked_fwd``. Returns ``(dq, dk, dgamma_q,
+    dgamma_k)``."""
+    lib = load_library()
     B, S, Hq, Hkv, D = _lw_inputs(q, k, gamma_q, gamma_k, pos_ids)
     T = B * S
-    dev = q.device
+    for n, t, ref in (("dq_out", dq_out, q), ("dk_out", dk_out, k)):
+        _need_cuda(n, t)
+        if t.shape != ref.shape or t.dtype != ref.dtype:
+            raise ValueError(f"{n} must match its input in shape and dtype")
+    rq = _token_vec("rstd_q", rstd_q.reshape(-1) if rstd_q is not None else None, T, q.device)
+    rk = _token_vec("rstd_k", rstd_k.reshape(-1) if rstd_k is not None else None, T, q.device)
     dq, dk = torch.empty_like(q), torch.empty_like(k)
     dgq = dgk = None
     if need_dgamma:
-        dgq = torch.zeros(Hq * D, dtype=torch.float32, device=dev)
-        dgk = torch.zeros(Hkv * D, dtype=torch.float32, device=dev)
+        dgq = torch.zeros(Hq * D, dtype=torch.float32, device=q.device)
+        dgk = torch.zeros(Hkv * D, dtype=torch.float32, device=q.device)
     if T == 0:
         return dq, dk, dgq, dgk
-    pos = _chunk_positions(pos_ids, B, S, dev)
-    qf, kf, dqof, dkof, dqf, dkf = (_flat_tokens(t) for t in (q, k, dq_out, dk_out, dq, dk))
-    rq, rk = rstd_q.reshape(T), rstd_k.reshape(T)
-    spans = token_chunks(T, chunks)
-    comp, comm = torch.cuda.current_stream(dev), _comm_stream(dev)
-    bufs = [torch.empty((2, t1 - t0), dtype=torch.float32, device=dev) for t0, t1 in spans]
-    done = [None] * len(spans)
-
-    def view(t, i):
-        t0, t1 = spans[i]
-        return t[t0:t1].unsqueeze(0)
+    c = _Chunks(q, k, chunks, pos_ids, min_chunk)
+    gq, gk = _ptr(gamma_q), _ptr(gamma_k)
+    fn = lib.qk_layerwise_norm_rope_bwd_acc if need_dgamma else lib.qk_layerwise_norm_rope_bwd
 
     def partial(i):
-        t0, t1 = spans[i]
-        qk_layerwise_bwd_dots(view(qf, i), view(kf, i), gamma_q, gamma_k,
-                              pos[t0:t1].unsqueeze(0), rq[t0:t1], rk[t0:t1], view(dqof, i),
-                              view(dkof, i), rotary_dim=rotary_dim, theta=theta,
-                              dot_q=bufs[i][0], dot_k=bufs[i][1], stream=comp)
-
-    def exch(i):
-        ev = torch.cuda.Event()
-        ev.record(comp)
-        with torch.cuda.stream(comm):
-            comm.wait_event(ev)
-            exchange(bufs[i], spans[i])
-            done[i] = torch.cuda.Event()
-            done[i].record(comm)
+        pq, pk = c.sums(i)
+        _ok(lib.qk_layerwise_bwd_dots(
+            c.rows(q, i, Hq), c.rows(k, i, Hkv), gq, gk, c.vec(c.pos, i), c.vec(rq, i),
+            c.vec(rk, i), c.rows(dq_out, i, Hq), c.rows(dk_out, i, Hkv), pq, pk, 1, c.n(i), Hq,
+            Hkv, D, int(rotary_dim), float(theta), c.dt, c.st), "qk_layerwise_bwd_dots")
 
     def finish(i):
-        t0, t1 = spans[i]
-        comp.wait_event(done[i])
-        qk_layerwise_norm_rope_bwd(
-            view(qf, i), view(kf, i), gamma_q, gamma_k, pos[t0:t1].unsqueeze(0), rq[t0:t1],
-            rk[t0:t1], view(dqof, i), view(dkof, i), bufs[i][0], bufs[i][1],
-            rotary_dim=rotary_dim, theta=theta, Hq_total=Hq_total, Hkv_total=Hkv_total,
-            dq=view(dqf, i), dk=view(dkf, i), dgamma_q=dgq, dgamma_k=dgk,
-            need_dgamma=need_dgamma, accumulate=need_dgamma, stream=comp)
+        c.wait(i)
+        pq, pk = c.sums(i)
+        _ok(fn(c.rows(q, i, Hq), c.rows(k, i, Hkv), gq, gk, c.vec(c.pos, i), c.vec(rq, i),
+               c.vec(rk, i), c.rows(dq_out, i, Hq), c.rows(dk_out, i, Hkv), pq, pk,
+               c.rows(dq, i, Hq), c.rows(dk, i, Hkv), _ptr(dgq), _ptr(dgk), 1, c.n(i), Hq, Hkv,
+               int(Hq_total), int(Hkv_total), D, int(rotary_dim), float(theta), c.dt, c.st),
+            "qk_layerwise_norm_rope_bwd")
 
-    run_chunked(len(spans), partial, exch, finish)
+    run_chunked(len(c.spans), partial, lambda i: c.exchange(i, exchange), finish)
     return dq, dk, dgq, dgk
 
 

@@ -563,7 +563,7 @@ template <int V> struct LwCsWork {
     }
 };
 
-template <typename T, int LPR, int MODE>
+template <typename T, int LPR, int MODE, int NBM>
 __global__ void __launch_bounds__((kLwCWMax + 1) * 32, 1)
     qknr_lw_pipe_kernel(const LwArgs a, const LwGeom g) {
     using IO = Io<T>;
@@ -580,6 +580,7 @@ __global__ void __launch_bounds__((kLwCWMax + 1) * 32, 1)
         return;
     }
     __shared__ int s_abort;  // a consumer warp gave up a wait: skip the dgamma phase
+    __shared__ __align__(8) uint64_t s_tgbar[kLwCWMax];  // one per token group: its warps' partials are in
     unsigned char *ring = smem + 128;
     float2 *parts_all = reinterpret_cast<float2 *>(smem + g.off_parts);
     if (threadIdx.x == 0) s_abort = 0;
@@ -601,8 +602,8 @@ __global__ void __launch_bounds__((kLwCWMax + 1) * 32, 1)
         for (int s = 0; s < g.NS; ++s) {
             lw_bar_init(bar0 + 8 * s, 32);                   // the producer warp's lanes
             lw_bar_init(bar0 + 8 * (g.NS + s), ncw);       // one per consumer warp
-            lw_bar_init(bar0 + 8 * (2 * g.NS + s), ncw);   // one per consumer warp
         }
+        for (int t = 0; t < g.NTG; ++t) lw_bar_init(lw_smem_u32(&s_tgbar[t]), g.G);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
@@ -680,24 +681,36 @@ __global__ void __launch_bounds__((kLwCWMax + 1) * 32, 1)
     }
 
     // -------------------------------------------------------------- consumers
+    // Token group tg (warps tg G .. tg G + G - 1) takes tokens tg, tg + NTG,
+    // ... of every stage, UA at a time; warp wb of the group owns head blocks
+    // wb, wb + G (at most NBM), so each lane keeps the same rows, elements
+    // and dgamma sums for the whole kernel. Per round a warp un-rotates dy,
+    // forms hh = g gamma and xh = x r, adds g xh to its dgamma sums and keeps
+    // hh, xh in registers; when the per-token sums come from this pass, the
+    // group's G warps post their partials and meet on the group's mbarrier,
+    // every warp adds the G partials in warp order, and then finishes dx
+    // from the registers (no second pass over the rows).
     const int tg = warp / g.G, wb = warp % g.G;
     const Lane<LPR, V> L(lane, a.D, a.R);
     const int offA = L.eA * E, offB = L.eB * E;
     const int hp = half >> 1;  // rotary pairs per token
     const bool local = MODE == kLwBwd && a.sq == nullptr && a.sk == nullptr;
     const bool need_parts = MODE == kLwDots || local;
-    constexpr int kUA = 2;  // tokens per partial-sum round
-    float2 acc[kLwNBMax][V];  // dgamma sums: pairs of the A vector, then of the B vector
+    constexpr int UA = NBM == 1 ? 2 : 1;  // tokens per round
+    const uint32_t tgbar = lw_smem_u32(&s_tgbar[tg]);
+    uint32_t tg_phase = 0;
+    float2 acc[NBM][V];  // dgamma sums: pairs of the A vector, then of the B vector
 #pragma unroll
-    for (int nb = 0; nb < kLwNBMax; ++nb)
+    for (int nb = 0; nb < NBM; ++nb)
 #pragma unroll
         for (int k = 0; k < V; ++k) acc[nb][k] = make_float2(0.f, 0.f);
+    bool aborted = false;
 
-    for (int i = 0; i < ntiles; ++i) {
+    for (int i = 0; i < ntiles && !aborted; ++i) {
         const int s = i % g.NS;
         const uint32_t ph = (uint32_t)(i / g.NS) & 1u;
         if (!lw_wait(bar0 + 8 * s, ph)) {
-            s_abort = 1;
+            aborted = true;
             break;
         }
         const int64_t t0 = t_lo + (int64_t)i * g.TT;
@@ -709,154 +722,149 @@ __global__ void __launch_bounds__((kLwCWMax + 1) * 32, 1)
         const float4 *sc = reinterpret_cast<const float4 *>(st + g.off_sc);
         float2 *parts = parts_all + (size_t)s * g.TT * g.G;
 
-        if (need_parts) {
-            // this warp's share of each token's (g gamma).(x r), kUA tokens
-            // per round so that their warp reductions overlap
-            for (int j0 = tg; j0 < na; j0 += kUA * g.NTG) {
-                float vq[kUA], vk[kUA];
+        for (int j0 = tg; j0 < na; j0 += UA * g.NTG) {
+            float2 hh[UA][NBM][V], xh[UA][NBM][V];  // pairs of A, then of B
+            float vq[UA], vk[UA];
 #pragma unroll
-                for (int u = 0; u < kUA; ++u) {
-                    const int j = j0 + u * g.NTG;
-                    vq[u] = vk[u] = 0.f;
-                    if (j >= na) continue;
-                    float4 c[V / 2];
-                    lane_cs4<V>(c, cs_st + j * hp, L, hp / (V / 2));
-                    const float4 sv = sc[j];
-                    const float r2q = sv.x, r2k = sv.y;
+            for (int u = 0; u < UA; ++u) {
+                const int j = j0 + u * g.NTG;
+                vq[u] = vk[u] = 0.f;
+                const bool tok_ok = j < na;
+                float4 c[V / 2];
+                lane_cs4<V>(c, cs_st + (tok_ok ? j : j0) * hp, L, hp / (V / 2));
+                const float4 sv = sc[tok_ok ? j : j0];
 #pragma unroll
-                    for (int nb = 0; nb < kLwNBMax; ++nb) {
-                        const int b = wb + nb * g.G;
-                        if (b >= g.HB) break;
-                        const int h = b * SLOTS + L.slot;
-                        if (!(L.on && h < H)) continue;
-                        const bool isq = h < a.Hq;
-                        const unsigned char *row = stage_row(xq, xk, j, h, a.Hq, a.Hkv, rowb);
-                        const unsigned char *drow = stage_row(dq0, dk0, j, h, a.Hq, a.Hkv, rowb);
-                        const unsigned char *grow = s_gamma + h * rowb;
-                        const Vec16 xa = ld16(row + offA), xb = ld16(row + offB);
-                        const Vec16 da = ld16(drow + offA), db = ld16(drow + offB);
-                        const Vec16 ga = ld16(grow + offA), gb = ld16(grow + offB);
-                        float2 p2 = make_float2(0.f, 0.f);
+                for (int nb = 0; nb < NBM; ++nb) {
+                    const int b = wb + nb * g.G;
+                    const int h = b * SLOTS + L.slot;
+                    const bool on = tok_ok && b < g.HB && L.on && h < H;
+                    const bool isq = h < a.Hq;
+                    const int hs = on ? h : 0;
+                    const unsigned char *row = stage_row(xq, xk, on ? j : 0, hs, a.Hq, a.Hkv, rowb);
+                    const unsigned char *drow = stage_row(dq0, dk0, on ? j : 0, hs, a.Hq, a.Hkv, rowb);
+                    const unsigned char *grow = s_gamma + hs * rowb;
+                    const Vec16 xa = ld16(row + offA), xb = ld16(row + offB);
+                    const Vec16 da = ld16(drow + offA), db = ld16(drow + offB);
+                    const Vec16 ga = ld16(grow + offA), gb = ld16(grow + offB);
+                    const float r = on ? (isq ? sv.x : sv.y) : 0.f;  // off rows add nothing
+                    const float2 r2 = make_float2(r, r);
+                    float2 p2 = make_float2(0.f, 0.f);
 #pragma unroll
-                        for (int k2 = 0; k2 < V / 2; ++k2) {
-                            const float2 c2 = make_float2(c[k2].x, c[k2].y);
-                            const float2 s2 = make_float2(c[k2].z, c[k2].w);
-                            const float2 ea = IO::get2(da, k2), eb = IO::get2(db, k2);
-                            const float2 gA = __ffma2_rn(ea, c2, __fmul2_rn(eb, s2));
-                            const float2 gB = __ffma2_rn(eb, c2, __fmul2_rn(ea, neg2f(s2)));
-                            p2 = __ffma2_rn(__fmul2_rn(gA, IO::get2(ga, k2)), IO::get2(xa, k2), p2);
-                            p2 = __ffma2_rn(__fmul2_rn(gB, IO::get2(gb, k2)), IO::get2(xb, k2), p2);
+                    for (int k2 = 0; k2 < V / 2; ++k2) {
+                        const float2 c2 = make_float2(c[k2].x, c[k2].y);
+                        const float2 s2 = make_float2(c[k2].z, c[k2].w);
+                        const float2 ea = IO::get2(da, k2), eb = IO::get2(db, k2);
+                        const float2 gA = __ffma2_rn(ea, c2, __fmul2_rn(eb, s2));
+                        const float2 gB = __ffma2_rn(eb, c2, __fmul2_rn(ea, neg2f(s2)));
+                        const float2 hA = __fmul2_rn(gA, IO::get2(ga, k2));
+                        const float2 hB = __fmul2_rn(gB, IO::get2(gb, k2));
+                        const float2 xA = __fmul2_rn(IO::get2(xa, k2), r2);
+                        const float2 xB = __fmul2_rn(IO::get2(xb, k2), r2);
+                        p2 = __ffma2_rn(hA, xA, p2);
+                        p2 = __ffma2_rn(hB, xB, p2);
+                        hh[u][nb][k2] = hA;
+                        hh[u][nb][V / 2 + k2] = hB;
+                        xh[u][nb][k2] = xA;
+                        xh[u][nb][V / 2 + k2] = xB;
+                        if (MODE == kLwBwd) {
+                            acc[nb][k2] = __ffma2_rn(gA, xA, acc[nb][k2]);
+                            acc[nb][V / 2 + k2] = __ffma2_rn(gB, xB, acc[nb][V / 2 + k2]);
                         }
-                        const float p = (p2.x + p2.y) * (isq ? r2q : r2k);
-                        vq[u] += isq ? p : 0.f;
-                        vk[u] += isq ? 0.f : p;
                     }
+                    const float pr = p2.x + p2.y;
+                    vq[u] += isq ? pr : 0.f;
+                    vk[u] += isq ? 0.f : pr;
                 }
+            }
+            float2 tot[UA];
+            if (need_parts) {
 #pragma unroll
                 for (int o = 16; o; o >>= 1)
 #pragma unroll
-                    for (int u = 0; u < kUA; ++u) {
+                    for (int u = 0; u < UA; ++u) {
                         vq[u] += __shfl_xor_sync(0xffffffffu, vq[u], o);
                         vk[u] += __shfl_xor_sync(0xffffffffu, vk[u], o);
                     }
                 if (lane == 0) {
 #pragma unroll
-                    for (int u = 0; u < kUA; ++u) {
+                    for (int u = 0; u < UA; ++u) {
                         const int j = j0 + u * g.NTG;
                         if (j < na) parts[j * g.G + wb] = make_float2(vq[u], vk[u]);
                     }
                 }
-            }
-            __syncwarp();
-            const uint32_t pbar = bar0 + 8 * (2 * g.NS + s);
-            if (lane == 0) lw_bar_arrive(pbar);
-            if (!lw_wait(pbar, ph)) {
-                s_abort = 1;
-                break;
-            }
-            if (MODE == kLwDots && warp == 0) {
-                // lane j: token j's total over the G warps, in warp order
-                for (int j = lane; j < na; j += 32) {
-                    const float2 tot = token_total(parts, j, g.G);
-                    if (a.Hq) a.wq[t0 + j] = tot.x;
-                    if (a.Hkv) a.wk[t0 + j] = tot.y;
+                // the group's G warps meet: every partial of these tokens is in
+                __syncwarp();
+                if (lane == 0) lw_bar_arrive(tgbar);
+                if (!lw_wait(tgbar, tg_phase)) {
+                    aborted = true;
+                    break;
                 }
-            }
-        }
-
-        if (MODE == kLwBwd) {
-            // per-token totals: lane j holds token j's (j < 32; TT <= 32)
-            float2 my_tot = make_float2(0.f, 0.f);
-            if (lane < na) {
-                if (local) {
-                    my_tot = token_total(parts, lane, g.G);
-                } else {
-                    const float4 v = sc[lane];
-                    my_tot = make_float2(v.z, v.w);
-                }
-            }
-            // two tokens per round, their work interleaved
-            for (int j0 = tg; j0 < na; j0 += 2 * g.NTG) {
+                tg_phase ^= 1u;
 #pragma unroll
-                for (int u = 0; u < 2; ++u) {
+                for (int u = 0; u < UA; ++u) {
                     const int j = j0 + u * g.NTG;
-                    const int jj = j < na ? j : j0;
-                    const float2 tot = make_float2(__shfl_sync(0xffffffffu, my_tot.x, jj),
-                                                   __shfl_sync(0xffffffffu, my_tot.y, jj));
+                    tot[u] = j < na ? token_total(parts, j, g.G) : make_float2(0.f, 0.f);
+                }
+                if (MODE == kLwDots) {
+                    if (wb == 0 && lane == 0) {
+#pragma unroll
+                        for (int u = 0; u < UA; ++u) {
+                            const int j = j0 + u * g.NTG;
+                            if (j >= na) continue;
+                            if (a.Hq) a.wq[t0 + j] = tot[u].x;
+                            if (a.Hkv) a.wk[t0 + j] = tot[u].y;
+                        }
+                    }
+                    continue;
+                }
+            } else {
+#pragma unroll
+                for (int u = 0; u < UA; ++u) {
+                    const int j = j0 + u * g.NTG;
+                    const float4 sv = sc[j < na ? j : j0];
+                    tot[u] = make_float2(sv.z, sv.w);
+                }
+            }
+            if (MODE == kLwBwd) {
+                // dx = r (hh - xh P / (H_total D)) from the registers
+#pragma unroll
+                for (int u = 0; u < UA; ++u) {
+                    const int j = j0 + u * g.NTG;
                     if (j >= na) continue;
                     const int64_t t = t0 + j;
                     const float4 sv = sc[j];
-                    const float rq = sv.x, rk = sv.y;
-                    // dx = r (hh - (x r) P / (H_total D)); nq, nk: the factors of x
-                    const float nq = -rq * tot.x * a.inv_q, nk = -rk * tot.y * a.inv_k;
-                    float4 c[V / 2];
-                    lane_cs4<V>(c, cs_st + j * hp, L, hp / (V / 2));
+                    const float nq = -tot[u].x * a.inv_q, nk = -tot[u].y * a.inv_k;
 #pragma unroll
-                    for (int nb = 0; nb < kLwNBMax; ++nb) {
+                    for (int nb = 0; nb < NBM; ++nb) {
                         const int b = wb + nb * g.G;
-                        if (b >= g.HB) break;
                         const int h = b * SLOTS + L.slot;
-                        if (!(L.on && h < H)) continue;
+                        if (!(b < g.HB && L.on && h < H)) continue;
                         const bool isq = h < a.Hq;
-                        const int hh = isq ? h : h - a.Hq;
-                        const unsigned char *row = stage_row(xq, xk, j, h, a.Hq, a.Hkv, rowb);
-                        const unsigned char *drow = stage_row(dq0, dk0, j, h, a.Hq, a.Hkv, rowb);
-                        const unsigned char *grow = s_gamma + h * rowb;
-                        char *out = (char *)(isq ? a.qo : a.ko) +
-                                    ((isq ? t * a.Hq : t * a.Hkv) + hh) * rowb;
-                        const Vec16 xa = ld16(row + offA), xb = ld16(row + offB);
-                        const Vec16 da = ld16(drow + offA), db = ld16(drow + offB);
-                        const Vec16 ga = ld16(grow + offA), gb = ld16(grow + offB);
-                        const float r = isq ? rq : rk, nd = isq ? nq : nk;
+                        const int hh_ = isq ? h : h - a.Hq;
+                        const float r = isq ? sv.x : sv.y, nd = isq ? nq : nk;
                         const float2 r2 = make_float2(r, r), nd2 = make_float2(nd, nd);
                         Vec16 oa, ob;
 #pragma unroll
                         for (int k2 = 0; k2 < V / 2; ++k2) {
-                            const float2 c2 = make_float2(c[k2].x, c[k2].y);
-                            const float2 s2 = make_float2(c[k2].z, c[k2].w);
-                            const float2 ea = IO::get2(da, k2), eb = IO::get2(db, k2);
-                            const float2 va = IO::get2(xa, k2), vb = IO::get2(xb, k2);
-                            const float2 gA = __ffma2_rn(ea, c2, __fmul2_rn(eb, s2));
-                            const float2 gB = __ffma2_rn(eb, c2, __fmul2_rn(ea, neg2f(s2)));
-                            const float2 hA = __fmul2_rn(gA, IO::get2(ga, k2));
-                            const float2 hB = __fmul2_rn(gB, IO::get2(gb, k2));
-                            const float2 oA = __fmul2_rn(r2, __ffma2_rn(va, nd2, hA));
-                            const float2 oB = __fmul2_rn(r2, __ffma2_rn(vb, nd2, hB));
-                            acc[nb][k2] = __ffma2_rn(__fmul2_rn(gA, va), r2, acc[nb][k2]);
-                            acc[nb][V / 2 + k2] =
-                                __ffma2_rn(__fmul2_rn(gB, vb), r2, acc[nb][V / 2 + k2]);
+                            const float2 oA = __fmul2_rn(r2, __ffma2_rn(xh[u][nb][k2], nd2, hh[u][nb][k2]));
+                            const float2 oB = __fmul2_rn(
+                                r2, __ffma2_rn(xh[u][nb][V / 2 + k2], nd2, hh[u][nb][V / 2 + k2]));
                             IO::put2(oa, k2, oA.x, oA.y);
                             IO::put2(ob, k2, oB.x, oB.y);
                         }
+                        char *out = (char *)(isq ? a.qo : a.ko) +
+                                    ((isq ? t * a.Hq : t * a.Hkv) + hh_) * rowb;
                         lw_st_stream(out + offA, oa);
                         lw_st_stream(out + offB, ob);
                     }
                 }
             }
         }
+        if (aborted) break;
         __syncwarp();
         if (lane == 0) lw_bar_arrive(bar0 + 8 * (g.NS + s));
     }
+    if (aborted) s_abort = 1;
 
     if (MODE == kLwBwd) {
         // dgamma: the token groups of this CTA own the same elements, so sum
@@ -870,8 +878,10 @@ __global__ void __launch_bounds__((kLwCWMax + 1) * 32, 1)
         if (s_abort) return;
         for (int e = threadIdx.x; e < nel; e += ct) s_red[e] = 0.f;
         asm volatile("bar.sync 1, %0;" ::"r"(ct) : "memory");
+        // the B vector of a rotary pair is e + R/2 elements on; the
+        // geometry's element offsets say where each pair sum belongs
 #pragma unroll
-        for (int nb = 0; nb < kLwNBMax; ++nb) {
+        for (int nb = 0; nb < NBM; ++nb) {
             const int b = wb + nb * g.G;
             if (b >= g.HB) break;
             const int h = b * SLOTS + L.slot;
@@ -1275,7 +1285,9 @@ qknr_status lw_tok_launch(const LwArgs &a, const LwTokGeom &g, int grid, int sme
 template <typename T, int LPR, int MODE>
 qknr_status lw_pipe_launch(const LwArgs &a, const LwGeom &g, int grid, int smem, int threads,
                            cudaStream_t st) {
-    auto kern = qknr_lw_pipe_kernel<T, LPR, MODE>;
+    // head blocks a warp owns: one (two tokens a round) or two (one a round)
+    auto kern = (g.HB + g.G - 1) / g.G <= 1 ? qknr_lw_pipe_kernel<T, LPR, MODE, 1>
+                                            : qknr_lw_pipe_kernel<T, LPR, MODE, 2>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return cuda_fail(e);
     kern<<<grid, threads, smem, st>>>(a, g);
