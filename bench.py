@@ -540,21 +540,32 @@ def layerwise_variants(w, dense, dev, timed, line):
     def no_exchange(buf, span):  # one GPU: the sums are already the totals
         return None
 
+    def graphed(fn):
+        # the chunked schedule's host work (a few calls and events per chunk)
+        # would dominate short calls; a training step captures it in a CUDA
+        # graph, and so does this measurement: one capture, timed replays
+        fn()
+        torch.cuda.synchronize(dev)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        torch.cuda.synchronize(dev)
+        keep.append(g)
+        return g.replay
+
+    keep = []
+
     def chunked_f(s):
-        def run():
-            qknr.layerwise_chunked_fwd(s.q, s.k, gq, gk, s.pos, rotary_dim=w.rotary_dim,
-                                       theta=w.theta, eps=w.eps, Hq_total=w.Hq, Hkv_total=w.Hkv,
-                                       exchange=no_exchange,
-                                       chunks=qknr.DEFAULT_EXCHANGE_CHUNKS)
-        return run
+        return graphed(lambda: qknr.layerwise_chunked_fwd(
+            s.q, s.k, gq, gk, s.pos, rotary_dim=w.rotary_dim, theta=w.theta, eps=w.eps,
+            Hq_total=w.Hq, Hkv_total=w.Hkv, exchange=no_exchange,
+            chunks=qknr.DEFAULT_EXCHANGE_CHUNKS))
 
     def chunked_b(s, b):
-        def run():
-            qknr.layerwise_chunked_bwd(s.q, s.k, gq, gk, s.pos, b["rq"], b["rk"], s.dqo, s.dko,
-                                       rotary_dim=w.rotary_dim, theta=w.theta, Hq_total=w.Hq,
-                                       Hkv_total=w.Hkv, exchange=no_exchange,
-                                       chunks=qknr.DEFAULT_EXCHANGE_CHUNKS)
-        return run
+        return graphed(lambda: qknr.layerwise_chunked_bwd(
+            s.q, s.k, gq, gk, s.pos, b["rq"], b["rk"], s.dqo, s.dko, rotary_dim=w.rotary_dim,
+            theta=w.theta, Hq_total=w.Hq, Hkv_total=w.Hkv, exchange=no_exchange,
+            chunks=qknr.DEFAULT_EXCHANGE_CHUNKS))
 
     return {
         "layerwise_one_pass": {"fwd": line(timed(one_f), fwd_b), "bwd": line(timed(one_b), bwd_b),
@@ -565,8 +576,9 @@ def layerwise_variants(w, dense, dev, timed, line):
         "layerwise_tp_chunked": {
             "fwd": line(timed([chunked_f(s) for s in dense]), fwd_b),
             "bwd": line(timed([chunked_b(s, b) for s, b in zip(dense, bufs)]), bwd_b),
-            "entry": f"layerwise_chunked_fwd / _bwd, {qknr.DEFAULT_EXCHANGE_CHUNKS} token chunks, "
-                     "side-stream exchange (here a no-op: one GPU holds every head)"},
+            "entry": f"layerwise_chunked_fwd / _bwd, up to {qknr.DEFAULT_EXCHANGE_CHUNKS} token "
+                     f"chunks of >= {qknr.MIN_CHUNK_TOKENS} tokens, side-stream exchange (here a "
+                     "no-op: one GPU holds every head), captured in a CUDA graph and replayed"},
     }
 
 

@@ -825,11 +825,21 @@ def _flat_tokens(t: torch.Tensor) -> torch.Tensor:
     return t.reshape((B * S,) + tuple(t.shape[2:]))
 
 
+_POSITIONS = {}
+
+
 def _chunk_positions(pos_ids, B: int, S: int, device) -> torch.Tensor:
-    """Every token's position as int32 [B*S] (the given ids, else s)."""
+    """Every token's position as int32 [B*S]: the given ids, else s within
+    the batch row (written once per shape and device, then reused)."""
     if pos_ids is not None:
         return pos_ids.reshape(B * S)
-    return (torch.arange(B * S, device=device, dtype=torch.int64) % S).to(torch.int32)
+    key = (B, S, str(torch.device(device)))
+    p = _POSITIONS.get(key)
+    if p is None:
+        p = (torch.arange(B * S, device=device, dtype=torch.int64) % S).to(torch.int32)
+        if not torch.cuda.is_current_stream_capturing():
+            _POSITIONS[key] = p
+    return p
 
 
 def _all_reduce_exchange(group):

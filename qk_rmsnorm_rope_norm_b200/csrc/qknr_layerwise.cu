@@ -1187,9 +1187,16 @@ bool lw_plan(int mode, const LwArgs &a, int esz, int lpr, int sms, LwGeom *g, in
     const int slots = 32 / lpr, H = a.Hq + a.Hkv;
     const int HB = (H + slots - 1) / slots;
     // head blocks per warp, warps per token, token groups: every warp owns
-    // NB blocks (the last one maybe fewer), at most kLwCWMax warps
-    const int NB = (HB + kLwCWMax - 1) / kLwCWMax;
+    // NB blocks (the last one maybe fewer), at most kLwCWMax warps. Two
+    // blocks a warp (one token a round instead of two) when that lets a
+    // quarter more consumer warps run: more warps hide the shared-memory and
+    // group-sync latencies (Llama-3-8B shape: 3 groups of 5 warps, not 1 of 10)
+    int NB = (HB + kLwCWMax - 1) / kLwCWMax;
     if (NB > kLwNBMax) return false;
+    if (NB == 1 && HB > 1) {
+        const int G1 = HB, G2 = (HB + 1) / 2;
+        if (4 * G2 * (kLwCWMax / G2) >= 5 * G1 * (kLwCWMax / G1)) NB = 2;
+    }
     const int G = (HB + NB - 1) / NB;
     const int NTG = kLwCWMax / G;
     const int64_t rowb = (int64_t)a.D * esz;

@@ -198,11 +198,22 @@ __device__ __forceinline__ int64_t box_start(int64_t t0, int64_t t_hi, int TT) {
 __device__ __forceinline__ void stg16(void *p, const Vec16 &v) {
     __stcs(reinterpret_cast<uint4 *>(p), make_uint4(v.w[0], v.w[1], v.w[2], v.w[3]));
 }
-__device__ __forceinline__ Vec16 lds16(const unsigned char *p) {
-    const uint4 v = *reinterpret_cast<const uint4 *>(p);
+// 16-byte shared-memory loads at 32-bit shared addresses (the consumers keep
+// every address in 32 bits). Volatile keeps them in order with the mbarrier
+// waits and arrivals around them.
+__device__ __forceinline__ Vec16 lds16(uint32_t addr) {
     Vec16 r;
-    r.w[0] = v.x; r.w[1] = v.y; r.w[2] = v.z; r.w[3] = v.w;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r.w[0]), "=r"(r.w[1]), "=r"(r.w[2]), "=r"(r.w[3])
+                 : "r"(addr));
     return r;
+}
+__device__ __forceinline__ float4 ldsf4(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(addr));
+    return v;
 }
 
 // Everything a CTA knows about its run of tokens.
@@ -293,21 +304,28 @@ __device__ __forceinline__ void producers_sync(int nthreads) {
     asm volatile("bar.sync 2, %0;" ::"r"(nthreads) : "memory");
 }
 
-// Consumer: the V/2 (cos, sin) float4 of unit u for one token; (1, 1, 0, 0)
-// on pass-through units.
-template <int V>
-__device__ __forceinline__ void unit_table(const float4 *tok, bool rot, int u, float4 *cs) {
-    constexpr int W = V / 2;
-    if (rot) {
-        const float4 *t = tok + W * u;
-        const int sh = (u * W) >> 3;
+// Consumer: shared-memory byte offsets of a register pair's (cos, sin) and
+// gamma operands, fixed for the kernel. The table of a token holds R/2V
+// units of V/2 float4 (c_2P, c_2P+1, s_2P, s_2P+1); unit w's float4 k sits at
+// W w + (k + ((w W) >> 3)) mod W (the rotation that spreads a shared-memory
+// phase over eight bank groups; W = V/2). A pass-through unit reads the
+// identity table (1, 1, 0, 0) instead. Gamma's first vector of the pair is
+// rows kb, kb + 1, ... of the fp32 table at column w (^ X in the B half), its
+// second vector rows W/2 - kb, ...: a float4 row is 32 float4 (512 bytes).
+template <int V, int X> struct PairOffsets {
+    static constexpr int W = V / 2;
+    uint32_t cs[W];   // from the token's table (rotary unit) or the identity table
+    uint32_t g1, g2;  // gamma, first and second vector, float4 j at + j * 512
+    __device__ __forceinline__ void set(int w, bool rot, int kb) {
+        const int sh = (w * W) >> 3;
 #pragma unroll
-        for (int k = 0; k < W; ++k) cs[k] = t[(k + sh) % W];
-    } else {
-#pragma unroll
-        for (int k = 0; k < W; ++k) cs[k] = make_float4(1.f, 1.f, 0.f, 0.f);
+        for (int k = 0; k < W; ++k)
+            cs[k] = rot ? (uint32_t)(W * w + ((k + sh) & (W - 1))) * 16u : (uint32_t)k * 16u;
+        const int k1 = kb, k2 = W / 2 - kb;
+        g1 = (uint32_t)(k1 * 32 + (w ^ (k1 >= W / 2 ? X : 0))) * 16u;
+        g2 = (uint32_t)(k2 * 32 + (w ^ (k2 >= W / 2 ? X : 0))) * 16u;
     }
-}
+};
 
 __device__ __forceinline__ float2 neg2(float2 v) { return make_float2(-v.x, -v.y); }
 __device__ __forceinline__ float2 lo2(float4 v) { return make_float2(v.x, v.y); }
@@ -407,18 +425,6 @@ __device__ __forceinline__ void fill_unit_gamma(float4 (*s_gl)[V / 2][32], const
     }
 }
 
-// gamma of a pair: float4 j < V/4 of its first vector, then of its second.
-template <int V, int X>
-__device__ __forceinline__ void pair_gamma(const float4 (*gl)[32], int w, int kb, float4 *gv) {
-    constexpr int W = V / 2;
-#pragma unroll
-    for (int j = 0; j < W / 2; ++j) {
-        const int k1 = kb + j, k2 = (W / 2 - kb) + j;
-        gv[j] = gl[k1][w ^ (k1 >= W / 2 ? X : 0)];
-        gv[W / 2 + j] = gl[k2][w ^ (k2 >= W / 2 ? X : 0)];
-    }
-}
-
 // Barrier set-up, before the CTA-wide __syncthreads.
 template <int NCW, int NPW>
 __device__ __forceinline__ void init_barriers(uint32_t full0, uint32_t empty0, const PipeGeom &g) {
@@ -451,6 +457,7 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g,
     __shared__ __align__(8) uint64_t bars[2 * kMaxStages];
     __shared__ uint64_t s_step[kMaxHalf];
     __shared__ __align__(16) float4 s_gl[2][W][32];
+    __shared__ __align__(16) float4 s_ident[W];  // (cos, sin) of a pass-through unit
     __shared__ volatile int s_abort;
 
     // tensor copies land on 128-byte boundaries (the stage offsets are
@@ -464,6 +471,7 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g,
     const uint32_t full0 = smem_u32(&bars[0]), empty0 = smem_u32(&bars[kMaxStages]);
     init_barriers<NCW, NPW>(full0, empty0, g);
     if (threadIdx.x == 0) s_abort = 0;
+    if (threadIdx.x < W) s_ident[threadIdx.x] = make_float4(1.f, 1.f, 0.f, 0.f);
     const int half = a.R >> 1;
     // the angle steps depend on the arguments only: taken before the wait
     for (int i = threadIdx.x; i < half; i += blockDim.x) s_step[i] = turn_step(i, a.R, a.theta);
@@ -549,20 +557,24 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g,
                                  threadIdx.x - NPW * 32, NCW * 32);
         consumers_sync(NCW * 32);
         const Pairs<LPR, V, U> L(lane, a.D, a.R);
-        int off1[U], off2[U];
+        uint32_t off1[U], off2[U];
         float sgn[U];  // sine sign of each pair (negated again for the inverse rotation)
+        PairOffsets<V, X> po[U];
 #pragma unroll
         for (int q = 0; q < U; ++q) {
-            off1[q] = L.first[q] * (int)sizeof(T);
-            off2[q] = L.second[q] * (int)sizeof(T);
+            off1[q] = (uint32_t)(L.first[q] * (int)sizeof(T));
+            off2[q] = (uint32_t)(L.second[q] * (int)sizeof(T));
             sgn[q] = (mode & kModeInverse) ? -L.sgn[q] : L.sgn[q];
+            po[q].set(L.w[q], L.rot[q], L.kb[q]);
         }
+        const uint32_t smem0 = smem_u32(smem), ident0 = smem_u32(&s_ident[0]);
+        const uint32_t gq0 = smem_u32(&s_gl[0][0][0]), gk0 = smem_u32(&s_gl[1][0][0]);
         const float inv_d = 1.0f / (float)a.D;
         int pc = 0;  // passes dealt before this tile, mod NCW
         for (int it = 0; it < run.ntiles; ++it) {
             const int s = it % g.NS;
             if (!mbar_wait(full0 + 8 * s, (it / g.NS) & 1, 0)) break;
-            const unsigned char *st = smem + (size_t)s * g.stage_bytes;
+            const uint32_t st = smem0 + (uint32_t)(s * g.stage_bytes);
             const int64_t t0 = run.t_lo + (int64_t)it * g.TT;
             const int na = (int)min((int64_t)g.TT, run.t_hi - t0);
 
@@ -574,7 +586,7 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g,
             char *out_k = (char *)a.ko + t0 * a.Hkv * rowb;
             float *r_q = a.rq + t0 * a.Hq;
             float *r_k = a.rk + t0 * a.Hkv;
-            const float4 *cs_tile = reinterpret_cast<const float4 *>(st + g.off_cs);
+            const uint32_t cs_tile = st + (uint32_t)g.off_cs;
             const TilePasses tp(na, a.Hq, a.Hkv, SLOTS);
             const int npass = tp.npass;
             int p = (warp - NPW) - pc;
@@ -584,7 +596,7 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g,
                 const int j = (isq ? p : p - tp.pq) * SLOTS + L.slot;
                 const bool valid = j < (isq ? tp.rows_q : tp.rows_k);
                 const TileRow tr(isq, valid ? j : 0, g);
-                const unsigned char *src = st + (tr.isq ? xq0 : g.off_k + xk0) + tr.jj * rowb;
+                const uint32_t src = st + (uint32_t)((tr.isq ? xq0 : g.off_k + xk0) + tr.jj * rowb);
                 Vec16 xa[U], xb[U];
 #pragma unroll
                 for (int q = 0; q < U; ++q) xa[q] = lds16(src + off1[q]);
@@ -626,13 +638,20 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g,
                     r = rsqrtf(fmaf(ss, inv_d, a.eps));
                 }
                 const float2 r2 = make_float2(r, r);
-                const float4 *tok = cs_tile + tr.tl * (half >> 1);
+                const uint32_t tok = cs_tile + (uint32_t)(tr.tl * (half >> 1) * 16);
+                const uint32_t gtab = tr.isq ? gq0 : gk0;
                 char *out = (tr.isq ? out_q : out_k) + tr.jj * rowb;
 #pragma unroll
                 for (int q = 0; q < U && !(mode & kModeStatsOnly); ++q) {
                     float4 cs[W], gv[W];
-                    unit_table<V>(tok, L.rot[q], L.w[q], cs);
-                    pair_gamma<V, X>(s_gl[tr.isq ? 0 : 1], L.w[q], L.kb[q], gv);
+                    const uint32_t cb = L.rot[q] ? tok : ident0;
+#pragma unroll
+                    for (int k = 0; k < W; ++k) cs[k] = ldsf4(cb + po[q].cs[k]);
+#pragma unroll
+                    for (int k = 0; k < W / 2; ++k) {
+                        gv[k] = ldsf4(gtab + po[q].g1 + 512u * k);
+                        gv[W / 2 + k] = ldsf4(gtab + po[q].g2 + 512u * k);
+                    }
                     // r (and the pair's sine sign) folded into cos and sin
                     const float rs = r * sgn[q];
                     const float2 rs2 = make_float2(rs, rs);
@@ -685,6 +704,7 @@ qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g,
     __shared__ __align__(8) uint64_t bars[2 * kMaxStages];
     __shared__ uint64_t s_step[kMaxHalf];
     __shared__ __align__(16) float4 s_gl[2][W][32];
+    __shared__ __align__(16) float4 s_ident[W];  // (cos, sin) of a pass-through unit
     __shared__ volatile int s_abort;
     __shared__ float s_dg[2][kMaxD];
 
@@ -699,6 +719,7 @@ qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g,
     const uint32_t full0 = smem_u32(&bars[0]), empty0 = smem_u32(&bars[kMaxStages]);
     init_barriers<NCW, NPW>(full0, empty0, g);
     if (threadIdx.x == 0) s_abort = 0;
+    if (threadIdx.x < W) s_ident[threadIdx.x] = make_float4(1.f, 1.f, 0.f, 0.f);
     for (int i = threadIdx.x; i < 2 * kMaxD; i += blockDim.x) (&s_dg[0][0])[i] = 0.f;
     const int half = a.R >> 1;
     // the angle steps depend on the arguments only: taken before the wait
@@ -800,9 +821,13 @@ qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g,
                                  threadIdx.x - NPW * 32, NCW * 32);
         consumers_sync(NCW * 32);
         const Pairs<LPR, V, 1> L(lane, a.D, a.R);
-        const int off1 = L.first[0] * (int)sizeof(T), off2 = L.second[0] * (int)sizeof(T);
-        const int uu = L.w[0];
+        const uint32_t off1 = (uint32_t)(L.first[0] * (int)sizeof(T));
+        const uint32_t off2 = (uint32_t)(L.second[0] * (int)sizeof(T));
         const float2 sg = make_float2(L.sgn[0], L.sgn[0]);
+        PairOffsets<V, X> po;
+        po.set(L.w[0], L.rot[0], L.kb[0]);
+        const uint32_t smem0 = smem_u32(smem), ident0 = smem_u32(&s_ident[0]);
+        const uint32_t gq0 = smem_u32(&s_gl[0][0][0]), gk0 = smem_u32(&s_gl[1][0][0]);
         const float inv_d = 1.0f / (float)a.D;
         // dgamma partial sums: [k] = elements (first + 2k, first + 2k + 1),
         // same for the second vector
@@ -813,7 +838,7 @@ qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g,
         for (int it = 0; it < run.ntiles; ++it) {
             const int s = it % g.NS;
             if (!mbar_wait(full0 + 8 * s, (it / g.NS) & 1, 0)) break;
-            const unsigned char *st = smem + (size_t)s * g.stage_bytes;
+            const uint32_t st = smem0 + (uint32_t)(s * g.stage_bytes);
             const int64_t t0 = run.t_lo + (int64_t)it * g.TT;
             const int na = (int)min((int64_t)g.TT, run.t_hi - t0);
 
@@ -823,7 +848,7 @@ qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g,
             const int xk0 = (tmap & 2) ? skip * a.Hkv * rowb : 0;
             char *out_q = (char *)a.dq + t0 * a.dqts;
             char *out_k = (char *)a.dk + t0 * a.dkts;
-            const float4 *cs_tile = reinterpret_cast<const float4 *>(st + g.off_cs);
+            const uint32_t cs_tile = st + (uint32_t)g.off_cs;
             const TilePasses tp(na, a.Hq, a.Hkv, SLOTS);
             const int npass = tp.npass;
             int p = (warp - NPW) - pc;
@@ -834,36 +859,93 @@ qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g,
                 const bool in = j < (isq ? tp.rows_q : tp.rows_k);
                 const bool valid = in && L.on[0];
                 const TileRow tr(isq, in ? j : 0, g);
-                const unsigned char *xs = st + (tr.isq ? xq0 : g.off_k + xk0) + tr.jj * rowb;
-                const unsigned char *ds = st + (tr.isq ? g.off_dq : g.off_dk) + tr.jj * rowb;
+                const uint32_t xs = st + (uint32_t)((tr.isq ? xq0 : g.off_k + xk0) + tr.jj * rowb);
+                const uint32_t ds = st + (uint32_t)((tr.isq ? g.off_dq : g.off_dk) + tr.jj * rowb);
                 const Vec16 xa = lds16(xs + off1), da = lds16(ds + off1);
                 const Vec16 xb = lds16(xs + off2), db = lds16(ds + off2);
-                float r = reinterpret_cast<const float *>(st + (tr.isq ? g.off_rq : g.off_rk))[tr.jj];
+                float r;
+                asm volatile("ld.shared.f32 %0, [%1];"
+                             : "=f"(r)
+                             : "r"(st + (uint32_t)((tr.isq ? g.off_rq : g.off_rk) + 4 * tr.jj)));
                 r = valid ? r : 0.f;  // rows past the tile and off lanes add nothing
                 float4 cs[W], gv[W];
-                unit_table<V>(cs_tile + tr.tl * (half >> 1), L.rot[0], uu, cs);
-                pair_gamma<V, X>(s_gl[tr.isq ? 0 : 1], uu, L.kb[0], gv);
-                const float2 r2 = make_float2(r, r);
-                float2 nmr2 = make_float2(0.f, 0.f);  // -mean * r (mean-centred variant)
-                if (LN) {
-                    float2 s0 = make_float2(0.f, 0.f);
+                const uint32_t cb = L.rot[0] ? cs_tile + (uint32_t)(tr.tl * (half >> 1) * 16) : ident0;
+                const uint32_t gtab = tr.isq ? gq0 : gk0;
 #pragma unroll
-                    for (int k = 0; k < W; ++k)
-                        s0 = __fadd2_rn(s0, __fadd2_rn(IO::get2(xa, k), IO::get2(xb, k)));
-                    const float mu = group_sum<LPR>(L.on[0] ? s0.x + s0.y : 0.f) * inv_d;
-                    nmr2 = make_float2(-mu * r, -mu * r);
+                for (int k = 0; k < W; ++k) cs[k] = ldsf4(cb + po.cs[k]);
+#pragma unroll
+                for (int k = 0; k < W / 2; ++k) {
+                    gv[k] = ldsf4(gtab + po.g1 + 512u * k);
+                    gv[W / 2 + k] = ldsf4(gtab + po.g2 + 512u * k);
                 }
-                float2 ha[W], hb[W], xha[W], xhb[W];
-                float2 d0 = make_float2(0.f, 0.f), d1 = make_float2(0.f, 0.f);
-                float2 e0 = make_float2(0.f, 0.f);  // sum of h (mean-centred variant)
+                const float2 r2 = make_float2(r, r);
+                if constexpr (LN) {
+                // one pass forms g (dy un-rotated) and the row sums of x,
+                // h = g gamma and h x; with mu = mean(x), xh = (x - mu) r:
+                //   <h, xh> / D = r (sum(h x) / D - mu mean(h))
+                //   dx = r (h - mean(h) - xh <h, xh> / D) = r h + A x + B
+                // so dx and the dgamma terms g xh come from x and g alone
+                float2 xA[W], xB[W], gAv[W], gBv[W];
+                float2 sx = make_float2(0.f, 0.f), sh = make_float2(0.f, 0.f);
+                float2 shx = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int k = 0; k < W; ++k) {
                     const float2 ga = (k & 1) ? hi2(gv[k >> 1]) : lo2(gv[k >> 1]);
                     const float2 gb = (k & 1) ? hi2(gv[W / 2 + (k >> 1)]) : lo2(gv[W / 2 + (k >> 1)]);
                     const float2 c = lo2(cs[k]), sn = __fmul2_rn(hi2(cs[k]), sg);
                     const float2 dA = IO::get2(da, k), dB = IO::get2(db, k);
-                    xha[k] = LN ? __ffma2_rn(IO::get2(xa, k), r2, nmr2) : __fmul2_rn(IO::get2(xa, k), r2);
-                    xhb[k] = LN ? __ffma2_rn(IO::get2(xb, k), r2, nmr2) : __fmul2_rn(IO::get2(xb, k), r2);
+                    xA[k] = IO::get2(xa, k);
+                    xB[k] = IO::get2(xb, k);
+                    gAv[k] = __ffma2_rn(dA, c, __fmul2_rn(dB, sn));
+                    gBv[k] = __ffma2_rn(dB, c, __fmul2_rn(dA, neg2(sn)));
+                    const float2 hA = __fmul2_rn(gAv[k], ga), hB = __fmul2_rn(gBv[k], gb);
+                    sx = __fadd2_rn(sx, __fadd2_rn(xA[k], xB[k]));
+                    sh = __fadd2_rn(sh, __fadd2_rn(hA, hB));
+                    shx = __ffma2_rn(hA, xA[k], __ffma2_rn(hB, xB[k], shx));
+                }
+                const float mu = group_sum<LPR>(L.on[0] ? sx.x + sx.y : 0.f) * inv_d;
+                const float mh = group_sum<LPR>(sh.x + sh.y) * inv_d;
+                const float dd = r * (group_sum<LPR>(shx.x + shx.y) * inv_d - mu * mh);
+                const float A = -r * r * dd, Bc = r * (r * dd * mu - mh);
+                const float2 A2 = make_float2(A, A), B2 = make_float2(Bc, Bc);
+                const float2 nmr2 = make_float2(-mu * r, -mu * r);
+                Vec16 oa, ob;
+#pragma unroll
+                for (int k = 0; k < W; ++k) {
+                    const float2 ga = (k & 1) ? hi2(gv[k >> 1]) : lo2(gv[k >> 1]);
+                    const float2 gb = (k & 1) ? hi2(gv[W / 2 + (k >> 1)]) : lo2(gv[W / 2 + (k >> 1)]);
+                    const float2 xhA = __ffma2_rn(xA[k], r2, nmr2), xhB = __ffma2_rn(xB[k], r2, nmr2);
+                    if (tr.isq) {
+                        aqa[k] = __ffma2_rn(gAv[k], xhA, aqa[k]);
+                        aqb[k] = __ffma2_rn(gBv[k], xhB, aqb[k]);
+                    } else {
+                        aka[k] = __ffma2_rn(gAv[k], xhA, aka[k]);
+                        akb[k] = __ffma2_rn(gBv[k], xhB, akb[k]);
+                    }
+                    const float2 va = __ffma2_rn(xA[k], A2, __ffma2_rn(__fmul2_rn(gAv[k], ga), r2, B2));
+                    const float2 vb = __ffma2_rn(xB[k], A2, __ffma2_rn(__fmul2_rn(gBv[k], gb), r2, B2));
+                    IO::put2(oa, k, va.x, va.y);
+                    IO::put2(ob, k, vb.x, vb.y);
+                }
+                if (valid) {
+                    // row (tl, h) of dq / dk, whose tokens may be strided
+                    const int hz = tr.isq ? a.Hq : a.Hkv;
+                    char *out = (tr.isq ? out_q : out_k) + (int64_t)tr.tl * (tr.isq ? a.dqts : a.dkts) +
+                                (tr.jj - tr.tl * hz) * rowb;
+                    stg16(out + off1, oa);
+                    stg16(out + off2, ob);
+                }
+                } else {
+                float2 ha[W], hb[W], xha[W], xhb[W];
+                float2 d0 = make_float2(0.f, 0.f), d1 = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int k = 0; k < W; ++k) {
+                    const float2 ga = (k & 1) ? hi2(gv[k >> 1]) : lo2(gv[k >> 1]);
+                    const float2 gb = (k & 1) ? hi2(gv[W / 2 + (k >> 1)]) : lo2(gv[W / 2 + (k >> 1)]);
+                    const float2 c = lo2(cs[k]), sn = __fmul2_rn(hi2(cs[k]), sg);
+                    const float2 dA = IO::get2(da, k), dB = IO::get2(db, k);
+                    xha[k] = __fmul2_rn(IO::get2(xa, k), r2);
+                    xhb[k] = __fmul2_rn(IO::get2(xb, k), r2);
                     const float2 gA = __ffma2_rn(dA, c, __fmul2_rn(dB, sn));
                     const float2 gB = __ffma2_rn(dB, c, __fmul2_rn(dA, neg2(sn)));
                     if (tr.isq) {
@@ -877,19 +959,15 @@ qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g,
                     hb[k] = __fmul2_rn(gB, gb);
                     d0 = __ffma2_rn(ha[k], xha[k], d0);
                     d1 = __ffma2_rn(hb[k], xhb[k], d1);
-                    if (LN) e0 = __fadd2_rn(e0, __fadd2_rn(ha[k], hb[k]));
                 }
                 const float dot = group_sum<LPR>((d0.x + d1.x) + (d0.y + d1.y)) * inv_d;
-                const float mh = LN ? group_sum<LPR>(e0.x + e0.y) * inv_d : 0.f;
                 if (valid) {
-                    const float2 nd = make_float2(-dot, -dot), nmh = make_float2(-mh, -mh);
+                    const float2 nd = make_float2(-dot, -dot);
                     Vec16 oa, ob;
 #pragma unroll
                     for (int k = 0; k < W; ++k) {
-                        const float2 pa = LN ? __fadd2_rn(ha[k], nmh) : ha[k];
-                        const float2 pb = LN ? __fadd2_rn(hb[k], nmh) : hb[k];
-                        const float2 va = __fmul2_rn(__ffma2_rn(xha[k], nd, pa), r2);
-                        const float2 vb = __fmul2_rn(__ffma2_rn(xhb[k], nd, pb), r2);
+                        const float2 va = __fmul2_rn(__ffma2_rn(xha[k], nd, ha[k]), r2);
+                        const float2 vb = __fmul2_rn(__ffma2_rn(xhb[k], nd, hb[k]), r2);
                         IO::put2(oa, k, va.x, va.y);
                         IO::put2(ob, k, vb.x, vb.y);
                     }
@@ -899,6 +977,7 @@ qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g,
                                 (tr.jj - tr.tl * hz) * rowb;
                     stg16(out + off1, oa);
                     stg16(out + off2, ob);
+                }
                 }
             }
             pc = (pc + npass) % NCW;
