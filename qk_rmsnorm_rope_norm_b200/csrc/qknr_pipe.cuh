@@ -308,19 +308,18 @@ __device__ __forceinline__ void producers_sync(int nthreads) {
 // gamma operands, fixed for the kernel. The table of a token holds R/2V
 // units of V/2 float4 (c_2P, c_2P+1, s_2P, s_2P+1); unit w's float4 k sits at
 // W w + (k + ((w W) >> 3)) mod W (the rotation that spreads a shared-memory
-// phase over eight bank groups; W = V/2). A pass-through unit reads the
-// identity table (1, 1, 0, 0) instead. Gamma's first vector of the pair is
+// phase over eight bank groups; W = V/2); a pass-through unit reads none and
+// takes (cos, sin) = (1, 0). Gamma's first vector of the pair is
 // rows kb, kb + 1, ... of the fp32 table at column w (^ X in the B half), its
 // second vector rows W/2 - kb, ...: a float4 row is 32 float4 (512 bytes).
 template <int V, int X> struct PairOffsets {
     static constexpr int W = V / 2;
-    uint32_t cs[W];   // from the token's table (rotary unit) or the identity table
+    uint32_t cs[W];   // from the token's table (rotary units)
     uint32_t g1, g2;  // gamma, first and second vector, float4 j at + j * 512
-    __device__ __forceinline__ void set(int w, bool rot, int kb) {
+    __device__ __forceinline__ void set(int w, int kb) {
         const int sh = (w * W) >> 3;
 #pragma unroll
-        for (int k = 0; k < W; ++k)
-            cs[k] = rot ? (uint32_t)(W * w + ((k + sh) & (W - 1))) * 16u : (uint32_t)k * 16u;
+        for (int k = 0; k < W; ++k) cs[k] = (uint32_t)(W * w + ((k + sh) & (W - 1))) * 16u;
         const int k1 = kb, k2 = W / 2 - kb;
         g1 = (uint32_t)(k1 * 32 + (w ^ (k1 >= W / 2 ? X : 0))) * 16u;
         g2 = (uint32_t)(k2 * 32 + (w ^ (k2 >= W / 2 ? X : 0))) * 16u;
@@ -457,7 +456,6 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g,
     __shared__ __align__(8) uint64_t bars[2 * kMaxStages];
     __shared__ uint64_t s_step[kMaxHalf];
     __shared__ __align__(16) float4 s_gl[2][W][32];
-    __shared__ __align__(16) float4 s_ident[W];  // (cos, sin) of a pass-through unit
     __shared__ volatile int s_abort;
 
     // tensor copies land on 128-byte boundaries (the stage offsets are
@@ -471,7 +469,6 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g,
     const uint32_t full0 = smem_u32(&bars[0]), empty0 = smem_u32(&bars[kMaxStages]);
     init_barriers<NCW, NPW>(full0, empty0, g);
     if (threadIdx.x == 0) s_abort = 0;
-    if (threadIdx.x < W) s_ident[threadIdx.x] = make_float4(1.f, 1.f, 0.f, 0.f);
     const int half = a.R >> 1;
     // the angle steps depend on the arguments only: taken before the wait
     for (int i = threadIdx.x; i < half; i += blockDim.x) s_step[i] = turn_step(i, a.R, a.theta);
@@ -565,9 +562,9 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g,
             off1[q] = (uint32_t)(L.first[q] * (int)sizeof(T));
             off2[q] = (uint32_t)(L.second[q] * (int)sizeof(T));
             sgn[q] = (mode & kModeInverse) ? -L.sgn[q] : L.sgn[q];
-            po[q].set(L.w[q], L.rot[q], L.kb[q]);
+            po[q].set(L.w[q], L.kb[q]);
         }
-        const uint32_t smem0 = smem_u32(smem), ident0 = smem_u32(&s_ident[0]);
+        const uint32_t smem0 = smem_u32(smem);
         const uint32_t gq0 = smem_u32(&s_gl[0][0][0]), gk0 = smem_u32(&s_gl[1][0][0]);
         const float inv_d = 1.0f / (float)a.D;
         int pc = 0;  // passes dealt before this tile, mod NCW
@@ -644,9 +641,13 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g,
 #pragma unroll
                 for (int q = 0; q < U && !(mode & kModeStatsOnly); ++q) {
                     float4 cs[W], gv[W];
-                    const uint32_t cb = L.rot[q] ? tok : ident0;
+                    if (L.rot[q]) {
 #pragma unroll
-                    for (int k = 0; k < W; ++k) cs[k] = ldsf4(cb + po[q].cs[k]);
+                        for (int k = 0; k < W; ++k) cs[k] = ldsf4(tok + po[q].cs[k]);
+                    } else {  // pass-through unit: (cos, sin) = (1, 0), no load
+#pragma unroll
+                        for (int k = 0; k < W; ++k) cs[k] = make_float4(1.f, 1.f, 0.f, 0.f);
+                    }
 #pragma unroll
                     for (int k = 0; k < W / 2; ++k) {
                         gv[k] = ldsf4(gtab + po[q].g1 + 512u * k);
@@ -704,7 +705,6 @@ qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g,
     __shared__ __align__(8) uint64_t bars[2 * kMaxStages];
     __shared__ uint64_t s_step[kMaxHalf];
     __shared__ __align__(16) float4 s_gl[2][W][32];
-    __shared__ __align__(16) float4 s_ident[W];  // (cos, sin) of a pass-through unit
     __shared__ volatile int s_abort;
     __shared__ float s_dg[2][kMaxD];
 
@@ -719,7 +719,6 @@ qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g,
     const uint32_t full0 = smem_u32(&bars[0]), empty0 = smem_u32(&bars[kMaxStages]);
     init_barriers<NCW, NPW>(full0, empty0, g);
     if (threadIdx.x == 0) s_abort = 0;
-    if (threadIdx.x < W) s_ident[threadIdx.x] = make_float4(1.f, 1.f, 0.f, 0.f);
     for (int i = threadIdx.x; i < 2 * kMaxD; i += blockDim.x) (&s_dg[0][0])[i] = 0.f;
     const int half = a.R >> 1;
     // the angle steps depend on the arguments only: taken before the wait
@@ -825,8 +824,8 @@ qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g,
         const uint32_t off2 = (uint32_t)(L.second[0] * (int)sizeof(T));
         const float2 sg = make_float2(L.sgn[0], L.sgn[0]);
         PairOffsets<V, X> po;
-        po.set(L.w[0], L.rot[0], L.kb[0]);
-        const uint32_t smem0 = smem_u32(smem), ident0 = smem_u32(&s_ident[0]);
+        po.set(L.w[0], L.kb[0]);
+        const uint32_t smem0 = smem_u32(smem);
         const uint32_t gq0 = smem_u32(&s_gl[0][0][0]), gk0 = smem_u32(&s_gl[1][0][0]);
         const float inv_d = 1.0f / (float)a.D;
         // dgamma partial sums: [k] = elements (first + 2k, first + 2k + 1),
@@ -869,10 +868,15 @@ qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g,
                              : "r"(st + (uint32_t)((tr.isq ? g.off_rq : g.off_rk) + 4 * tr.jj)));
                 r = valid ? r : 0.f;  // rows past the tile and off lanes add nothing
                 float4 cs[W], gv[W];
-                const uint32_t cb = L.rot[0] ? cs_tile + (uint32_t)(tr.tl * (half >> 1) * 16) : ident0;
-                const uint32_t gtab = tr.isq ? gq0 : gk0;
+                if (L.rot[0]) {
+                    const uint32_t cb = cs_tile + (uint32_t)(tr.tl * (half >> 1) * 16);
 #pragma unroll
-                for (int k = 0; k < W; ++k) cs[k] = ldsf4(cb + po.cs[k]);
+                    for (int k = 0; k < W; ++k) cs[k] = ldsf4(cb + po.cs[k]);
+                } else {  // pass-through unit: (cos, sin) = (1, 0), no load
+#pragma unroll
+                    for (int k = 0; k < W; ++k) cs[k] = make_float4(1.f, 1.f, 0.f, 0.f);
+                }
+                const uint32_t gtab = tr.isq ? gq0 : gk0;
 #pragma unroll
                 for (int k = 0; k < W / 2; ++k) {
                     gv[k] = ldsf4(gtab + po.g1 + 512u * k);
