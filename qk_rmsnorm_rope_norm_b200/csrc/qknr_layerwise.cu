@@ -476,14 +476,6 @@ __device__ __forceinline__ void lw_st_stream(void *p, const Vec16 &v) {
     __stcs(reinterpret_cast<uint4 *>(p), make_uint4(v.w[0], v.w[1], v.w[2], v.w[3]));
 }
 
-// Stage row of token j, head h (local Q heads, then K heads) in section
-// `q0` (Q rows) / `k0` (K rows).
-__device__ __forceinline__ const unsigned char *stage_row(const unsigned char *q0,
-                                                          const unsigned char *k0, int j, int h,
-                                                          int Hq, int Hkv, int rowb) {
-    return h < Hq ? q0 + (j * Hq + h) * rowb : k0 + (j * Hkv + (h - Hq)) * rowb;
-}
-
 __device__ __forceinline__ float2 neg2f(float2 v) { return make_float2(-v.x, -v.y); }
 
 // Token j's sums over all heads: its G per-warp partials added in warp order
@@ -498,16 +490,56 @@ __device__ __forceinline__ float2 token_total(const float2 *parts, int j, int G)
     return tot;
 }
 
-// A lane's (cos, sin) pairs for elements eA .. eA + V - 1 of token table
-// `tok` (float4 per pair, pair k of unit w at k U + w, U = hp / (V / 2));
-// (1, 1, 0, 0) on lanes past the rotary span.
-template <int V, typename LaneT>
-__device__ __forceinline__ void lane_cs4(float4 (&c)[V / 2], const float4 *tok, const LaneT &L,
-                                         int U) {
-    const int w = L.eA / V;
+// Shared-memory loads at 32-bit shared addresses (the pipelined consumers
+// keep every shared address in 32 bits). Volatile keeps them in order with
+// the mbarrier waits and arrivals around them.
+__device__ __forceinline__ Vec16 lw_lds16(uint32_t addr) {
+    Vec16 r;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r.w[0]), "=r"(r.w[1]), "=r"(r.w[2]), "=r"(r.w[3])
+                 : "r"(addr));
+    return r;
+}
+__device__ __forceinline__ float4 lw_ldsf4(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ float2 lw_ldsf2(uint32_t addr) {
+    float2 v;
+    asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
+    return v;
+}
+// Row h of token j in a stage whose Q rows start at q0 and K rows at k0.
+__device__ __forceinline__ uint32_t stage_row32(uint32_t q0, uint32_t k0, int j, int h, int Hq,
+                                                int Hkv, int rowb) {
+    return h < Hq ? q0 + (uint32_t)((j * Hq + h) * rowb) : k0 + (uint32_t)((j * Hkv + (h - Hq)) * rowb);
+}
+// A lane's (cos, sin) pairs for elements eA .. eA + V - 1 come from its
+// token's table: float4 per pair, pair k of unit w at k U + w (U = hp / (V/2)
+// rotating units). The byte offsets are fixed for the kernel; lanes past the
+// rotary span load none and take (1, 1, 0, 0).
+template <int V> struct LwCsOffsets {
+    uint32_t o[V / 2];
+    template <typename LaneT>
+    __device__ __forceinline__ LwCsOffsets(const LaneT &L, int U) {
+        const int w = L.eA / V;
 #pragma unroll
-    for (int k = 0; k < V / 2; ++k)
-        c[k] = L.rot ? tok[k * U + w] : make_float4(1.f, 1.f, 0.f, 0.f);
+        for (int k = 0; k < V / 2; ++k) o[k] = (uint32_t)(k * U + w) * 16u;
+    }
+};
+template <int V, typename LaneT>
+__device__ __forceinline__ void lane_cs4_32(float4 (&c)[V / 2], uint32_t tok,
+                                            const LwCsOffsets<V> &co, const LaneT &L) {
+    if (L.rot) {
+#pragma unroll
+        for (int k = 0; k < V / 2; ++k) c[k] = lw_ldsf4(tok + co.o[k]);
+    } else {
+#pragma unroll
+        for (int k = 0; k < V / 2; ++k) c[k] = make_float4(1.f, 1.f, 0.f, 0.f);
+    }
 }
 
 // The producer warp's share of a stage's (cos, sin) table: pair P of a token
@@ -692,8 +724,10 @@ __global__ void __launch_bounds__((kLwCWMax + 1) * 32, 1)
     // from the registers (no second pass over the rows).
     const int tg = warp / g.G, wb = warp % g.G;
     const Lane<LPR, V> L(lane, a.D, a.R);
-    const int offA = L.eA * E, offB = L.eB * E;
+    const uint32_t offA = (uint32_t)(L.eA * E), offB = (uint32_t)(L.eB * E);
     const int hp = half >> 1;  // rotary pairs per token
+    const LwCsOffsets<V> co(L, hp / (V / 2));
+    const uint32_t ring32 = lw_smem_u32(ring), gam32 = lw_smem_u32(s_gamma);
     const bool local = MODE == kLwBwd && a.sq == nullptr && a.sk == nullptr;
     const bool need_parts = MODE == kLwDots || local;
     constexpr int UA = NBM == 1 ? 2 : 1;  // tokens per round
@@ -715,11 +749,10 @@ __global__ void __launch_bounds__((kLwCWMax + 1) * 32, 1)
         }
         const int64_t t0 = t_lo + (int64_t)i * g.TT;
         const int na = (int)min((int64_t)g.TT, t_hi - t0);
-        const unsigned char *st = ring + (size_t)s * g.stage_bytes;
-        const unsigned char *xq = st, *xk = st + g.off_k;
-        const unsigned char *dq0 = st + g.off_dq, *dk0 = st + g.off_dk;
-        const float4 *cs_st = reinterpret_cast<const float4 *>(st + g.off_cs);
-        const float4 *sc = reinterpret_cast<const float4 *>(st + g.off_sc);
+        const uint32_t st = ring32 + (uint32_t)(s * g.stage_bytes);
+        const uint32_t xq = st, xk = st + (uint32_t)g.off_k;
+        const uint32_t dq0 = st + (uint32_t)g.off_dq, dk0 = st + (uint32_t)g.off_dk;
+        const uint32_t cs_st = st + (uint32_t)g.off_cs, sc = st + (uint32_t)g.off_sc;
         float2 *parts = parts_all + (size_t)s * g.TT * g.G;
 
         for (int j0 = tg; j0 < na; j0 += UA * g.NTG) {
@@ -731,8 +764,9 @@ __global__ void __launch_bounds__((kLwCWMax + 1) * 32, 1)
                 vq[u] = vk[u] = 0.f;
                 const bool tok_ok = j < na;
                 float4 c[V / 2];
-                lane_cs4<V>(c, cs_st + (tok_ok ? j : j0) * hp, L, hp / (V / 2));
-                const float4 sv = sc[tok_ok ? j : j0];
+                const int jt = tok_ok ? j : j0;
+                lane_cs4_32<V>(c, cs_st + (uint32_t)(jt * hp * 16), co, L);
+                const float4 sv = lw_ldsf4(sc + (uint32_t)(jt * 16));
 #pragma unroll
                 for (int nb = 0; nb < NBM; ++nb) {
                     const int b = wb + nb * g.G;
@@ -740,12 +774,12 @@ __global__ void __launch_bounds__((kLwCWMax + 1) * 32, 1)
                     const bool on = tok_ok && b < g.HB && L.on && h < H;
                     const bool isq = h < a.Hq;
                     const int hs = on ? h : 0;
-                    const unsigned char *row = stage_row(xq, xk, on ? j : 0, hs, a.Hq, a.Hkv, rowb);
-                    const unsigned char *drow = stage_row(dq0, dk0, on ? j : 0, hs, a.Hq, a.Hkv, rowb);
-                    const unsigned char *grow = s_gamma + hs * rowb;
-                    const Vec16 xa = ld16(row + offA), xb = ld16(row + offB);
-                    const Vec16 da = ld16(drow + offA), db = ld16(drow + offB);
-                    const Vec16 ga = ld16(grow + offA), gb = ld16(grow + offB);
+                    const uint32_t row = stage_row32(xq, xk, on ? j : 0, hs, a.Hq, a.Hkv, rowb);
+                    const uint32_t drow = stage_row32(dq0, dk0, on ? j : 0, hs, a.Hq, a.Hkv, rowb);
+                    const uint32_t grow = gam32 + (uint32_t)(hs * rowb);
+                    const Vec16 xa = lw_lds16(row + offA), xb = lw_lds16(row + offB);
+                    const Vec16 da = lw_lds16(drow + offA), db = lw_lds16(drow + offB);
+                    const Vec16 ga = lw_lds16(grow + offA), gb = lw_lds16(grow + offB);
                     const float r = on ? (isq ? sv.x : sv.y) : 0.f;  // off rows add nothing
                     const float2 r2 = make_float2(r, r);
                     float2 p2 = make_float2(0.f, 0.f);
@@ -821,7 +855,7 @@ __global__ void __launch_bounds__((kLwCWMax + 1) * 32, 1)
 #pragma unroll
                 for (int u = 0; u < UA; ++u) {
                     const int j = j0 + u * g.NTG;
-                    const float4 sv = sc[j < na ? j : j0];
+                    const float4 sv = lw_ldsf4(sc + (uint32_t)((j < na ? j : j0) * 16));
                     tot[u] = make_float2(sv.z, sv.w);
                 }
             }
@@ -832,7 +866,7 @@ __global__ void __launch_bounds__((kLwCWMax + 1) * 32, 1)
                     const int j = j0 + u * g.NTG;
                     if (j >= na) continue;
                     const int64_t t = t0 + j;
-                    const float4 sv = sc[j];
+                    const float4 sv = lw_ldsf4(sc + (uint32_t)(j * 16));
                     const float nq = -tot[u].x * a.inv_q, nk = -tot[u].y * a.inv_k;
 #pragma unroll
                     for (int nb = 0; nb < NBM; ++nb) {
@@ -928,9 +962,9 @@ struct LwTokGeom {
 // Sums of x^2 over the rows of one token held in shared memory (Q rows at
 // xq, K rows at xk), the warp totals in every lane.
 template <typename T, int LPR>
-__device__ __forceinline__ float2 tok_sumsq(const unsigned char *xq, const unsigned char *xk,
+__device__ __forceinline__ float2 tok_sumsq(uint32_t xq, uint32_t xk,
                                             const Lane<LPR, Io<T>::V> &L, int Hq, int H,
-                                            int rowb, int offA, int offB) {
+                                            int rowb, uint32_t offA, uint32_t offB) {
     using IO = Io<T>;
     constexpr int V = IO::V, SLOTS = 32 / LPR;
     float2 pq = make_float2(0.f, 0.f), pk = make_float2(0.f, 0.f);
@@ -938,8 +972,8 @@ __device__ __forceinline__ float2 tok_sumsq(const unsigned char *xq, const unsig
         const int h = p + L.slot;
         if (!(L.on && h < H)) continue;
         const bool isq = h < Hq;
-        const unsigned char *row = isq ? xq + h * rowb : xk + (h - Hq) * rowb;
-        const Vec16 xa = ld16(row + offA), xb = ld16(row + offB);
+        const uint32_t row = isq ? xq + (uint32_t)(h * rowb) : xk + (uint32_t)((h - Hq) * rowb);
+        const Vec16 xa = lw_lds16(row + offA), xb = lw_lds16(row + offB);
         float2 s0 = make_float2(0.f, 0.f);
 #pragma unroll
         for (int k2 = 0; k2 < V / 2; ++k2) {
@@ -1063,30 +1097,32 @@ __global__ void __launch_bounds__((kLwCWMax + 1) * 32, 1)
 
     // ---------------------------------------------------------------- consumers
     const Lane<LPR, V> L(lane, a.D, a.R);
-    const int offA = L.eA * E, offB = L.eB * E;
+    const uint32_t offA = (uint32_t)(L.eA * E), offB = (uint32_t)(L.eB * E);
     // the sums use the lane layout without a rotary span (the statistics
     // call has none), so every call adds the same terms in the same order
     const Lane<LPR, V> Ls(lane, a.D, 0);
-    const int offAs = Ls.eA * E, offBs = Ls.eB * E;
+    const uint32_t offAs = (uint32_t)(Ls.eA * E), offBs = (uint32_t)(Ls.eB * E);
     const int hp = half >> 1;  // rotary pairs per token
+    const LwCsOffsets<V> co(L, hp / (V / 2));
+    const uint32_t ring32 = lw_smem_u32(ring), gam32 = lw_smem_u32(s_gamma);
     int pc = 0;                // tokens dealt before this stage, mod ncw
     for (int i = 0; i < ntiles; ++i) {
         const int s = i % g.NS;
         if (!lw_wait(bar0 + 8 * s, (uint32_t)(i / g.NS) & 1u)) break;
         const int64_t t0 = t_lo + (int64_t)i * g.TT;
         const int na = (int)min((int64_t)g.TT, t_hi - t0);
-        const unsigned char *st = ring + (size_t)s * g.stage_bytes;
+        const uint32_t st = ring32 + (uint32_t)(s * g.stage_bytes);
         int j = warp - pc;
         if (j < 0) j += ncw;
         for (; j < na; j += ncw) {
             const int64_t t = t0 + j;
-            const unsigned char *xq = st + j * a.Hq * rowb;
-            const unsigned char *xk = st + g.off_k + j * a.Hkv * rowb;
+            const uint32_t xq = st + (uint32_t)(j * a.Hq * rowb);
+            const uint32_t xk = st + (uint32_t)(g.off_k + j * a.Hkv * rowb);
             float2 tot;
             if (MODE == kTokStats || local) {
                 tot = tok_sumsq<T, LPR>(xq, xk, Ls, a.Hq, H, rowb, offAs, offBs);
             } else {
-                tot = reinterpret_cast<const float2 *>(st + g.off_sc)[j];
+                tot = lw_ldsf2(st + (uint32_t)(g.off_sc + 8 * j));
             }
             if (MODE == kTokStats) {
                 if (lane == 0) {
@@ -1102,17 +1138,16 @@ __global__ void __launch_bounds__((kLwCWMax + 1) * 32, 1)
                 if (a.Hkv) a.wk[t] = rk;
             }
             float4 c[V / 2];
-            lane_cs4<V>(c, reinterpret_cast<const float4 *>(st + g.off_cs) + j * hp, L,
-                        hp / (V / 2));
+            lane_cs4_32<V>(c, st + (uint32_t)(g.off_cs + j * hp * 16), co, L);
             for (int p = 0; p < H; p += SLOTS) {
                 const int h = p + L.slot;
                 if (!(L.on && h < H)) continue;
                 const bool isq = h < a.Hq;
                 const int hh = isq ? h : h - a.Hq;
-                const unsigned char *row = isq ? xq + h * rowb : xk + hh * rowb;
-                const unsigned char *grow = s_gamma + h * rowb;
-                const Vec16 xa = ld16(row + offA), xb = ld16(row + offB);
-                const Vec16 ga = ld16(grow + offA), gb = ld16(grow + offB);
+                const uint32_t row = isq ? xq + (uint32_t)(h * rowb) : xk + (uint32_t)(hh * rowb);
+                const uint32_t grow = gam32 + (uint32_t)(h * rowb);
+                const Vec16 xa = lw_lds16(row + offA), xb = lw_lds16(row + offB);
+                const Vec16 ga = lw_lds16(grow + offA), gb = lw_lds16(grow + offB);
                 const float r = isq ? rq : rk;
                 const float2 r2 = make_float2(r, r);
                 Vec16 ya, yb;

@@ -314,3 +314,16 @@ def test_plan_query_validation(lib):
     # the bench shapes: pipelined, one CTA per SM at most
     assert lib.qk_norm_rope_plan(1, 1, 65536, 32, 8, 128, 32, BF16, 0, 148, 0, pp) == OK
     assert plan[0] == 1 and plan[11] == 148 and plan[13] == (plan[3] + plan[4]) * 32
+
+
+def test_layerwise_bwd_acc_validation(lib):
+    # the accumulating backward checks its arguments exactly like the backward
+    def bwd(fn, Hq=4, dgq=P(17), dq=P(15)):
+        return fn(P(1), P(2), P(3), P(4), None, P(7), P(8), P(11), P(12), P(13), P(14), dq,
+                  P(16), dgq, P(18), 2, 8, Hq, 2, 512, 2, 128, 128, 1e4, BF16, None)
+
+    for fn in (lib.qk_layerwise_norm_rope_bwd, lib.qk_layerwise_norm_rope_bwd_acc):
+        assert bwd(fn, Hq=511) == UNSUP
+        assert bwd(fn, dq=P(11, 16)) == INVALID
+        assert bwd(fn, dgq=P(17, 2)) == ALIGN
+        assert bwd(fn, dq=None) == INVALID
