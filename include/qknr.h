@@ -120,8 +120,8 @@ QKNR_API qknr_status qk_norm_rope_fwd(const void *q, const void *k,
  * rstd and the upstream gradients dq_out/dk_out, writes
  *   dq, dk            gradients w.r.t. q and k (may equal dq_out, dk_out)
  *   dgamma_q/dgamma_k fp32 [D] gradients w.r.t. gamma, OVERWRITTEN (the
- *                     call zeroes them on `stream` first); either may be
- *                     NULL to skip it.
+ *                     call zeroes them on `stream` first, by a small kernel
+ *                     of its own); either may be NULL to skip it.
  * Per row, with g the inverse rotation of dy and xh = x * r:
  *   dgamma_d += g_d * xh_d;   h = g * gamma;
  *   dx = r * (h - xh * <h, xh> / D).

@@ -296,32 +296,21 @@ bool pipe_disabled() {
     return e && e[0] == '1';
 }
 
-// Programmatic dependent launch of the pipelined kernels (they wait for the
-// previous kernel of the stream before touching global memory and let the
-// next one start its prologue early); QKNR_PDL=0 launches them plainly.
-bool pdl_enabled() {
-    static const bool on = [] {
-        const char *e = std::getenv("QKNR_PDL");
-        return !(e && e[0] == '0');
-    }();
-    return on;
+}  // namespace
+
+// na floats at a and nb at b set to zero on the stream (either may be null
+// with a count of 0), by one programmatic-dependent launch.
+qknr_status zero_f32(float *a, int64_t na, float *b, int64_t nb, cudaStream_t st) {
+    if (!a) na = 0;
+    if (!b) nb = 0;
+    if (na + nb == 0) return QKNR_OK;
+    const int64_t blocks = (na + nb + 2047) / 2048;
+    const cudaError_t e =
+        launch_pdl(qknr_zero_kernel, (int)(blocks < 16 ? blocks : 16), 256, 0, st, a, na, b, nb);
+    return e == cudaSuccess ? QKNR_OK : cuda_fail(e);
 }
 
-template <typename... P, typename... A>
-cudaError_t launch_pipe(void (*kern)(P...), int grid, int threads, int smem, cudaStream_t st,
-                        A &&...args) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)grid);
-    cfg.blockDim = dim3((unsigned)threads);
-    cfg.dynamicSmemBytes = (size_t)smem;
-    cfg.stream = st;
-    cudaLaunchAttribute at[1];
-    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    at[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = at;
-    cfg.numAttrs = pdl_enabled() ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, kern, std::forward<A>(args)...);
-}
+namespace {
 
 // cuTensorMapEncodeTiled from the driver, looked up once.
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
@@ -387,7 +376,7 @@ qknr_status launch_fwd_pipe_tm(const FwdArgs &a, const PipeGeom &g, const CUtens
     *launched = true;
     typename MapsArg<TM>::type maps{};
     if constexpr (TM) maps = TensorMaps{mq, mk};
-    cudaError_t e = launch_pipe(kern, grid, (NCW + kProducerWarps) * 32, smem, st, a, g, maps);
+    cudaError_t e = launch_pdl(kern, grid, (NCW + kProducerWarps) * 32, smem, st, a, g, maps);
     return e == cudaSuccess ? QKNR_OK : cuda_fail(e);
 }
 
@@ -403,7 +392,7 @@ qknr_status launch_bwd_pipe_tm(const BwdArgs &a, const PipeGeom &g, const CUtens
     *launched = true;
     typename MapsArg<TM>::type maps{};
     if constexpr (TM) maps = TensorMaps{mq, mk};
-    cudaError_t e = launch_pipe(kern, grid, (NCW + kProducerWarps) * 32, smem, st, a, g, maps);
+    cudaError_t e = launch_pdl(kern, grid, (NCW + kProducerWarps) * 32, smem, st, a, g, maps);
     return e == cudaSuccess ? QKNR_OK : cuda_fail(e);
 }
 
@@ -666,14 +655,9 @@ qknr_status bwd_impl(const void *q, const void *k, int64_t q_ts, int64_t k_ts,
     if (check_overlaps(all, 13, 9, may_equal) != QKNR_OK) return QKNR_ERR_INVALID_ARG;
 
     cudaStream_t cs = (cudaStream_t)stream;
-    if (dgamma_q) {
-        cudaError_t ce = cudaMemsetAsync(dgamma_q, 0, (size_t)D * 4, cs);
-        if (ce != cudaSuccess) return cuda_fail(ce);
-    }
-    if (dgamma_k) {
-        cudaError_t ce = cudaMemsetAsync(dgamma_k, 0, (size_t)D * 4, cs);
-        if (ce != cudaSuccess) return cuda_fail(ce);
-    }
+    // dgamma is accumulated by atomics, so it starts from zero; one small
+    // kernel clears both (chained to the backward launch that follows)
+    if ((st = zero_f32(dgamma_q, D, dgamma_k, D, cs)) != QKNR_OK) return st;
     if (!work) return QKNR_OK;
 
     BwdArgs a{};

@@ -32,6 +32,9 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <cstdlib>
+#include <utility>
+
 namespace qknr {
 
 constexpr int kWarps = 8;
@@ -46,6 +49,48 @@ constexpr int kMaxHalf = kMaxD / 2;
 #ifndef QKNR_BWD_MIN_CTAS
 #define QKNR_BWD_MIN_CTAS 2
 #endif
+
+// Programmatic dependent launch. The pipelined kernels (per-head and
+// layerwise) and the dgamma zeroing kernel are launched with programmatic
+// stream serialization allowed, so a kernel's CTAs may start while the
+// previous kernel of the stream is still finishing: everything before
+// grid_dep_wait() touches only the CTA's own shared memory (and, on the
+// misaligned-shared-memory error path, the library's own error flag), and no
+// input or output is read or written before it returns (the previous kernel
+// has then completed and its writes are visible). grid_dep_launch() lets the
+// next kernel of the stream start its own prologue once every CTA of this one
+// has passed that point. Both are no-ops for a launch without the attribute.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// QKNR_PDL=0 in the environment launches those kernels plainly.
+inline bool pdl_enabled() {
+    static const bool on = [] {
+        const char *e = std::getenv("QKNR_PDL");
+        return !(e && e[0] == '0');
+    }();
+    return on;
+}
+
+// Launch with programmatic stream serialization (unless disabled). Only for
+// kernels that call grid_dep_wait() before their first global access.
+template <typename... P, typename... A>
+cudaError_t launch_pdl(void (*kern)(P...), int grid, int threads, int smem, cudaStream_t st,
+                       A &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3((unsigned)threads);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = pdl_enabled() ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<A>(args)...);
+}
 
 // Forward variants (FwdArgs::mode bits).
 constexpr int kModeRopeOnly = 1;  // rotation alone: r = 1, gamma = 1, no rstd written

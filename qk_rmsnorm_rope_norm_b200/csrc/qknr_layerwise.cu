@@ -36,6 +36,8 @@
 namespace qknr {
 
 qknr_status cuda_fail(cudaError_t e);  // defined beside the per-head entry points
+// zeroes two float ranges by one kernel launch (beside the per-head entry points)
+qknr_status zero_f32(float *a, int64_t na, float *b, int64_t nb, cudaStream_t st);
 
 namespace {
 
@@ -622,14 +624,6 @@ __global__ void __launch_bounds__((kLwCWMax + 1) * 32, 1)
     const int ntiles = t_hi > t_lo ? (int)((t_hi - t_lo + g.TT - 1) / g.TT) : 0;
     const int H = a.Hq + a.Hkv, rowb = a.D * E;
     unsigned char *s_gamma = smem + g.off_gamma;  // every CTA reads the weights once
-    {
-        const int nq = a.Hq * rowb / 16, nk = a.Hkv * rowb / 16;
-        for (int i = threadIdx.x; i < nq + nk; i += nthr) {
-            const Vec16 v = i < nq ? ld16((const char *)a.gq + 16 * i)
-                                   : ld16((const char *)a.gk + 16 * (i - nq));
-            st16(s_gamma + 16 * i, v);
-        }
-    }
     if (threadIdx.x == 0) {
         for (int s = 0; s < g.NS; ++s) {
             lw_bar_init(bar0 + 8 * s, 32);                   // the producer warp's lanes
@@ -637,6 +631,16 @@ __global__ void __launch_bounds__((kLwCWMax + 1) * 32, 1)
         }
         for (int t = 0; t < g.NTG; ++t) lw_bar_init(lw_smem_u32(&s_tgbar[t]), g.G);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    grid_dep_wait();  // no global memory is touched above this line
+    grid_dep_launch();
+    {
+        const int nq = a.Hq * rowb / 16, nk = a.Hkv * rowb / 16;
+        for (int i = threadIdx.x; i < nq + nk; i += nthr) {
+            const Vec16 v = i < nq ? ld16((const char *)a.gq + 16 * i)
+                                   : ld16((const char *)a.gk + 16 * (i - nq));
+            st16(s_gamma + 16 * i, v);
+        }
     }
     __syncthreads();
 
@@ -1016,6 +1020,15 @@ __global__ void __launch_bounds__((kLwCWMax + 1) * 32, 1)
     const int ntiles = t_hi > t_lo ? (int)((t_hi - t_lo + g.TT - 1) / g.TT) : 0;
     const int H = a.Hq + a.Hkv, rowb = a.D * E;
     const unsigned char *s_gamma = smem + g.off_gamma;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < g.NS; ++s) {
+            lw_bar_init(bar0 + 8 * s, 32);              // the producer warp's lanes
+            lw_bar_init(bar0 + 8 * (g.NS + s), ncw);    // one per consumer warp
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    grid_dep_wait();  // no global memory is touched above this line
+    grid_dep_launch();
     if (MODE == kTokFwd) {  // every CTA reads the weights once
         const int nq = a.Hq * rowb / 16, nk = a.Hkv * rowb / 16;
         for (int i = threadIdx.x; i < nq + nk; i += nthr) {
@@ -1023,13 +1036,6 @@ __global__ void __launch_bounds__((kLwCWMax + 1) * 32, 1)
                                    : ld16((const char *)a.gk + 16 * (i - nq));
             st16(smem + g.off_gamma + 16 * i, v);
         }
-    }
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < g.NS; ++s) {
-            lw_bar_init(bar0 + 8 * s, 32);              // the producer warp's lanes
-            lw_bar_init(bar0 + 8 * (g.NS + s), ncw);    // one per consumer warp
-        }
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
     const bool local = a.sq == nullptr && a.sk == nullptr;
@@ -1320,8 +1326,8 @@ qknr_status lw_tok_launch(const LwArgs &a, const LwTokGeom &g, int grid, int sme
     auto kern = qknr_lw_tok_kernel<T, LPR, MODE>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return cuda_fail(e);
-    kern<<<grid, threads, smem, st>>>(a, g);
-    return cuda_status();
+    e = launch_pdl(kern, grid, threads, smem, st, a, g);
+    return e == cudaSuccess ? QKNR_OK : cuda_fail(e);
 }
 
 template <typename T, int LPR, int MODE>
@@ -1332,8 +1338,8 @@ qknr_status lw_pipe_launch(const LwArgs &a, const LwGeom &g, int grid, int smem,
                                             : qknr_lw_pipe_kernel<T, LPR, MODE, 2>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return cuda_fail(e);
-    kern<<<grid, threads, smem, st>>>(a, g);
-    return cuda_status();
+    e = launch_pdl(kern, grid, threads, smem, st, a, g);
+    return e == cudaSuccess ? QKNR_OK : cuda_fail(e);
 }
 
 template <typename T, int LPR>
@@ -1642,13 +1648,10 @@ qknr_status lw_bwd_impl(const void *q, const void *k, const void *gamma_q, const
         if (!disjoint(outs, ins)) return QKNR_ERR_INVALID_ARG;
     }
     cudaStream_t st = (cudaStream_t)stream;
-    cudaError_t ce;
-    if (zero_dgamma && dgamma_q && Hq &&
-        (ce = cudaMemsetAsync(dgamma_q, 0, (size_t)Hq * D * 4, st)) != cudaSuccess)
-        return cuda_fail(ce);
-    if (zero_dgamma && dgamma_k && Hkv &&
-        (ce = cudaMemsetAsync(dgamma_k, 0, (size_t)Hkv * D * 4, st)) != cudaSuccess)
-        return cuda_fail(ce);
+    if (zero_dgamma) {
+        const qknr_status zs = zero_f32(dgamma_q, (int64_t)Hq * D, dgamma_k, (int64_t)Hkv * D, st);
+        if (zs != QKNR_OK) return zs;
+    }
     if (!work) return QKNR_OK;
     LwArgs a{};
     a.q = q; a.k = k; a.gq = gamma_q; a.gk = gamma_k; a.pos = pos_ids;

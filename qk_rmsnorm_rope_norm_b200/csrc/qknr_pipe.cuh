@@ -123,18 +123,20 @@ __global__ void qknr_wait_selftest_kernel(long long limit) {
     fence_mbar_init();
     mbar_wait(b, 0, 256, limit);
 }
-// Programmatic dependent launch. The pipelined kernels are launched with
-// programmatic stream serialization allowed, so a kernel's CTAs may start
-// while the previous kernel of the stream is still finishing: everything
-// before grid_dep_wait() touches only the CTA's own shared memory (and, on
-// the misaligned-shared-memory error path, the library's own error flag), and
-// no input or output is read or written before it returns (the previous
-// kernel has then completed and its writes are visible). grid_dep_launch() lets the next
-// kernel of the stream start its own prologue once every CTA of this one has
-// passed that point. Both are no-ops for a launch without the attribute.
-__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void grid_dep_launch() {
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+// Zeroes the dgamma accumulators ahead of a backward launch. Launched with
+// programmatic stream serialization like the pipelined kernels, it overlaps
+// the previous kernel's tail, and the backward that follows overlaps its own
+// prologue with this one; two memset nodes in its place would end both
+// overlaps (about 6 us of launch gaps a backward call on B200).
+__global__ void __launch_bounds__(256) qknr_zero_kernel(float *a, int64_t na, float *b,
+                                                        int64_t nb) {
+    grid_dep_wait();  // the previous kernel of the stream may still use a or b
+    grid_dep_launch();
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < na + nb; i += stride) {
+        if (i < na) a[i] = 0.f;
+        else b[i - na] = 0.f;
+    }
 }
 
 // Named barrier over the consumer warps only (id 1; id 0 is __syncthreads).
