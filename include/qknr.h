@@ -425,7 +425,7 @@ QKNR_API qknr_status qk_layerwise_geometry(int mode, int B, int S, int Hq, int H
  * forward / backward (qk_layernorm_rope_*). strided: bit 0 (1) when q (k)
  * has a token stride other than its dense one. sms: the SM count to plan
  * for; smem_optin: shared memory per block available by opt-in (0: 227 KB,
- * B200's). plan (14 int64, caller-owned) receives
+ * B200's). plan (15 int64, caller-owned) receives
  *   [0] 1 if the plan is the pipelined kernel, 0 if the plain-load kernel
  *       (then only [1], [2], [5] and [13] are set); the library follows it
  *       on a device with these limits unless QKNR_SIMPLE_KERNELS=1,
@@ -433,7 +433,9 @@ QKNR_API qknr_status qk_layerwise_geometry(int mode, int B, int S, int Hq, int H
  *   [3] consumer warps, [4] producer warps, [5] 1 if mean-centred,
  *   [6] tensor-copy mask (bit 0 q, bit 1 k), [7] tokens per tile,
  *   [8] stages in the ring, [9] bytes per stage, [10] tokens per CTA,
- *   [11] CTAs, [12] dynamic shared memory bytes, [13] threads per CTA.
+ *   [11] CTAs, [12] dynamic shared memory bytes, [13] threads per CTA,
+ *   [14] tokens of each CTA's first tile (a forward without tensor copies
+ *       starts on half a tile; otherwise [7]).
  * The pipelined kernels are named qknr_fwd_pipe_kernel<T, [1], [2], [3],
  * [4], [5], [6] != 0> and qknr_bwd_pipe_kernel<T, [1], [3], [4], [5],
  * [6] != 0>. Shapes are checked as for the entry points; a bad kind,

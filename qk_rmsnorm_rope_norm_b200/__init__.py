@@ -1083,7 +1083,7 @@ def layerwise_geometry(mode: str, B: int, S: int, Hq: int, Hkv: int, D: int, rot
 
 
 _PLAN_KEYS = ("pipelined", "lpr", "units", "consumer_warps", "producer_warps", "ln", "tmap",
-              "TT", "NS", "stage_bytes", "tpc", "grid", "smem", "threads")
+              "TT", "NS", "stage_bytes", "tpc", "grid", "smem", "threads", "first_tile")
 _PLAN_KINDS = {"fwd": 0, "bwd": 1, "ln_fwd": 2, "ln_bwd": 3}
 
 

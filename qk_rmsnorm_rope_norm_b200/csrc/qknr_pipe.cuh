@@ -51,8 +51,9 @@ struct PipeGeom {
     int off_cs;        // (cos, sin) table, TT * R/2 float2
     int off_rq, off_rk;  // backward: saved inverse RMS of Q and K rows
     uint32_t mq, mk;   // jj / Hq == umulhi(jj, mq) (mq == 0: Hq == 1); same for Hkv
-    int64_t tpc;       // tokens per CTA (a multiple of TT)
+    int64_t tpc;       // tokens per CTA
     int tmap;          // bit 0 (1): Q (K) rows arrive by 3-D tensor copy (strided input)
+    int h0;            // tokens of a CTA's first tile when shorter than TT (0: TT)
 };
 
 // ------------------------------------------------------------ PTX helpers
@@ -218,14 +219,26 @@ __device__ __forceinline__ float4 ldsf4(uint32_t addr) {
     return v;
 }
 
-// Everything a CTA knows about its run of tokens.
+// Everything a CTA knows about its run of tokens: tile 0 holds h0 tokens
+// (a shorter first tile lets the consumers start on a partly filled ring
+// instead of waiting for a whole stage), every later tile TT, the last one
+// what remains.
 struct Run {
     int64_t t_lo, t_hi;
-    int ntiles;
+    int ntiles, h0, TT;
     __device__ __forceinline__ Run(int64_t T, const PipeGeom &g) {
         t_lo = (int64_t)blockIdx.x * g.tpc;
         t_hi = min(T, t_lo + g.tpc);
-        ntiles = t_hi > t_lo ? (int)((t_hi - t_lo + g.TT - 1) / g.TT) : 0;
+        TT = g.TT;
+        const int64_t L = t_hi - t_lo;
+        h0 = (g.h0 > 0 && L > g.TT) ? g.h0 : g.TT;
+        ntiles = L > 0 ? (L <= h0 ? 1 : 1 + (int)((L - h0 + g.TT - 1) / g.TT)) : 0;
+    }
+    __device__ __forceinline__ int64_t start(int it) const {
+        return it == 0 ? t_lo : t_lo + h0 + (int64_t)(it - 1) * TT;
+    }
+    __device__ __forceinline__ int count(int it) const {
+        return (int)min((int64_t)(it == 0 ? h0 : TT), t_hi - start(it));
     }
 };
 
@@ -490,8 +503,8 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g,
         // copies of tile `it` into its stage, counted on the stage's barrier
         auto issue = [&](int it) {
             const int s = it % g.NS;
-            const int64_t t0 = run.t_lo + (int64_t)it * g.TT;
-            const int na = (int)min((int64_t)g.TT, run.t_hi - t0);
+            const int64_t t0 = run.start(it);
+            const int na = run.count(it);
             unsigned char *st = smem + (size_t)s * g.stage_bytes;
             const uint32_t bq = (uint32_t)(na * a.Hq * rowb), bk = (uint32_t)(na * a.Hkv * rowb);
             // a tensor copy moves its whole box of TT tokens
@@ -515,18 +528,17 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g,
             for (int it = 0; it < first; ++it) issue(it);
         int issued = first;
         int s_row = run.ntiles ? (int)(run.t_lo % a.S) : 0;  // row position of the tile's first token
-        int32_t pos_next = tile_pos(a.pos, a.S, run.t_lo, s_row,
-                                    (int)min((int64_t)g.TT, run.t_hi - run.t_lo), lane);
+        int32_t pos_next = tile_pos(a.pos, a.S, run.t_lo, s_row, run.ntiles ? run.count(0) : 0, lane);
         for (int it = 0; it < run.ntiles; ++it) {
             const int s = it % g.NS;
-            const int64_t t0 = run.t_lo + (int64_t)it * g.TT;
-            const int na = (int)min((int64_t)g.TT, run.t_hi - t0);
+            const int64_t t0 = run.start(it);
+            const int na = run.count(it);
             const int32_t pos = pos_next;
-            s_row += g.TT;
+            s_row += na;
             while (s_row >= a.S) s_row -= a.S;
             if (it + 1 < run.ntiles) {
-                const int64_t t1 = t0 + g.TT;
-                pos_next = tile_pos(a.pos, a.S, t1, s_row, (int)min((int64_t)g.TT, run.t_hi - t1), lane);
+                const int64_t t1 = t0 + na;
+                pos_next = tile_pos(a.pos, a.S, t1, s_row, run.count(it + 1), lane);
             }
             if (it >= first) {
                 // warp 0 waits for the stage and refills it; the others block
@@ -574,8 +586,8 @@ qknr_fwd_pipe_kernel(const FwdArgs a, const PipeGeom g,
             const int s = it % g.NS;
             if (!mbar_wait(full0 + 8 * s, (it / g.NS) & 1, 0)) break;
             const uint32_t st = smem0 + (uint32_t)(s * g.stage_bytes);
-            const int64_t t0 = run.t_lo + (int64_t)it * g.TT;
-            const int na = (int)min((int64_t)g.TT, run.t_hi - t0);
+            const int64_t t0 = run.start(it);
+            const int na = run.count(it);
 
             // tokens of a tensor-copy box before the tile (partial last tile)
             const int skip = (int)(t0 - box_start(t0, run.t_hi, g.TT));
@@ -740,8 +752,8 @@ qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g,
         const uint64_t pol = evict_first_policy();
         auto issue = [&](int it) {
             const int s = it % g.NS;
-            const int64_t t0 = run.t_lo + (int64_t)it * g.TT;
-            const int na = (int)min((int64_t)g.TT, run.t_hi - t0);
+            const int64_t t0 = run.start(it);
+            const int na = run.count(it);
             unsigned char *st = smem + (size_t)s * g.stage_bytes;
             const uint32_t bq = (uint32_t)(na * a.Hq * rowb), bk = (uint32_t)(na * a.Hkv * rowb);
             // inverse RMS: the 16-byte multiple of each block (the
@@ -772,18 +784,17 @@ qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g,
             for (int it = 0; it < first; ++it) issue(it);
         int issued = first;
         int s_row = run.ntiles ? (int)(run.t_lo % a.S) : 0;  // row position of the tile's first token
-        int32_t pos_next = tile_pos(a.pos, a.S, run.t_lo, s_row,
-                                    (int)min((int64_t)g.TT, run.t_hi - run.t_lo), lane);
+        int32_t pos_next = tile_pos(a.pos, a.S, run.t_lo, s_row, run.ntiles ? run.count(0) : 0, lane);
         for (int it = 0; it < run.ntiles; ++it) {
             const int s = it % g.NS;
-            const int64_t t0 = run.t_lo + (int64_t)it * g.TT;
-            const int na = (int)min((int64_t)g.TT, run.t_hi - t0);
+            const int64_t t0 = run.start(it);
+            const int na = run.count(it);
             const int32_t pos = pos_next;
-            s_row += g.TT;
+            s_row += na;
             while (s_row >= a.S) s_row -= a.S;
             if (it + 1 < run.ntiles) {
-                const int64_t t1 = t0 + g.TT;
-                pos_next = tile_pos(a.pos, a.S, t1, s_row, (int)min((int64_t)g.TT, run.t_hi - t1), lane);
+                const int64_t t1 = t0 + na;
+                pos_next = tile_pos(a.pos, a.S, t1, s_row, run.count(it + 1), lane);
             }
             if (it >= first) {
                 // warp 0 waits for the stage and refills it; the others block
@@ -840,8 +851,8 @@ qknr_bwd_pipe_kernel(const BwdArgs a, const PipeGeom g,
             const int s = it % g.NS;
             if (!mbar_wait(full0 + 8 * s, (it / g.NS) & 1, 0)) break;
             const uint32_t st = smem0 + (uint32_t)(s * g.stage_bytes);
-            const int64_t t0 = run.t_lo + (int64_t)it * g.TT;
-            const int na = (int)min((int64_t)g.TT, run.t_hi - t0);
+            const int64_t t0 = run.start(it);
+            const int na = run.count(it);
 
             // tokens of a tensor-copy box before the tile (partial last tile)
             const int skip = (int)(t0 - box_start(t0, run.t_hi, g.TT));

@@ -99,7 +99,7 @@ def test_sixteen_byte_rows_accepted(lib, dt, D, R):
     # query makes no CUDA call)
     assert fwd(lib, B=0, D=D, R=R, dt=dt) == OK
     assert bwd(lib, B=0, D=D, R=R, dt=dt, dgq=None, dgk=None) == OK
-    plan = (ctypes.c_int64 * 14)()
+    plan = (ctypes.c_int64 * 15)()
     for kind in range(4):
         assert lib.qk_norm_rope_plan(kind, 2, 8, 4, 2, D, R, dt, 0, 148, 0,
                                      ctypes.cast(plan, ctypes.c_void_p)) == OK
@@ -303,7 +303,7 @@ def test_wait_selftest_validation(lib):
 
 
 def test_plan_query_validation(lib):
-    plan = (ctypes.c_int64 * 14)()
+    plan = (ctypes.c_int64 * 15)()
     pp = ctypes.cast(plan, ctypes.c_void_p)
     assert lib.qk_norm_rope_plan(4, 2, 8, 4, 2, 64, 64, BF16, 0, 148, 0, pp) == INVALID
     assert lib.qk_norm_rope_plan(0, 2, 8, 4, 2, 64, 64, BF16, 4, 148, 0, pp) == INVALID
@@ -314,6 +314,13 @@ def test_plan_query_validation(lib):
     # the bench shapes: pipelined, one CTA per SM at most
     assert lib.qk_norm_rope_plan(1, 1, 65536, 32, 8, 128, 32, BF16, 0, 148, 0, pp) == OK
     assert plan[0] == 1 and plan[11] == 148 and plan[13] == (plan[3] + plan[4]) * 32
+    assert plan[14] == plan[7]  # the backward runs whole tiles
+    # the forward starts each CTA on half a tile, unless tensor copies
+    # (strided inputs) move whole boxes
+    assert lib.qk_norm_rope_plan(0, 1, 65536, 32, 8, 128, 32, BF16, 0, 148, 0, pp) == OK
+    assert plan[0] == 1 and plan[14] == plan[7] // 2 and plan[7] >= 2
+    assert lib.qk_norm_rope_plan(0, 1, 65536, 32, 8, 128, 32, BF16, 3, 148, 0, pp) == OK
+    assert plan[6] == 3 and plan[14] == plan[7]
 
 
 def test_layerwise_bwd_acc_validation(lib):
