@@ -878,7 +878,8 @@ def main():
                      "traffic": ncu_traffic(dom_kernel, w.name),
                      "algorithmic_bytes": cb[dom], "peak_source": peak_src},
         "clocks": r["clocks"],
-        "gpu_launches": 2 * args.steps,
+        # per step: the forward, the kernel that clears dgamma, the backward
+        "gpu_launches": 3 * args.steps,
     }
     if r["e2e"] is not None:
         e = r["e2e"]
