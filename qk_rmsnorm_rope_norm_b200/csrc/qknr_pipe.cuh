@@ -278,6 +278,7 @@ __device__ __forceinline__ void tile_angles(float *__restrict__ cs,
                                             const uint64_t *__restrict__ s_step, int half,
                                             int na, int32_t pos, int pw, int lane) {
     constexpr int NW = 32 * NPW;
+    if (half <= 0) return;  // no rotary span (NoPE): no table
     const int w = pw * 32 + lane;
     if (half <= NW) {
         const int G = NW / half;
