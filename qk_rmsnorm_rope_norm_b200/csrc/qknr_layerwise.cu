@@ -42,7 +42,7 @@ qknr_status zero_f32(float *a, int64_t na, float *b, int64_t nb, cudaStream_t st
 namespace {
 
 constexpr int kLwMaxDgammaBytes = 200 * 1024;
-constexpr int kLwGeomLen = 19;  // entries qk_layerwise_geometry writes
+constexpr int kLwGeomLen = 20;  // entries qk_layerwise_geometry writes
 
 struct LwArgs {
     const void *q, *k;        // this rank's heads: [T, Hq, D], [T, Hkv, D]
@@ -961,6 +961,27 @@ struct LwTokGeom {
     int off_gamma;              // gamma_q then gamma_k rows, I/O dtype
     int ncw;                    // consumer warps
     int64_t tpc;                // tokens per CTA
+    int h0;                     // tokens of a CTA's first tile when shorter than TT (0: TT)
+};
+
+// A CTA's tiles: the first holds h (a shorter first tile lets the consumers
+// start before a whole stage has landed), every later one TT, the last what
+// remains.
+struct LwTiles {
+    int64_t t_lo, t_hi;
+    int TT, h, n;
+    __device__ __forceinline__ LwTiles(int64_t lo, int64_t hi, int tt, int h0)
+        : t_lo(lo), t_hi(hi), TT(tt) {
+        const int64_t len = hi - lo;
+        h = (h0 > 0 && len > tt) ? h0 : tt;
+        n = len > 0 ? (len <= h ? 1 : 1 + (int)((len - h + tt - 1) / tt)) : 0;
+    }
+    __device__ __forceinline__ int64_t start(int i) const {
+        return i == 0 ? t_lo : t_lo + h + (int64_t)(i - 1) * TT;
+    }
+    __device__ __forceinline__ int count(int i) const {
+        return (int)min((int64_t)(i == 0 ? h : TT), t_hi - start(i));
+    }
 };
 
 // Sums of x^2 over the rows of one token held in shared memory (Q rows at
@@ -1017,7 +1038,8 @@ __global__ void __launch_bounds__((kLwCWMax + 1) * 32, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t t_lo = (int64_t)blockIdx.x * g.tpc;
     const int64_t t_hi = min(a.T, t_lo + g.tpc);
-    const int ntiles = t_hi > t_lo ? (int)((t_hi - t_lo + g.TT - 1) / g.TT) : 0;
+    const LwTiles tiles(t_lo, t_hi, g.TT, g.h0);
+    const int ntiles = tiles.n;
     const int H = a.Hq + a.Hkv, rowb = a.D * E;
     const unsigned char *s_gamma = smem + g.off_gamma;
     if (threadIdx.x == 0) {
@@ -1050,8 +1072,8 @@ __global__ void __launch_bounds__((kLwCWMax + 1) * 32, 1)
         for (int i = 0; i < ntiles; ++i) {
             const int s = i % g.NS;
             const uint32_t ph = (uint32_t)(i / g.NS) & 1u;
-            const int64_t t0 = t_lo + (int64_t)i * g.TT;
-            const int na = (int)min((int64_t)g.TT, t_hi - t0);
+            const int64_t t0 = tiles.start(i);
+            const int na = tiles.count(i);
             // per-token values, loaded before the wait for the slot
             float2 v = make_float2(0.f, 0.f);
             int32_t pos = 0;
@@ -1071,7 +1093,7 @@ __global__ void __launch_bounds__((kLwCWMax + 1) * 32, 1)
                     }
                 }
             }
-            s_cur += g.TT;
+            s_cur += na;
             while (s_cur >= a.S) s_cur -= a.S;
             if (i >= g.NS && !lw_wait(bar0 + 8 * (g.NS + s), ph ^ 1u)) break;
             unsigned char *st = ring + (size_t)s * g.stage_bytes;
@@ -1115,8 +1137,8 @@ __global__ void __launch_bounds__((kLwCWMax + 1) * 32, 1)
     for (int i = 0; i < ntiles; ++i) {
         const int s = i % g.NS;
         if (!lw_wait(bar0 + 8 * s, (uint32_t)(i / g.NS) & 1u)) break;
-        const int64_t t0 = t_lo + (int64_t)i * g.TT;
-        const int na = (int)min((int64_t)g.TT, t_hi - t0);
+        const int64_t t0 = tiles.start(i);
+        const int na = tiles.count(i);
         const uint32_t st = ring32 + (uint32_t)(s * g.stage_bytes);
         int j = warp - pc;
         if (j < 0) j += ncw;
@@ -1310,6 +1332,7 @@ bool lw_tok_plan(const LwArgs &a, int esz, int sms, LwTokGeom *g, int *grid, int
     g->off_sc = (int)off_sc;
     g->off_gamma = 128 + (int)(NS * stage);
     g->ncw = kLwCWMax;
+    g->h0 = TT >= 2 ? (int)(TT / 2) : 0;  // half a first tile (see LwTiles)
     const int64_t tiles = (a.T + TT - 1) / TT;
     int64_t nb = tiles < (int64_t)sms ? tiles : (int64_t)sms;
     g->tpc = (a.T + nb - 1) / nb;
@@ -1504,7 +1527,7 @@ extern "C" qknr_status qk_layerwise_geometry(int mode, int B, int S, int Hq, int
         const int64_t v[kLwGeomLen] = {1, lpr, t.TT, t.NS, t.stage_bytes, t.off_k, 0, 0,
                                        t.off_cs, t.off_sc, 0, t.off_gamma, 1, t.ncw,
                                        (Hq + Hkv + 32 / lpr - 1) / (32 / lpr), t.tpc, grid, smem,
-                                       thr};
+                                       thr, t.h0 ? t.h0 : t.TT};
         for (int i = 0; i < kLwGeomLen; ++i) geom[i] = v[i];
         return QKNR_OK;
     }
@@ -1513,7 +1536,7 @@ extern "C" qknr_status qk_layerwise_geometry(int mode, int B, int S, int Hq, int
         return QKNR_OK;
     const int64_t v[kLwGeomLen] = {1, lpr, g.TT, g.NS, g.stage_bytes, g.off_k, g.off_dq,
                                    g.off_dk, g.off_cs, g.off_sc, g.off_parts, g.off_gamma, g.G,
-                                   g.NTG, g.HB, g.tpc, grid, smem, thr};
+                                   g.NTG, g.HB, g.tpc, grid, smem, thr, g.TT};
     for (int i = 0; i < kLwGeomLen; ++i) geom[i] = v[i];
     return QKNR_OK;
 }

@@ -400,8 +400,9 @@ def test_layerwise_chunked_schedule_vs_oracle(cuda, name, over, chunks):
 
 
 def test_layerwise_partial_last_stage_vs_oracle(cuda):
-    """A shape whose CTA runs end in a partial stage (tokens per CTA not a
-    multiple of the stage's tokens) and whose grid is below the SM count:
+    """A shape whose CTA runs end in a partial stage (the tokens after the
+    first tile not a multiple of the stage's tokens) and whose grid is below
+    the SM count:
     the launch plan says so, and every element matches the oracle."""
     sms = torch.cuda.get_device_properties(cuda).multi_processor_count
     inp, gq, gk = lw_inputs("llama3-8b-qknorm", B=1, S=1500)
@@ -409,7 +410,10 @@ def test_layerwise_partial_last_stage_vs_oracle(cuda):
     for mode in ("bwd", "tok"):
         g = qknr.layerwise_geometry(mode, w.B, w.S, w.Hq, w.Hkv, w.D, w.rotary_dim,
                                     torch.bfloat16, sms)
-        assert g["pipelined"] and g["tpc"] % g["TT"] != 0 and g["grid"] < sms, (mode, g)
+        # after a first tile of first_tile tokens, whole tiles of TT, then
+        # a partial one
+        assert g["pipelined"] and g["grid"] < sms, (mode, g)
+        assert g["tpc"] > g["TT"] and (g["tpc"] - g["first_tile"]) % g["TT"] != 0, (mode, g)
     for local in (False, True):
         check_vs_oracle(inp, gq, gk, run_ranks(inp, gq, gk, cuda, world=1, local=local))
     check_vs_oracle(inp, gq, gk, run_ranks(inp, gq, gk, cuda, world=2))

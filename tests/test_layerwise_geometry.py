@@ -48,6 +48,7 @@ def replay(mode, B, S, Hq, Hkv, D, R, dtype, sms=148):
     T = B * S
     lpr, TT, NS, stage = g["lpr"], g["TT"], g["NS"], g["stage_bytes"]
     G, NTG, HB = g["G"], g["NTG"], g["HB"]
+    assert g["first_tile"] == TT  # the head-block pipeline runs whole tiles
     slots = 32 // lpr
     # lane layout and warp split
     assert lpr & (lpr - 1) == 0 and lpr >= Dv2 and (lpr == 1 or lpr // 2 < Dv2)
@@ -214,12 +215,17 @@ def replay_tok(B, S, Hq, Hkv, D, R, dtype, sms=148):
     grid, tpc = g["grid"], g["tpc"]
     assert 1 <= grid <= sms and (grid - 1) * tpc < T <= grid * tpc
     seen = set()
+    # each CTA's first tile holds half a tile (whole when TT == 1), later
+    # tiles TT, the last what remains; a run of at most TT is one tile
+    h0 = g["first_tile"]
+    assert h0 == (TT // 2 if TT >= 2 else TT)
     for cta in range(grid):
         t_lo, t_hi = cta * tpc, min(T, (cta + 1) * tpc)
+        h = h0 if t_hi - t_lo > TT else TT
+        starts = [t_lo] + list(range(t_lo + h, t_hi, TT)) if t_hi - t_lo > h else [t_lo]
         pc = 0
-        for i in range(ceil_div(t_hi - t_lo, TT)):
-            t0 = t_lo + i * TT
-            na = min(TT, t_hi - t0)
+        for i, t0 in enumerate(starts):
+            na = min(h if i == 0 else TT, t_hi - t0)
             assert 1 <= na <= TT and t0 + na <= T
             for w in range(ncw):
                 j = (w - pc) % ncw
