@@ -605,42 +605,71 @@ def copy_floor_ms(traffic_bytes: int, dev, n: int = 20) -> float:
 
 
 def run_e2e(args, w, inp, dev, cfg, world):
-    """Public API from pinned host buffers: H2D inputs, fwd, bwd, D2H outputs."""
+    """Public API from pinned host buffers: every step copies its inputs
+    host -> device, runs the forward and the backward, and copies all their
+    results device -> host. Two slots of device buffers and three streams
+    pipeline the steps the way a training loop's loader does: step i + 1's
+    inputs cross PCIe host -> device while step i's results cross it device
+    -> host (the link is full duplex), and a step's kernels run in between.
+    Every step still moves all of its bytes both ways."""
     import qk_rmsnorm_rope_norm_b200 as qknr
     host_in = {n: getattr(inp, n).pin_memory() for n in ("q", "k", "dq_out", "dk_out")}
     gq, gk = inp.gamma_q.to(dev), inp.gamma_k.to(dev)
     pos = None if inp.pos is None else inp.pos.to(dev)
-    d = {n: torch.empty_like(t, device=dev) for n, t in host_in.items()}
     out_shapes = {"q_out": (inp.q.shape, inp.q.dtype), "k_out": (inp.k.shape, inp.k.dtype),
                   "rstd_q": ((w.B, w.S, w.Hq), torch.float32),
                   "rstd_k": ((w.B, w.S, w.Hkv), torch.float32),
                   "dq": (inp.q.shape, inp.q.dtype), "dk": (inp.k.shape, inp.k.dtype),
                   "dgamma_q": ((w.D,), torch.float32), "dgamma_k": ((w.D,), torch.float32)}
     host_out = {n: torch.empty(s, dtype=dt).pin_memory() for n, (s, dt) in out_shapes.items()}
+    slots = []
+    for _ in range(2):
+        d = {n: torch.empty_like(t, device=dev) for n, t in host_in.items()}
+        d.update({n: torch.empty(s, dtype=dt, device=dev) for n, (s, dt) in out_shapes.items()})
+        slots.append(d)
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
     d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+    s_in, s_run, s_out = (torch.cuda.Stream(dev) for _ in range(3))
+    ev = {(k, i): torch.cuda.Event() for k in ("in", "run", "out") for i in range(2)}
+    used = [False, False]
 
-    def step():
-        for n, t in host_in.items():
-            d[n].copy_(t, non_blocking=True)
-        qo, ko, rq, rk = qknr.qk_norm_rope_fwd(d["q"], d["k"], gq, gk, pos, **cfg)
-        dq, dk, dgq, dgk = qknr.qk_norm_rope_bwd(d["q"], d["k"], gq, gk, pos, rq, rk,
-                                                 d["dq_out"], d["dk_out"], **cfg)
-        for n, t in (("q_out", qo), ("k_out", ko), ("rstd_q", rq), ("rstd_k", rk),
-                     ("dq", dq), ("dk", dk), ("dgamma_q", dgq), ("dgamma_k", dgk)):
-            host_out[n].copy_(t, non_blocking=True)
+    def step(i):
+        sl = i % 2
+        d = slots[sl]
+        with torch.cuda.stream(s_in):
+            if used[sl]:
+                s_in.wait_event(ev["run", sl])  # the slot's inputs are read
+            for n, t in host_in.items():
+                d[n].copy_(t, non_blocking=True)
+            ev["in", sl].record(s_in)
+        s_run.wait_event(ev["in", sl])
+        if used[sl]:
+            s_run.wait_event(ev["out", sl])  # the slot's results are out
+        qknr.qk_norm_rope_fwd(d["q"], d["k"], gq, gk, pos, q_out=d["q_out"], k_out=d["k_out"],
+                              rstd_q=d["rstd_q"], rstd_k=d["rstd_k"], stream=s_run, **cfg)
+        qknr.qk_norm_rope_bwd(d["q"], d["k"], gq, gk, pos, d["rstd_q"], d["rstd_k"],
+                              d["dq_out"], d["dk_out"], dq=d["dq"], dk=d["dk"],
+                              dgamma_q=d["dgamma_q"], dgamma_k=d["dgamma_k"], stream=s_run,
+                              **cfg)
+        ev["run", sl].record(s_run)
+        s_out.wait_event(ev["run", sl])
+        with torch.cuda.stream(s_out):
+            for n, t in host_out.items():
+                t.copy_(d[n], non_blocking=True)
+            ev["out", sl].record(s_out)
+        used[sl] = True
 
     E = max(1, min(args.steps, args.e2e_steps))
-    for _ in range(3):
-        step()
+    for i in range(3):
+        step(i)
     torch.cuda.synchronize(dev)
     if world > 1:
         torch.distributed.barrier()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
-    for _ in range(E):
-        step()
-    b.record()
+    a.record(s_in)
+    for i in range(E):
+        step(3 + i)
+    b.record(s_out)  # after the last step's results reached the host
     torch.cuda.synchronize(dev)
     ms = max_over_ranks([a.elapsed_time(b) / E], world, dev)[0]
     return dict(ms=ms, steps=E, h2d=h2d, d2h=d2h)
@@ -885,7 +914,11 @@ def main():
         e = r["e2e"]
         line["e2e"] = {"value": aggregate_tokens_per_s(world, tokens, e["ms"]), "unit": "tokens/s",
                        "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"],
-                       "ms_per_step": e["ms"], "steps": e["steps"]}
+                       "ms_per_step": e["ms"], "steps": e["steps"],
+                       "schedule": "public API calls on pinned host buffers; two device "
+                                   "buffer slots and three streams, so step i+1's "
+                                   "host-to-device copies overlap step i's device-to-host "
+                                   "copies"}
     line["cpu_baseline"] = cpu
     if per_config is not None:
         line["per_config"] = per_config

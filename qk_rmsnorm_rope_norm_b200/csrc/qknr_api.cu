@@ -157,8 +157,10 @@ void geometry(const void *kernel, std::atomic<int> *cache, int64_t T, int *grid,
 // more than 128 bytes per lane group (LPR * U > 4: Llama-3-8B and partial
 // RoPE shapes 3-5% faster than with 12); 12 (512 threads, so 128 registers a
 // thread) for the forward on short rows (Qwen2.5-0.5B shape 7% faster), for
-// every backward (equal or up to 6% faster) and for the mean-centred kernels
-// (which spill at 96 registers).
+// every backward (14 or 16 fit in 96 registers without spills but run 2-5%
+// slower) and for the mean-centred kernels (which spill at 96 registers).
+// Four producer warps: with two, the forward's angle tables take longer to
+// fill (Qwen2.5-0.5B-shaped forward 7% slower).
 constexpr int kFwdPipeWarps = QKNR_FWD_PIPE_WARPS;
 constexpr int kFwdPipeWarpsShortRow = 12;
 constexpr int kBwdPipeWarps = QKNR_BWD_PIPE_WARPS;

@@ -2,25 +2,28 @@
 //
 // Same arithmetic as qknr_kernels.cuh; what changes is how bytes reach the
 // SMs. A persistent CTA owns a contiguous run of tokens and streams it in
-// tiles of TT tokens through a ring of NS shared-memory stages:
+// tiles through a ring of NS shared-memory stages (the forward's first tile
+// holds half the tokens of the others, see Run):
 //
-//  * warp NCW is the producer: one lane arms the stage's "full" mbarrier
-//    with the expected byte count and issues bulk asynchronous copies
-//    (cp.async.bulk, the TMA engine, no tensor map: every block of a tile is
-//    one contiguous run of global memory) for the tile's Q rows and K rows
-//    (and, backward, the upstream gradients and saved inverse RMS); its 32
-//    lanes meanwhile compute the tile's rotary (cos, sin) table into the
-//    stage, then all arrive on "full";
-//  * warps 0..NCW-1 are consumers: they wait on "full", walk the tile's rows
-//    (row passes dealt round-robin across the consumer warps, continuing
-//    across tiles), write results straight to global memory with 16-byte
-//    stores, and arrive on the stage's "empty" mbarrier so the producer can
-//    refill it.
+//  * warps 0..NPW-1 are the producers: lane 0 of warp 0 arms the stage's
+//    "full" mbarrier with the expected byte count and issues asynchronous
+//    bulk copies for the tile's Q rows and K rows (and, backward, the
+//    upstream gradients and saved inverse RMS): cp.async.bulk, the TMA
+//    engine, one contiguous run of global memory a block, or a 3-D tensor
+//    copy when Q / K are strided slices of a fused QKV buffer. All NPW * 32
+//    producer lanes meanwhile compute the tile's rotary (cos, sin) table
+//    into the stage, then arrive on "full";
+//  * the NCW warps after them are consumers: they wait on "full", walk the
+//    tile's rows (row passes dealt round-robin across the consumer warps,
+//    continuing across tiles), write results straight to global memory
+//    with 16-byte stores, and arrive on the stage's "empty" mbarrier so the
+//    producers can refill it.
 //
-// Memory parallelism therefore comes from the copy engine (NS stages of
-// ~16-32 KB in flight per CTA) rather than from registers, and the consumer
-// registers hold gamma, the row and the dgamma partial sums in fp32, with
-// packed FP32x2 arithmetic (FFMA2/FMUL2) on element pairs.
+// Memory parallelism therefore comes from the copy engine (two or three
+// stages of ~80 KB in flight per CTA) rather than from registers, and the
+// consumer registers hold the row and the dgamma partial sums in fp32
+// (gamma and the angle table are read from shared memory), with packed
+// FP32x2 arithmetic (FFMA2/FMUL2) on element pairs.
 //
 // Every mbarrier wait is bounded (about 2-4 s of SM clock cycles); on expiry
 // the thread records an error in g_qknr_pipe_error and leaves its loop, and
