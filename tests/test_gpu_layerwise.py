@@ -417,3 +417,51 @@ def test_layerwise_partial_last_stage_vs_oracle(cuda):
     for local in (False, True):
         check_vs_oracle(inp, gq, gk, run_ranks(inp, gq, gk, cuda, world=1, local=local))
     check_vs_oracle(inp, gq, gk, run_ranks(inp, gq, gk, cuda, world=2))
+
+
+def test_layerwise_offsets_past_4gib_sampled(cuda):
+    """One rank holding every head, q of 4.3 GB (1,048,613 tokens x 16 heads
+    x 128 dims, bf16): offsets past 2^31 elements and 2^32 bytes. The rows
+    repeat one seeded 4,096-token block along the tokens, positions are s,
+    so every token's output differs. Outputs, rstd and dX of sampled tokens
+    (the ends, both sides of the 2^31- and 2^32-byte offsets of q, random
+    ones) against the oracle; dgamma is checked at the sizes above."""
+    import numpy as np
+    base_inp, gq, gk = lw_inputs("llama3-8b-qknorm", B=1, S=4096, Hq=16, Hkv=4, rotary_dim=64)
+    w = base_inp.w
+    T = 2 ** 20 + 37
+    reps = -(-T // w.S)
+
+    def big(t):
+        return t.to(cuda).repeat(1, reps, 1, 1)[:, :T].contiguous()
+
+    q, k = big(base_inp.q), big(base_inp.k)
+    dqo, dko = big(base_inp.dq_out), big(base_inp.dk_out)
+    assert q.numel() * q.element_size() > 2 ** 32
+    cfg = dict(rotary_dim=w.rotary_dim, theta=w.theta, Hq_total=w.Hq, Hkv_total=w.Hkv)
+    qo, ko, rq, rk = qknr.qk_layerwise_norm_rope_fwd(q, k, gq.to(cuda), gk.to(cuda), None, None,
+                                                     None, eps=w.eps, **cfg)
+    dq, dk, _, _ = qknr.qk_layerwise_norm_rope_bwd(q, k, gq.to(cuda), gk.to(cuda), None, rq, rk,
+                                                   dqo, dko, None, None, **cfg)
+    torch.cuda.synchronize()
+    tok_bytes = w.Hq * w.D * 2
+    edges = [0, 1, T - 2, T - 1]
+    for b in (2 ** 31, 2 ** 32):
+        t = b // tok_bytes
+        edges += [t - 1, t, t + 1]
+    pick = np.unique(np.concatenate([edges, np.random.default_rng(6).choice(T, 96,
+                                                                           replace=False)]))
+    idx = torch.from_numpy(pick).to(cuda)
+    base = torch.from_numpy(pick % w.S)
+    o = oracle.get()
+    got = {"q_out": qo, "k_out": ko, "dq": dq, "dk": dk, "rstd_q": rq, "rstd_k": rk}
+    for name, x, g, dy, H in (("q", base_inp.q, gq, base_inp.dq_out, w.Hq),
+                              ("k", base_inp.k, gk, base_inp.dk_out, w.Hkv)):
+        st = parity.Stats(w.dtype, H * w.D)
+        y, r = o.lw_fwd(x[0, base], g, pick, w.rotary_dim, w.theta, w.eps)
+        dx, _ = o.lw_bwd(x[0, base], g, dy[0, base], pick, w.rotary_dim, w.theta, w.eps)
+        sel = lambda t: oracle.as_f64(t.reshape(T, -1).index_select(0, idx).cpu())
+        st.elem(f"{name}_out", sel(got[f"{name}_out"]).reshape(y.shape), y)
+        st.elem(f"d{name}", sel(got[f"d{name}"]).reshape(dx.shape), dx)
+        st.rstd(sel(got[f"rstd_{name}"]).reshape(-1), np.asarray(r).reshape(-1))
+        st.check()

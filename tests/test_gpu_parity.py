@@ -13,6 +13,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import parity
 import workloads
 import qk_rmsnorm_rope_norm_b200 as qknr
@@ -330,3 +331,56 @@ def test_simple_and_pipelined_agree(cuda):
 
 def test_no_pipeline_timeouts(cuda):
     assert qknr.pipeline_error() == 0
+
+
+def test_offsets_past_4gib_sampled(cuda):
+    """A q tensor of 4.3 GB (1,048,613 tokens x 16 heads x 128 dims, bf16):
+    element offsets past 2^31 and byte offsets past 2^32 in every pointer
+    the kernels form. The rows repeat one seeded 4,096-token block along the
+    tokens; positions are s (up to 2^20), so no two tokens give the same
+    output. Forward outputs, rstd, dq and dk of sampled tokens (the ends,
+    both sides of the 2^31- and 2^32-byte offsets of q, random ones) against
+    the oracle; dgamma sums over every row and is checked at the sizes
+    above."""
+    B0 = workloads.make_inputs("llama3-8b-qknorm", B=1, S=4096, Hq=16, Hkv=4, rotary_dim=64)
+    w = B0.w
+    T = 2 ** 20 + 37
+    reps = -(-T // w.S)
+
+    def big(t):
+        return t.to(cuda).repeat(1, reps, 1, 1)[:, :T].contiguous()
+
+    q, k, dqo, dko = big(B0.q), big(B0.k), big(B0.dq_out), big(B0.dk_out)
+    gq, gk = B0.gamma_q.to(cuda), B0.gamma_k.to(cuda)
+    assert q.numel() * q.element_size() > 2 ** 32
+    cfg = dict(rotary_dim=w.rotary_dim, theta=w.theta, eps=w.eps)
+    qo, ko, rq, rk = qknr.qk_norm_rope_fwd(q, k, gq, gk, None, **cfg)
+    dq, dk, _, _ = qknr.qk_norm_rope_bwd(q, k, gq, gk, None, rq, rk, dqo, dko, **cfg)
+    torch.cuda.synchronize()
+    tok_bytes = w.Hq * w.D * 2
+    edges = [0, 1, T - 2, T - 1]
+    for b in (2 ** 31, 2 ** 32):
+        t = b // tok_bytes
+        edges += [t - 1, t, t + 1]
+    rng = np.random.default_rng(5)
+    pick = np.unique(np.concatenate([edges, rng.choice(T, 96, replace=False)]))
+    idx = torch.from_numpy(pick).to(cuda)
+    base = torch.from_numpy(pick % w.S)
+    orc = oracle.get()
+    ref_q, ref_k, ref_rq, ref_rk = orc.fwd(B0.q[0, base], B0.k[0, base], B0.gamma_q, B0.gamma_k,
+                                          pick.astype(np.int64), w.rotary_dim, w.theta, w.eps)
+    ref_dq, ref_dk, _, _ = orc.bwd(B0.q[0, base], B0.k[0, base], B0.gamma_q, B0.gamma_k,
+                                   pick.astype(np.int64), B0.dq_out[0, base], B0.dk_out[0, base],
+                                   w.rotary_dim, w.theta, w.eps)
+
+    def rows(t):
+        return oracle.as_f64(t[0].index_select(0, idx).cpu())
+
+    st = parity.Stats(w.dtype, w.D)
+    st.elem("q_out", rows(qo), ref_q)
+    st.elem("k_out", rows(ko), ref_k)
+    st.elem("dq", rows(dq), ref_dq)
+    st.elem("dk", rows(dk), ref_dk)
+    st.rstd(rows(rq).reshape(-1), np.asarray(ref_rq).reshape(-1))
+    st.rstd(rows(rk).reshape(-1), np.asarray(ref_rk).reshape(-1))
+    st.check()
