@@ -17,16 +17,20 @@
 //             dgamma[h D + d] += g x r_t, g = R^T dy
 //
 // The exchange itself (an all-reduce of one fp32 per token and tensor) is
-// the caller's: NCCL through torch.distributed in the Python binding. A rank
-// holding every head passes no totals and gets one pass each way.
+// the caller's: NCCL through torch.distributed in the Python binding, token
+// chunk by token chunk on a side stream so that each chunk's all-reduce
+// overlaps the next chunk's statistics. A rank holding every head passes no
+// totals and gets one pass each way.
 //
-// Two kernel families. Plain-load kernels: one warp walks all of a token's
-// local heads, so each per-token sum is one warp reduction; gamma rows are
-// read with the same 16-byte vectors as x rows (they are cached; every token
-// reuses them). They serve the statistics and the forward, and every shape
-// the pipeline below does not take. Pipelined kernels (further down): the
-// dots and the backward, staged through shared memory by bulk copies, with
-// dgamma summed in registers.
+// Three kernel families, all staged through shared memory by bulk copies
+// except the last. The token-per-warp pipeline (qknr_lw_tok_kernel) takes
+// the statistics and the forward: a warp owns whole tokens, so each
+// per-token sum is one warp reduction. The head-block pipeline
+// (qknr_lw_pipe_kernel) takes the dots and the backward: a warp owns fixed
+// head blocks of a token group, so dgamma is summed in registers, and the
+// group's warps meet per token for the sum. Plain-load kernels (one warp
+// walks all of a token's local heads with 16-byte loads) take every shape
+// neither pipeline fits.
 #include "qknr.h"
 #include "qknr_kernels.cuh"
 
@@ -944,8 +948,8 @@ __global__ void __launch_bounds__((kLwCWMax + 1) * 32, 1)
 
 // ------------------------------------------------------------------------
 // Pipelined statistics and forward. One producer warp streams stages of TT
-// whole tokens (a stage's Q rows and K rows are two contiguous ranges) into
-// the ring with bulk copies and writes the stage's per-token totals (second
+// whole tokens (a CTA's first stage holds half as many; a stage's Q rows and
+// K rows are two contiguous ranges) into the ring with bulk copies and writes the stage's per-token totals (second
 // phase of a sharded call) and (cos, sin) table. Each consumer warp takes
 // whole tokens, dealt round-robin and continuing across stages: it sums x^2
 // over the token's rows in shared memory (one warp reduction per tensor, no

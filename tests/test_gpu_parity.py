@@ -333,7 +333,8 @@ def test_no_pipeline_timeouts(cuda):
     assert qknr.pipeline_error() == 0
 
 
-def test_offsets_past_4gib_sampled(cuda):
+@pytest.mark.parametrize("family", ["pipelined", "plain"])
+def test_offsets_past_4gib_sampled(cuda, family, monkeypatch):
     """A q tensor of 4.3 GB (1,048,613 tokens x 16 heads x 128 dims, bf16):
     element offsets past 2^31 and byte offsets past 2^32 in every pointer
     the kernels form. The rows repeat one seeded 4,096-token block along the
@@ -341,7 +342,9 @@ def test_offsets_past_4gib_sampled(cuda):
     output. Forward outputs, rstd, dq and dk of sampled tokens (the ends,
     both sides of the 2^31- and 2^32-byte offsets of q, random ones) against
     the oracle; dgamma sums over every row and is checked at the sizes
-    above."""
+    above. Both kernel families."""
+    if family == "plain":
+        monkeypatch.setenv("QKNR_SIMPLE_KERNELS", "1")
     B0 = workloads.make_inputs("llama3-8b-qknorm", B=1, S=4096, Hq=16, Hkv=4, rotary_dim=64)
     w = B0.w
     T = 2 ** 20 + 37
