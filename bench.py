@@ -475,9 +475,11 @@ def layerwise_variants(w, dense, dev, timed, line):
     rank holds every head, one launch each way. "tp_phases": the sequence a
     tensor-parallel rank runs (stats, then normalise; dots, then backward),
     here with every head on one GPU and no exchange between the phases, so it
-    times the extra pass over the rows that sharding costs. Bytes are the
-    op's contract bytes (each row read once and written once, dy read once,
-    rstd [T] per tensor)."""
+    times the extra pass over the rows that sharding costs. "tp_rank": the
+    same sequence on one rank's head slice (TP 8, 4 or 2), the shape a real
+    sharded rank runs. "tp_chunked": the binding's chunked exchange schedule.
+    Bytes are the op's contract bytes (each row read once and written once,
+    dy read once, rstd [T] per tensor)."""
     import qk_rmsnorm_rope_norm_b200 as qknr
     lib = qknr.load_library()
     P = qknr._ptr
@@ -567,7 +569,67 @@ def layerwise_variants(w, dense, dev, timed, line):
             theta=w.theta, Hq_total=w.Hq, Hkv_total=w.Hkv, exchange=no_exchange,
             chunks=qknr.DEFAULT_EXCHANGE_CHUNKS))
 
+    # one rank of a tensor-parallel group on its own head slice: the two
+    # phases it runs (stats, then normalise; dots, then backward), with the
+    # exchange between them a no-op on one GPU. TP = the largest of 8, 4, 2
+    # that divides both head counts.
+    tp = next((t for t in (8, 4, 2) if w.Hq % t == 0 and w.Hkv % t == 0), 1)
+    hq, hk = w.Hq // tp, w.Hkv // tp
+    gq_r, gk_r = gq[: hq * w.D], gk[: hk * w.D]
+    ranks = []
+    for s in dense:
+        r = dict(q=s.q[:, :, :hq].contiguous(), k=s.k[:, :, :hk].contiguous(),
+                 dqo=s.dqo[:, :, :hq].contiguous(), dko=s.dko[:, :, :hk].contiguous(),
+                 pos=s.pos, rq=torch.empty(T, device=dev), rk=torch.empty(T, device=dev),
+                 dgq=torch.empty(hq * w.D, device=dev), dgk=torch.empty(hk * w.D, device=dev))
+        r.update(qo=torch.empty_like(r["q"]), ko=torch.empty_like(r["k"]),
+                 dq=torch.empty_like(r["q"]), dk=torch.empty_like(r["k"]))
+        # one checked pass through the Python API validates every buffer
+        r["sq"], r["sk"] = qknr.qk_layerwise_stats(r["q"], r["k"])
+        qknr.qk_layerwise_norm_rope_fwd(r["q"], r["k"], gq_r, gk_r, r["pos"], r["sq"], r["sk"],
+                                        rotary_dim=w.rotary_dim, theta=w.theta, eps=w.eps,
+                                        Hq_total=w.Hq, Hkv_total=w.Hkv, q_out=r["qo"],
+                                        k_out=r["ko"], rstd_q=r["rq"], rstd_k=r["rk"])
+        qknr.qk_layerwise_norm_rope_bwd(r["q"], r["k"], gq_r, gk_r, r["pos"], r["rq"], r["rk"],
+                                        r["dqo"], r["dko"], r["sq"], r["sk"],
+                                        rotary_dim=w.rotary_dim, theta=w.theta, Hq_total=w.Hq,
+                                        Hkv_total=w.Hkv, dq=r["dq"], dk=r["dk"],
+                                        dgamma_q=r["dgq"], dgamma_k=r["dgk"])
+        ranks.append(r)
+    torch.cuda.synchronize(dev)
+    rank_f = [seq(C(lib.qk_layerwise_stats,
+                    (P(r["q"]), P(r["k"]), P(r["sq"]), P(r["sk"]), w.B, w.S, hq, hk, w.D, dt, st),
+                    "lw stats", r),
+                  C(lib.qk_layerwise_norm_rope_fwd,
+                    (P(r["q"]), P(r["k"]), P(gq_r), P(gk_r), P(r["pos"]), P(r["sq"]), P(r["sk"]),
+                     P(r["qo"]), P(r["ko"]), P(r["rq"]), P(r["rk"]), w.B, w.S, hq, hk, w.Hq,
+                     w.Hkv, w.D, w.rotary_dim, float(w.theta), float(w.eps), dt, st),
+                    "lw fwd", r))
+              for r in ranks]
+    rank_b = [seq(C(lib.qk_layerwise_bwd_dots,
+                    (P(r["q"]), P(r["k"]), P(gq_r), P(gk_r), P(r["pos"]), P(r["rq"]), P(r["rk"]),
+                     P(r["dqo"]), P(r["dko"]), P(r["sq"]), P(r["sk"]), w.B, w.S, hq, hk, w.D,
+                     w.rotary_dim, float(w.theta), dt, st),
+                    "lw dots", r),
+                  C(lib.qk_layerwise_norm_rope_bwd,
+                    (P(r["q"]), P(r["k"]), P(gq_r), P(gk_r), P(r["pos"]), P(r["rq"]), P(r["rk"]),
+                     P(r["dqo"]), P(r["dko"]), P(r["sq"]), P(r["sk"]), P(r["dq"]), P(r["dk"]),
+                     P(r["dgq"]), P(r["dgk"]), w.B, w.S, hq, hk, w.Hq, w.Hkv, w.D,
+                     w.rotary_dim, float(w.theta), dt, st),
+                    "lw bwd", r))
+              for r in ranks]
+    Hr = hq + hk
+    fwd_r = 2 * T * Hr * w.D * e + 4 * T * 2 + pos_b + Hr * w.D * e
+    bwd_r = 3 * T * Hr * w.D * e + 4 * T * 2 + pos_b + Hr * w.D * e
+    rank_line = {"fwd": line(timed(rank_f), fwd_r), "bwd": line(timed(rank_b), bwd_r),
+                 "tp": tp, "heads": f"{hq} + {hk}",
+                 "entry": f"one rank of a TP={tp} group on its {hq} + {hk} head slice: "
+                          "qk_layerwise_stats + _fwd; qk_layerwise_bwd_dots + _bwd (the "
+                          "exchange between them a no-op); bytes are the slice's one-pass bytes"}
+    del ranks
+
     return {
+        "layerwise_tp_rank": rank_line,
         "layerwise_one_pass": {"fwd": line(timed(one_f), fwd_b), "bwd": line(timed(one_b), bwd_b),
                                "entry": "qk_layerwise_norm_rope_fwd / _bwd, sums NULL"},
         "layerwise_tp_phases": {"fwd": line(timed(two_f), fwd_b),
