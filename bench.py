@@ -639,7 +639,8 @@ def layerwise_variants(w, dense, dev, timed, line):
             "fwd": line(timed([chunked_f(s) for s in dense]), fwd_b),
             "bwd": line(timed([chunked_b(s, b) for s, b in zip(dense, bufs)]), bwd_b),
             "entry": f"layerwise_chunked_fwd / _bwd, up to {qknr.DEFAULT_EXCHANGE_CHUNKS} token "
-                     f"chunks of >= {qknr.MIN_CHUNK_TOKENS} tokens, side-stream exchange (here a "
+                     f"chunks of >= {qknr.MIN_CHUNK_TOKENS} tokens and >= "
+                     f"{qknr.MIN_CHUNK_BYTES >> 20} MiB of rows, side-stream exchange (here a "
                      "no-op: one GPU holds every head), captured in a CUDA graph and replayed"},
     }
 

@@ -32,8 +32,8 @@ __all__ = ["qk_norm_rope_fwd", "qk_norm_rope_bwd", "qknr_strerror", "QKNormRoPE"
            "qk_layerwise_stats", "qk_layerwise_norm_rope_fwd", "qk_layerwise_bwd_dots",
            "qk_layerwise_norm_rope_bwd", "QKLayerwiseNormRoPE", "qk_layerwise_norm_rope",
            "all_reduce_stats", "layerwise_geometry", "launch_plan", "kernel_name",
-           "wait_selftest", "token_chunks", "run_chunked", "layerwise_chunked_fwd",
-           "layerwise_chunked_bwd", "MIN_CHUNK_TOKENS"]
+           "wait_selftest", "token_chunks", "chunk_count", "run_chunked", "layerwise_chunked_fwd",
+           "layerwise_chunked_bwd", "MIN_CHUNK_TOKENS", "MIN_CHUNK_BYTES"]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libqknr.so")
@@ -851,16 +851,36 @@ def _all_reduce_exchange(group):
 
 
 MIN_CHUNK_TOKENS = 4096  # a chunk's kernels should outlast their launch and event overhead
+# Rows (this rank's Q and K) a chunk should hold. Chunk i's exchange is
+# hidden only behind chunk i + 1's statistics pass, so a chunk whose
+# statistics take less than one small all-reduce (a few to ~15 us across
+# NVSwitch) adds exposed exchanges instead of hiding one; 96 MiB of rows is
+# ~15 us of HBM time for the statistics pass on B200.
+MIN_CHUNK_BYTES = 96 << 20
+
+
+def chunk_count(T: int, row_bytes: int, chunks: int, min_chunk: int = MIN_CHUNK_TOKENS,
+                min_chunk_bytes: int = MIN_CHUNK_BYTES) -> int:
+    """Token chunks of a sharded layerwise call: at most ``chunks``, each of
+    at least ``min_chunk`` tokens and (when > 0) ``min_chunk_bytes`` of the
+    rank's rows (``row_bytes`` over all T tokens); at least one."""
+    if T <= 0:
+        return 1
+    n = min(int(chunks), T // max(1, int(min_chunk)))
+    if min_chunk_bytes > 0:
+        n = min(n, int(row_bytes) // int(min_chunk_bytes))
+    return max(1, n)
 
 
 class _Chunks:
     """Token chunks of one sharded layerwise call and the direct library
     arguments of each chunk (the tensors are checked once, by the caller)."""
 
-    def __init__(self, q, k, chunks, pos_ids, min_chunk):
+    def __init__(self, q, k, chunks, pos_ids, min_chunk, min_chunk_bytes):
         B, S, Hq, Hkv, D = _shape(q, k)
         self.T = T = B * S
-        n = max(1, min(int(chunks), T // max(1, int(min_chunk)))) if T else 1
+        n = chunk_count(T, T * (Hq + Hkv) * D * q.element_size(), chunks, min_chunk,
+                        min_chunk_bytes)
         self.spans = token_chunks(T, n)
         self.dev = q.device
         self.Hq, self.Hkv, self.D = Hq, Hkv, D
@@ -911,14 +931,17 @@ def _ok(st: int, where: str):
 
 def layerwise_chunked_fwd(q, k, gamma_q, gamma_k, pos_ids, *, rotary_dim: int, theta: float,
                           eps: float, Hq_total: int, Hkv_total: int, exchange, chunks: int = 4,
-                          min_chunk: int = MIN_CHUNK_TOKENS):
+                          min_chunk: int = MIN_CHUNK_TOKENS,
+                          min_chunk_bytes: int = MIN_CHUNK_BYTES):
     """Forward of a rank holding a slice of the heads, in token chunks:
     stats of chunk i -> ``exchange(buf, (t0, t1))`` of its [2, n] partial
     sums (q row, k row) of tokens [t0, t1), on a side stream (the default
     exchange is an all-reduce over the group) -> normalise and rotate chunk
     i, with chunk i's exchange overlapping chunk i + 1's statistics
     (``run_chunked``). The tokens are cut into ``chunks`` runs of at least
-    ``min_chunk`` tokens (fewer runs for short calls). Returns ``(q_out, k_out,
+    ``min_chunk`` tokens and ``min_chunk_bytes`` bytes of this rank's rows
+    (fewer runs for short calls or narrow slices; one run is the plain
+    stats -> exchange -> normalise sequence). Returns ``(q_out, k_out,
     rstd_q, rstd_k)``, rstd fp32 [B*S]."""
     lib = load_library()
     B, S, Hq, Hkv, D = _lw_inputs(q, k, gamma_q, gamma_k, pos_ids)
@@ -928,7 +951,7 @@ def layerwise_chunked_fwd(q, k, gamma_q, gamma_k, pos_ids, *, rotary_dim: int, t
     rstd_k = torch.empty(T, dtype=torch.float32, device=q.device)
     if T == 0:
         return q_out, k_out, rstd_q, rstd_k
-    c = _Chunks(q, k, chunks, pos_ids, min_chunk)
+    c = _Chunks(q, k, chunks, pos_ids, min_chunk, min_chunk_bytes)
     gq, gk = _ptr(gamma_q), _ptr(gamma_k)
 
     def partial(i):
@@ -952,7 +975,8 @@ def layerwise_chunked_fwd(q, k, gamma_q, gamma_k, pos_ids, *, rotary_dim: int, t
 def layerwise_chunked_bwd(q, k, gamma_q, gamma_k, pos_ids, rstd_q, rstd_k, dq_out, dk_out, *,
                           rotary_dim: int, theta: float, Hq_total: int, Hkv_total: int,
                           exchange, chunks: int = 4, need_dgamma: bool = True,
-                          min_chunk: int = MIN_CHUNK_TOKENS):
+                          min_chunk: int = MIN_CHUNK_TOKENS,
+                          min_chunk_bytes: int = MIN_CHUNK_BYTES):
     """Backward of a rank holding a slice of the heads, in token chunks:
     dots of chunk i -> ``exchange(buf, (t0, t1))`` -> dx and the chunk's
     dgamma share (added into one dgamma per tensor, zeroed once), overlapped
@@ -974,7 +998,7 @@ def layerwise_chunked_bwd(q, k, gamma_q, gamma_k, pos_ids, rstd_q, rstd_k, dq_ou
         dgk = torch.zeros(Hkv * D, dtype=torch.float32, device=q.device)
     if T == 0:
         return dq, dk, dgq, dgk
-    c = _Chunks(q, k, chunks, pos_ids, min_chunk)
+    c = _Chunks(q, k, chunks, pos_ids, min_chunk, min_chunk_bytes)
     gq, gk = _ptr(gamma_q), _ptr(gamma_k)
     fn = lib.qk_layerwise_norm_rope_bwd_acc if need_dgamma else lib.qk_layerwise_norm_rope_bwd
 

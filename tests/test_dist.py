@@ -236,3 +236,23 @@ def test_token_chunks_cover_every_token():
             assert spans[0][0] == 0 and spans[-1][1] == T
             assert all(a[1] == b[0] for a, b in zip(spans, spans[1:]))
             assert all(t1 > t0 for t0, t1 in spans) or T == 0
+
+
+def test_chunk_count_rule():
+    """A sharded layerwise call is cut into at most `chunks` token runs, each
+    of at least MIN_CHUNK_TOKENS tokens and MIN_CHUNK_BYTES of the rank's
+    rows, and always at least one."""
+    import qk_rmsnorm_rope_norm_b200 as qknr
+    row = lambda T, H, D=128, e=2: T * H * D * e
+    # every head of the Llama-3-8B and 64k partial-RoPE shapes: byte floor
+    # 96 MiB -> 3 and 4 (the cap) chunks
+    assert qknr.chunk_count(32768, row(32768, 40), 4) == 3
+    assert qknr.chunk_count(65536, row(65536, 40), 4) == 4
+    # one TP-8 rank of the Llama-3-8B shape (4 + 1 heads, 42 MB of rows):
+    # a single run, the plain stats -> exchange -> normalise sequence
+    assert qknr.chunk_count(32768, row(32768, 5), 4) == 1
+    # the token floor binds on short calls; both floors off: the cap
+    assert qknr.chunk_count(8191, row(8191, 400), 4) == 1
+    assert qknr.chunk_count(100, row(100, 5), 7, min_chunk=1, min_chunk_bytes=0) == 7
+    assert qknr.chunk_count(3, row(3, 5), 7, min_chunk=1, min_chunk_bytes=0) == 3
+    assert qknr.chunk_count(0, 0, 4) == 1

@@ -377,14 +377,14 @@ def test_layerwise_chunked_schedule_vs_oracle(cuda, name, over, chunks):
     fw = [qknr.layerwise_chunked_fwd(s["q"], s["k"], s["gq"], s["gk"], pos, eps=w.eps,
                                      Hq_total=w.Hq, Hkv_total=w.Hkv,
                                      exchange=exchange_with(stats[1 - r]), chunks=chunks,
-                                     min_chunk=1, **cfg)
+                                     min_chunk=1, min_chunk_bytes=0, **cfg)
           for r, s in enumerate(sl)]
     dots = [qknr.qk_layerwise_bwd_dots(s["q"], s["k"], s["gq"], s["gk"], pos, f[2], f[3],
                                        s["dqo"], s["dko"], **cfg) for s, f in zip(sl, fw)]
     bw = [qknr.layerwise_chunked_bwd(s["q"], s["k"], s["gq"], s["gk"], pos, f[2], f[3],
                                      s["dqo"], s["dko"], Hq_total=w.Hq, Hkv_total=w.Hkv,
                                      exchange=exchange_with(dots[1 - r]), chunks=chunks,
-                                     min_chunk=1, **cfg)
+                                     min_chunk=1, min_chunk_bytes=0, **cfg)
           for r, (s, f) in enumerate(zip(sl, fw))]
     torch.cuda.synchronize()
     cat = lambda xs, d: torch.cat(xs, dim=d).cpu()
