@@ -401,10 +401,12 @@ struct LwGeom {
     int TT, NS, stage_bytes;
     int off_k, off_dq, off_dk, off_cs;  // sections of a stage (Q rows at 0)
     int off_sc;                         // stage: per-token scalars float4 {rq, rk, sq, sk}
+    int off_pos;                        // stage: token positions, int32
     int off_parts;                      // per-token partial sums [NS][TT][G] float2
     int off_gamma;                      // gamma_q then gamma_k rows, I/O dtype
     int G, NTG, HB;                     // warps per token, token groups, head blocks
     int64_t tpc;                        // tokens per CTA
+    int cs_by_consumers;                // each warp fills its tokens' (cos, sin) table
 };
 
 __device__ __forceinline__ uint32_t lw_smem_u32(const void *p) {
@@ -705,7 +707,9 @@ __global__ void __launch_bounds__((kLwCWMax + 1) * 32, 1)
                             full, pol);
             }
             if (lane < na) reinterpret_cast<float4 *>(st + g.off_sc)[lane] = v;
-            if (need_cs) {
+            if (need_cs && g.cs_by_consumers) {
+                if (lane < na) reinterpret_cast<int32_t *>(st + g.off_pos)[lane] = pos;
+            } else if (need_cs) {
                 if (lane < na) s_pos[lane] = pos;
                 __syncwarp();
                 csw.fill(reinterpret_cast<float4 *>(st + g.off_cs), s_pos, s_step, na, lane);
@@ -773,6 +777,24 @@ __global__ void __launch_bounds__((kLwCWMax + 1) * 32, 1)
                 const bool tok_ok = j < na;
                 float4 c[V / 2];
                 const int jt = tok_ok ? j : j0;
+                if (NBM == 1 && half > 0 && g.cs_by_consumers && tok_ok) {
+                    // every warp of the token's group fills the whole table
+                    // before reading it (the same values, so the group's
+                    // concurrent fills of one entry agree); planned only for
+                    // one head block a warp, the register-lighter instance
+                    const unsigned char *stg = ring + (size_t)s * g.stage_bytes;
+                    const int32_t m = reinterpret_cast<const int32_t *>(stg + g.off_pos)[j];
+                    float4 *tab = reinterpret_cast<float4 *>(ring + (size_t)s * g.stage_bytes +
+                                                             g.off_cs) + j * hp;
+                    for (int P = lane; P < hp; P += 32) {
+                        const int pw = P / (V / 2);
+                        const int dst = (P - pw * (V / 2)) * (hp / (V / 2)) + pw;
+                        const float2 c0 = rope_cos_sin_fixed(m, s_step[2 * P]);
+                        const float2 c1 = rope_cos_sin_fixed(m, s_step[2 * P + 1]);
+                        tab[dst] = make_float4(c0.x, c1.x, c0.y, c1.y);
+                    }
+                    __syncwarp();
+                }
                 lane_cs4_32<V>(c, cs_st + (uint32_t)(jt * hp * 16), co, L);
                 const float4 sv = lw_ldsf4(sc + (uint32_t)(jt * 16));
 #pragma unroll
@@ -962,10 +984,12 @@ enum LwTokMode { kTokStats = 0, kTokFwd = 1 };
 struct LwTokGeom {
     int TT, NS, stage_bytes;
     int off_k, off_cs, off_sc;  // sections of a stage (Q rows at 0); scalars float2 {sq, sk}
+    int off_pos;                // the stage's token positions, int32
     int off_gamma;              // gamma_q then gamma_k rows, I/O dtype
     int ncw;                    // consumer warps
     int64_t tpc;                // tokens per CTA
     int h0;                     // tokens of a CTA's first tile when shorter than TT (0: TT)
+    int cs_by_consumers;        // each consumer warp fills its tokens' (cos, sin) table
 };
 
 // A CTA's tiles: the first holds h (a shorter first tile lets the consumers
@@ -1112,7 +1136,9 @@ __global__ void __launch_bounds__((kLwCWMax + 1) * 32, 1)
                             full, pol);
             }
             if (totals && lane < na) reinterpret_cast<float2 *>(st + g.off_sc)[lane] = v;
-            if (half > 0) {
+            if (half > 0 && g.cs_by_consumers) {
+                if (lane < na) reinterpret_cast<int32_t *>(st + g.off_pos)[lane] = pos;
+            } else if (half > 0) {
                 if (lane < na) s_pos[lane] = pos;
                 __syncwarp();
                 csw.fill(reinterpret_cast<float4 *>(st + g.off_cs), s_pos, s_step, na, lane);
@@ -1168,6 +1194,22 @@ __global__ void __launch_bounds__((kLwCWMax + 1) * 32, 1)
             if (lane == 0) {
                 if (a.Hq) a.wq[t] = rq;
                 if (a.Hkv) a.wk[t] = rk;
+            }
+            if (half > 0 && g.cs_by_consumers) {
+                // this warp owns token j: its lanes fill the token's table
+                // (pair P at the same entry as the producer's fill would)
+                const int32_t m = reinterpret_cast<const int32_t *>(
+                    ring + (size_t)s * g.stage_bytes + g.off_pos)[j];
+                float4 *tab = reinterpret_cast<float4 *>(ring + (size_t)s * g.stage_bytes +
+                                                         g.off_cs) + j * hp;
+                for (int P = lane; P < hp; P += 32) {
+                    const int pw = P / (V / 2);
+                    const int dst = (P - pw * (V / 2)) * (hp / (V / 2)) + pw;
+                    const float2 c0 = rope_cos_sin_fixed(m, s_step[2 * P]);
+                    const float2 c1 = rope_cos_sin_fixed(m, s_step[2 * P + 1]);
+                    tab[dst] = make_float4(c0.x, c1.x, c0.y, c1.y);
+                }
+                __syncwarp();
             }
             float4 c[V / 2];
             lane_cs4_32<V>(c, st + (uint32_t)(g.off_cs + j * hp * 16), co, L);
@@ -1269,13 +1311,13 @@ bool lw_plan(int mode, const LwArgs &a, int esz, int lpr, int sms, LwGeom *g, in
     const int64_t rowb = (int64_t)a.D * esz;
     const int64_t xq = (int64_t)a.Hq * rowb, xk = (int64_t)a.Hkv * rowb;  // per token
     const int64_t csb = (int64_t)(a.R / 2) * 8;
-    const int64_t per = 2 * (xq + xk) + csb + 16;  // rows, gradients, angles, scalars
+    const int64_t per = 2 * (xq + xk) + csb + 16 + 4;  // rows, gradients, angles, scalars, position
     int64_t TT = kLwStageTarget / per;
     TT = TT > kMaxTileTokensLw ? kMaxTileTokensLw : TT;
     TT = (TT / NTG) * NTG;
     if (TT < NTG) TT = NTG;
     if (TT > kMaxTileTokensLw) return false;
-    const int64_t stage = ((TT * per + 127) / 128) * 128;
+    const int64_t stage = ((TT * per + 127) / 128) * 128;  // the position section is last
     const int64_t gbytes = ((xq + xk + 127) / 128) * 128;
     const int64_t budget = kLwSmemBytes - 128 - TT * G * 8 * kLwMaxStages - 128 - gbytes;
     int64_t NS = (budget < kLwRingBytes ? budget : kLwRingBytes) / stage;
@@ -1290,6 +1332,10 @@ bool lw_plan(int mode, const LwArgs &a, int esz, int lpr, int sms, LwGeom *g, in
     g->off_dk = (int)(TT * (2 * xq + xk));
     g->off_cs = (int)(TT * 2 * (xq + xk));
     g->off_sc = g->off_cs + (int)(TT * csb);
+    g->off_pos = g->off_sc + (int)(TT * 16);
+    // few rows a token: the consumer warps fill their tokens' (cos, sin)
+    // tables, as in the token pipeline (see lw_tok_plan)
+    g->cs_by_consumers = (a.R > 0 && NB == 1 && xq + xk < 32 * (int64_t)a.R) ? 1 : 0;
     g->off_parts = 128 + (int)(NS * stage);
     g->off_gamma = g->off_parts + (int)(((NS * TT * G * 8 + 127) / 128) * 128);
     g->G = G;
@@ -1317,12 +1363,13 @@ bool lw_tok_plan(const LwArgs &a, int esz, int sms, LwTokGeom *g, int *grid, int
     const int64_t rowb = (int64_t)a.D * esz;
     const int64_t xq = (int64_t)a.Hq * rowb, xk = (int64_t)a.Hkv * rowb;  // per token
     const int64_t csb = (int64_t)(a.R / 2) * 8;
-    const int64_t per = xq + xk + csb + 8;  // rows, angles, totals
+    const int64_t per = xq + xk + csb + 8 + 4;  // rows, angles, totals, position
     int64_t TT = kLwTokStageTarget / per;
     TT = TT > kMaxTileTokensLw ? kMaxTileTokensLw : (TT < 1 ? 1 : TT);
     const int64_t off_cs = TT * (xq + xk);
     const int64_t off_sc = off_cs + TT * csb;
-    const int64_t stage = ((off_sc + TT * 8 + 127) / 128) * 128;
+    const int64_t off_pos = off_sc + TT * 8;
+    const int64_t stage = ((off_pos + TT * 4 + 127) / 128) * 128;
     const int64_t gbytes = ((xq + xk + 127) / 128) * 128;
     const int64_t budget = kLwSmemBytes - 128 - gbytes;
     int64_t NS = (budget < kLwRingBytes ? budget : kLwRingBytes) / stage;
@@ -1334,9 +1381,17 @@ bool lw_tok_plan(const LwArgs &a, int esz, int sms, LwTokGeom *g, int *grid, int
     g->off_k = (int)(TT * xq);
     g->off_cs = (int)off_cs;
     g->off_sc = (int)off_sc;
+    g->off_pos = (int)off_pos;
     g->off_gamma = 128 + (int)(NS * stage);
     g->ncw = kLwCWMax;
     g->h0 = TT >= 2 ? (int)(TT / 2) : 0;  // half a first tile (see LwTiles)
+    // The one producer warp fills every token's (cos, sin) table of the CTA,
+    // two angles a lane for each four pairs of dims: when a token's rows are
+    // few (a tensor-parallel rank's head slice), that outlasts the rows'
+    // transfer, so the consumer warps fill the tables of their own tokens
+    // instead (Llama-3-8B shape at 4 + 1 heads: the producer-filled forward
+    // ran at 15% DRAM throughput, its consumers waiting on stages).
+    g->cs_by_consumers = (a.R > 0 && xq + xk < 32 * (int64_t)a.R) ? 1 : 0;
     const int64_t tiles = (a.T + TT - 1) / TT;
     int64_t nb = tiles < (int64_t)sms ? tiles : (int64_t)sms;
     g->tpc = (a.T + nb - 1) / nb;
