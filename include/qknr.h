@@ -395,7 +395,7 @@ QKNR_API qknr_status qk_layerwise_norm_rope_bwd_acc(const void *q, const void *k
  * 2: the statistics and the forward (qk_layerwise_stats,
  * qk_layerwise_norm_rope_fwd: one warp per token, so [12] is 1 and [13]
  * the consumer warps, with no dQ_out / dK_out or partial-sum sections);
- * sms: the SM count to plan for. geom (20 int64, caller-owned) receives
+ * sms: the SM count to plan for. geom (22 int64, caller-owned) receives
  *   [0] 1 if the plan for `sms` SMs is the pipelined kernel, 0 if it is
  *       the plain-load kernel (then the rest is 0); this is the plan the
  *       library follows on a device with `sms` SMs unless the environment
@@ -408,7 +408,10 @@ QKNR_API qknr_status qk_layerwise_norm_rope_bwd_acc(const void *q, const void *k
  *   [12] warps per token, [13] token groups, [14] head blocks,
  *   [15] tokens per CTA, [16] CTAs, [17] dynamic shared memory bytes,
  *   [18] threads per CTA, [19] tokens of each CTA's first tile (the
- *       token pipeline starts on half a tile; the head-block one on [2]).
+ *       token pipeline starts on half a tile; the head-block one on [2]),
+ *   [20] 1 when the consumer warps fill their own tokens' (cos, sin)
+ *       tables (few rows a token), 0 when the producer warp fills them,
+ *   [21] offset of the stage's token positions (int32 each).
  * Shapes are checked as for qk_layerwise_norm_rope_bwd (with the totals
  * equal to the local head counts); a bad mode, sms or NULL geom is
  * QKNR_ERR_INVALID_ARG.

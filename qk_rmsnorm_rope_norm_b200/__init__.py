@@ -1088,7 +1088,7 @@ def qk_layerwise_norm_rope(q, k, gamma_q, gamma_k, pos_ids=None, *, rotary_dim: 
 
 _GEOM_KEYS = ("pipelined", "lpr", "TT", "NS", "stage_bytes", "off_k", "off_dq", "off_dk",
               "off_cs", "off_sc", "off_parts", "off_gamma", "G", "NTG", "HB", "tpc", "grid",
-              "smem", "threads", "first_tile")
+              "smem", "threads", "first_tile", "cs_by_consumers", "off_pos")
 
 
 def layerwise_geometry(mode: str, B: int, S: int, Hq: int, Hkv: int, D: int, rotary_dim: int,

@@ -46,7 +46,7 @@ qknr_status zero_f32(float *a, int64_t na, float *b, int64_t nb, cudaStream_t st
 namespace {
 
 constexpr int kLwMaxDgammaBytes = 200 * 1024;
-constexpr int kLwGeomLen = 20;  // entries qk_layerwise_geometry writes
+constexpr int kLwGeomLen = 22;  // entries qk_layerwise_geometry writes
 
 struct LwArgs {
     const void *q, *k;        // this rank's heads: [T, Hq, D], [T, Hkv, D]
@@ -1586,7 +1586,7 @@ extern "C" qknr_status qk_layerwise_geometry(int mode, int B, int S, int Hq, int
         const int64_t v[kLwGeomLen] = {1, lpr, t.TT, t.NS, t.stage_bytes, t.off_k, 0, 0,
                                        t.off_cs, t.off_sc, 0, t.off_gamma, 1, t.ncw,
                                        (Hq + Hkv + 32 / lpr - 1) / (32 / lpr), t.tpc, grid, smem,
-                                       thr, t.h0 ? t.h0 : t.TT};
+                                       thr, t.h0 ? t.h0 : t.TT, t.cs_by_consumers, t.off_pos};
         for (int i = 0; i < kLwGeomLen; ++i) geom[i] = v[i];
         return QKNR_OK;
     }
@@ -1595,7 +1595,8 @@ extern "C" qknr_status qk_layerwise_geometry(int mode, int B, int S, int Hq, int
         return QKNR_OK;
     const int64_t v[kLwGeomLen] = {1, lpr, g.TT, g.NS, g.stage_bytes, g.off_k, g.off_dq,
                                    g.off_dk, g.off_cs, g.off_sc, g.off_parts, g.off_gamma, g.G,
-                                   g.NTG, g.HB, g.tpc, grid, smem, thr, g.TT};
+                                   g.NTG, g.HB, g.tpc, grid, smem, thr, g.TT, g.cs_by_consumers,
+                                   g.off_pos};
     for (int i = 0; i < kLwGeomLen; ++i) geom[i] = v[i];
     return QKNR_OK;
 }

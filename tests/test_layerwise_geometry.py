@@ -62,9 +62,15 @@ def replay(mode, B, S, Hq, Hkv, D, R, dtype, sms=148):
     assert g["off_dk"] == TT * (2 * Hq + Hkv) * rowb
     assert g["off_cs"] == 2 * TT * H * rowb
     assert g["off_sc"] == g["off_cs"] + TT * (R // 2) * 8
-    assert g["off_sc"] + 16 * TT <= stage and stage % 128 == 0
-    for k in ("off_k", "off_dq", "off_dk", "off_cs", "off_sc"):
+    assert g["off_pos"] == g["off_sc"] + 16 * TT
+    assert g["off_pos"] + 4 * TT <= stage and stage % 128 == 0
+    for k in ("off_k", "off_dq", "off_dk", "off_cs", "off_sc", "off_pos"):
         assert g[k] % 16 == 0, k
+    # who fills the (cos, sin) tables: the consumer warps for few rows a
+    # token, and only when a warp owns one head block (the kernel instance
+    # that carries the fill)
+    narrow = R > 0 and H * rowb < 32 * R
+    assert g["cs_by_consumers"] == int(narrow and ceil_div(HB, G) == 1), g
     assert 2 * TT * H * rowb <= TX_LIMIT
     # ring, partial-sum table, gamma table
     assert NS >= 2 and g["off_parts"] == 128 + NS * stage
@@ -182,9 +188,14 @@ def replay_tok(B, S, Hq, Hkv, D, R, dtype, sms=148):
     assert 1 <= TT <= 32
     assert g["off_k"] == TT * Hq * rowb and g["off_cs"] == TT * H * rowb
     assert g["off_sc"] == g["off_cs"] + TT * (R // 2) * 8
-    assert g["off_sc"] + 8 * TT <= stage and stage % 128 == 0
+    assert g["off_pos"] == g["off_sc"] + 8 * TT
+    assert g["off_pos"] + 4 * TT <= stage and stage % 128 == 0
     for k in ("off_k", "off_cs", "off_sc"):
         assert g[k] % 16 == 0, k
+    assert g["off_pos"] % 4 == 0
+    # the consumer warps fill their tokens' (cos, sin) tables for few rows
+    # a token, the producer warp otherwise
+    assert g["cs_by_consumers"] == int(R > 0 and H * rowb < 32 * R), g
     assert TT * H * rowb <= TX_LIMIT
     assert NS >= 2 and g["off_gamma"] == 128 + NS * stage
     assert g["smem"] >= g["off_gamma"] + H * rowb and g["smem"] <= SMEM_LIMIT
