@@ -21,7 +21,9 @@ max over ranks.
 Rank 0 prints one JSON line. ``per_config`` times the other workloads the
 same way (their own rings, forward and backward each). ``e2e`` repeats the
 step through the public Python API from pinned host buffers (inputs copied
-in, every output copied back, inside the timed region). ``cpu_baseline``
+in, every output copied back, inside the timed region; two device slots and
+three streams let one step's host-to-device copies overlap the previous
+step's device-to-host copies). ``cpu_baseline``
 times the CPU oracle on a bounded sample of the same workload, on one host
 core and on all of them.
 """
